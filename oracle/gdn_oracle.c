@@ -1,0 +1,408 @@
+/*
+ * gdn_oracle.c -- plain, slow, fp64 CPU oracle of the Gated DeltaNet
+ * recurrent-state update and of the single-token recurrent layer around it.
+ *
+ * TEST INFRASTRUCTURE. Only the tests, the smoke check and the benchmark's
+ * CPU-baseline leg load this file's library. The CUDA library never links,
+ * includes or calls it, and this file includes nothing from the CUDA side.
+ *
+ * Every value is held in double. Inputs arrive as double arrays (the callers
+ * widen fp32 data exactly), outputs leave as double arrays. The loops follow
+ * the pages' step order with no blocking, fusion or reordering; sums run in
+ * ascending index order.
+ *
+ * Sources (page title, section):
+ *   [S] "Red Lite dev15c -- Gated DeltaNet recurrent-state parity",
+ *       section "Pinned llama.cpp semantics": value head h reads Q/K of key
+ *       head h % 16; state layout M[j][i] = S[i][j]; one token runs the five
+ *       numbered steps; the output uses the updated state.
+ *   [L] "Red Lite dev15e -- complete recurrent DeltaNet layer composition",
+ *       opening list and section "M4 field result": conv/prestate path with
+ *       beta/decay transforms and Q/K L2 normalisation, the recurrence, then
+ *       gated RMSNorm with ssm_norm.weight and SiLU(z); geometry
+ *       channels=8192, qk=2048, value=4096, heads(k/v)=16/32, conv cache.
+ *   [P] "Red Lite dev15a -- DeltaNet projection field validation", section
+ *       "Validation boundary": stage order conv-state shift, ssm_conv1d,
+ *       SiLU, Q/K/V split, per-head Q/K L2 normalisation.
+ *   [B] "Module linear_core" (cortiq_engine), entry "gdn_forward_batch":
+ *       the recurrence runs sequentially over positions and is elementwise
+ *       identical to the one-position path.
+ *
+ * Readings where the pages are silent (each is listed with its reason in the
+ * design notes): gate is a log-decay applied as exp(gate); the output scale
+ * 1/sqrt(128) is 1/sqrt(dk); the conv window is (ring[0..K-2], x) oldest
+ * first with tap t multiplying window[t], no bias, and the ring keeps raw
+ * (pre-conv) inputs; q | k | v are contiguous head-major slices of the conv
+ * output; L2 normalisation is x / max(||x||, l2_eps); beta = sigmoid(b);
+ * gate = -exp(A_log) * softplus(a + dt_bias); the tail is
+ * o * (mean(o^2) + eps)^(-1/2) * w[j] * SiLU(z) with one weight vector of
+ * length dv shared by all heads.
+ *
+ * Return codes: 0 on success, -1 on a bad argument (nothing is written),
+ * -2 when a scratch allocation fails.
+ */
+#include <math.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+
+/* ------------------------------------------------------------------------ */
+/* The recurrence for one value head and one token. [S], steps 1-5.         */
+/* M is [dv][dk] (row j = value index, i = key index, M[j][i] = S[i][j]).   */
+/* ------------------------------------------------------------------------ */
+static int gdn_head_token(double *M, const double *q, const double *k,
+                          const double *v, double beta, double gate,
+                          double *out, int64_t dk, int64_t dv)
+{
+    double *sk = (double *)malloc((size_t)dv * sizeof(double));
+    double *delta = (double *)malloc((size_t)dv * sizeof(double));
+    if (!sk || !delta) {
+        free(sk);
+        free(delta);
+        return -2;
+    }
+
+    /* step 1: M *= exp(gate[h]) */
+    const double decay = exp(gate);
+    for (int64_t j = 0; j < dv; ++j)
+        for (int64_t i = 0; i < dk; ++i)
+            M[j * dk + i] *= decay;
+
+    /* step 2: sk[j] = dot(M[j], k), on the decayed state */
+    for (int64_t j = 0; j < dv; ++j) {
+        double acc = 0.0;
+        for (int64_t i = 0; i < dk; ++i)
+            acc += M[j * dk + i] * k[i];
+        sk[j] = acc;
+    }
+
+    /* step 3: delta[j] = (v[j] - sk[j]) * beta[h] */
+    for (int64_t j = 0; j < dv; ++j)
+        delta[j] = (v[j] - sk[j]) * beta;
+
+    /* step 4: M[j][i] += delta[j] * k[i] */
+    for (int64_t j = 0; j < dv; ++j)
+        for (int64_t i = 0; i < dk; ++i)
+            M[j * dk + i] += delta[j] * k[i];
+
+    /* step 5: out[j] = dot(M[j], q) / sqrt(dk), on the updated state */
+    const double scale_div = sqrt((double)dk);
+    for (int64_t j = 0; j < dv; ++j) {
+        double acc = 0.0;
+        for (int64_t i = 0; i < dk; ++i)
+            acc += M[j * dk + i] * q[i];
+        out[j] = acc / scale_div;
+    }
+
+    free(sk);
+    free(delta);
+    return 0;
+}
+
+static int dims_ok(int64_t Hk, int64_t Hv, int64_t dk, int64_t dv)
+{
+    return Hk > 0 && Hv > 0 && dk > 0 && dv > 0 && Hv % Hk == 0;
+}
+
+/*
+ * Batched single-token decode over L layers x B sequences x Hv value heads.
+ *   state [L][B][Hv][dv][dk]  in/out
+ *   q, k  [L][B][Hk][dk]
+ *   v     [L][B][Hv][dv]
+ *   beta, gate [L][B][Hv]
+ *   out   [L][B][Hv][dv]      (only the listed units are written)
+ * units: flat unit indices u = (l*B + b)*Hv + h to compute, or NULL for all.
+ * [S]: each (layer, sequence, value head) is an independent recurrence; the
+ * value head h takes q/k of key head h % Hk.
+ */
+int oracle_gdn_step(double *state, const double *q, const double *k,
+                    const double *v, const double *beta, const double *gate,
+                    double *out, int64_t L, int64_t B, int64_t Hk, int64_t Hv,
+                    int64_t dk, int64_t dv, const int64_t *units,
+                    int64_t n_units)
+{
+    if (L < 0 || B < 0 || !dims_ok(Hk, Hv, dk, dv))
+        return -1;
+    const int64_t total = L * B * Hv;
+    const int64_t count = units ? n_units : total;
+    for (int64_t n = 0; n < count; ++n) {
+        const int64_t u = units ? units[n] : n;
+        if (u < 0 || u >= total)
+            return -1;
+    }
+    for (int64_t n = 0; n < count; ++n) {
+        const int64_t u = units ? units[n] : n;
+        const int64_t lb = u / Hv;           /* l*B + b */
+        const int64_t h = u % Hv;
+        const int64_t g = h % Hk;            /* key head read by value head h */
+        const double *qg = q + (lb * Hk + g) * dk;
+        const double *kg = k + (lb * Hk + g) * dk;
+        int rc = gdn_head_token(state + u * dv * dk, qg, kg, v + u * dv,
+                                beta[u], gate[u], out + u * dv, dk, dv);
+        if (rc)
+            return rc;
+    }
+    return 0;
+}
+
+/*
+ * Sequential prefill over T positions, [B]: position t runs the one-token
+ * recurrence on the state left by position t-1.
+ *   state [B][Hv][dv][dk]  in: initial, out: final
+ *   q, k  [B][T][Hk][dk]
+ *   v     [B][T][Hv][dv]
+ *   beta, gate [B][T][Hv]
+ *   out   [B][T][Hv][dv]
+ * units: flat indices u = b*Hv + h, or NULL for all.
+ */
+int oracle_gdn_prefill(double *state, const double *q, const double *k,
+                       const double *v, const double *beta, const double *gate,
+                       double *out, int64_t B, int64_t T, int64_t Hk,
+                       int64_t Hv, int64_t dk, int64_t dv,
+                       const int64_t *units, int64_t n_units)
+{
+    if (B < 0 || T < 0 || !dims_ok(Hk, Hv, dk, dv))
+        return -1;
+    const int64_t total = B * Hv;
+    const int64_t count = units ? n_units : total;
+    for (int64_t n = 0; n < count; ++n) {
+        const int64_t u = units ? units[n] : n;
+        if (u < 0 || u >= total)
+            return -1;
+    }
+    for (int64_t n = 0; n < count; ++n) {
+        const int64_t u = units ? units[n] : n;
+        const int64_t b = u / Hv;
+        const int64_t h = u % Hv;
+        const int64_t g = h % Hk;
+        double *M = state + u * dv * dk;
+        for (int64_t t = 0; t < T; ++t) {
+            const int64_t bt = b * T + t;
+            int rc = gdn_head_token(M, q + (bt * Hk + g) * dk,
+                                    k + (bt * Hk + g) * dk,
+                                    v + (bt * Hv + h) * dv,
+                                    beta[bt * Hv + h], gate[bt * Hv + h],
+                                    out + (bt * Hv + h) * dv, dk, dv);
+            if (rc)
+                return rc;
+        }
+    }
+    return 0;
+}
+
+/* ------------------------------------------------------------------------ */
+/* Prestate pieces, [L] and [P].                                             */
+/* ------------------------------------------------------------------------ */
+
+/* SiLU(x) = x * sigmoid(x) */
+static double silu(double x) { return x / (1.0 + exp(-x)); }
+
+/* sigmoid(x) = 1 / (1 + e^-x) */
+static double sigmoid(double x) { return 1.0 / (1.0 + exp(-x)); }
+
+/* softplus(x) = ln(1 + e^x), written as max(x,0) + ln(1 + e^-|x|) */
+static double softplus(double x)
+{
+    return (x > 0.0 ? x : 0.0) + log1p(exp(-fabs(x)));
+}
+
+/*
+ * Causal depthwise conv1d over one token with the conv-state ring, [P]
+ * ("conv-state shift, real F32 ssm_conv1d").
+ *   x    [C]        this token's pre-conv input (mixed q|k|v)
+ *   ring [K-1][C]   in/out; slot 0 is the oldest past input
+ *   w    [C][K]     tap t multiplies window[t], window = (ring[0..K-2], x)
+ *   y    [C]        conv output (before SiLU)
+ * The ring afterwards holds (ring[1..K-2], x): the raw inputs, shifted.
+ */
+static void conv_ring_token(const double *x, double *ring, const double *w,
+                            double *y, int64_t C, int64_t K)
+{
+    for (int64_t c = 0; c < C; ++c) {
+        double acc = 0.0;
+        for (int64_t t = 0; t < K; ++t) {
+            const double win = (t < K - 1) ? ring[t * C + c] : x[c];
+            acc += w[c * K + t] * win;
+        }
+        y[c] = acc;
+    }
+    for (int64_t c = 0; c < C; ++c) {
+        for (int64_t t = 0; t + 1 < K - 1; ++t)
+            ring[t * C + c] = ring[(t + 1) * C + c];
+        if (K > 1)
+            ring[(K - 2) * C + c] = x[c];
+    }
+}
+
+/* x /= max(||x||_2, eps), [L] "Q/K L2 normalization" */
+static void l2_normalize(double *x, int64_t n, double eps)
+{
+    double ss = 0.0;
+    for (int64_t i = 0; i < n; ++i)
+        ss += x[i] * x[i];
+    double norm = sqrt(ss);
+    if (norm < eps)
+        norm = eps;
+    for (int64_t i = 0; i < n; ++i)
+        x[i] = x[i] / norm;
+}
+
+/*
+ * Prestate of one token of one sequence, [L] and [P]:
+ *   conv (with ring shift) -> SiLU -> split q|k|v -> L2(q), L2(k) per key
+ *   head -> beta = sigmoid(b_in), gate = -exp(A_log) * softplus(a + dt_bias).
+ *   x [C = 2*Hk*dk + Hv*dv], ring [K-1][C] in/out, conv_w [C][K],
+ *   a_in, b_in, A_log, dt_bias [Hv].
+ * Outputs: q, k [Hk][dk], v [Hv][dv], beta, gate [Hv].
+ */
+static int prestate_token(const double *x, double *ring, const double *conv_w,
+                          const double *a_in, const double *b_in,
+                          const double *A_log, const double *dt_bias,
+                          double l2_eps, double *q, double *k, double *v,
+                          double *beta, double *gate, int64_t Hk, int64_t Hv,
+                          int64_t dk, int64_t dv, int64_t K)
+{
+    const int64_t C = 2 * Hk * dk + Hv * dv;
+    double *y = (double *)malloc((size_t)C * sizeof(double));
+    if (!y)
+        return -2;
+    conv_ring_token(x, ring, conv_w, y, C, K);
+    for (int64_t c = 0; c < C; ++c)
+        y[c] = silu(y[c]);
+    memcpy(q, y, (size_t)(Hk * dk) * sizeof(double));
+    memcpy(k, y + Hk * dk, (size_t)(Hk * dk) * sizeof(double));
+    memcpy(v, y + 2 * Hk * dk, (size_t)(Hv * dv) * sizeof(double));
+    free(y);
+    for (int64_t g = 0; g < Hk; ++g) {
+        l2_normalize(q + g * dk, dk, l2_eps);
+        l2_normalize(k + g * dk, dk, l2_eps);
+    }
+    for (int64_t h = 0; h < Hv; ++h) {
+        beta[h] = sigmoid(b_in[h]);
+        gate[h] = -exp(A_log[h]) * softplus(a_in[h] + dt_bias[h]);
+    }
+    return 0;
+}
+
+/*
+ * Gated RMSNorm tail of one head, [L] ("gated RMSNorm with ssm_norm.weight
+ * and SiLU(z)"): y[j] = o[j] * (mean(o^2) + eps)^(-1/2) * w[j] * SiLU(z[j]).
+ */
+static void gated_rmsnorm_head(const double *o, const double *z,
+                               const double *w, double eps, double *y,
+                               int64_t dv)
+{
+    double ss = 0.0;
+    for (int64_t j = 0; j < dv; ++j)
+        ss += o[j] * o[j];
+    const double inv_rms = 1.0 / sqrt(ss / (double)dv + eps);
+    for (int64_t j = 0; j < dv; ++j)
+        y[j] = o[j] * inv_rms * w[j] * silu(z[j]);
+}
+
+/*
+ * Stage entry: prestate for the listed sequences (NULL = all B).
+ *   x [B][C], ring [B][K-1][C] in/out, conv_w [C][K], a_in, b_in [B][Hv],
+ *   A_log, dt_bias [Hv]; outputs q, k [B][Hk][dk], v [B][Hv][dv],
+ *   beta, gate [B][Hv].
+ */
+int oracle_gdn_prestate(const double *x, double *ring, const double *conv_w,
+                        const double *a_in, const double *b_in,
+                        const double *A_log, const double *dt_bias,
+                        double l2_eps, double *q, double *k, double *v,
+                        double *beta, double *gate, int64_t B, int64_t Hk,
+                        int64_t Hv, int64_t dk, int64_t dv, int64_t K,
+                        const int64_t *seqs, int64_t n_seqs)
+{
+    if (B < 0 || K < 1 || !dims_ok(Hk, Hv, dk, dv))
+        return -1;
+    const int64_t C = 2 * Hk * dk + Hv * dv;
+    const int64_t count = seqs ? n_seqs : B;
+    for (int64_t n = 0; n < count; ++n) {
+        const int64_t b = seqs ? seqs[n] : n;
+        if (b < 0 || b >= B)
+            return -1;
+    }
+    for (int64_t n = 0; n < count; ++n) {
+        const int64_t b = seqs ? seqs[n] : n;
+        int rc = prestate_token(x + b * C, ring + b * (K - 1) * C, conv_w,
+                                a_in + b * Hv, b_in + b * Hv, A_log, dt_bias,
+                                l2_eps, q + b * Hk * dk, k + b * Hk * dk,
+                                v + b * Hv * dv, beta + b * Hv, gate + b * Hv,
+                                Hk, Hv, dk, dv, K);
+        if (rc)
+            return rc;
+    }
+    return 0;
+}
+
+/*
+ * Stage entry: gated RMSNorm tail over rows of dv values.
+ *   o, z, y [n_rows][dv]; w [dv] shared by every row.
+ */
+int oracle_gated_rmsnorm(const double *o, const double *z, const double *w,
+                         double eps, double *y, int64_t n_rows, int64_t dv)
+{
+    if (n_rows < 0 || dv <= 0)
+        return -1;
+    for (int64_t r = 0; r < n_rows; ++r)
+        gated_rmsnorm_head(o + r * dv, z + r * dv, w, eps, y + r * dv, dv);
+    return 0;
+}
+
+/*
+ * The single-token recurrent layer, [L]: prestate -> recurrence [S] for
+ * every value head -> gated RMSNorm tail, for the listed sequences.
+ *   mixed_qkv [B][C]; z [B][Hv*dv]; a_in, b_in [B][Hv]
+ *   ring [B][K-1][C] in/out; conv_w [C][K]; A_log, dt_bias [Hv]; norm_w [dv]
+ *   state [B][Hv][dv][dk] in/out; out [B][Hv*dv]
+ */
+int oracle_gdn_layer_decode(const double *mixed_qkv, const double *z,
+                            const double *a_in, const double *b_in,
+                            double *ring, const double *conv_w,
+                            const double *A_log, const double *dt_bias,
+                            const double *norm_w, double l2_eps,
+                            double norm_eps, double *state, double *out,
+                            int64_t B, int64_t Hk, int64_t Hv, int64_t dk,
+                            int64_t dv, int64_t K, const int64_t *seqs,
+                            int64_t n_seqs)
+{
+    if (B < 0 || K < 1 || !dims_ok(Hk, Hv, dk, dv))
+        return -1;
+    const int64_t C = 2 * Hk * dk + Hv * dv;
+    const int64_t count = seqs ? n_seqs : B;
+    for (int64_t n = 0; n < count; ++n) {
+        const int64_t b = seqs ? seqs[n] : n;
+        if (b < 0 || b >= B)
+            return -1;
+    }
+    double *q = (double *)malloc((size_t)(Hk * dk) * sizeof(double));
+    double *k = (double *)malloc((size_t)(Hk * dk) * sizeof(double));
+    double *v = (double *)malloc((size_t)(Hv * dv) * sizeof(double));
+    double *beta = (double *)malloc((size_t)Hv * sizeof(double));
+    double *gate = (double *)malloc((size_t)Hv * sizeof(double));
+    double *o = (double *)malloc((size_t)dv * sizeof(double));
+    int rc = (q && k && v && beta && gate && o) ? 0 : -2;
+    for (int64_t n = 0; rc == 0 && n < count; ++n) {
+        const int64_t b = seqs ? seqs[n] : n;
+        rc = prestate_token(mixed_qkv + b * C, ring + b * (K - 1) * C, conv_w,
+                            a_in + b * Hv, b_in + b * Hv, A_log, dt_bias,
+                            l2_eps, q, k, v, beta, gate, Hk, Hv, dk, dv, K);
+        for (int64_t h = 0; rc == 0 && h < Hv; ++h) {
+            const int64_t g = h % Hk;
+            rc = gdn_head_token(state + (b * Hv + h) * dv * dk, q + g * dk,
+                                k + g * dk, v + h * dv, beta[h], gate[h], o,
+                                dk, dv);
+            if (rc == 0)
+                gated_rmsnorm_head(o, z + b * Hv * dv + h * dv, norm_w,
+                                   norm_eps, out + b * Hv * dv + h * dv, dv);
+        }
+    }
+    free(q);
+    free(k);
+    free(v);
+    free(beta);
+    free(gate);
+    free(o);
+    return rc;
+}

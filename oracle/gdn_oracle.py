@@ -1,0 +1,187 @@
+"""ctypes wrapper around ``libgdn_oracle.so`` (built from ``gdn_oracle.c``).
+
+TEST INFRASTRUCTURE. The wrapper only marshals arrays: every input is widened
+to a C-contiguous float64 copy (fp32 data widens exactly), every output comes
+back as a new float64 array, and the caller's arrays are never modified. All
+arithmetic is in the C file; see its header for the passages each function
+follows.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional, Sequence
+
+import numpy as np
+
+from . import build as _build
+
+_I64 = ctypes.c_int64
+_DBL = ctypes.c_double
+_PD = ctypes.POINTER(ctypes.c_double)
+_PI = ctypes.POINTER(ctypes.c_int64)
+
+
+def _f64(a) -> np.ndarray:
+    return np.ascontiguousarray(np.asarray(a, dtype=np.float64)).copy()
+
+
+def _ptr(a: np.ndarray):
+    return a.ctypes.data_as(_PD)
+
+
+def _units(units: Optional[Sequence[int]]):
+    if units is None:
+        return None, 0, None
+    arr = np.ascontiguousarray(np.asarray(units, dtype=np.int64))
+    return arr.ctypes.data_as(_PI), int(arr.size), arr
+
+
+class OracleError(RuntimeError):
+    pass
+
+
+def _check(rc: int, what: str) -> None:
+    if rc == -1:
+        raise OracleError(f"{what}: bad argument")
+    if rc == -2:
+        raise OracleError(f"{what}: out of memory")
+    if rc != 0:
+        raise OracleError(f"{what}: status {rc}")
+
+
+class Oracle:
+    """Handle on one build of the oracle library (the default, or a given .so)."""
+
+    def __init__(self, so_path: Optional[str] = None):
+        if so_path is None:
+            so_path = _build.build()
+        self.path = so_path
+        lib = ctypes.CDLL(os.path.abspath(so_path))
+        lib.oracle_gdn_step.restype = ctypes.c_int
+        lib.oracle_gdn_step.argtypes = [_PD, _PD, _PD, _PD, _PD, _PD, _PD,
+                                        _I64, _I64, _I64, _I64, _I64, _I64, _PI, _I64]
+        lib.oracle_gdn_prefill.restype = ctypes.c_int
+        lib.oracle_gdn_prefill.argtypes = [_PD, _PD, _PD, _PD, _PD, _PD, _PD,
+                                           _I64, _I64, _I64, _I64, _I64, _I64, _PI, _I64]
+        lib.oracle_gdn_prestate.restype = ctypes.c_int
+        lib.oracle_gdn_prestate.argtypes = [_PD, _PD, _PD, _PD, _PD, _PD, _PD, _DBL,
+                                            _PD, _PD, _PD, _PD, _PD,
+                                            _I64, _I64, _I64, _I64, _I64, _I64, _PI, _I64]
+        lib.oracle_gated_rmsnorm.restype = ctypes.c_int
+        lib.oracle_gated_rmsnorm.argtypes = [_PD, _PD, _PD, _DBL, _PD, _I64, _I64]
+        lib.oracle_gdn_layer_decode.restype = ctypes.c_int
+        lib.oracle_gdn_layer_decode.argtypes = [_PD, _PD, _PD, _PD, _PD, _PD, _PD, _PD, _PD,
+                                                _DBL, _DBL, _PD, _PD,
+                                                _I64, _I64, _I64, _I64, _I64, _I64, _PI, _I64]
+        self.lib = lib
+
+    # -- recurrence ---------------------------------------------------------
+    def step(self, state, q, k, v, beta, gate, units=None):
+        """One token for every (layer, sequence, value head) unit.
+
+        Shapes: state [L,B,Hv,dv,dk]; q, k [L,B,Hk,dk]; v [L,B,Hv,dv];
+        beta, gate [L,B,Hv]. Returns (new_state, out [L,B,Hv,dv]); units that
+        are not listed keep their state and get zero output.
+        """
+        st = _f64(state)
+        L, B, Hv, dv, dk = st.shape
+        Hk = np.shape(q)[2]
+        qq, kk, vv, bb, gg = _f64(q), _f64(k), _f64(v), _f64(beta), _f64(gate)
+        assert qq.shape == (L, B, Hk, dk) and kk.shape == qq.shape
+        assert vv.shape == (L, B, Hv, dv) and bb.shape == (L, B, Hv) and gg.shape == bb.shape
+        out = np.zeros((L, B, Hv, dv), dtype=np.float64)
+        up, nu, _keep = _units(units)
+        rc = self.lib.oracle_gdn_step(_ptr(st), _ptr(qq), _ptr(kk), _ptr(vv), _ptr(bb),
+                                      _ptr(gg), _ptr(out), L, B, Hk, Hv, dk, dv, up, nu)
+        _check(rc, "oracle_gdn_step")
+        return st, out
+
+    def prefill(self, state, q, k, v, beta, gate, units=None):
+        """T positions in order, for every (sequence, value head) unit.
+
+        Shapes: state [B,Hv,dv,dk]; q, k [B,T,Hk,dk]; v [B,T,Hv,dv];
+        beta, gate [B,T,Hv]. Returns (final_state, out [B,T,Hv,dv]).
+        """
+        st = _f64(state)
+        B, Hv, dv, dk = st.shape
+        qq, kk, vv, bb, gg = _f64(q), _f64(k), _f64(v), _f64(beta), _f64(gate)
+        T, Hk = qq.shape[1], qq.shape[2]
+        assert qq.shape == (B, T, Hk, dk) and kk.shape == qq.shape
+        assert vv.shape == (B, T, Hv, dv) and bb.shape == (B, T, Hv) and gg.shape == bb.shape
+        out = np.zeros((B, T, Hv, dv), dtype=np.float64)
+        up, nu, _keep = _units(units)
+        rc = self.lib.oracle_gdn_prefill(_ptr(st), _ptr(qq), _ptr(kk), _ptr(vv), _ptr(bb),
+                                         _ptr(gg), _ptr(out), B, T, Hk, Hv, dk, dv, up, nu)
+        _check(rc, "oracle_gdn_prefill")
+        return st, out
+
+    # -- layer pieces -------------------------------------------------------
+    def prestate(self, mixed_qkv, ring, conv_w, a, b, A_log, dt_bias, *, Hk, Hv, dk, dv,
+                 l2_eps=1e-6, seqs=None):
+        """Conv + ring shift, SiLU, split, L2 norm, beta and gate.
+
+        Shapes: mixed_qkv [B,C]; ring [B,K-1,C]; conv_w [C,K]; a, b [B,Hv];
+        A_log, dt_bias [Hv]. Returns dict(q [B,Hk,dk], k, v [B,Hv,dv],
+        beta [B,Hv], gate [B,Hv], ring [B,K-1,C]).
+        """
+        x, rg, w = _f64(mixed_qkv), _f64(ring), _f64(conv_w)
+        B, C = x.shape
+        K = w.shape[1]
+        assert C == 2 * Hk * dk + Hv * dv and rg.shape == (B, K - 1, C) and w.shape == (C, K)
+        aa, bb, al, dt = _f64(a), _f64(b), _f64(A_log), _f64(dt_bias)
+        q = np.zeros((B, Hk, dk)); k = np.zeros((B, Hk, dk)); v = np.zeros((B, Hv, dv))
+        beta = np.zeros((B, Hv)); gate = np.zeros((B, Hv))
+        sp, ns, _keep = _units(seqs)
+        rc = self.lib.oracle_gdn_prestate(_ptr(x), _ptr(rg), _ptr(w), _ptr(aa), _ptr(bb),
+                                          _ptr(al), _ptr(dt), float(l2_eps), _ptr(q), _ptr(k),
+                                          _ptr(v), _ptr(beta), _ptr(gate),
+                                          B, Hk, Hv, dk, dv, K, sp, ns)
+        _check(rc, "oracle_gdn_prestate")
+        return dict(q=q, k=k, v=v, beta=beta, gate=gate, ring=rg)
+
+    def gated_rmsnorm(self, o, z, w, eps=1e-6):
+        """Tail over the last axis: o, z [..., dv]; w [dv]."""
+        oo, zz, ww = _f64(o), _f64(z), _f64(w)
+        dv = oo.shape[-1]
+        assert zz.shape == oo.shape and ww.shape == (dv,)
+        y = np.zeros_like(oo)
+        rc = self.lib.oracle_gated_rmsnorm(_ptr(oo), _ptr(zz), _ptr(ww), float(eps), _ptr(y),
+                                           oo.size // dv, dv)
+        _check(rc, "oracle_gated_rmsnorm")
+        return y
+
+    def layer_decode(self, mixed_qkv, z, a, b, ring, conv_w, A_log, dt_bias, norm_w, state,
+                     *, Hk, l2_eps=1e-6, norm_eps=1e-6, seqs=None):
+        """Prestate -> recurrence -> gated RMSNorm tail, one token per sequence.
+
+        Shapes: mixed_qkv [B,C]; z [B,Hv*dv]; a, b [B,Hv]; ring [B,K-1,C];
+        conv_w [C,K]; A_log, dt_bias [Hv]; norm_w [dv]; state [B,Hv,dv,dk].
+        Returns (out [B,Hv*dv], new_ring, new_state).
+        """
+        st = _f64(state)
+        B, Hv, dv, dk = st.shape
+        x, zz, aa, bb = _f64(mixed_qkv), _f64(z), _f64(a), _f64(b)
+        rg, w, al, dt, nw = _f64(ring), _f64(conv_w), _f64(A_log), _f64(dt_bias), _f64(norm_w)
+        C, K = w.shape
+        assert x.shape == (B, C) and C == 2 * Hk * dk + Hv * dv
+        assert zz.shape == (B, Hv * dv) and rg.shape == (B, K - 1, C) and nw.shape == (dv,)
+        out = np.zeros((B, Hv * dv))
+        sp, ns, _keep = _units(seqs)
+        rc = self.lib.oracle_gdn_layer_decode(_ptr(x), _ptr(zz), _ptr(aa), _ptr(bb), _ptr(rg),
+                                              _ptr(w), _ptr(al), _ptr(dt), _ptr(nw),
+                                              float(l2_eps), float(norm_eps), _ptr(st),
+                                              _ptr(out), B, Hk, Hv, dk, dv, K, sp, ns)
+        _check(rc, "oracle_gdn_layer_decode")
+        return out, rg, st
+
+
+_DEFAULT: Optional[Oracle] = None
+
+
+def load() -> Oracle:
+    """The oracle built from this directory's source (built on first use)."""
+    global _DEFAULT
+    if _DEFAULT is None:
+        _DEFAULT = Oracle()
+    return _DEFAULT

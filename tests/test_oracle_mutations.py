@@ -1,0 +1,90 @@
+"""Plant plausible mistakes in copies of the oracle's C source and check that
+the pins catch every one of them.
+
+Each mutation edits exactly one spot of ``oracle/gdn_oracle.c`` (the target
+text must occur once), is compiled into a temporary library with the same
+flags as the real build, and is run through all pins in
+``oracle_pins.ALL_PINS``. A mutation that no pin detects means the pins have
+a blind spot. Every edit keeps all memory accesses in bounds.
+"""
+import os
+import tempfile
+
+import pytest
+
+from oracle import build as oracle_build
+from oracle.gdn_oracle import Oracle, OracleError
+from oracle_pins import ALL_PINS
+
+MUTATIONS = [
+    # recurrence, "Pinned llama.cpp semantics" steps 1-5
+    ("decay dropped", "M[j * dk + i] *= decay;", "M[j * dk + i] *= 1.0;"),
+    ("decay uses -gate", "const double decay = exp(gate);", "const double decay = exp(-gate);"),
+    ("sk reads q", "acc += M[j * dk + i] * k[i];\n        sk[j] = acc;",
+     "acc += M[j * dk + i] * q[i];\n        sk[j] = acc;"),
+    ("delta sign", "delta[j] = (v[j] - sk[j]) * beta;", "delta[j] = (sk[j] - v[j]) * beta;"),
+    ("beta dropped", "delta[j] = (v[j] - sk[j]) * beta;", "delta[j] = (v[j] - sk[j]);"),
+    ("update sign", "M[j * dk + i] += delta[j] * k[i];", "M[j * dk + i] -= delta[j] * k[i];"),
+    ("update writes q", "M[j * dk + i] += delta[j] * k[i];", "M[j * dk + i] += delta[j] * q[i];"),
+    ("output reads k", "acc += M[j * dk + i] * q[i];\n        out[j]",
+     "acc += M[j * dk + i] * k[i];\n        out[j]"),
+    ("output scale dropped", "out[j] = acc / scale_div;", "out[j] = acc;"),
+    ("output scale 1/dk", "const double scale_div = sqrt((double)dk);",
+     "const double scale_div = (double)dk;"),
+    ("step broadcast h/2", "const int64_t g = h % Hk;            /* key head read by value head h */",
+     "const int64_t g = h / (Hv / Hk);"),
+    ("prefill broadcast h/2", "const int64_t g = h % Hk;\n        double *M",
+     "const int64_t g = h / (Hv / Hk);\n        double *M"),
+    ("prefill order reversed", "const int64_t bt = b * T + t;",
+     "const int64_t bt = b * T + (T - 1 - t);"),
+    # prestate
+    ("conv taps reversed", "acc += w[c * K + t] * win;", "acc += w[c * K + (K - 1 - t)] * win;"),
+    ("ring not refreshed", "ring[(K - 2) * C + c] = x[c];",
+     "ring[(K - 2) * C + c] = ring[(K - 2) * C + c];"),
+    ("ring stores conv output", "ring[(K - 2) * C + c] = x[c];", "ring[(K - 2) * C + c] = y[c];"),
+    ("silu is sigmoid", "static double silu(double x) { return x / (1.0 + exp(-x)); }",
+     "static double silu(double x) { return 1.0 / (1.0 + exp(-x)); }"),
+    ("softplus lost max", "return (x > 0.0 ? x : 0.0) + log1p(exp(-fabs(x)));",
+     "return log1p(exp(-fabs(x)));"),
+    ("gate sign", "gate[h] = -exp(A_log[h]) *", "gate[h] = exp(A_log[h]) *"),
+    ("gate drops dt_bias", "softplus(a_in[h] + dt_bias[h]);", "softplus(a_in[h]);"),
+    ("beta not squashed", "beta[h] = sigmoid(b_in[h]);", "beta[h] = b_in[h];"),
+    ("no L2 norm", "x[i] = x[i] / norm;", "x[i] = x[i];"),
+    ("q takes k slice", "memcpy(q, y, ", "memcpy(q, y + Hk * dk, "),
+    # tail
+    ("rms eps outside sqrt", "1.0 / sqrt(ss / (double)dv + eps);",
+     "1.0 / (sqrt(ss / (double)dv) + eps);"),
+    ("rms sum not mean", "1.0 / sqrt(ss / (double)dv + eps);", "1.0 / sqrt(ss + eps);"),
+    ("tail weight dropped", "y[j] = o[j] * inv_rms * w[j] * silu(z[j]);",
+     "y[j] = o[j] * inv_rms * silu(z[j]);"),
+    ("tail gate not silu", "y[j] = o[j] * inv_rms * w[j] * silu(z[j]);",
+     "y[j] = o[j] * inv_rms * w[j] * z[j];"),
+    ("layer broadcast h/2", "const int64_t g = h % Hk;\n            rc = gdn_head_token",
+     "const int64_t g = h / (Hv / Hk);\n            rc = gdn_head_token"),
+    ("layer tail reads head 0 z", "z + b * Hv * dv + h * dv, norm_w", "z + b * Hv * dv, norm_w"),
+]
+
+
+@pytest.fixture(scope="module")
+def source():
+    with open(oracle_build.SOURCE) as fh:
+        return fh.read()
+
+
+@pytest.mark.parametrize("name,old,new", MUTATIONS, ids=[m[0] for m in MUTATIONS])
+def test_mutation_is_caught(source, name, old, new):
+    assert source.count(old) == 1, f"mutation target for '{name}' must occur exactly once"
+    with tempfile.TemporaryDirectory() as tmp:
+        src = os.path.join(tmp, "mutant.c")
+        lib = os.path.join(tmp, "libmutant.so")
+        with open(src, "w") as fh:
+            fh.write(source.replace(old, new))
+        oracle_build.build(src, lib, force=True)
+        mutant = Oracle(lib)
+        caught = []
+        for pin in ALL_PINS:
+            try:
+                pin(mutant)
+            except (AssertionError, OracleError) as exc:
+                caught.append(f"{pin.__name__}: {str(exc).splitlines()[0][:80]}")
+        assert caught, f"no pin detects mutation '{name}'"
