@@ -1,0 +1,597 @@
+"""Benchmark of the Gated DeltaNet recurrent-state update on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+One step is one batched decode token through ``gdn_step`` over the B = 64
+workload (64 sequences x 32 value heads x 128 x 128 fp32 state, one layer).
+The timed region holds exactly K steps, bracketed by a barrier and a device
+synchronisation on both sides and timed with CUDA events on the launching
+stream; with N ranks each rank runs its own B = 64 batch (weak scaling, no
+collective on the data path) and the slowest rank's time is used.
+
+Printed (rank 0, one JSON line): state GB/s over all ranks, layer-tokens/s,
+the roofline of the step kernel against the measured HBM copy bandwidth, an
+end-to-end figure through the C ABI with the per-step inputs copied from
+pinned host memory and the output copied back, NVML clock samples taken
+during the timed region, the fp64 CPU oracle timed on this host as a
+reported baseline, and (N = 1) the other four workloads measured the same way.
+
+``--impl reference`` times the CPU oracle alone on the same workload and
+metric (rank 0 only; other ranks exit at once).
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import sys
+import threading
+import time
+from typing import Dict, List, Optional
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "gdn_step state GB/s and % of HBM peak; layer-tokens/s at B=64 decode"
+UNIT = "GB/s"
+HEADLINE = "decode_l1_b64"
+L2_BYTES = 126 * 1024 * 1024
+FALLBACK_HBM_GBS = 6650.0
+STATE_BYTES_PER_HEAD = 128 * 128 * 4
+
+# Algorithmic bytes of one value-head token of gdn_step: state read + write,
+# v in, out, beta and gate, and q/k of its key head shared by Hv / Hk value heads.
+def step_bytes(L: int, B: int, Hk: int = 16, Hv: int = 32, d: int = 128) -> int:
+    heads = L * B * Hv
+    return heads * (2 * d * d * 4 + 2 * d * 4 + 2 * 4) + L * B * Hk * 2 * d * 4
+
+
+def prefill_bytes(B: int, T: int, Hk: int = 16, Hv: int = 32, d: int = 128) -> int:
+    return (2 * B * Hv * d * d * 4 + B * T * (Hk * 2 * d * 4 + Hv * (2 * d * 4 + 2 * 4)))
+
+
+def prefill_flops(B: int, T: int, Hv: int = 32, d: int = 128) -> int:
+    # per state element and position: decay (1), sk (2), update (2), output (2)
+    return 7 * B * T * Hv * d * d
+
+
+def layer_bytes(B: int, Hk: int = 16, Hv: int = 32, d: int = 128, K: int = 4) -> int:
+    C = 2 * Hk * d + Hv * d
+    return (B * Hv * d * d * 4 * 2 + B * (K - 1) * C * 4 * 2 + B * C * 4 + B * Hv * d * 4 * 2
+            + B * Hv * 4 * 2 + C * K * 4 + Hv * 4 * 2 + d * 4)
+
+
+# --------------------------------------------------------------------------
+# host-side helpers (no GPU needed; covered by the CPU tests)
+# --------------------------------------------------------------------------
+def dist_env() -> Dict[str, int]:
+    return dict(rank=int(os.environ.get("RANK", 0)), world=int(os.environ.get("WORLD_SIZE", 1)),
+                local_rank=int(os.environ.get("LOCAL_RANK", 0)))
+
+
+def rank_seed(base: int, rank: int) -> int:
+    """Each rank draws its own batch (weak scaling): distinct, reproducible seeds."""
+    return base + 7919 * rank
+
+
+def max_over_ranks(value: float, device=None) -> float:
+    """The largest value over all ranks (identity without a process group)."""
+    import torch
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return float(value)
+    t = torch.tensor([float(value)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def throughput(units_per_rank: float, n_ranks: int, seconds: float) -> float:
+    """Whole-job throughput: units processed by all ranks over the slowest rank's time."""
+    return units_per_rank * n_ranks / seconds if seconds > 0 else float("nan")
+
+
+def measured_peaks() -> Dict[str, object]:
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as fh:
+            p = json.load(fh)
+        return dict(hbm_gbs=float(p["hbm_gbs"]), source="measured")
+    except (OSError, KeyError, ValueError):
+        return dict(hbm_gbs=FALLBACK_HBM_GBS, source="fallback")
+
+
+def kernel_source_digest(names: List[str]) -> str:
+    """Short hash of kernel sources; a stored ncu traffic figure is used only
+    while the source it was taken from is unchanged."""
+    h = hashlib.sha256()
+    for n in names:
+        with open(os.path.join(ROOT, "linear_attention_recurrence_04_b200", "csrc", n), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def stored_traffic(kernel: str, digest: str) -> Optional[float]:
+    """DRAM bytes per launch from the committed ncu summary, if still current."""
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    try:
+        with open(path) as fh:
+            rec = json.load(fh).get(kernel)
+    except (OSError, ValueError):
+        return None
+    if not rec or rec.get("source_digest") != digest:
+        return None
+    return float(rec["dram_bytes_per_launch"])
+
+
+REASON_BITS = {
+    0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap",
+    0x8: "hw_slowdown", 0x10: "sync_boost", 0x20: "sw_thermal_slowdown",
+    0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown",
+    0x100: "display_clock_setting",
+}
+
+
+def decode_reasons(mask: int) -> List[str]:
+    return [name for bit, name in REASON_BITS.items() if mask & bit]
+
+
+class ClockSampler:
+    """Samples SM clock and clock-event reasons through NVML in a thread."""
+
+    def __init__(self, device_index: int, period_s: float = 0.005):
+        self.period = period_s
+        self.samples: List[int] = []
+        self.reasons = 0
+        self.max_mhz: Optional[int] = None
+        self._stop = threading.Event()
+        self._thread = None
+        self._nvml = None
+        self._handle = None
+        try:
+            import pynvml
+            import torch
+            pynvml.nvmlInit()
+            self._nvml = pynvml
+            try:
+                uuid = str(torch.cuda.get_device_properties(device_index).uuid)
+                self._handle = pynvml.nvmlDeviceGetHandleByUUID(
+                    uuid if uuid.startswith("GPU-") else "GPU-" + uuid)
+            except Exception:
+                self._handle = pynvml.nvmlDeviceGetHandleByIndex(device_index)
+            self.max_mhz = int(pynvml.nvmlDeviceGetMaxClockInfo(self._handle,
+                                                                pynvml.NVML_CLOCK_SM))
+        except Exception:
+            self._nvml = None
+
+    def _sample(self):
+        p = self._nvml
+        self.samples.append(int(p.nvmlDeviceGetClockInfo(self._handle, p.NVML_CLOCK_SM)))
+        try:
+            mask = p.nvmlDeviceGetCurrentClocksEventReasons(self._handle)
+        except AttributeError:
+            mask = p.nvmlDeviceGetCurrentClocksThrottleReasons(self._handle)
+        self.reasons |= int(mask)
+
+    def _run(self):
+        while not self._stop.is_set():
+            try:
+                self._sample()
+            except Exception:
+                break
+            self._stop.wait(self.period)
+
+    def __enter__(self):
+        if self._nvml is not None:
+            self._thread = threading.Thread(target=self._run, daemon=True)
+            self._thread.start()
+        return self
+
+    def __exit__(self, *exc):
+        self._stop.set()
+        if self._thread is not None:
+            self._thread.join()
+            if not self.samples:
+                self._sample()
+
+    def summary(self) -> Dict[str, object]:
+        if self._nvml is None:
+            return dict(sm_mhz=None, sm_max_mhz=None, reasons=["nvml_unavailable"], samples=0)
+        med = float(np.median(self.samples)) if self.samples else None
+        reasons = [r for r in decode_reasons(self.reasons) if r != "gpu_idle"]
+        return dict(sm_mhz=med, sm_max_mhz=self.max_mhz, reasons=reasons,
+                    samples=len(self.samples))
+
+
+# --------------------------------------------------------------------------
+# GPU measurement
+# --------------------------------------------------------------------------
+def _to_dev(d: Dict[str, np.ndarray], device) -> Dict[str, "torch.Tensor"]:
+    import torch
+    return {k: torch.from_numpy(np.ascontiguousarray(v)).to(device) for k, v in d.items()}
+
+
+def _sets_for(bytes_per_set: int) -> int:
+    """Rotating input sets so the sets together exceed 4x the L2."""
+    return max(1, min(64, math.ceil(4 * L2_BYTES / max(bytes_per_set, 1))))
+
+
+def capture(launches, device):
+    """A CUDA graph holding the given launches (callables), in order."""
+    import torch
+    g = torch.cuda.CUDAGraph()
+    side = torch.cuda.Stream(device)
+    with torch.cuda.graph(g, stream=side):
+        for fn in launches:
+            fn()
+    return g
+
+
+def time_launches(launch, n_sets: int, steps: int, warmup: int, stream,
+                  graph: bool = False) -> float:
+    """Run `launch(i)` for warmup + steps iterations, rotating input set
+    i % n_sets; return the device seconds of the timed steps. With
+    graph=True the timed steps are captured once into a CUDA graph and
+    replayed, so host launch overhead does not enter the timing."""
+    import torch
+    for i in range(warmup):
+        launch(i % n_sets)
+    torch.cuda.synchronize()
+    g = None
+    if graph and steps > 0:
+        g = capture([(lambda j=j: launch((warmup + j) % n_sets)) for j in range(steps)],
+                    stream.device)
+        torch.cuda.synchronize()
+    start = torch.cuda.Event(enable_timing=True)
+    end = torch.cuda.Event(enable_timing=True)
+    start.record(stream)
+    if g is not None:
+        g.replay()
+    else:
+        for i in range(steps):
+            launch((warmup + i) % n_sets)
+    end.record(stream)
+    torch.cuda.synchronize()
+    return start.elapsed_time(end) / 1e3
+
+
+def bench_step_workload(name: str, steps: int, warmup: int, device, seed_offset: int = 0,
+                        graph: bool = True):
+    import torch
+    from linear_attention_recurrence_04_b200 import gdn, inputs
+    w = inputs.WORKLOADS[name]
+    L, B = w.sizes["L"], w.sizes["B"]
+    d = inputs.decode_inputs(L, B, seed=w.seed + seed_offset)
+    base = _to_dev(d, device)
+    nbytes = step_bytes(L, B)
+    n_sets = _sets_for(nbytes)
+    sets = [base] + [{k: v.clone() for k, v in base.items()} for _ in range(n_sets - 1)]
+    outs = [torch.empty_like(s["v"]) for s in sets]
+    stream = torch.cuda.current_stream(device)
+
+    def launch(i):
+        s = sets[i]
+        gdn.step(s["state"], s["q"], s["k"], s["v"], s["beta"], s["gate"], outs[i])
+
+    secs = time_launches(launch, n_sets, steps, warmup, stream, graph=graph)
+    return dict(seconds=secs, bytes=nbytes, state_bytes=L * B * 32 * STATE_BYTES_PER_HEAD,
+                layer_tokens=L * B, n_sets=n_sets, set_bytes=nbytes, sets=sets, outs=outs, d=d)
+
+
+def bench_e2e(d: Dict[str, np.ndarray], steps: int, warmup: int, device):
+    """gdn_step through the C ABI with each step's q, k, v, beta, gate copied
+    from pinned host memory and the output copied back to pinned host memory,
+    all inside the timed region. The recurrent state stays resident on the
+    device, as a decode cache does."""
+    import torch
+    from linear_attention_recurrence_04_b200 import gdn
+    host = {k: torch.from_numpy(np.ascontiguousarray(d[k])).pin_memory()
+            for k in ("q", "k", "v", "beta", "gate")}
+    state_bytes = d["state"].nbytes
+    n_sets = _sets_for(state_bytes)
+    states = [torch.from_numpy(d["state"]).to(device) for _ in range(n_sets)]
+    dev_in = {k: torch.empty(v.shape, dtype=v.dtype, device=device) for k, v in host.items()}
+    out_dev = torch.empty(d["v"].shape, dtype=torch.float32, device=device)
+    out_host = torch.empty(d["v"].shape, dtype=torch.float32).pin_memory()
+    stream = torch.cuda.current_stream(device)
+
+    def launch(i):
+        for k, v in host.items():
+            dev_in[k].copy_(v, non_blocking=True)
+        gdn.step(states[i], dev_in["q"], dev_in["k"], dev_in["v"], dev_in["beta"],
+                 dev_in["gate"], out_dev)
+        out_host.copy_(out_dev, non_blocking=True)
+
+    secs = time_launches(launch, n_sets, steps, warmup, stream)
+    h2d = sum(v.numel() * v.element_size() for v in host.values())
+    d2h = out_host.numel() * out_host.element_size()
+    return secs, h2d, d2h
+
+
+def bench_prefill(steps: int, warmup: int, device):
+    """Each launch starts from the zero state (restored outside the timed
+    interval); the launches alone are timed, one event pair each."""
+    import torch
+    from linear_attention_recurrence_04_b200 import gdn, inputs
+    w = inputs.WORKLOADS["prefill_b4_t4096"]
+    B, T = w.sizes["B"], w.sizes["T"]
+    t = _to_dev(w.draw(), device)
+    out = torch.empty_like(t["v"])
+    state0 = t["state"].clone()
+    stream = torch.cuda.current_stream(device)
+    total = 0.0
+    for i in range(warmup + steps):
+        t["state"].copy_(state0)
+        a = torch.cuda.Event(enable_timing=True)
+        b = torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        gdn.prefill(t["state"], t["q"], t["k"], t["v"], t["beta"], t["gate"], out)
+        b.record(stream)
+        torch.cuda.synchronize()
+        if i >= warmup:
+            total += a.elapsed_time(b) / 1e3
+    return dict(seconds=total, launches=steps, bytes=prefill_bytes(B, T),
+                flops=prefill_flops(B, T), tokens=B * T)
+
+
+def bench_layer(steps: int, warmup: int, device):
+    import torch
+    from linear_attention_recurrence_04_b200 import gdn, inputs
+    w = inputs.WORKLOADS["layer_decode_b256"]
+    B = w.sizes["B"]
+    t = _to_dev(w.draw(), device)
+    out = torch.empty_like(t["z"])
+    order = ("mixed_qkv", "z", "a", "b", "conv_ring", "conv_w", "A_log", "dt_bias", "norm_w",
+             "state")
+    stream = torch.cuda.current_stream(device)
+
+    def launch(i):
+        gdn.layer_decode(*(t[n] for n in order), out, Hk=16)
+
+    secs = time_launches(launch, 1, steps, warmup, stream, graph=True)
+    return dict(seconds=secs, launches=steps, bytes=layer_bytes(B), tokens=B)
+
+
+def cpu_oracle_baseline(name: str, budget_s: float, max_units: Optional[int] = None):
+    """Time the fp64 oracle as it stands on a bounded sample of the workload:
+    whole decode steps over the first `units` (layer, sequence, head) units,
+    repeated until `budget_s` has elapsed (at least once)."""
+    import oracle
+    from linear_attention_recurrence_04_b200 import inputs
+    o = oracle.load()
+    w = inputs.WORKLOADS[name]
+    L, B = w.sizes["L"], w.sizes["B"]
+    d = inputs.decode_inputs(L, B, seed=w.seed)
+    total_units = L * B * 32
+    units = np.arange(total_units if max_units is None else min(max_units, total_units))
+    st = d["state"]
+    reps, elapsed = 0, 0.0
+    while reps == 0 or elapsed < budget_s:
+        t0 = time.perf_counter()
+        o.step(st, d["q"], d["k"], d["v"], d["beta"], d["gate"], units=units)
+        elapsed += time.perf_counter() - t0
+        reps += 1
+    state_bytes = reps * len(units) * STATE_BYTES_PER_HEAD * 2
+    return dict(value=state_bytes / elapsed / 1e9, unit=UNIT, cores=1, kind="oracle",
+                sample=(f"{reps} pass(es) of the fp64 C oracle over {len(units)} of "
+                        f"{total_units} value-head units of {name}, single thread, "
+                        f"{elapsed:.1f} s"),
+                seconds=elapsed, units=int(len(units)), reps=reps)
+
+
+# --------------------------------------------------------------------------
+# arms
+# --------------------------------------------------------------------------
+def config_block(n_sets: int, set_bytes: int) -> Dict[str, object]:
+    return {"workload": HEADLINE, "L": 1, "B": 64, "Hk": 16, "Hv": 32, "dk": 128, "dv": 128,
+            "state_bytes": 64 * 32 * STATE_BYTES_PER_HEAD,
+            "l2": f"rotating {n_sets} input sets of {set_bytes / 2**20:.0f} MiB "
+                  f"(> 4x the 126 MB L2)",
+            "parallelism": "independent batches per rank"}
+
+
+def run_reference(args) -> int:
+    env = dist_env()
+    if env["rank"] != 0:
+        return 0
+    n_steps = args.steps + args.warmup
+    # size each step so the whole run stays within about two minutes
+    probe = cpu_oracle_baseline(HEADLINE, 0.0, max_units=64)
+    per_unit = probe["seconds"] / probe["units"]
+    units = int(max(1, min(2048, 120.0 / max(n_steps, 1) / per_unit)))
+    import oracle
+    from linear_attention_recurrence_04_b200 import inputs
+    o = oracle.load()
+    w = inputs.WORKLOADS[HEADLINE]
+    d = inputs.decode_inputs(1, 64, seed=w.seed)
+    sel = np.arange(units)
+    st = d["state"]
+    for _ in range(args.warmup):
+        st, _out = o.step(st, d["q"], d["k"], d["v"], d["beta"], d["gate"], units=sel)
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        st, _out = o.step(st, d["q"], d["k"], d["v"], d["beta"], d["gate"], units=sel)
+    secs = time.perf_counter() - t0
+    value = args.steps * units * STATE_BYTES_PER_HEAD * 2 / secs / 1e9
+    sample = (f"each step: the fp64 C oracle over {units} of 2048 value-head units of "
+              f"{HEADLINE}, single thread")
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": env["world"],
+        "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": secs / max(args.steps, 1) * 1e3, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": config_block(1, 0) | {"l2": "n/a (host)"}, "impl": "reference",
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": 1, "kind": "oracle",
+                         "sample": sample},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def run_ours(args) -> int:
+    import torch
+    import torch.distributed as dist
+    from datetime import timedelta
+    from linear_attention_recurrence_04_b200 import gdn
+
+    env = dist_env()
+    if not torch.cuda.is_available():
+        raise SystemExit("bench.py needs a CUDA device (there is no CPU path)")
+    torch.cuda.set_device(env["local_rank"])
+    device = torch.device("cuda", env["local_rank"])
+    gdn.load_library()
+    if env["world"] > 1:
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120),
+                                device_id=device)
+
+    def barrier():
+        if env["world"] > 1:
+            dist.barrier(device_ids=[env["local_rank"]])
+
+    # ---- headline: device-resident gdn_step, B = 64 -------------------
+    res = bench_step_workload(HEADLINE, 0, args.warmup, device,
+                              seed_offset=rank_seed(0, env["rank"]))
+    sets, outs = res["sets"], res["outs"]
+    n_sets = res["n_sets"]
+    stream = torch.cuda.current_stream(device)
+
+    def launch(i):
+        s = sets[i]
+        gdn.step(s["state"], s["q"], s["k"], s["v"], s["beta"], s["gate"], outs[i])
+
+    # the K timed launches, captured once into a CUDA graph (no host launch
+    # overhead inside the timed region); the same K launches eager, for reference
+    graph = capture([(lambda j=j: launch(j % n_sets)) for j in range(args.steps)], device)
+    torch.cuda.synchronize()
+    start = torch.cuda.Event(enable_timing=True)
+    end = torch.cuda.Event(enable_timing=True)
+    barrier()
+    torch.cuda.synchronize()
+    with ClockSampler(env["local_rank"]) as clocks:
+        start.record(stream)
+        graph.replay()
+        end.record(stream)
+        torch.cuda.synchronize()
+    barrier()
+    secs = max_over_ranks(start.elapsed_time(end) / 1e3, device)
+    del graph
+    eager_secs = max_over_ranks(time_launches(launch, n_sets, args.steps, 3, stream), device)
+    per_launch = secs / max(args.steps, 1)
+    state_total = res["state_bytes"] * args.steps
+    value = throughput(state_total / 1e9, env["world"], secs)
+    tokens_per_s = throughput(res["layer_tokens"] * args.steps, env["world"], secs)
+    peaks = measured_peaks()
+    achieved = res["bytes"] / per_launch / 1e9
+    digest = kernel_source_digest(["gdn_step.cu", "gdn_common.cuh"])
+
+    # ---- end to end through the C ABI with host buffers --------------
+    e2e_steps = max(args.steps, 1)
+    barrier()
+    e2e_secs, h2d, d2h = bench_e2e(res["d"], e2e_steps, args.warmup, device)
+    e2e_secs = max_over_ranks(e2e_secs, device)
+    e2e_value = throughput(res["state_bytes"] * e2e_steps / 1e9, env["world"], e2e_secs)
+    del sets, outs, res["sets"], res["outs"]
+    torch.cuda.empty_cache()
+
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": env["world"],
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": per_launch * 1e3,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
+        "data": "synthetic (seeded numpy draws: state N(0,0.05^2), unit q/k, v N(0,1), "
+                "beta sigmoid(N(0,1)), gate U(-1,0))",
+        "config": config_block(n_sets, res["set_bytes"]),
+        "layer_tokens_per_s": tokens_per_s,
+        "timing": "CUDA graph of the K launches, replayed once between CUDA events",
+        "eager_ms_per_step": eager_secs / max(args.steps, 1) * 1e3,
+        "hbm_frac_of_measured": achieved / peaks["hbm_gbs"],
+        "hbm_frac_of_8tbs_nominal": achieved / 8000.0,
+        "roofline": {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"],
+                     "peak_source": peaks["source"], "unit": "GB/s",
+                     "frac": achieved / peaks["hbm_gbs"],
+                     "traffic": stored_traffic("gdn_step", digest),
+                     "algorithmic_bytes_per_launch": res["bytes"],
+                     "kernel": "gdn::step_kernel", "kernel_source_digest": digest},
+        "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d,
+                "d2h_bytes_per_step": d2h},
+        "gpu_launches": args.steps,
+        "clocks": clocks.summary(),
+    }
+
+    if env["world"] == 1 and not args.no_extras:
+        extras = {}
+        r0 = bench_step_workload("decode_l1_b1", 2000, 50, device)
+        extras["decode_l1_b1"] = _step_extra(r0, 2000, peaks)
+        del r0
+        r2 = bench_step_workload("decode_l36_b16", 20, 3, device)
+        extras["decode_l36_b16"] = _step_extra(r2, 20, peaks)
+        del r2
+        torch.cuda.empty_cache()
+        p = bench_prefill(5, 3, device)
+        alu_peak = 148 * 128 * 2 * (line["clocks"]["sm_max_mhz"] or 1965) * 1e6 / 1e12
+        extras["prefill_b4_t4096"] = {
+            "ms_per_launch": p["seconds"] / p["launches"] * 1e3,
+            "tokens_per_s": p["tokens"] * p["launches"] / p["seconds"],
+            "gb_s": p["bytes"] * p["launches"] / p["seconds"] / 1e9,
+            "fp32_tflops": p["flops"] * p["launches"] / p["seconds"] / 1e12,
+            "roofline": {"bound": "alu", "peak": alu_peak, "unit": "TFLOP/s",
+                         "frac": p["flops"] * p["launches"] / p["seconds"] / 1e12 / alu_peak},
+        }
+        torch.cuda.empty_cache()
+        lay = bench_layer(20, 3, device)
+        gbs = lay["bytes"] * lay["launches"] / lay["seconds"] / 1e9
+        extras["layer_decode_b256"] = {
+            "ms_per_launch": lay["seconds"] / lay["launches"] * 1e3,
+            "layer_tokens_per_s": lay["tokens"] * lay["launches"] / lay["seconds"],
+            "gb_s": gbs, "roofline": {"bound": "hbm", "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                                      "frac": gbs / peaks["hbm_gbs"]},
+        }
+        line["workloads"] = extras
+
+    if env["rank"] == 0 and env["world"] == 1 and not args.no_cpu_baseline:
+        cb = cpu_oracle_baseline(HEADLINE, args.cpu_budget)
+        line["cpu_baseline"] = {k: cb[k] for k in ("value", "unit", "cores", "kind", "sample")}
+
+    if env["world"] > 1:
+        barrier()
+        dist.destroy_process_group()
+    if env["rank"] == 0:
+        print(json.dumps(line), flush=True)
+    return 0
+
+
+def _step_extra(r, steps, peaks):
+    per = r["seconds"] / steps
+    gbs = r["bytes"] / per / 1e9
+    return {"ms_per_launch": per * 1e3, "state_gb_s": r["state_bytes"] / per / 1e9,
+            "layer_tokens_per_s": r["layer_tokens"] / per, "gb_s": gbs,
+            "roofline": {"bound": "hbm", "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                         "frac": gbs / peaks["hbm_gbs"]},
+            "l2": f"rotating {r['n_sets']} input sets"}
+
+
+def main(argv=None) -> int:
+    ap = argparse.ArgumentParser(description=__doc__.splitlines()[0])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=2000)
+    ap.add_argument("--warmup", type=int, default=100)
+    ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
+    ap.add_argument("--cpu-budget", type=float, default=10.0,
+                    help="seconds of CPU time for the oracle baseline sample")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-extras", action="store_true",
+                    help="skip the other four workloads (headline only)")
+    args = ap.parse_args(argv)
+    if args.warmup < 3:
+        ap.error("--warmup must be at least 3")
+    if args.impl == "reference":
+        return run_reference(args)
+    return run_ours(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,142 @@
+/*
+ * gdn.h -- C ABI of libgdn.so: the Gated DeltaNet recurrent-state update on
+ * NVIDIA B200 (sm_100a).
+ *
+ * The operation (page "Red Lite dev15c -- Gated DeltaNet recurrent-state
+ * parity", section "Pinned llama.cpp semantics"): for every value head h,
+ * with q and k taken from key head h % Hk and the fp32 state held transposed
+ * as M[j][i] = S[i][j] (row j = value index, i = key index), one token does
+ *   1. M *= exp(gate[h])
+ *   2. sk[j] = dot(M[j], k)
+ *   3. delta[j] = (v[j] - sk[j]) * beta[h]
+ *   4. M[j][i] += delta[j] * k[i]
+ *   5. out[j] = dot(M[j], q) / sqrt(dk)      (the updated state)
+ *
+ * Conventions shared by every entry point
+ *   - All tensors are dense, C-contiguous, row-major float32 in DEVICE
+ *     memory of the current CUDA device; no pointer may be a host pointer.
+ *   - The caller allocates and frees every buffer. The library allocates no
+ *     memory, never synchronises, and enqueues its kernels on `stream`
+ *     (a cudaStream_t; NULL means the legacy default stream). Results are
+ *     ready once the stream reaches that point.
+ *   - Supported geometry: dk = dv = 128, Hk >= 1, Hv a multiple of Hk,
+ *     conv kernel K = 4. Other values return GDN_ERR_UNSUPPORTED.
+ *   - `state` and `conv_ring` are updated in place and must not overlap any
+ *     other argument; `out` must not overlap any argument either
+ *     (GDN_ERR_ALIAS otherwise). Read-only inputs may share memory.
+ *   - Alignment: state, q, k, v, out, mixed_qkv, z, conv_ring and conv_w
+ *     must be 16-byte aligned; the per-head scalars (beta, gate, a, b,
+ *     A_log, dt_bias) and norm_w need 4-byte alignment.
+ *   - Arguments are checked on the host before anything is enqueued; on any
+ *     error nothing is written and nothing is launched. A problem with no
+ *     work (a zero size) returns GDN_OK without touching any pointer.
+ *   - Sizes are int64_t. Kernel faults are asynchronous and surface at the
+ *     caller's next synchronisation, as for any CUDA kernel.
+ *   - Thread safety: calls from several host threads are safe; calls that
+ *     update the same state buffer must be ordered by the caller.
+ */
+#ifndef GDN_H
+#define GDN_H
+
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum gdn_status {
+    GDN_OK = 0,
+    GDN_ERR_NULL = 1,        /* a required pointer is NULL                     */
+    GDN_ERR_SHAPE = 2,       /* a negative size, or Hv not a multiple of Hk    */
+    GDN_ERR_UNSUPPORTED = 3, /* dk, dv or K outside what the kernels implement */
+    GDN_ERR_ALIGN = 4,       /* a pointer violates the alignment rule above    */
+    GDN_ERR_OVERFLOW = 5,    /* an element count does not fit the index type   */
+    GDN_ERR_CUDA = 6,        /* the CUDA runtime refused the launch            */
+    GDN_ERR_ALIAS = 7        /* out, state or conv_ring overlaps an argument   */
+} gdn_status;
+
+/* Static English text for a status code (never NULL). */
+const char *gdn_status_string(int status);
+
+/* Text describing the last failed call on this host thread ("" if none).
+ * The pointer stays valid until the next call of this library on the same
+ * thread. */
+const char *gdn_last_error(void);
+
+/*
+ * gdn_step -- one decode token for L layers x B sequences x Hv value heads,
+ * in a single launch. Each (layer, sequence, value head) is an independent
+ * recurrence; value head h reads q/k of key head h % Hk.
+ * ("Red Lite dev15c -- Gated DeltaNet recurrent-state parity", section
+ * "Pinned llama.cpp semantics", steps 1-5.)
+ *
+ *   state [L][B][Hv][dv][dk]  in/out, transposed layout M[j][i]
+ *   q, k  [L][B][Hk][dk]      query and key (the kernel does not normalise)
+ *   v     [L][B][Hv][dv]
+ *   beta  [L][B][Hv]          write strength (used as given)
+ *   gate  [L][B][Hv]          log-decay: the state is scaled by exp(gate)
+ *   out   [L][B][Hv][dv]      out[j] = dot(M_new[j], q) / sqrt(dk)
+ */
+gdn_status gdn_step(float *state, const float *q, const float *k, const float *v,
+                    const float *beta, const float *gate, float *out,
+                    int64_t L, int64_t B, int64_t Hk, int64_t Hv, int64_t dk,
+                    int64_t dv, void *stream);
+
+/*
+ * gdn_prefill -- T positions per sequence, run in order: position t starts
+ * from the state left by position t-1, so the result equals T calls of
+ * gdn_step with L = 1. ("Module linear_core", entry "gdn_forward_batch":
+ * the recurrence runs sequentially over positions and is elementwise
+ * identical to the one-position path; steps as for gdn_step.)
+ *
+ *   state [B][Hv][dv][dk]  in: initial state, out: state after position T-1
+ *   q, k  [B][T][Hk][dk]
+ *   v     [B][T][Hv][dv]
+ *   beta, gate [B][T][Hv]
+ *   out   [B][T][Hv][dv]
+ */
+gdn_status gdn_prefill(float *state, const float *q, const float *k, const float *v,
+                       const float *beta, const float *gate, float *out,
+                       int64_t B, int64_t T, int64_t Hk, int64_t Hv, int64_t dk,
+                       int64_t dv, void *stream);
+
+/*
+ * gdn_layer_decode -- the single-token recurrent layer between the input
+ * projections and the output projection, fused in one launch
+ * ("Red Lite dev15e -- complete recurrent DeltaNet layer composition",
+ * opening list; stage order from "Red Lite dev15a -- DeltaNet projection
+ * field validation", section "Validation boundary"):
+ *   1. causal depthwise conv over the window (conv_ring[0..K-2], mixed_qkv),
+ *      oldest first, tap t of conv_w multiplying window[t], no bias; the
+ *      ring then holds (conv_ring[1..K-2], mixed_qkv): raw inputs, shifted;
+ *   2. SiLU; split into q [Hk][dk] | k [Hk][dk] | v [Hv][dv] (contiguous,
+ *      head-major);
+ *   3. q and k of each key head scaled by 1 / max(||x||_2, l2_eps);
+ *   4. beta = sigmoid(b), gate = -exp(A_log) * softplus(a + dt_bias);
+ *   5. the recurrence of gdn_step for every value head;
+ *   6. gated RMSNorm per value head:
+ *      out[j] = o[j] / sqrt(mean(o^2) + norm_eps) * norm_w[j] * SiLU(z[j]).
+ *
+ *   mixed_qkv [B][C], C = 2*Hk*dk + Hv*dv   pre-conv input of this token
+ *   z         [B][Hv*dv]                    output gate input
+ *   a, b      [B][Hv]                       raw decay / write-strength inputs
+ *   conv_ring [B][K-1][C]                   in/out; slot 0 is the oldest
+ *   conv_w    [C][K]
+ *   A_log, dt_bias [Hv]
+ *   norm_w    [dv]                          shared by all value heads
+ *   state     [B][Hv][dv][dk]               in/out
+ *   out       [B][Hv*dv]
+ */
+gdn_status gdn_layer_decode(const float *mixed_qkv, const float *z, const float *a,
+                            const float *b, float *conv_ring, const float *conv_w,
+                            const float *A_log, const float *dt_bias,
+                            const float *norm_w, float l2_eps, float norm_eps,
+                            float *state, float *out, int64_t B, int64_t Hk,
+                            int64_t Hv, int64_t dk, int64_t dv, int64_t K,
+                            void *stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* GDN_H */

@@ -1,0 +1,270 @@
+// gdn_api.cu -- the extern "C" entry points of libgdn.so (declared in
+// include/gdn.h): host-side argument checks, then one kernel launch each.
+#include <atomic>
+#include <cstdarg>
+#include <cstdint>
+#include <cstdio>
+#include <cstring>
+
+#include <cuda_runtime.h>
+
+#include "gdn.h"
+#include "gdn_common.cuh"
+#include "gdn_internal.h"
+
+namespace gdn {
+
+namespace {
+
+thread_local char g_last_error[512] = "";
+
+gdn_status fail(gdn_status st, const char* fmt, ...) {
+    va_list ap;
+    va_start(ap, fmt);
+    vsnprintf(g_last_error, sizeof(g_last_error), fmt, ap);
+    va_end(ap);
+    return st;
+}
+
+constexpr int kMaxDevices = 64;
+std::atomic<int> g_sm_count[kMaxDevices];
+
+// Checked product of non-negative sizes; false on overflow of int64.
+bool mul_ok(int64_t a, int64_t b, int64_t* r) {
+    if (a < 0 || b < 0) return false;
+    if (a != 0 && b > INT64_MAX / a) return false;
+    *r = a * b;
+    return true;
+}
+
+struct Span {
+    const void* p;
+    int64_t bytes;
+    const char* name;
+};
+
+bool overlaps(const Span& x, const Span& y) {
+    if (!x.p || !y.p || x.bytes == 0 || y.bytes == 0) return false;
+    const uintptr_t a0 = reinterpret_cast<uintptr_t>(x.p), a1 = a0 + x.bytes;
+    const uintptr_t b0 = reinterpret_cast<uintptr_t>(y.p), b1 = b0 + y.bytes;
+    return a0 < b1 && b0 < a1;
+}
+
+bool aligned(const void* p, uintptr_t n) { return (reinterpret_cast<uintptr_t>(p) % n) == 0; }
+
+gdn_status check_geometry(int64_t Hk, int64_t Hv, int64_t dk, int64_t dv) {
+    if (Hk <= 0 || Hv <= 0) return fail(GDN_ERR_SHAPE, "Hk=%lld and Hv=%lld must be positive",
+                                        (long long)Hk, (long long)Hv);
+    if (Hv % Hk != 0) return fail(GDN_ERR_SHAPE, "Hv=%lld is not a multiple of Hk=%lld",
+                                  (long long)Hv, (long long)Hk);
+    if (dk != kDk || dv != kDv)
+        return fail(GDN_ERR_UNSUPPORTED, "dk=%lld dv=%lld: only dk = dv = 128 is implemented",
+                    (long long)dk, (long long)dv);
+    if (Hv > (1 << 20)) return fail(GDN_ERR_OVERFLOW, "Hv=%lld is too large", (long long)Hv);
+    return GDN_OK;
+}
+
+// `out` must not overlap anything; a buffer updated in place (the first
+// `n_inplace` entries of `in`) must not overlap any other entry either.
+gdn_status check_spans(const Span* in, int n_in, int n_inplace, const Span& out) {
+    for (int i = 0; i < n_in; ++i)
+        if (overlaps(in[i], out))
+            return fail(GDN_ERR_ALIAS, "out overlaps %s", in[i].name);
+    for (int i = 0; i < n_inplace; ++i)
+        for (int j = 0; j < n_in; ++j)
+            if (j != i && overlaps(in[i], in[j]))
+                return fail(GDN_ERR_ALIAS, "%s (updated in place) overlaps %s", in[i].name,
+                            in[j].name);
+    return GDN_OK;
+}
+
+gdn_status launched(cudaError_t err, const char* what) {
+    if (err != cudaSuccess)
+        return fail(GDN_ERR_CUDA, "%s: %s (%s)", what, cudaGetErrorString(err),
+                    cudaGetErrorName(err));
+    g_last_error[0] = '\0';
+    return GDN_OK;
+}
+
+}  // namespace
+
+int device_sm_count() {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0) return 148;
+    if (dev < kMaxDevices) {
+        const int cached = g_sm_count[dev].load(std::memory_order_relaxed);
+        if (cached > 0) return cached;
+    }
+    int n = 0;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0)
+        n = 148;
+    if (dev < kMaxDevices) g_sm_count[dev].store(n, std::memory_order_relaxed);
+    return n;
+}
+
+namespace {
+
+struct OccEntry {
+    std::atomic<const void*> kernel{nullptr};
+    std::atomic<int> threads{0};
+    std::atomic<int> per_sm{0};
+};
+constexpr int kOccSlots = 16;
+OccEntry g_occ[kMaxDevices][kOccSlots];
+
+}  // namespace
+
+cudaError_t resident_ctas_per_sm(const void* kernel, int threads, int* per_sm) {
+    int dev = 0;
+    cudaError_t err = cudaGetDevice(&dev);
+    if (err != cudaSuccess) return err;
+    if (dev >= 0 && dev < kMaxDevices) {
+        for (int i = 0; i < kOccSlots; ++i) {
+            OccEntry& e = g_occ[dev][i];
+            if (e.kernel.load(std::memory_order_acquire) == kernel &&
+                e.threads.load(std::memory_order_relaxed) == threads) {
+                const int v = e.per_sm.load(std::memory_order_relaxed);
+                if (v > 0) { *per_sm = v; return cudaSuccess; }
+            }
+        }
+    }
+    int n = 0;
+    err = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, kernel, threads, 0);
+    if (err != cudaSuccess) return err;
+    if (n < 1) n = 1;
+    *per_sm = n;
+    if (dev >= 0 && dev < kMaxDevices) {
+        for (int i = 0; i < kOccSlots; ++i) {
+            OccEntry& e = g_occ[dev][i];
+            const void* expected = nullptr;
+            if (e.kernel.compare_exchange_strong(expected, kernel, std::memory_order_acq_rel) ||
+                expected == kernel) {
+                e.threads.store(threads, std::memory_order_relaxed);
+                e.per_sm.store(n, std::memory_order_relaxed);
+                break;
+            }
+        }
+    }
+    return cudaSuccess;
+}
+
+}  // namespace gdn
+
+using namespace gdn;
+
+extern "C" {
+
+const char* gdn_status_string(int status) {
+    switch (status) {
+        case GDN_OK: return "ok";
+        case GDN_ERR_NULL: return "a required pointer is NULL";
+        case GDN_ERR_SHAPE: return "invalid shape";
+        case GDN_ERR_UNSUPPORTED: return "unsupported geometry";
+        case GDN_ERR_ALIGN: return "misaligned pointer";
+        case GDN_ERR_OVERFLOW: return "size overflow";
+        case GDN_ERR_CUDA: return "CUDA launch error";
+        case GDN_ERR_ALIAS: return "output overlaps an input";
+        default: return "unknown status";
+    }
+}
+
+const char* gdn_last_error(void) { return g_last_error; }
+
+gdn_status gdn_step(float* state, const float* q, const float* k, const float* v,
+                    const float* beta, const float* gate, float* out, int64_t L, int64_t B,
+                    int64_t Hk, int64_t Hv, int64_t dk, int64_t dv, void* stream) {
+    if (L < 0 || B < 0) return fail(GDN_ERR_SHAPE, "negative L=%lld or B=%lld", (long long)L,
+                                    (long long)B);
+    gdn_status st = check_geometry(Hk, Hv, dk, dv);
+    if (st != GDN_OK) return st;
+    int64_t lb = 0, heads = 0, state_n = 0, qk_n = 0, v_n = 0;
+    if (!mul_ok(L, B, &lb) || !mul_ok(lb, Hv, &heads) || !mul_ok(heads, dv * dk, &state_n) ||
+        !mul_ok(lb, Hk * dk, &qk_n) || !mul_ok(heads, dv, &v_n) || state_n > INT64_MAX / 8)
+        return fail(GDN_ERR_OVERFLOW, "L*B*Hv*dv*dk overflows int64");
+    if (heads == 0) { g_last_error[0] = '\0'; return GDN_OK; }
+    if (!state || !q || !k || !v || !beta || !gate || !out)
+        return fail(GDN_ERR_NULL, "gdn_step: a tensor pointer is NULL");
+    if (!aligned(state, 16) || !aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) ||
+        !aligned(out, 16) || !aligned(beta, 4) || !aligned(gate, 4))
+        return fail(GDN_ERR_ALIGN, "gdn_step: state/q/k/v/out need 16-byte, beta/gate 4-byte alignment");
+    const Span ins[] = {{state, state_n * 4, "state"}, {q, qk_n * 4, "q"}, {k, qk_n * 4, "k"},
+                        {v, v_n * 4, "v"}, {beta, heads * 4, "beta"}, {gate, heads * 4, "gate"}};
+    st = check_spans(ins, 6, 1, Span{out, v_n * 4, "out"});
+    if (st != GDN_OK) return st;
+    StepArgs a{state, q, k, v, beta, gate, out, heads, static_cast<int>(Hk), static_cast<int>(Hv)};
+    return launched(launch_step(a, static_cast<cudaStream_t>(stream)), "gdn_step");
+}
+
+gdn_status gdn_prefill(float* state, const float* q, const float* k, const float* v,
+                       const float* beta, const float* gate, float* out, int64_t B, int64_t T,
+                       int64_t Hk, int64_t Hv, int64_t dk, int64_t dv, void* stream) {
+    if (B < 0 || T < 0) return fail(GDN_ERR_SHAPE, "negative B=%lld or T=%lld", (long long)B,
+                                    (long long)T);
+    gdn_status st = check_geometry(Hk, Hv, dk, dv);
+    if (st != GDN_OK) return st;
+    int64_t bt = 0, heads = 0, state_n = 0, qk_n = 0, v_n = 0, bh = 0;
+    if (!mul_ok(B, T, &bt) || !mul_ok(B, Hv, &heads) || !mul_ok(heads, dv * dk, &state_n) ||
+        !mul_ok(bt, Hk * dk, &qk_n) || !mul_ok(bt, Hv * dv, &v_n) || !mul_ok(bt, Hv, &bh) ||
+        v_n > INT64_MAX / 8 || qk_n > INT64_MAX / 8)
+        return fail(GDN_ERR_OVERFLOW, "B*T*Hv*dv overflows int64");
+    // One warp per 8 rows of a head pair; the grid must fit gridDim.x.
+    if (heads * (kDv / 8) > INT32_MAX)
+        return fail(GDN_ERR_OVERFLOW, "B*Hv=%lld exceeds the launch grid", (long long)heads);
+    if (bt == 0 || heads == 0) { g_last_error[0] = '\0'; return GDN_OK; }
+    if (!state || !q || !k || !v || !beta || !gate || !out)
+        return fail(GDN_ERR_NULL, "gdn_prefill: a tensor pointer is NULL");
+    if (!aligned(state, 16) || !aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) ||
+        !aligned(out, 16) || !aligned(beta, 4) || !aligned(gate, 4))
+        return fail(GDN_ERR_ALIGN, "gdn_prefill: state/q/k/v/out need 16-byte, beta/gate 4-byte alignment");
+    const Span ins[] = {{state, state_n * 4, "state"}, {q, qk_n * 4, "q"}, {k, qk_n * 4, "k"},
+                        {v, v_n * 4, "v"}, {beta, bh * 4, "beta"}, {gate, bh * 4, "gate"}};
+    st = check_spans(ins, 6, 1, Span{out, v_n * 4, "out"});
+    if (st != GDN_OK) return st;
+    PrefillArgs a{state, q, k, v, beta, gate, out, B, T, static_cast<int>(Hk), static_cast<int>(Hv)};
+    return launched(launch_prefill(a, static_cast<cudaStream_t>(stream)), "gdn_prefill");
+}
+
+gdn_status gdn_layer_decode(const float* mixed_qkv, const float* z, const float* a,
+                            const float* b, float* conv_ring, const float* conv_w,
+                            const float* A_log, const float* dt_bias, const float* norm_w,
+                            float l2_eps, float norm_eps, float* state, float* out, int64_t B,
+                            int64_t Hk, int64_t Hv, int64_t dk, int64_t dv, int64_t K,
+                            void* stream) {
+    if (B < 0) return fail(GDN_ERR_SHAPE, "negative B=%lld", (long long)B);
+    gdn_status st = check_geometry(Hk, Hv, dk, dv);
+    if (st != GDN_OK) return st;
+    if (K != kConvK) return fail(GDN_ERR_UNSUPPORTED, "K=%lld: only a conv kernel of 4 is implemented",
+                                 (long long)K);
+    if (!layer_decode_supports(static_cast<int>(Hv / Hk)))
+        return fail(GDN_ERR_UNSUPPORTED, "Hv/Hk=%lld: the fused layer supports 1, 2 or 4",
+                    (long long)(Hv / Hk));
+    const int64_t C = 2 * Hk * dk + Hv * dv;
+    int64_t x_n = 0, z_n = 0, bh = 0, ring_n = 0, state_n = 0, grid = 0;
+    if (!mul_ok(B, C, &x_n) || !mul_ok(B, Hv * dv, &z_n) || !mul_ok(B, Hv, &bh) ||
+        !mul_ok(x_n, K - 1, &ring_n) || !mul_ok(bh, dv * dk, &state_n) || !mul_ok(B, Hk, &grid) ||
+        state_n > INT64_MAX / 8 || ring_n > INT64_MAX / 8)
+        return fail(GDN_ERR_OVERFLOW, "B*Hv*dv*dk overflows int64");
+    if (grid > INT32_MAX) return fail(GDN_ERR_OVERFLOW, "B*Hk=%lld exceeds the launch grid",
+                                      (long long)grid);
+    if (B == 0) { g_last_error[0] = '\0'; return GDN_OK; }
+    if (!mixed_qkv || !z || !a || !b || !conv_ring || !conv_w || !A_log || !dt_bias || !norm_w ||
+        !state || !out)
+        return fail(GDN_ERR_NULL, "gdn_layer_decode: a tensor pointer is NULL");
+    if (!aligned(mixed_qkv, 16) || !aligned(z, 16) || !aligned(conv_ring, 16) ||
+        !aligned(conv_w, 16) || !aligned(state, 16) || !aligned(out, 16) || !aligned(a, 4) ||
+        !aligned(b, 4) || !aligned(A_log, 4) || !aligned(dt_bias, 4) || !aligned(norm_w, 4))
+        return fail(GDN_ERR_ALIGN, "gdn_layer_decode: alignment rule violated");
+    const Span ins[] = {{state, state_n * 4, "state"}, {conv_ring, ring_n * 4, "conv_ring"},
+                        {mixed_qkv, x_n * 4, "mixed_qkv"}, {z, z_n * 4, "z"}, {a, bh * 4, "a"},
+                        {b, bh * 4, "b"}, {conv_w, C * K * 4, "conv_w"},
+                        {A_log, Hv * 4, "A_log"}, {dt_bias, Hv * 4, "dt_bias"},
+                        {norm_w, dv * 4, "norm_w"}};
+    st = check_spans(ins, 10, 2, Span{out, z_n * 4, "out"});
+    if (st != GDN_OK) return st;
+    LayerArgs args{mixed_qkv, z, a, b, conv_ring, conv_w, A_log, dt_bias, norm_w, l2_eps,
+                   norm_eps, state, out, B, static_cast<int>(Hk), static_cast<int>(Hv)};
+    return launched(launch_layer_decode(args, static_cast<cudaStream_t>(stream)),
+                    "gdn_layer_decode");
+}
+
+}  // extern "C"

@@ -1,0 +1,71 @@
+// gdn_internal.h -- launchers behind the C ABI (not exported).
+#pragma once
+
+#include <cstdint>
+#include <cuda_runtime.h>
+
+namespace gdn {
+
+struct StepArgs {
+    float* state;
+    const float* q;
+    const float* k;
+    const float* v;
+    const float* beta;
+    const float* gate;
+    float* out;
+    int64_t n_heads;   // L * B * Hv
+    int Hk;
+    int Hv;
+};
+
+struct PrefillArgs {
+    float* state;
+    const float* q;
+    const float* k;
+    const float* v;
+    const float* beta;
+    const float* gate;
+    float* out;
+    int64_t B;
+    int64_t T;
+    int Hk;
+    int Hv;
+};
+
+struct LayerArgs {
+    const float* mixed_qkv;
+    const float* z;
+    const float* a;
+    const float* b;
+    float* conv_ring;
+    const float* conv_w;
+    const float* A_log;
+    const float* dt_bias;
+    const float* norm_w;
+    float l2_eps;
+    float norm_eps;
+    float* state;
+    float* out;
+    int64_t B;
+    int Hk;
+    int Hv;
+};
+
+// Each launcher enqueues its kernel on `stream` and returns the launch status.
+cudaError_t launch_step(const StepArgs& a, cudaStream_t stream);
+cudaError_t launch_prefill(const PrefillArgs& a, cudaStream_t stream);
+cudaError_t launch_layer_decode(const LayerArgs& a, cudaStream_t stream);
+
+// Value-heads-per-key-head ratios the fused layer kernel is compiled for.
+bool layer_decode_supports(int G);
+
+// Number of SMs of the current device, cached per device.
+int device_sm_count();
+
+// Resident CTAs per SM of `kernel` at `threads` threads and no dynamic shared
+// memory on the current device (at least 1), cached per (device, kernel) so a
+// launch inside stream capture makes no occupancy query.
+cudaError_t resident_ctas_per_sm(const void* kernel, int threads, int* per_sm);
+
+}  // namespace gdn

@@ -1,0 +1,153 @@
+// gdn_step.cu -- batched single-token Gated DeltaNet decode.
+//
+// Page "Red Lite dev15c -- Gated DeltaNet recurrent-state parity", section
+// "Pinned llama.cpp semantics": per value head h (q/k of key head h % Hk),
+// with M[j][i] = S[i][j],
+//   1. M *= exp(gate)   2. sk[j] = M[j].k   3. delta[j] = (v[j] - sk[j]) beta
+//   4. M[j] += delta[j] k   5. out[j] = M_new[j].q / sqrt(128).
+//
+// Design: every row j of M is independent once k, q, v[j], beta and gate are
+// known, so the kernel streams rows. A warp owns R consecutive rows of one
+// head; lane l holds columns [4l, 4l+4) of each row as one float4, so a row
+// is one coalesced 512-byte access. All R row loads are issued before any
+// arithmetic, the five steps run in registers (two warp-shuffle reductions
+// per row), and each row is written back once: the state crosses HBM exactly
+// once in each direction per token. Warps walk row groups with a grid-stride
+// loop over a persistent grid of (SMs x resident CTAs), prefetching the next
+// group's rows while the current group computes.
+#include "gdn_common.cuh"
+#include "gdn_internal.h"
+
+#ifndef GDN_STEP_ROWS
+#define GDN_STEP_ROWS 8          // rows per warp task
+#endif
+#ifndef GDN_STEP_THREADS
+#define GDN_STEP_THREADS 256     // threads per CTA
+#endif
+#ifndef GDN_STEP_PREFETCH
+#define GDN_STEP_PREFETCH 1      // load the next task's rows before computing
+#endif
+
+namespace gdn {
+
+namespace {
+
+template <int R>
+struct RowTask {
+    int64_t head;   // flat (layer, sequence, value head)
+    int row0;       // first row j of the task
+};
+
+template <int R>
+__device__ __forceinline__ RowTask<R> decode_task(int64_t task) {
+    constexpr int kTasksPerHead = kDv / R;
+    RowTask<R> t;
+    t.head = task / kTasksPerHead;
+    t.row0 = static_cast<int>(task - t.head * kTasksPerHead) * R;
+    return t;
+}
+
+template <int R>
+__device__ __forceinline__ void load_rows(float4 (&m)[R], const float* state, RowTask<R> t,
+                                          int lane) {
+    const float* rows = state + (t.head * kDv + t.row0) * kDk + lane * 4;
+#pragma unroll
+    for (int r = 0; r < R; ++r) m[r] = ld_stream(rows + r * kDk);
+}
+
+// Steps 1-5 on R rows held in registers; writes the rows and R outputs.
+template <int R>
+__device__ __forceinline__ void update_rows(float4 (&m)[R], float* __restrict__ state,
+                                            const float* __restrict__ q,
+                                            const float* __restrict__ k,
+                                            const float* __restrict__ v,
+                                            const float* __restrict__ beta,
+                                            const float* __restrict__ gate,
+                                            float* __restrict__ out, RowTask<R> t, int Hk,
+                                            int Hv, int lane) {
+    const int64_t lb = t.head / Hv;
+    const int h = static_cast<int>(t.head - lb * Hv);
+    const int64_t key = (lb * Hk + (h % Hk)) * kDk + lane * 4;
+    const float4 k4 = ld_ro4(k + key);
+    const float4 q4 = ld_ro4(q + key);
+    const float decay = expf(gate[t.head]);
+    const float bt = beta[t.head];
+    const int64_t vrow = t.head * kDv + t.row0;
+    const float v_lane = lane < R ? v[vrow + lane] : 0.0f;
+    float* rows = state + vrow * kDk + lane * 4;
+    float o_lane = 0.0f;
+#pragma unroll
+    for (int r = 0; r < R; ++r) {
+        float4 x = m[r];
+        // step 1: decay
+        x.x *= decay; x.y *= decay; x.z *= decay; x.w *= decay;
+        // step 2: sk = M[j].k on the decayed row
+        const float sk = warp_sum(dot4(x, k4));
+        // step 3: delta
+        const float delta = (__shfl_sync(kFull, v_lane, r) - sk) * bt;
+        // step 4: rank-1 update
+        x.x = fmaf(delta, k4.x, x.x);
+        x.y = fmaf(delta, k4.y, x.y);
+        x.z = fmaf(delta, k4.z, x.z);
+        x.w = fmaf(delta, k4.w, x.w);
+        // step 5: output from the updated row
+        const float o = warp_sum(dot4(x, q4)) * kOutScale;
+        if (lane == r) o_lane = o;
+        st_stream(rows + r * kDk, x);
+    }
+    if (lane < R) out[vrow + lane] = o_lane;
+}
+
+template <int R>
+__global__ void __launch_bounds__(GDN_STEP_THREADS)
+step_kernel(float* __restrict__ state, const float* __restrict__ q, const float* __restrict__ k,
+            const float* __restrict__ v, const float* __restrict__ beta,
+            const float* __restrict__ gate, float* __restrict__ out, int64_t n_tasks, int Hk,
+            int Hv) {
+    const int lane = threadIdx.x & 31;
+    const int64_t warps_per_cta = blockDim.x >> 5;
+    const int64_t stride = static_cast<int64_t>(gridDim.x) * warps_per_cta;
+    int64_t task = static_cast<int64_t>(blockIdx.x) * warps_per_cta + (threadIdx.x >> 5);
+    if (task >= n_tasks) return;
+    float4 m[R];
+    load_rows<R>(m, state, decode_task<R>(task), lane);
+    for (; task < n_tasks; task += stride) {
+        const RowTask<R> cur = decode_task<R>(task);
+#if GDN_STEP_PREFETCH
+        float4 nxt[R];
+        const bool more = task + stride < n_tasks;
+        if (more) load_rows<R>(nxt, state, decode_task<R>(task + stride), lane);
+        update_rows<R>(m, state, q, k, v, beta, gate, out, cur, Hk, Hv, lane);
+        if (more) {
+#pragma unroll
+            for (int r = 0; r < R; ++r) m[r] = nxt[r];
+        }
+#else
+        update_rows<R>(m, state, q, k, v, beta, gate, out, cur, Hk, Hv, lane);
+        if (task + stride < n_tasks) load_rows<R>(m, state, decode_task<R>(task + stride), lane);
+#endif
+    }
+}
+
+}  // namespace
+
+cudaError_t launch_step(const StepArgs& a, cudaStream_t stream) {
+    constexpr int R = GDN_STEP_ROWS;
+    static_assert(kDv % R == 0 && R <= 32, "rows per task must divide dv");
+    const int64_t n_tasks = a.n_heads * (kDv / R);
+    if (n_tasks == 0) return cudaSuccess;
+    constexpr int threads = GDN_STEP_THREADS;
+    constexpr int warps_per_cta = threads / 32;
+    int per_sm = 0;
+    cudaError_t err = resident_ctas_per_sm(reinterpret_cast<const void*>(&step_kernel<R>),
+                                           threads, &per_sm);
+    if (err != cudaSuccess) return err;
+    const int64_t needed = (n_tasks + warps_per_cta - 1) / warps_per_cta;
+    const int64_t resident = static_cast<int64_t>(device_sm_count()) * per_sm;
+    const int grid = static_cast<int>(needed < resident ? needed : resident);
+    step_kernel<R><<<grid, threads, 0, stream>>>(a.state, a.q, a.k, a.v, a.beta, a.gate, a.out,
+                                                 n_tasks, a.Hk, a.Hv);
+    return cudaGetLastError();
+}
+
+}  // namespace gdn

@@ -1,0 +1,193 @@
+"""ctypes binding of ``libgdn.so`` (C ABI in ``include/gdn.h``).
+
+Argument marshalling only: each function checks that the torch tensors are
+float32, contiguous and on one CUDA device, passes their device pointers and
+the current stream to the C entry point of the same name, and raises
+``GdnError`` on a non-zero status. Every step of the computation runs in the
+library's CUDA kernels. There is no CPU path: if the library is missing the
+first call raises.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional, Sequence
+
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+_LIB_NAME = "libgdn.so"
+
+_VP = ctypes.c_void_p
+_I64 = ctypes.c_int64
+_F32 = ctypes.c_float
+
+STATUS = {
+    0: "GDN_OK", 1: "GDN_ERR_NULL", 2: "GDN_ERR_SHAPE", 3: "GDN_ERR_UNSUPPORTED",
+    4: "GDN_ERR_ALIGN", 5: "GDN_ERR_OVERFLOW", 6: "GDN_ERR_CUDA", 7: "GDN_ERR_ALIAS",
+}
+
+# Every symbol that include/gdn.h declares.
+EXPORTS = ("gdn_status_string", "gdn_last_error", "gdn_step", "gdn_prefill", "gdn_layer_decode")
+
+
+class GdnError(RuntimeError):
+    """A non-zero gdn_status from the library."""
+
+    def __init__(self, func: str, status: int, detail: str):
+        self.status = status
+        self.code = STATUS.get(status, str(status))
+        super().__init__(f"{func}: {self.code}: {detail}")
+
+
+_lib: Optional[ctypes.CDLL] = None
+
+
+def library_path() -> str:
+    return os.environ.get("GDN_LIBRARY", os.path.join(_PKG, _LIB_NAME))
+
+
+def load_library(path: Optional[str] = None) -> ctypes.CDLL:
+    """Load (once) and return the library; raises if it has not been built."""
+    global _lib
+    if _lib is not None and path is None:
+        return _lib
+    p = path or library_path()
+    if not os.path.exists(p):
+        raise FileNotFoundError(
+            f"{p} is missing: build it with `python -m linear_attention_recurrence_04_b200.build`"
+            " (there is no CPU fallback)")
+    lib = ctypes.CDLL(p)
+    lib.gdn_status_string.restype = ctypes.c_char_p
+    lib.gdn_status_string.argtypes = [ctypes.c_int]
+    lib.gdn_last_error.restype = ctypes.c_char_p
+    lib.gdn_last_error.argtypes = []
+    lib.gdn_step.restype = ctypes.c_int
+    lib.gdn_step.argtypes = [_VP] * 7 + [_I64] * 6 + [_VP]
+    lib.gdn_prefill.restype = ctypes.c_int
+    lib.gdn_prefill.argtypes = [_VP] * 7 + [_I64] * 6 + [_VP]
+    lib.gdn_layer_decode.restype = ctypes.c_int
+    lib.gdn_layer_decode.argtypes = [_VP] * 9 + [_F32, _F32] + [_VP, _VP] + [_I64] * 6 + [_VP]
+    if path is None:
+        _lib = lib
+    return lib
+
+
+def status_string(status: int) -> str:
+    return load_library().gdn_status_string(int(status)).decode()
+
+
+def _raise_on(func: str, status: int) -> None:
+    if status != 0:
+        lib = load_library()
+        raise GdnError(func, status, lib.gdn_last_error().decode())
+
+
+def _dev(tensors: Sequence[torch.Tensor], names: Sequence[str]) -> torch.device:
+    device = tensors[0].device
+    for t, n in zip(tensors, names):
+        if not isinstance(t, torch.Tensor):
+            raise TypeError(f"{n} must be a torch.Tensor")
+        if t.dtype is not torch.float32:
+            raise TypeError(f"{n} must be float32, got {t.dtype}")
+        if not t.is_cuda:
+            raise ValueError(f"{n} must be a CUDA tensor")
+        if not t.is_contiguous():
+            raise ValueError(f"{n} must be contiguous")
+        if t.device != device:
+            raise ValueError(f"{n} is on {t.device}, expected {device}")
+    return device
+
+
+def _call(device: torch.device, fn, *args) -> int:
+    """Call `fn` with `device` current (switching only when it is not)."""
+    if torch.cuda.current_device() == device.index:
+        return fn(*args)
+    with torch.cuda.device(device):
+        return fn(*args)
+
+
+def _ptr(t: torch.Tensor) -> int:
+    return t.data_ptr() if t.numel() else 0
+
+
+def _stream(device: torch.device, stream: Optional[torch.cuda.Stream]) -> int:
+    s = stream if stream is not None else torch.cuda.current_stream(device)
+    return s.cuda_stream
+
+
+def step(state, q, k, v, beta, gate, out=None, *, stream=None):
+    """One decode token: state [L,B,Hv,128,128] (updated in place), q/k
+    [L,B,Hk,128], v [L,B,Hv,128], beta/gate [L,B,Hv]. Returns out [L,B,Hv,128]."""
+    if state.dim() != 5:
+        raise ValueError("state must be [L, B, Hv, dv, dk]")
+    L, B, Hv, dv, dk = state.shape
+    Hk = q.shape[2]
+    if out is None:
+        out = torch.empty((L, B, Hv, dv), dtype=torch.float32, device=state.device)
+    names = ("state", "q", "k", "v", "beta", "gate", "out")
+    tensors = (state, q, k, v, beta, gate, out)
+    device = _dev(tensors, names)
+    expect = dict(q=(L, B, Hk, dk), k=(L, B, Hk, dk), v=(L, B, Hv, dv), beta=(L, B, Hv),
+                  gate=(L, B, Hv), out=(L, B, Hv, dv))
+    for n, t in zip(names[1:], tensors[1:]):
+        if tuple(t.shape) != expect[n]:
+            raise ValueError(f"{n} has shape {tuple(t.shape)}, expected {expect[n]}")
+    st = _call(device, load_library().gdn_step, *(_ptr(t) for t in tensors), L, B, Hk, Hv, dk,
+               dv, _stream(device, stream))
+    _raise_on("gdn_step", st)
+    return out
+
+
+def prefill(state, q, k, v, beta, gate, out=None, *, stream=None):
+    """T positions in order: state [B,Hv,128,128] (initial -> final, in place),
+    q/k [B,T,Hk,128], v [B,T,Hv,128], beta/gate [B,T,Hv]. Returns out [B,T,Hv,128]."""
+    if state.dim() != 4:
+        raise ValueError("state must be [B, Hv, dv, dk]")
+    B, Hv, dv, dk = state.shape
+    T, Hk = q.shape[1], q.shape[2]
+    if out is None:
+        out = torch.empty((B, T, Hv, dv), dtype=torch.float32, device=state.device)
+    names = ("state", "q", "k", "v", "beta", "gate", "out")
+    tensors = (state, q, k, v, beta, gate, out)
+    device = _dev(tensors, names)
+    expect = dict(q=(B, T, Hk, dk), k=(B, T, Hk, dk), v=(B, T, Hv, dv), beta=(B, T, Hv),
+                  gate=(B, T, Hv), out=(B, T, Hv, dv))
+    for n, t in zip(names[1:], tensors[1:]):
+        if tuple(t.shape) != expect[n]:
+            raise ValueError(f"{n} has shape {tuple(t.shape)}, expected {expect[n]}")
+    st = _call(device, load_library().gdn_prefill, *(_ptr(t) for t in tensors), B, T, Hk, Hv,
+               dk, dv, _stream(device, stream))
+    _raise_on("gdn_prefill", st)
+    return out
+
+
+def layer_decode(mixed_qkv, z, a, b, conv_ring, conv_w, A_log, dt_bias, norm_w, state,
+                 out=None, *, Hk: int, l2_eps: float = 1e-6, norm_eps: float = 1e-6,
+                 stream=None):
+    """Fused prestate + recurrence + gated RMSNorm for one token per sequence.
+
+    mixed_qkv [B,C]; z [B,Hv*128]; a, b [B,Hv]; conv_ring [B,K-1,C] (in place);
+    conv_w [C,K]; A_log, dt_bias [Hv]; norm_w [128]; state [B,Hv,128,128]
+    (in place). Returns out [B,Hv*128]."""
+    if state.dim() != 4:
+        raise ValueError("state must be [B, Hv, dv, dk]")
+    B, Hv, dv, dk = state.shape
+    C, K = conv_w.shape
+    if out is None:
+        out = torch.empty((B, Hv * dv), dtype=torch.float32, device=state.device)
+    names = ("mixed_qkv", "z", "a", "b", "conv_ring", "conv_w", "A_log", "dt_bias", "norm_w",
+             "state", "out")
+    tensors = (mixed_qkv, z, a, b, conv_ring, conv_w, A_log, dt_bias, norm_w, state, out)
+    device = _dev(tensors, names)
+    expect = dict(mixed_qkv=(B, C), z=(B, Hv * dv), a=(B, Hv), b=(B, Hv),
+                  conv_ring=(B, K - 1, C), A_log=(Hv,), dt_bias=(Hv,), norm_w=(dv,),
+                  out=(B, Hv * dv))
+    for n, t in zip(names, tensors):
+        if n in expect and tuple(t.shape) != expect[n]:
+            raise ValueError(f"{n} has shape {tuple(t.shape)}, expected {expect[n]}")
+    ptrs = [_ptr(t) for t in tensors]
+    st = _call(device, load_library().gdn_layer_decode, *ptrs[:9], float(l2_eps),
+               float(norm_eps), ptrs[9], ptrs[10], B, Hk, Hv, dk, dv, K, _stream(device, stream))
+    _raise_on("gdn_layer_decode", st)
+    return out

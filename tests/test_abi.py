@@ -1,0 +1,123 @@
+"""The C ABI without a GPU: the library loads, exports every symbol that
+include/gdn.h declares, and rejects bad arguments on the host before any
+CUDA call (these calls never reach a launch)."""
+import ctypes
+import os
+import re
+import subprocess
+
+import pytest
+
+from linear_attention_recurrence_04_b200 import build as gdn_build
+from linear_attention_recurrence_04_b200 import gdn
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "gdn.h")
+
+OK, NULL, SHAPE, UNSUP, ALIGN, OVERFLOW, CUDA, ALIAS = range(8)
+
+
+@pytest.fixture(scope="module")
+def lib():
+    gdn_build.build()
+    return gdn.load_library()
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(gdn_[a-z_]+)\s*\(", text)))
+
+
+def test_header_declares_the_binding_exports():
+    assert declared_functions() == sorted(gdn.EXPORTS)
+
+
+def test_library_exports_every_declared_symbol(lib):
+    out = subprocess.run(["nm", "-D", "--defined-only", gdn.library_path()], check=True,
+                         capture_output=True, text=True).stdout
+    exported = {line.split()[-1] for line in out.splitlines() if line.strip()}
+    for name in declared_functions():
+        assert name in exported, f"{name} not exported"
+        assert hasattr(lib, name)
+
+
+def test_status_strings(lib):
+    for code in range(8):
+        assert gdn.status_string(code)
+    assert gdn.status_string(99) == "unknown status"
+
+
+# Fake, 16-byte aligned device addresses 4 GiB apart: never dereferenced,
+# every call below fails its checks before any launch.
+def fake(i):
+    return (i + 1) << 32
+
+
+A16, A16b, A16c = fake(0), fake(1), fake(2)
+
+
+def step_call(lib, state=A16, q=A16b, k=A16c, v=fake(3), beta=fake(4), gate=fake(5),
+              out=fake(6), L=1, B=1, Hk=16, Hv=32, dk=128, dv=128):
+    return lib.gdn_step(state, q, k, v, beta, gate, out, L, B, Hk, Hv, dk, dv, None)
+
+
+def test_step_argument_checks(lib):
+    assert step_call(lib, L=-1) == SHAPE
+    assert step_call(lib, Hv=24, Hk=16) == SHAPE
+    assert step_call(lib, Hk=0) == SHAPE
+    assert step_call(lib, dk=64) == UNSUP
+    assert step_call(lib, dv=256) == UNSUP
+    assert step_call(lib, q=0) == NULL
+    assert step_call(lib, out=0) == NULL
+    assert step_call(lib, state=A16 + 4) == ALIGN
+    assert step_call(lib, beta=fake(4) + 2) == ALIGN
+    assert step_call(lib, L=1 << 40, B=1 << 40) == OVERFLOW
+    # out inside the state buffer; state overlapping q
+    assert step_call(lib, out=A16 + 4096) == ALIAS
+    assert step_call(lib, q=A16 + 1024) == ALIAS
+    # read-only inputs may share memory
+    assert step_call(lib, k=A16b, q=A16b, out=0) == NULL
+    assert b"NULL" in lib.gdn_last_error() or lib.gdn_last_error()
+    # empty problems succeed without touching the (null) pointers
+    assert lib.gdn_step(0, 0, 0, 0, 0, 0, 0, 0, 5, 16, 32, 128, 128, None) == OK
+    assert lib.gdn_step(0, 0, 0, 0, 0, 0, 0, 3, 0, 16, 32, 128, 128, None) == OK
+
+
+def test_prefill_argument_checks(lib):
+    f = lambda **kw: lib.gdn_prefill(kw.get("state", A16), A16b, A16c, fake(3), fake(4),
+                                     fake(5), kw.get("out", fake(6)), kw.get("B", 1),
+                                     kw.get("T", 4), kw.get("Hk", 16), kw.get("Hv", 32),
+                                     128, 128, None)
+    assert f(T=-1) == SHAPE
+    assert f(Hv=17) == SHAPE
+    assert f(state=0) == NULL
+    assert f(state=A16 + 8) == ALIGN
+    assert f(out=A16b) == ALIAS
+    assert lib.gdn_prefill(0, 0, 0, 0, 0, 0, 0, 2, 0, 16, 32, 128, 128, None) == OK
+    assert lib.gdn_prefill(0, 0, 0, 0, 0, 0, 0, 0, 9, 16, 32, 128, 128, None) == OK
+
+
+def test_layer_argument_checks(lib):
+    def f(B=1, Hk=16, Hv=32, K=4, state=A16, out=fake(10), ring=fake(5)):
+        return lib.gdn_layer_decode(A16b, A16c, fake(3), fake(4), ring, fake(6), fake(7),
+                                    fake(8), fake(9), ctypes.c_float(1e-6), ctypes.c_float(1e-6),
+                                    state, out, B, Hk, Hv, 128, 128, K, None)
+    assert f(B=-2) == SHAPE
+    assert f(K=3) == UNSUP
+    assert f(Hk=4, Hv=32) == UNSUP          # 8 value heads per key head: not compiled
+    assert f(state=0) == NULL
+    assert f(state=A16 + 4) == ALIGN
+    assert f(out=A16b + 64) == ALIAS        # inside mixed_qkv
+    assert f(ring=A16c + 16) == ALIAS       # conv ring overlapping z
+    assert lib.gdn_layer_decode(0, 0, 0, 0, 0, 0, 0, 0, 0, ctypes.c_float(1e-6),
+                                ctypes.c_float(1e-6), 0, 0, 0, 16, 32, 128, 128, 4, None) == OK
+
+
+def test_binding_rejects_cpu_tensors():
+    import torch
+    st = torch.zeros(1, 1, 32, 128, 128)
+    q = torch.zeros(1, 1, 16, 128)
+    with pytest.raises(ValueError):
+        gdn.step(st, q, q, torch.zeros(1, 1, 32, 128), torch.zeros(1, 1, 32),
+                 torch.zeros(1, 1, 32), out=torch.zeros(1, 1, 32, 128))

@@ -1,0 +1,108 @@
+"""gdn_prefill on the GPU against the fp64 oracle (through the C ABI)."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from linear_attention_recurrence_04_b200 import gdn, inputs
+from parity import assert_parity
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def o():
+    return oracle.load()
+
+
+def to_dev(d):
+    return {k: torch.from_numpy(np.ascontiguousarray(v)).cuda() for k, v in d.items()}
+
+
+def run_gpu(d):
+    t = to_dev(d)
+    out = gdn.prefill(t["state"], t["q"], t["k"], t["v"], t["beta"], t["gate"])
+    torch.cuda.synchronize()
+    return t["state"].cpu().numpy(), out.cpu().numpy()
+
+
+@pytest.mark.parametrize("B,T,Hk,Hv,std", [(2, 37, 16, 32, 0.05), (1, 5, 4, 4, 0.05),
+                                           (3, 9, 2, 6, 0.0), (1, 16, 2, 8, 0.05),
+                                           (1, 1, 16, 32, 0.05)])
+def test_prefill_small_full_parity(o, B, T, Hk, Hv, std):
+    d = inputs.prefill_inputs(B, T, Hk=Hk, Hv=Hv, seed=500 + B * 100 + T, state_std=std)
+    st_ref, out_ref = o.prefill(d["state"], d["q"], d["k"], d["v"], d["beta"], d["gate"])
+    st, out = run_gpu(d)
+    assert_parity(out, out_ref, "prefill out")
+    assert_parity(st, st_ref, "prefill state")
+
+
+def test_prefill_one_position_equals_step():
+    d = inputs.prefill_inputs(3, 1, seed=61, state_std=0.05)
+    st_p, out_p = run_gpu(d)
+    # prefill's [B, T=1, ...] is step's [L=1, B, ...]
+    s = {"state": d["state"][None]}
+    for n in ("q", "k", "v", "beta", "gate"):
+        s[n] = d[n][:, 0][None]
+    t = to_dev(s)
+    out_s = gdn.step(t["state"], t["q"], t["k"], t["v"], t["beta"], t["gate"])
+    torch.cuda.synchronize()
+    assert_parity(out_p[:, 0], out_s[0].cpu().numpy().astype(np.float64), "T=1 out vs step")
+    assert_parity(st_p, t["state"][0].cpu().numpy().astype(np.float64), "T=1 state vs step")
+
+
+def test_prefill_resume_matches_one_pass(o):
+    """prefill(T1) then prefill(T2) from the returned state == oracle prefill(T1 + T2)."""
+    d = inputs.prefill_inputs(2, 50, seed=62, state_std=0.05)
+    t = to_dev(d)
+    cut = 23
+    sl = lambda x, a, b: x[:, a:b].contiguous()
+    o1 = gdn.prefill(t["state"], sl(t["q"], 0, cut), sl(t["k"], 0, cut), sl(t["v"], 0, cut),
+                     sl(t["beta"], 0, cut), sl(t["gate"], 0, cut))
+    o2 = gdn.prefill(t["state"], sl(t["q"], cut, 50), sl(t["k"], cut, 50), sl(t["v"], cut, 50),
+                     sl(t["beta"], cut, 50), sl(t["gate"], cut, 50))
+    torch.cuda.synchronize()
+    st_ref, out_ref = o.prefill(d["state"], d["q"], d["k"], d["v"], d["beta"], d["gate"])
+    assert_parity(torch.cat([o1, o2], 1).cpu().numpy(), out_ref, "resumed out")
+    assert_parity(t["state"].cpu().numpy(), st_ref, "resumed state")
+
+
+def test_prefill_decay_extremes(o):
+    """Runs of no decay, of decay to exactly zero (gate = -200), and of mild
+    growth (gate > 0), which push the kernel's running scale through both of
+    its fold-back bounds."""
+    d = inputs.prefill_inputs(1, 300, seed=63, state_std=0.05)
+    d["gate"][0, :100, :] = 0.0
+    d["gate"][0, 100, :] = -200.0
+    d["gate"][0, 101:200, :] = -0.45     # the scale shrinks past 2^-40 and folds
+    d["gate"][0, 200:300, :] = 0.3       # and grows past 2^40 and folds
+    d["beta"][0, 200:300, :] *= 0.01     # keep the state bounded while it grows
+    st_ref, out_ref = o.prefill(d["state"], d["q"], d["k"], d["v"], d["beta"], d["gate"])
+    st, out = run_gpu(d)
+    scale = max(1.0, float(np.max(np.abs(st_ref))))
+    assert_parity(out / scale, out_ref / scale, "extreme out (scaled)")
+    assert_parity(st / scale, st_ref / scale, "extreme state (scaled)")
+
+
+def test_prefill_empty():
+    st = torch.zeros(2, 32, 128, 128, device="cuda")
+    q = torch.zeros(2, 0, 16, 128, device="cuda")
+    out = gdn.prefill(st, q, q, torch.zeros(2, 0, 32, 128, device="cuda"),
+                      torch.zeros(2, 0, 32, device="cuda"), torch.zeros(2, 0, 32, device="cuda"))
+    assert out.shape == (2, 0, 32, 128) and not st.any()
+
+
+def test_prefill_full_workload_sampled(o):
+    """B = 4 x T = 4096 in the benchmark's launch shape; 6 (sequence, head)
+    units recomputed by the oracle over all 4096 positions."""
+    d = inputs.WORKLOADS["prefill_b4_t4096"].draw()
+    st, out = run_gpu(d)
+    assert np.all(np.isfinite(out)) and np.all(np.isfinite(st))
+    B, Hv = d["state"].shape[:2]
+    units = [0, 17, 31, 32 + 5, 2 * 32 + 16, B * Hv - 1]
+    st_ref, out_ref = o.prefill(d["state"], d["q"], d["k"], d["v"], d["beta"], d["gate"],
+                                units=units)
+    for u in units:
+        b, h = divmod(u, Hv)
+        assert_parity(out[b, :, h], out_ref[b, :, h], f"full prefill out b{b} h{h}")
+        assert_parity(st[b, h], st_ref[b, h], f"full prefill state b{b} h{h}")
