@@ -268,7 +268,8 @@ def bench_step_workload(name: str, steps: int, warmup: int, device, seed_offset:
     d = inputs.decode_inputs(L, B, seed=w.seed + seed_offset)
     base = _to_dev(d, device)
     nbytes = step_bytes(L, B)
-    n_sets = _sets_for(nbytes)
+    footprint = sum(v.nbytes for v in d.values()) + d["v"].nbytes   # inputs + out
+    n_sets = _sets_for(footprint)
     sets = [base] + [{k: v.clone() for k, v in base.items()} for _ in range(n_sets - 1)]
     outs = [torch.empty_like(s["v"]) for s in sets]
     stream = torch.cuda.current_stream(device)
@@ -279,7 +280,8 @@ def bench_step_workload(name: str, steps: int, warmup: int, device, seed_offset:
 
     secs = time_launches(launch, n_sets, steps, warmup, stream, graph=graph)
     return dict(seconds=secs, bytes=nbytes, state_bytes=L * B * 32 * STATE_BYTES_PER_HEAD,
-                layer_tokens=L * B, n_sets=n_sets, set_bytes=nbytes, sets=sets, outs=outs, d=d)
+                layer_tokens=L * B, n_sets=n_sets, set_bytes=footprint, sets=sets, outs=outs,
+                d=d)
 
 
 def bench_e2e(d: Dict[str, np.ndarray], steps: int, warmup: int, device):
