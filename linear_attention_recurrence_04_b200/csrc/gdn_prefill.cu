@@ -10,10 +10,11 @@
 //  * The state never leaves the chip between positions. Row j of a head only
 //    needs k, q, v[j], beta and gate of each position, so a head's 128 x 128
 //    state splits into independent rows. A warp owns 8 rows of NH value heads
-//    that share one key head (h, h + Hk, ...): lane l holds a 32-column slice
-//    of each of its NH rows in registers (4 lanes per row), so each k/q value
-//    it reads serves NH rows; a row's dot products reduce over its 4 lanes
-//    with two shuffles.
+//    that share one key head (h, h + Hk, ...): 4 lanes share a row, each
+//    holding a 32-column slice of each of its NH rows in registers, so each
+//    k/q value a lane reads serves NH rows; a row's dot products reduce over
+//    its 4 lanes with two shuffles. (Eight lanes per row, 16 columns each,
+//    doubles the resident warps but measured slower.)
 //  * Work balance: the warps ("units") are dealt to one CTA per SM in
 //    contiguous runs whose lengths differ by at most one, so every SM carries
 //    the same number of rows. A run covers at most two (sequence, key head,
@@ -21,7 +22,14 @@
 //  * Inputs are staged in shared memory S stages of TS positions ahead with
 //    16-byte asynchronous copies (cp.async), shared by all warps of the CTA:
 //    k and q rows once per group and position, each warp's v rows, beta and
-//    gate. The copy of stage s + S - 1 overlaps the arithmetic of stage s.
+//    gate. Positions past T are zero-filled. The decays exp(gate) of a stage
+//    are computed once per warp (one per lane) and broadcast by shuffle.
+//  * Software pipeline across positions: after the rank-1 update of position
+//    t, one pass over the register-resident rows makes both the output dot
+//    W.q_t and the next position's key dot W.k_{t+1} (both read the same
+//    updated row), and the 4-lane reductions of out_t and sk_{t+1} run as one
+//    batch at the top of the next iteration. The dependency chain per
+//    position is then: reduce -> scalar delta -> one fused pass.
 //  * Algebra in place of step 1 (same result up to rounding): head h's state
 //    is held as s * W with a per-head scalar s, so the decay is s *= e (one
 //    multiply per head, not per element). With W held:
@@ -35,14 +43,14 @@
 #include "gdn_common.cuh"
 #include "gdn_internal.h"
 
-#ifndef GDN_PREFILL_TS
-#define GDN_PREFILL_TS 16          // positions per stage
-#endif
 #ifndef GDN_PREFILL_STAGES
-#define GDN_PREFILL_STAGES 3       // stages in flight
+#define GDN_PREFILL_STAGES 4       // stages in flight (at least 3)
 #endif
 #ifndef GDN_PREFILL_MAX_WARPS
 #define GDN_PREFILL_MAX_WARPS 8    // units (warps) per CTA at most
+#endif
+#ifndef GDN_PREFILL_LPR
+#define GDN_PREFILL_LPR 4          // lanes per state row (4 or 8)
 #endif
 #ifndef GDN_PREFILL_FMA2
 #define GDN_PREFILL_FMA2 1         // packed f32x2 FMAs for the per-element work
@@ -52,24 +60,26 @@ namespace gdn {
 
 namespace {
 
-constexpr int kTS = GDN_PREFILL_TS;
+constexpr int kTS = 16;                         // positions per stage
 constexpr int kStages = GDN_PREFILL_STAGES;
 constexpr int kMaxWarps = GDN_PREFILL_MAX_WARPS;
-constexpr int kRowsPerUnit = 8;                 // 8 rows x 4 lanes = one warp
+constexpr int kLPR = GDN_PREFILL_LPR;           // lanes sharing one state row
+constexpr int kRowsPerUnit = 32 / kLPR;         // rows of a head per warp
 constexpr int kUnitsPerHead = kDv / kRowsPerUnit;
-constexpr int kChunks = 8;                      // float4 chunks per lane per row
+constexpr int kChunks = kDk / 4 / kLPR;         // float4 chunks per lane per row
 constexpr int kMaxGroups = 2;                   // groups one CTA's run can touch
 constexpr int kMaxRows = kMaxWarps * kRowsPerUnit;
 constexpr float kScaleLo = 0x1p-40f;
 constexpr float kScaleHi = 0x1p40f;
 static_assert(kMaxWarps <= kUnitsPerHead, "a run must span at most two groups");
-static_assert((kTS & (kTS - 1)) == 0, "positions per stage must be a power of two");
+static_assert(kStages >= 3, "the pipeline reads one stage ahead");
+static_assert(kLPR == 4 || kLPR == 8, "4 or 8 lanes per row");
 
 // Shared-memory image of one stage.
 template <int NH>
 struct Stage {
     float kq[kMaxGroups][kTS][2][kDk];          // [group][pos][k|q][col]
-    float v[kMaxGroups][kTS][NH][kMaxRows];     // rows [row_lo, row_hi) of the group
+    float v[kMaxGroups][kTS][NH][kMaxRows];     // rows [row_lo, row_lo + rows) of the group
     float bg[kMaxGroups][kTS][NH][2];           // beta, gate
 };
 
@@ -83,7 +93,9 @@ struct Group {
     int rows;
 };
 
-__device__ __forceinline__ int chunk_col(int i, int c) { return 16 * i + 4 * c; }
+// Lane c of a row holds the float4 chunks {kLPR i + c}, so one warp-wide
+// 16-byte load of k or q touches 16 kLPR contiguous bytes.
+__device__ __forceinline__ int chunk_col(int i, int c) { return 4 * (kLPR * i + c); }
 
 __device__ __forceinline__ void cp_async16(void* smem, const void* gmem) {
     const unsigned s = static_cast<unsigned>(__cvta_generic_to_shared(smem));
@@ -99,16 +111,10 @@ __device__ __forceinline__ void cp_async_wait() {
     asm volatile("cp.async.wait_group %0;\n" ::"n"(N) : "memory");
 }
 
-// d = a * b + c on two lanes of packed floats.
+// d = a * b + c on two lanes of packed floats (one packed f32x2 FMA).
 __device__ __forceinline__ float2 fma2(float2 a, float2 b, float2 c) {
 #if GDN_PREFILL_FMA2
-    float2 d;
-    asm("{\n\t.reg .b64 ra, rb, rc, rd;\n\t"
-        "mov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\tmov.b64 rc, {%6, %7};\n\t"
-        "fma.rn.f32x2 rd, ra, rb, rc;\n\tmov.b64 {%0, %1}, rd;\n\t}"
-        : "=f"(d.x), "=f"(d.y)
-        : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y), "f"(c.x), "f"(c.y));
-    return d;
+    return __ffma2_rn(a, b, c);
 #else
     return make_float2(fmaf(a.x, b.x, c.x), fmaf(a.y, b.y, c.y));
 #endif
@@ -116,6 +122,8 @@ __device__ __forceinline__ float2 fma2(float2 a, float2 b, float2 c) {
 
 __device__ __forceinline__ float2 lo2(float4 v) { return make_float2(v.x, v.y); }
 __device__ __forceinline__ float2 hi2(float4 v) { return make_float2(v.z, v.w); }
+__device__ __forceinline__ float4 ld_s4(const float* p) { return *reinterpret_cast<const float4*>(p); }
+__device__ __forceinline__ float sum4(float2 a, float2 b) { return (a.x + a.y) + (b.x + b.y); }
 
 template <int NH>
 __global__ void __launch_bounds__(32 * kMaxWarps, 1)
@@ -125,28 +133,24 @@ prefill_kernel(float* __restrict__ state, const float* __restrict__ q,
                float* __restrict__ out, int64_t T, int Hk, int Hv, int units_lo, int n_big) {
     extern __shared__ __align__(16) unsigned char smem_raw[];
     Stage<NH>* stages = reinterpret_cast<Stage<NH>*>(smem_raw);
+    __shared__ Group grp_of[kMaxGroups];
 
     const int tid = threadIdx.x;
     const int nthreads = blockDim.x;
     const int warp = tid >> 5;
     const int lane = tid & 31;
-    const int p = lane >> 2;
-    const int c = lane & 3;
+    const int p = lane / kLPR;                  // row within the warp's rows
+    const int c = lane % kLPR;                  // column slice
 
     // This CTA's run of units: [u0, u0 + count).
     const int cta = blockIdx.x;
     const int64_t u0 = static_cast<int64_t>(cta) * units_lo + (cta < n_big ? cta : n_big);
     const int count = units_lo + (cta < n_big ? 1 : 0);
     const int groups_per_key = (Hv / Hk) / NH;
-
-    // The (at most two) groups the run touches.
-    Group grp_of[kMaxGroups];
     const int64_t gid0 = u0 / kUnitsPerHead;
-    const int64_t gid1 = (u0 + count - 1) / kUnitsPerHead;
-    const int n_groups = static_cast<int>(gid1 - gid0) + 1;
-#pragma unroll
-    for (int gi = 0; gi < kMaxGroups; ++gi) {
-        const int64_t gid = gid0 + gi;
+    const int n_groups = static_cast<int>((u0 + count - 1) / kUnitsPerHead - gid0) + 1;
+    if (tid < kMaxGroups) {
+        const int64_t gid = gid0 + tid;
         int64_t rest = gid;
         Group G;
         G.grp = static_cast<int>(rest % groups_per_key);
@@ -158,48 +162,54 @@ prefill_kernel(float* __restrict__ state, const float* __restrict__ q,
                                                                    : u0 + count;
         G.row_lo = static_cast<int>(first - gid * kUnitsPerHead) * kRowsPerUnit;
         G.rows = static_cast<int>(last - first) * kRowsPerUnit;
-        grp_of[gi] = G;
+        grp_of[tid] = G;
     }
+    __syncthreads();
 
-    // ---- stage loader: every thread issues a share of the copies --------
+    // ---- stage loader: every thread issues a share of the copies; positions
+    //      at or past T are zero-filled ------------------------------------
     auto load_stage = [&](int64_t t0, Stage<NH>& st) {
 #pragma unroll
         for (int gi = 0; gi < kMaxGroups; ++gi) {
             if (gi >= n_groups) break;
             const Group G = grp_of[gi];
-            // k and q rows: TS positions x 2 x 32 chunks of 16 bytes
-            for (int idx = tid; idx < kTS * 64; idx += nthreads) {
+            for (int idx = tid; idx < kTS * 64; idx += nthreads) {        // k, q rows
                 const int chunk = idx & 31;
                 const int which = (idx >> 5) & 1;
                 const int tp = idx >> 6;
                 const int64_t t = t0 + tp;
+                float* dst = &st.kq[gi][tp][which][chunk * 4];
                 if (t < T) {
-                    const float* src = (which ? q : k) + ((G.b * T + t) * Hk + G.g) * kDk + chunk * 4;
-                    cp_async16(&st.kq[gi][tp][which][chunk * 4], src);
+                    cp_async16(dst, (which ? q : k) + ((G.b * T + t) * Hk + G.g) * kDk + chunk * 4);
+                } else {
+                    *reinterpret_cast<float4*>(dst) = make_float4(0.f, 0.f, 0.f, 0.f);
                 }
             }
-            // v rows of the run, for each of the NH heads
-            const int vchunks = G.rows / 4;
+            const int vchunks = G.rows / 4;                              // v rows
             for (int idx = tid; idx < kTS * NH * vchunks; idx += nthreads) {
                 const int chunk = idx % vchunks;
                 const int n = (idx / vchunks) % NH;
                 const int tp = idx / (vchunks * NH);
                 const int64_t t = t0 + tp;
+                float* dst = &st.v[gi][tp][n][chunk * 4];
                 if (t < T) {
                     const int h = G.g + (G.grp * NH + n) * Hk;
-                    const float* src = v + ((G.b * T + t) * Hv + h) * kDv + G.row_lo + chunk * 4;
-                    cp_async16(&st.v[gi][tp][n][chunk * 4], src);
+                    cp_async16(dst, v + ((G.b * T + t) * Hv + h) * kDv + G.row_lo + chunk * 4);
+                } else {
+                    *reinterpret_cast<float4*>(dst) = make_float4(0.f, 0.f, 0.f, 0.f);
                 }
             }
-            // beta and gate
-            for (int idx = tid; idx < kTS * NH * 2; idx += nthreads) {
+            for (int idx = tid; idx < kTS * NH * 2; idx += nthreads) {    // beta, gate
                 const int which = idx & 1;
                 const int n = (idx >> 1) % NH;
                 const int tp = (idx >> 1) / NH;
                 const int64_t t = t0 + tp;
+                float* dst = &st.bg[gi][tp][n][which];
                 if (t < T) {
                     const int h = G.g + (G.grp * NH + n) * Hk;
-                    cp_async4(&st.bg[gi][tp][n][which], (which ? gate : beta) + (G.b * T + t) * Hv + h);
+                    cp_async4(dst, (which ? gate : beta) + (G.b * T + t) * Hv + h);
+                } else {
+                    *dst = 0.0f;
                 }
             }
         }
@@ -209,19 +219,24 @@ prefill_kernel(float* __restrict__ state, const float* __restrict__ q,
     const bool active = warp < count;
     const int64_t unit = u0 + warp;
     const int gi = active ? static_cast<int>(unit / kUnitsPerHead - gid0) : 0;
-    const Group G = gi == 0 ? grp_of[0] : grp_of[1];
+    const Group G = grp_of[gi];
     const int rb = static_cast<int>(unit % kUnitsPerHead);
     const int j = rb * kRowsPerUnit + p;                 // row within the head
     const int vrow = j - G.row_lo;                       // row within the staged v
     int hidx[NH];
 #pragma unroll
     for (int n = 0; n < NH; ++n) hidx[n] = G.g + (G.grp * NH + n) * Hk;
+    // out of position t, head n, row j: out_base[n] + t * out_stride
+    const int64_t out_stride = static_cast<int64_t>(Hv) * kDv;
+    float* out_base[NH];
+#pragma unroll
+    for (int n = 0; n < NH; ++n) out_base[n] = out + (G.b * T * Hv + hidx[n]) * kDv + j;
 
     // Prologue: request the first S - 1 stages, then load the state rows.
-    const int64_t n_stages_total = (T + kTS - 1) / kTS;
+    const int64_t n_stages = (T + kTS - 1) / kTS;
 #pragma unroll
-    for (int s = 0; s < kStages - 1; ++s) {
-        if (s < n_stages_total) load_stage(static_cast<int64_t>(s) * kTS, stages[s]);
+    for (int s2 = 0; s2 < kStages - 1; ++s2) {
+        if (s2 < n_stages) load_stage(static_cast<int64_t>(s2) * kTS, stages[s2]);
         cp_async_commit();
     }
 
@@ -237,101 +252,136 @@ prefill_kernel(float* __restrict__ state, const float* __restrict__ q,
         }
     }
 
-    for (int64_t s = 0; s < n_stages_total; ++s) {
-        cp_async_wait<kStages - 2>();       // this thread's copies of stage s landed
-        __syncthreads();                     // ... and everyone's; stage s-1 is free
+    // Loop-carried partial sums: a = W.k of the coming position, o = W.q of
+    // the previous position (its store is pending), s_out = its scale.
+    float2 a_lo[NH], a_hi[NH], o_lo[NH], o_hi[NH];
+    float s_out[NH];
+    bool out_pending = false;
+    int64_t t_out = 0;
+
+    for (int64_t s = 0; s < n_stages; ++s) {
+        cp_async_wait<kStages - 3>();       // this thread's copies of stages s, s+1 landed
+        __syncthreads();                     // ... and everyone's; stage s-1 is consumed
         {
             const int64_t nxt = s + kStages - 1;
-            if (nxt < n_stages_total) load_stage(nxt * kTS, stages[nxt % kStages]);
+            if (nxt < n_stages) load_stage(nxt * kTS, stages[nxt % kStages]);
             cp_async_commit();
         }
+        if (!active) continue;
         const Stage<NH>& st = stages[s % kStages];
+        const Stage<NH>& st_next = stages[(s + 1) % kStages];
         const int64_t t0 = s * kTS;
         const int tp_end = (T - t0) < kTS ? static_cast<int>(T - t0) : kTS;
-        if (active) {
-            for (int tp = 0; tp < tp_end; ++tp) {
-                float4 kk[kChunks], qq[kChunks];
+
+        // decays of this stage, one per lane: lane tp + kTS n holds exp(gate)
+        const float e_lane = (lane < kTS * NH) ? expf(st.bg[gi][lane % kTS][lane / kTS][1]) : 1.0f;
+
+        if (s == 0) {
+            // first key dot: a = W.k_0
 #pragma unroll
-                for (int i = 0; i < kChunks; ++i) {
-                    kk[i] = *reinterpret_cast<const float4*>(&st.kq[gi][tp][0][chunk_col(i, c)]);
-                    qq[i] = *reinterpret_cast<const float4*>(&st.kq[gi][tp][1][chunk_col(i, c)]);
-                }
-                const int64_t bt = G.b * T + t0 + tp;
-                // The NH heads are independent: each phase below runs for all
-                // of them before the next, so their dependency chains overlap.
-                float s_new[NH], sk[NH], vj[NH], bn[NH];
-                float2 a0[NH], a1[NH];
+            for (int n = 0; n < NH; ++n) a_lo[n] = a_hi[n] = make_float2(0.f, 0.f);
+#pragma unroll
+            for (int i = 0; i < kChunks; ++i) {
+                const float4 kv = ld_s4(&st.kq[gi][0][0][chunk_col(i, c)]);
 #pragma unroll
                 for (int n = 0; n < NH; ++n) {
-                    vj[n] = st.v[gi][tp][n][vrow];
-                    bn[n] = st.bg[gi][tp][n][0];
-                    // step 1 as a scale update
-                    s_new[n] = sc[n] * expf(st.bg[gi][tp][n][1]);
-                    // step 2: W.k (the scale enters below)
-                    a0[n] = make_float2(0.f, 0.f);
-                    a1[n] = make_float2(0.f, 0.f);
-#pragma unroll
-                    for (int i = 0; i < kChunks; ++i) {
-                        a0[n] = fma2(lo2(w[n][i]), lo2(kk[i]), a0[n]);
-                        a1[n] = fma2(hi2(w[n][i]), hi2(kk[i]), a1[n]);
-                    }
-                }
-                float delta[NH];
-                bool fold = false;
-#pragma unroll
-                for (int n = 0; n < NH; ++n) {
-                    // sk = s_new (W.k) whether or not the scale is folded below
-                    sk[n] = s_new[n] * group_sum<4>((a0[n].x + a0[n].y) + (a1[n].x + a1[n].y));
-                    delta[n] = (vj[n] - sk[n]) * bn[n];                  // step 3
-                    fold |= !(s_new[n] >= kScaleLo && s_new[n] <= kScaleHi);
-                }
-                if (fold) {          // rare, and uniform across the warp
-#pragma unroll
-                    for (int n = 0; n < NH; ++n) {
-                        if (!(s_new[n] >= kScaleLo && s_new[n] <= kScaleHi)) {
-#pragma unroll
-                            for (int i = 0; i < kChunks; ++i) {
-                                w[n][i].x *= s_new[n]; w[n][i].y *= s_new[n];
-                                w[n][i].z *= s_new[n]; w[n][i].w *= s_new[n];
-                            }
-                            s_new[n] = 1.0f;
-                        }
-                    }
-                }
-                float2 o0[NH], o1[NH];
-#pragma unroll
-                for (int n = 0; n < NH; ++n) {
-                    sc[n] = s_new[n];
-                    // step 4: W += (delta / s) k
-                    const float cf = delta[n] * __frcp_rn(sc[n]);
-                    const float2 cf2 = make_float2(cf, cf);
-#pragma unroll
-                    for (int i = 0; i < kChunks; ++i) {
-                        const float2 lo = fma2(cf2, lo2(kk[i]), lo2(w[n][i]));
-                        const float2 hi = fma2(cf2, hi2(kk[i]), hi2(w[n][i]));
-                        w[n][i] = make_float4(lo.x, lo.y, hi.x, hi.y);
-                    }
-                    // step 5: W_new.q
-                    o0[n] = make_float2(0.f, 0.f);
-                    o1[n] = make_float2(0.f, 0.f);
-#pragma unroll
-                    for (int i = 0; i < kChunks; ++i) {
-                        o0[n] = fma2(lo2(w[n][i]), lo2(qq[i]), o0[n]);
-                        o1[n] = fma2(hi2(w[n][i]), hi2(qq[i]), o1[n]);
-                    }
-                }
-#pragma unroll
-                for (int n = 0; n < NH; ++n) {
-                    const float o = sc[n] * group_sum<4>((o0[n].x + o0[n].y) + (o1[n].x + o1[n].y)) * kOutScale;
-                    if (c == (n & 3)) out[(bt * Hv + hidx[n]) * kDv + j] = o;
+                    a_lo[n] = fma2(lo2(w[n][i]), lo2(kv), a_lo[n]);
+                    a_hi[n] = fma2(hi2(w[n][i]), hi2(kv), a_hi[n]);
                 }
             }
+        }
+
+        for (int tp = 0; tp < tp_end; ++tp) {
+            const int64_t t = t0 + tp;
+            // (a) batched reductions: sk of t, and out of t-1
+            float A[NH], O[NH];
+#pragma unroll
+            for (int n = 0; n < NH; ++n) {
+                A[n] = sum4(a_lo[n], a_hi[n]);
+                O[n] = out_pending ? sum4(o_lo[n], o_hi[n]) : 0.0f;
+            }
+#pragma unroll
+            for (int n = 0; n < NH; ++n) {
+                A[n] = group_sum<kLPR>(A[n]);
+                O[n] = group_sum<kLPR>(O[n]);
+            }
+            if (out_pending) {
+#pragma unroll
+                for (int n = 0; n < NH; ++n)
+                    if (c == (n & 3)) out_base[n][t_out * out_stride] = s_out[n] * O[n] * kOutScale;
+            }
+            // (b) scalar part of position t (step 1 as a scale update, steps 2-3)
+            float cf[NH];
+            bool fold = false;
+            float s_new[NH];
+#pragma unroll
+            for (int n = 0; n < NH; ++n) {
+                const float e = __shfl_sync(kFull, e_lane, tp + kTS * n);
+                s_new[n] = sc[n] * e;
+                const float sk = s_new[n] * A[n];
+                cf[n] = (st.v[gi][tp][n][vrow] - sk) * st.bg[gi][tp][n][0];   // delta
+                fold |= !(s_new[n] >= kScaleLo && s_new[n] <= kScaleHi);
+            }
+            if (fold) {          // rare, and uniform across the warp
+#pragma unroll
+                for (int n = 0; n < NH; ++n) {
+                    if (!(s_new[n] >= kScaleLo && s_new[n] <= kScaleHi)) {
+#pragma unroll
+                        for (int i = 0; i < kChunks; ++i) {
+                            w[n][i].x *= s_new[n]; w[n][i].y *= s_new[n];
+                            w[n][i].z *= s_new[n]; w[n][i].w *= s_new[n];
+                        }
+                        s_new[n] = 1.0f;
+                    }
+                }
+            }
+#pragma unroll
+            for (int n = 0; n < NH; ++n) {
+                sc[n] = s_new[n];
+                cf[n] *= __frcp_rn(sc[n]);                                   // delta / s
+                s_out[n] = sc[n];
+            }
+            // (c) one pass: step 4 for t, then W.q_t (step 5) and W.k_{t+1}
+            const bool has_next = t + 1 < T;
+            const float* kn = (tp + 1 < kTS) ? &st.kq[gi][tp + 1][0][0] : &st_next.kq[gi][0][0][0];
+#pragma unroll
+            for (int n = 0; n < NH; ++n) {
+                o_lo[n] = o_hi[n] = a_lo[n] = a_hi[n] = make_float2(0.f, 0.f);
+            }
+#pragma unroll
+            for (int i = 0; i < kChunks; ++i) {
+                const float4 kv = ld_s4(&st.kq[gi][tp][0][chunk_col(i, c)]);
+                const float4 qv = ld_s4(&st.kq[gi][tp][1][chunk_col(i, c)]);
+                const float4 nv = has_next ? ld_s4(kn + chunk_col(i, c)) : make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+                for (int n = 0; n < NH; ++n) {
+                    const float2 cf2 = make_float2(cf[n], cf[n]);
+                    const float2 lo = fma2(cf2, lo2(kv), lo2(w[n][i]));
+                    const float2 hi = fma2(cf2, hi2(kv), hi2(w[n][i]));
+                    w[n][i] = make_float4(lo.x, lo.y, hi.x, hi.y);
+                    o_lo[n] = fma2(lo, lo2(qv), o_lo[n]);
+                    o_hi[n] = fma2(hi, hi2(qv), o_hi[n]);
+                    a_lo[n] = fma2(lo, lo2(nv), a_lo[n]);
+                    a_hi[n] = fma2(hi, hi2(nv), a_hi[n]);
+                }
+            }
+            out_pending = true;
+            t_out = t;
         }
     }
     cp_async_wait<0>();
 
-    // Write the final state back with the scale folded in.
     if (active) {
+        // the last position's output
+        if (out_pending) {
+            float O[NH];
+#pragma unroll
+            for (int n = 0; n < NH; ++n) O[n] = group_sum<kLPR>(sum4(o_lo[n], o_hi[n]));
+#pragma unroll
+            for (int n = 0; n < NH; ++n)
+                if (c == (n & 3)) out_base[n][t_out * out_stride] = s_out[n] * O[n] * kOutScale;
+        }
+        // the final state, scale folded in
 #pragma unroll
         for (int n = 0; n < NH; ++n) {
             float* row = state + ((G.b * Hv + hidx[n]) * kDv + j) * kDk;
