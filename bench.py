@@ -66,6 +66,15 @@ def layer_bytes(B: int, Hk: int = 16, Hv: int = 32, d: int = 128, K: int = 4) ->
             + B * Hv * 4 * 2 + C * K * 4 + Hv * 4 * 2 + d * 4)
 
 
+def layer_pair_bytes(B: int, Hk: int = 16, Hv: int = 32, d: int = 128, K: int = 4) -> int:
+    """State read once and written twice (committed + scratch), ring likewise,
+    and two positions of activations and outputs."""
+    C = 2 * Hk * d + Hv * d
+    return (B * Hv * d * d * 4 * 3 + B * (K - 1) * C * 4 * 3
+            + 2 * (B * C * 4 + B * Hv * d * 4 * 2 + B * Hv * 4 * 2)
+            + C * K * 4 + Hv * 4 * 2 + d * 4)
+
+
 # --------------------------------------------------------------------------
 # host-side helpers (no GPU needed; covered by the CPU tests)
 # --------------------------------------------------------------------------
@@ -358,6 +367,29 @@ def bench_layer(steps: int, warmup: int, device):
     return dict(seconds=secs, launches=steps, bytes=layer_bytes(B), tokens=B)
 
 
+def bench_layer_pair(steps: int, warmup: int, device):
+    import torch
+    from linear_attention_recurrence_04_b200 import gdn, inputs
+    B = 256
+    d = inputs.layer_inputs(B, seed=1005)
+    d2 = inputs.layer_inputs(B, seed=1006)
+    for n in ("mixed_qkv", "z", "a", "b"):
+        d[n] = np.stack([d[n], d2[n]], axis=1)
+    t = _to_dev(d, device)
+    sring = torch.empty_like(t["conv_ring"])
+    sstate = torch.empty_like(t["state"])
+    out = torch.empty((B, 2, 32 * 128), dtype=torch.float32, device=device)
+    order = ("mixed_qkv", "z", "a", "b", "conv_ring", "conv_w", "A_log", "dt_bias", "norm_w",
+             "state")
+    stream = torch.cuda.current_stream(device)
+
+    def launch(i):
+        gdn.layer_pair(*(t[n] for n in order), sring, sstate, out, Hk=16)
+
+    secs = time_launches(launch, 1, steps, warmup, stream, graph=True)
+    return dict(seconds=secs, launches=steps, bytes=layer_pair_bytes(B), tokens=2 * B)
+
+
 def cpu_oracle_baseline(name: str, budget_s: float, max_units: Optional[int] = None):
     """Time the fp64 oracle as it stands on a bounded sample of the workload:
     whole decode steps over the first `units` (layer, sequence, head) units,
@@ -549,6 +581,14 @@ def run_ours(args) -> int:
         extras["layer_decode_b256"] = {
             "ms_per_launch": lay["seconds"] / lay["launches"] * 1e3,
             "layer_tokens_per_s": lay["tokens"] * lay["launches"] / lay["seconds"],
+            "gb_s": gbs, "roofline": {"bound": "hbm", "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                                      "frac": gbs / peaks["hbm_gbs"]},
+        }
+        pr = bench_layer_pair(20, 3, device)
+        gbs = pr["bytes"] * pr["launches"] / pr["seconds"] / 1e9
+        extras["layer_pair_b256"] = {
+            "ms_per_launch": pr["seconds"] / pr["launches"] * 1e3,
+            "layer_tokens_per_s": pr["tokens"] * pr["launches"] / pr["seconds"],
             "gb_s": gbs, "roofline": {"bound": "hbm", "peak": peaks["hbm_gbs"], "unit": "GB/s",
                                       "frac": gbs / peaks["hbm_gbs"]},
         }

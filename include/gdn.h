@@ -22,8 +22,9 @@
  *   - Supported geometry: dk = dv = 128, Hk >= 1, Hv a multiple of Hk,
  *     conv kernel K = 4. Other values return GDN_ERR_UNSUPPORTED.
  *   - `state` and `conv_ring` are updated in place and must not overlap any
- *     other argument; `out` must not overlap any argument either
- *     (GDN_ERR_ALIAS otherwise). Read-only inputs may share memory.
+ *     other argument; `out` and the scratch outputs must not overlap any
+ *     argument either (GDN_ERR_ALIAS otherwise). Read-only inputs may share
+ *     memory.
  *   - Alignment: state, q, k, v, out, mixed_qkv, z, conv_ring and conv_w
  *     must be 16-byte aligned; the per-head scalars (beta, gate, a, b,
  *     A_log, dt_bias) and norm_w need 4-byte alignment.
@@ -52,7 +53,7 @@ typedef enum gdn_status {
     GDN_ERR_ALIGN = 4,       /* a pointer violates the alignment rule above    */
     GDN_ERR_OVERFLOW = 5,    /* an element count does not fit the index type   */
     GDN_ERR_CUDA = 6,        /* the CUDA runtime refused the launch            */
-    GDN_ERR_ALIAS = 7        /* out, state or conv_ring overlaps an argument   */
+    GDN_ERR_ALIAS = 7        /* an output or in-place buffer overlaps another  */
 } gdn_status;
 
 /* Static English text for a status code (never NULL). */
@@ -134,6 +135,40 @@ gdn_status gdn_layer_decode(const float *mixed_qkv, const float *z, const float 
                             float *state, float *out, int64_t B, int64_t Hk,
                             int64_t Hv, int64_t dk, int64_t dv, int64_t K,
                             void *stream);
+
+/*
+ * gdn_layer_pair -- the fused layer for two consecutive positions of each
+ * sequence, for speculative verification ("Module linear_core", entry
+ * "gdn_pair": lane 1 commits into the state, lane 2 is tentative in scratch,
+ * the conv ring and the recurrent state moving together). Position 0 runs
+ * gdn_layer_decode's six stages and commits: conv_ring and state are updated
+ * in place. Position 1 continues from that committed result; the ring and
+ * state it leaves are written to scratch_ring and scratch_state, and the
+ * live buffers keep position 0's result. To accept the draft the caller
+ * makes the scratch buffers live (swap pointers or copy); to reject it, it
+ * ignores them. The result equals gdn_layer_decode on position 0 followed
+ * by gdn_layer_decode on position 1 applied to copies of the updated
+ * buffers; each state row is read once and written twice.
+ *
+ *   mixed_qkv     [B][2][C]
+ *   z             [B][2][Hv*dv]
+ *   a, b          [B][2][Hv]
+ *   conv_ring     [B][K-1][C]        in/out: after position 0
+ *   conv_w        [C][K];  A_log, dt_bias [Hv];  norm_w [dv]
+ *   state         [B][Hv][dv][dk]    in/out: after position 0
+ *   scratch_ring  [B][K-1][C]        out: after position 1
+ *   scratch_state [B][Hv][dv][dk]    out: after position 1
+ *   out           [B][2][Hv*dv]      both positions' outputs
+ * scratch_ring and scratch_state are caller-allocated outputs, 16-byte
+ * aligned, and must not overlap any other argument.
+ */
+gdn_status gdn_layer_pair(const float *mixed_qkv, const float *z, const float *a,
+                          const float *b, float *conv_ring, const float *conv_w,
+                          const float *A_log, const float *dt_bias,
+                          const float *norm_w, float l2_eps, float norm_eps,
+                          float *state, float *scratch_ring, float *scratch_state,
+                          float *out, int64_t B, int64_t Hk, int64_t Hv, int64_t dk,
+                          int64_t dv, int64_t K, void *stream);
 
 #ifdef __cplusplus
 }

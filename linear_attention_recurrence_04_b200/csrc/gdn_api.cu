@@ -224,47 +224,94 @@ gdn_status gdn_prefill(float* state, const float* q, const float* k, const float
     return launched(launch_prefill(a, static_cast<cudaStream_t>(stream)), "gdn_prefill");
 }
 
+namespace {
+
+// Shared checks of the fused layer entry points; npos = 1 (decode) or 2 (pair).
+gdn_status check_layer(const char* fn, int npos, const float* mixed_qkv, const float* z,
+                       const float* a, const float* b, const float* conv_ring,
+                       const float* conv_w, const float* A_log, const float* dt_bias,
+                       const float* norm_w, const float* state, const float* scratch_ring,
+                       const float* scratch_state, const float* out, int64_t B, int64_t Hk,
+                       int64_t Hv, int64_t dk, int64_t dv, int64_t K, bool* empty) {
+    *empty = false;
+    if (B < 0) return fail(GDN_ERR_SHAPE, "%s: negative B=%lld", fn, (long long)B);
+    gdn_status st = check_geometry(Hk, Hv, dk, dv);
+    if (st != GDN_OK) return st;
+    if (K != kConvK) return fail(GDN_ERR_UNSUPPORTED, "%s: K=%lld: only a conv kernel of 4 is implemented",
+                                 fn, (long long)K);
+    if (!layer_decode_supports(static_cast<int>(Hv / Hk)))
+        return fail(GDN_ERR_UNSUPPORTED, "%s: Hv/Hk=%lld: the fused layer supports 1, 2 or 4",
+                    fn, (long long)(Hv / Hk));
+    const int64_t C = 2 * Hk * dk + Hv * dv;
+    int64_t x_n = 0, z_n = 0, bh = 0, ring_n = 0, state_n = 0, grid = 0;
+    if (!mul_ok(B * npos, C, &x_n) || !mul_ok(B * npos, Hv * dv, &z_n) ||
+        !mul_ok(B * npos, Hv, &bh) || !mul_ok(B, (K - 1) * C, &ring_n) ||
+        !mul_ok(B * Hv, dv * dk, &state_n) || !mul_ok(B, Hk, &grid) ||
+        B > INT64_MAX / 8 / Hv || state_n > INT64_MAX / 8 || ring_n > INT64_MAX / 8)
+        return fail(GDN_ERR_OVERFLOW, "%s: B*Hv*dv*dk overflows int64", fn);
+    if (grid > INT32_MAX) return fail(GDN_ERR_OVERFLOW, "%s: B*Hk=%lld exceeds the launch grid",
+                                      fn, (long long)grid);
+    if (B == 0) { *empty = true; return GDN_OK; }
+    if (!mixed_qkv || !z || !a || !b || !conv_ring || !conv_w || !A_log || !dt_bias || !norm_w ||
+        !state || !out || (npos == 2 && (!scratch_ring || !scratch_state)))
+        return fail(GDN_ERR_NULL, "%s: a tensor pointer is NULL", fn);
+    if (!aligned(mixed_qkv, 16) || !aligned(z, 16) || !aligned(conv_ring, 16) ||
+        !aligned(conv_w, 16) || !aligned(state, 16) || !aligned(out, 16) || !aligned(a, 4) ||
+        !aligned(b, 4) || !aligned(A_log, 4) || !aligned(dt_bias, 4) || !aligned(norm_w, 4) ||
+        (npos == 2 && (!aligned(scratch_ring, 16) || !aligned(scratch_state, 16))))
+        return fail(GDN_ERR_ALIGN, "%s: alignment rule violated", fn);
+    const Span ins[] = {{state, state_n * 4, "state"}, {conv_ring, ring_n * 4, "conv_ring"},
+                        {scratch_state, npos == 2 ? state_n * 4 : 0, "scratch_state"},
+                        {scratch_ring, npos == 2 ? ring_n * 4 : 0, "scratch_ring"},
+                        {mixed_qkv, x_n * 4, "mixed_qkv"}, {z, z_n * 4, "z"}, {a, bh * 4, "a"},
+                        {b, bh * 4, "b"}, {conv_w, C * K * 4, "conv_w"},
+                        {A_log, Hv * 4, "A_log"}, {dt_bias, Hv * 4, "dt_bias"},
+                        {norm_w, dv * 4, "norm_w"}};
+    return check_spans(ins, 12, 4, Span{out, z_n * 4, "out"});
+}
+
+}  // namespace
+
 gdn_status gdn_layer_decode(const float* mixed_qkv, const float* z, const float* a,
                             const float* b, float* conv_ring, const float* conv_w,
                             const float* A_log, const float* dt_bias, const float* norm_w,
                             float l2_eps, float norm_eps, float* state, float* out, int64_t B,
                             int64_t Hk, int64_t Hv, int64_t dk, int64_t dv, int64_t K,
                             void* stream) {
-    if (B < 0) return fail(GDN_ERR_SHAPE, "negative B=%lld", (long long)B);
-    gdn_status st = check_geometry(Hk, Hv, dk, dv);
-    if (st != GDN_OK) return st;
-    if (K != kConvK) return fail(GDN_ERR_UNSUPPORTED, "K=%lld: only a conv kernel of 4 is implemented",
-                                 (long long)K);
-    if (!layer_decode_supports(static_cast<int>(Hv / Hk)))
-        return fail(GDN_ERR_UNSUPPORTED, "Hv/Hk=%lld: the fused layer supports 1, 2 or 4",
-                    (long long)(Hv / Hk));
-    const int64_t C = 2 * Hk * dk + Hv * dv;
-    int64_t x_n = 0, z_n = 0, bh = 0, ring_n = 0, state_n = 0, grid = 0;
-    if (!mul_ok(B, C, &x_n) || !mul_ok(B, Hv * dv, &z_n) || !mul_ok(B, Hv, &bh) ||
-        !mul_ok(x_n, K - 1, &ring_n) || !mul_ok(bh, dv * dk, &state_n) || !mul_ok(B, Hk, &grid) ||
-        state_n > INT64_MAX / 8 || ring_n > INT64_MAX / 8)
-        return fail(GDN_ERR_OVERFLOW, "B*Hv*dv*dk overflows int64");
-    if (grid > INT32_MAX) return fail(GDN_ERR_OVERFLOW, "B*Hk=%lld exceeds the launch grid",
-                                      (long long)grid);
-    if (B == 0) { g_last_error[0] = '\0'; return GDN_OK; }
-    if (!mixed_qkv || !z || !a || !b || !conv_ring || !conv_w || !A_log || !dt_bias || !norm_w ||
-        !state || !out)
-        return fail(GDN_ERR_NULL, "gdn_layer_decode: a tensor pointer is NULL");
-    if (!aligned(mixed_qkv, 16) || !aligned(z, 16) || !aligned(conv_ring, 16) ||
-        !aligned(conv_w, 16) || !aligned(state, 16) || !aligned(out, 16) || !aligned(a, 4) ||
-        !aligned(b, 4) || !aligned(A_log, 4) || !aligned(dt_bias, 4) || !aligned(norm_w, 4))
-        return fail(GDN_ERR_ALIGN, "gdn_layer_decode: alignment rule violated");
-    const Span ins[] = {{state, state_n * 4, "state"}, {conv_ring, ring_n * 4, "conv_ring"},
-                        {mixed_qkv, x_n * 4, "mixed_qkv"}, {z, z_n * 4, "z"}, {a, bh * 4, "a"},
-                        {b, bh * 4, "b"}, {conv_w, C * K * 4, "conv_w"},
-                        {A_log, Hv * 4, "A_log"}, {dt_bias, Hv * 4, "dt_bias"},
-                        {norm_w, dv * 4, "norm_w"}};
-    st = check_spans(ins, 10, 2, Span{out, z_n * 4, "out"});
-    if (st != GDN_OK) return st;
+    bool empty = false;
+    gdn_status st = check_layer("gdn_layer_decode", 1, mixed_qkv, z, a, b, conv_ring, conv_w,
+                                A_log, dt_bias, norm_w, state, nullptr, nullptr, out, B, Hk,
+                                Hv, dk, dv, K, &empty);
+    if (st != GDN_OK || empty) {
+        if (st == GDN_OK) g_last_error[0] = '\0';
+        return st;
+    }
     LayerArgs args{mixed_qkv, z, a, b, conv_ring, conv_w, A_log, dt_bias, norm_w, l2_eps,
-                   norm_eps, state, out, B, static_cast<int>(Hk), static_cast<int>(Hv)};
+                   norm_eps, state, out, B, static_cast<int>(Hk), static_cast<int>(Hv),
+                   nullptr, nullptr};
     return launched(launch_layer_decode(args, static_cast<cudaStream_t>(stream)),
                     "gdn_layer_decode");
+}
+
+gdn_status gdn_layer_pair(const float* mixed_qkv, const float* z, const float* a, const float* b,
+                          float* conv_ring, const float* conv_w, const float* A_log,
+                          const float* dt_bias, const float* norm_w, float l2_eps,
+                          float norm_eps, float* state, float* scratch_ring,
+                          float* scratch_state, float* out, int64_t B, int64_t Hk, int64_t Hv,
+                          int64_t dk, int64_t dv, int64_t K, void* stream) {
+    bool empty = false;
+    gdn_status st = check_layer("gdn_layer_pair", 2, mixed_qkv, z, a, b, conv_ring, conv_w,
+                                A_log, dt_bias, norm_w, state, scratch_ring, scratch_state, out,
+                                B, Hk, Hv, dk, dv, K, &empty);
+    if (st != GDN_OK || empty) {
+        if (st == GDN_OK) g_last_error[0] = '\0';
+        return st;
+    }
+    LayerArgs args{mixed_qkv, z, a, b, conv_ring, conv_w, A_log, dt_bias, norm_w, l2_eps,
+                   norm_eps, state, out, B, static_cast<int>(Hk), static_cast<int>(Hv),
+                   scratch_ring, scratch_state};
+    return launched(launch_layer_pair(args, static_cast<cudaStream_t>(stream)),
+                    "gdn_layer_pair");
 }
 
 }  // extern "C"

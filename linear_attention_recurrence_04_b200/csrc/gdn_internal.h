@@ -50,12 +50,15 @@ struct LayerArgs {
     int64_t B;
     int Hk;
     int Hv;
+    float* scratch_ring;    // pair only: ring after the tentative position
+    float* scratch_state;   // pair only: state after the tentative position
 };
 
 // Each launcher enqueues its kernel on `stream` and returns the launch status.
 cudaError_t launch_step(const StepArgs& a, cudaStream_t stream);
 cudaError_t launch_prefill(const PrefillArgs& a, cudaStream_t stream);
 cudaError_t launch_layer_decode(const LayerArgs& a, cudaStream_t stream);
+cudaError_t launch_layer_pair(const LayerArgs& a, cudaStream_t stream);
 
 // Value-heads-per-key-head ratios the fused layer kernel is compiled for.
 bool layer_decode_supports(int G);

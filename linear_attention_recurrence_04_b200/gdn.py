@@ -28,7 +28,8 @@ STATUS = {
 }
 
 # Every symbol that include/gdn.h declares.
-EXPORTS = ("gdn_status_string", "gdn_last_error", "gdn_step", "gdn_prefill", "gdn_layer_decode")
+EXPORTS = ("gdn_status_string", "gdn_last_error", "gdn_step", "gdn_prefill", "gdn_layer_decode",
+           "gdn_layer_pair")
 
 
 class GdnError(RuntimeError):
@@ -68,6 +69,8 @@ def load_library(path: Optional[str] = None) -> ctypes.CDLL:
     lib.gdn_prefill.argtypes = [_VP] * 7 + [_I64] * 6 + [_VP]
     lib.gdn_layer_decode.restype = ctypes.c_int
     lib.gdn_layer_decode.argtypes = [_VP] * 9 + [_F32, _F32] + [_VP, _VP] + [_I64] * 6 + [_VP]
+    lib.gdn_layer_pair.restype = ctypes.c_int
+    lib.gdn_layer_pair.argtypes = [_VP] * 9 + [_F32, _F32] + [_VP] * 4 + [_I64] * 6 + [_VP]
     if path is None:
         _lib = lib
     return lib
@@ -191,3 +194,40 @@ def layer_decode(mixed_qkv, z, a, b, conv_ring, conv_w, A_log, dt_bias, norm_w, 
                float(norm_eps), ptrs[9], ptrs[10], B, Hk, Hv, dk, dv, K, _stream(device, stream))
     _raise_on("gdn_layer_decode", st)
     return out
+
+
+def layer_pair(mixed_qkv, z, a, b, conv_ring, conv_w, A_log, dt_bias, norm_w, state,
+               scratch_ring=None, scratch_state=None, out=None, *, Hk: int, l2_eps: float = 1e-6,
+               norm_eps: float = 1e-6, stream=None):
+    """Two positions per sequence for speculative verification.
+
+    Position 0 commits into conv_ring and state (in place); position 1's ring
+    and state go to scratch_ring and scratch_state. Activations are
+    [B, 2, ...]. Returns (out [B, 2, Hv*128], scratch_ring, scratch_state).
+    """
+    if state.dim() != 4:
+        raise ValueError("state must be [B, Hv, dv, dk]")
+    B, Hv, dv, dk = state.shape
+    C, K = conv_w.shape
+    if scratch_ring is None:
+        scratch_ring = torch.empty_like(conv_ring)
+    if scratch_state is None:
+        scratch_state = torch.empty_like(state)
+    if out is None:
+        out = torch.empty((B, 2, Hv * dv), dtype=torch.float32, device=state.device)
+    names = ("mixed_qkv", "z", "a", "b", "conv_ring", "conv_w", "A_log", "dt_bias", "norm_w",
+             "state", "scratch_ring", "scratch_state", "out")
+    tensors = (mixed_qkv, z, a, b, conv_ring, conv_w, A_log, dt_bias, norm_w, state,
+               scratch_ring, scratch_state, out)
+    device = _dev(tensors, names)
+    expect = dict(mixed_qkv=(B, 2, C), z=(B, 2, Hv * dv), a=(B, 2, Hv), b=(B, 2, Hv),
+                  conv_ring=(B, K - 1, C), A_log=(Hv,), dt_bias=(Hv,), norm_w=(dv,),
+                  scratch_ring=(B, K - 1, C), scratch_state=(B, Hv, dv, dk), out=(B, 2, Hv * dv))
+    for n, t in zip(names, tensors):
+        if n in expect and tuple(t.shape) != expect[n]:
+            raise ValueError(f"{n} has shape {tuple(t.shape)}, expected {expect[n]}")
+    ptrs = [_ptr(t) for t in tensors]
+    st = _call(device, load_library().gdn_layer_pair, *ptrs[:9], float(l2_eps), float(norm_eps),
+               *ptrs[9:13], B, Hk, Hv, dk, dv, K, _stream(device, stream))
+    _raise_on("gdn_layer_pair", st)
+    return out, scratch_ring, scratch_state

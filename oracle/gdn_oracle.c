@@ -26,7 +26,10 @@
  *       SiLU, Q/K/V split, per-head Q/K L2 normalisation.
  *   [B] "Module linear_core" (cortiq_engine), entry "gdn_forward_batch":
  *       the recurrence runs sequentially over positions and is elementwise
- *       identical to the one-position path.
+ *       identical to the one-position path; entry "gdn_pair": a fused
+ *       two-position forward for speculative verification, where lane 1
+ *       commits into the state and lane 2 is tentative in scratch, the conv
+ *       ring and the recurrent state moving together.
  *
  * Readings where the pages are silent (each is listed with its reason in the
  * design notes): gate is a log-decay applied as exp(gate); the output scale
@@ -405,4 +408,68 @@ int oracle_gdn_layer_decode(const double *mixed_qkv, const double *z,
     free(gate);
     free(o);
     return rc;
+}
+
+/*
+ * Two-position speculative verify of the single-token layer, [B] entry
+ * "gdn_pair" and [L]: position 1 runs the layer and commits (ring and state
+ * are updated in place); position 2 continues from that committed result
+ * and its ring and state go to scratch (the caller keeps them on accept and
+ * drops them on reject). Plainly: two calls of the one-token layer, the
+ * first on the live buffers, the second on copies of them.
+ *   mixed_qkv [B][2][C]; z [B][2][Hv*dv]; a_in, b_in [B][2][Hv]
+ *   ring [B][K-1][C] in/out; state [B][Hv][dv][dk] in/out
+ *   scratch_ring [B][K-1][C] out; scratch_state [B][Hv][dv][dk] out
+ *   out [B][2][Hv*dv]
+ */
+int oracle_gdn_layer_pair(const double *mixed_qkv, const double *z,
+                          const double *a_in, const double *b_in,
+                          double *ring, const double *conv_w,
+                          const double *A_log, const double *dt_bias,
+                          const double *norm_w, double l2_eps,
+                          double norm_eps, double *state,
+                          double *scratch_ring, double *scratch_state,
+                          double *out, int64_t B, int64_t Hk, int64_t Hv,
+                          int64_t dk, int64_t dv, int64_t K,
+                          const int64_t *seqs, int64_t n_seqs)
+{
+    if (B < 0 || K < 1 || !dims_ok(Hk, Hv, dk, dv))
+        return -1;
+    const int64_t C = 2 * Hk * dk + Hv * dv;
+    const int64_t count = seqs ? n_seqs : B;
+    for (int64_t n = 0; n < count; ++n) {
+        const int64_t b = seqs ? seqs[n] : n;
+        if (b < 0 || b >= B)
+            return -1;
+    }
+    for (int64_t n = 0; n < count; ++n) {
+        const int64_t b = seqs ? seqs[n] : n;
+        double *rg = ring + b * (K - 1) * C;
+        double *st = state + b * Hv * dv * dk;
+        double *srg = scratch_ring + b * (K - 1) * C;
+        double *sst = scratch_state + b * Hv * dv * dk;
+        /* lane 1: commits into the live ring and state */
+        int rc = oracle_gdn_layer_decode(mixed_qkv + (b * 2 + 0) * C,
+                                         z + (b * 2 + 0) * Hv * dv,
+                                         a_in + (b * 2 + 0) * Hv,
+                                         b_in + (b * 2 + 0) * Hv, rg, conv_w,
+                                         A_log, dt_bias, norm_w, l2_eps,
+                                         norm_eps, st, out + (b * 2 + 0) * Hv * dv,
+                                         1, Hk, Hv, dk, dv, K, NULL, 0);
+        if (rc)
+            return rc;
+        /* lane 2: continues on copies of the committed ring and state */
+        memcpy(srg, rg, (size_t)((K - 1) * C) * sizeof(double));
+        memcpy(sst, st, (size_t)(Hv * dv * dk) * sizeof(double));
+        rc = oracle_gdn_layer_decode(mixed_qkv + (b * 2 + 1) * C,
+                                     z + (b * 2 + 1) * Hv * dv,
+                                     a_in + (b * 2 + 1) * Hv,
+                                     b_in + (b * 2 + 1) * Hv, srg, conv_w, A_log,
+                                     dt_bias, norm_w, l2_eps, norm_eps, sst,
+                                     out + (b * 2 + 1) * Hv * dv, 1, Hk, Hv, dk,
+                                     dv, K, NULL, 0);
+        if (rc)
+            return rc;
+    }
+    return 0;
 }

@@ -74,6 +74,10 @@ class Oracle:
         lib.oracle_gdn_layer_decode.argtypes = [_PD, _PD, _PD, _PD, _PD, _PD, _PD, _PD, _PD,
                                                 _DBL, _DBL, _PD, _PD,
                                                 _I64, _I64, _I64, _I64, _I64, _I64, _PI, _I64]
+        lib.oracle_gdn_layer_pair.restype = ctypes.c_int
+        lib.oracle_gdn_layer_pair.argtypes = [_PD, _PD, _PD, _PD, _PD, _PD, _PD, _PD, _PD,
+                                              _DBL, _DBL, _PD, _PD, _PD, _PD,
+                                              _I64, _I64, _I64, _I64, _I64, _I64, _PI, _I64]
         self.lib = lib
 
     # -- recurrence ---------------------------------------------------------
@@ -174,6 +178,35 @@ class Oracle:
                                               _ptr(out), B, Hk, Hv, dk, dv, K, sp, ns)
         _check(rc, "oracle_gdn_layer_decode")
         return out, rg, st
+
+
+    def layer_pair(self, mixed_qkv, z, a, b, ring, conv_w, A_log, dt_bias, norm_w, state, *,
+                   Hk, l2_eps=1e-6, norm_eps=1e-6, seqs=None):
+        """Two positions per sequence: position 1 commits, position 2 is tentative.
+
+        Shapes: mixed_qkv [B,2,C]; z [B,2,Hv*dv]; a, b [B,2,Hv]; ring [B,K-1,C];
+        conv_w [C,K]; A_log, dt_bias [Hv]; norm_w [dv]; state [B,Hv,dv,dk].
+        Returns (out [B,2,Hv*dv], ring, state, scratch_ring, scratch_state):
+        ring/state after position 1, scratch_* after position 2.
+        """
+        st = _f64(state)
+        B, Hv, dv, dk = st.shape
+        x, zz, aa, bb = _f64(mixed_qkv), _f64(z), _f64(a), _f64(b)
+        rg, w, al, dt, nw = _f64(ring), _f64(conv_w), _f64(A_log), _f64(dt_bias), _f64(norm_w)
+        C, K = w.shape
+        assert x.shape == (B, 2, C) and C == 2 * Hk * dk + Hv * dv
+        assert zz.shape == (B, 2, Hv * dv) and aa.shape == (B, 2, Hv) and bb.shape == aa.shape
+        assert rg.shape == (B, K - 1, C) and nw.shape == (dv,)
+        out = np.zeros((B, 2, Hv * dv))
+        srg = np.zeros_like(rg)
+        sst = np.zeros_like(st)
+        sp, ns, _keep = _units(seqs)
+        rc = self.lib.oracle_gdn_layer_pair(_ptr(x), _ptr(zz), _ptr(aa), _ptr(bb), _ptr(rg),
+                                            _ptr(w), _ptr(al), _ptr(dt), _ptr(nw), float(l2_eps),
+                                            float(norm_eps), _ptr(st), _ptr(srg), _ptr(sst),
+                                            _ptr(out), B, Hk, Hv, dk, dv, K, sp, ns)
+        _check(rc, "oracle_gdn_layer_pair")
+        return out, rg, st, srg, sst
 
 
 _DEFAULT: Optional[Oracle] = None

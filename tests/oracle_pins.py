@@ -350,6 +350,51 @@ def pin_layer_library(o):
     _close(out, want, 1e-11, "layer out")
 
 
+def _torch_layer(c, x, z, a, b, ring, state):
+    """One token of the layer from torch routines and the product-form
+    recurrence; returns (out [B, Hv*dv], new ring, new state)."""
+    Hk, Hv, dk, dv = c["Hk"], c["Hv"], c["dk"], c["dv"]
+    q, k, v, beta, gate, ring_t = _torch_prestate(x, ring, c["w"], a, b, c["A_log"],
+                                                  c["dt_bias"], Hk, Hv, dk, dv, 1e-6)
+    B = x.shape[0]
+    out = np.zeros((B, Hv * dv))
+    st = np.zeros_like(state)
+    for bb in range(B):
+        for h in range(Hv):
+            g = h % Hk
+            st[bb, h], on = textbook_head(state[bb, h], q[bb, g], k[bb, g], v[bb, h],
+                                          beta[bb, h], gate[bb, h])
+            zt = torch.from_numpy(z[bb, h * dv:(h + 1) * dv])
+            y = F.rms_norm(torch.from_numpy(on), (dv,), weight=torch.from_numpy(c["norm_w"]),
+                           eps=1e-6) * F.silu(zt)
+            out[bb, h * dv:(h + 1) * dv] = y.numpy()
+    return out, ring_t, st
+
+
+def pin_layer_pair_library(o):
+    """Speculative two-position verify ("Module linear_core", gdn_pair):
+    position 1 commits (ring and state), position 2 continues from the
+    committed result into scratch; checked against the torch composition
+    applied twice."""
+    c = _layer_case(25)
+    r = _rng(26)
+    B, C = c["x"].shape
+    Hv, dv = c["Hv"], c["dv"]
+    x2 = np.stack([c["x"], r.normal(size=(B, C))], axis=1)
+    z2 = np.stack([c["z"], r.normal(size=(B, Hv * dv))], axis=1)
+    a2 = np.stack([c["a"], r.normal(size=(B, Hv))], axis=1)
+    b2 = np.stack([c["b"], r.normal(size=(B, Hv))], axis=1)
+    out, ring, st, sring, sst = o.layer_pair(x2, z2, a2, b2, c["ring"], c["w"], c["A_log"],
+                                             c["dt_bias"], c["norm_w"], c["state"], Hk=c["Hk"])
+    o1, r1, s1 = _torch_layer(c, x2[:, 0], z2[:, 0], a2[:, 0], b2[:, 0], c["ring"], c["state"])
+    o2, r2, s2 = _torch_layer(c, x2[:, 1], z2[:, 1], a2[:, 1], b2[:, 1], r1, s1)
+    _close(out[:, 0], o1, 1e-11, "pair out 1")
+    _close(out[:, 1], o2, 1e-11, "pair out 2")
+    assert np.array_equal(ring, r1) and np.array_equal(sring, r2), "pair rings"
+    _close(st, s1, 1e-12, "pair committed state")
+    _close(sst, s2, 1e-12, "pair scratch state")
+
+
 ALL_PINS = [
     pin_golden_step_cases,
     pin_delta_rule_closed_form,
@@ -363,4 +408,5 @@ ALL_PINS = [
     pin_prestate_special_values,
     pin_tail_library,
     pin_layer_library,
+    pin_layer_pair_library,
 ]

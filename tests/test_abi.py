@@ -121,3 +121,21 @@ def test_binding_rejects_cpu_tensors():
     with pytest.raises(ValueError):
         gdn.step(st, q, q, torch.zeros(1, 1, 32, 128), torch.zeros(1, 1, 32),
                  torch.zeros(1, 1, 32), out=torch.zeros(1, 1, 32, 128))
+
+
+def test_layer_pair_argument_checks(lib):
+    def f(B=1, Hk=16, Hv=32, K=4, state=A16, sring=fake(11), sstate=fake(12), out=fake(10)):
+        return lib.gdn_layer_pair(A16b, A16c, fake(3), fake(4), fake(5), fake(6), fake(7),
+                                  fake(8), fake(9), ctypes.c_float(1e-6), ctypes.c_float(1e-6),
+                                  state, sring, sstate, out, B, Hk, Hv, 128, 128, K, None)
+    assert f(B=-1) == SHAPE
+    assert f(K=5) == UNSUP
+    assert f(sring=0) == NULL
+    assert f(sstate=0) == NULL
+    assert f(sstate=fake(12) + 8) == ALIGN
+    assert f(sstate=A16 + 65536) == ALIAS           # scratch state inside the live state
+    assert f(sring=fake(5) + 16) == ALIAS           # scratch ring inside the live ring
+    assert f(out=A16b + 32768 + 64) == ALIAS        # out inside mixed_qkv [1][2][8192]
+    assert lib.gdn_layer_pair(0, 0, 0, 0, 0, 0, 0, 0, 0, ctypes.c_float(1e-6),
+                              ctypes.c_float(1e-6), 0, 0, 0, 0, 0, 16, 32, 128, 128, 4,
+                              None) == OK

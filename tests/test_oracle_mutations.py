@@ -62,6 +62,11 @@ MUTATIONS = [
     ("layer broadcast h/2", "const int64_t g = h % Hk;\n            rc = gdn_head_token",
      "const int64_t g = h / (Hv / Hk);\n            rc = gdn_head_token"),
     ("layer tail reads head 0 z", "z + b * Hv * dv + h * dv, norm_w", "z + b * Hv * dv, norm_w"),
+    # two-position verify
+    ("pair lane 2 reuses lane 1 input", "rc = oracle_gdn_layer_decode(mixed_qkv + (b * 2 + 1) * C,",
+     "rc = oracle_gdn_layer_decode(mixed_qkv + (b * 2 + 0) * C,"),
+    ("pair scratch starts from lane-2 ring slot", "memcpy(srg, rg, (size_t)((K - 1) * C) * sizeof(double));",
+     "memcpy(srg, rg, (size_t)((K - 1) * C) * sizeof(double)); srg[0] = srg[1];"),
 ]
 
 
