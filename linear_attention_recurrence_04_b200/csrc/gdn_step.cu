@@ -7,7 +7,7 @@
 //   4. M[j] += delta[j] k   5. out[j] = M_new[j].q / sqrt(128).
 //
 // Design: every row j of M is independent once k, q, v[j], beta and gate are
-// known, so the kernel streams rows. A warp owns R consecutive rows of one
+// known, so the kernel streams rows. A warp owns R = 4 consecutive rows of one
 // head; lane l holds columns [4l, 4l+4) of each row as one float4, so a row
 // is one coalesced 512-byte access. All R row loads are issued before any
 // arithmetic, the five steps run in registers (two warp-shuffle reductions
@@ -19,7 +19,7 @@
 #include "gdn_internal.h"
 
 #ifndef GDN_STEP_ROWS
-#define GDN_STEP_ROWS 8          // rows per warp task
+#define GDN_STEP_ROWS 4          // rows per warp task
 #endif
 #ifndef GDN_STEP_THREADS
 #define GDN_STEP_THREADS 256     // threads per CTA
@@ -27,6 +27,7 @@
 #ifndef GDN_STEP_PREFETCH
 #define GDN_STEP_PREFETCH 1      // load the next task's rows before computing
 #endif
+
 
 namespace gdn {
 
@@ -138,11 +139,11 @@ cudaError_t launch_step(const StepArgs& a, cudaStream_t stream) {
     if (n_tasks == 0) return cudaSuccess;
     constexpr int threads = GDN_STEP_THREADS;
     constexpr int warps_per_cta = threads / 32;
+    const int64_t needed = (n_tasks + warps_per_cta - 1) / warps_per_cta;
     int per_sm = 0;
     cudaError_t err = resident_ctas_per_sm(reinterpret_cast<const void*>(&step_kernel<R>),
                                            threads, &per_sm);
     if (err != cudaSuccess) return err;
-    const int64_t needed = (n_tasks + warps_per_cta - 1) / warps_per_cta;
     const int64_t resident = static_cast<int64_t>(device_sm_count()) * per_sm;
     const int grid = static_cast<int>(needed < resident ? needed : resident);
     step_kernel<R><<<grid, threads, 0, stream>>>(a.state, a.q, a.k, a.v, a.beta, a.gate, a.out,
