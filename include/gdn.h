@@ -170,6 +170,28 @@ gdn_status gdn_layer_pair(const float *mixed_qkv, const float *z, const float *a
                           float *out, int64_t B, int64_t Hk, int64_t Hv, int64_t dk,
                           int64_t dv, int64_t K, void *stream);
 
+/*
+ * gdn_linear_bf16 -- dense projection on the tensor cores:
+ *   y[M][N] = x[M][K] . w[N][K]^T
+ * with bf16 inputs and fp32 accumulation and output. These are the layer's
+ * projections ("Red Lite dev15e -- complete recurrent DeltaNet layer
+ * composition", opening list: attn_qkv 2048 -> 8192, attn_gate 2048 ->
+ * 4096, ssm_ba 2048 -> 64, ssm_out 4096 -> 2048), here with dense bf16
+ * weights, run as matrix-matrix products over a batch of positions
+ * ("Module linear_core", entry "gdn_forward_batch").
+ *
+ *   x       [M][K] bf16 (uint16 bit patterns), row-major, 16-byte aligned
+ *   w       [N][K] bf16, row-major (the usual [out][in] weight layout)
+ *   y       [M][N] fp32 output, 16-byte aligned, must not overlap x or w
+ *   K       a multiple of 8 (16-byte rows for the tensor-memory copies);
+ *           K = 0 gives y = 0
+ *   status  optional device pointer to a zero-initialised 32-bit word; if a
+ *           kernel-internal wait ever times out (2 s) a non-zero bit is ORed
+ *           into it and the kernel returns without hanging. NULL: not reported.
+ */
+gdn_status gdn_linear_bf16(const void *x, const void *w, float *y, int64_t M, int64_t N,
+                           int64_t K, uint32_t *status, void *stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -6,8 +6,8 @@ torch device tensors to it; it loads the library on first use and raises if
 the library is missing: there is no CPU fallback. ``inputs`` draws the seeded
 synthetic workloads and needs neither the library nor a GPU.
 """
-_BINDING = ("GdnError", "step", "prefill", "layer_decode", "layer_pair", "library_path",
-            "status_string")
+_BINDING = ("GdnError", "step", "prefill", "layer_decode", "layer_pair", "linear_bf16",
+            "library_path", "status_string")
 
 
 def __getattr__(name):

@@ -314,4 +314,32 @@ gdn_status gdn_layer_pair(const float* mixed_qkv, const float* z, const float* a
                     "gdn_layer_pair");
 }
 
+gdn_status gdn_linear_bf16(const void* x, const void* w, float* y, int64_t M, int64_t N,
+                           int64_t K, uint32_t* status, void* stream) {
+    if (M < 0 || N < 0 || K < 0)
+        return fail(GDN_ERR_SHAPE, "gdn_linear_bf16: negative M=%lld N=%lld K=%lld", (long long)M,
+                    (long long)N, (long long)K);
+    if (K % 8 != 0)
+        return fail(GDN_ERR_UNSUPPORTED, "gdn_linear_bf16: K=%lld must be a multiple of 8", (long long)K);
+    if (M > (int64_t)65535 * 128 || N > INT32_MAX / 2 || K > INT32_MAX / 2)
+        return fail(GDN_ERR_OVERFLOW, "gdn_linear_bf16: M, N or K too large");
+    int64_t xy = 0, xk = 0, wk = 0;
+    if (!mul_ok(M, N, &xy) || !mul_ok(M, K, &xk) || !mul_ok(N, K, &wk))
+        return fail(GDN_ERR_OVERFLOW, "gdn_linear_bf16: size overflow");
+    if (M == 0 || N == 0) { g_last_error[0] = '\0'; return GDN_OK; }
+    if (!y || (K > 0 && (!x || !w)))
+        return fail(GDN_ERR_NULL, "gdn_linear_bf16: a tensor pointer is NULL");
+    if (!aligned(y, 16) || (K > 0 && (!aligned(x, 16) || !aligned(w, 16))) ||
+        (status && !aligned(status, 4)))
+        return fail(GDN_ERR_ALIGN, "gdn_linear_bf16: x, w, y need 16-byte alignment");
+    const Span ins[] = {{x, xk * 2, "x"}, {w, wk * 2, "w"}, {status, status ? 4 : 0, "status"}};
+    gdn_status st = check_spans(ins, 3, 0, Span{y, xy * 4, "y"});
+    if (st != GDN_OK) return st;
+    if (K == 0)    // an empty sum: y = 0
+        return launched(cudaMemsetAsync(y, 0, static_cast<size_t>(xy) * 4,
+                                        static_cast<cudaStream_t>(stream)), "gdn_linear_bf16");
+    LinearArgs a{x, w, y, M, N, K, status};
+    return launched(launch_linear_bf16(a, static_cast<cudaStream_t>(stream)), "gdn_linear_bf16");
+}
+
 }  // extern "C"

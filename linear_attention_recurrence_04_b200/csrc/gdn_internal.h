@@ -54,11 +54,22 @@ struct LayerArgs {
     float* scratch_state;   // pair only: state after the tentative position
 };
 
+struct LinearArgs {
+    const void* x;     // [M][K] bf16
+    const void* w;     // [N][K] bf16
+    float* y;          // [M][N]
+    int64_t M;
+    int64_t N;
+    int64_t K;
+    uint32_t* status;  // optional device word for timeout bits
+};
+
 // Each launcher enqueues its kernel on `stream` and returns the launch status.
 cudaError_t launch_step(const StepArgs& a, cudaStream_t stream);
 cudaError_t launch_prefill(const PrefillArgs& a, cudaStream_t stream);
 cudaError_t launch_layer_decode(const LayerArgs& a, cudaStream_t stream);
 cudaError_t launch_layer_pair(const LayerArgs& a, cudaStream_t stream);
+cudaError_t launch_linear_bf16(const LinearArgs& a, cudaStream_t stream);
 
 // Value-heads-per-key-head ratios the fused layer kernel is compiled for.
 bool layer_decode_supports(int G);

@@ -1,0 +1,247 @@
+// gdn_linear.cu -- dense projection y[M][N] (fp32) = x[M][K] (bf16) . W[N][K]^T
+// (bf16) on the sm_100a tensor cores.
+//
+// These are the layer's input and output projections ("Red Lite dev15e --
+// complete recurrent DeltaNet layer composition", opening list: attn_qkv
+// 2048 -> 8192, attn_gate 2048 -> 4096, ssm_ba 2048 -> 64, ssm_out 4096 ->
+// 2048), here with dense bf16 weights; "Module linear_core", entry
+// "gdn_forward_batch", runs them as matrix-matrix products over a batch of
+// positions.
+//
+// Design (one 128 x BN output tile per CTA, BN = 256, 192 threads):
+//   warp 0      one thread issues TMA loads of 128 x 64 tiles of x and W
+//               (128-byte swizzle) into an S-stage shared-memory ring;
+//   warp 1      owns the TMEM accumulator (BN fp32 columns x 128 lanes) and
+//               one thread issues tcgen05.mma (bf16, M = 128, N = BN, K = 16)
+//               per 32-byte K step; a tcgen05.commit per stage frees the slot
+//               back to the producer, a final one signals the epilogue;
+//   warps 2-5   read the accumulator with tcgen05.ld (each warp its TMEM lane
+//               quarter, i.e. 32 rows) and store fp32 rows.
+// Tiles past M, N or K are zero-filled by TMA and masked on store. Every
+// mbarrier wait gives up after 2 s, ORs an error bit into the caller's
+// status word (if given), lets in-flight copies land and frees TMEM.
+#include <cuda.h>
+
+#include "gdn_common.cuh"
+#include "gdn_internal.h"
+#include "gdn_tc.cuh"
+
+#ifndef GDN_LINEAR_BN
+#define GDN_LINEAR_BN 256        // output tile width (TMEM columns)
+#endif
+#ifndef GDN_LINEAR_STAGES
+#define GDN_LINEAR_STAGES (GDN_LINEAR_BN == 256 ? 4 : 6)
+#endif
+
+namespace gdn {
+
+namespace {
+
+constexpr int kBM = 128;
+constexpr int kBK = 64;                  // 64 bf16 = one 128-byte swizzle row
+constexpr int kStages = GDN_LINEAR_STAGES;
+constexpr int kThreads = 192;
+
+template <int BN>
+struct LinearSmem {
+    static constexpr uint32_t kA = kBM * kBK * 2;
+    static constexpr uint32_t kB = BN * kBK * 2;
+    static constexpr uint32_t kStage = kA + kB;
+    static constexpr size_t kDynamic = static_cast<size_t>(kStage) * kStages + 1024;
+};
+
+template <int BN>
+__global__ void __launch_bounds__(kThreads, 1)
+linear_bf16_kernel(const __grid_constant__ CUtensorMap tmap_x,
+                   const __grid_constant__ CUtensorMap tmap_w, float* __restrict__ y, int M,
+                   int N, int K, uint32_t* __restrict__ status) {
+    using L = LinearSmem<BN>;
+    extern __shared__ uint8_t smem_raw[];
+    __shared__ __align__(8) uint64_t full[kStages];
+    __shared__ __align__(8) uint64_t empty[kStages];
+    __shared__ __align__(8) uint64_t done;
+    __shared__ uint32_t tmem_slot;
+    __shared__ int issued, consumed, failed;
+
+    // 1024-byte aligned base for the swizzled tiles
+    const uint32_t raw = tc::smem_u32(smem_raw);
+    const uint32_t base = (raw + 1023u) & ~1023u;
+
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+    const int m0 = blockIdx.y * kBM;
+    const int n0 = blockIdx.x * BN;
+    const int n_kt = (K + kBK - 1) / kBK;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < kStages; ++s) {
+            tc::mbar_init(tc::smem_u32(&full[s]), 1);
+            tc::mbar_init(tc::smem_u32(&empty[s]), 1);
+        }
+        tc::mbar_init(tc::smem_u32(&done), 1);
+        tc::fence_mbar_init();
+        issued = 0;
+        consumed = 0;
+        failed = 0;
+    }
+    if (warp == 1) {
+        tc::tmem_alloc(tc::smem_u32(&tmem_slot), BN);
+        tc::tmem_relinquish();
+    }
+    tc::tc_fence_before();
+    __syncthreads();
+    tc::tc_fence_after();
+    const uint32_t tmem = tmem_slot;
+
+    if (warp == 0 && lane == 0) {
+        // ---- producer --------------------------------------------------------
+        tc::prefetch_tmap(&tmap_x);
+        tc::prefetch_tmap(&tmap_w);
+        for (int kt = 0; kt < n_kt; ++kt) {
+            const int s = kt % kStages;
+            const uint32_t ph = (kt / kStages) & 1;
+            if (!tc::mbar_wait(tc::smem_u32(&empty[s]), ph ^ 1)) {
+                if (status) atomicOr(status, tc::kTimeoutProducer);
+                atomicExch(&failed, 1);
+                break;
+            }
+            if (*reinterpret_cast<volatile int*>(&failed)) break;
+            const uint32_t a = base + s * L::kStage;
+            tc::mbar_arrive_expect_tx(tc::smem_u32(&full[s]), L::kStage);
+            tc::tma_load_2d(a, &tmap_x, tc::smem_u32(&full[s]), kt * kBK, m0);
+            tc::tma_load_2d(a + L::kA, &tmap_w, tc::smem_u32(&full[s]), kt * kBK, n0);
+            issued = kt + 1;
+        }
+    } else if (warp == 1 && lane == 0) {
+        // ---- MMA issuer ------------------------------------------------------
+        const uint32_t idesc = tc::idesc_bf16_f32(kBM, BN);
+        bool ok = true;
+        for (int kt = 0; kt < n_kt; ++kt) {
+            const int s = kt % kStages;
+            const uint32_t ph = (kt / kStages) & 1;
+            if (!tc::mbar_wait(tc::smem_u32(&full[s]), ph) ||
+                *reinterpret_cast<volatile int*>(&failed)) {
+                if (status) atomicOr(status, tc::kTimeoutMma);
+                atomicExch(&failed, 1);
+                ok = false;
+                break;
+            }
+            consumed = kt + 1;
+            tc::tc_fence_after();
+            const uint32_t a = base + s * L::kStage;
+            const uint32_t b = a + L::kA;
+#pragma unroll
+            for (int kk = 0; kk < kBK / 16; ++kk) {
+                tc::mma_bf16(tmem, tc::desc_k_sw128(a + kk * 32), tc::desc_k_sw128(b + kk * 32),
+                             idesc, (kt > 0 || kk > 0) ? 1u : 0u);
+            }
+            tc::mma_commit(tc::smem_u32(&empty[s]));      // slot free once these MMAs finish
+        }
+        if (ok) tc::mma_commit(tc::smem_u32(&done));     // accumulator complete
+    } else if (warp >= 2) {
+        // ---- epilogue: TMEM -> registers -> global ---------------------------
+        const int quarter = warp & 3;                      // TMEM lanes 32 q .. 32 q + 31
+        if (!tc::mbar_wait(tc::smem_u32(&done), 0)) {
+            if (status) atomicOr(status, tc::kTimeoutEpilogue);
+            atomicExch(&failed, 1);
+        } else {
+            tc::tc_fence_after();
+            const int row = m0 + quarter * 32 + lane;
+            const bool row_ok = row < M;
+            float* yrow = y + static_cast<int64_t>(row) * N;
+#pragma unroll 1
+            for (int c0 = 0; c0 < BN; c0 += 32) {
+                uint32_t r[32];
+                tc::tmem_ld_32x32b_x32(tmem + (static_cast<uint32_t>(quarter * 32) << 16) + c0, r);
+                tc::tmem_ld_wait();
+                const int col = n0 + c0;
+                if (!row_ok || col >= N) continue;
+                if (col + 32 <= N && (N & 3) == 0) {
+#pragma unroll
+                    for (int j = 0; j < 32; j += 4) {
+                        *reinterpret_cast<float4*>(yrow + col + j) =
+                            make_float4(__uint_as_float(r[j]), __uint_as_float(r[j + 1]),
+                                        __uint_as_float(r[j + 2]), __uint_as_float(r[j + 3]));
+                    }
+                } else {
+#pragma unroll
+                    for (int j = 0; j < 32; ++j)
+                        if (col + j < N) yrow[col + j] = __uint_as_float(r[j]);
+                }
+            }
+        }
+    }
+
+    // On failure, let copies that were issued but never consumed land before
+    // the shared memory goes away (bounded like every other wait).
+    __syncthreads();
+    if (threadIdx.x == 0 && failed) {
+        for (int kt = consumed; kt < issued; ++kt)
+            tc::mbar_wait(tc::smem_u32(&full[kt % kStages]), (kt / kStages) & 1);
+    }
+    tc::tc_fence_before();
+    __syncthreads();
+    tc::tc_fence_after();
+    if (warp == 1) tc::tmem_dealloc(tmem, BN);
+}
+
+// cuTensorMapEncodeTiled through the runtime's driver entry point (no link
+// against libcuda).
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                   const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                   const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                   CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+    static EncodeTiledFn fn = nullptr;
+    if (!fn) {
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+                cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(p);
+    }
+    return fn;
+}
+
+// Row-major bf16 matrix [rows][K] as a 2D tensor map with box [box_rows][64].
+bool make_tmap(CUtensorMap* map, const void* ptr, int64_t rows, int64_t K, int box_rows) {
+    EncodeTiledFn fn = encode_fn();
+    if (!fn) return false;
+    const cuuint64_t dims[2] = {static_cast<cuuint64_t>(K), static_cast<cuuint64_t>(rows)};
+    const cuuint64_t strides[1] = {static_cast<cuuint64_t>(K) * 2};
+    const cuuint32_t box[2] = {static_cast<cuuint32_t>(kBK), static_cast<cuuint32_t>(box_rows)};
+    const cuuint32_t estr[2] = {1, 1};
+    return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(ptr), dims, strides, box,
+              estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) ==
+           CUDA_SUCCESS;
+}
+
+template <int BN>
+cudaError_t launch_bn(const LinearArgs& a, cudaStream_t stream) {
+    CUtensorMap tx, tw;
+    if (!make_tmap(&tx, a.x, a.M, a.K, kBM) || !make_tmap(&tw, a.w, a.N, a.K, BN))
+        return cudaErrorInvalidValue;
+    const size_t smem = LinearSmem<BN>::kDynamic;
+    cudaError_t err = cudaFuncSetAttribute(linear_bf16_kernel<BN>,
+                                           cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                           static_cast<int>(smem));
+    if (err != cudaSuccess) return err;
+    const dim3 grid(static_cast<unsigned>((a.N + BN - 1) / BN),
+                    static_cast<unsigned>((a.M + kBM - 1) / kBM));
+    linear_bf16_kernel<BN><<<grid, kThreads, smem, stream>>>(tx, tw, a.y, static_cast<int>(a.M),
+                                                             static_cast<int>(a.N),
+                                                             static_cast<int>(a.K), a.status);
+    return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_linear_bf16(const LinearArgs& a, cudaStream_t stream) {
+    if (a.M == 0 || a.N == 0) return cudaSuccess;
+    return launch_bn<GDN_LINEAR_BN>(a, stream);
+}
+
+}  // namespace gdn

@@ -29,7 +29,7 @@ STATUS = {
 
 # Every symbol that include/gdn.h declares.
 EXPORTS = ("gdn_status_string", "gdn_last_error", "gdn_step", "gdn_prefill", "gdn_layer_decode",
-           "gdn_layer_pair")
+           "gdn_layer_pair", "gdn_linear_bf16")
 
 
 class GdnError(RuntimeError):
@@ -71,6 +71,8 @@ def load_library(path: Optional[str] = None) -> ctypes.CDLL:
     lib.gdn_layer_decode.argtypes = [_VP] * 9 + [_F32, _F32] + [_VP, _VP] + [_I64] * 6 + [_VP]
     lib.gdn_layer_pair.restype = ctypes.c_int
     lib.gdn_layer_pair.argtypes = [_VP] * 9 + [_F32, _F32] + [_VP] * 4 + [_I64] * 6 + [_VP]
+    lib.gdn_linear_bf16.restype = ctypes.c_int
+    lib.gdn_linear_bf16.argtypes = [_VP, _VP, _VP, _I64, _I64, _I64, _VP, _VP]
     if path is None:
         _lib = lib
     return lib
@@ -231,3 +233,32 @@ def layer_pair(mixed_qkv, z, a, b, conv_ring, conv_w, A_log, dt_bias, norm_w, st
                *ptrs[9:13], B, Hk, Hv, dk, dv, K, _stream(device, stream))
     _raise_on("gdn_layer_pair", st)
     return out, scratch_ring, scratch_state
+
+
+def linear_bf16(x, w, y=None, *, status=None, stream=None):
+    """y = x @ w.T on the tensor cores: x [M, K] bf16, w [N, K] bf16, y [M, N]
+    fp32. `status`, if given, is a zero-initialised int32 CUDA tensor that
+    receives timeout bits (see include/gdn.h)."""
+    if x.dim() != 2 or w.dim() != 2 or x.shape[1] != w.shape[1]:
+        raise ValueError("x must be [M, K] and w [N, K]")
+    M, K = x.shape
+    N = w.shape[0]
+    for n, t in (("x", x), ("w", w)):
+        if t.dtype is not torch.bfloat16 or not t.is_cuda or not t.is_contiguous():
+            raise TypeError(f"{n} must be a contiguous bfloat16 CUDA tensor")
+    if y is None:
+        y = torch.empty((M, N), dtype=torch.float32, device=x.device)
+    device = _dev((y,), ("y",))
+    if x.device != device or w.device != device:
+        raise ValueError("x, w and y must be on one device")
+    if tuple(y.shape) != (M, N):
+        raise ValueError(f"y has shape {tuple(y.shape)}, expected {(M, N)}")
+    sp = 0
+    if status is not None:
+        if status.dtype is not torch.int32 or status.device != device or status.numel() != 1:
+            raise TypeError("status must be a one-element int32 tensor on the same device")
+        sp = status.data_ptr()
+    st = _call(device, load_library().gdn_linear_bf16, _ptr(x), _ptr(w), _ptr(y), M, N, K, sp,
+               _stream(device, stream))
+    _raise_on("gdn_linear_bf16", st)
+    return y

@@ -26,7 +26,7 @@ def lib():
 def declared_functions():
     text = open(HEADER).read()
     text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
-    return sorted(set(re.findall(r"\b(gdn_[a-z_]+)\s*\(", text)))
+    return sorted(set(re.findall(r"\b(gdn_[a-z0-9_]+)\s*\(", text)))
 
 
 def test_header_declares_the_binding_exports():
@@ -139,3 +139,15 @@ def test_layer_pair_argument_checks(lib):
     assert lib.gdn_layer_pair(0, 0, 0, 0, 0, 0, 0, 0, 0, ctypes.c_float(1e-6),
                               ctypes.c_float(1e-6), 0, 0, 0, 0, 0, 16, 32, 128, 128, 4,
                               None) == OK
+
+
+def test_linear_argument_checks(lib):
+    f = lambda x=fake(1), w=fake(2), y=fake(3), M=4, N=4, K=16, st=0: lib.gdn_linear_bf16(
+        x, w, y, M, N, K, st, None)
+    assert f(K=12) == UNSUP
+    assert f(M=-1) == SHAPE
+    assert f(x=0) == NULL
+    assert f(y=fake(3) + 8) == ALIGN
+    assert f(y=fake(1) + 16) == ALIAS
+    assert f(M=1 << 30) == OVERFLOW
+    assert lib.gdn_linear_bf16(0, 0, 0, 0, 7, 16, 0, None) == OK

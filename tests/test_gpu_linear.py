@@ -1,0 +1,63 @@
+"""gdn_linear_bf16 (tcgen05 + TMA projection GEMM) against an fp64 matmul of
+the same bf16 values, through the C ABI."""
+import numpy as np
+import pytest
+import torch
+
+from linear_attention_recurrence_04_b200 import gdn
+
+pytestmark = pytest.mark.gpu
+
+
+def bf16_pair(M, N, K, seed, scale=1.0):
+    g = torch.Generator().manual_seed(seed)
+    x = (torch.randn(M, K, generator=g) * scale).to(torch.bfloat16)
+    w = (torch.randn(N, K, generator=g) / K ** 0.5).to(torch.bfloat16)
+    return x, w
+
+
+def check(x, w, y):
+    xd = x.to(torch.float64).numpy()
+    wd = w.to(torch.float64).numpy()
+    ref = xd @ wd.T
+    mag = np.abs(xd) @ np.abs(wd).T                 # sum of |products| per element
+    err = np.abs(y.cpu().numpy().astype(np.float64) - ref)
+    # fp32 accumulation of exact bf16 x bf16 products: a few units of fp32
+    # rounding relative to the sum of magnitudes
+    bound = 4e-7 * np.sqrt(x.shape[1]) * mag + 1e-30
+    worst = float(np.max(err / bound)) if err.size else 0.0
+    assert worst <= 1.0, f"error {worst:.2f} x bound (max abs {err.max():.3e})"
+    return float(err.max())
+
+
+@pytest.mark.parametrize("M,N,K", [(128, 128, 64), (200, 300, 136), (1, 8, 8), (129, 257, 64),
+                                   (256, 4096 + 64, 2048), (513, 2048, 4096)])
+def test_linear_parity(M, N, K):
+    x, w = bf16_pair(M, N, K, seed=M + N + K)
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    y = gdn.linear_bf16(x.cuda(), w.cuda(), status=status)
+    torch.cuda.synchronize()
+    assert int(status.item()) == 0
+    check(x, w, y)
+
+
+def test_linear_large_sampled():
+    """A projection-sized product (4096 x 8192 x 2048): sampled rows checked."""
+    M, N, K = 4096, 8192, 2048
+    x, w = bf16_pair(M, N, K, seed=7)
+    y = gdn.linear_bf16(x.cuda(), w.cuda())
+    torch.cuda.synchronize()
+    rows = torch.tensor([0, 1, 127, 128, 2049, 4095])
+    check(x[rows], w, y[rows.cuda()])
+
+
+def test_linear_k_zero_and_empty():
+    x = torch.zeros(3, 0, dtype=torch.bfloat16, device="cuda")
+    w = torch.zeros(5, 0, dtype=torch.bfloat16, device="cuda")
+    y = torch.full((3, 5), 7.0, device="cuda")
+    gdn.linear_bf16(x, w, y)
+    torch.cuda.synchronize()
+    assert torch.count_nonzero(y) == 0
+    e = gdn.linear_bf16(torch.zeros(0, 16, dtype=torch.bfloat16, device="cuda"),
+                        torch.zeros(4, 16, dtype=torch.bfloat16, device="cuda"))
+    assert e.shape == (0, 4)
