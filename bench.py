@@ -432,6 +432,34 @@ def bench_layer_pair(steps: int, warmup: int, device):
     return dict(seconds=secs, launches=steps, bytes=layer_pair_bytes(B), tokens=2 * B)
 
 
+def bench_forward_batch(steps: int, warmup: int, device):
+    """The layer over B = 4 x T = 4096 positions with dense bf16 projections
+    (D = 2048), graph-replayed; the ring and state advance from call to call."""
+    import torch
+    from linear_attention_recurrence_04_b200 import gdn, inputs
+    w = inputs.FORWARD_WORKLOAD
+    B, T = w.sizes["B"], w.sizes["T"]
+    d = w.draw()
+    bf = ("hidden", "w_qkv", "w_z", "w_ba", "w_out")
+    t = {k: (torch.from_numpy(v).to(device).to(torch.bfloat16) if k in bf
+             else torch.from_numpy(v).to(device)) for k, v in d.items()}
+    D = t["hidden"].shape[2]
+    out = torch.empty((B, T, D), dtype=torch.float32, device=device)
+    ws = torch.empty(gdn.forward_batch_workspace_size(B, T), dtype=torch.uint8, device=device)
+    stream = torch.cuda.current_stream(device)
+
+    def launch(i):
+        gdn.forward_batch(t["hidden"], t["w_qkv"], t["w_z"], t["w_ba"], t["w_out"],
+                          t["conv_ring"], t["conv_w"], t["A_log"], t["dt_bias"], t["norm_w"],
+                          t["state"], out, ws, Hk=16)
+
+    secs = time_launches(launch, 1, steps, warmup, stream, graph=True)
+    C, HD, Hv = 8192, 4096, 32
+    gemm_flops = 2 * B * T * D * (C + HD + 2 * Hv) + 2 * B * T * HD * D
+    return dict(seconds=secs, launches=steps, tokens=B * T, gemm_flops=gemm_flops,
+                rec_flops=prefill_flops(B, T))
+
+
 def cpu_oracle_baseline(name: str, budget_s: float, max_units: Optional[int] = None):
     """Time the fp64 oracle as it stands on a bounded sample of the workload:
     whole decode steps over the first `units` (layer, sequence, head) units,
@@ -633,6 +661,15 @@ def run_ours(args) -> int:
             "layer_tokens_per_s": pr["tokens"] * pr["launches"] / pr["seconds"],
             "gb_s": gbs, "roofline": {"bound": "hbm", "peak": peaks["hbm_gbs"], "unit": "GB/s",
                                       "frac": gbs / peaks["hbm_gbs"]},
+        }
+        torch.cuda.empty_cache()
+        fb = bench_forward_batch(5, 2, device)
+        per = fb["seconds"] / fb["launches"]
+        extras["forward_batch_b4_t4096"] = {
+            "ms_per_launch": per * 1e3,
+            "tokens_per_s": fb["tokens"] / per,
+            "projection_tflops": fb["gemm_flops"] / per / 1e12,
+            "note": "D=2048 bf16 projections on tcgen05 + conv + sequential recurrence + tail",
         }
         line["workloads"] = extras
 

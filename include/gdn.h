@@ -39,6 +39,7 @@
 #ifndef GDN_H
 #define GDN_H
 
+#include <stddef.h>
 #include <stdint.h>
 
 #ifdef __cplusplus
@@ -191,6 +192,44 @@ gdn_status gdn_layer_pair(const float *mixed_qkv, const float *z, const float *a
  */
 gdn_status gdn_linear_bf16(const void *x, const void *w, float *y, int64_t M, int64_t N,
                            int64_t K, uint32_t *status, void *stream);
+
+/*
+ * gdn_forward_batch -- the recurrent layer over T consecutive positions of
+ * each of B sequences, with dense bf16 projections ("Module linear_core",
+ * entry "gdn_forward_batch": the qkv/z/a/b and out_proj projections are
+ * matrix-matrix products over the batch while the recurrence runs
+ * sequentially over positions; stages as in gdn_layer_decode). Per position,
+ * in order:
+ *   mixed = W_qkv h,  z = W_z h,  (b | a) = W_ba h        (tensor-core GEMMs)
+ *   stages 1-6 of gdn_layer_decode (conv with ring, SiLU, split, L2 norms,
+ *   beta/gate, recurrence, gated RMSNorm), the recurrence carried across
+ *   positions as in gdn_prefill;
+ *   y rounded to bf16, out = W_out y                        (tensor-core GEMM)
+ *
+ *   hidden    [B][T][D] bf16        D a multiple of 8
+ *   w_qkv     [C][D] bf16, C = 2*Hk*dk + Hv*dv
+ *   w_z       [Hv*dv][D] bf16
+ *   w_ba      [2*Hv][D] bf16        rows 0..Hv-1 give b, rows Hv..2Hv-1 give a
+ *   w_out     [D][Hv*dv] bf16
+ *   conv_ring [B][K-1][C] in/out    after position T-1
+ *   conv_w [C][K]; A_log, dt_bias [Hv]; norm_w [dv]   (fp32)
+ *   state     [B][Hv][dv][dk] in/out
+ *   out       [B][T][D] fp32
+ *   workspace device scratch of at least gdn_forward_batch_workspace_size()
+ *             bytes, 256-byte aligned, owned by the caller; its contents on
+ *             entry do not matter and are undefined afterwards
+ *   status    optional zero-initialised device word for timeout bits (see
+ *             gdn_linear_bf16)
+ */
+size_t gdn_forward_batch_workspace_size(int64_t B, int64_t T, int64_t Hk, int64_t Hv,
+                                        int64_t dk, int64_t dv);
+gdn_status gdn_forward_batch(const void *hidden, const void *w_qkv, const void *w_z,
+                             const void *w_ba, const void *w_out, float *conv_ring,
+                             const float *conv_w, const float *A_log, const float *dt_bias,
+                             const float *norm_w, float l2_eps, float norm_eps, float *state,
+                             float *out, void *workspace, size_t workspace_bytes, int64_t B,
+                             int64_t T, int64_t D, int64_t Hk, int64_t Hv, int64_t dk,
+                             int64_t dv, int64_t K, uint32_t *status, void *stream);
 
 #ifdef __cplusplus
 }

@@ -342,4 +342,64 @@ gdn_status gdn_linear_bf16(const void* x, const void* w, float* y, int64_t M, in
     return launched(launch_linear_bf16(a, static_cast<cudaStream_t>(stream)), "gdn_linear_bf16");
 }
 
+size_t gdn_forward_batch_workspace_size(int64_t B, int64_t T, int64_t Hk, int64_t Hv,
+                                        int64_t dk, int64_t dv) {
+    if (B < 0 || T < 0 || Hk <= 0 || Hv <= 0 || Hv % Hk != 0 || dk != kDk || dv != kDv ||
+        Hv > (1 << 20) || B > (int64_t)65535 * 128 || T > (int64_t)65535 * 128 ||
+        B * T > (int64_t)65535 * 128)
+        return 0;
+    return forward_batch_layout(B, T, static_cast<int>(Hk), static_cast<int>(Hv)).total;
+}
+
+gdn_status gdn_forward_batch(const void* hidden, const void* w_qkv, const void* w_z,
+                             const void* w_ba, const void* w_out, float* conv_ring,
+                             const float* conv_w, const float* A_log, const float* dt_bias,
+                             const float* norm_w, float l2_eps, float norm_eps, float* state,
+                             float* out, void* workspace, size_t workspace_bytes, int64_t B,
+                             int64_t T, int64_t D, int64_t Hk, int64_t Hv, int64_t dk,
+                             int64_t dv, int64_t K, uint32_t* status, void* stream) {
+    const char* fn = "gdn_forward_batch";
+    if (B < 0 || T < 0 || D < 0) return fail(GDN_ERR_SHAPE, "%s: negative B, T or D", fn);
+    gdn_status st = check_geometry(Hk, Hv, dk, dv);
+    if (st != GDN_OK) return st;
+    if (K != kConvK) return fail(GDN_ERR_UNSUPPORTED, "%s: K=%lld: only a conv kernel of 4 is implemented",
+                                 fn, (long long)K);
+    if (D == 0 || D % 8 != 0)
+        return fail(GDN_ERR_UNSUPPORTED, "%s: D=%lld must be a positive multiple of 8", fn, (long long)D);
+    if (B > (int64_t)65535 * 128 || T > (int64_t)65535 * 128 || B * T > (int64_t)65535 * 128 ||
+        D > (1 << 24))
+        return fail(GDN_ERR_OVERFLOW, "%s: B*T=%lld or D too large", fn, (long long)(B * T));
+    const int64_t BT = B * T;
+    const int64_t C = 2 * Hk * dk + Hv * dv;
+    const int64_t HD = Hv * dv;
+    if (BT == 0) { g_last_error[0] = '\0'; return GDN_OK; }
+    const size_t need = forward_batch_layout(B, T, static_cast<int>(Hk), static_cast<int>(Hv)).total;
+    if (!hidden || !w_qkv || !w_z || !w_ba || !w_out || !conv_ring || !conv_w || !A_log ||
+        !dt_bias || !norm_w || !state || !out || !workspace)
+        return fail(GDN_ERR_NULL, "%s: a tensor pointer is NULL", fn);
+    if (workspace_bytes < need)
+        return fail(GDN_ERR_SHAPE, "%s: workspace of %zu bytes, %zu needed", fn, workspace_bytes, need);
+    if (!aligned(hidden, 16) || !aligned(w_qkv, 16) || !aligned(w_z, 16) || !aligned(w_ba, 16) ||
+        !aligned(w_out, 16) || !aligned(conv_ring, 16) || !aligned(conv_w, 16) ||
+        !aligned(state, 16) || !aligned(out, 16) || !aligned(workspace, 256) ||
+        !aligned(A_log, 4) || !aligned(dt_bias, 4) || !aligned(norm_w, 4) ||
+        (status && !aligned(status, 4)))
+        return fail(GDN_ERR_ALIGN, "%s: alignment rule violated (workspace needs 256 bytes)", fn);
+    const Span ins[] = {{state, B * Hv * dv * dk * 4, "state"},
+                        {conv_ring, B * (K - 1) * C * 4, "conv_ring"},
+                        {workspace, static_cast<int64_t>(need), "workspace"},
+                        {status, status ? 4 : 0, "status"},
+                        {hidden, BT * D * 2, "hidden"}, {w_qkv, C * D * 2, "w_qkv"},
+                        {w_z, HD * D * 2, "w_z"}, {w_ba, 2 * Hv * D * 2, "w_ba"},
+                        {w_out, D * HD * 2, "w_out"}, {conv_w, C * K * 4, "conv_w"},
+                        {A_log, Hv * 4, "A_log"}, {dt_bias, Hv * 4, "dt_bias"},
+                        {norm_w, dv * 4, "norm_w"}};
+    st = check_spans(ins, 13, 4, Span{out, BT * D * 4, "out"});
+    if (st != GDN_OK) return st;
+    ForwardBatchArgs a{hidden, w_qkv, w_z, w_ba, w_out, conv_ring, conv_w, A_log, dt_bias, norm_w,
+                       l2_eps, norm_eps, state, out, workspace, B, T, D, static_cast<int>(Hk),
+                       static_cast<int>(Hv), status};
+    return launched(launch_forward_batch(a, static_cast<cudaStream_t>(stream)), fn);
+}
+
 }  // extern "C"

@@ -1,0 +1,208 @@
+// gdn_forward_batch.cu -- the recurrent layer over T positions of B sequences
+// with dense projections.
+//
+// Page "Module linear_core", entry "gdn_forward_batch": the qkv/z/a/b and
+// out_proj projections are matrix-matrix products over the batch, and the
+// recurrence runs sequentially over positions, elementwise as the
+// one-position path; stages from "Red Lite dev15e -- complete recurrent
+// DeltaNet layer composition" (opening list) and "Red Lite dev15a --
+// DeltaNet projection field validation" ("Validation boundary").
+//
+// Pipeline (every stage a kernel of this library, on the caller's stream):
+//   1. mixed = hidden . W_qkv^T, z = hidden . W_z^T, ba = hidden . W_ba^T
+//      (tcgen05 GEMMs, bf16 in, fp32 out, into the workspace);
+//   2. conv_seq: per (sequence, channel) one thread walks the positions with
+//      the conv ring in registers, replacing mixed with SiLU(conv) in place
+//      and leaving the last K-1 raw inputs in the ring;
+//   3. qk_norm_gates: per position, L2-normalise each q and k head in place
+//      and form beta = sigmoid(b), gate = -exp(A_log) softplus(a + dt_bias);
+//   4. the sequential prefill recurrence, reading q, k, v straight out of the
+//      conv buffer (row stride C), writing o [B][T][Hv][dv];
+//   5. tail: per (position, value head) gated RMSNorm in double, rounded to
+//      bf16 (the output projection's input type);
+//   6. out = y . W_out^T (tcgen05 GEMM).
+#include <cuda_bf16.h>
+
+#include "gdn_common.cuh"
+#include "gdn_internal.h"
+
+namespace gdn {
+
+namespace {
+
+// 2. causal depthwise conv over positions, SiLU, in place; ring update.
+__global__ void __launch_bounds__(256)
+conv_seq_kernel(float* __restrict__ act, float* __restrict__ ring,
+                const float* __restrict__ conv_w, int64_t B, int64_t T, int64_t C) {
+    const int64_t idx = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+    if (idx >= B * C) return;
+    const int64_t b = idx / C;
+    const int64_t c = idx - b * C;
+    float* rg = ring + b * (kConvK - 1) * C + c;
+    float w0 = rg[0], w1 = rg[C], w2 = rg[2 * C];      // raw inputs, oldest first
+    const float4 w = ld_ro4(conv_w + c * kConvK);
+    float* col = act + b * T * C + c;
+    // Positions in blocks of kSeqBlock: all loads of a block are issued
+    // before any of its (sequential) conv steps, so the memory latency is
+    // paid once per block rather than once per position.
+    constexpr int kSeqBlock = 16;
+    for (int64_t t0 = 0; t0 < T; t0 += kSeqBlock) {
+        const int n = (T - t0) < kSeqBlock ? static_cast<int>(T - t0) : kSeqBlock;
+        float xs[kSeqBlock];
+#pragma unroll
+        for (int i = 0; i < kSeqBlock; ++i) xs[i] = (i < n) ? col[(t0 + i) * C] : 0.0f;
+#pragma unroll
+        for (int i = 0; i < kSeqBlock; ++i) {
+            if (i < n) {
+                const float x = xs[i];
+                const float y = fmaf(w.w, x, fmaf(w.z, w2, fmaf(w.y, w1, w.x * w0)));
+                col[(t0 + i) * C] = siluf_acc(y);
+                w0 = w1;
+                w1 = w2;
+                w2 = x;
+            }
+        }
+    }
+    rg[0] = w0;
+    rg[C] = w1;
+    rg[2 * C] = w2;
+}
+
+// 3. per position: L2-normalise the 2 Hk q/k heads (one warp each, in turn)
+//    and compute the Hv decay gates and write strengths.
+__global__ void __launch_bounds__(256)
+qk_norm_gates_kernel(float* __restrict__ act, const float* __restrict__ ba,
+                     const float* __restrict__ A_log, const float* __restrict__ dt_bias,
+                     float* __restrict__ beta, float* __restrict__ gate, int64_t C, int Hk,
+                     int Hv, float l2_eps) {
+    const int64_t bt = blockIdx.x;
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+    const int n_warps = blockDim.x >> 5;
+    float* row = act + bt * C;
+    for (int vec = warp; vec < 2 * Hk; vec += n_warps) {
+        float4* p = reinterpret_cast<float4*>(row + static_cast<int64_t>(vec) * kDk) + lane;
+        float4 x = *p;
+        float ss = fmaf(x.x, x.x, fmaf(x.y, x.y, fmaf(x.z, x.z, x.w * x.w)));
+        ss = warp_sum(ss);
+        const float inv = 1.0f / fmaxf(sqrtf(ss), l2_eps);
+        x.x *= inv; x.y *= inv; x.z *= inv; x.w *= inv;
+        *p = x;
+    }
+    for (int h = threadIdx.x; h < Hv; h += blockDim.x) {
+        const float bv = ba[bt * 2 * Hv + h];
+        const float av = ba[bt * 2 * Hv + Hv + h];
+        beta[bt * Hv + h] = sigmoidf_acc(bv);
+        gate[bt * Hv + h] = -expf(A_log[h]) * softplusf_acc(av + dt_bias[h]);
+    }
+}
+
+__device__ __forceinline__ double warp_sum_d(double x) {
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) x += __shfl_xor_sync(kFull, x, off);
+    return x;
+}
+
+// 5. gated RMSNorm per (position, value head) in double; y in bf16.
+__global__ void __launch_bounds__(256)
+tail_bf16_kernel(const float* __restrict__ o, const float* __restrict__ z,
+                 const float* __restrict__ norm_w, __nv_bfloat16* __restrict__ y, int64_t rows,
+                 float norm_eps) {
+    const int64_t r = static_cast<int64_t>(blockIdx.x) * (blockDim.x >> 5) + (threadIdx.x >> 5);
+    if (r >= rows) return;                                   // r = (b t) * Hv + h
+    const int lane = threadIdx.x & 31;
+    const float4 ov = ld_ro4(o + r * kDv + lane * 4);
+    const float4 zv = ld_ro4(z + r * kDv + lane * 4);
+    const float4 wv = ld_ro4(norm_w + lane * 4);
+    const double o4[4] = {ov.x, ov.y, ov.z, ov.w};
+    const double z4[4] = {zv.x, zv.y, zv.z, zv.w};
+    const double w4[4] = {wv.x, wv.y, wv.z, wv.w};
+    double ss = 0.0;
+#pragma unroll
+    for (int i = 0; i < 4; ++i) ss = fma(o4[i], o4[i], ss);
+    ss = warp_sum_d(ss);
+    const double inv_rms = 1.0 / sqrt(ss / static_cast<double>(kDv) + static_cast<double>(norm_eps));
+    __nv_bfloat16 out4[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        const double silu = z4[i] / (1.0 + exp(-z4[i]));
+        out4[i] = __double2bfloat16(o4[i] * inv_rms * w4[i] * silu);
+    }
+    *reinterpret_cast<uint2*>(y + r * kDv + lane * 4) = *reinterpret_cast<const uint2*>(out4);
+}
+
+size_t align256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
+
+}  // namespace
+
+ForwardBatchLayout forward_batch_layout(int64_t B, int64_t T, int Hk, int Hv) {
+    const int64_t BT = B * T;
+    const int64_t C = static_cast<int64_t>(2 * Hk) * kDk + static_cast<int64_t>(Hv) * kDv;
+    const int64_t HD = static_cast<int64_t>(Hv) * kDv;
+    ForwardBatchLayout L;
+    size_t off = 0;
+    L.act = off;   off = align256(off + BT * C * 4);
+    L.z = off;     off = align256(off + BT * HD * 4);
+    L.ba = off;    off = align256(off + BT * 2 * Hv * 4);
+    L.beta = off;  off = align256(off + BT * Hv * 4);
+    L.gate = off;  off = align256(off + BT * Hv * 4);
+    L.o = off;     off = align256(off + BT * HD * 4);
+    L.y = off;     off = align256(off + BT * HD * 2);
+    L.total = off;
+    return L;
+}
+
+cudaError_t launch_forward_batch(const ForwardBatchArgs& a, cudaStream_t stream) {
+    const int64_t BT = a.B * a.T;
+    if (BT == 0) return cudaSuccess;
+    const int64_t C = static_cast<int64_t>(2 * a.Hk) * kDk + static_cast<int64_t>(a.Hv) * kDv;
+    const int64_t HD = static_cast<int64_t>(a.Hv) * kDv;
+    const ForwardBatchLayout L = forward_batch_layout(a.B, a.T, a.Hk, a.Hv);
+    char* ws = static_cast<char*>(a.workspace);
+    float* act = reinterpret_cast<float*>(ws + L.act);
+    float* z = reinterpret_cast<float*>(ws + L.z);
+    float* ba = reinterpret_cast<float*>(ws + L.ba);
+    float* beta = reinterpret_cast<float*>(ws + L.beta);
+    float* gate = reinterpret_cast<float*>(ws + L.gate);
+    float* o = reinterpret_cast<float*>(ws + L.o);
+    __nv_bfloat16* y = reinterpret_cast<__nv_bfloat16*>(ws + L.y);
+
+    // 1. input projections
+    cudaError_t err;
+    if ((err = launch_linear_bf16(LinearArgs{a.hidden, a.w_qkv, act, BT, C, a.D, a.status}, stream)))
+        return err;
+    if ((err = launch_linear_bf16(LinearArgs{a.hidden, a.w_z, z, BT, HD, a.D, a.status}, stream)))
+        return err;
+    if ((err = launch_linear_bf16(LinearArgs{a.hidden, a.w_ba, ba, BT, 2 * a.Hv, a.D, a.status},
+                                  stream)))
+        return err;
+    // 2. conv over positions with the ring, SiLU
+    {
+        const int64_t n = a.B * C;
+        conv_seq_kernel<<<static_cast<unsigned>((n + 255) / 256), 256, 0, stream>>>(
+            act, a.conv_ring, a.conv_w, a.B, a.T, C);
+        if ((err = cudaGetLastError())) return err;
+    }
+    // 3. q/k L2 norm, beta and gate
+    qk_norm_gates_kernel<<<static_cast<unsigned>(BT), 256, 0, stream>>>(
+        act, ba, a.A_log, a.dt_bias, beta, gate, C, a.Hk, a.Hv, a.l2_eps);
+    if ((err = cudaGetLastError())) return err;
+    // 4. the sequential recurrence, reading q, k, v from the conv rows
+    {
+        PrefillArgs p{a.state, act, act + static_cast<int64_t>(a.Hk) * kDk,
+                      act + static_cast<int64_t>(2 * a.Hk) * kDk, beta, gate, o, a.B, a.T, a.Hk,
+                      a.Hv, C, C, a.Hv};
+        if ((err = launch_prefill(p, stream))) return err;
+    }
+    // 5. gated RMSNorm tail -> bf16
+    {
+        const int64_t rows = BT * a.Hv;
+        tail_bf16_kernel<<<static_cast<unsigned>((rows + 7) / 8), 256, 0, stream>>>(
+            o, z, a.norm_w, y, rows, a.norm_eps);
+        if ((err = cudaGetLastError())) return err;
+    }
+    // 6. output projection
+    return launch_linear_bf16(LinearArgs{y, a.w_out, a.out, BT, a.D, HD, a.status}, stream);
+}
+
+}  // namespace gdn

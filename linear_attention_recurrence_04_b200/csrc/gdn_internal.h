@@ -31,6 +31,12 @@ struct PrefillArgs {
     int64_t T;
     int Hk;
     int Hv;
+    // Elements between consecutive positions of q and k, of v, and of
+    // beta/gate; 0 selects the contiguous layouts [B][T][Hk][dk],
+    // [B][T][Hv][dv] and [B][T][Hv].
+    int64_t qk_stride = 0;
+    int64_t v_stride = 0;
+    int64_t bg_stride = 0;
 };
 
 struct LayerArgs {
@@ -64,12 +70,43 @@ struct LinearArgs {
     uint32_t* status;  // optional device word for timeout bits
 };
 
+struct ForwardBatchArgs {
+    const void* hidden;    // [B][T][D] bf16
+    const void* w_qkv;     // [C][D] bf16
+    const void* w_z;       // [Hv*dv][D] bf16
+    const void* w_ba;      // [2*Hv][D] bf16: rows 0..Hv-1 give b, Hv..2Hv-1 give a
+    const void* w_out;     // [D][Hv*dv] bf16
+    float* conv_ring;
+    const float* conv_w;
+    const float* A_log;
+    const float* dt_bias;
+    const float* norm_w;
+    float l2_eps;
+    float norm_eps;
+    float* state;
+    float* out;            // [B][T][D]
+    void* workspace;
+    int64_t B;
+    int64_t T;
+    int64_t D;
+    int Hk;
+    int Hv;
+    uint32_t* status;
+};
+
+// Byte offsets of the forward-batch intermediates inside the workspace.
+struct ForwardBatchLayout {
+    size_t act, z, ba, beta, gate, o, y, total;
+};
+ForwardBatchLayout forward_batch_layout(int64_t B, int64_t T, int Hk, int Hv);
+
 // Each launcher enqueues its kernel on `stream` and returns the launch status.
 cudaError_t launch_step(const StepArgs& a, cudaStream_t stream);
 cudaError_t launch_prefill(const PrefillArgs& a, cudaStream_t stream);
 cudaError_t launch_layer_decode(const LayerArgs& a, cudaStream_t stream);
 cudaError_t launch_layer_pair(const LayerArgs& a, cudaStream_t stream);
 cudaError_t launch_linear_bf16(const LinearArgs& a, cudaStream_t stream);
+cudaError_t launch_forward_batch(const ForwardBatchArgs& a, cudaStream_t stream);
 
 // Value-heads-per-key-head ratios the fused layer kernel is compiled for.
 bool layer_decode_supports(int G);

@@ -130,7 +130,8 @@ __global__ void __launch_bounds__(32 * kMaxWarps, 1)
 prefill_kernel(float* __restrict__ state, const float* __restrict__ q,
                const float* __restrict__ k, const float* __restrict__ v,
                const float* __restrict__ beta, const float* __restrict__ gate,
-               float* __restrict__ out, int64_t T, int Hk, int Hv, int units_lo, int n_big) {
+               float* __restrict__ out, int64_t T, int Hk, int Hv, int units_lo, int n_big,
+               int64_t qk_stride, int64_t v_stride, int64_t bg_stride) {
     extern __shared__ __align__(16) unsigned char smem_raw[];
     Stage<NH>* stages = reinterpret_cast<Stage<NH>*>(smem_raw);
     __shared__ Group grp_of[kMaxGroups];
@@ -180,7 +181,7 @@ prefill_kernel(float* __restrict__ state, const float* __restrict__ q,
                 const int64_t t = t0 + tp;
                 float* dst = &st.kq[gi][tp][which][chunk * 4];
                 if (t < T) {
-                    cp_async16(dst, (which ? q : k) + ((G.b * T + t) * Hk + G.g) * kDk + chunk * 4);
+                    cp_async16(dst, (which ? q : k) + (G.b * T + t) * qk_stride + G.g * kDk + chunk * 4);
                 } else {
                     *reinterpret_cast<float4*>(dst) = make_float4(0.f, 0.f, 0.f, 0.f);
                 }
@@ -194,7 +195,7 @@ prefill_kernel(float* __restrict__ state, const float* __restrict__ q,
                 float* dst = &st.v[gi][tp][n][chunk * 4];
                 if (t < T) {
                     const int h = G.g + (G.grp * NH + n) * Hk;
-                    cp_async16(dst, v + ((G.b * T + t) * Hv + h) * kDv + G.row_lo + chunk * 4);
+                    cp_async16(dst, v + (G.b * T + t) * v_stride + h * kDv + G.row_lo + chunk * 4);
                 } else {
                     *reinterpret_cast<float4*>(dst) = make_float4(0.f, 0.f, 0.f, 0.f);
                 }
@@ -207,7 +208,7 @@ prefill_kernel(float* __restrict__ state, const float* __restrict__ q,
                 float* dst = &st.bg[gi][tp][n][which];
                 if (t < T) {
                     const int h = G.g + (G.grp * NH + n) * Hk;
-                    cp_async4(dst, (which ? gate : beta) + (G.b * T + t) * Hv + h);
+                    cp_async4(dst, (which ? gate : beta) + (G.b * T + t) * bg_stride + h);
                 } else {
                     *dst = 0.0f;
                 }
@@ -412,8 +413,12 @@ cudaError_t launch_nh(const PrefillArgs& a, cudaStream_t stream) {
                                            cudaFuncAttributeMaxDynamicSharedMemorySize,
                                            static_cast<int>(smem));
     if (err != cudaSuccess) return err;
+    const int64_t qk_stride = a.qk_stride ? a.qk_stride : static_cast<int64_t>(a.Hk) * kDk;
+    const int64_t v_stride = a.v_stride ? a.v_stride : static_cast<int64_t>(a.Hv) * kDv;
+    const int64_t bg_stride = a.bg_stride ? a.bg_stride : a.Hv;
     prefill_kernel<NH><<<static_cast<unsigned>(grid), 32 * warps, smem, stream>>>(
-        a.state, a.q, a.k, a.v, a.beta, a.gate, a.out, a.T, a.Hk, a.Hv, units_lo, n_big);
+        a.state, a.q, a.k, a.v, a.beta, a.gate, a.out, a.T, a.Hk, a.Hv, units_lo, n_big,
+        qk_stride, v_stride, bg_stride);
     return cudaGetLastError();
 }
 

@@ -29,7 +29,8 @@ STATUS = {
 
 # Every symbol that include/gdn.h declares.
 EXPORTS = ("gdn_status_string", "gdn_last_error", "gdn_step", "gdn_prefill", "gdn_layer_decode",
-           "gdn_layer_pair", "gdn_linear_bf16")
+           "gdn_layer_pair", "gdn_linear_bf16", "gdn_forward_batch_workspace_size",
+           "gdn_forward_batch")
 
 
 class GdnError(RuntimeError):
@@ -73,6 +74,11 @@ def load_library(path: Optional[str] = None) -> ctypes.CDLL:
     lib.gdn_layer_pair.argtypes = [_VP] * 9 + [_F32, _F32] + [_VP] * 4 + [_I64] * 6 + [_VP]
     lib.gdn_linear_bf16.restype = ctypes.c_int
     lib.gdn_linear_bf16.argtypes = [_VP, _VP, _VP, _I64, _I64, _I64, _VP, _VP]
+    lib.gdn_forward_batch_workspace_size.restype = ctypes.c_size_t
+    lib.gdn_forward_batch_workspace_size.argtypes = [_I64] * 6
+    lib.gdn_forward_batch.restype = ctypes.c_int
+    lib.gdn_forward_batch.argtypes = ([_VP] * 10 + [_F32, _F32] + [_VP, _VP, _VP, ctypes.c_size_t]
+                                      + [_I64] * 8 + [_VP, _VP])
     if path is None:
         _lib = lib
     return lib
@@ -262,3 +268,49 @@ def linear_bf16(x, w, y=None, *, status=None, stream=None):
                _stream(device, stream))
     _raise_on("gdn_linear_bf16", st)
     return y
+
+
+def forward_batch_workspace_size(B: int, T: int, Hk: int = 16, Hv: int = 32) -> int:
+    return int(load_library().gdn_forward_batch_workspace_size(B, T, Hk, Hv, 128, 128))
+
+
+def forward_batch(hidden, w_qkv, w_z, w_ba, w_out, conv_ring, conv_w, A_log, dt_bias, norm_w,
+                  state, out=None, workspace=None, *, Hk: int, l2_eps: float = 1e-6,
+                  norm_eps: float = 1e-6, status=None, stream=None):
+    """The layer over T positions with dense bf16 projections.
+
+    hidden [B, T, D] bf16; w_qkv [C, D], w_z [Hv*128, D], w_ba [2*Hv, D],
+    w_out [D, Hv*128] bf16; conv_ring [B, K-1, C] and state [B, Hv, 128, 128]
+    are updated in place. `workspace` (uint8 CUDA tensor) is allocated here
+    if not given. Returns out [B, T, D] fp32."""
+    B, T, D = hidden.shape
+    Hv = state.shape[1]
+    C, K = conv_w.shape
+    for n, t in (("hidden", hidden), ("w_qkv", w_qkv), ("w_z", w_z), ("w_ba", w_ba),
+                 ("w_out", w_out)):
+        if t.dtype is not torch.bfloat16 or not t.is_cuda or not t.is_contiguous():
+            raise TypeError(f"{n} must be a contiguous bfloat16 CUDA tensor")
+    if out is None:
+        out = torch.empty((B, T, D), dtype=torch.float32, device=hidden.device)
+    names = ("conv_ring", "conv_w", "A_log", "dt_bias", "norm_w", "state", "out")
+    tensors = (conv_ring, conv_w, A_log, dt_bias, norm_w, state, out)
+    device = _dev(tensors, names)
+    need = forward_batch_workspace_size(B, T, Hk, Hv)
+    if workspace is None:
+        workspace = torch.empty(max(need, 1), dtype=torch.uint8, device=device)
+    if workspace.dtype is not torch.uint8 or workspace.device != device:
+        raise TypeError("workspace must be a uint8 tensor on the same device")
+    expect = dict(w_qkv=(C, D), w_z=(Hv * 128, D), w_ba=(2 * Hv, D), w_out=(D, Hv * 128),
+                  conv_ring=(B, K - 1, C), out=(B, T, D))
+    for n, t in (("w_qkv", w_qkv), ("w_z", w_z), ("w_ba", w_ba), ("w_out", w_out),
+                 ("conv_ring", conv_ring), ("out", out)):
+        if tuple(t.shape) != expect[n]:
+            raise ValueError(f"{n} has shape {tuple(t.shape)}, expected {expect[n]}")
+    sp = status.data_ptr() if status is not None else 0
+    st = _call(device, load_library().gdn_forward_batch, _ptr(hidden), _ptr(w_qkv), _ptr(w_z),
+               _ptr(w_ba), _ptr(w_out), _ptr(conv_ring), _ptr(conv_w), _ptr(A_log),
+               _ptr(dt_bias), _ptr(norm_w), float(l2_eps), float(norm_eps), _ptr(state),
+               _ptr(out), workspace.data_ptr(), workspace.numel(), B, T, D, Hk, Hv, 128, 128, K,
+               sp, _stream(device, stream))
+    _raise_on("gdn_forward_batch", st)
+    return out

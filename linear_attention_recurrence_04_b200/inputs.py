@@ -105,6 +105,43 @@ def layer_inputs(B: int, *, Hk: int = HK, Hv: int = HV, dk: int = DK, dv: int = 
     )
 
 
+def to_bf16_values(x: np.ndarray) -> np.ndarray:
+    """float32 array of the nearest bfloat16 values (round half to even), a
+    dtype conversion so the GPU (as bf16) and the oracle (as fp64) read the
+    same numbers."""
+    u = np.ascontiguousarray(x, dtype=np.float32).view(np.uint32).astype(np.uint64)
+    u = (u + 0x7FFF + ((u >> 16) & 1)) & 0xFFFF0000
+    return u.astype(np.uint32).view(np.float32)
+
+
+def forward_inputs(B: int, T: int, *, D: int = 2048, Hk: int = HK, Hv: int = HV, dk: int = DK,
+                   dv: int = DV, K: int = KCONV, seed: int = 1007,
+                   state_std: float = 0.0) -> Dict[str, np.ndarray]:
+    """A layer over T positions with dense projections: hidden ~ N(0, 1),
+    weights ~ N(0, 1/fan_in) (all bf16-representable float32), conv ring
+    ~ N(0, 1), conv weight ~ N(0, 0.25^2), A_log ~ U(-1, 1),
+    dt_bias ~ N(0, 0.1^2), norm weight ~ 1 + N(0, 0.1^2), state zero (or
+    N(0, state_std^2))."""
+    r = np.random.default_rng(seed)
+    C = 2 * Hk * dk + Hv * dv
+    HD = Hv * dv
+    bf = lambda a: to_bf16_values(a.astype(np.float32))
+    return dict(
+        hidden=bf(r.normal(size=(B, T, D))),
+        w_qkv=bf(r.normal(0.0, D ** -0.5, (C, D))),
+        w_z=bf(r.normal(0.0, D ** -0.5, (HD, D))),
+        w_ba=bf(r.normal(0.0, D ** -0.5, (2 * Hv, D))),
+        w_out=bf(r.normal(0.0, HD ** -0.5, (D, HD))),
+        conv_ring=_f32(r.normal(size=(B, K - 1, C))),
+        conv_w=_f32(r.normal(0.0, 0.25, (C, K))),
+        A_log=_f32(r.uniform(-1.0, 1.0, Hv)),
+        dt_bias=_f32(r.normal(0.0, 0.1, Hv)),
+        norm_w=_f32(1.0 + r.normal(0.0, 0.1, dv)),
+        state=(_f32(r.normal(0.0, state_std, (B, Hv, dv, dk))) if state_std > 0
+               else np.zeros((B, Hv, dv, dk), np.float32)),
+    )
+
+
 @dataclass(frozen=True)
 class Workload:
     """One named synthetic workload and how to draw it."""
@@ -120,6 +157,8 @@ class Workload:
             return prefill_inputs(self.sizes["B"], self.sizes["T"], seed=self.seed)
         if self.kind == "layer":
             return layer_inputs(self.sizes["B"], seed=self.seed)
+        if self.kind == "forward":
+            return forward_inputs(self.sizes["B"], self.sizes["T"], seed=self.seed)
         raise ValueError(self.kind)
 
 
@@ -132,3 +171,6 @@ WORKLOADS = {
     "prefill_b4_t4096": Workload("prefill_b4_t4096", "prefill", dict(B=4, T=4096), seed=1003),
     "layer_decode_b256": Workload("layer_decode_b256", "layer", dict(B=256), seed=1004),
 }
+
+# The batched layer forward with dense projections (D = 2048 hidden).
+FORWARD_WORKLOAD = Workload("forward_batch_b4_t4096", "forward", dict(B=4, T=4096), seed=1007)

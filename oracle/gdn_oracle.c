@@ -29,7 +29,9 @@
  *       identical to the one-position path; entry "gdn_pair": a fused
  *       two-position forward for speculative verification, where lane 1
  *       commits into the state and lane 2 is tentative in scratch, the conv
- *       ring and the recurrent state moving together.
+ *       ring and the recurrent state moving together; entry
+ *       "gdn_forward_batch" also names the layer's projections (qkv, z, a/b,
+ *       out_proj) as matrix products over a batch of positions.
  *
  * Readings where the pages are silent (each is listed with its reason in the
  * design notes): gate is a log-decay applied as exp(gate); the output scale
@@ -472,4 +474,102 @@ int oracle_gdn_layer_pair(const double *mixed_qkv, const double *z,
             return rc;
     }
     return 0;
+}
+
+/* Nearest bf16 value (round half to even) of x, for normal-range x: keep 8
+ * significant bits of the binary significand. */
+static double round_to_bf16(double x)
+{
+    if (x == 0.0 || !isfinite(x))
+        return x;
+    int e;
+    const double m = frexp(x, &e);          /* x = m 2^e, 0.5 <= |m| < 1 */
+    return ldexp(nearbyint(ldexp(m, 8)), e - 8);
+}
+
+/*
+ * The layer for T positions of B sequences with dense projections, [L] and
+ * [B] entry "gdn_forward_batch". Position by position, in order:
+ *   mixed = W_qkv h_t,  z = W_z h_t,  (b_in | a_in) = W_ba h_t   (matvecs)
+ *   prestate -> recurrence of every value head -> gated RMSNorm tail (as in
+ *   oracle_gdn_layer_decode), then out_t = W_out y_t.
+ * The tail output y is rounded to bf16 before the output projection when
+ * round_y is non-zero (the precision the projection consumes).
+ *   hidden [B][T][D]; W_qkv [C][D], C = 2*Hk*dk + Hv*dv; W_z [Hv*dv][D];
+ *   W_ba [2*Hv][D] (rows 0..Hv-1 give b, rows Hv..2Hv-1 give a);
+ *   W_out [D][Hv*dv]; ring [B][K-1][C] in/out; state [B][Hv][dv][dk] in/out;
+ *   out [B][T][D].
+ */
+int oracle_gdn_forward_batch(const double *hidden, const double *W_qkv,
+                             const double *W_z, const double *W_ba,
+                             const double *W_out, double *ring,
+                             const double *conv_w, const double *A_log,
+                             const double *dt_bias, const double *norm_w,
+                             double l2_eps, double norm_eps, double *state,
+                             double *out, int64_t B, int64_t T, int64_t D,
+                             int64_t Hk, int64_t Hv, int64_t dk, int64_t dv,
+                             int64_t K, int round_y, const int64_t *seqs,
+                             int64_t n_seqs)
+{
+    if (B < 0 || T < 0 || D <= 0 || K < 1 || !dims_ok(Hk, Hv, dk, dv))
+        return -1;
+    const int64_t C = 2 * Hk * dk + Hv * dv;
+    const int64_t HD = Hv * dv;
+    const int64_t count = seqs ? n_seqs : B;
+    for (int64_t n = 0; n < count; ++n) {
+        const int64_t b = seqs ? seqs[n] : n;
+        if (b < 0 || b >= B)
+            return -1;
+    }
+    double *mixed = (double *)malloc((size_t)C * sizeof(double));
+    double *z = (double *)malloc((size_t)HD * sizeof(double));
+    double *ab = (double *)malloc((size_t)(2 * Hv) * sizeof(double));
+    double *y = (double *)malloc((size_t)HD * sizeof(double));
+    int rc = (mixed && z && ab && y) ? 0 : -2;
+    for (int64_t n = 0; rc == 0 && n < count; ++n) {
+        const int64_t b = seqs ? seqs[n] : n;
+        for (int64_t t = 0; rc == 0 && t < T; ++t) {
+            const double *h = hidden + (b * T + t) * D;
+            for (int64_t r = 0; r < C; ++r) {
+                double acc = 0.0;
+                for (int64_t i = 0; i < D; ++i)
+                    acc += W_qkv[r * D + i] * h[i];
+                mixed[r] = acc;
+            }
+            for (int64_t r = 0; r < HD; ++r) {
+                double acc = 0.0;
+                for (int64_t i = 0; i < D; ++i)
+                    acc += W_z[r * D + i] * h[i];
+                z[r] = acc;
+            }
+            for (int64_t r = 0; r < 2 * Hv; ++r) {
+                double acc = 0.0;
+                for (int64_t i = 0; i < D; ++i)
+                    acc += W_ba[r * D + i] * h[i];
+                ab[r] = acc;
+            }
+            /* b_in = ab[0..Hv), a_in = ab[Hv..2Hv) */
+            rc = oracle_gdn_layer_decode(mixed, z, ab + Hv, ab, ring + b * (K - 1) * C,
+                                         conv_w, A_log, dt_bias, norm_w, l2_eps,
+                                         norm_eps, state + b * Hv * dv * dk, y, 1, Hk,
+                                         Hv, dk, dv, K, NULL, 0);
+            if (rc)
+                break;
+            if (round_y)
+                for (int64_t r = 0; r < HD; ++r)
+                    y[r] = round_to_bf16(y[r]);
+            double *o = out + (b * T + t) * D;
+            for (int64_t r = 0; r < D; ++r) {
+                double acc = 0.0;
+                for (int64_t i = 0; i < HD; ++i)
+                    acc += W_out[r * HD + i] * y[i];
+                o[r] = acc;
+            }
+        }
+    }
+    free(mixed);
+    free(z);
+    free(ab);
+    free(y);
+    return rc;
 }

@@ -78,6 +78,9 @@ class Oracle:
         lib.oracle_gdn_layer_pair.argtypes = [_PD, _PD, _PD, _PD, _PD, _PD, _PD, _PD, _PD,
                                               _DBL, _DBL, _PD, _PD, _PD, _PD,
                                               _I64, _I64, _I64, _I64, _I64, _I64, _PI, _I64]
+        lib.oracle_gdn_forward_batch.restype = ctypes.c_int
+        lib.oracle_gdn_forward_batch.argtypes = [_PD] * 10 + [_DBL, _DBL, _PD, _PD] + [_I64] * 8 + \
+            [ctypes.c_int, _PI, _I64]
         self.lib = lib
 
     # -- recurrence ---------------------------------------------------------
@@ -207,6 +210,35 @@ class Oracle:
                                             _ptr(out), B, Hk, Hv, dk, dv, K, sp, ns)
         _check(rc, "oracle_gdn_layer_pair")
         return out, rg, st, srg, sst
+
+
+    def forward_batch(self, hidden, W_qkv, W_z, W_ba, W_out, ring, conv_w, A_log, dt_bias,
+                      norm_w, state, *, Hk, l2_eps=1e-6, norm_eps=1e-6, round_y=True,
+                      seqs=None):
+        """T positions of the layer with dense projections.
+
+        Shapes: hidden [B,T,D]; W_qkv [C,D]; W_z [Hv*dv,D]; W_ba [2*Hv,D];
+        W_out [D,Hv*dv]; ring [B,K-1,C]; conv_w [C,K]; A_log, dt_bias [Hv];
+        norm_w [dv]; state [B,Hv,dv,dk]. Returns (out [B,T,D], ring, state).
+        """
+        st = _f64(state)
+        B, Hv, dv, dk = st.shape
+        hh = _f64(hidden)
+        T, D = hh.shape[1], hh.shape[2]
+        wq, wz, wb, wo = _f64(W_qkv), _f64(W_z), _f64(W_ba), _f64(W_out)
+        rg, w, al, dt, nw = _f64(ring), _f64(conv_w), _f64(A_log), _f64(dt_bias), _f64(norm_w)
+        C, K = w.shape
+        assert hh.shape == (B, T, D) and wq.shape == (C, D) and wz.shape == (Hv * dv, D)
+        assert wb.shape == (2 * Hv, D) and wo.shape == (D, Hv * dv) and rg.shape == (B, K - 1, C)
+        out = np.zeros((B, T, D))
+        sp, ns, _keep = _units(seqs)
+        rc = self.lib.oracle_gdn_forward_batch(_ptr(hh), _ptr(wq), _ptr(wz), _ptr(wb), _ptr(wo),
+                                               _ptr(rg), _ptr(w), _ptr(al), _ptr(dt), _ptr(nw),
+                                               float(l2_eps), float(norm_eps),
+                                               _ptr(st), _ptr(out), B, T, D, Hk, Hv, dk, dv, K,
+                                               int(bool(round_y)), sp, ns)
+        _check(rc, "oracle_gdn_forward_batch")
+        return out, rg, st
 
 
 _DEFAULT: Optional[Oracle] = None

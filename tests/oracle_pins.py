@@ -395,6 +395,44 @@ def pin_layer_pair_library(o):
     _close(sst, s2, 1e-12, "pair scratch state")
 
 
+
+
+
+def _bf16_exact(x):
+    """Round an fp64 array to bf16 values (kept in fp64) with torch."""
+    return torch.from_numpy(x).to(torch.bfloat16).to(torch.float64).numpy()
+
+
+def pin_forward_batch_library(o):
+    """T positions of the layer with dense projections ("Module linear_core",
+    gdn_forward_batch): projections as matmuls, each position through the
+    torch-built layer, the tail output rounded to bf16 by torch, then the
+    output projection; on non-square heads with Hv = 2 Hk."""
+    c = _layer_case(27, B=2)
+    r = _rng(28)
+    Hk, Hv, dk, dv = c["Hk"], c["Hv"], c["dk"], c["dv"]
+    C = c["x"].shape[1]
+    B, T, D = 2, 5, 24
+    hidden = _bf16_exact(r.normal(size=(B, T, D)))
+    Wq = _bf16_exact(r.normal(0, D ** -0.5, (C, D)))
+    Wz = _bf16_exact(r.normal(0, D ** -0.5, (Hv * dv, D)))
+    Wba = _bf16_exact(r.normal(0, D ** -0.5, (2 * Hv, D)))
+    Wo = _bf16_exact(r.normal(0, (Hv * dv) ** -0.5, (D, Hv * dv)))
+    out, ring, st = o.forward_batch(hidden, Wq, Wz, Wba, Wo, c["ring"], c["w"], c["A_log"],
+                                    c["dt_bias"], c["norm_w"], c["state"], Hk=Hk)
+    ring_t, st_t = c["ring"].copy(), c["state"].copy()
+    for t in range(T):
+        h = hidden[:, t]
+        mixed = h @ Wq.T
+        z = h @ Wz.T
+        ba = h @ Wba.T
+        y, ring_t, st_t = _torch_layer(c, mixed, z, ba[:, Hv:], ba[:, :Hv], ring_t, st_t)
+        want = _bf16_exact(y) @ Wo.T
+        _close(out[:, t], want, 1e-12, f"forward_batch out t{t}")
+    assert np.array_equal(ring, ring_t), "forward_batch ring"
+    _close(st, st_t, 1e-12, "forward_batch state")
+
+
 ALL_PINS = [
     pin_golden_step_cases,
     pin_delta_rule_closed_form,
@@ -409,4 +447,5 @@ ALL_PINS = [
     pin_tail_library,
     pin_layer_library,
     pin_layer_pair_library,
+    pin_forward_batch_library,
 ]

@@ -151,3 +151,21 @@ def test_linear_argument_checks(lib):
     assert f(y=fake(1) + 16) == ALIAS
     assert f(M=1 << 30) == OVERFLOW
     assert lib.gdn_linear_bf16(0, 0, 0, 0, 7, 16, 0, None) == OK
+
+
+def test_forward_batch_argument_checks(lib):
+    ws = lib.gdn_forward_batch_workspace_size(2, 3, 16, 32, 128, 128)
+    assert ws > 2 * 3 * (8192 + 4096 + 4096) * 4
+    assert lib.gdn_forward_batch_workspace_size(2, 3, 16, 32, 64, 128) == 0
+
+    def f(D=64, ws_bytes=ws, workspace=fake(20), K=4, out=fake(13)):
+        return lib.gdn_forward_batch(fake(1), fake(2), fake(3), fake(4), fake(5), fake(6),
+                                     fake(7), fake(8), fake(9), fake(10), ctypes.c_float(1e-6),
+                                     ctypes.c_float(1e-6), fake(12), out, workspace, ws_bytes,
+                                     2, 3, D, 16, 32, 128, 128, K, 0, None)
+    assert f(D=60) == UNSUP
+    assert f(K=2) == UNSUP
+    assert f(ws_bytes=ws - 1) == SHAPE
+    assert f(workspace=0) == NULL
+    assert f(workspace=fake(20) + 16) == ALIGN
+    assert f(out=fake(20) + 256) == ALIAS

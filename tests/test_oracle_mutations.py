@@ -67,6 +67,12 @@ MUTATIONS = [
      "rc = oracle_gdn_layer_decode(mixed_qkv + (b * 2 + 0) * C,"),
     ("pair scratch starts from lane-2 ring slot", "memcpy(srg, rg, (size_t)((K - 1) * C) * sizeof(double));",
      "memcpy(srg, rg, (size_t)((K - 1) * C) * sizeof(double)); srg[0] = srg[1];"),
+    # batched forward with projections
+    ("forward a/b swapped", "rc = oracle_gdn_layer_decode(mixed, z, ab + Hv, ab,",
+     "rc = oracle_gdn_layer_decode(mixed, z, ab, ab + Hv,"),
+    ("forward y not rounded", "y[r] = round_to_bf16(y[r]);", "y[r] = y[r];"),
+    ("bf16 keeps 9 bits", "return ldexp(nearbyint(ldexp(m, 8)), e - 8);",
+     "return ldexp(nearbyint(ldexp(m, 9)), e - 9);"),
 ]
 
 
