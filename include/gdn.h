@@ -231,6 +231,33 @@ gdn_status gdn_forward_batch(const void *hidden, const void *w_qkv, const void *
                              int64_t T, int64_t D, int64_t Hk, int64_t Hv, int64_t dk,
                              int64_t dv, int64_t K, uint32_t *status, void *stream);
 
+/*
+ * gdn_forward_batch_noalloc -- gdn_forward_batch without a caller-provided
+ * workspace, for callers that cannot allocate device memory (a plugin whose
+ * host program owns every device allocation and offers no hook, code held to
+ * a memory budget fixed before it runs, or a latency-critical path where an
+ * allocation is not allowed). There is no counterpart on the source pages:
+ * it is a deployment variant of the same layer. Arguments and results are
+ * those of gdn_forward_batch without `workspace` and `workspace_bytes`.
+ *
+ * The workspace is a 16 MiB array built into the library (held on every GPU
+ * that loads the library until the process exits). B*T positions whose
+ * gdn_forward_batch_workspace_size() exceeds 16 MiB (about 226 positions at
+ * Hk = 16, Hv = 32, dk = dv = 128) are rejected with GDN_ERR_UNSUPPORTED and
+ * a message; nothing is launched. The first call on a device looks up the
+ * array's device address; make that call before any stream capture. Every
+ * call uses the same array, so calls whose GPU work overlaps (other streams,
+ * other host threads on the same device) race and must be ordered by the
+ * caller. The library performs no allocation of any kind for this call.
+ */
+gdn_status gdn_forward_batch_noalloc(const void *hidden, const void *w_qkv, const void *w_z,
+                                     const void *w_ba, const void *w_out, float *conv_ring,
+                                     const float *conv_w, const float *A_log,
+                                     const float *dt_bias, const float *norm_w, float l2_eps,
+                                     float norm_eps, float *state, float *out, int64_t B,
+                                     int64_t T, int64_t D, int64_t Hk, int64_t Hv, int64_t dk,
+                                     int64_t dv, int64_t K, uint32_t *status, void *stream);
+
 #ifdef __cplusplus
 }
 #endif

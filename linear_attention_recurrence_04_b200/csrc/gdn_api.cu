@@ -88,6 +88,11 @@ gdn_status launched(cudaError_t err, const char* what) {
 
 }  // namespace
 
+int report_error(int status, const char* message) {
+    snprintf(g_last_error, sizeof(g_last_error), "%s", message);
+    return status;
+}
+
 int device_sm_count() {
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0) return 148;

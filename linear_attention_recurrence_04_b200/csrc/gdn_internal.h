@@ -111,6 +111,10 @@ cudaError_t launch_forward_batch(const ForwardBatchArgs& a, cudaStream_t stream)
 // Value-heads-per-key-head ratios the fused layer kernel is compiled for.
 bool layer_decode_supports(int G);
 
+// Records `message` as this host thread's gdn_last_error() text and returns
+// `status` (for entry points defined outside gdn_api.cu).
+int report_error(int status, const char* message);
+
 // Number of SMs of the current device, cached per device.
 int device_sm_count();
 

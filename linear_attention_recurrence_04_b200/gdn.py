@@ -30,7 +30,7 @@ STATUS = {
 # Every symbol that include/gdn.h declares.
 EXPORTS = ("gdn_status_string", "gdn_last_error", "gdn_step", "gdn_prefill", "gdn_layer_decode",
            "gdn_layer_pair", "gdn_linear_bf16", "gdn_forward_batch_workspace_size",
-           "gdn_forward_batch")
+           "gdn_forward_batch", "gdn_forward_batch_noalloc")
 
 
 class GdnError(RuntimeError):
@@ -79,6 +79,9 @@ def load_library(path: Optional[str] = None) -> ctypes.CDLL:
     lib.gdn_forward_batch.restype = ctypes.c_int
     lib.gdn_forward_batch.argtypes = ([_VP] * 10 + [_F32, _F32] + [_VP, _VP, _VP, ctypes.c_size_t]
                                       + [_I64] * 8 + [_VP, _VP])
+    lib.gdn_forward_batch_noalloc.restype = ctypes.c_int
+    lib.gdn_forward_batch_noalloc.argtypes = ([_VP] * 10 + [_F32, _F32] + [_VP, _VP]
+                                              + [_I64] * 8 + [_VP, _VP])
     if path is None:
         _lib = lib
     return lib
@@ -313,4 +316,32 @@ def forward_batch(hidden, w_qkv, w_z, w_ba, w_out, conv_ring, conv_w, A_log, dt_
                _ptr(out), workspace.data_ptr(), workspace.numel(), B, T, D, Hk, Hv, 128, 128, K,
                sp, _stream(device, stream))
     _raise_on("gdn_forward_batch", st)
+    return out
+
+
+def forward_batch_noalloc(hidden, w_qkv, w_z, w_ba, w_out, conv_ring, conv_w, A_log, dt_bias,
+                          norm_w, state, out, *, Hk: int, l2_eps: float = 1e-6,
+                          norm_eps: float = 1e-6, status=None, stream=None):
+    """forward_batch with the library's built-in scratch instead of a
+    workspace (see gdn_forward_batch_noalloc in include/gdn.h): for callers
+    that cannot allocate device memory. `out` must be given; nothing is
+    allocated here."""
+    B, T, D = hidden.shape
+    Hv = state.shape[1]
+    C, K = conv_w.shape
+    for n, t in (("hidden", hidden), ("w_qkv", w_qkv), ("w_z", w_z), ("w_ba", w_ba),
+                 ("w_out", w_out)):
+        if t.dtype is not torch.bfloat16 or not t.is_cuda or not t.is_contiguous():
+            raise TypeError(f"{n} must be a contiguous bfloat16 CUDA tensor")
+    names = ("conv_ring", "conv_w", "A_log", "dt_bias", "norm_w", "state", "out")
+    tensors = (conv_ring, conv_w, A_log, dt_bias, norm_w, state, out)
+    device = _dev(tensors, names)
+    if tuple(out.shape) != (B, T, D):
+        raise ValueError(f"out has shape {tuple(out.shape)}, expected {(B, T, D)}")
+    sp = status.data_ptr() if status is not None else 0
+    st = _call(device, load_library().gdn_forward_batch_noalloc, _ptr(hidden), _ptr(w_qkv),
+               _ptr(w_z), _ptr(w_ba), _ptr(w_out), _ptr(conv_ring), _ptr(conv_w), _ptr(A_log),
+               _ptr(dt_bias), _ptr(norm_w), float(l2_eps), float(norm_eps), _ptr(state),
+               _ptr(out), B, T, D, Hk, Hv, 128, 128, K, sp, _stream(device, stream))
+    _raise_on("gdn_forward_batch_noalloc", st)
     return out
