@@ -32,6 +32,11 @@
  *       ring and the recurrent state moving together; entry
  *       "gdn_forward_batch" also names the layer's projections (qkv, z, a/b,
  *       out_proj) as matrix products over a batch of positions.
+ *   [SC] "Module linear_core", struct "ShortConvWeights" and entries
+ *       "short_conv_forward", "short_conv_forward_batch",
+ *       "short_conv_pair": the LFM2 short-convolution mixer, whose only
+ *       state is the causal conv ring of the last kernel-1 gated inputs per
+ *       channel.
  *
  * Readings where the pages are silent (each is listed with its reason in the
  * design notes): gate is a log-decay applied as exp(gate); the output scale
@@ -571,5 +576,139 @@ int oracle_gdn_forward_batch(const double *hidden, const double *W_qkv,
     free(z);
     free(ab);
     free(y);
+    return rc;
+}
+
+/* ------------------------------------------------------------------------ */
+/* LFM2 short-convolution mixer. [SC] "Module linear_core", struct          */
+/* "ShortConvWeights" and entries "short_conv_forward",                     */
+/* "short_conv_forward_batch", "short_conv_pair": no recurrent state, only  */
+/* the causal conv ring holding the last K-1 gated inputs of each channel;   */
+/* in_proj and out_proj are matrix products, the conv walks the positions    */
+/* in order. Readings (the pages give no formula): in_proj maps D to 3D     */
+/* rows split into the input gate bg = rows [0, D), the output gate         */
+/* cg = rows [D, 2D) and the value xv = rows [2D, 3D); the gated input is   */
+/* u = bg * xv; conv = sum_t conv_w[d][t] * window[t] over the window       */
+/* (ring[0..K-2], u) oldest first, no bias; y = cg * conv; out = W_out y.   */
+/* ------------------------------------------------------------------------ */
+
+/* One position of one sequence: h [D] -> o [D]; ring [K-1][D] advances. */
+static int short_conv_token(const double *h, const double *W_in,
+                            const double *W_out, double *ring,
+                            const double *conv_w, double *o, int64_t D,
+                            int64_t K, int round_y, double *proj, double *y,
+                            double *window)
+{
+    for (int64_t r = 0; r < 3 * D; ++r) {
+        double acc = 0.0;
+        for (int64_t i = 0; i < D; ++i)
+            acc += W_in[r * D + i] * h[i];
+        proj[r] = acc;
+    }
+    const double *bg = proj;
+    const double *cg = proj + D;
+    const double *xv = proj + 2 * D;
+    for (int64_t d = 0; d < D; ++d) {
+        for (int64_t t = 0; t < K - 1; ++t)
+            window[t] = ring[t * D + d];
+        window[K - 1] = bg[d] * xv[d];
+        double conv = 0.0;
+        for (int64_t t = 0; t < K; ++t)
+            conv += conv_w[d * K + t] * window[t];
+        for (int64_t t = 0; t < K - 1; ++t)
+            ring[t * D + d] = window[t + 1];
+        y[d] = cg[d] * conv;
+        if (round_y)
+            y[d] = round_to_bf16(y[d]);
+    }
+    for (int64_t r = 0; r < D; ++r) {
+        double acc = 0.0;
+        for (int64_t i = 0; i < D; ++i)
+            acc += W_out[r * D + i] * y[i];
+        o[r] = acc;
+    }
+    return 0;
+}
+
+/*
+ * T positions of B sequences, [SC] "short_conv_forward_batch" (T = 1 is
+ * "short_conv_forward"). hidden [B][T][D]; W_in [3D][D]; W_out [D][D];
+ * ring [B][K-1][D] in/out; conv_w [D][K]; out [B][T][D]. round_y rounds y
+ * to the nearest bf16 value (ties to even) before the output projection.
+ * seqs (optional) restricts the work to the listed sequences.
+ */
+int oracle_short_conv_forward_batch(const double *hidden, const double *W_in,
+                                    const double *W_out, double *ring,
+                                    const double *conv_w, double *out,
+                                    int64_t B, int64_t T, int64_t D, int64_t K,
+                                    int round_y, const int64_t *seqs,
+                                    int64_t n_seqs)
+{
+    if (B < 0 || T < 0 || D <= 0 || K < 1)
+        return -1;
+    const int64_t count = seqs ? n_seqs : B;
+    for (int64_t n = 0; n < count; ++n) {
+        const int64_t b = seqs ? seqs[n] : n;
+        if (b < 0 || b >= B)
+            return -1;
+    }
+    double *proj = (double *)malloc((size_t)(3 * D) * sizeof(double));
+    double *y = (double *)malloc((size_t)D * sizeof(double));
+    double *window = (double *)malloc((size_t)K * sizeof(double));
+    int rc = (proj && y && window) ? 0 : -2;
+    for (int64_t n = 0; rc == 0 && n < count; ++n) {
+        const int64_t b = seqs ? seqs[n] : n;
+        for (int64_t t = 0; rc == 0 && t < T; ++t)
+            rc = short_conv_token(hidden + (b * T + t) * D, W_in, W_out,
+                                  ring + b * (K - 1) * D, conv_w,
+                                  out + (b * T + t) * D, D, K, round_y, proj, y,
+                                  window);
+    }
+    free(proj);
+    free(y);
+    free(window);
+    return rc;
+}
+
+/*
+ * Two positions per sequence, [SC] "short_conv_pair": position 0 commits
+ * into ring; position 1 continues from a copy of the committed ring and
+ * leaves its ring in scratch_ring [B][K-1][D]. hidden [B][2][D],
+ * out [B][2][D].
+ */
+int oracle_short_conv_pair(const double *hidden, const double *W_in,
+                           const double *W_out, double *ring,
+                           double *scratch_ring, const double *conv_w,
+                           double *out, int64_t B, int64_t D, int64_t K,
+                           int round_y, const int64_t *seqs, int64_t n_seqs)
+{
+    if (B < 0 || D <= 0 || K < 1)
+        return -1;
+    const int64_t count = seqs ? n_seqs : B;
+    for (int64_t n = 0; n < count; ++n) {
+        const int64_t b = seqs ? seqs[n] : n;
+        if (b < 0 || b >= B)
+            return -1;
+    }
+    double *proj = (double *)malloc((size_t)(3 * D) * sizeof(double));
+    double *y = (double *)malloc((size_t)D * sizeof(double));
+    double *window = (double *)malloc((size_t)K * sizeof(double));
+    int rc = (proj && y && window) ? 0 : -2;
+    for (int64_t n = 0; rc == 0 && n < count; ++n) {
+        const int64_t b = seqs ? seqs[n] : n;
+        double *rg = ring + b * (K - 1) * D;
+        double *srg = scratch_ring + b * (K - 1) * D;
+        rc = short_conv_token(hidden + (b * 2) * D, W_in, W_out, rg, conv_w,
+                              out + (b * 2) * D, D, K, round_y, proj, y, window);
+        if (rc)
+            break;
+        memcpy(srg, rg, (size_t)((K - 1) * D) * sizeof(double));
+        rc = short_conv_token(hidden + (b * 2 + 1) * D, W_in, W_out, srg, conv_w,
+                              out + (b * 2 + 1) * D, D, K, round_y, proj, y,
+                              window);
+    }
+    free(proj);
+    free(y);
+    free(window);
     return rc;
 }

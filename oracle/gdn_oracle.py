@@ -81,6 +81,11 @@ class Oracle:
         lib.oracle_gdn_forward_batch.restype = ctypes.c_int
         lib.oracle_gdn_forward_batch.argtypes = [_PD] * 10 + [_DBL, _DBL, _PD, _PD] + [_I64] * 8 + \
             [ctypes.c_int, _PI, _I64]
+        lib.oracle_short_conv_forward_batch.restype = ctypes.c_int
+        lib.oracle_short_conv_forward_batch.argtypes = [_PD] * 6 + [_I64] * 4 + \
+            [ctypes.c_int, _PI, _I64]
+        lib.oracle_short_conv_pair.restype = ctypes.c_int
+        lib.oracle_short_conv_pair.argtypes = [_PD] * 7 + [_I64] * 3 + [ctypes.c_int, _PI, _I64]
         self.lib = lib
 
     # -- recurrence ---------------------------------------------------------
@@ -239,6 +244,52 @@ class Oracle:
                                                int(bool(round_y)), sp, ns)
         _check(rc, "oracle_gdn_forward_batch")
         return out, rg, st
+
+
+    # -- LFM2 short-convolution mixer ----------------------------------------
+    def short_conv_forward_batch(self, hidden, W_in, W_out, ring, conv_w, *, round_y=True,
+                                 seqs=None):
+        """T positions of the short-conv mixer.
+
+        Shapes: hidden [B,T,D]; W_in [3D,D] (rows: input gate | output gate |
+        value); W_out [D,D]; ring [B,K-1,D] (gated inputs, oldest first);
+        conv_w [D,K]. Returns (out [B,T,D], ring).
+        """
+        hh = _f64(hidden)
+        B, T, D = hh.shape
+        wi, wo, rg, w = _f64(W_in), _f64(W_out), _f64(ring), _f64(conv_w)
+        K = w.shape[1]
+        assert wi.shape == (3 * D, D) and wo.shape == (D, D) and w.shape == (D, K)
+        assert rg.shape == (B, K - 1, D)
+        out = np.zeros((B, T, D))
+        sp, ns, _keep = _units(seqs)
+        rc = self.lib.oracle_short_conv_forward_batch(_ptr(hh), _ptr(wi), _ptr(wo), _ptr(rg),
+                                                      _ptr(w), _ptr(out), B, T, D, K,
+                                                      int(bool(round_y)), sp, ns)
+        _check(rc, "oracle_short_conv_forward_batch")
+        return out, rg
+
+    def short_conv_pair(self, hidden, W_in, W_out, ring, conv_w, *, round_y=True, seqs=None):
+        """Two positions per sequence: position 0 commits, position 1 is tentative.
+
+        Shapes: hidden [B,2,D]; the rest as short_conv_forward_batch.
+        Returns (out [B,2,D], ring after position 0, scratch_ring after
+        position 1).
+        """
+        hh = _f64(hidden)
+        B, two, D = hh.shape
+        assert two == 2
+        wi, wo, rg, w = _f64(W_in), _f64(W_out), _f64(ring), _f64(conv_w)
+        K = w.shape[1]
+        assert wi.shape == (3 * D, D) and wo.shape == (D, D) and rg.shape == (B, K - 1, D)
+        out = np.zeros((B, 2, D))
+        srg = np.zeros_like(rg)
+        sp, ns, _keep = _units(seqs)
+        rc = self.lib.oracle_short_conv_pair(_ptr(hh), _ptr(wi), _ptr(wo), _ptr(rg), _ptr(srg),
+                                             _ptr(w), _ptr(out), B, D, K, int(bool(round_y)),
+                                             sp, ns)
+        _check(rc, "oracle_short_conv_pair")
+        return out, rg, srg
 
 
 _DEFAULT: Optional[Oracle] = None

@@ -433,6 +433,83 @@ def pin_forward_batch_library(o):
     _close(st, st_t, 1e-12, "forward_batch state")
 
 
+def _lfm2_mixer(W_in, W_out, conv_w):
+    """The transformers library's LFM2 short-conv mixer in float64, holding
+    the given weights (no biases, the library's default)."""
+    from transformers.models.lfm2.configuration_lfm2 import Lfm2Config
+    from transformers.models.lfm2.modeling_lfm2 import Lfm2ShortConv
+    D, K = conv_w.shape
+    m = Lfm2ShortConv(Lfm2Config(hidden_size=D, conv_L_cache=K, conv_bias=False), 0).double()
+    with torch.no_grad():
+        m.in_proj.weight.copy_(torch.from_numpy(W_in))
+        m.out_proj.weight.copy_(torch.from_numpy(W_out))
+        m.conv.weight.copy_(torch.from_numpy(conv_w).reshape(D, 1, K))
+    return m
+
+
+def _lfm2_run(W_in, W_out, conv_w, hidden):
+    """(out, y) of the library mixer over whole sequences from an empty
+    history; y (the gated conv output) is read by running the mixer again
+    with an identity output projection."""
+    D = conv_w.shape[0]
+    with torch.no_grad():
+        h = torch.from_numpy(hidden)
+        out = _lfm2_mixer(W_in, W_out, conv_w).slow_forward(h).numpy()
+        y = _lfm2_mixer(W_in, np.eye(D), conv_w).slow_forward(h).numpy()
+    return out, y
+
+
+def _short_conv_case(seed, B, T, D, K):
+    r = _rng(seed)
+    return dict(hidden=r.normal(size=(B, T, D)), W_in=r.normal(0, D ** -0.5, (3 * D, D)),
+                W_out=r.normal(0, D ** -0.5, (D, D)), conv_w=r.normal(0, 0.5, (D, K)))
+
+
+def pin_short_conv_library(o):
+    """LFM2 short-conv mixer ("Module linear_core", short_conv_forward_batch):
+    from an empty ring, the oracle over T1 positions and then, resuming from
+    its ring, over T2 more equals the transformers library's LFM2 mixer run
+    over all T1 + T2 positions; the ring then holds the last K-1 gated inputs
+    (input gate times value, computed here with a matmul); with y rounded to
+    bf16 (by torch) the output is W_out y."""
+    for K in (3, 4, 2):
+        B, T1, T2, D = 2, 4, 3, 12
+        c = _short_conv_case(30 + K, B, T1 + T2, D, K)
+        want, y = _lfm2_run(c["W_in"], c["W_out"], c["conv_w"], c["hidden"])
+        ring0 = np.zeros((B, K - 1, D))
+        args = (c["W_in"], c["W_out"])
+        out1, ring1 = o.short_conv_forward_batch(c["hidden"][:, :T1], *args, ring0, c["conv_w"],
+                                                 round_y=False)
+        out2, ring2 = o.short_conv_forward_batch(c["hidden"][:, T1:], *args, ring1, c["conv_w"],
+                                                 round_y=False)
+        _close(np.concatenate([out1, out2], axis=1), want, 1e-12, f"short_conv out K={K}")
+        proj = c["hidden"] @ c["W_in"].T
+        gated = proj[..., :D] * proj[..., 2 * D:]
+        _close(ring2, gated[:, T1 + T2 - (K - 1):], 1e-12, f"short_conv ring K={K}")
+        out_r, _ = o.short_conv_forward_batch(c["hidden"], *args, ring0, c["conv_w"])
+        _close(out_r, _bf16_exact(y) @ c["W_out"].T, 1e-12, f"short_conv bf16 y K={K}")
+
+
+def pin_short_conv_pair_library(o):
+    """Speculative two-position verify of the short-conv mixer ("Module
+    linear_core", short_conv_pair): after P positions, position P commits its
+    ring and position P + 1 continues into scratch; outputs and both rings
+    against the library mixer over P + 2 positions and the gated inputs."""
+    B, P, D, K = 3, 5, 10, 3
+    c = _short_conv_case(34, B, P + 2, D, K)
+    want, _ = _lfm2_run(c["W_in"], c["W_out"], c["conv_w"], c["hidden"])
+    args = (c["W_in"], c["W_out"])
+    _, ring = o.short_conv_forward_batch(c["hidden"][:, :P], *args, np.zeros((B, K - 1, D)),
+                                         c["conv_w"], round_y=False)
+    out, ring_c, ring_s = o.short_conv_pair(c["hidden"][:, P:], *args, ring, c["conv_w"],
+                                            round_y=False)
+    _close(out, want[:, P:], 1e-12, "short_conv_pair out")
+    proj = c["hidden"] @ c["W_in"].T
+    gated = proj[..., :D] * proj[..., 2 * D:]
+    _close(ring_c, gated[:, P + 1 - (K - 1):P + 1], 1e-12, "short_conv_pair committed ring")
+    _close(ring_s, gated[:, P + 2 - (K - 1):P + 2], 1e-12, "short_conv_pair scratch ring")
+
+
 ALL_PINS = [
     pin_golden_step_cases,
     pin_delta_rule_closed_form,
@@ -448,4 +525,6 @@ ALL_PINS = [
     pin_layer_library,
     pin_layer_pair_library,
     pin_forward_batch_library,
+    pin_short_conv_library,
+    pin_short_conv_pair_library,
 ]

@@ -73,6 +73,17 @@ MUTATIONS = [
     ("forward y not rounded", "y[r] = round_to_bf16(y[r]);", "y[r] = y[r];"),
     ("bf16 keeps 9 bits", "return ldexp(nearbyint(ldexp(m, 8)), e - 8);",
      "return ldexp(nearbyint(ldexp(m, 9)), e - 9);"),
+    # LFM2 short-conv mixer
+    ("short conv gates swapped", "const double *bg = proj;", "const double *bg = proj + D;"),
+    ("short conv input gate dropped", "window[K - 1] = bg[d] * xv[d];", "window[K - 1] = xv[d];"),
+    ("short conv output gate dropped", "y[d] = cg[d] * conv;", "y[d] = conv;"),
+    ("short conv taps reversed", "conv += conv_w[d * K + t] * window[t];",
+     "conv += conv_w[d * K + (K - 1 - t)] * window[t];"),
+    ("short conv ring not shifted", "ring[t * D + d] = window[t + 1];",
+     "ring[t * D + d] = window[t];"),
+    ("short conv y not rounded", "y[d] = round_to_bf16(y[d]);", "y[d] = y[d];"),
+    ("short conv pair lane 2 commits", "rc = short_conv_token(hidden + (b * 2 + 1) * D, W_in, W_out, srg,",
+     "rc = short_conv_token(hidden + (b * 2 + 1) * D, W_in, W_out, rg,"),
 ]
 
 
