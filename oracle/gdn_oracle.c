@@ -32,6 +32,9 @@
  *       ring and the recurrent state moving together; entry
  *       "gdn_forward_batch" also names the layer's projections (qkv, z, a/b,
  *       out_proj) as matrix products over a batch of positions.
+ *   [K] "Module linear_core", struct "KdaWeights" and entries "kda_forward"
+ *       and "kda_forward_batch": the KDA recurrence with the same
+ *       one-position and sequential-batch contract (no equations given).
  *   [SC] "Module linear_core", struct "ShortConvWeights" and entries
  *       "short_conv_forward", "short_conv_forward_batch",
  *       "short_conv_pair": the LFM2 short-convolution mixer, whose only
@@ -711,4 +714,141 @@ int oracle_short_conv_pair(const double *hidden, const double *W_in,
     free(y);
     free(window);
     return rc;
+}
+
+/* ------------------------------------------------------------------------ */
+/* KDA core: the delta-rule recurrence with a decay per key channel.        */
+/* [K] "Module linear_core", entries "kda_forward" (one position, advances  */
+/* the state) and "kda_forward_batch" (the recurrence sequential per        */
+/* position). The pages give no equations; the reading is the published    */
+/* Kimi Delta Attention update S_t = (I - b k k^T) Diag(a_t) S_{t-1}        */
+/* + b k v^T, o_t = S_t^T q_t, with a_t = exp(g_t) per key channel and the  */
+/* scale 1/sqrt(dk) of the one-position path. In the transposed layout      */
+/* M[j][i] = S[i][j] the five steps of [S] hold with step 1 decaying column */
+/* i by exp(g[i]).                                                          */
+/* ------------------------------------------------------------------------ */
+static int kda_head_token(double *M, const double *q, const double *k,
+                          const double *v, double beta, const double *g,
+                          double *out, int64_t dk, int64_t dv)
+{
+    double *sk = (double *)malloc((size_t)dv * sizeof(double));
+    double *delta = (double *)malloc((size_t)dv * sizeof(double));
+    double *alpha = (double *)malloc((size_t)dk * sizeof(double));
+    if (!sk || !delta || !alpha) {
+        free(sk);
+        free(delta);
+        free(alpha);
+        return -2;
+    }
+
+    /* step 1: column i of M decays by exp(g[i]) */
+    for (int64_t i = 0; i < dk; ++i)
+        alpha[i] = exp(g[i]);
+    for (int64_t j = 0; j < dv; ++j)
+        for (int64_t i = 0; i < dk; ++i)
+            M[j * dk + i] *= alpha[i];
+
+    /* step 2: sk[j] = dot(M[j], k) on the decayed state */
+    for (int64_t j = 0; j < dv; ++j) {
+        double dot = 0.0;
+        for (int64_t i = 0; i < dk; ++i)
+            dot += M[j * dk + i] * k[i];
+        sk[j] = dot;
+    }
+
+    /* step 3: delta[j] = (v[j] - sk[j]) * beta */
+    for (int64_t j = 0; j < dv; ++j)
+        delta[j] = beta * (v[j] - sk[j]);
+
+    /* step 4: M[j][i] += delta[j] * k[i] */
+    for (int64_t j = 0; j < dv; ++j)
+        for (int64_t i = 0; i < dk; ++i)
+            M[j * dk + i] += k[i] * delta[j];
+
+    /* step 5: out[j] = dot(M[j], q) / sqrt(dk) on the updated state */
+    const double root_dk = sqrt((double)dk);
+    for (int64_t j = 0; j < dv; ++j) {
+        double dot = 0.0;
+        for (int64_t i = 0; i < dk; ++i)
+            dot += M[j * dk + i] * q[i];
+        out[j] = dot / root_dk;
+    }
+
+    free(sk);
+    free(delta);
+    free(alpha);
+    return 0;
+}
+
+/*
+ * KDA decode over L layers x B sequences x Hv value heads, [K]
+ * "kda_forward". Shapes as oracle_gdn_step except
+ *   g [L][B][Hv][dk]   log-decay per value head and key channel.
+ * Value head h reads q/k of key head h % Hk.
+ */
+int oracle_kda_step(double *state, const double *q, const double *k,
+                    const double *v, const double *beta, const double *g,
+                    double *out, int64_t L, int64_t B, int64_t Hk, int64_t Hv,
+                    int64_t dk, int64_t dv, const int64_t *units,
+                    int64_t n_units)
+{
+    if (L < 0 || B < 0 || !dims_ok(Hk, Hv, dk, dv))
+        return -1;
+    const int64_t total = L * B * Hv;
+    const int64_t count = units ? n_units : total;
+    for (int64_t n = 0; n < count; ++n) {
+        const int64_t u = units ? units[n] : n;
+        if (u < 0 || u >= total)
+            return -1;
+    }
+    for (int64_t n = 0; n < count; ++n) {
+        const int64_t u = units ? units[n] : n;
+        const int64_t lb = u / Hv;
+        const int64_t key = lb * Hk + (u % Hv) % Hk;
+        int rc = kda_head_token(state + u * dv * dk, q + key * dk, k + key * dk,
+                                v + u * dv, beta[u], g + u * dk, out + u * dv,
+                                dk, dv);
+        if (rc)
+            return rc;
+    }
+    return 0;
+}
+
+/*
+ * KDA over T positions in order, [K] "kda_forward_batch": position t runs the
+ * one-position update on the state left by position t-1.
+ *   state [B][Hv][dv][dk]; q, k [B][T][Hk][dk]; v [B][T][Hv][dv];
+ *   beta [B][T][Hv]; g [B][T][Hv][dk]; out [B][T][Hv][dv].
+ */
+int oracle_kda_prefill(double *state, const double *q, const double *k,
+                       const double *v, const double *beta, const double *g,
+                       double *out, int64_t B, int64_t T, int64_t Hk,
+                       int64_t Hv, int64_t dk, int64_t dv,
+                       const int64_t *units, int64_t n_units)
+{
+    if (B < 0 || T < 0 || !dims_ok(Hk, Hv, dk, dv))
+        return -1;
+    const int64_t total = B * Hv;
+    const int64_t count = units ? n_units : total;
+    for (int64_t n = 0; n < count; ++n) {
+        const int64_t u = units ? units[n] : n;
+        if (u < 0 || u >= total)
+            return -1;
+    }
+    for (int64_t n = 0; n < count; ++n) {
+        const int64_t u = units ? units[n] : n;
+        const int64_t b = u / Hv;
+        const int64_t h = u % Hv;
+        double *M = state + u * dv * dk;
+        for (int64_t t = 0; t < T; ++t) {
+            const int64_t row = (b * T + t) * Hv + h;     /* (b, t, h) */
+            const int64_t key = (b * T + t) * Hk + h % Hk;
+            int rc = kda_head_token(M, q + key * dk, k + key * dk, v + row * dv,
+                                    beta[row], g + row * dk, out + row * dv, dk,
+                                    dv);
+            if (rc)
+                return rc;
+        }
+    }
+    return 0;
 }

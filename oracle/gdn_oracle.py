@@ -81,6 +81,10 @@ class Oracle:
         lib.oracle_gdn_forward_batch.restype = ctypes.c_int
         lib.oracle_gdn_forward_batch.argtypes = [_PD] * 10 + [_DBL, _DBL, _PD, _PD] + [_I64] * 8 + \
             [ctypes.c_int, _PI, _I64]
+        for name in ("oracle_kda_step", "oracle_kda_prefill"):
+            fn = getattr(lib, name)
+            fn.restype = ctypes.c_int
+            fn.argtypes = [_PD] * 7 + [_I64] * 6 + [_PI, _I64]
         lib.oracle_short_conv_forward_batch.restype = ctypes.c_int
         lib.oracle_short_conv_forward_batch.argtypes = [_PD] * 6 + [_I64] * 4 + \
             [ctypes.c_int, _PI, _I64]
@@ -245,6 +249,46 @@ class Oracle:
         _check(rc, "oracle_gdn_forward_batch")
         return out, rg, st
 
+
+    # -- KDA core ---------------------------------------------------------------
+    def kda_step(self, state, q, k, v, beta, g, units=None):
+        """One KDA token per (layer, sequence, value head) unit.
+
+        Shapes: state [L,B,Hv,dv,dk]; q, k [L,B,Hk,dk]; v [L,B,Hv,dv];
+        beta [L,B,Hv]; g [L,B,Hv,dk] (log-decay per key channel).
+        Returns (new_state, out [L,B,Hv,dv]).
+        """
+        st = _f64(state)
+        L, B, Hv, dv, dk = st.shape
+        Hk = np.shape(q)[2]
+        qq, kk, vv, bb, gg = _f64(q), _f64(k), _f64(v), _f64(beta), _f64(g)
+        assert qq.shape == (L, B, Hk, dk) and kk.shape == qq.shape
+        assert vv.shape == (L, B, Hv, dv) and bb.shape == (L, B, Hv)
+        assert gg.shape == (L, B, Hv, dk)
+        out = np.zeros((L, B, Hv, dv), dtype=np.float64)
+        up, nu, _keep = _units(units)
+        rc = self.lib.oracle_kda_step(_ptr(st), _ptr(qq), _ptr(kk), _ptr(vv), _ptr(bb),
+                                      _ptr(gg), _ptr(out), L, B, Hk, Hv, dk, dv, up, nu)
+        _check(rc, "oracle_kda_step")
+        return st, out
+
+    def kda_prefill(self, state, q, k, v, beta, g, units=None):
+        """T KDA positions in order. Shapes: state [B,Hv,dv,dk]; q, k
+        [B,T,Hk,dk]; v [B,T,Hv,dv]; beta [B,T,Hv]; g [B,T,Hv,dk].
+        Returns (final_state, out [B,T,Hv,dv])."""
+        st = _f64(state)
+        B, Hv, dv, dk = st.shape
+        T, Hk = np.shape(q)[1], np.shape(q)[2]
+        qq, kk, vv, bb, gg = _f64(q), _f64(k), _f64(v), _f64(beta), _f64(g)
+        assert qq.shape == (B, T, Hk, dk) and kk.shape == qq.shape
+        assert vv.shape == (B, T, Hv, dv) and bb.shape == (B, T, Hv)
+        assert gg.shape == (B, T, Hv, dk)
+        out = np.zeros((B, T, Hv, dv), dtype=np.float64)
+        up, nu, _keep = _units(units)
+        rc = self.lib.oracle_kda_prefill(_ptr(st), _ptr(qq), _ptr(kk), _ptr(vv), _ptr(bb),
+                                         _ptr(gg), _ptr(out), B, T, Hk, Hv, dk, dv, up, nu)
+        _check(rc, "oracle_kda_prefill")
+        return st, out
 
     # -- LFM2 short-convolution mixer ----------------------------------------
     def short_conv_forward_batch(self, hidden, W_in, W_out, ring, conv_w, *, round_y=True,

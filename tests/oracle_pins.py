@@ -510,6 +510,93 @@ def pin_short_conv_pair_library(o):
     _close(ring_s, gated[:, P + 2 - (K - 1):P + 2], 1e-12, "short_conv_pair scratch ring")
 
 
+def _kda_textbook(M, q, k, v, beta, g, dk):
+    """One KDA position on one head in the product form
+    M_new = M Diag(exp g) (I - beta k k^T) + beta v k^T, out = M_new q / sqrt(dk)."""
+    A = np.diag(np.exp(g)) @ (np.eye(dk) - beta * np.outer(k, k))
+    M_new = M @ A + beta * np.outer(v, k)
+    return M_new, M_new @ q / math.sqrt(dk)
+
+
+def pin_kda_textbook(o):
+    """KDA ("Module linear_core", kda_forward / kda_forward_batch; the
+    published delta rule with a decay per key channel): random non-square
+    heads with Hv = 2 Hk, one position and a 5-position sequence, against the
+    product form with value head h reading key head h % Hk and its own
+    per-channel decay."""
+    r = _rng(40)
+    L, B, Hk, Hv, dk, dv = 1, 2, 2, 4, 8, 6
+    M = r.normal(0, 0.3, (L, B, Hv, dv, dk))
+    q = _unit_rows(r.normal(size=(L, B, Hk, dk)))
+    k = _unit_rows(r.normal(size=(L, B, Hk, dk)))
+    v = r.normal(size=(L, B, Hv, dv))
+    beta = r.uniform(0.1, 0.9, (L, B, Hv))
+    g = r.uniform(-1.5, 0, (L, B, Hv, dk))
+    st, out = o.kda_step(M, q, k, v, beta, g)
+    for b in range(B):
+        for h in range(Hv):
+            Mn, on = _kda_textbook(M[0, b, h], q[0, b, h % Hk], k[0, b, h % Hk], v[0, b, h],
+                                   beta[0, b, h], g[0, b, h], dk)
+            _close(st[0, b, h], Mn, 1e-13, f"kda step state b{b} h{h}")
+            _close(out[0, b, h], on, 1e-13, f"kda step out b{b} h{h}")
+    T = 5
+    M0 = r.normal(0, 0.3, (B, Hv, dv, dk))
+    q = _unit_rows(r.normal(size=(B, T, Hk, dk)))
+    k = _unit_rows(r.normal(size=(B, T, Hk, dk)))
+    v = r.normal(size=(B, T, Hv, dv))
+    beta = r.uniform(0.1, 0.9, (B, T, Hv))
+    g = r.uniform(-1.5, 0, (B, T, Hv, dk))
+    st, out = o.kda_prefill(M0, q, k, v, beta, g)
+    for b in range(B):
+        for h in range(Hv):
+            Mt = M0[b, h]
+            for t in range(T):
+                Mt, ot = _kda_textbook(Mt, q[b, t, h % Hk], k[b, t, h % Hk], v[b, t, h],
+                                       beta[b, t, h], g[b, t, h], dk)
+                _close(out[b, t, h], ot, 1e-12, f"kda prefill out b{b} t{t} h{h}")
+            _close(st[b, h], Mt, 1e-12, f"kda prefill state b{b} h{h}")
+
+
+def pin_kda_channel_marker(o):
+    """k = 0 (no write) and a decay on key channel 3 only: column 3 of every
+    row shrinks by exp(-30) and every other entry is left exactly as it was;
+    the output reads the decayed state."""
+    r = _rng(41)
+    dk, dv = 8, 5
+    M = r.normal(size=(1, 1, 1, dv, dk))
+    g = np.zeros((1, 1, 1, dk))
+    g[..., 3] = -30.0
+    q = _unit_rows(r.normal(size=(1, 1, 1, dk)))
+    st, out = o.kda_step(M, q, np.zeros((1, 1, 1, dk)), r.normal(size=(1, 1, 1, dv)),
+                         np.full((1, 1, 1), 0.5), g)
+    keep = np.ones(dk, bool)
+    keep[3] = False
+    assert np.array_equal(st[..., keep], M[..., keep]), "kda marker: other channels changed"
+    _close(st[..., 3] / M[..., 3], np.full((1, 1, 1, dv), math.exp(-30.0)), 1e-15,
+           "kda marker: decayed channel")
+    _close(out, st @ q[0, 0, 0] / math.sqrt(dk), 1e-15, "kda marker: out")
+
+
+def pin_kda_closed_form(o):
+    """No decay (g = 0), beta = 1, |k| = 1: the delta rule stores v at k, so
+    M_new k = v, and with q = k the output is v / sqrt(dk); with a uniform
+    decay the update equals the scalar-gated one (gdn_step)."""
+    r = _rng(42)
+    dk, dv = 16, 12
+    M = r.normal(size=(1, 1, 1, dv, dk))
+    k = _unit_rows(r.normal(size=(1, 1, 1, dk)))
+    v = r.normal(size=(1, 1, 1, dv))
+    st, out = o.kda_step(M, k, k, v, np.ones((1, 1, 1)), np.zeros((1, 1, 1, dk)))
+    _close(st[0, 0, 0] @ k[0, 0, 0], v[0, 0, 0], 1e-12, "kda closed form M k")
+    _close(out[0, 0, 0], v[0, 0, 0] / math.sqrt(dk), 1e-12, "kda closed form out")
+    gate = np.full((1, 1, 1), -0.7)
+    q = _unit_rows(r.normal(size=(1, 1, 1, dk)))
+    st_k, out_k = o.kda_step(M, q, k, v, np.full((1, 1, 1), 0.3), np.full((1, 1, 1, dk), -0.7))
+    st_g, out_g = o.step(M, q, k, v, np.full((1, 1, 1), 0.3), gate)
+    _close(st_k, st_g, 1e-14, "kda uniform decay state")
+    _close(out_k, out_g, 1e-14, "kda uniform decay out")
+
+
 ALL_PINS = [
     pin_golden_step_cases,
     pin_delta_rule_closed_form,
@@ -525,6 +612,9 @@ ALL_PINS = [
     pin_layer_library,
     pin_layer_pair_library,
     pin_forward_batch_library,
+    pin_kda_textbook,
+    pin_kda_channel_marker,
+    pin_kda_closed_form,
     pin_short_conv_library,
     pin_short_conv_pair_library,
 ]

@@ -169,3 +169,32 @@ def test_forward_batch_argument_checks(lib):
     assert f(workspace=0) == NULL
     assert f(workspace=fake(20) + 16) == ALIGN
     assert f(out=fake(20) + 256) == ALIAS
+
+
+def test_short_conv_argument_checks(lib):
+    ws = lib.gdn_short_conv_workspace_size(2, 3, 64)
+    assert ws >= 2 * 3 * 64 * (3 * 4 + 2)
+    assert lib.gdn_short_conv_workspace_size(2, 3, 60) == 0
+    assert lib.gdn_short_conv_workspace_size(70000, 1, 64) == 0
+
+    def f(D=64, ws_bytes=ws, workspace=fake(20), K=3, out=fake(13), T=3, B=2):
+        return lib.gdn_short_conv_forward_batch(fake(1), fake(2), fake(3), fake(4), fake(5), out,
+                                                workspace, ws_bytes, B, T, D, K, 0, None)
+    assert f(D=60) == UNSUP
+    assert f(K=1) == UNSUP and f(K=5) == UNSUP
+    assert f(T=-1) == SHAPE
+    assert f(B=70000) == OVERFLOW
+    assert f(ws_bytes=ws - 1) == SHAPE
+    assert f(workspace=0) == NULL
+    assert f(workspace=fake(20) + 16) == ALIGN
+    assert f(out=fake(20) + 256) == ALIAS
+    assert f(out=fake(4)) == ALIAS                      # out over the ring
+    # one position and the two-position verify go through the same checks
+    ws1 = lib.gdn_short_conv_workspace_size(2, 1, 64)
+    assert lib.gdn_short_conv_forward(fake(1), fake(2), fake(3), fake(4), fake(5), fake(13),
+                                      fake(20), ws1 - 1, 2, 64, 3, 0, None) == SHAPE
+    ws2 = lib.gdn_short_conv_workspace_size(2, 2, 64)
+    assert lib.gdn_short_conv_pair(fake(1), fake(2), fake(3), fake(4), 0, fake(5), fake(13),
+                                   fake(20), ws2, 2, 64, 3, 0, None) == NULL
+    assert lib.gdn_short_conv_pair(fake(1), fake(2), fake(3), fake(4), fake(4), fake(5), fake(13),
+                                   fake(20), ws2, 2, 64, 3, 0, None) == ALIAS

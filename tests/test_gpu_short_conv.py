@@ -1,0 +1,189 @@
+"""The LFM2 short-conv mixer (gdn_short_conv_forward_batch / _forward / _pair)
+on the GPU against the fp64 oracle, through the C ABI.
+
+Tolerances. Both sides round y = cg * conv to bf16 before the output
+projection; where the two unrounded values straddle a rounding boundary they
+differ by one bf16 ulp on a few of the D terms of an output, which moves an
+output of RMS ~0.4 by well under 1e-3: the bound is 2e-3 absolute (the one
+the forward-batch tests use). A ring slot holds u = bg * xv, two outputs of
+the fp32 input projection: its error is bounded by |xv| e_bg + |bg| e_xv plus
+one fp32 rounding, where e_r is the projection's bound, a few fp32 units times
+sqrt(D) relative to the sum of |h_i W_ri|. Slots carried over from the input
+ring must be identical. Runs that must be elementwise identical (the same
+positions in one call or in several) are compared bit for bit."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from linear_attention_recurrence_04_b200 import gdn, inputs
+
+pytestmark = pytest.mark.gpu
+
+BF16 = ("hidden", "w_in", "w_out")
+OUT_ABS = 2e-3
+
+
+@pytest.fixture(scope="module")
+def o():
+    return oracle.load()
+
+
+def to_dev(d):
+    t = {}
+    for k, v in d.items():
+        x = torch.from_numpy(np.ascontiguousarray(v)).cuda()
+        t[k] = x.to(torch.bfloat16) if k in BF16 else x
+    return t
+
+
+def gpu_batch(t, hidden=None):
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    out = gdn.short_conv_forward_batch(t["hidden"] if hidden is None else hidden, t["w_in"],
+                                       t["w_out"], t["conv_ring"], t["conv_w"], status=status)
+    torch.cuda.synchronize()
+    assert int(status.item()) == 0
+    return out
+
+
+def check_out(gpu, ref, what):
+    gpu = np.asarray(gpu, np.float64)
+    assert np.all(np.isfinite(gpu)), f"{what}: non-finite"
+    err = np.abs(gpu - ref)
+    assert err.max() <= OUT_ABS, f"{what}: max abs {err.max():.3e} > {OUT_ABS}"
+
+
+def check_ring(gpu_ring, ring_in, hidden, w_in, ref_ring, last, what):
+    """Slot s of the ring holds the gated input of position last - (K-2) + s;
+    positions before 0 come from `ring_in` unchanged."""
+    h = hidden.astype(np.float64)
+    W = w_in.astype(np.float64)
+    D = h.shape[2]
+    K1 = ref_ring.shape[1]
+    gpu_ring = np.asarray(gpu_ring, np.float64)
+    for slot in range(K1):
+        t = last - (K1 - 1) + slot
+        if t < 0:
+            assert np.array_equal(gpu_ring[:, slot], ring_in[:, K1 + t]), f"{what}: carried slot"
+            continue
+        proj = h[:, t] @ W.T
+        mag = np.abs(h[:, t]) @ np.abs(W).T
+        e = 4e-7 * np.sqrt(D) * mag
+        bg, xv = proj[:, :D], proj[:, 2 * D:]
+        bound = np.abs(xv) * e[:, :D] + np.abs(bg) * e[:, 2 * D:] + e[:, :D] * e[:, 2 * D:] \
+            + 2.0 ** -23 * np.abs(bg * xv) + 1e-30
+        err = np.abs(gpu_ring[:, slot] - ref_ring[:, slot])
+        assert np.all(err <= bound), f"{what}: slot {slot} error {np.max(err / bound):.2f} x bound"
+
+
+@pytest.mark.parametrize("B,T,D,K", [(3, 1, 64, 3), (2, 5, 256, 2), (2, 37, 64, 4),
+                                     (3, 70, 256, 3), (1, 33, 320, 3)])
+def test_forward_batch_matches_oracle(o, B, T, D, K):
+    d = inputs.short_conv_inputs(B, T, D=D, K=K, seed=1400 + T)
+    t = to_dev(d)
+    out = gpu_batch(t)
+    ref_out, ref_ring = o.short_conv_forward_batch(d["hidden"], d["w_in"], d["w_out"],
+                                                   d["conv_ring"], d["conv_w"])
+    check_out(out.cpu().numpy(), ref_out, f"B{B} T{T} D{D} K{K} out")
+    check_ring(t["conv_ring"].cpu().numpy(), d["conv_ring"], d["hidden"], d["w_in"], ref_ring,
+               T - 1, f"B{B} T{T} D{D} K{K} ring")
+
+
+def test_chunks_and_single_positions_are_elementwise_identical():
+    """20 + 30 positions, and 50 single-position calls, give exactly the
+    outputs and ring of one 50-position call."""
+    B, T, D, K = 2, 50, 128, 3
+    d = inputs.short_conv_inputs(B, T, D=D, K=K, seed=1450)
+    whole = to_dev(d)
+    out_whole = gpu_batch(whole)
+    parts = to_dev(d)
+    o1 = gpu_batch(parts, parts["hidden"][:, :20].contiguous())
+    o2 = gpu_batch(parts, parts["hidden"][:, 20:].contiguous())
+    assert torch.equal(torch.cat([o1, o2], dim=1), out_whole), "chunked outputs"
+    assert torch.equal(parts["conv_ring"], whole["conv_ring"]), "chunked ring"
+    single = to_dev(d)
+    outs = []
+    for s in range(T):
+        outs.append(gdn.short_conv_forward(single["hidden"][:, s].contiguous(), single["w_in"],
+                                           single["w_out"], single["conv_ring"],
+                                           single["conv_w"]))
+    torch.cuda.synchronize()
+    assert torch.equal(torch.stack(outs, dim=1), out_whole), "single-position outputs"
+    assert torch.equal(single["conv_ring"], whole["conv_ring"]), "single-position ring"
+
+
+@pytest.mark.parametrize("K", [2, 3, 4])
+def test_pair_matches_oracle(o, K):
+    B, D = 5, 192
+    d = inputs.short_conv_inputs(B, 2, D=D, K=K, seed=1460 + K)
+    t = to_dev(d)
+    scratch = torch.full_like(t["conv_ring"], float("nan"))
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    out = gdn.short_conv_pair(t["hidden"], t["w_in"], t["w_out"], t["conv_ring"], scratch,
+                              t["conv_w"], status=status)
+    torch.cuda.synchronize()
+    assert int(status.item()) == 0
+    ref_out, ref_ring, ref_scratch = o.short_conv_pair(d["hidden"], d["w_in"], d["w_out"],
+                                                       d["conv_ring"], d["conv_w"])
+    check_out(out.cpu().numpy(), ref_out, f"pair K{K} out")
+    check_ring(t["conv_ring"].cpu().numpy(), d["conv_ring"], d["hidden"], d["w_in"], ref_ring, 0,
+               f"pair K{K} committed ring")
+    check_ring(scratch.cpu().numpy(), d["conv_ring"], d["hidden"], d["w_in"], ref_scratch, 1,
+               f"pair K{K} scratch ring")
+    # the pair's outputs are those of a two-position batch, bit for bit
+    t2 = to_dev(d)
+    out2 = gpu_batch(t2)
+    assert torch.equal(out, out2), "pair vs two-position batch"
+    assert torch.equal(scratch, t2["conv_ring"]), "scratch ring vs two-position batch ring"
+
+
+def test_empty_batch_is_a_no_op():
+    d = inputs.short_conv_inputs(2, 1, D=64, seed=1470)
+    t = to_dev(d)
+    ring0 = t["conv_ring"].clone()
+    out = gdn.short_conv_forward_batch(t["hidden"][:, :0].contiguous(), t["w_in"], t["w_out"],
+                                       t["conv_ring"], t["conv_w"])
+    torch.cuda.synchronize()
+    assert out.shape == (2, 0, 64)
+    assert torch.equal(t["conv_ring"], ring0)
+
+
+def test_decode_b64_full_size(o):
+    """The benchmark's decode launch (64 sequences, D = 2048, K = 3), every
+    sequence against the oracle."""
+    w = inputs.SHORT_CONV_WORKLOADS["short_conv_decode_b64"]
+    d = w.draw()
+    t = to_dev(d)
+    out = gdn.short_conv_forward(t["hidden"][:, 0].contiguous(), t["w_in"], t["w_out"],
+                                 t["conv_ring"], t["conv_w"])
+    torch.cuda.synchronize()
+    ref_out, ref_ring = o.short_conv_forward_batch(d["hidden"], d["w_in"], d["w_out"],
+                                                   d["conv_ring"], d["conv_w"])
+    check_out(out.cpu().numpy(), ref_out[:, 0], "decode_b64 out")
+    check_ring(t["conv_ring"].cpu().numpy(), d["conv_ring"], d["hidden"], d["w_in"], ref_ring, 0,
+               "decode_b64 ring")
+
+
+def test_batch_b4_t4096_full_size_sampled(o):
+    """The benchmark's 4 x 4096-position launch. Sequence 0's first 40
+    positions against the oracle from the true ring; for every sequence the
+    last 12 positions against the oracle started 12 positions early from an
+    arbitrary ring (after K-1 positions the window no longer reaches it), and
+    the final rings."""
+    w = inputs.SHORT_CONV_WORKLOADS["short_conv_batch_b4_t4096"]
+    d = w.draw()
+    t = to_dev(d)
+    out = gpu_batch(t).cpu().numpy()
+    B, T, D = d["hidden"].shape
+    K = d["conv_w"].shape[1]
+    head = {k: (v[:1, :40] if k == "hidden" else v[:1] if k == "conv_ring" else v)
+            for k, v in d.items()}
+    ref_head, _ = o.short_conv_forward_batch(head["hidden"], d["w_in"], d["w_out"],
+                                             head["conv_ring"], d["conv_w"])
+    check_out(out[:1, :40], ref_head, "batch_b4_t4096 head")
+    tail_h = d["hidden"][:, T - 12:]
+    ref_tail, ref_ring = o.short_conv_forward_batch(tail_h, d["w_in"], d["w_out"],
+                                                    np.zeros_like(d["conv_ring"]), d["conv_w"])
+    check_out(out[:, T - 12 + (K - 1):], ref_tail[:, K - 1:], "batch_b4_t4096 tail")
+    check_ring(t["conv_ring"].cpu().numpy(), None, tail_h, d["w_in"], ref_ring, 11,
+               "batch_b4_t4096 ring")

@@ -73,6 +73,19 @@ MUTATIONS = [
     ("forward y not rounded", "y[r] = round_to_bf16(y[r]);", "y[r] = y[r];"),
     ("bf16 keeps 9 bits", "return ldexp(nearbyint(ldexp(m, 8)), e - 8);",
      "return ldexp(nearbyint(ldexp(m, 9)), e - 9);"),
+    # KDA core
+    ("kda decay per row", "M[j * dk + i] *= alpha[i];", "M[j * dk + i] *= alpha[j % dk];"),
+    ("kda decay dropped", "alpha[i] = exp(g[i]);", "alpha[i] = 1.0;"),
+    ("kda decay sign", "alpha[i] = exp(g[i]);", "alpha[i] = exp(-g[i]);"),
+    ("kda sk reads q", "dot += M[j * dk + i] * k[i];", "dot += M[j * dk + i] * q[i];"),
+    ("kda delta sign", "delta[j] = beta * (v[j] - sk[j]);", "delta[j] = beta * (sk[j] - v[j]);"),
+    ("kda update writes q", "M[j * dk + i] += k[i] * delta[j];", "M[j * dk + i] += q[i] * delta[j];"),
+    ("kda output unscaled", "out[j] = dot / root_dk;", "out[j] = dot;"),
+    ("kda step decay of the key head", "beta[u], g + u * dk,", "beta[u], g + key * dk,"),
+    ("kda prefill decay of position 0", "beta[row], g + row * dk,",
+     "beta[row], g + (b * T * Hv + h) * dk,"),
+    ("kda prefill broadcast h/2", "const int64_t key = (b * T + t) * Hk + h % Hk;",
+     "const int64_t key = (b * T + t) * Hk + h / (Hv / Hk);"),
     # LFM2 short-conv mixer
     ("short conv gates swapped", "const double *bg = proj;", "const double *bg = proj + D;"),
     ("short conv input gate dropped", "window[K - 1] = bg[d] * xv[d];", "window[K - 1] = xv[d];"),
