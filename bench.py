@@ -42,6 +42,7 @@ UNIT = "GB/s"
 HEADLINE = "decode_l1_b64"
 L2_BYTES = 126 * 1024 * 1024
 FALLBACK_HBM_GBS = 6650.0
+FALLBACK_BF16_TFLOPS = 1590.0
 STATE_BYTES_PER_HEAD = 128 * 128 * 4
 
 # Algorithmic bytes of one value-head token of gdn_step: state read + write,
@@ -73,6 +74,25 @@ def layer_pair_bytes(B: int, Hk: int = 16, Hv: int = 32, d: int = 128, K: int = 
     return (B * Hv * d * d * 4 * 3 + B * (K - 1) * C * 4 * 3
             + 2 * (B * C * 4 + B * Hv * d * 4 * 2 + B * Hv * 4 * 2)
             + C * K * 4 + Hv * 4 * 2 + d * 4)
+
+
+def kda_step_bytes(L: int, B: int, Hk: int = 16, Hv: int = 32, d: int = 128) -> int:
+    """gdn_step's bytes with the scalar gate replaced by a log-decay per key
+    channel (d floats per value head)."""
+    return step_bytes(L, B, Hk, Hv, d) + L * B * Hv * (d - 1) * 4
+
+
+def short_conv_bytes(B: int, T: int, D: int = 2048, K: int = 3, pair: bool = False) -> int:
+    """One launch of the short-conv mixer: both weight matrices (bf16) once,
+    hidden in and out, the ring read and written (twice for the verify's
+    committed and scratch rings), the conv weight."""
+    rings = 3 if pair else 2
+    return (3 * D * D * 2 + D * D * 2 + B * T * D * 2 + B * T * D * 4
+            + rings * B * (K - 1) * D * 4 + D * K * 4)
+
+
+def short_conv_flops(B: int, T: int, D: int = 2048) -> int:
+    return 2 * B * T * D * 3 * D + 2 * B * T * D * D
 
 
 # --------------------------------------------------------------------------
@@ -109,9 +129,10 @@ def measured_peaks() -> Dict[str, object]:
     try:
         with open(path) as fh:
             p = json.load(fh)
-        return dict(hbm_gbs=float(p["hbm_gbs"]), source="measured")
+        return dict(hbm_gbs=float(p["hbm_gbs"]), bf16_tflops=float(p["bf16_tflops"]),
+                    source="measured")
     except (OSError, KeyError, ValueError):
-        return dict(hbm_gbs=FALLBACK_HBM_GBS, source="fallback")
+        return dict(hbm_gbs=FALLBACK_HBM_GBS, bf16_tflops=FALLBACK_BF16_TFLOPS, source="fallback")
 
 
 def kernel_source_digest(names: List[str]) -> str:
@@ -391,44 +412,140 @@ def bench_prefill(steps: int, warmup: int, device):
                 flops=prefill_flops(B, T), tokens=B * T)
 
 
-def bench_layer(steps: int, warmup: int, device):
+def _bf16_dev(d: Dict[str, np.ndarray], bf16_names, device) -> Dict[str, "torch.Tensor"]:
+    import torch
+    return {k: (torch.from_numpy(v).to(device).to(torch.bfloat16) if k in bf16_names
+                else torch.from_numpy(v).to(device)) for k, v in d.items()}
+
+
+def build_case(name: str, device):
+    """(launch(i), meta) for one named workload on seeded synthetic inputs
+    resident on `device`; `launch` issues one call of the library on the
+    current stream. Used by the benchmark legs and by --profile-case."""
     import torch
     from linear_attention_recurrence_04_b200 import gdn, inputs
-    w = inputs.WORKLOADS["layer_decode_b256"]
-    B = w.sizes["B"]
-    t = _to_dev(w.draw(), device)
-    out = torch.empty_like(t["z"])
+    if name in inputs.WORKLOADS and inputs.WORKLOADS[name].kind == "step":
+        w = inputs.WORKLOADS[name]
+        t = _to_dev(w.draw(), device)
+        out = torch.empty_like(t["v"])
+        return (lambda i: gdn.step(t["state"], t["q"], t["k"], t["v"], t["beta"], t["gate"],
+                                   out)), dict(tensors=t)
+    if name == "prefill_b4_t4096":
+        w = inputs.WORKLOADS[name]
+        t = _to_dev(w.draw(), device)
+        out = torch.empty_like(t["v"])
+        return (lambda i: gdn.prefill(t["state"], t["q"], t["k"], t["v"], t["beta"], t["gate"],
+                                      out)), dict(tensors=t, B=w.sizes["B"], T=w.sizes["T"])
     order = ("mixed_qkv", "z", "a", "b", "conv_ring", "conv_w", "A_log", "dt_bias", "norm_w",
              "state")
+    if name == "layer_decode_b256":
+        w = inputs.WORKLOADS[name]
+        t = _to_dev(w.draw(), device)
+        out = torch.empty_like(t["z"])
+        return (lambda i: gdn.layer_decode(*(t[n] for n in order), out, Hk=16)), \
+            dict(B=w.sizes["B"])
+    if name == "layer_pair_b256":
+        B = 256
+        d = inputs.layer_inputs(B, seed=1005)
+        d2 = inputs.layer_inputs(B, seed=1006)
+        for n in ("mixed_qkv", "z", "a", "b"):
+            d[n] = np.stack([d[n], d2[n]], axis=1)
+        t = _to_dev(d, device)
+        sring = torch.empty_like(t["conv_ring"])
+        sstate = torch.empty_like(t["state"])
+        out = torch.empty((B, 2, 32 * 128), dtype=torch.float32, device=device)
+        return (lambda i: gdn.layer_pair(*(t[n] for n in order), sring, sstate, out, Hk=16)), \
+            dict(B=B)
+    if name == "forward_batch_b4_t4096":
+        w = inputs.FORWARD_WORKLOAD
+        B, T = w.sizes["B"], w.sizes["T"]
+        t = _bf16_dev(w.draw(), ("hidden", "w_qkv", "w_z", "w_ba", "w_out"), device)
+        D = t["hidden"].shape[2]
+        out = torch.empty((B, T, D), dtype=torch.float32, device=device)
+        ws = torch.empty(gdn.forward_batch_workspace_size(B, T), dtype=torch.uint8,
+                         device=device)
+
+        def launch(i):
+            gdn.forward_batch(t["hidden"], t["w_qkv"], t["w_z"], t["w_ba"], t["w_out"],
+                              t["conv_ring"], t["conv_w"], t["A_log"], t["dt_bias"],
+                              t["norm_w"], t["state"], out, ws, Hk=16)
+        return launch, dict(B=B, T=T, D=D)
+    if name in inputs.KDA_WORKLOADS:
+        w = inputs.KDA_WORKLOADS[name]
+        t = _to_dev(w.draw(), device)
+        out = torch.empty_like(t["v"])
+        fn = gdn.kda_step if w.kind == "kda_step" else gdn.kda_prefill
+        return (lambda i: fn(t["state"], t["q"], t["k"], t["v"], t["beta"], t["g"], out)), \
+            dict(sizes=w.sizes, tensors=t)
+    if name in inputs.SHORT_CONV_WORKLOADS:
+        w = inputs.SHORT_CONV_WORKLOADS[name]
+        B, T, D, K = (w.sizes[k] for k in ("B", "T", "D", "K"))
+        t = _bf16_dev(w.draw(), ("hidden", "w_in", "w_out"), device)
+        meta = dict(B=B, T=T, D=D, K=K)
+        if name == "short_conv_pair_b64":
+            out = torch.empty((B, 2, D), dtype=torch.float32, device=device)
+            ws = torch.empty(gdn.short_conv_workspace_size(B, 2, D), dtype=torch.uint8,
+                             device=device)
+            sring = torch.empty_like(t["conv_ring"])
+            return (lambda i: gdn.short_conv_pair(t["hidden"], t["w_in"], t["w_out"],
+                                                  t["conv_ring"], sring, t["conv_w"], out,
+                                                  ws)), meta
+        out = torch.empty((B, T, D), dtype=torch.float32, device=device)
+        ws = torch.empty(gdn.short_conv_workspace_size(B, T, D), dtype=torch.uint8,
+                         device=device)
+        if T == 1:
+            h1, o1 = t["hidden"][:, 0], out[:, 0]
+            return (lambda i: gdn.short_conv_forward(h1, t["w_in"], t["w_out"], t["conv_ring"],
+                                                     t["conv_w"], o1, ws)), meta
+        return (lambda i: gdn.short_conv_forward_batch(t["hidden"], t["w_in"], t["w_out"],
+                                                       t["conv_ring"], t["conv_w"], out,
+                                                       ws)), meta
+    if name == "linear_bf16_m16384_n8192_k2048":
+        M, N, K = 16384, 8192, 2048
+        r = np.random.default_rng(1010)
+        x = torch.from_numpy(inputs.to_bf16_values(r.normal(size=(M, K)))).to(device)
+        wt = torch.from_numpy(inputs.to_bf16_values(r.normal(0, K ** -0.5, (N, K)))).to(device)
+        x, wt = x.to(torch.bfloat16), wt.to(torch.bfloat16)
+        y = torch.empty((M, N), dtype=torch.float32, device=device)
+        return (lambda i: gdn.linear_bf16(x, wt, y)), dict(flops=2 * M * N * K)
+    raise KeyError(f"unknown case {name!r}")
+
+
+PROFILE_CASES = ("decode_l1_b1", "decode_l1_b64", "decode_l36_b16", "prefill_b4_t4096",
+                 "layer_decode_b256", "layer_pair_b256", "forward_batch_b4_t4096",
+                 "linear_bf16_m16384_n8192_k2048", "short_conv_decode_b64", "short_conv_pair_b64",
+                 "short_conv_batch_b4_t4096", "kda_decode_b64", "kda_prefill_b4_t4096")
+
+
+def run_profile_case(name: str, launches: int) -> int:
+    """Run `launches` calls of one case and exit (no timing): the program
+    that ncu captures for the summaries kept with the sources."""
+    import torch
+    if not torch.cuda.is_available():
+        raise SystemExit("bench.py needs a CUDA device (there is no CPU path)")
+    device = torch.device("cuda", 0)
+    launch, _ = build_case(name, device)
+    for i in range(launches):
+        launch(i)
+    torch.cuda.synchronize()
+    print(f"ok {name} x{launches}")
+    return 0
+
+
+def bench_layer(steps: int, warmup: int, device):
+    import torch
+    launch, meta = build_case("layer_decode_b256", device)
     stream = torch.cuda.current_stream(device)
-
-    def launch(i):
-        gdn.layer_decode(*(t[n] for n in order), out, Hk=16)
-
     secs = time_launches(launch, 1, steps, warmup, stream, graph=True)
-    return dict(seconds=secs, launches=steps, bytes=layer_bytes(B), tokens=B)
+    return dict(seconds=secs, launches=steps, bytes=layer_bytes(meta["B"]), tokens=meta["B"])
 
 
 def bench_layer_pair(steps: int, warmup: int, device):
     import torch
-    from linear_attention_recurrence_04_b200 import gdn, inputs
-    B = 256
-    d = inputs.layer_inputs(B, seed=1005)
-    d2 = inputs.layer_inputs(B, seed=1006)
-    for n in ("mixed_qkv", "z", "a", "b"):
-        d[n] = np.stack([d[n], d2[n]], axis=1)
-    t = _to_dev(d, device)
-    sring = torch.empty_like(t["conv_ring"])
-    sstate = torch.empty_like(t["state"])
-    out = torch.empty((B, 2, 32 * 128), dtype=torch.float32, device=device)
-    order = ("mixed_qkv", "z", "a", "b", "conv_ring", "conv_w", "A_log", "dt_bias", "norm_w",
-             "state")
+    launch, meta = build_case("layer_pair_b256", device)
     stream = torch.cuda.current_stream(device)
-
-    def launch(i):
-        gdn.layer_pair(*(t[n] for n in order), sring, sstate, out, Hk=16)
-
     secs = time_launches(launch, 1, steps, warmup, stream, graph=True)
+    B = meta["B"]
     return dict(seconds=secs, launches=steps, bytes=layer_pair_bytes(B), tokens=2 * B)
 
 
@@ -436,28 +553,62 @@ def bench_forward_batch(steps: int, warmup: int, device):
     """The layer over B = 4 x T = 4096 positions with dense bf16 projections
     (D = 2048), graph-replayed; the ring and state advance from call to call."""
     import torch
-    from linear_attention_recurrence_04_b200 import gdn, inputs
-    w = inputs.FORWARD_WORKLOAD
-    B, T = w.sizes["B"], w.sizes["T"]
-    d = w.draw()
-    bf = ("hidden", "w_qkv", "w_z", "w_ba", "w_out")
-    t = {k: (torch.from_numpy(v).to(device).to(torch.bfloat16) if k in bf
-             else torch.from_numpy(v).to(device)) for k, v in d.items()}
-    D = t["hidden"].shape[2]
-    out = torch.empty((B, T, D), dtype=torch.float32, device=device)
-    ws = torch.empty(gdn.forward_batch_workspace_size(B, T), dtype=torch.uint8, device=device)
+    launch, meta = build_case("forward_batch_b4_t4096", device)
+    B, T, D = meta["B"], meta["T"], meta["D"]
     stream = torch.cuda.current_stream(device)
-
-    def launch(i):
-        gdn.forward_batch(t["hidden"], t["w_qkv"], t["w_z"], t["w_ba"], t["w_out"],
-                          t["conv_ring"], t["conv_w"], t["A_log"], t["dt_bias"], t["norm_w"],
-                          t["state"], out, ws, Hk=16)
-
     secs = time_launches(launch, 1, steps, warmup, stream, graph=True)
     C, HD, Hv = 8192, 4096, 32
     gemm_flops = 2 * B * T * D * (C + HD + 2 * Hv) + 2 * B * T * HD * D
     return dict(seconds=secs, launches=steps, tokens=B * T, gemm_flops=gemm_flops,
                 rec_flops=prefill_flops(B, T))
+
+
+def bench_short_conv(name: str, steps: int, warmup: int, device, peaks):
+    """One short-conv workload, graph-replayed; HBM roofline for the decode
+    and verify launches (weight streaming), tensor roofline for the batch."""
+    import torch
+    launch, m = build_case(name, device)
+    stream = torch.cuda.current_stream(device)
+    secs = time_launches(launch, 1, steps, warmup, stream, graph=True)
+    per = secs / steps
+    B, T, D, K = m["B"], m["T"], m["D"], m["K"]
+    r = {"ms_per_launch": per * 1e3, "tokens_per_s": B * T / per}
+    if T <= 2:
+        gbs = short_conv_bytes(B, T, D, K, pair=(name == "short_conv_pair_b64")) / per / 1e9
+        r.update(gb_s=gbs, roofline={"bound": "hbm", "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                                     "frac": gbs / peaks["hbm_gbs"]})
+    else:
+        tf = short_conv_flops(B, T, D) / per / 1e12
+        r.update(tflops=tf, roofline={"bound": "tensor", "peak": peaks["bf16_tflops"],
+                                      "unit": "TFLOP/s", "frac": tf / peaks["bf16_tflops"]})
+    return r
+
+
+def bench_kda(steps_decode: int, steps_prefill: int, device, peaks, alu_peak):
+    """The KDA core: the B = 64 decode token (HBM roofline) and the
+    4 x 4096-position prefill (fp32 ALU roofline), graph-replayed; the
+    prefill's state carries over from launch to launch, which changes no
+    work per launch."""
+    import torch
+    stream = torch.cuda.current_stream(device)
+    launch, m = build_case("kda_decode_b64", device)
+    per = time_launches(launch, 1, steps_decode, 10, stream, graph=True) / steps_decode
+    L, B = m["sizes"]["L"], m["sizes"]["B"]
+    gbs = kda_step_bytes(L, B) / per / 1e9
+    res = {"kda_decode_b64": {
+        "ms_per_launch": per * 1e3, "layer_tokens_per_s": L * B / per, "gb_s": gbs,
+        "roofline": {"bound": "hbm", "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                     "frac": gbs / peaks["hbm_gbs"]}}}
+    del launch, m
+    torch.cuda.empty_cache()
+    launch, m = build_case("kda_prefill_b4_t4096", device)
+    per = time_launches(launch, 1, steps_prefill, 3, stream, graph=True) / steps_prefill
+    B, T = m["sizes"]["B"], m["sizes"]["T"]
+    tf = prefill_flops(B, T) / per / 1e12
+    res["kda_prefill_b4_t4096"] = {
+        "ms_per_launch": per * 1e3, "tokens_per_s": B * T / per, "fp32_tflops": tf,
+        "roofline": {"bound": "alu", "peak": alu_peak, "unit": "TFLOP/s", "frac": tf / alu_peak}}
+    return res
 
 
 def cpu_oracle_baseline(name: str, budget_s: float, max_units: Optional[int] = None):
@@ -671,6 +822,13 @@ def run_ours(args) -> int:
             "projection_tflops": fb["gemm_flops"] / per / 1e12,
             "note": "D=2048 bf16 projections on tcgen05 + conv + sequential recurrence + tail",
         }
+        torch.cuda.empty_cache()
+        for name in ("short_conv_decode_b64", "short_conv_pair_b64"):
+            extras[name] = bench_short_conv(name, 200, 10, device, peaks)
+        extras["short_conv_batch_b4_t4096"] = bench_short_conv("short_conv_batch_b4_t4096", 10, 3,
+                                                               device, peaks)
+        torch.cuda.empty_cache()
+        extras.update(bench_kda(200, 5, device, peaks, alu_peak))
         line["workloads"] = extras
 
     if env["rank"] == 0 and env["world"] == 1 and not args.no_cpu_baseline:
@@ -704,9 +862,14 @@ def main(argv=None) -> int:
     ap.add_argument("--cpu-budget", type=float, default=10.0,
                     help="seconds of CPU time for the oracle baseline sample")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--profile-case", choices=PROFILE_CASES, default=None,
+                    help="run --launches calls of one case without timing (for ncu) and exit")
+    ap.add_argument("--launches", type=int, default=3)
     ap.add_argument("--no-extras", action="store_true",
                     help="skip the other four workloads (headline only)")
     args = ap.parse_args(argv)
+    if args.profile_case:
+        return run_profile_case(args.profile_case, args.launches)
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")
     if args.impl == "reference":

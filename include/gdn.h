@@ -258,6 +258,84 @@ gdn_status gdn_forward_batch_noalloc(const void *hidden, const void *w_qkv, cons
                                      int64_t T, int64_t D, int64_t Hk, int64_t Hv, int64_t dk,
                                      int64_t dv, int64_t K, uint32_t *status, void *stream);
 
+/*
+ * gdn_kda_step / gdn_kda_prefill -- the KDA core ("Module linear_core",
+ * entries "kda_forward": one position, advances the state, and
+ * "kda_forward_batch": the recurrence sequential per position, elementwise
+ * identical to the one-position path). The pages give no equations; the
+ * update implemented is the published Kimi Delta Attention rule, the
+ * delta rule with a decay per key channel. In the layout of gdn_step
+ * (M[j][i] = S[i][j]), per value head h reading key head h % Hk:
+ *   1. M[j][i] *= exp(g[h][i])  2. sk[j] = M[j].k  3. delta[j] = (v[j] - sk[j]) beta
+ *   4. M[j] += delta[j] k       5. out[j] = M_new[j].q / sqrt(dk)
+ * Arguments, layouts, ownership and errors are those of gdn_step and
+ * gdn_prefill, except the log-decay:
+ *   gdn_kda_step:    g [L][B][Hv][dk]
+ *   gdn_kda_prefill: g [B][T][Hv][dk]   (contiguous)
+ * g must be 16-byte aligned. Values at or below 0 are expected (decays in
+ * (0, 1]); others are applied as given.
+ */
+gdn_status gdn_kda_step(float *state, const float *q, const float *k, const float *v,
+                        const float *beta, const float *g, float *out, int64_t L, int64_t B,
+                        int64_t Hk, int64_t Hv, int64_t dk, int64_t dv, void *stream);
+gdn_status gdn_kda_prefill(float *state, const float *q, const float *k, const float *v,
+                           const float *beta, const float *g, float *out, int64_t B, int64_t T,
+                           int64_t Hk, int64_t Hv, int64_t dk, int64_t dv, void *stream);
+
+/*
+ * The LFM2 short-convolution mixer ("Module linear_core", struct
+ * "ShortConvWeights": no recurrent state, the only state is the causal conv
+ * ring holding the last kernel-1 gated inputs of every channel; entries
+ * "short_conv_forward", "short_conv_forward_batch" and "short_conv_pair").
+ * The pages give no formula; the mixer implemented is, per position t and
+ * channel d:
+ *   (bg | cg | xv) = W_in h_t        rows [0,D) | [D,2D) | [2D,3D) of W_in
+ *   u = bg[d] * xv[d]                the gated input, rounded to fp32
+ *   conv = sum_{tau<K} conv_w[d][tau] * window[tau],
+ *          window = (ring[0..K-2], u) oldest first, no bias
+ *   y = cg[d] * conv                 rounded to bf16
+ *   out_t = W_out y                  (tensor-core GEMMs, fp32 accumulation)
+ * and the ring drops its oldest slot and appends u.
+ *
+ *   hidden    [B][T][D] bf16        D a positive multiple of 8
+ *   w_in      [3D][D] bf16
+ *   w_out     [D][D] bf16
+ *   conv_ring [B][K-1][D] fp32 in/out, slot 0 oldest
+ *   conv_w    [D][K] fp32, tap 0 multiplies the oldest slot; K in {2, 3, 4}
+ *   out       [B][T][D] fp32
+ *   workspace device scratch of gdn_short_conv_workspace_size(B, T, D) bytes,
+ *             256-byte aligned, owned by the caller; contents on entry do
+ *             not matter and are undefined afterwards
+ *   status    optional zero-initialised device word for timeout bits (see
+ *             gdn_linear_bf16)
+ * All pointers are device pointers, 16-byte aligned. conv_ring is updated in
+ * place and may overlap nothing else; out may overlap no argument.
+ * gdn_short_conv_workspace_size returns 0 for an invalid shape.
+ *
+ * gdn_short_conv_forward_batch runs T positions in order; conv_ring ends as
+ * the ring after position T-1 (T = 0 does nothing).
+ * gdn_short_conv_forward is the same call for one position per sequence:
+ * hidden [B][D], out [B][D].
+ * gdn_short_conv_pair is the two-position verify: hidden [B][2][D],
+ * out [B][2][D]; conv_ring receives the ring after position 0 (committed)
+ * and scratch_ring [B][K-1][D] the ring after position 1 (tentative, to be
+ * swapped in on acceptance). scratch_ring may overlap nothing else.
+ */
+size_t gdn_short_conv_workspace_size(int64_t B, int64_t T, int64_t D);
+gdn_status gdn_short_conv_forward_batch(const void *hidden, const void *w_in, const void *w_out,
+                                        float *conv_ring, const float *conv_w, float *out,
+                                        void *workspace, size_t workspace_bytes, int64_t B,
+                                        int64_t T, int64_t D, int64_t K, uint32_t *status,
+                                        void *stream);
+gdn_status gdn_short_conv_forward(const void *hidden, const void *w_in, const void *w_out,
+                                  float *conv_ring, const float *conv_w, float *out,
+                                  void *workspace, size_t workspace_bytes, int64_t B, int64_t D,
+                                  int64_t K, uint32_t *status, void *stream);
+gdn_status gdn_short_conv_pair(const void *hidden, const void *w_in, const void *w_out,
+                               float *conv_ring, float *scratch_ring, const float *conv_w,
+                               float *out, void *workspace, size_t workspace_bytes, int64_t B,
+                               int64_t D, int64_t K, uint32_t *status, void *stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -7,7 +7,10 @@ the library is missing: there is no CPU fallback. ``inputs`` draws the seeded
 synthetic workloads and needs neither the library nor a GPU.
 """
 _BINDING = ("GdnError", "step", "prefill", "layer_decode", "layer_pair", "linear_bf16",
-            "forward_batch", "forward_batch_workspace_size", "library_path", "status_string")
+            "forward_batch", "forward_batch_workspace_size", "forward_batch_noalloc",
+            "short_conv_forward", "short_conv_forward_batch", "short_conv_pair",
+            "short_conv_workspace_size", "kda_step", "kda_prefill", "library_path",
+            "status_string")
 
 
 def __getattr__(name):

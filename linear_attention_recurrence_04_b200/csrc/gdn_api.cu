@@ -175,58 +175,108 @@ const char* gdn_status_string(int status) {
 
 const char* gdn_last_error(void) { return g_last_error; }
 
-gdn_status gdn_step(float* state, const float* q, const float* k, const float* v,
-                    const float* beta, const float* gate, float* out, int64_t L, int64_t B,
-                    int64_t Hk, int64_t Hv, int64_t dk, int64_t dv, void* stream) {
-    if (L < 0 || B < 0) return fail(GDN_ERR_SHAPE, "negative L=%lld or B=%lld", (long long)L,
-                                    (long long)B);
+}  // extern "C"
+
+namespace {
+
+// Checks shared by the decode entries: gdn_step (one log-decay per head,
+// gate_w = 1) and gdn_kda_step (one per head and key channel, gate_w = dk).
+gdn_status step_call(const char* fn, float* state, const float* q, const float* k,
+                     const float* v, const float* beta, const float* gate, float* out,
+                     int64_t L, int64_t B, int64_t Hk, int64_t Hv, int64_t dk, int64_t dv,
+                     bool channel_decay, void* stream) {
+    if (L < 0 || B < 0) return fail(GDN_ERR_SHAPE, "%s: negative L=%lld or B=%lld", fn,
+                                    (long long)L, (long long)B);
     gdn_status st = check_geometry(Hk, Hv, dk, dv);
     if (st != GDN_OK) return st;
-    int64_t lb = 0, heads = 0, state_n = 0, qk_n = 0, v_n = 0;
+    int64_t lb = 0, heads = 0, state_n = 0, qk_n = 0, v_n = 0, gate_n = 0;
     if (!mul_ok(L, B, &lb) || !mul_ok(lb, Hv, &heads) || !mul_ok(heads, dv * dk, &state_n) ||
-        !mul_ok(lb, Hk * dk, &qk_n) || !mul_ok(heads, dv, &v_n) || state_n > INT64_MAX / 8)
-        return fail(GDN_ERR_OVERFLOW, "L*B*Hv*dv*dk overflows int64");
+        !mul_ok(lb, Hk * dk, &qk_n) || !mul_ok(heads, dv, &v_n) ||
+        !mul_ok(heads, channel_decay ? dk : 1, &gate_n) || state_n > INT64_MAX / 8)
+        return fail(GDN_ERR_OVERFLOW, "%s: L*B*Hv*dv*dk overflows int64", fn);
     if (heads == 0) { g_last_error[0] = '\0'; return GDN_OK; }
     if (!state || !q || !k || !v || !beta || !gate || !out)
-        return fail(GDN_ERR_NULL, "gdn_step: a tensor pointer is NULL");
+        return fail(GDN_ERR_NULL, "%s: a tensor pointer is NULL", fn);
     if (!aligned(state, 16) || !aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) ||
-        !aligned(out, 16) || !aligned(beta, 4) || !aligned(gate, 4))
-        return fail(GDN_ERR_ALIGN, "gdn_step: state/q/k/v/out need 16-byte, beta/gate 4-byte alignment");
+        !aligned(out, 16) || !aligned(beta, 4) || !aligned(gate, channel_decay ? 16 : 4))
+        return fail(GDN_ERR_ALIGN, "%s: state/q/k/v/out%s need 16-byte, beta%s 4-byte alignment",
+                    fn, channel_decay ? "/g" : "", channel_decay ? "" : "/gate");
     const Span ins[] = {{state, state_n * 4, "state"}, {q, qk_n * 4, "q"}, {k, qk_n * 4, "k"},
-                        {v, v_n * 4, "v"}, {beta, heads * 4, "beta"}, {gate, heads * 4, "gate"}};
+                        {v, v_n * 4, "v"}, {beta, heads * 4, "beta"},
+                        {gate, gate_n * 4, channel_decay ? "g" : "gate"}};
     st = check_spans(ins, 6, 1, Span{out, v_n * 4, "out"});
     if (st != GDN_OK) return st;
     StepArgs a{state, q, k, v, beta, gate, out, heads, static_cast<int>(Hk), static_cast<int>(Hv)};
-    return launched(launch_step(a, static_cast<cudaStream_t>(stream)), "gdn_step");
+    const cudaStream_t s = static_cast<cudaStream_t>(stream);
+    return launched(channel_decay ? launch_kda_step(a, s) : launch_step(a, s), fn);
+}
+
+// Checks shared by the multi-position entries gdn_prefill and gdn_kda_prefill.
+gdn_status prefill_call(const char* fn, float* state, const float* q, const float* k,
+                        const float* v, const float* beta, const float* gate, float* out,
+                        int64_t B, int64_t T, int64_t Hk, int64_t Hv, int64_t dk, int64_t dv,
+                        bool channel_decay, void* stream) {
+    if (B < 0 || T < 0) return fail(GDN_ERR_SHAPE, "%s: negative B=%lld or T=%lld", fn,
+                                    (long long)B, (long long)T);
+    gdn_status st = check_geometry(Hk, Hv, dk, dv);
+    if (st != GDN_OK) return st;
+    int64_t bt = 0, heads = 0, state_n = 0, qk_n = 0, v_n = 0, bh = 0, gate_n = 0;
+    if (!mul_ok(B, T, &bt) || !mul_ok(B, Hv, &heads) || !mul_ok(heads, dv * dk, &state_n) ||
+        !mul_ok(bt, Hk * dk, &qk_n) || !mul_ok(bt, Hv * dv, &v_n) || !mul_ok(bt, Hv, &bh) ||
+        !mul_ok(bh, channel_decay ? dk : 1, &gate_n) || v_n > INT64_MAX / 8 ||
+        qk_n > INT64_MAX / 8 || gate_n > INT64_MAX / 8)
+        return fail(GDN_ERR_OVERFLOW, "%s: B*T*Hv*dv overflows int64", fn);
+    // One warp per 8 rows of a head (pair); the grid must fit gridDim.x.
+    if (heads * (kDv / 8) > INT32_MAX)
+        return fail(GDN_ERR_OVERFLOW, "%s: B*Hv=%lld exceeds the launch grid", fn,
+                    (long long)heads);
+    if (bt == 0 || heads == 0) { g_last_error[0] = '\0'; return GDN_OK; }
+    if (!state || !q || !k || !v || !beta || !gate || !out)
+        return fail(GDN_ERR_NULL, "%s: a tensor pointer is NULL", fn);
+    if (!aligned(state, 16) || !aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) ||
+        !aligned(out, 16) || !aligned(beta, 4) || !aligned(gate, channel_decay ? 16 : 4))
+        return fail(GDN_ERR_ALIGN, "%s: state/q/k/v/out%s need 16-byte, beta%s 4-byte alignment",
+                    fn, channel_decay ? "/g" : "", channel_decay ? "" : "/gate");
+    const Span ins[] = {{state, state_n * 4, "state"}, {q, qk_n * 4, "q"}, {k, qk_n * 4, "k"},
+                        {v, v_n * 4, "v"}, {beta, bh * 4, "beta"},
+                        {gate, gate_n * 4, channel_decay ? "g" : "gate"}};
+    st = check_spans(ins, 6, 1, Span{out, v_n * 4, "out"});
+    if (st != GDN_OK) return st;
+    PrefillArgs a{state, q, k, v, beta, gate, out, B, T, static_cast<int>(Hk), static_cast<int>(Hv)};
+    const cudaStream_t s = static_cast<cudaStream_t>(stream);
+    return launched(channel_decay ? launch_kda_prefill(a, s) : launch_prefill(a, s), fn);
+}
+
+}  // namespace
+
+extern "C" {
+
+gdn_status gdn_step(float* state, const float* q, const float* k, const float* v,
+                    const float* beta, const float* gate, float* out, int64_t L, int64_t B,
+                    int64_t Hk, int64_t Hv, int64_t dk, int64_t dv, void* stream) {
+    return step_call("gdn_step", state, q, k, v, beta, gate, out, L, B, Hk, Hv, dk, dv, false,
+                     stream);
 }
 
 gdn_status gdn_prefill(float* state, const float* q, const float* k, const float* v,
                        const float* beta, const float* gate, float* out, int64_t B, int64_t T,
                        int64_t Hk, int64_t Hv, int64_t dk, int64_t dv, void* stream) {
-    if (B < 0 || T < 0) return fail(GDN_ERR_SHAPE, "negative B=%lld or T=%lld", (long long)B,
-                                    (long long)T);
-    gdn_status st = check_geometry(Hk, Hv, dk, dv);
-    if (st != GDN_OK) return st;
-    int64_t bt = 0, heads = 0, state_n = 0, qk_n = 0, v_n = 0, bh = 0;
-    if (!mul_ok(B, T, &bt) || !mul_ok(B, Hv, &heads) || !mul_ok(heads, dv * dk, &state_n) ||
-        !mul_ok(bt, Hk * dk, &qk_n) || !mul_ok(bt, Hv * dv, &v_n) || !mul_ok(bt, Hv, &bh) ||
-        v_n > INT64_MAX / 8 || qk_n > INT64_MAX / 8)
-        return fail(GDN_ERR_OVERFLOW, "B*T*Hv*dv overflows int64");
-    // One warp per 8 rows of a head pair; the grid must fit gridDim.x.
-    if (heads * (kDv / 8) > INT32_MAX)
-        return fail(GDN_ERR_OVERFLOW, "B*Hv=%lld exceeds the launch grid", (long long)heads);
-    if (bt == 0 || heads == 0) { g_last_error[0] = '\0'; return GDN_OK; }
-    if (!state || !q || !k || !v || !beta || !gate || !out)
-        return fail(GDN_ERR_NULL, "gdn_prefill: a tensor pointer is NULL");
-    if (!aligned(state, 16) || !aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) ||
-        !aligned(out, 16) || !aligned(beta, 4) || !aligned(gate, 4))
-        return fail(GDN_ERR_ALIGN, "gdn_prefill: state/q/k/v/out need 16-byte, beta/gate 4-byte alignment");
-    const Span ins[] = {{state, state_n * 4, "state"}, {q, qk_n * 4, "q"}, {k, qk_n * 4, "k"},
-                        {v, v_n * 4, "v"}, {beta, bh * 4, "beta"}, {gate, bh * 4, "gate"}};
-    st = check_spans(ins, 6, 1, Span{out, v_n * 4, "out"});
-    if (st != GDN_OK) return st;
-    PrefillArgs a{state, q, k, v, beta, gate, out, B, T, static_cast<int>(Hk), static_cast<int>(Hv)};
-    return launched(launch_prefill(a, static_cast<cudaStream_t>(stream)), "gdn_prefill");
+    return prefill_call("gdn_prefill", state, q, k, v, beta, gate, out, B, T, Hk, Hv, dk, dv,
+                        false, stream);
+}
+
+gdn_status gdn_kda_step(float* state, const float* q, const float* k, const float* v,
+                        const float* beta, const float* g, float* out, int64_t L, int64_t B,
+                        int64_t Hk, int64_t Hv, int64_t dk, int64_t dv, void* stream) {
+    return step_call("gdn_kda_step", state, q, k, v, beta, g, out, L, B, Hk, Hv, dk, dv, true,
+                     stream);
+}
+
+gdn_status gdn_kda_prefill(float* state, const float* q, const float* k, const float* v,
+                           const float* beta, const float* g, float* out, int64_t B, int64_t T,
+                           int64_t Hk, int64_t Hv, int64_t dk, int64_t dv, void* stream) {
+    return prefill_call("gdn_kda_prefill", state, q, k, v, beta, g, out, B, T, Hk, Hv, dk, dv,
+                        true, stream);
 }
 
 namespace {
@@ -405,6 +455,95 @@ gdn_status gdn_forward_batch(const void* hidden, const void* w_qkv, const void* 
                        l2_eps, norm_eps, state, out, workspace, B, T, D, static_cast<int>(Hk),
                        static_cast<int>(Hv), status};
     return launched(launch_forward_batch(a, static_cast<cudaStream_t>(stream)), fn);
+}
+
+size_t gdn_short_conv_workspace_size(int64_t B, int64_t T, int64_t D) {
+    if (B < 0 || T < 0 || D <= 0 || D % 8 != 0 || D > (1 << 24) || B > 65535 ||
+        T > (int64_t)65535 * 128 || B * T > (int64_t)65535 * 128)
+        return 0;
+    return short_conv_layout(B, T, D).total;
+}
+
+}  // extern "C"
+
+namespace {
+
+// Shared checks of the three short-conv entries; n_commit positions go to
+// conv_ring, the ring after the last position to scratch_ring (if given).
+gdn_status short_conv_call(const char* fn, const void* hidden, const void* w_in,
+                           const void* w_out, float* conv_ring, float* scratch_ring,
+                           const float* conv_w, float* out, void* workspace,
+                           size_t workspace_bytes, int64_t B, int64_t T, int64_t D, int64_t K,
+                           int64_t n_commit, uint32_t* status, void* stream) {
+    if (B < 0 || T < 0 || D < 0) return fail(GDN_ERR_SHAPE, "%s: negative B, T or D", fn);
+    if (K < 2 || K > 4)
+        return fail(GDN_ERR_UNSUPPORTED, "%s: K=%lld: conv kernels of 2, 3 or 4 are implemented",
+                    fn, (long long)K);
+    if (D == 0 || D % 8 != 0)
+        return fail(GDN_ERR_UNSUPPORTED, "%s: D=%lld must be a positive multiple of 8", fn,
+                    (long long)D);
+    if (B > 65535 || T > (int64_t)65535 * 128 || B * T > (int64_t)65535 * 128 || D > (1 << 24))
+        return fail(GDN_ERR_OVERFLOW, "%s: B=%lld, B*T=%lld or D too large", fn, (long long)B,
+                    (long long)(B * T));
+    const int64_t BT = B * T;
+    if (BT == 0) { g_last_error[0] = '\0'; return GDN_OK; }
+    const size_t need = short_conv_layout(B, T, D).total;
+    if (!hidden || !w_in || !w_out || !conv_ring || !conv_w || !out || !workspace)
+        return fail(GDN_ERR_NULL, "%s: a tensor pointer is NULL", fn);
+    if (workspace_bytes < need)
+        return fail(GDN_ERR_SHAPE, "%s: workspace of %zu bytes, %zu needed", fn, workspace_bytes,
+                    need);
+    if (!aligned(hidden, 16) || !aligned(w_in, 16) || !aligned(w_out, 16) ||
+        !aligned(conv_ring, 16) || !aligned(conv_w, 16) || !aligned(out, 16) ||
+        (scratch_ring && !aligned(scratch_ring, 16)) || !aligned(workspace, 256) ||
+        (status && !aligned(status, 4)))
+        return fail(GDN_ERR_ALIGN, "%s: alignment rule violated (workspace needs 256 bytes)", fn);
+    const int64_t ring_bytes = B * (K - 1) * D * 4;
+    const Span ins[] = {{conv_ring, ring_bytes, "conv_ring"},
+                        {scratch_ring, scratch_ring ? ring_bytes : 0, "scratch_ring"},
+                        {workspace, static_cast<int64_t>(need), "workspace"},
+                        {status, status ? 4 : 0, "status"},
+                        {hidden, BT * D * 2, "hidden"}, {w_in, 3 * D * D * 2, "w_in"},
+                        {w_out, D * D * 2, "w_out"}, {conv_w, D * K * 4, "conv_w"}};
+    gdn_status st = check_spans(ins, 8, 4, Span{out, BT * D * 4, "out"});
+    if (st != GDN_OK) return st;
+    ShortConvArgs a{hidden, w_in, w_out, conv_ring, scratch_ring, conv_w, out, workspace,
+                    B, T, D, static_cast<int>(K), n_commit, status};
+    return launched(launch_short_conv(a, static_cast<cudaStream_t>(stream)), fn);
+}
+
+}  // namespace
+
+extern "C" {
+
+gdn_status gdn_short_conv_forward_batch(const void* hidden, const void* w_in, const void* w_out,
+                                        float* conv_ring, const float* conv_w, float* out,
+                                        void* workspace, size_t workspace_bytes, int64_t B,
+                                        int64_t T, int64_t D, int64_t K, uint32_t* status,
+                                        void* stream) {
+    return short_conv_call("gdn_short_conv_forward_batch", hidden, w_in, w_out, conv_ring,
+                           nullptr, conv_w, out, workspace, workspace_bytes, B, T, D, K, T,
+                           status, stream);
+}
+
+gdn_status gdn_short_conv_forward(const void* hidden, const void* w_in, const void* w_out,
+                                  float* conv_ring, const float* conv_w, float* out,
+                                  void* workspace, size_t workspace_bytes, int64_t B, int64_t D,
+                                  int64_t K, uint32_t* status, void* stream) {
+    return short_conv_call("gdn_short_conv_forward", hidden, w_in, w_out, conv_ring, nullptr,
+                           conv_w, out, workspace, workspace_bytes, B, 1, D, K, 1, status,
+                           stream);
+}
+
+gdn_status gdn_short_conv_pair(const void* hidden, const void* w_in, const void* w_out,
+                               float* conv_ring, float* scratch_ring, const float* conv_w,
+                               float* out, void* workspace, size_t workspace_bytes, int64_t B,
+                               int64_t D, int64_t K, uint32_t* status, void* stream) {
+    if (B > 0 && !scratch_ring)
+        return fail(GDN_ERR_NULL, "gdn_short_conv_pair: scratch_ring is NULL");
+    return short_conv_call("gdn_short_conv_pair", hidden, w_in, w_out, conv_ring, scratch_ring,
+                           conv_w, out, workspace, workspace_bytes, B, 2, D, K, 1, status,
+                           stream);
 }
 
 }  // extern "C"

@@ -31,7 +31,9 @@ namespace gdn {
 namespace {
 
 // 2. causal depthwise conv over positions, SiLU, in place; ring update.
-__global__ void __launch_bounds__(256)
+constexpr int kConvThreads = 64;          // small blocks: B*C threads spread over every SM
+
+__global__ void __launch_bounds__(kConvThreads)
 conv_seq_kernel(float* __restrict__ act, float* __restrict__ ring,
                 const float* __restrict__ conv_w, int64_t B, int64_t T, int64_t C) {
     const int64_t idx = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
@@ -44,8 +46,9 @@ conv_seq_kernel(float* __restrict__ act, float* __restrict__ ring,
     float* col = act + b * T * C + c;
     // Positions in blocks of kSeqBlock: all loads of a block are issued
     // before any of its (sequential) conv steps, so the memory latency is
-    // paid once per block rather than once per position.
-    constexpr int kSeqBlock = 16;
+    // paid once per block rather than once per position, with enough bytes
+    // in flight per SM to keep HBM busy.
+    constexpr int kSeqBlock = 64;
     for (int64_t t0 = 0; t0 < T; t0 += kSeqBlock) {
         const int n = (T - t0) < kSeqBlock ? static_cast<int>(T - t0) : kSeqBlock;
         float xs[kSeqBlock];
@@ -103,7 +106,9 @@ __device__ __forceinline__ double warp_sum_d(double x) {
     return x;
 }
 
-// 5. gated RMSNorm per (position, value head) in double; y in bf16.
+// 5. gated RMSNorm per (position, value head); y in bf16. The sum of squares
+//    and 1/rms are taken in double, the gate in fp32: y is rounded to bf16
+//    (relative step 2^-8) right after, far coarser than fp32's error.
 __global__ void __launch_bounds__(256)
 tail_bf16_kernel(const float* __restrict__ o, const float* __restrict__ z,
                  const float* __restrict__ norm_w, __nv_bfloat16* __restrict__ y, int64_t rows,
@@ -114,20 +119,19 @@ tail_bf16_kernel(const float* __restrict__ o, const float* __restrict__ z,
     const float4 ov = ld_ro4(o + r * kDv + lane * 4);
     const float4 zv = ld_ro4(z + r * kDv + lane * 4);
     const float4 wv = ld_ro4(norm_w + lane * 4);
-    const double o4[4] = {ov.x, ov.y, ov.z, ov.w};
-    const double z4[4] = {zv.x, zv.y, zv.z, zv.w};
-    const double w4[4] = {wv.x, wv.y, wv.z, wv.w};
+    const float o4[4] = {ov.x, ov.y, ov.z, ov.w};
+    const float z4[4] = {zv.x, zv.y, zv.z, zv.w};
+    const float w4[4] = {wv.x, wv.y, wv.z, wv.w};
     double ss = 0.0;
 #pragma unroll
-    for (int i = 0; i < 4; ++i) ss = fma(o4[i], o4[i], ss);
+    for (int i = 0; i < 4; ++i) ss = fma(static_cast<double>(o4[i]), static_cast<double>(o4[i]), ss);
     ss = warp_sum_d(ss);
-    const double inv_rms = 1.0 / sqrt(ss / static_cast<double>(kDv) + static_cast<double>(norm_eps));
+    const float inv_rms =
+        static_cast<float>(1.0 / sqrt(ss / static_cast<double>(kDv) + static_cast<double>(norm_eps)));
     __nv_bfloat16 out4[4];
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {
-        const double silu = z4[i] / (1.0 + exp(-z4[i]));
-        out4[i] = __double2bfloat16(o4[i] * inv_rms * w4[i] * silu);
-    }
+    for (int i = 0; i < 4; ++i)
+        out4[i] = __float2bfloat16_rn(o4[i] * inv_rms * w4[i] * siluf_acc(z4[i]));
     *reinterpret_cast<uint2*>(y + r * kDv + lane * 4) = *reinterpret_cast<const uint2*>(out4);
 }
 
@@ -179,7 +183,8 @@ cudaError_t launch_forward_batch(const ForwardBatchArgs& a, cudaStream_t stream)
     // 2. conv over positions with the ring, SiLU
     {
         const int64_t n = a.B * C;
-        conv_seq_kernel<<<static_cast<unsigned>((n + 255) / 256), 256, 0, stream>>>(
+        conv_seq_kernel<<<static_cast<unsigned>((n + kConvThreads - 1) / kConvThreads),
+                          kConvThreads, 0, stream>>>(
             act, a.conv_ring, a.conv_w, a.B, a.T, C);
         if ((err = cudaGetLastError())) return err;
     }

@@ -100,13 +100,38 @@ struct ForwardBatchLayout {
 };
 ForwardBatchLayout forward_batch_layout(int64_t B, int64_t T, int Hk, int Hv);
 
+// The LFM2 short-conv mixer over T positions (gdn_short_conv.cu).
+struct ShortConvArgs {
+    const void* hidden;    // [B][T][D] bf16
+    const void* w_in;      // [3D][D] bf16: input gate | output gate | value rows
+    const void* w_out;     // [D][D] bf16
+    float* conv_ring;      // [B][K-1][D] gated inputs, oldest first (in/out)
+    float* scratch_ring;   // [B][K-1][D] ring after the last position, or null
+    const float* conv_w;   // [D][K]
+    float* out;            // [B][T][D] fp32
+    void* workspace;       // short_conv_layout(B, T, D).total bytes, 256-aligned
+    int64_t B, T, D;
+    int K;                 // 2, 3 or 4
+    int64_t n_commit;      // conv_ring receives the ring after position n_commit - 1
+    uint32_t* status;
+};
+struct ShortConvLayout {
+    size_t proj, y, total;
+};
+ShortConvLayout short_conv_layout(int64_t B, int64_t T, int64_t D);
+
 // Each launcher enqueues its kernel on `stream` and returns the launch status.
 cudaError_t launch_step(const StepArgs& a, cudaStream_t stream);
+// KDA core: StepArgs / PrefillArgs with `gate` holding a log-decay per key
+// channel, [..][Hv][dk] (contiguous).
+cudaError_t launch_kda_step(const StepArgs& a, cudaStream_t stream);
+cudaError_t launch_kda_prefill(const PrefillArgs& a, cudaStream_t stream);
 cudaError_t launch_prefill(const PrefillArgs& a, cudaStream_t stream);
 cudaError_t launch_layer_decode(const LayerArgs& a, cudaStream_t stream);
 cudaError_t launch_layer_pair(const LayerArgs& a, cudaStream_t stream);
 cudaError_t launch_linear_bf16(const LinearArgs& a, cudaStream_t stream);
 cudaError_t launch_forward_batch(const ForwardBatchArgs& a, cudaStream_t stream);
+cudaError_t launch_short_conv(const ShortConvArgs& a, cudaStream_t stream);
 
 // Value-heads-per-key-head ratios the fused layer kernel is compiled for.
 bool layer_decode_supports(int G);

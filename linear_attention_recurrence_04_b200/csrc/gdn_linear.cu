@@ -8,7 +8,9 @@
 // "gdn_forward_batch", runs them as matrix-matrix products over a batch of
 // positions.
 //
-// Design (one 128 x BN output tile per CTA, BN = 256, 192 threads):
+// Design (one 128 x BN output tile per CTA, 192 threads; BN is 256, 128 or 64,
+// the widest whose grid still covers every SM once -- a decode-sized product
+// with few rows gets narrow tiles so that more SMs stream the weights):
 //   warp 0      one thread issues TMA loads of 128 x 64 tiles of x and W
 //               (128-byte swizzle) into an S-stage shared-memory ring;
 //   warp 1      owns the TMEM accumulator (BN fp32 columns x 128 lanes) and
@@ -27,10 +29,7 @@
 #include "gdn_tc.cuh"
 
 #ifndef GDN_LINEAR_BN
-#define GDN_LINEAR_BN 256        // output tile width (TMEM columns)
-#endif
-#ifndef GDN_LINEAR_STAGES
-#define GDN_LINEAR_STAGES (GDN_LINEAR_BN == 256 ? 4 : 6)
+#define GDN_LINEAR_BN 0          // 0: choose the tile width per launch; else force 64/128/256
 #endif
 
 namespace gdn {
@@ -39,11 +38,13 @@ namespace {
 
 constexpr int kBM = 128;
 constexpr int kBK = 64;                  // 64 bf16 = one 128-byte swizzle row
-constexpr int kStages = GDN_LINEAR_STAGES;
 constexpr int kThreads = 192;
 
+// Shared-memory ring per tile width: 4 stages of 48 KB (BN = 256), 6 of
+// 32 KB (128), 8 of 24 KB (64).
 template <int BN>
 struct LinearSmem {
+    static constexpr int kStages = BN == 256 ? 4 : (BN == 128 ? 6 : 8);
     static constexpr uint32_t kA = kBM * kBK * 2;
     static constexpr uint32_t kB = BN * kBK * 2;
     static constexpr uint32_t kStage = kA + kB;
@@ -56,6 +57,7 @@ linear_bf16_kernel(const __grid_constant__ CUtensorMap tmap_x,
                    const __grid_constant__ CUtensorMap tmap_w, float* __restrict__ y, int M,
                    int N, int K, uint32_t* __restrict__ status) {
     using L = LinearSmem<BN>;
+    constexpr int kStages = L::kStages;
     extern __shared__ uint8_t smem_raw[];
     __shared__ __align__(8) uint64_t full[kStages];
     __shared__ __align__(8) uint64_t empty[kStages];
@@ -241,7 +243,17 @@ cudaError_t launch_bn(const LinearArgs& a, cudaStream_t stream) {
 
 cudaError_t launch_linear_bf16(const LinearArgs& a, cudaStream_t stream) {
     if (a.M == 0 || a.N == 0) return cudaSuccess;
-    return launch_bn<GDN_LINEAR_BN>(a, stream);
+    int bn = GDN_LINEAR_BN;
+    if (bn == 0) {
+        const int64_t sms = device_sm_count();
+        const int64_t m_tiles = (a.M + kBM - 1) / kBM;
+        bn = 64;
+        if (m_tiles * ((a.N + 255) / 256) >= sms) bn = 256;
+        else if (m_tiles * ((a.N + 127) / 128) >= sms) bn = 128;
+    }
+    if (bn == 256) return launch_bn<256>(a, stream);
+    if (bn == 128) return launch_bn<128>(a, stream);
+    return launch_bn<64>(a, stream);
 }
 
 }  // namespace gdn

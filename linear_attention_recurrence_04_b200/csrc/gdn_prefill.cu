@@ -40,6 +40,12 @@
 //    folded back into W (W *= s, s = 1); a decay that underflows to zero
 //    folds to W = 0 exactly as step 1 would. W * s is written back at the
 //    end, so the stored state has its ordinary meaning.
+//  * KDA ("Module linear_core", entry "kda_forward_batch"; the published Kimi
+//    Delta Attention update) is the same pipeline with a log-decay per key
+//    channel, g [B][T][Hv][dk]: one head per warp (NH = 1), no running scale,
+//    and each stage also carries alpha = exp(g) and alpha * k, converted in
+//    place from the staged g one stage ahead. Per element and position:
+//    W *= alpha_t, W += delta k_t, o += W q_t, a += W (alpha_{t+1} k_{t+1}).
 #include "gdn_common.cuh"
 #include "gdn_internal.h"
 
@@ -75,13 +81,20 @@ static_assert(kMaxWarps <= kUnitsPerHead, "a run must span at most two groups");
 static_assert(kStages >= 3, "the pipeline reads one stage ahead");
 static_assert(kLPR == 4 || kLPR == 8, "4 or 8 lanes per row");
 
-// Shared-memory image of one stage.
-template <int NH>
+// Shared-memory image of one stage. kCh (per-channel decay): alpha holds g
+// as copied, then exp(g); ka holds exp(g) * k. Without kCh both are stubs.
+template <int NH, bool kCh>
 struct Stage {
     float kq[kMaxGroups][kTS][2][kDk];          // [group][pos][k|q][col]
     float v[kMaxGroups][kTS][NH][kMaxRows];     // rows [row_lo, row_lo + rows) of the group
     float bg[kMaxGroups][kTS][NH][2];           // beta, gate
+    float alpha[kCh ? kMaxGroups : 1][kCh ? kTS : 1][NH][kCh ? kDk : 4];
+    float ka[kCh ? kMaxGroups : 1][kCh ? kTS : 1][NH][kCh ? kDk : 4];
 };
+
+// Stages in flight: the per-channel stages are larger, so three of them.
+template <bool kCh>
+constexpr int stages_for() { return kCh ? 3 : kStages; }
 
 // One group of the CTA's run: (sequence b, key head g, head group grp) and the
 // rows of it that the run covers.
@@ -125,15 +138,18 @@ __device__ __forceinline__ float2 hi2(float4 v) { return make_float2(v.z, v.w); 
 __device__ __forceinline__ float4 ld_s4(const float* p) { return *reinterpret_cast<const float4*>(p); }
 __device__ __forceinline__ float sum4(float2 a, float2 b) { return (a.x + a.y) + (b.x + b.y); }
 
-template <int NH>
+template <int NH, bool kCh>
 __global__ void __launch_bounds__(32 * kMaxWarps, 1)
 prefill_kernel(float* __restrict__ state, const float* __restrict__ q,
                const float* __restrict__ k, const float* __restrict__ v,
                const float* __restrict__ beta, const float* __restrict__ gate,
                float* __restrict__ out, int64_t T, int Hk, int Hv, int units_lo, int n_big,
                int64_t qk_stride, int64_t v_stride, int64_t bg_stride) {
+    static_assert(!kCh || NH == 1, "per-channel decay runs one head per warp");
+    constexpr int S = stages_for<kCh>();
+    using StageT = Stage<NH, kCh>;
     extern __shared__ __align__(16) unsigned char smem_raw[];
-    Stage<NH>* stages = reinterpret_cast<Stage<NH>*>(smem_raw);
+    StageT* stages = reinterpret_cast<StageT*>(smem_raw);
     __shared__ Group grp_of[kMaxGroups];
 
     const int tid = threadIdx.x;
@@ -169,7 +185,7 @@ prefill_kernel(float* __restrict__ state, const float* __restrict__ q,
 
     // ---- stage loader: every thread issues a share of the copies; positions
     //      at or past T are zero-filled ------------------------------------
-    auto load_stage = [&](int64_t t0, Stage<NH>& st) {
+    auto load_stage = [&](int64_t t0, StageT& st) {
 #pragma unroll
         for (int gi = 0; gi < kMaxGroups; ++gi) {
             if (gi >= n_groups) break;
@@ -206,11 +222,41 @@ prefill_kernel(float* __restrict__ state, const float* __restrict__ q,
                 const int tp = (idx >> 1) / NH;
                 const int64_t t = t0 + tp;
                 float* dst = &st.bg[gi][tp][n][which];
-                if (t < T) {
+                if (t < T && !(kCh && which)) {
                     const int h = G.g + (G.grp * NH + n) * Hk;
                     cp_async4(dst, (which ? gate : beta) + (G.b * T + t) * bg_stride + h);
                 } else {
                     *dst = 0.0f;
+                }
+            }
+            if constexpr (kCh) {                                         // g rows
+                for (int idx = tid; idx < kTS * NH * 32; idx += nthreads) {
+                    const int chunk = idx & 31;
+                    const int n = (idx >> 5) % NH;
+                    const int tp = (idx >> 5) / NH;
+                    const int64_t t = t0 + tp;
+                    float* dst = &st.alpha[gi][tp][n][chunk * 4];
+                    if (t < T) {
+                        const int h = G.g + (G.grp * NH + n) * Hk;
+                        cp_async16(dst, gate + ((G.b * T + t) * Hv + h) * kDk + chunk * 4);
+                    } else {
+                        *reinterpret_cast<float4*>(dst) = make_float4(0.f, 0.f, 0.f, 0.f);
+                    }
+                }
+            }
+        }
+    };
+    // kCh: alpha = exp(g) and ka = alpha * k of a landed stage, in place.
+    auto convert_stage = [&](StageT& st) {
+        if constexpr (kCh) {
+            for (int gi2 = 0; gi2 < n_groups; ++gi2) {
+                for (int idx = tid; idx < kTS * NH * kDk; idx += nthreads) {
+                    const int col = idx % kDk;
+                    const int n = (idx / kDk) % NH;
+                    const int tp = idx / (kDk * NH);
+                    const float a = expf(st.alpha[gi2][tp][n][col]);
+                    st.alpha[gi2][tp][n][col] = a;
+                    st.ka[gi2][tp][n][col] = a * st.kq[gi2][tp][0][col];
                 }
             }
         }
@@ -236,7 +282,7 @@ prefill_kernel(float* __restrict__ state, const float* __restrict__ q,
     // Prologue: request the first S - 1 stages, then load the state rows.
     const int64_t n_stages = (T + kTS - 1) / kTS;
 #pragma unroll
-    for (int s2 = 0; s2 < kStages - 1; ++s2) {
+    for (int s2 = 0; s2 < S - 1; ++s2) {
         if (s2 < n_stages) load_stage(static_cast<int64_t>(s2) * kTS, stages[s2]);
         cp_async_commit();
     }
@@ -261,21 +307,29 @@ prefill_kernel(float* __restrict__ state, const float* __restrict__ q,
     int64_t t_out = 0;
 
     for (int64_t s = 0; s < n_stages; ++s) {
-        cp_async_wait<kStages - 3>();       // this thread's copies of stages s, s+1 landed
+        cp_async_wait<S - 3>();             // this thread's copies of stages s, s+1 landed
         __syncthreads();                     // ... and everyone's; stage s-1 is consumed
         {
-            const int64_t nxt = s + kStages - 1;
-            if (nxt < n_stages) load_stage(nxt * kTS, stages[nxt % kStages]);
+            const int64_t nxt = s + S - 1;
+            if (nxt < n_stages) load_stage(nxt * kTS, stages[nxt % S]);
             cp_async_commit();
         }
+        if constexpr (kCh) {
+            // stage s+1 (and, first, stage 0) gets its decays before any warp
+            // reads its first key product for the next-position dot
+            if (s == 0) convert_stage(stages[0]);
+            if (s + 1 < n_stages) convert_stage(stages[(s + 1) % S]);
+            __syncthreads();
+        }
         if (!active) continue;
-        const Stage<NH>& st = stages[s % kStages];
-        const Stage<NH>& st_next = stages[(s + 1) % kStages];
+        const StageT& st = stages[s % S];
+        const StageT& st_next = stages[(s + 1) % S];
         const int64_t t0 = s * kTS;
         const int tp_end = (T - t0) < kTS ? static_cast<int>(T - t0) : kTS;
 
         // decays of this stage, one per lane: lane tp + kTS n holds exp(gate)
-        const float e_lane = (lane < kTS * NH) ? expf(st.bg[gi][lane % kTS][lane / kTS][1]) : 1.0f;
+        const float e_lane =
+            (!kCh && lane < kTS * NH) ? expf(st.bg[gi][lane % kTS][lane / kTS][1]) : 1.0f;
 
         if (s == 0) {
             // first key dot: a = W.k_0
@@ -283,9 +337,10 @@ prefill_kernel(float* __restrict__ state, const float* __restrict__ q,
             for (int n = 0; n < NH; ++n) a_lo[n] = a_hi[n] = make_float2(0.f, 0.f);
 #pragma unroll
             for (int i = 0; i < kChunks; ++i) {
-                const float4 kv = ld_s4(&st.kq[gi][0][0][chunk_col(i, c)]);
 #pragma unroll
                 for (int n = 0; n < NH; ++n) {
+                    const float4 kv = kCh ? ld_s4(&st.ka[gi][0][n][chunk_col(i, c)])
+                                          : ld_s4(&st.kq[gi][0][0][chunk_col(i, c)]);
                     a_lo[n] = fma2(lo2(w[n][i]), lo2(kv), a_lo[n]);
                     a_hi[n] = fma2(hi2(w[n][i]), hi2(kv), a_hi[n]);
                 }
@@ -317,7 +372,7 @@ prefill_kernel(float* __restrict__ state, const float* __restrict__ q,
             float s_new[NH];
 #pragma unroll
             for (int n = 0; n < NH; ++n) {
-                const float e = __shfl_sync(kFull, e_lane, tp + kTS * n);
+                const float e = kCh ? 1.0f : __shfl_sync(kFull, e_lane, tp + kTS * n);
                 s_new[n] = sc[n] * e;
                 const float sk = s_new[n] * A[n];
                 cf[n] = (st.v[gi][tp][n][vrow] - sk) * st.bg[gi][tp][n][0];   // delta
@@ -345,6 +400,9 @@ prefill_kernel(float* __restrict__ state, const float* __restrict__ q,
             // (c) one pass: step 4 for t, then W.q_t (step 5) and W.k_{t+1}
             const bool has_next = t + 1 < T;
             const float* kn = (tp + 1 < kTS) ? &st.kq[gi][tp + 1][0][0] : &st_next.kq[gi][0][0][0];
+            const float* kan = nullptr;     // decay * key of the next position (kCh)
+            if constexpr (kCh)
+                kan = (tp + 1 < kTS) ? &st.ka[gi][tp + 1][0][0] : &st_next.ka[gi][0][0][0];
 #pragma unroll
             for (int n = 0; n < NH; ++n) {
                 o_lo[n] = o_hi[n] = a_lo[n] = a_hi[n] = make_float2(0.f, 0.f);
@@ -357,13 +415,25 @@ prefill_kernel(float* __restrict__ state, const float* __restrict__ q,
 #pragma unroll
                 for (int n = 0; n < NH; ++n) {
                     const float2 cf2 = make_float2(cf[n], cf[n]);
-                    const float2 lo = fma2(cf2, lo2(kv), lo2(w[n][i]));
-                    const float2 hi = fma2(cf2, hi2(kv), hi2(w[n][i]));
+                    float4 wv = w[n][i];
+                    float4 next = nv;
+                    if constexpr (kCh) {
+                        // step 1 per channel, and the next key with its decay
+                        const float4 al = ld_s4(&st.alpha[gi][tp][n][chunk_col(i, c)]);
+                        const float2 z2 = make_float2(0.f, 0.f);
+                        const float2 dl = fma2(lo2(wv), lo2(al), z2);
+                        const float2 dh = fma2(hi2(wv), hi2(al), z2);
+                        wv = make_float4(dl.x, dl.y, dh.x, dh.y);
+                        next = has_next ? ld_s4(kan + n * kDk + chunk_col(i, c))
+                                        : make_float4(0.f, 0.f, 0.f, 0.f);
+                    }
+                    const float2 lo = fma2(cf2, lo2(kv), lo2(wv));
+                    const float2 hi = fma2(cf2, hi2(kv), hi2(wv));
                     w[n][i] = make_float4(lo.x, lo.y, hi.x, hi.y);
                     o_lo[n] = fma2(lo, lo2(qv), o_lo[n]);
                     o_hi[n] = fma2(hi, hi2(qv), o_hi[n]);
-                    a_lo[n] = fma2(lo, lo2(nv), a_lo[n]);
-                    a_hi[n] = fma2(hi, hi2(nv), a_hi[n]);
+                    a_lo[n] = fma2(lo, lo2(next), a_lo[n]);
+                    a_hi[n] = fma2(hi, hi2(next), a_hi[n]);
                 }
             }
             out_pending = true;
@@ -396,7 +466,7 @@ prefill_kernel(float* __restrict__ state, const float* __restrict__ q,
     }
 }
 
-template <int NH>
+template <int NH, bool kCh>
 cudaError_t launch_nh(const PrefillArgs& a, cudaStream_t stream) {
     const int G = a.Hv / a.Hk;
     const int64_t n_units = a.B * a.Hk * (G / NH) * kUnitsPerHead;
@@ -408,15 +478,15 @@ cudaError_t launch_nh(const PrefillArgs& a, cudaStream_t stream) {
     const int units_lo = static_cast<int>(n_units / grid);
     const int n_big = static_cast<int>(n_units % grid);
     const int warps = units_lo + (n_big > 0 ? 1 : 0);
-    const size_t smem = sizeof(Stage<NH>) * kStages;
-    cudaError_t err = cudaFuncSetAttribute(prefill_kernel<NH>,
+    const size_t smem = sizeof(Stage<NH, kCh>) * stages_for<kCh>();
+    cudaError_t err = cudaFuncSetAttribute(prefill_kernel<NH, kCh>,
                                            cudaFuncAttributeMaxDynamicSharedMemorySize,
                                            static_cast<int>(smem));
     if (err != cudaSuccess) return err;
     const int64_t qk_stride = a.qk_stride ? a.qk_stride : static_cast<int64_t>(a.Hk) * kDk;
     const int64_t v_stride = a.v_stride ? a.v_stride : static_cast<int64_t>(a.Hv) * kDv;
     const int64_t bg_stride = a.bg_stride ? a.bg_stride : a.Hv;
-    prefill_kernel<NH><<<static_cast<unsigned>(grid), 32 * warps, smem, stream>>>(
+    prefill_kernel<NH, kCh><<<static_cast<unsigned>(grid), 32 * warps, smem, stream>>>(
         a.state, a.q, a.k, a.v, a.beta, a.gate, a.out, a.T, a.Hk, a.Hv, units_lo, n_big,
         qk_stride, v_stride, bg_stride);
     return cudaGetLastError();
@@ -426,7 +496,11 @@ cudaError_t launch_nh(const PrefillArgs& a, cudaStream_t stream) {
 
 cudaError_t launch_prefill(const PrefillArgs& a, cudaStream_t stream) {
     const int G = a.Hv / a.Hk;
-    return (G % 2 == 0) ? launch_nh<2>(a, stream) : launch_nh<1>(a, stream);
+    return (G % 2 == 0) ? launch_nh<2, false>(a, stream) : launch_nh<1, false>(a, stream);
+}
+
+cudaError_t launch_kda_prefill(const PrefillArgs& a, cudaStream_t stream) {
+    return launch_nh<1, true>(a, stream);
 }
 
 }  // namespace gdn

@@ -1,0 +1,181 @@
+// gdn_short_conv.cu -- the LFM2 short-convolution mixer over T positions of B
+// sequences ("Module linear_core", struct "ShortConvWeights" and entries
+// "short_conv_forward", "short_conv_forward_batch", "short_conv_pair").
+//
+// The mixer has no recurrent state: its only state is the causal conv ring,
+// the last K-1 gated inputs of every channel. Per position t and channel d:
+//   (bg | cg | xv) = W_in h_t            rows [0,D) | [D,2D) | [2D,3D)
+//   u_t[d]  = bg[d] * xv[d]              (the gated input the ring keeps)
+//   conv[d] = sum_tau conv_w[d][tau] * window[tau],
+//             window = (u_{t-K+1} .. u_t), entries before position 0 from the ring
+//   y_t[d]  = cg[d] * conv[d]            (rounded to bf16, out_proj's input type)
+//   out_t   = W_out y_t
+//
+// Pipeline (each stage a kernel of this library, on the caller's stream):
+//   1. proj = hidden . W_in^T          (tcgen05 GEMM, fp32 out, workspace)
+//   2. gate_conv: every (sequence, 32-position tile, channel) in parallel --
+//      u is a function of proj alone, so no position waits for another; each
+//      thread rebuilds its K-1 halo from proj (or from the ring before
+//      position 0) with the same fp32 product, so every tile sees exactly the
+//      ring values a position-by-position walk would hold;
+//   3. ring_update: per (sequence, channel), the ring after position
+//      n_commit - 1 goes to conv_ring and, for the two-position verify, the
+//      ring after the last position to scratch_ring (a separate kernel so
+//      that no tile of step 2 can read a ring slot that was already replaced);
+//   4. out = y . W_out^T              (tcgen05 GEMM).
+// u is rounded to fp32 (the ring's type) before it enters the window; the
+// window sum and the output gate run in double, and y is rounded once.
+#include <cuda_bf16.h>
+
+#include "gdn_common.cuh"
+#include "gdn_internal.h"
+
+namespace gdn {
+
+namespace {
+
+constexpr int kConvTile = 32;            // positions per thread in gate_conv
+
+template <int K>
+__global__ void __launch_bounds__(256)
+short_conv_gate_kernel(const float* __restrict__ proj, const float* __restrict__ ring,
+                       const float* __restrict__ conv_w, __nv_bfloat16* __restrict__ y,
+                       int64_t B, int64_t T, int64_t D) {
+    const int64_t d = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+    if (d >= D) return;
+    const int64_t b = blockIdx.z;
+    const int64_t t0 = static_cast<int64_t>(blockIdx.y) * kConvTile;
+    const int64_t D3 = 3 * D;
+    const float* pb = proj + b * T * D3 + d;          // (b, t, d) at pb[t * D3]
+    double w[K];
+#pragma unroll
+    for (int tau = 0; tau < K; ++tau) w[tau] = conv_w[d * K + tau];
+    // window[0..K-2] = u at positions t0-K+1 .. t0-1
+    float win[K - 1];
+#pragma unroll
+    for (int i = 0; i < K - 1; ++i) {
+        const int64_t t = t0 - (K - 1) + i;
+        if (t >= 0) {
+            win[i] = __fmul_rn(pb[t * D3], pb[t * D3 + 2 * D]);
+        } else {
+            // slot K-1+t of the ring holds u at position t (t = -1 newest)
+            win[i] = ring[(b * (K - 1) + (K - 1 + t)) * D + d];
+        }
+    }
+    const int n = static_cast<int>((T - t0) < kConvTile ? (T - t0) : kConvTile);
+    // all loads of the tile first, then the sequential window walk
+    float bg[kConvTile], cg[kConvTile], xv[kConvTile];
+#pragma unroll
+    for (int i = 0; i < kConvTile; ++i) {
+        if (i < n) {
+            const float* p = pb + (t0 + i) * D3;
+            bg[i] = p[0];
+            cg[i] = p[D];
+            xv[i] = p[2 * D];
+        }
+    }
+    __nv_bfloat16* yb = y + (b * T + t0) * D + d;
+#pragma unroll
+    for (int i = 0; i < kConvTile; ++i) {
+        if (i < n) {
+            const float u = __fmul_rn(bg[i], xv[i]);
+            double conv = 0.0;
+#pragma unroll
+            for (int tau = 0; tau < K - 1; ++tau) conv = fma(w[tau], static_cast<double>(win[tau]), conv);
+            conv = fma(w[K - 1], static_cast<double>(u), conv);
+            yb[static_cast<int64_t>(i) * D] = __double2bfloat16(static_cast<double>(cg[i]) * conv);
+#pragma unroll
+            for (int tau = 0; tau < K - 2; ++tau) win[tau] = win[tau + 1];
+            win[K - 2] = u;
+        }
+    }
+}
+
+// For one (sequence, channel): the ring after position n_commit - 1 (its K-1
+// newest gated inputs) into `ring`, and the ring after position T - 1 into
+// `scratch_ring` when one is given; gated inputs come from proj and, before
+// position 0, from the old ring. Every read precedes every write of the
+// thread's own column, so the update is safe in place.
+template <int K>
+__global__ void __launch_bounds__(256)
+short_conv_ring_kernel(const float* __restrict__ proj, float* ring, float* scratch_ring,
+                       int64_t B, int64_t T, int64_t D, int64_t n_commit) {
+    const int64_t idx = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+    if (idx >= B * D) return;
+    const int64_t b = idx / D;
+    const int64_t d = idx - b * D;
+    const int64_t D3 = 3 * D;
+    const float* pb = proj + b * T * D3 + d;
+    float* rg = ring + b * (K - 1) * D + d;
+    float old[K - 1];
+#pragma unroll
+    for (int i = 0; i < K - 1; ++i) old[i] = rg[i * D];
+    // gated input at position t; slot K-1+t of the old ring before position 0
+    auto u_at = [&](int64_t t) -> float {
+        return t >= 0 ? __fmul_rn(pb[t * D3], pb[t * D3 + 2 * D]) : old[K - 1 + t];
+    };
+    float committed[K - 1], tentative[K - 1];
+#pragma unroll
+    for (int i = 0; i < K - 1; ++i) {
+        committed[i] = u_at(n_commit - (K - 1) + i);
+        tentative[i] = u_at(T - (K - 1) + i);
+    }
+#pragma unroll
+    for (int i = 0; i < K - 1; ++i) rg[i * D] = committed[i];
+    if (scratch_ring) {
+        float* sg = scratch_ring + b * (K - 1) * D + d;
+#pragma unroll
+        for (int i = 0; i < K - 1; ++i) sg[i * D] = tentative[i];
+    }
+}
+
+size_t align256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
+
+template <int K>
+cudaError_t launch_conv(const ShortConvArgs& a, float* proj, __nv_bfloat16* y,
+                        cudaStream_t stream) {
+    const dim3 grid(static_cast<unsigned>((a.D + 255) / 256),
+                    static_cast<unsigned>((a.T + kConvTile - 1) / kConvTile),
+                    static_cast<unsigned>(a.B));
+    short_conv_gate_kernel<K><<<grid, 256, 0, stream>>>(proj, a.conv_ring, a.conv_w, y, a.B,
+                                                        a.T, a.D);
+    cudaError_t err = cudaGetLastError();
+    if (err != cudaSuccess) return err;
+    const int64_t n = a.B * a.D;
+    short_conv_ring_kernel<K><<<static_cast<unsigned>((n + 255) / 256), 256, 0, stream>>>(
+        proj, a.conv_ring, a.scratch_ring, a.B, a.T, a.D, a.n_commit);
+    return cudaGetLastError();
+}
+
+}  // namespace
+
+ShortConvLayout short_conv_layout(int64_t B, int64_t T, int64_t D) {
+    const int64_t BT = B * T;
+    ShortConvLayout L;
+    L.proj = 0;
+    L.y = align256(static_cast<size_t>(BT) * 3 * D * 4);
+    L.total = align256(L.y + static_cast<size_t>(BT) * D * 2);
+    return L;
+}
+
+cudaError_t launch_short_conv(const ShortConvArgs& a, cudaStream_t stream) {
+    const int64_t BT = a.B * a.T;
+    if (BT == 0) return cudaSuccess;
+    const ShortConvLayout L = short_conv_layout(a.B, a.T, a.D);
+    char* ws = static_cast<char*>(a.workspace);
+    float* proj = reinterpret_cast<float*>(ws + L.proj);
+    __nv_bfloat16* y = reinterpret_cast<__nv_bfloat16*>(ws + L.y);
+    cudaError_t err = launch_linear_bf16(LinearArgs{a.hidden, a.w_in, proj, BT, 3 * a.D, a.D,
+                                                    a.status}, stream);
+    if (err != cudaSuccess) return err;
+    switch (a.K) {
+        case 2: err = launch_conv<2>(a, proj, y, stream); break;
+        case 3: err = launch_conv<3>(a, proj, y, stream); break;
+        case 4: err = launch_conv<4>(a, proj, y, stream); break;
+        default: return cudaErrorInvalidValue;
+    }
+    if (err != cudaSuccess) return err;
+    return launch_linear_bf16(LinearArgs{y, a.w_out, a.out, BT, a.D, a.D, a.status}, stream);
+}
+
+}  // namespace gdn

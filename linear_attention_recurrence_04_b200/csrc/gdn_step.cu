@@ -15,6 +15,11 @@
 // once in each direction per token. Warps walk row groups with a grid-stride
 // loop over a persistent grid of (SMs x resident CTAs), prefetching the next
 // group's rows while the current group computes.
+//
+// The same kernel with a decay per key channel is the KDA core ("Module
+// linear_core", entry "kda_forward"; the published Kimi Delta Attention
+// update): step 1 becomes M[j][i] *= exp(g[i]), g [.., Hv, dk], so each lane
+// scales its four columns by their own factors; steps 2-5 are unchanged.
 #include "gdn_common.cuh"
 #include "gdn_internal.h"
 
@@ -57,7 +62,9 @@ __device__ __forceinline__ void load_rows(float4 (&m)[R], const float* state, Ro
 }
 
 // Steps 1-5 on R rows held in registers; writes the rows and R outputs.
-template <int R>
+// kChannelDecay: gate holds a log-decay per key channel ([head][dk]) instead
+// of one per head.
+template <int R, bool kChannelDecay>
 __device__ __forceinline__ void update_rows(float4 (&m)[R], float* __restrict__ state,
                                             const float* __restrict__ q,
                                             const float* __restrict__ k,
@@ -71,7 +78,14 @@ __device__ __forceinline__ void update_rows(float4 (&m)[R], float* __restrict__ 
     const int64_t key = (lb * Hk + (h % Hk)) * kDk + lane * 4;
     const float4 k4 = ld_ro4(k + key);
     const float4 q4 = ld_ro4(q + key);
-    const float decay = expf(gate[t.head]);
+    float4 decay;
+    if constexpr (kChannelDecay) {
+        const float4 g4 = ld_ro4(gate + t.head * kDk + lane * 4);
+        decay = make_float4(expf(g4.x), expf(g4.y), expf(g4.z), expf(g4.w));
+    } else {
+        const float e = expf(gate[t.head]);
+        decay = make_float4(e, e, e, e);
+    }
     const float bt = beta[t.head];
     const int64_t vrow = t.head * kDv + t.row0;
     const float v_lane = lane < R ? v[vrow + lane] : 0.0f;
@@ -81,7 +95,7 @@ __device__ __forceinline__ void update_rows(float4 (&m)[R], float* __restrict__ 
     for (int r = 0; r < R; ++r) {
         float4 x = m[r];
         // step 1: decay
-        x.x *= decay; x.y *= decay; x.z *= decay; x.w *= decay;
+        x.x *= decay.x; x.y *= decay.y; x.z *= decay.z; x.w *= decay.w;
         // step 2: sk = M[j].k on the decayed row
         const float sk = warp_sum(dot4(x, k4));
         // step 3: delta
@@ -99,7 +113,7 @@ __device__ __forceinline__ void update_rows(float4 (&m)[R], float* __restrict__ 
     if (lane < R) out[vrow + lane] = o_lane;
 }
 
-template <int R>
+template <int R, bool kChannelDecay>
 __global__ void __launch_bounds__(GDN_STEP_THREADS)
 step_kernel(float* __restrict__ state, const float* __restrict__ q, const float* __restrict__ k,
             const float* __restrict__ v, const float* __restrict__ beta,
@@ -118,21 +132,20 @@ step_kernel(float* __restrict__ state, const float* __restrict__ q, const float*
         float4 nxt[R];
         const bool more = task + stride < n_tasks;
         if (more) load_rows<R>(nxt, state, decode_task<R>(task + stride), lane);
-        update_rows<R>(m, state, q, k, v, beta, gate, out, cur, Hk, Hv, lane);
+        update_rows<R, kChannelDecay>(m, state, q, k, v, beta, gate, out, cur, Hk, Hv, lane);
         if (more) {
 #pragma unroll
             for (int r = 0; r < R; ++r) m[r] = nxt[r];
         }
 #else
-        update_rows<R>(m, state, q, k, v, beta, gate, out, cur, Hk, Hv, lane);
+        update_rows<R, kChannelDecay>(m, state, q, k, v, beta, gate, out, cur, Hk, Hv, lane);
         if (task + stride < n_tasks) load_rows<R>(m, state, decode_task<R>(task + stride), lane);
 #endif
     }
 }
 
-}  // namespace
-
-cudaError_t launch_step(const StepArgs& a, cudaStream_t stream) {
+template <bool kChannelDecay>
+cudaError_t launch_rows(const StepArgs& a, cudaStream_t stream) {
     constexpr int R = GDN_STEP_ROWS;
     static_assert(kDv % R == 0 && R <= 32, "rows per task must divide dv");
     const int64_t n_tasks = a.n_heads * (kDv / R);
@@ -141,14 +154,25 @@ cudaError_t launch_step(const StepArgs& a, cudaStream_t stream) {
     constexpr int warps_per_cta = threads / 32;
     const int64_t needed = (n_tasks + warps_per_cta - 1) / warps_per_cta;
     int per_sm = 0;
-    cudaError_t err = resident_ctas_per_sm(reinterpret_cast<const void*>(&step_kernel<R>),
-                                           threads, &per_sm);
+    cudaError_t err = resident_ctas_per_sm(
+        reinterpret_cast<const void*>(&step_kernel<R, kChannelDecay>), threads, &per_sm);
     if (err != cudaSuccess) return err;
     const int64_t resident = static_cast<int64_t>(device_sm_count()) * per_sm;
     const int grid = static_cast<int>(needed < resident ? needed : resident);
-    step_kernel<R><<<grid, threads, 0, stream>>>(a.state, a.q, a.k, a.v, a.beta, a.gate, a.out,
-                                                 n_tasks, a.Hk, a.Hv);
+    step_kernel<R, kChannelDecay><<<grid, threads, 0, stream>>>(a.state, a.q, a.k, a.v, a.beta,
+                                                                a.gate, a.out, n_tasks, a.Hk,
+                                                                a.Hv);
     return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_step(const StepArgs& a, cudaStream_t stream) {
+    return launch_rows<false>(a, stream);
+}
+
+cudaError_t launch_kda_step(const StepArgs& a, cudaStream_t stream) {
+    return launch_rows<true>(a, stream);
 }
 
 }  // namespace gdn

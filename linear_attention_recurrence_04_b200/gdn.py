@@ -30,7 +30,9 @@ STATUS = {
 # Every symbol that include/gdn.h declares.
 EXPORTS = ("gdn_status_string", "gdn_last_error", "gdn_step", "gdn_prefill", "gdn_layer_decode",
            "gdn_layer_pair", "gdn_linear_bf16", "gdn_forward_batch_workspace_size",
-           "gdn_forward_batch", "gdn_forward_batch_noalloc")
+           "gdn_forward_batch", "gdn_forward_batch_noalloc", "gdn_short_conv_workspace_size",
+           "gdn_short_conv_forward_batch", "gdn_short_conv_forward", "gdn_short_conv_pair",
+           "gdn_kda_step", "gdn_kda_prefill")
 
 
 class GdnError(RuntimeError):
@@ -82,6 +84,18 @@ def load_library(path: Optional[str] = None) -> ctypes.CDLL:
     lib.gdn_forward_batch_noalloc.restype = ctypes.c_int
     lib.gdn_forward_batch_noalloc.argtypes = ([_VP] * 10 + [_F32, _F32] + [_VP, _VP]
                                               + [_I64] * 8 + [_VP, _VP])
+    for name in ("gdn_kda_step", "gdn_kda_prefill"):
+        getattr(lib, name).restype = ctypes.c_int
+        getattr(lib, name).argtypes = [_VP] * 7 + [_I64] * 6 + [_VP]
+    lib.gdn_short_conv_workspace_size.restype = ctypes.c_size_t
+    lib.gdn_short_conv_workspace_size.argtypes = [_I64] * 3
+    lib.gdn_short_conv_forward_batch.restype = ctypes.c_int
+    lib.gdn_short_conv_forward_batch.argtypes = ([_VP] * 7 + [ctypes.c_size_t] + [_I64] * 4
+                                                 + [_VP, _VP])
+    lib.gdn_short_conv_forward.restype = ctypes.c_int
+    lib.gdn_short_conv_forward.argtypes = [_VP] * 7 + [ctypes.c_size_t] + [_I64] * 3 + [_VP, _VP]
+    lib.gdn_short_conv_pair.restype = ctypes.c_int
+    lib.gdn_short_conv_pair.argtypes = [_VP] * 8 + [ctypes.c_size_t] + [_I64] * 3 + [_VP, _VP]
     if path is None:
         _lib = lib
     return lib
@@ -344,4 +358,137 @@ def forward_batch_noalloc(hidden, w_qkv, w_z, w_ba, w_out, conv_ring, conv_w, A_
                _ptr(dt_bias), _ptr(norm_w), float(l2_eps), float(norm_eps), _ptr(state),
                _ptr(out), B, T, D, Hk, Hv, 128, 128, K, sp, _stream(device, stream))
     _raise_on("gdn_forward_batch_noalloc", st)
+    return out
+
+
+# -- KDA core ----------------------------------------------------------------
+
+def kda_step(state, q, k, v, beta, g, out=None, *, stream=None):
+    """One KDA decode token: state [L,B,Hv,128,128] (updated in place), q/k
+    [L,B,Hk,128], v [L,B,Hv,128], beta [L,B,Hv], g [L,B,Hv,128] (log-decay per
+    key channel). Returns out [L,B,Hv,128]."""
+    if state.dim() != 5:
+        raise ValueError("state must be [L, B, Hv, dv, dk]")
+    L, B, Hv, dv, dk = state.shape
+    Hk = q.shape[2]
+    if out is None:
+        out = torch.empty((L, B, Hv, dv), dtype=torch.float32, device=state.device)
+    names = ("state", "q", "k", "v", "beta", "g", "out")
+    tensors = (state, q, k, v, beta, g, out)
+    device = _dev(tensors, names)
+    expect = dict(q=(L, B, Hk, dk), k=(L, B, Hk, dk), v=(L, B, Hv, dv), beta=(L, B, Hv),
+                  g=(L, B, Hv, dk), out=(L, B, Hv, dv))
+    for n, t in zip(names[1:], tensors[1:]):
+        if tuple(t.shape) != expect[n]:
+            raise ValueError(f"{n} has shape {tuple(t.shape)}, expected {expect[n]}")
+    st = _call(device, load_library().gdn_kda_step, *(_ptr(t) for t in tensors), L, B, Hk, Hv,
+               dk, dv, _stream(device, stream))
+    _raise_on("gdn_kda_step", st)
+    return out
+
+
+def kda_prefill(state, q, k, v, beta, g, out=None, *, stream=None):
+    """T KDA positions in order: state [B,Hv,128,128] (initial -> final, in
+    place), q/k [B,T,Hk,128], v [B,T,Hv,128], beta [B,T,Hv], g [B,T,Hv,128].
+    Returns out [B,T,Hv,128]."""
+    if state.dim() != 4:
+        raise ValueError("state must be [B, Hv, dv, dk]")
+    B, Hv, dv, dk = state.shape
+    T, Hk = q.shape[1], q.shape[2]
+    if out is None:
+        out = torch.empty((B, T, Hv, dv), dtype=torch.float32, device=state.device)
+    names = ("state", "q", "k", "v", "beta", "g", "out")
+    tensors = (state, q, k, v, beta, g, out)
+    device = _dev(tensors, names)
+    expect = dict(q=(B, T, Hk, dk), k=(B, T, Hk, dk), v=(B, T, Hv, dv), beta=(B, T, Hv),
+                  g=(B, T, Hv, dk), out=(B, T, Hv, dv))
+    for n, t in zip(names[1:], tensors[1:]):
+        if tuple(t.shape) != expect[n]:
+            raise ValueError(f"{n} has shape {tuple(t.shape)}, expected {expect[n]}")
+    st = _call(device, load_library().gdn_kda_prefill, *(_ptr(t) for t in tensors), B, T, Hk,
+               Hv, dk, dv, _stream(device, stream))
+    _raise_on("gdn_kda_prefill", st)
+    return out
+
+
+# -- LFM2 short-convolution mixer ------------------------------------------
+
+def short_conv_workspace_size(B: int, T: int, D: int) -> int:
+    return int(load_library().gdn_short_conv_workspace_size(B, T, D))
+
+
+def _short_conv_args(hidden, w_in, w_out, conv_ring, conv_w, out, workspace, T, npos_out):
+    """Checks shared by the short-conv calls; returns (device, B, D, K, out, workspace)."""
+    B, D = hidden.shape[0], hidden.shape[-1]
+    K = conv_w.shape[1]
+    for n, t in (("hidden", hidden), ("w_in", w_in), ("w_out", w_out)):
+        if t.dtype is not torch.bfloat16 or not t.is_cuda or not t.is_contiguous():
+            raise TypeError(f"{n} must be a contiguous bfloat16 CUDA tensor")
+    if out is None:
+        out = torch.empty(npos_out, dtype=torch.float32, device=hidden.device)
+    device = _dev((conv_ring, conv_w, out), ("conv_ring", "conv_w", "out"))
+    if hidden.device != device or w_in.device != device or w_out.device != device:
+        raise ValueError("all tensors must be on one device")
+    expect = dict(w_in=(3 * D, D), w_out=(D, D), conv_ring=(B, K - 1, D), conv_w=(D, K),
+                  out=tuple(npos_out))
+    for n, t in (("w_in", w_in), ("w_out", w_out), ("conv_ring", conv_ring), ("conv_w", conv_w),
+                 ("out", out)):
+        if tuple(t.shape) != expect[n]:
+            raise ValueError(f"{n} has shape {tuple(t.shape)}, expected {expect[n]}")
+    need = short_conv_workspace_size(B, T, D)
+    if workspace is None:
+        workspace = torch.empty(max(need, 1), dtype=torch.uint8, device=device)
+    if workspace.dtype is not torch.uint8 or workspace.device != device:
+        raise TypeError("workspace must be a uint8 tensor on the same device")
+    return device, B, D, K, out, workspace
+
+
+def short_conv_forward_batch(hidden, w_in, w_out, conv_ring, conv_w, out=None, workspace=None,
+                             *, status=None, stream=None):
+    """T positions of the short-conv mixer: hidden [B, T, D] bf16, w_in
+    [3D, D] and w_out [D, D] bf16, conv_ring [B, K-1, D] (updated in place),
+    conv_w [D, K]. Returns out [B, T, D] fp32."""
+    B, T, D = hidden.shape
+    device, B, D, K, out, workspace = _short_conv_args(hidden, w_in, w_out, conv_ring, conv_w,
+                                                       out, workspace, T, (B, T, D))
+    sp = status.data_ptr() if status is not None else 0
+    st = _call(device, load_library().gdn_short_conv_forward_batch, _ptr(hidden), _ptr(w_in),
+               _ptr(w_out), _ptr(conv_ring), _ptr(conv_w), _ptr(out), workspace.data_ptr(),
+               workspace.numel(), B, T, D, K, sp, _stream(device, stream))
+    _raise_on("gdn_short_conv_forward_batch", st)
+    return out
+
+
+def short_conv_forward(hidden, w_in, w_out, conv_ring, conv_w, out=None, workspace=None, *,
+                       status=None, stream=None):
+    """One position per sequence: hidden [B, D] bf16. Returns out [B, D] fp32."""
+    B, D = hidden.shape
+    device, B, D, K, out, workspace = _short_conv_args(hidden, w_in, w_out, conv_ring, conv_w,
+                                                       out, workspace, 1, (B, D))
+    sp = status.data_ptr() if status is not None else 0
+    st = _call(device, load_library().gdn_short_conv_forward, _ptr(hidden), _ptr(w_in),
+               _ptr(w_out), _ptr(conv_ring), _ptr(conv_w), _ptr(out), workspace.data_ptr(),
+               workspace.numel(), B, D, K, sp, _stream(device, stream))
+    _raise_on("gdn_short_conv_forward", st)
+    return out
+
+
+def short_conv_pair(hidden, w_in, w_out, conv_ring, scratch_ring, conv_w, out=None,
+                    workspace=None, *, status=None, stream=None):
+    """Two-position verify: hidden [B, 2, D] bf16; conv_ring receives the ring
+    after position 0, scratch_ring [B, K-1, D] the ring after position 1.
+    Returns out [B, 2, D] fp32."""
+    B, two, D = hidden.shape
+    if two != 2:
+        raise ValueError("hidden must be [B, 2, D]")
+    device, B, D, K, out, workspace = _short_conv_args(hidden, w_in, w_out, conv_ring, conv_w,
+                                                       out, workspace, 2, (B, 2, D))
+    _dev((scratch_ring,), ("scratch_ring",))
+    if tuple(scratch_ring.shape) != tuple(conv_ring.shape) or scratch_ring.device != device:
+        raise ValueError("scratch_ring must match conv_ring in shape and device")
+    sp = status.data_ptr() if status is not None else 0
+    st = _call(device, load_library().gdn_short_conv_pair, _ptr(hidden), _ptr(w_in),
+               _ptr(w_out), _ptr(conv_ring), _ptr(scratch_ring), _ptr(conv_w), _ptr(out),
+               workspace.data_ptr(), workspace.numel(), B, D, K, sp, _stream(device, stream))
+    _raise_on("gdn_short_conv_pair", st)
     return out

@@ -105,6 +105,31 @@ def layer_inputs(B: int, *, Hk: int = HK, Hv: int = HV, dk: int = DK, dv: int = 
     )
 
 
+def kda_decode_inputs(L: int, B: int, *, seed: int = 1013, g_low: float = -1.0,
+                      **kw) -> Dict[str, np.ndarray]:
+    """decode_inputs plus a log-decay per key channel g ~ U(g_low, 0)
+    [L, B, Hv, dk] (the KDA core's gate; the scalar gate is dropped)."""
+    d = decode_inputs(L, B, seed=seed, **kw)
+    r = np.random.default_rng([seed, 1])
+    L_, B_, Hv = d["beta"].shape
+    dk = d["q"].shape[-1]
+    d["g"] = _f32(r.uniform(g_low, 0.0, (L_, B_, Hv, dk)))
+    del d["gate"]
+    return d
+
+
+def kda_prefill_inputs(B: int, T: int, *, seed: int = 1014, g_low: float = -0.5,
+                       **kw) -> Dict[str, np.ndarray]:
+    """prefill_inputs plus g ~ U(g_low, 0) [B, T, Hv, dk] per key channel."""
+    d = prefill_inputs(B, T, seed=seed, **kw)
+    r = np.random.default_rng([seed, 1])
+    B_, T_, Hv = d["beta"].shape
+    dk = d["q"].shape[-1]
+    d["g"] = _f32(r.uniform(g_low, 0.0, (B_, T_, Hv, dk)))
+    del d["gate"]
+    return d
+
+
 def to_bf16_values(x: np.ndarray) -> np.ndarray:
     """float32 array of the nearest bfloat16 values (round half to even), a
     dtype conversion so the GPU (as bf16) and the oracle (as fp64) read the
@@ -142,11 +167,28 @@ def forward_inputs(B: int, T: int, *, D: int = 2048, Hk: int = HK, Hv: int = HV,
     )
 
 
+def short_conv_inputs(B: int, T: int, *, D: int = 2048, K: int = 3, seed: int = 1008,
+                      ring_std: float = 1.0) -> Dict[str, np.ndarray]:
+    """The LFM2 short-conv mixer over T positions: hidden ~ N(0, 1),
+    w_in ~ N(0, 1/D) [3D, D], w_out ~ N(0, 1/D) [D, D] (all bf16-representable
+    float32), conv ring of gated inputs ~ N(0, ring_std^2) [B, K-1, D], conv
+    weight ~ N(0, 0.25^2) [D, K]."""
+    r = np.random.default_rng(seed)
+    bf = lambda a: to_bf16_values(a.astype(np.float32))
+    return dict(
+        hidden=bf(r.normal(size=(B, T, D))),
+        w_in=bf(r.normal(0.0, D ** -0.5, (3 * D, D))),
+        w_out=bf(r.normal(0.0, D ** -0.5, (D, D))),
+        conv_ring=_f32(r.normal(0.0, ring_std, (B, K - 1, D))),
+        conv_w=_f32(r.normal(0.0, 0.25, (D, K))),
+    )
+
+
 @dataclass(frozen=True)
 class Workload:
     """One named synthetic workload and how to draw it."""
     name: str
-    kind: str                     # "step" | "prefill" | "layer"
+    kind: str                     # "step" | "prefill" | "layer" | "forward" | "short_conv" | "kda_*"
     sizes: Dict[str, int] = field(default_factory=dict)
     seed: int = 1000
 
@@ -159,6 +201,13 @@ class Workload:
             return layer_inputs(self.sizes["B"], seed=self.seed)
         if self.kind == "forward":
             return forward_inputs(self.sizes["B"], self.sizes["T"], seed=self.seed)
+        if self.kind == "kda_step":
+            return kda_decode_inputs(self.sizes["L"], self.sizes["B"], seed=self.seed)
+        if self.kind == "kda_prefill":
+            return kda_prefill_inputs(self.sizes["B"], self.sizes["T"], seed=self.seed)
+        if self.kind == "short_conv":
+            return short_conv_inputs(self.sizes["B"], self.sizes["T"], D=self.sizes["D"],
+                                     K=self.sizes["K"], seed=self.seed)
         raise ValueError(self.kind)
 
 
@@ -174,3 +223,22 @@ WORKLOADS = {
 
 # The batched layer forward with dense projections (D = 2048 hidden).
 FORWARD_WORKLOAD = Workload("forward_batch_b4_t4096", "forward", dict(B=4, T=4096), seed=1007)
+
+# The KDA core at the recurrent layer's geometry: one decode token for 64
+# sequences, and 4 x 4096 positions from a zero state.
+KDA_WORKLOADS = {
+    "kda_decode_b64": Workload("kda_decode_b64", "kda_step", dict(L=1, B=64), seed=1013),
+    "kda_prefill_b4_t4096": Workload("kda_prefill_b4_t4096", "kda_prefill", dict(B=4, T=4096),
+                                     seed=1014),
+}
+
+# The LFM2 short-conv mixer at the same hidden size: one decode position for 64
+# sequences, the two-position verify for 64 sequences, and 4 x 4096 positions.
+SHORT_CONV_WORKLOADS = {
+    "short_conv_decode_b64": Workload("short_conv_decode_b64", "short_conv",
+                                      dict(B=64, T=1, D=2048, K=3), seed=1008),
+    "short_conv_pair_b64": Workload("short_conv_pair_b64", "short_conv",
+                                    dict(B=64, T=2, D=2048, K=3), seed=1012),
+    "short_conv_batch_b4_t4096": Workload("short_conv_batch_b4_t4096", "short_conv",
+                                          dict(B=4, T=4096, D=2048, K=3), seed=1009),
+}

@@ -198,3 +198,21 @@ def test_short_conv_argument_checks(lib):
                                    fake(20), ws2, 2, 64, 3, 0, None) == NULL
     assert lib.gdn_short_conv_pair(fake(1), fake(2), fake(3), fake(4), fake(4), fake(5), fake(13),
                                    fake(20), ws2, 2, 64, 3, 0, None) == ALIAS
+
+
+def test_kda_argument_checks(lib):
+    def step(g=fake(6), L=1, dk=128):
+        return lib.gdn_kda_step(fake(1), fake(2), fake(3), fake(4), fake(5), g, fake(7), L, 2, 16,
+                                32, dk, 128, None)
+    assert step(dk=64) == UNSUP
+    assert step(L=-1) == SHAPE
+    assert step(g=0) == NULL
+    assert step(g=fake(6) + 4) == ALIGN          # g is read 16 bytes at a time
+    assert step(g=fake(1) + 16) == ALIAS         # g inside the state (updated in place)
+
+    def pre(g=fake(6), T=3):
+        return lib.gdn_kda_prefill(fake(1), fake(2), fake(3), fake(4), fake(5), g, fake(7), 2, T,
+                                   16, 32, 128, 128, None)
+    assert pre(T=-2) == SHAPE
+    assert pre(g=0) == NULL
+    assert pre(g=fake(6) + 8) == ALIGN

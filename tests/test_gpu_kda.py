@@ -1,0 +1,103 @@
+"""The KDA core (gdn_kda_step, gdn_kda_prefill) on the GPU against the fp64
+oracle, through the C ABI, with the library tolerance: |gpu - ref| <= 1e-5
+everywhere and relative 1e-4 where |ref| > 1e-3."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from linear_attention_recurrence_04_b200 import gdn, inputs
+from parity import assert_parity
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def o():
+    return oracle.load()
+
+
+def to_dev(d):
+    return {k: torch.from_numpy(np.ascontiguousarray(v)).cuda() for k, v in d.items()}
+
+
+def gpu_step(d):
+    t = to_dev(d)
+    out = gdn.kda_step(t["state"], t["q"], t["k"], t["v"], t["beta"], t["g"])
+    torch.cuda.synchronize()
+    return t["state"].cpu().numpy(), out.cpu().numpy()
+
+
+def gpu_prefill(d):
+    t = to_dev(d)
+    out = gdn.kda_prefill(t["state"], t["q"], t["k"], t["v"], t["beta"], t["g"])
+    torch.cuda.synchronize()
+    return t["state"].cpu().numpy(), out.cpu().numpy()
+
+
+@pytest.mark.parametrize("L,B,Hk,Hv", [(1, 3, 16, 32), (2, 2, 4, 4), (1, 1, 2, 6)])
+def test_kda_step_parity(o, L, B, Hk, Hv):
+    d = inputs.kda_decode_inputs(L, B, Hk=Hk, Hv=Hv, seed=1500 + 10 * L + B)
+    st_ref, out_ref = o.kda_step(d["state"], d["q"], d["k"], d["v"], d["beta"], d["g"])
+    st, out = gpu_step(d)
+    assert_parity(out, out_ref, "kda step out")
+    assert_parity(st, st_ref, "kda step state")
+
+
+def test_kda_step_decode_b64_full_size(o):
+    """The benchmark's decode launch, every unit against the oracle."""
+    d = inputs.KDA_WORKLOADS["kda_decode_b64"].draw()
+    st_ref, out_ref = o.kda_step(d["state"], d["q"], d["k"], d["v"], d["beta"], d["g"])
+    st, out = gpu_step(d)
+    assert_parity(out, out_ref, "kda decode_b64 out")
+    assert_parity(st, st_ref, "kda decode_b64 state")
+
+
+def test_kda_uniform_decay_equals_gdn_step():
+    """With the same log-decay on every channel the KDA update is the scalar
+    one of gdn_step."""
+    d = inputs.kda_decode_inputs(1, 4, seed=1510)
+    d["g"] = np.repeat(d["g"][..., :1], d["g"].shape[-1], axis=-1).copy()
+    st_k, out_k = gpu_step(d)
+    t = to_dev(d)
+    out_g = gdn.step(t["state"], t["q"], t["k"], t["v"], t["beta"], t["g"][..., 0].contiguous())
+    torch.cuda.synchronize()
+    assert_parity(out_k, out_g.cpu().numpy().astype(np.float64), "uniform decay out")
+    assert_parity(st_k, t["state"].cpu().numpy().astype(np.float64), "uniform decay state")
+
+
+@pytest.mark.parametrize("B,T,Hk,Hv,std", [(2, 37, 16, 32, 0.05), (1, 16, 4, 4, 0.0),
+                                           (3, 9, 2, 6, 0.05), (1, 1, 16, 32, 0.05),
+                                           (1, 49, 8, 8, 0.05)])
+def test_kda_prefill_parity(o, B, T, Hk, Hv, std):
+    d = inputs.kda_prefill_inputs(B, T, Hk=Hk, Hv=Hv, seed=1600 + T, state_std=std)
+    st_ref, out_ref = o.kda_prefill(d["state"], d["q"], d["k"], d["v"], d["beta"], d["g"])
+    st, out = gpu_prefill(d)
+    assert_parity(out, out_ref, "kda prefill out")
+    assert_parity(st, st_ref, "kda prefill state")
+
+
+def test_kda_prefill_one_position_equals_step():
+    d = inputs.kda_prefill_inputs(3, 1, seed=1620, state_std=0.05)
+    st_p, out_p = gpu_prefill(d)
+    s = {"state": d["state"][None]}
+    for n in ("q", "k", "v", "beta", "g"):
+        s[n] = d[n][:, 0][None]
+    st_s, out_s = gpu_step(s)
+    assert_parity(out_p[:, 0], out_s[0].astype(np.float64), "T=1 out vs kda step")
+    assert_parity(st_p, st_s[0].astype(np.float64), "T=1 state vs kda step")
+
+
+def test_kda_prefill_b4_t4096_full_size_sampled(o):
+    """The benchmark's 4 x 4096-position launch: two (sequence, value head)
+    units over all positions and their final states against the oracle."""
+    d = inputs.KDA_WORKLOADS["kda_prefill_b4_t4096"].draw()
+    st, out = gpu_prefill(d)
+    Hv = d["state"].shape[1]
+    units = [0, 3 * Hv + Hv - 1]
+    st_ref, out_ref = o.kda_prefill(d["state"], d["q"], d["k"], d["v"], d["beta"], d["g"],
+                                    units=units)
+    for u in units:
+        b, h = divmod(u, Hv)
+        assert_parity(out[b, :, h], out_ref[b, :, h], f"kda prefill b{b} h{h} out")
+        assert_parity(st[b, h], st_ref[b, h], f"kda prefill b{b} h{h} state")
