@@ -61,6 +61,9 @@
 #ifndef GDN_PREFILL_FMA2
 #define GDN_PREFILL_FMA2 1         // packed f32x2 FMAs for the per-element work
 #endif
+#ifndef GDN_PREFILL_NH
+#define GDN_PREFILL_NH 0           // value heads per warp: 0 = 2 when Hv/Hk is even, else 1
+#endif
 
 namespace gdn {
 
@@ -496,7 +499,8 @@ cudaError_t launch_nh(const PrefillArgs& a, cudaStream_t stream) {
 
 cudaError_t launch_prefill(const PrefillArgs& a, cudaStream_t stream) {
     const int G = a.Hv / a.Hk;
-    return (G % 2 == 0) ? launch_nh<2, false>(a, stream) : launch_nh<1, false>(a, stream);
+    const bool two = GDN_PREFILL_NH == 0 ? (G % 2 == 0) : (GDN_PREFILL_NH == 2 && G % 2 == 0);
+    return two ? launch_nh<2, false>(a, stream) : launch_nh<1, false>(a, stream);
 }
 
 cudaError_t launch_kda_prefill(const PrefillArgs& a, cudaStream_t stream) {
