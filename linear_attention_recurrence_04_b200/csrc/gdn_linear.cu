@@ -8,20 +8,26 @@
 // "gdn_forward_batch", runs them as matrix-matrix products over a batch of
 // positions.
 //
-// Design (one 128 x BN output tile per CTA, 192 threads; BN is 256, 128 or 64,
-// the widest whose grid still covers every SM once -- a decode-sized product
-// with few rows gets narrow tiles so that more SMs stream the weights):
+// Design (persistent: one CTA per SM walks 128 x BN output tiles, 192
+// threads; BN is 256, 128 or 64, the widest whose tile count still covers
+// every SM once -- a decode-sized product with few rows gets narrow tiles so
+// that more SMs stream the weights):
 //   warp 0      one thread issues TMA loads of 128 x 64 tiles of x and W
-//               (128-byte swizzle) into an S-stage shared-memory ring;
-//   warp 1      owns the TMEM accumulator (BN fp32 columns x 128 lanes) and
-//               one thread issues tcgen05.mma (bf16, M = 128, N = BN, K = 16)
-//               per 32-byte K step; a tcgen05.commit per stage frees the slot
-//               back to the producer, a final one signals the epilogue;
-//   warps 2-5   read the accumulator with tcgen05.ld (each warp its TMEM lane
-//               quarter, i.e. 32 rows) and store fp32 rows.
-// Tiles past M, N or K are zero-filled by TMA and masked on store. Every
-// mbarrier wait gives up after 2 s, ORs an error bit into the caller's
-// status word (if given), lets in-flight copies land and frees TMEM.
+//               (128-byte swizzle) into an S-stage shared-memory ring that
+//               runs on across tiles;
+//   warp 1      owns two TMEM accumulators (2 x BN fp32 columns x 128 lanes);
+//               one thread issues tcgen05.mma (bf16, M = 128, N = BN,
+//               K = 16) per 32-byte K step into the tile's accumulator; a
+//               tcgen05.commit per stage frees the slot back to the producer,
+//               one per tile hands the accumulator to the epilogue;
+//   warps 2-5   read an accumulator with tcgen05.ld (each warp its TMEM lane
+//               quarter, i.e. 32 rows), store fp32 rows, and release it: while
+//               they drain tile i, the MMAs of tile i+1 fill the other one.
+// Tiles past M, N or K are zero-filled by TMA and masked on store. An
+// element's K order never depends on the tile width, the tile's place or M,
+// so a row's result is the same in any batch. Every mbarrier wait gives up
+// after 2 s, ORs an error bit into the caller's status word (if given), lets
+// in-flight copies land and frees TMEM.
 #include <cuda.h>
 
 #include "gdn_common.cuh"
@@ -61,9 +67,11 @@ linear_bf16_kernel(const __grid_constant__ CUtensorMap tmap_x,
     extern __shared__ uint8_t smem_raw[];
     __shared__ __align__(8) uint64_t full[kStages];
     __shared__ __align__(8) uint64_t empty[kStages];
-    __shared__ __align__(8) uint64_t done;
+    __shared__ __align__(8) uint64_t acc_full[2];      // MMA -> epilogue, per accumulator
+    __shared__ __align__(8) uint64_t acc_empty[2];     // epilogue -> MMA
     __shared__ uint32_t tmem_slot;
-    __shared__ int issued, consumed, failed;
+    __shared__ int64_t issued, consumed;
+    __shared__ int failed;
 
     // 1024-byte aligned base for the swizzled tiles
     const uint32_t raw = tc::smem_u32(smem_raw);
@@ -71,90 +79,118 @@ linear_bf16_kernel(const __grid_constant__ CUtensorMap tmap_x,
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
-    const int m0 = blockIdx.y * kBM;
-    const int n0 = blockIdx.x * BN;
     const int n_kt = (K + kBK - 1) / kBK;
+    const int tiles_n = (N + BN - 1) / BN;
+    const int n_tiles = tiles_n * ((M + kBM - 1) / kBM);
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < kStages; ++s) {
             tc::mbar_init(tc::smem_u32(&full[s]), 1);
             tc::mbar_init(tc::smem_u32(&empty[s]), 1);
         }
-        tc::mbar_init(tc::smem_u32(&done), 1);
+        for (int a = 0; a < 2; ++a) {
+            tc::mbar_init(tc::smem_u32(&acc_full[a]), 1);
+            tc::mbar_init(tc::smem_u32(&acc_empty[a]), 4);   // one arrival per epilogue warp
+        }
         tc::fence_mbar_init();
         issued = 0;
         consumed = 0;
         failed = 0;
     }
     if (warp == 1) {
-        tc::tmem_alloc(tc::smem_u32(&tmem_slot), BN);
+        tc::tmem_alloc(tc::smem_u32(&tmem_slot), 2 * BN);
         tc::tmem_relinquish();
     }
     tc::tc_fence_before();
     __syncthreads();
     tc::tc_fence_after();
     const uint32_t tmem = tmem_slot;
+    volatile int* vfailed = &failed;
 
     if (warp == 0 && lane == 0) {
-        // ---- producer --------------------------------------------------------
+        // ---- producer: k-steps of every tile, through the stage ring --------
         tc::prefetch_tmap(&tmap_x);
         tc::prefetch_tmap(&tmap_w);
-        for (int kt = 0; kt < n_kt; ++kt) {
-            const int s = kt % kStages;
-            const uint32_t ph = (kt / kStages) & 1;
-            if (!tc::mbar_wait(tc::smem_u32(&empty[s]), ph ^ 1)) {
-                if (status) atomicOr(status, tc::kTimeoutProducer);
-                atomicExch(&failed, 1);
-                break;
+        int64_t g = 0;                                     // k-steps issued so far
+        for (int tile = blockIdx.x; tile < n_tiles && !*vfailed; tile += gridDim.x) {
+            const int m0 = (tile / tiles_n) * kBM;
+            const int n0 = (tile % tiles_n) * BN;
+            for (int kt = 0; kt < n_kt; ++kt, ++g) {
+                const int s = static_cast<int>(g % kStages);
+                const uint32_t ph = static_cast<uint32_t>(g / kStages) & 1u;
+                if (!tc::mbar_wait(tc::smem_u32(&empty[s]), ph ^ 1)) {
+                    if (status) atomicOr(status, tc::kTimeoutProducer);
+                    atomicExch(&failed, 1);
+                    break;
+                }
+                if (*vfailed) break;
+                const uint32_t a = base + s * L::kStage;
+                tc::mbar_arrive_expect_tx(tc::smem_u32(&full[s]), L::kStage);
+                tc::tma_load_2d(a, &tmap_x, tc::smem_u32(&full[s]), kt * kBK, m0);
+                tc::tma_load_2d(a + L::kA, &tmap_w, tc::smem_u32(&full[s]), kt * kBK, n0);
+                issued = g + 1;
             }
-            if (*reinterpret_cast<volatile int*>(&failed)) break;
-            const uint32_t a = base + s * L::kStage;
-            tc::mbar_arrive_expect_tx(tc::smem_u32(&full[s]), L::kStage);
-            tc::tma_load_2d(a, &tmap_x, tc::smem_u32(&full[s]), kt * kBK, m0);
-            tc::tma_load_2d(a + L::kA, &tmap_w, tc::smem_u32(&full[s]), kt * kBK, n0);
-            issued = kt + 1;
         }
     } else if (warp == 1 && lane == 0) {
-        // ---- MMA issuer ------------------------------------------------------
+        // ---- MMA issuer: tile li accumulates into accumulator li & 1 -------
         const uint32_t idesc = tc::idesc_bf16_f32(kBM, BN);
+        int64_t g = 0;
         bool ok = true;
-        for (int kt = 0; kt < n_kt; ++kt) {
-            const int s = kt % kStages;
-            const uint32_t ph = (kt / kStages) & 1;
-            if (!tc::mbar_wait(tc::smem_u32(&full[s]), ph) ||
-                *reinterpret_cast<volatile int*>(&failed)) {
+        int li = 0;
+        for (int tile = blockIdx.x; ok && tile < n_tiles; tile += gridDim.x, ++li) {
+            const int acc = li & 1;
+            const uint32_t d = tmem + static_cast<uint32_t>(acc * BN);
+            if (!tc::mbar_wait(tc::smem_u32(&acc_empty[acc]), ((li >> 1) & 1) ^ 1) || *vfailed) {
                 if (status) atomicOr(status, tc::kTimeoutMma);
                 atomicExch(&failed, 1);
-                ok = false;
                 break;
             }
-            consumed = kt + 1;
             tc::tc_fence_after();
-            const uint32_t a = base + s * L::kStage;
-            const uint32_t b = a + L::kA;
+            for (int kt = 0; kt < n_kt; ++kt, ++g) {
+                const int s = static_cast<int>(g % kStages);
+                const uint32_t ph = static_cast<uint32_t>(g / kStages) & 1u;
+                if (!tc::mbar_wait(tc::smem_u32(&full[s]), ph) || *vfailed) {
+                    if (status) atomicOr(status, tc::kTimeoutMma);
+                    atomicExch(&failed, 1);
+                    ok = false;
+                    break;
+                }
+                consumed = g + 1;
+                tc::tc_fence_after();
+                const uint32_t a = base + s * L::kStage;
+                const uint32_t b = a + L::kA;
 #pragma unroll
-            for (int kk = 0; kk < kBK / 16; ++kk) {
-                tc::mma_bf16(tmem, tc::desc_k_sw128(a + kk * 32), tc::desc_k_sw128(b + kk * 32),
-                             idesc, (kt > 0 || kk > 0) ? 1u : 0u);
+                for (int kk = 0; kk < kBK / 16; ++kk) {
+                    tc::mma_bf16(d, tc::desc_k_sw128(a + kk * 32), tc::desc_k_sw128(b + kk * 32),
+                                 idesc, (kt > 0 || kk > 0) ? 1u : 0u);
+                }
+                tc::mma_commit(tc::smem_u32(&empty[s]));   // slot free once these MMAs finish
             }
-            tc::mma_commit(tc::smem_u32(&empty[s]));      // slot free once these MMAs finish
+            if (ok) tc::mma_commit(tc::smem_u32(&acc_full[acc]));   // accumulator complete
         }
-        if (ok) tc::mma_commit(tc::smem_u32(&done));     // accumulator complete
     } else if (warp >= 2) {
-        // ---- epilogue: TMEM -> registers -> global ---------------------------
+        // ---- epilogue: TMEM -> registers -> global, then release ------------
         const int quarter = warp & 3;                      // TMEM lanes 32 q .. 32 q + 31
-        if (!tc::mbar_wait(tc::smem_u32(&done), 0)) {
-            if (status) atomicOr(status, tc::kTimeoutEpilogue);
-            atomicExch(&failed, 1);
-        } else {
+        int li = 0;
+        for (int tile = blockIdx.x; tile < n_tiles; tile += gridDim.x, ++li) {
+            const int acc = li & 1;
+            if (!tc::mbar_wait(tc::smem_u32(&acc_full[acc]), (li >> 1) & 1) || *vfailed) {
+                if (status) atomicOr(status, tc::kTimeoutEpilogue);
+                atomicExch(&failed, 1);
+                break;
+            }
             tc::tc_fence_after();
+            const int m0 = (tile / tiles_n) * kBM;
+            const int n0 = (tile % tiles_n) * BN;
             const int row = m0 + quarter * 32 + lane;
             const bool row_ok = row < M;
             float* yrow = y + static_cast<int64_t>(row) * N;
+            const uint32_t src = tmem + static_cast<uint32_t>(acc * BN) +
+                                 (static_cast<uint32_t>(quarter * 32) << 16);
 #pragma unroll 1
             for (int c0 = 0; c0 < BN; c0 += 32) {
                 uint32_t r[32];
-                tc::tmem_ld_32x32b_x32(tmem + (static_cast<uint32_t>(quarter * 32) << 16) + c0, r);
+                tc::tmem_ld_32x32b_x32(src + c0, r);
                 tc::tmem_ld_wait();
                 const int col = n0 + c0;
                 if (!row_ok || col >= N) continue;
@@ -171,6 +207,10 @@ linear_bf16_kernel(const __grid_constant__ CUtensorMap tmap_x,
                         if (col + j < N) yrow[col + j] = __uint_as_float(r[j]);
                 }
             }
+            // every read of this accumulator has completed: hand it back
+            tc::tc_fence_before();
+            __syncwarp();
+            if (lane == 0) tc::mbar_arrive(tc::smem_u32(&acc_empty[acc]));
         }
     }
 
@@ -178,13 +218,14 @@ linear_bf16_kernel(const __grid_constant__ CUtensorMap tmap_x,
     // the shared memory goes away (bounded like every other wait).
     __syncthreads();
     if (threadIdx.x == 0 && failed) {
-        for (int kt = consumed; kt < issued; ++kt)
-            tc::mbar_wait(tc::smem_u32(&full[kt % kStages]), (kt / kStages) & 1);
+        for (int64_t g = consumed; g < issued; ++g)
+            tc::mbar_wait(tc::smem_u32(&full[g % kStages]),
+                          static_cast<uint32_t>(g / kStages) & 1u);
     }
     tc::tc_fence_before();
     __syncthreads();
     tc::tc_fence_after();
-    if (warp == 1) tc::tmem_dealloc(tmem, BN);
+    if (warp == 1) tc::tmem_dealloc(tmem, 2 * BN);
 }
 
 // cuTensorMapEncodeTiled through the runtime's driver entry point (no link
@@ -231,8 +272,10 @@ cudaError_t launch_bn(const LinearArgs& a, cudaStream_t stream) {
                                            cudaFuncAttributeMaxDynamicSharedMemorySize,
                                            static_cast<int>(smem));
     if (err != cudaSuccess) return err;
-    const dim3 grid(static_cast<unsigned>((a.N + BN - 1) / BN),
-                    static_cast<unsigned>((a.M + kBM - 1) / kBM));
+    const int64_t tiles = ((a.N + BN - 1) / BN) * ((a.M + kBM - 1) / kBM);
+    if (tiles > INT32_MAX) return cudaErrorInvalidValue;
+    const int64_t sms = device_sm_count();
+    const unsigned grid = static_cast<unsigned>(tiles < sms ? tiles : sms);
     linear_bf16_kernel<BN><<<grid, kThreads, smem, stream>>>(tx, tw, a.y, static_cast<int>(a.M),
                                                              static_cast<int>(a.N),
                                                              static_cast<int>(a.K), a.status);
