@@ -220,6 +220,8 @@ gdn_status gdn_linear_bf16(const void *x, const void *w, float *y, int64_t M, in
  *             entry do not matter and are undefined afterwards
  *   status    optional zero-initialised device word for timeout bits (see
  *             gdn_linear_bf16)
+ * Limits: B <= 65535, T <= 65535 * 32, B*T <= 65535 * 128 (GDN_ERR_OVERFLOW
+ * otherwise; the workspace size function returns 0).
  */
 size_t gdn_forward_batch_workspace_size(int64_t B, int64_t T, int64_t Hk, int64_t Hv,
                                         int64_t dk, int64_t dv);
@@ -242,7 +244,7 @@ gdn_status gdn_forward_batch(const void *hidden, const void *w_qkv, const void *
  *
  * The workspace is a 16 MiB array built into the library (held on every GPU
  * that loads the library until the process exits). B*T positions whose
- * gdn_forward_batch_workspace_size() exceeds 16 MiB (about 226 positions at
+ * gdn_forward_batch_workspace_size() exceeds 16 MiB (about 215 positions at
  * Hk = 16, Hv = 32, dk = dv = 128) are rejected with GDN_ERR_UNSUPPORTED and
  * a message; nothing is launched. The first call on a device looks up the
  * array's device address; make that call before any stream capture. Every
@@ -310,7 +312,8 @@ gdn_status gdn_kda_prefill(float *state, const float *q, const float *k, const f
  *             gdn_linear_bf16)
  * All pointers are device pointers, 16-byte aligned. conv_ring is updated in
  * place and may overlap nothing else; out may overlap no argument.
- * gdn_short_conv_workspace_size returns 0 for an invalid shape.
+ * Limits: B <= 65535, T <= 65535 * 32, B*T <= 65535 * 128 (GDN_ERR_OVERFLOW
+ * otherwise). gdn_short_conv_workspace_size returns 0 for an invalid shape.
  *
  * gdn_short_conv_forward_batch runs T positions in order; conv_ring ends as
  * the ring after position T-1 (T = 0 does nothing).

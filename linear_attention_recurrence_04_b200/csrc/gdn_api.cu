@@ -400,7 +400,7 @@ gdn_status gdn_linear_bf16(const void* x, const void* w, float* y, int64_t M, in
 size_t gdn_forward_batch_workspace_size(int64_t B, int64_t T, int64_t Hk, int64_t Hv,
                                         int64_t dk, int64_t dv) {
     if (B < 0 || T < 0 || Hk <= 0 || Hv <= 0 || Hv % Hk != 0 || dk != kDk || dv != kDv ||
-        Hv > (1 << 20) || B > (int64_t)65535 * 128 || T > (int64_t)65535 * 128 ||
+        Hv > (1 << 20) || B > 65535 || T > (int64_t)65535 * 32 ||
         B * T > (int64_t)65535 * 128)
         return 0;
     return forward_batch_layout(B, T, static_cast<int>(Hk), static_cast<int>(Hv)).total;
@@ -421,9 +421,11 @@ gdn_status gdn_forward_batch(const void* hidden, const void* w_qkv, const void* 
                                  fn, (long long)K);
     if (D == 0 || D % 8 != 0)
         return fail(GDN_ERR_UNSUPPORTED, "%s: D=%lld must be a positive multiple of 8", fn, (long long)D);
-    if (B > (int64_t)65535 * 128 || T > (int64_t)65535 * 128 || B * T > (int64_t)65535 * 128 ||
-        D > (1 << 24))
-        return fail(GDN_ERR_OVERFLOW, "%s: B*T=%lld or D too large", fn, (long long)(B * T));
+    // B*T rows of the projection GEMMs (M tiles of 128); the conv walks tiles
+    // of 32 positions in one grid dimension, and the sequences in another.
+    if (B > 65535 || T > (int64_t)65535 * 32 || B * T > (int64_t)65535 * 128 || D > (1 << 24))
+        return fail(GDN_ERR_OVERFLOW, "%s: B=%lld, T=%lld, B*T or D too large", fn, (long long)B,
+                    (long long)T);
     const int64_t BT = B * T;
     const int64_t C = 2 * Hk * dk + Hv * dv;
     const int64_t HD = Hv * dv;
@@ -459,7 +461,7 @@ gdn_status gdn_forward_batch(const void* hidden, const void* w_qkv, const void* 
 
 size_t gdn_short_conv_workspace_size(int64_t B, int64_t T, int64_t D) {
     if (B < 0 || T < 0 || D <= 0 || D % 8 != 0 || D > (1 << 24) || B > 65535 ||
-        T > (int64_t)65535 * 128 || B * T > (int64_t)65535 * 128)
+        T > (int64_t)65535 * 32 || B * T > (int64_t)65535 * 128)
         return 0;
     return short_conv_layout(B, T, D).total;
 }
@@ -482,9 +484,10 @@ gdn_status short_conv_call(const char* fn, const void* hidden, const void* w_in,
     if (D == 0 || D % 8 != 0)
         return fail(GDN_ERR_UNSUPPORTED, "%s: D=%lld must be a positive multiple of 8", fn,
                     (long long)D);
-    if (B > 65535 || T > (int64_t)65535 * 128 || B * T > (int64_t)65535 * 128 || D > (1 << 24))
-        return fail(GDN_ERR_OVERFLOW, "%s: B=%lld, B*T=%lld or D too large", fn, (long long)B,
-                    (long long)(B * T));
+    // the gate/conv kernel walks tiles of 32 positions in one grid dimension
+    if (B > 65535 || T > (int64_t)65535 * 32 || B * T > (int64_t)65535 * 128 || D > (1 << 24))
+        return fail(GDN_ERR_OVERFLOW, "%s: B=%lld, T=%lld, B*T or D too large", fn, (long long)B,
+                    (long long)T);
     const int64_t BT = B * T;
     if (BT == 0) { g_last_error[0] = '\0'; return GDN_OK; }
     const size_t need = short_conv_layout(B, T, D).total;

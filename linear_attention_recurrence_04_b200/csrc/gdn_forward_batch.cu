@@ -11,9 +11,9 @@
 // Pipeline (every stage a kernel of this library, on the caller's stream):
 //   1. mixed = hidden . W_qkv^T, z = hidden . W_z^T, ba = hidden . W_ba^T
 //      (tcgen05 GEMMs, bf16 in, fp32 out, into the workspace);
-//   2. conv_seq: per (sequence, channel) one thread walks the positions with
-//      the conv ring in registers, replacing mixed with SiLU(conv) in place
-//      and leaving the last K-1 raw inputs in the ring;
+//   2. conv: the positions in parallel tiles, in place after a halo pass that
+//      saves the K-1 raw inputs before each tile; mixed becomes SiLU(conv) and
+//      the ring ends as the last K-1 raw inputs;
 //   3. qk_norm_gates: per position, L2-normalise each q and k head in place
 //      and form beta = sigmoid(b), gate = -exp(A_log) softplus(a + dt_bias);
 //   4. the sequential prefill recurrence, reading q, k, v straight out of the
@@ -30,45 +30,70 @@ namespace gdn {
 
 namespace {
 
-// 2. causal depthwise conv over positions, SiLU, in place; ring update.
-constexpr int kConvThreads = 64;          // small blocks: B*C threads spread over every SM
+// 2. causal depthwise conv over positions, SiLU, in place, with the ring.
+//    Every output needs only the K-1 raw inputs before it, so the positions
+//    run in parallel in tiles of kConvTile; to convolve in place, the K-1 raw
+//    inputs before each tile are copied out first (conv_halo_kernel), then
+//    every (sequence, tile, channel) thread convolves its tile
+//    (conv_tile_kernel). The halo pass also forms the ring the call leaves
+//    behind (slot n_tiles), which the tile-0 thread of each channel writes
+//    after it has read the old ring -- the only thread that reads it.
+constexpr int kConvTile = 32;
 
-__global__ void __launch_bounds__(kConvThreads)
-conv_seq_kernel(float* __restrict__ act, float* __restrict__ ring,
-                const float* __restrict__ conv_w, int64_t B, int64_t T, int64_t C) {
-    const int64_t idx = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
-    if (idx >= B * C) return;
-    const int64_t b = idx / C;
-    const int64_t c = idx - b * C;
-    float* rg = ring + b * (kConvK - 1) * C + c;
-    float w0 = rg[0], w1 = rg[C], w2 = rg[2 * C];      // raw inputs, oldest first
+__global__ void __launch_bounds__(256)
+conv_halo_kernel(const float* __restrict__ act, const float* __restrict__ ring,
+                 float* __restrict__ halo, int64_t T, int64_t C, int n_tiles) {
+    const int64_t c = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+    if (c >= C) return;
+    const int j = blockIdx.y + 1;                        // tiles 1 .. n_tiles (n_tiles: the ring)
+    const int64_t b = blockIdx.z;
+    const int64_t end = j < n_tiles ? static_cast<int64_t>(j) * kConvTile : T;
+    float* dst = halo + ((b * (n_tiles + 1) + j) * (kConvK - 1)) * C + c;
+#pragma unroll
+    for (int i = 0; i < kConvK - 1; ++i) {
+        const int64_t t = end - (kConvK - 1) + i;        // raw input position (slot i)
+        dst[i * C] = t >= 0 ? act[(b * T + t) * C + c]
+                            : ring[(b * (kConvK - 1) + (kConvK - 1 + t)) * C + c];
+    }
+}
+
+__global__ void __launch_bounds__(256)
+conv_tile_kernel(float* __restrict__ act, float* __restrict__ ring,
+                 const float* __restrict__ halo, const float* __restrict__ conv_w, int64_t T,
+                 int64_t C, int n_tiles) {
+    const int64_t c = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+    if (c >= C) return;
+    const int j = blockIdx.y;
+    const int64_t b = blockIdx.z;
+    const int64_t t0 = static_cast<int64_t>(j) * kConvTile;
+    const int n = (T - t0) < kConvTile ? static_cast<int>(T - t0) : kConvTile;
     const float4 w = ld_ro4(conv_w + c * kConvK);
-    float* col = act + b * T * C + c;
-    // Positions in blocks of kSeqBlock: all loads of a block are issued
-    // before any of its (sequential) conv steps, so the memory latency is
-    // paid once per block rather than once per position, with enough bytes
-    // in flight per SM to keep HBM busy.
-    constexpr int kSeqBlock = 64;
-    for (int64_t t0 = 0; t0 < T; t0 += kSeqBlock) {
-        const int n = (T - t0) < kSeqBlock ? static_cast<int>(T - t0) : kSeqBlock;
-        float xs[kSeqBlock];
+    const float* hs = j == 0 ? ring + b * (kConvK - 1) * C + c
+                             : halo + ((b * (n_tiles + 1) + j) * (kConvK - 1)) * C + c;
+    float w0 = hs[0], w1 = hs[C], w2 = hs[2 * C];        // raw inputs, oldest first
+    float* col = act + (b * T + t0) * C + c;
+    float xs[kConvTile];
 #pragma unroll
-        for (int i = 0; i < kSeqBlock; ++i) xs[i] = (i < n) ? col[(t0 + i) * C] : 0.0f;
+    for (int i = 0; i < kConvTile; ++i) xs[i] = (i < n) ? col[static_cast<int64_t>(i) * C] : 0.0f;
 #pragma unroll
-        for (int i = 0; i < kSeqBlock; ++i) {
-            if (i < n) {
-                const float x = xs[i];
-                const float y = fmaf(w.w, x, fmaf(w.z, w2, fmaf(w.y, w1, w.x * w0)));
-                col[(t0 + i) * C] = siluf_acc(y);
-                w0 = w1;
-                w1 = w2;
-                w2 = x;
-            }
+    for (int i = 0; i < kConvTile; ++i) {
+        if (i < n) {
+            const float x = xs[i];
+            const float y = fmaf(w.w, x, fmaf(w.z, w2, fmaf(w.y, w1, w.x * w0)));
+            col[static_cast<int64_t>(i) * C] = siluf_acc(y);
+            w0 = w1;
+            w1 = w2;
+            w2 = x;
         }
     }
-    rg[0] = w0;
-    rg[C] = w1;
-    rg[2 * C] = w2;
+    if (j == 0) {            // the ring after the call (this thread read the old one above)
+        const float* nr = halo + ((b * (n_tiles + 1) + n_tiles) * (kConvK - 1)) * C + c;
+        float* rg = ring + b * (kConvK - 1) * C + c;
+        const float r0 = nr[0], r1 = nr[C], r2 = nr[2 * C];
+        rg[0] = r0;
+        rg[C] = r1;
+        rg[2 * C] = r2;
+    }
 }
 
 // 3. per position: L2-normalise the 2 Hk q/k heads (one warp each, in turn)
@@ -152,6 +177,8 @@ ForwardBatchLayout forward_batch_layout(int64_t B, int64_t T, int Hk, int Hv) {
     L.gate = off;  off = align256(off + BT * Hv * 4);
     L.o = off;     off = align256(off + BT * HD * 4);
     L.y = off;     off = align256(off + BT * HD * 2);
+    const int64_t n_tiles = (T + kConvTile - 1) / kConvTile;
+    L.halo = off;  off = align256(off + B * (n_tiles + 1) * (kConvK - 1) * C * 4);
     L.total = off;
     return L;
 }
@@ -170,6 +197,7 @@ cudaError_t launch_forward_batch(const ForwardBatchArgs& a, cudaStream_t stream)
     float* gate = reinterpret_cast<float*>(ws + L.gate);
     float* o = reinterpret_cast<float*>(ws + L.o);
     __nv_bfloat16* y = reinterpret_cast<__nv_bfloat16*>(ws + L.y);
+    float* halo = reinterpret_cast<float*>(ws + L.halo);
 
     // 1. input projections
     cudaError_t err;
@@ -180,12 +208,17 @@ cudaError_t launch_forward_batch(const ForwardBatchArgs& a, cudaStream_t stream)
     if ((err = launch_linear_bf16(LinearArgs{a.hidden, a.w_ba, ba, BT, 2 * a.Hv, a.D, a.status},
                                   stream)))
         return err;
-    // 2. conv over positions with the ring, SiLU
+    // 2. conv over positions with the ring, SiLU (halo pass, then in place)
     {
-        const int64_t n = a.B * C;
-        conv_seq_kernel<<<static_cast<unsigned>((n + kConvThreads - 1) / kConvThreads),
-                          kConvThreads, 0, stream>>>(
-            act, a.conv_ring, a.conv_w, a.B, a.T, C);
+        const int n_tiles = static_cast<int>((a.T + kConvTile - 1) / kConvTile);
+        const unsigned cblocks = static_cast<unsigned>((C + 255) / 256);
+        conv_halo_kernel<<<dim3(cblocks, static_cast<unsigned>(n_tiles),
+                                static_cast<unsigned>(a.B)), 256, 0, stream>>>(
+            act, a.conv_ring, halo, a.T, C, n_tiles);
+        if ((err = cudaGetLastError())) return err;
+        conv_tile_kernel<<<dim3(cblocks, static_cast<unsigned>(n_tiles),
+                                static_cast<unsigned>(a.B)), 256, 0, stream>>>(
+            act, a.conv_ring, halo, a.conv_w, a.T, C, n_tiles);
         if ((err = cudaGetLastError())) return err;
     }
     // 3. q/k L2 norm, beta and gate

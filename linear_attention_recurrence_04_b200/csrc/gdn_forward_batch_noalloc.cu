@@ -32,7 +32,7 @@
 #include "gdn_common.cuh"
 #include "gdn_internal.h"
 
-// The built-in scratch: 16 MiB, enough for about 226 positions of the
+// The built-in scratch: 16 MiB, enough for about 215 positions of the
 // pages' geometry (Hk = 16, Hv = 32, dk = dv = 128).
 static constexpr size_t kStaticScratchBytes = static_cast<size_t>(16) << 20;
 static __device__ __align__(256) unsigned char g_forward_scratch[kStaticScratchBytes];

@@ -96,7 +96,7 @@ struct ForwardBatchArgs {
 
 // Byte offsets of the forward-batch intermediates inside the workspace.
 struct ForwardBatchLayout {
-    size_t act, z, ba, beta, gate, o, y, total;
+    size_t act, z, ba, beta, gate, o, y, halo, total;
 };
 ForwardBatchLayout forward_batch_layout(int64_t B, int64_t T, int Hk, int Hv);
 

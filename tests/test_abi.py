@@ -216,3 +216,14 @@ def test_kda_argument_checks(lib):
     assert pre(T=-2) == SHAPE
     assert pre(g=0) == NULL
     assert pre(g=fake(6) + 8) == ALIGN
+
+
+def test_tile_grid_limits(lib):
+    """The conv kernels walk tiles of 32 positions in one grid dimension, so
+    T above 65535 * 32 is refused before any launch."""
+    T = 65535 * 32 + 1
+    assert lib.gdn_forward_batch_workspace_size(1, T, 16, 32, 128, 128) == 0
+    assert lib.gdn_short_conv_workspace_size(1, T, 64) == 0
+    assert lib.gdn_forward_batch_workspace_size(1, T - 1, 16, 32, 128, 128) > 0
+    assert lib.gdn_short_conv_forward_batch(fake(1), fake(2), fake(3), fake(4), fake(5), fake(13),
+                                            fake(20), 1 << 40, 1, T, 64, 3, 0, None) == OVERFLOW
