@@ -14,7 +14,9 @@ the roofline of the step kernel against the measured HBM copy bandwidth, an
 end-to-end figure through the C ABI with the per-step inputs copied from
 pinned host memory and the output copied back, NVML clock samples taken
 during the timed region, the fp64 CPU oracle timed on this host as a
-reported baseline, and (N = 1) the other four workloads measured the same way.
+reported baseline, and (N = 1) the other workloads (36-layer and B = 1 decode,
+prefill, fused layer and verify, batched forward, KDA core, short-conv mixer)
+measured the same way, each with its roofline.
 
 ``--impl reference`` times the CPU oracle alone on the same workload and
 metric (rank 0 only; other ranks exit at once).
@@ -563,6 +565,22 @@ def bench_forward_batch(steps: int, warmup: int, device):
                 rec_flops=prefill_flops(B, T))
 
 
+def forward_batch_roofline(fb, seconds: float, peaks, alu_peak: float) -> Dict[str, object]:
+    """The stages of the batched forward run one after another, so its ideal
+    time is the sum of each stage's own bound: the projection GEMMs at the
+    bf16 tensor peak, the recurrence at the FP32 ALU peak, and the conv
+    (read + write of the qkv activations), the q/k norms (read + write of q
+    and k) and the tail (o and z in, bf16 y out) at the HBM peak."""
+    BT, C, HD, QK = fb["tokens"], 8192, 4096, 4096
+    hbm_bytes = BT * (2 * C * 4 + 2 * QK * 4 + 2 * HD * 4 + HD * 2)
+    parts = {"gemm_ms": fb["gemm_flops"] / (peaks["bf16_tflops"] * 1e12) * 1e3,
+             "recurrence_ms": fb["rec_flops"] / (alu_peak * 1e12) * 1e3,
+             "elementwise_ms": hbm_bytes / (peaks["hbm_gbs"] * 1e9) * 1e3}
+    ideal = sum(parts.values())
+    return {"bound": "sum of stage bounds (tensor + alu + hbm)", "ideal_ms": ideal,
+            "frac": ideal / (seconds * 1e3), **parts}
+
+
 def bench_short_conv(name: str, steps: int, warmup: int, device, peaks):
     """One short-conv workload, graph-replayed; HBM roofline for the decode
     and verify launches (weight streaming), tensor roofline for the batch."""
@@ -820,6 +838,7 @@ def run_ours(args) -> int:
             "ms_per_launch": per * 1e3,
             "tokens_per_s": fb["tokens"] / per,
             "projection_tflops": fb["gemm_flops"] / per / 1e12,
+            "roofline": forward_batch_roofline(fb, per, peaks, alu_peak),
             "note": "D=2048 bf16 projections on tcgen05 + conv + sequential recurrence + tail",
         }
         torch.cuda.empty_cache()

@@ -339,6 +339,25 @@ gdn_status gdn_short_conv_pair(const void *hidden, const void *w_in, const void 
                                float *out, void *workspace, size_t workspace_bytes, int64_t B,
                                int64_t D, int64_t K, uint32_t *status, void *stream);
 
+/*
+ * gdn_selftest_bounded_wait -- a check of the library's failure detection,
+ * with no counterpart on the source pages. Every tensor-core kernel of the
+ * library (gdn_linear_bf16 and the calls built on it) waits on mbarriers with
+ * a time limit; a wait that runs out sets a bit in the caller's status word
+ * and the kernel returns, leaving the context usable. This call runs that
+ * same bounded wait in a one-thread kernel on an mbarrier that expects one
+ * arrival: with arrive = 0 nothing arrives and the wait must give up after
+ * limit_ns nanoseconds (0 < limit_ns <= 2e9, the library's own limit); with
+ * arrive = 1 the thread arrives first and the wait returns at once.
+ *   result  device words [2]: result[0] = 0 (completed) or 1 (timed out,
+ *           the producer-timeout bit of gdn_linear_bf16's status word);
+ *           result[1] = microseconds waited. 4-byte aligned.
+ * Errors: GDN_ERR_NULL, GDN_ERR_UNSUPPORTED (limit out of range),
+ * GDN_ERR_ALIGN, GDN_ERR_CUDA (launch refused).
+ */
+gdn_status gdn_selftest_bounded_wait(uint32_t *result, uint64_t limit_ns, int arrive,
+                                     void *stream);
+
 #ifdef __cplusplus
 }
 #endif

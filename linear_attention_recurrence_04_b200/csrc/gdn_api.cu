@@ -7,6 +7,7 @@
 #include <cstring>
 
 #include <cuda_runtime.h>
+#include <nvtx3/nvToolsExt.h>
 
 #include "gdn.h"
 #include "gdn_common.cuh"
@@ -17,6 +18,15 @@ namespace gdn {
 namespace {
 
 thread_local char g_last_error[512] = "";
+
+// An NVTX range over one entry point (named after it), so a timeline tool
+// shows each library call; free when no tool is attached.
+struct NvtxRange {
+    explicit NvtxRange(const char* name) { nvtxRangePushA(name); }
+    ~NvtxRange() { nvtxRangePop(); }
+    NvtxRange(const NvtxRange&) = delete;
+    NvtxRange& operator=(const NvtxRange&) = delete;
+};
 
 gdn_status fail(gdn_status st, const char* fmt, ...) {
     va_list ap;
@@ -185,6 +195,7 @@ gdn_status step_call(const char* fn, float* state, const float* q, const float* 
                      const float* v, const float* beta, const float* gate, float* out,
                      int64_t L, int64_t B, int64_t Hk, int64_t Hv, int64_t dk, int64_t dv,
                      bool channel_decay, void* stream) {
+    NvtxRange nvtx_range(fn);
     if (L < 0 || B < 0) return fail(GDN_ERR_SHAPE, "%s: negative L=%lld or B=%lld", fn,
                                     (long long)L, (long long)B);
     gdn_status st = check_geometry(Hk, Hv, dk, dv);
@@ -216,6 +227,7 @@ gdn_status prefill_call(const char* fn, float* state, const float* q, const floa
                         const float* v, const float* beta, const float* gate, float* out,
                         int64_t B, int64_t T, int64_t Hk, int64_t Hv, int64_t dk, int64_t dv,
                         bool channel_decay, void* stream) {
+    NvtxRange nvtx_range(fn);
     if (B < 0 || T < 0) return fail(GDN_ERR_SHAPE, "%s: negative B=%lld or T=%lld", fn,
                                     (long long)B, (long long)T);
     gdn_status st = check_geometry(Hk, Hv, dk, dv);
@@ -333,6 +345,7 @@ gdn_status gdn_layer_decode(const float* mixed_qkv, const float* z, const float*
                             float l2_eps, float norm_eps, float* state, float* out, int64_t B,
                             int64_t Hk, int64_t Hv, int64_t dk, int64_t dv, int64_t K,
                             void* stream) {
+    NvtxRange nvtx_range("gdn_layer_decode");
     bool empty = false;
     gdn_status st = check_layer("gdn_layer_decode", 1, mixed_qkv, z, a, b, conv_ring, conv_w,
                                 A_log, dt_bias, norm_w, state, nullptr, nullptr, out, B, Hk,
@@ -354,6 +367,7 @@ gdn_status gdn_layer_pair(const float* mixed_qkv, const float* z, const float* a
                           float norm_eps, float* state, float* scratch_ring,
                           float* scratch_state, float* out, int64_t B, int64_t Hk, int64_t Hv,
                           int64_t dk, int64_t dv, int64_t K, void* stream) {
+    NvtxRange nvtx_range("gdn_layer_pair");
     bool empty = false;
     gdn_status st = check_layer("gdn_layer_pair", 2, mixed_qkv, z, a, b, conv_ring, conv_w,
                                 A_log, dt_bias, norm_w, state, scratch_ring, scratch_state, out,
@@ -371,6 +385,7 @@ gdn_status gdn_layer_pair(const float* mixed_qkv, const float* z, const float* a
 
 gdn_status gdn_linear_bf16(const void* x, const void* w, float* y, int64_t M, int64_t N,
                            int64_t K, uint32_t* status, void* stream) {
+    NvtxRange nvtx_range("gdn_linear_bf16");
     if (M < 0 || N < 0 || K < 0)
         return fail(GDN_ERR_SHAPE, "gdn_linear_bf16: negative M=%lld N=%lld K=%lld", (long long)M,
                     (long long)N, (long long)K);
@@ -413,6 +428,7 @@ gdn_status gdn_forward_batch(const void* hidden, const void* w_qkv, const void* 
                              float* out, void* workspace, size_t workspace_bytes, int64_t B,
                              int64_t T, int64_t D, int64_t Hk, int64_t Hv, int64_t dk,
                              int64_t dv, int64_t K, uint32_t* status, void* stream) {
+    NvtxRange nvtx_range("gdn_forward_batch");
     const char* fn = "gdn_forward_batch";
     if (B < 0 || T < 0 || D < 0) return fail(GDN_ERR_SHAPE, "%s: negative B, T or D", fn);
     gdn_status st = check_geometry(Hk, Hv, dk, dv);
@@ -477,6 +493,7 @@ gdn_status short_conv_call(const char* fn, const void* hidden, const void* w_in,
                            const float* conv_w, float* out, void* workspace,
                            size_t workspace_bytes, int64_t B, int64_t T, int64_t D, int64_t K,
                            int64_t n_commit, uint32_t* status, void* stream) {
+    NvtxRange nvtx_range(fn);
     if (B < 0 || T < 0 || D < 0) return fail(GDN_ERR_SHAPE, "%s: negative B, T or D", fn);
     if (K < 2 || K > 4)
         return fail(GDN_ERR_UNSUPPORTED, "%s: K=%lld: conv kernels of 2, 3 or 4 are implemented",

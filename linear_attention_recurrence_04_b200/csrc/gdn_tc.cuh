@@ -57,12 +57,14 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
         : "memory");
     return ok != 0;
 }
-// Wait for the phase with the given parity to complete; false on timeout.
-__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity) {
+// Wait for the phase with the given parity to complete; false once
+// `limit_ns` of %globaltimer have passed without it.
+__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity,
+                                          uint64_t limit_ns = kWaitLimitNs) {
     if (mbar_try_wait(bar, parity)) return true;
     const uint64_t t0 = global_timer();
     while (!mbar_try_wait(bar, parity)) {
-        if (global_timer() - t0 > kWaitLimitNs) return false;
+        if (global_timer() - t0 > limit_ns) return false;
     }
     return true;
 }

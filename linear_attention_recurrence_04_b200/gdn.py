@@ -32,7 +32,7 @@ EXPORTS = ("gdn_status_string", "gdn_last_error", "gdn_step", "gdn_prefill", "gd
            "gdn_layer_pair", "gdn_linear_bf16", "gdn_forward_batch_workspace_size",
            "gdn_forward_batch", "gdn_forward_batch_noalloc", "gdn_short_conv_workspace_size",
            "gdn_short_conv_forward_batch", "gdn_short_conv_forward", "gdn_short_conv_pair",
-           "gdn_kda_step", "gdn_kda_prefill")
+           "gdn_kda_step", "gdn_kda_prefill", "gdn_selftest_bounded_wait")
 
 
 class GdnError(RuntimeError):
@@ -87,6 +87,8 @@ def load_library(path: Optional[str] = None) -> ctypes.CDLL:
     for name in ("gdn_kda_step", "gdn_kda_prefill"):
         getattr(lib, name).restype = ctypes.c_int
         getattr(lib, name).argtypes = [_VP] * 7 + [_I64] * 6 + [_VP]
+    lib.gdn_selftest_bounded_wait.restype = ctypes.c_int
+    lib.gdn_selftest_bounded_wait.argtypes = [_VP, ctypes.c_uint64, ctypes.c_int, _VP]
     lib.gdn_short_conv_workspace_size.restype = ctypes.c_size_t
     lib.gdn_short_conv_workspace_size.argtypes = [_I64] * 3
     lib.gdn_short_conv_forward_batch.restype = ctypes.c_int
@@ -492,3 +494,19 @@ def short_conv_pair(hidden, w_in, w_out, conv_ring, scratch_ring, conv_w, out=No
                workspace.data_ptr(), workspace.numel(), B, D, K, sp, _stream(device, stream))
     _raise_on("gdn_short_conv_pair", st)
     return out
+
+
+# -- failure detection -------------------------------------------------------
+
+def selftest_bounded_wait(limit_ns: int, arrive: bool = False, *, device=None, stream=None):
+    """Run the library's bounded mbarrier wait on a barrier that nothing
+    arrives at (or, with arrive=True, one that completes at once). Returns
+    (timed_out, microseconds_waited) after synchronising the stream."""
+    device = torch.device("cuda", torch.cuda.current_device()) if device is None else device
+    result = torch.zeros(2, dtype=torch.int32, device=device)
+    st = _call(device, load_library().gdn_selftest_bounded_wait, result.data_ptr(), int(limit_ns),
+               1 if arrive else 0, _stream(device, stream))
+    _raise_on("gdn_selftest_bounded_wait", st)
+    torch.cuda.synchronize(device)
+    r = result.cpu().tolist()
+    return bool(r[0]), int(r[1]) & 0xFFFFFFFF

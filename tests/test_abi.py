@@ -227,3 +227,10 @@ def test_tile_grid_limits(lib):
     assert lib.gdn_forward_batch_workspace_size(1, T - 1, 16, 32, 128, 128) > 0
     assert lib.gdn_short_conv_forward_batch(fake(1), fake(2), fake(3), fake(4), fake(5), fake(13),
                                             fake(20), 1 << 40, 1, T, 64, 3, 0, None) == OVERFLOW
+
+
+def test_selftest_bounded_wait_argument_checks(lib):
+    assert lib.gdn_selftest_bounded_wait(0, 1000, 0, None) == NULL
+    assert lib.gdn_selftest_bounded_wait(fake(1), 0, 0, None) == UNSUP
+    assert lib.gdn_selftest_bounded_wait(fake(1), 2_000_000_001, 0, None) == UNSUP
+    assert lib.gdn_selftest_bounded_wait(fake(1) + 2, 1000, 0, None) == ALIGN
