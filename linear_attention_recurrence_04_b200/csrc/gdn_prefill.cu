@@ -42,9 +42,10 @@
 //    end, so the stored state has its ordinary meaning.
 //  * KDA ("Module linear_core", entry "kda_forward_batch"; the published Kimi
 //    Delta Attention update) is the same pipeline with a log-decay per key
-//    channel, g [B][T][Hv][dk]: one head per warp (NH = 1), no running scale,
-//    and each stage also carries alpha = exp(g) and alpha * k, converted in
-//    place from the staged g one stage ahead. Per element and position:
+//    channel, g [B][T][Hv][dk]: no running scale, and each stage also carries
+//    alpha = exp(g) and alpha * k per value head, converted in place from the
+//    staged g one stage ahead (stages of 8 positions, so that two value heads
+//    per warp still fit). Per element and position:
 //    W *= alpha_t, W += delta k_t, o += W q_t, a += W (alpha_{t+1} k_{t+1}).
 #include "gdn_common.cuh"
 #include "gdn_internal.h"
@@ -69,7 +70,8 @@ namespace gdn {
 
 namespace {
 
-constexpr int kTS = 16;                         // positions per stage
+constexpr int kTS = 16;                         // positions per stage (scalar decay)
+constexpr int kTSChannel = 8;                   // positions per stage (per-channel decay)
 constexpr int kStages = GDN_PREFILL_STAGES;
 constexpr int kMaxWarps = GDN_PREFILL_MAX_WARPS;
 constexpr int kLPR = GDN_PREFILL_LPR;           // lanes sharing one state row
@@ -88,14 +90,15 @@ static_assert(kLPR == 4 || kLPR == 8, "4 or 8 lanes per row");
 // as copied, then exp(g); ka holds exp(g) * k. Without kCh both are stubs.
 template <int NH, bool kCh>
 struct Stage {
-    float kq[kMaxGroups][kTS][2][kDk];          // [group][pos][k|q][col]
-    float v[kMaxGroups][kTS][NH][kMaxRows];     // rows [row_lo, row_lo + rows) of the group
-    float bg[kMaxGroups][kTS][NH][2];           // beta, gate
-    float alpha[kCh ? kMaxGroups : 1][kCh ? kTS : 1][NH][kCh ? kDk : 4];
-    float ka[kCh ? kMaxGroups : 1][kCh ? kTS : 1][NH][kCh ? kDk : 4];
+    static constexpr int TS = kCh ? kTSChannel : kTS;   // positions per stage
+    float kq[kMaxGroups][TS][2][kDk];          // [group][pos][k|q][col]
+    float v[kMaxGroups][TS][NH][kMaxRows];     // rows [row_lo, row_lo + rows) of the group
+    float bg[kMaxGroups][TS][NH][2];           // beta, gate
+    float alpha[kCh ? kMaxGroups : 1][kCh ? TS : 1][NH][kCh ? kDk : 4];
+    float ka[kCh ? kMaxGroups : 1][kCh ? TS : 1][NH][kCh ? kDk : 4];
 };
 
-// Stages in flight: the per-channel stages are larger, so three of them.
+// Stages in flight: the per-channel stages carry more per position, so three.
 template <bool kCh>
 constexpr int stages_for() { return kCh ? 3 : kStages; }
 
@@ -148,8 +151,8 @@ prefill_kernel(float* __restrict__ state, const float* __restrict__ q,
                const float* __restrict__ beta, const float* __restrict__ gate,
                float* __restrict__ out, int64_t T, int Hk, int Hv, int units_lo, int n_big,
                int64_t qk_stride, int64_t v_stride, int64_t bg_stride) {
-    static_assert(!kCh || NH == 1, "per-channel decay runs one head per warp");
     constexpr int S = stages_for<kCh>();
+    constexpr int TS = kCh ? kTSChannel : kTS;      // positions per stage
     using StageT = Stage<NH, kCh>;
     extern __shared__ __align__(16) unsigned char smem_raw[];
     StageT* stages = reinterpret_cast<StageT*>(smem_raw);
@@ -193,7 +196,7 @@ prefill_kernel(float* __restrict__ state, const float* __restrict__ q,
         for (int gi = 0; gi < kMaxGroups; ++gi) {
             if (gi >= n_groups) break;
             const Group G = grp_of[gi];
-            for (int idx = tid; idx < kTS * 64; idx += nthreads) {        // k, q rows
+            for (int idx = tid; idx < TS * 64; idx += nthreads) {        // k, q rows
                 const int chunk = idx & 31;
                 const int which = (idx >> 5) & 1;
                 const int tp = idx >> 6;
@@ -206,7 +209,7 @@ prefill_kernel(float* __restrict__ state, const float* __restrict__ q,
                 }
             }
             const int vchunks = G.rows / 4;                              // v rows
-            for (int idx = tid; idx < kTS * NH * vchunks; idx += nthreads) {
+            for (int idx = tid; idx < TS * NH * vchunks; idx += nthreads) {
                 const int chunk = idx % vchunks;
                 const int n = (idx / vchunks) % NH;
                 const int tp = idx / (vchunks * NH);
@@ -219,7 +222,7 @@ prefill_kernel(float* __restrict__ state, const float* __restrict__ q,
                     *reinterpret_cast<float4*>(dst) = make_float4(0.f, 0.f, 0.f, 0.f);
                 }
             }
-            for (int idx = tid; idx < kTS * NH * 2; idx += nthreads) {    // beta, gate
+            for (int idx = tid; idx < TS * NH * 2; idx += nthreads) {    // beta, gate
                 const int which = idx & 1;
                 const int n = (idx >> 1) % NH;
                 const int tp = (idx >> 1) / NH;
@@ -233,7 +236,7 @@ prefill_kernel(float* __restrict__ state, const float* __restrict__ q,
                 }
             }
             if constexpr (kCh) {                                         // g rows
-                for (int idx = tid; idx < kTS * NH * 32; idx += nthreads) {
+                for (int idx = tid; idx < TS * NH * 32; idx += nthreads) {
                     const int chunk = idx & 31;
                     const int n = (idx >> 5) % NH;
                     const int tp = (idx >> 5) / NH;
@@ -253,7 +256,7 @@ prefill_kernel(float* __restrict__ state, const float* __restrict__ q,
     auto convert_stage = [&](StageT& st) {
         if constexpr (kCh) {
             for (int gi2 = 0; gi2 < n_groups; ++gi2) {
-                for (int idx = tid; idx < kTS * NH * kDk; idx += nthreads) {
+                for (int idx = tid; idx < TS * NH * kDk; idx += nthreads) {
                     const int col = idx % kDk;
                     const int n = (idx / kDk) % NH;
                     const int tp = idx / (kDk * NH);
@@ -283,10 +286,10 @@ prefill_kernel(float* __restrict__ state, const float* __restrict__ q,
     for (int n = 0; n < NH; ++n) out_base[n] = out + (G.b * T * Hv + hidx[n]) * kDv + j;
 
     // Prologue: request the first S - 1 stages, then load the state rows.
-    const int64_t n_stages = (T + kTS - 1) / kTS;
+    const int64_t n_stages = (T + TS - 1) / TS;
 #pragma unroll
     for (int s2 = 0; s2 < S - 1; ++s2) {
-        if (s2 < n_stages) load_stage(static_cast<int64_t>(s2) * kTS, stages[s2]);
+        if (s2 < n_stages) load_stage(static_cast<int64_t>(s2) * TS, stages[s2]);
         cp_async_commit();
     }
 
@@ -314,7 +317,7 @@ prefill_kernel(float* __restrict__ state, const float* __restrict__ q,
         __syncthreads();                     // ... and everyone's; stage s-1 is consumed
         {
             const int64_t nxt = s + S - 1;
-            if (nxt < n_stages) load_stage(nxt * kTS, stages[nxt % S]);
+            if (nxt < n_stages) load_stage(nxt * TS, stages[nxt % S]);
             cp_async_commit();
         }
         if constexpr (kCh) {
@@ -327,12 +330,12 @@ prefill_kernel(float* __restrict__ state, const float* __restrict__ q,
         if (!active) continue;
         const StageT& st = stages[s % S];
         const StageT& st_next = stages[(s + 1) % S];
-        const int64_t t0 = s * kTS;
-        const int tp_end = (T - t0) < kTS ? static_cast<int>(T - t0) : kTS;
+        const int64_t t0 = s * TS;
+        const int tp_end = (T - t0) < TS ? static_cast<int>(T - t0) : TS;
 
-        // decays of this stage, one per lane: lane tp + kTS n holds exp(gate)
+        // decays of this stage, one per lane: lane tp + TS n holds exp(gate)
         const float e_lane =
-            (!kCh && lane < kTS * NH) ? expf(st.bg[gi][lane % kTS][lane / kTS][1]) : 1.0f;
+            (!kCh && lane < TS * NH) ? expf(st.bg[gi][lane % TS][lane / TS][1]) : 1.0f;
 
         if (s == 0) {
             // first key dot: a = W.k_0
@@ -375,7 +378,7 @@ prefill_kernel(float* __restrict__ state, const float* __restrict__ q,
             float s_new[NH];
 #pragma unroll
             for (int n = 0; n < NH; ++n) {
-                const float e = kCh ? 1.0f : __shfl_sync(kFull, e_lane, tp + kTS * n);
+                const float e = kCh ? 1.0f : __shfl_sync(kFull, e_lane, tp + TS * n);
                 s_new[n] = sc[n] * e;
                 const float sk = s_new[n] * A[n];
                 cf[n] = (st.v[gi][tp][n][vrow] - sk) * st.bg[gi][tp][n][0];   // delta
@@ -402,10 +405,10 @@ prefill_kernel(float* __restrict__ state, const float* __restrict__ q,
             }
             // (c) one pass: step 4 for t, then W.q_t (step 5) and W.k_{t+1}
             const bool has_next = t + 1 < T;
-            const float* kn = (tp + 1 < kTS) ? &st.kq[gi][tp + 1][0][0] : &st_next.kq[gi][0][0][0];
+            const float* kn = (tp + 1 < TS) ? &st.kq[gi][tp + 1][0][0] : &st_next.kq[gi][0][0][0];
             const float* kan = nullptr;     // decay * key of the next position (kCh)
             if constexpr (kCh)
-                kan = (tp + 1 < kTS) ? &st.ka[gi][tp + 1][0][0] : &st_next.ka[gi][0][0][0];
+                kan = (tp + 1 < TS) ? &st.ka[gi][tp + 1][0][0] : &st_next.ka[gi][0][0][0];
 #pragma unroll
             for (int n = 0; n < NH; ++n) {
                 o_lo[n] = o_hi[n] = a_lo[n] = a_hi[n] = make_float2(0.f, 0.f);
@@ -504,7 +507,8 @@ cudaError_t launch_prefill(const PrefillArgs& a, cudaStream_t stream) {
 }
 
 cudaError_t launch_kda_prefill(const PrefillArgs& a, cudaStream_t stream) {
-    return launch_nh<1, true>(a, stream);
+    const int G = a.Hv / a.Hk;
+    return (G % 2 == 0) ? launch_nh<2, true>(a, stream) : launch_nh<1, true>(a, stream);
 }
 
 }  // namespace gdn
