@@ -63,30 +63,37 @@ short_conv_gate_kernel(const float* __restrict__ proj, const float* __restrict__
         }
     }
     const int n = static_cast<int>((T - t0) < kConvTile ? (T - t0) : kConvTile);
-    // all loads of the tile first, then the sequential window walk
-    float bg[kConvTile], cg[kConvTile], xv[kConvTile];
-#pragma unroll
-    for (int i = 0; i < kConvTile; ++i) {
-        if (i < n) {
-            const float* p = pb + (t0 + i) * D3;
-            bg[i] = p[0];
-            cg[i] = p[D];
-            xv[i] = p[2 * D];
-        }
-    }
+    // Blocks of kSub positions: all loads of a block first, then the window
+    // walk. A decode call (one position) runs one block, not the whole tile.
+    constexpr int kSub = 8;
     __nv_bfloat16* yb = y + (b * T + t0) * D + d;
+#pragma unroll 1
+    for (int i0 = 0; i0 < n; i0 += kSub) {
+        float bg[kSub], cg[kSub], xv[kSub];
 #pragma unroll
-    for (int i = 0; i < kConvTile; ++i) {
-        if (i < n) {
-            const float u = __fmul_rn(bg[i], xv[i]);
-            double conv = 0.0;
+        for (int i = 0; i < kSub; ++i) {
+            if (i0 + i < n) {
+                const float* p = pb + (t0 + i0 + i) * D3;
+                bg[i] = p[0];
+                cg[i] = p[D];
+                xv[i] = p[2 * D];
+            }
+        }
 #pragma unroll
-            for (int tau = 0; tau < K - 1; ++tau) conv = fma(w[tau], static_cast<double>(win[tau]), conv);
-            conv = fma(w[K - 1], static_cast<double>(u), conv);
-            yb[static_cast<int64_t>(i) * D] = __double2bfloat16(static_cast<double>(cg[i]) * conv);
+        for (int i = 0; i < kSub; ++i) {
+            if (i0 + i < n) {
+                const float u = __fmul_rn(bg[i], xv[i]);
+                double conv = 0.0;
 #pragma unroll
-            for (int tau = 0; tau < K - 2; ++tau) win[tau] = win[tau + 1];
-            win[K - 2] = u;
+                for (int tau = 0; tau < K - 1; ++tau)
+                    conv = fma(w[tau], static_cast<double>(win[tau]), conv);
+                conv = fma(w[K - 1], static_cast<double>(u), conv);
+                yb[static_cast<int64_t>(i0 + i) * D] =
+                    __double2bfloat16(static_cast<double>(cg[i]) * conv);
+#pragma unroll
+                for (int tau = 0; tau < K - 2; ++tau) win[tau] = win[tau + 1];
+                win[K - 2] = u;
+            }
         }
     }
 }

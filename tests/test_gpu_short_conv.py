@@ -112,6 +112,20 @@ def test_chunks_and_single_positions_are_elementwise_identical():
     assert torch.equal(single["conv_ring"], whole["conv_ring"]), "single-position ring"
 
 
+@pytest.mark.parametrize("B,T,D", [(3, 5, 1024), (2, 1, 1088), (7, 9, 1088)])
+def test_wide_hidden_matches_oracle(o, B, T, D):
+    """Hidden sizes of 16 and 17 k-steps of 64 (the last one ragged in
+    groups of 8), one position and several."""
+    d = inputs.short_conv_inputs(B, T, D=D, K=3, seed=1480 + D + T)
+    t = to_dev(d)
+    out = gpu_batch(t)
+    ref_out, ref_ring = o.short_conv_forward_batch(d["hidden"], d["w_in"], d["w_out"],
+                                                   d["conv_ring"], d["conv_w"])
+    check_out(out.cpu().numpy(), ref_out, f"B{B} T{T} D{D} out")
+    check_ring(t["conv_ring"].cpu().numpy(), d["conv_ring"], d["hidden"], d["w_in"], ref_ring,
+               T - 1, f"B{B} T{T} D{D} ring")
+
+
 @pytest.mark.parametrize("K", [2, 3, 4])
 def test_pair_matches_oracle(o, K):
     B, D = 5, 192
