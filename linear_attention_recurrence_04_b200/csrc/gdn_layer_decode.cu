@@ -80,6 +80,37 @@ __device__ __forceinline__ void cp_async_wait() {
     asm volatile("cp.async.wait_group %0;\n" ::"n"(N) : "memory");
 }
 
+// One halving step of warp_sum_many: a lane keeps one half of its HALF * 2
+// values (the upper half if its `o` bit is set) and adds its partner's
+// copy of that half, sending the other.
+template <int HALF>
+__device__ __forceinline__ void fold_step(double* v, int lane, int o) {
+    const bool up = (lane & o) != 0;
+#pragma unroll
+    for (int i = 0; i < HALF; ++i) {
+        const double send = up ? v[i] : v[i + HALF];
+        const double keep = up ? v[i + HALF] : v[i];
+        v[i] = keep + __shfl_xor_sync(kFull, send, o);
+    }
+}
+
+// Sums each of the N values v[0..N-1] over the warp's 32 lanes (N a power of
+// two, at most 32) with N - 1 + log2(32 / N) shuffles instead of 5 N. Lane L
+// returns the total of value L >> (5 - log2 N).
+template <int N>
+__device__ __forceinline__ double warp_sum_many(double (&v)[N], int lane) {
+    static_assert(N >= 1 && N <= 32 && (N & (N - 1)) == 0, "N must be a power of two <= 32");
+    int o = 16;
+    if constexpr (N >= 32) { fold_step<16>(v, lane, o); o >>= 1; }
+    if constexpr (N >= 16) { fold_step<8>(v, lane, o); o >>= 1; }
+    if constexpr (N >= 8) { fold_step<4>(v, lane, o); o >>= 1; }
+    if constexpr (N >= 4) { fold_step<2>(v, lane, o); o >>= 1; }
+    if constexpr (N >= 2) { fold_step<1>(v, lane, o); o >>= 1; }
+    double s = v[0];
+    for (; o >= 1; o >>= 1) s += __shfl_xor_sync(kFull, s, o);
+    return s;
+}
+
 struct D4 {
     double x, y, z, w;
 };
@@ -263,39 +294,63 @@ layer_kernel(const float* __restrict__ mixed_qkv, const float* __restrict__ z,
         double o_lane[NPOS];
 #pragma unroll
         for (int ps = 0; ps < NPOS; ++ps) o_lane[ps] = 0.0;
+        // dot products of the task's input rows with k and q of every
+        // position, in double, reduced over the warp RG rows at a time: value
+        // (rr * NPOS + ps) * 2 + {0: m.k, 1: m.q} ends on lane value << kShift
+        constexpr int RG = (NPOS == 2 && R % 2 == 0) ? 2 : R;   // rows reduced together
+        constexpr int kVals = RG * NPOS * 2;
+        constexpr int kShift = kVals == 32 ? 0 : kVals == 16 ? 1 : kVals == 8 ? 2 : kVals == 4 ? 3 : 4;
 #pragma unroll
-        for (int r = 0; r < R; ++r) {
-            const float4 x = m[r * 32];
-            // dot products of the input row, in double
-            const double mk0 = warp_sum_d(dot_fd(x, kd[0]));
-            const double mq0 = warp_sum_d(dot_fd(x, qd[0]));
-            const double d0 = (s_v[0][hh][row0 + r] - e0 * mk0) * b0;      // steps 1-3
-            const double out0 = (e0 * mq0 + d0 * kq00) * static_cast<double>(kOutScale);
-            if (lane == r) o_lane[0] = out0;
-            // step 4 for position 0, stored to the live state
-            const float d0f = static_cast<float>(d0);
-            float4 m1;
-            m1.x = fmaf(d0f, kf0.x, e0f * x.x);
-            m1.y = fmaf(d0f, kf0.y, e0f * x.y);
-            m1.z = fmaf(d0f, kf0.z, e0f * x.z);
-            m1.w = fmaf(d0f, kf0.w, e0f * x.w);
-            st_stream(state + off + r * kDk, m1);
-            if (NPOS == 2) {
-                const double e1 = s_decay[NPOS - 1][hh], b1 = s_beta[NPOS - 1][hh];
-                const double mk1 = warp_sum_d(dot_fd(x, kd[NPOS - 1]));
-                const double mq1 = warp_sum_d(dot_fd(x, qd[NPOS - 1]));
-                const double m1k1 = e0 * mk1 + d0 * kk01;
-                const double m1q1 = e0 * mq1 + d0 * kq01;
-                const double d1 = (s_v[NPOS - 1][hh][row0 + r] - e1 * m1k1) * b1;
-                const double out1 = (e1 * m1q1 + d1 * kq11) * static_cast<double>(kOutScale);
-                if (lane == r) o_lane[NPOS - 1] = out1;
-                const float e1f = static_cast<float>(e1), d1f = static_cast<float>(d1);
-                float4 m2;
-                m2.x = fmaf(d1f, kf1.x, e1f * m1.x);
-                m2.y = fmaf(d1f, kf1.y, e1f * m1.y);
-                m2.z = fmaf(d1f, kf1.z, e1f * m1.z);
-                m2.w = fmaf(d1f, kf1.w, e1f * m1.w);
-                st_stream(scratch_state + off + r * kDk, m2);
+        for (int rg = 0; rg < R; rg += RG) {
+            float4 xs[RG];
+            double dots[kVals];
+#pragma unroll
+            for (int rr = 0; rr < RG; ++rr) {
+                xs[rr] = m[(rg + rr) * 32];
+#pragma unroll
+                for (int ps = 0; ps < NPOS; ++ps) {
+                    dots[(rr * NPOS + ps) * 2] = dot_fd(xs[rr], kd[ps]);
+                    dots[(rr * NPOS + ps) * 2 + 1] = dot_fd(xs[rr], qd[ps]);
+                }
+            }
+            const double tot = warp_sum_many<kVals>(dots, lane);
+            auto dot_of = [&](int rr, int ps, int which) -> double {
+                return __shfl_sync(kFull, tot, ((rr * NPOS + ps) * 2 + which) << kShift);
+            };
+#pragma unroll
+            for (int rr = 0; rr < RG; ++rr) {
+                const int r = rg + rr;
+                const float4 x = xs[rr];
+                const double mk0 = dot_of(rr, 0, 0);
+                const double mq0 = dot_of(rr, 0, 1);
+                const double d0 = (s_v[0][hh][row0 + r] - e0 * mk0) * b0;      // steps 1-3
+                const double out0 = (e0 * mq0 + d0 * kq00) * static_cast<double>(kOutScale);
+                if (lane == r) o_lane[0] = out0;
+                // step 4 for position 0, stored to the live state
+                const float d0f = static_cast<float>(d0);
+                float4 m1;
+                m1.x = fmaf(d0f, kf0.x, e0f * x.x);
+                m1.y = fmaf(d0f, kf0.y, e0f * x.y);
+                m1.z = fmaf(d0f, kf0.z, e0f * x.z);
+                m1.w = fmaf(d0f, kf0.w, e0f * x.w);
+                st_stream(state + off + r * kDk, m1);
+                if (NPOS == 2) {
+                    const double e1 = s_decay[NPOS - 1][hh], b1 = s_beta[NPOS - 1][hh];
+                    const double mk1 = dot_of(rr, NPOS - 1, 0);
+                    const double mq1 = dot_of(rr, NPOS - 1, 1);
+                    const double m1k1 = e0 * mk1 + d0 * kk01;
+                    const double m1q1 = e0 * mq1 + d0 * kq01;
+                    const double d1 = (s_v[NPOS - 1][hh][row0 + r] - e1 * m1k1) * b1;
+                    const double out1 = (e1 * m1q1 + d1 * kq11) * static_cast<double>(kOutScale);
+                    if (lane == r) o_lane[NPOS - 1] = out1;
+                    const float e1f = static_cast<float>(e1), d1f = static_cast<float>(d1);
+                    float4 m2;
+                    m2.x = fmaf(d1f, kf1.x, e1f * m1.x);
+                    m2.y = fmaf(d1f, kf1.y, e1f * m1.y);
+                    m2.z = fmaf(d1f, kf1.z, e1f * m1.z);
+                    m2.w = fmaf(d1f, kf1.w, e1f * m1.w);
+                    st_stream(scratch_state + off + r * kDk, m2);
+                }
             }
         }
         if (lane < R) {
