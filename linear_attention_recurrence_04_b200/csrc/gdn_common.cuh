@@ -46,6 +46,43 @@ __device__ __forceinline__ float group_sum(float x) {
     return x;
 }
 
+// One halving step of warp_sum_many: a lane keeps one half of its 2 HALF
+// values (the upper half if its `o` bit is set), adds its partner's copy of
+// that half, and sends the other half.
+template <int HALF, typename T>
+__device__ __forceinline__ void fold_step(T* v, int lane, int o) {
+    const bool up = (lane & o) != 0;
+#pragma unroll
+    for (int i = 0; i < HALF; ++i) {
+        const T send = up ? v[i] : v[i + HALF];
+        const T keep = up ? v[i + HALF] : v[i];
+        v[i] = keep + __shfl_xor_sync(kFull, send, o);
+    }
+}
+
+// Sums each of the N values v[0..N-1] over the warp's 32 lanes (N a power of
+// two, at most 32) with N - 1 + log2(32 / N) shuffles instead of 5 N. Lane L
+// returns the total of value L >> (5 - log2 N).
+template <int N, typename T>
+__device__ __forceinline__ T warp_sum_many(T (&v)[N], int lane) {
+    static_assert(N >= 1 && N <= 32 && (N & (N - 1)) == 0, "N must be a power of two <= 32");
+    int o = 16;
+    if constexpr (N >= 32) { fold_step<16>(v, lane, o); o >>= 1; }
+    if constexpr (N >= 16) { fold_step<8>(v, lane, o); o >>= 1; }
+    if constexpr (N >= 8) { fold_step<4>(v, lane, o); o >>= 1; }
+    if constexpr (N >= 4) { fold_step<2>(v, lane, o); o >>= 1; }
+    if constexpr (N >= 2) { fold_step<1>(v, lane, o); o >>= 1; }
+    T s = v[0];
+    for (; o >= 1; o >>= 1) s += __shfl_xor_sync(kFull, s, o);
+    return s;
+}
+
+// The lane that warp_sum_many<N> leaves value `i`'s total on.
+template <int N>
+__device__ __forceinline__ int sum_many_lane(int i) {
+    return i << (N == 32 ? 0 : N == 16 ? 1 : N == 8 ? 2 : N == 4 ? 3 : N == 2 ? 4 : 5);
+}
+
 __device__ __forceinline__ float sigmoidf_acc(float x) { return 1.0f / (1.0f + expf(-x)); }
 __device__ __forceinline__ float siluf_acc(float x) { return x / (1.0f + expf(-x)); }
 // softplus(x) = ln(1 + e^x) = max(x, 0) + ln(1 + e^-|x|)

@@ -80,37 +80,6 @@ __device__ __forceinline__ void cp_async_wait() {
     asm volatile("cp.async.wait_group %0;\n" ::"n"(N) : "memory");
 }
 
-// One halving step of warp_sum_many: a lane keeps one half of its HALF * 2
-// values (the upper half if its `o` bit is set) and adds its partner's
-// copy of that half, sending the other.
-template <int HALF>
-__device__ __forceinline__ void fold_step(double* v, int lane, int o) {
-    const bool up = (lane & o) != 0;
-#pragma unroll
-    for (int i = 0; i < HALF; ++i) {
-        const double send = up ? v[i] : v[i + HALF];
-        const double keep = up ? v[i + HALF] : v[i];
-        v[i] = keep + __shfl_xor_sync(kFull, send, o);
-    }
-}
-
-// Sums each of the N values v[0..N-1] over the warp's 32 lanes (N a power of
-// two, at most 32) with N - 1 + log2(32 / N) shuffles instead of 5 N. Lane L
-// returns the total of value L >> (5 - log2 N).
-template <int N>
-__device__ __forceinline__ double warp_sum_many(double (&v)[N], int lane) {
-    static_assert(N >= 1 && N <= 32 && (N & (N - 1)) == 0, "N must be a power of two <= 32");
-    int o = 16;
-    if constexpr (N >= 32) { fold_step<16>(v, lane, o); o >>= 1; }
-    if constexpr (N >= 16) { fold_step<8>(v, lane, o); o >>= 1; }
-    if constexpr (N >= 8) { fold_step<4>(v, lane, o); o >>= 1; }
-    if constexpr (N >= 4) { fold_step<2>(v, lane, o); o >>= 1; }
-    if constexpr (N >= 2) { fold_step<1>(v, lane, o); o >>= 1; }
-    double s = v[0];
-    for (; o >= 1; o >>= 1) s += __shfl_xor_sync(kFull, s, o);
-    return s;
-}
-
 struct D4 {
     double x, y, z, w;
 };
@@ -295,11 +264,10 @@ layer_kernel(const float* __restrict__ mixed_qkv, const float* __restrict__ z,
 #pragma unroll
         for (int ps = 0; ps < NPOS; ++ps) o_lane[ps] = 0.0;
         // dot products of the task's input rows with k and q of every
-        // position, in double, reduced over the warp RG rows at a time: value
-        // (rr * NPOS + ps) * 2 + {0: m.k, 1: m.q} ends on lane value << kShift
+        // position, in double, reduced over the warp RG rows at a time (value
+        // (rr * NPOS + ps) * 2 + {0: m.k, 1: m.q})
         constexpr int RG = (NPOS == 2 && R % 2 == 0) ? 2 : R;   // rows reduced together
         constexpr int kVals = RG * NPOS * 2;
-        constexpr int kShift = kVals == 32 ? 0 : kVals == 16 ? 1 : kVals == 8 ? 2 : kVals == 4 ? 3 : 4;
 #pragma unroll
         for (int rg = 0; rg < R; rg += RG) {
             float4 xs[RG];
@@ -315,7 +283,7 @@ layer_kernel(const float* __restrict__ mixed_qkv, const float* __restrict__ z,
             }
             const double tot = warp_sum_many<kVals>(dots, lane);
             auto dot_of = [&](int rr, int ps, int which) -> double {
-                return __shfl_sync(kFull, tot, ((rr * NPOS + ps) * 2 + which) << kShift);
+                return __shfl_sync(kFull, tot, sum_many_lane<kVals>((rr * NPOS + ps) * 2 + which));
             };
 #pragma unroll
             for (int rr = 0; rr < RG; ++rr) {

@@ -10,8 +10,9 @@
 // known, so the kernel streams rows. A warp owns R = 4 consecutive rows of one
 // head; lane l holds columns [4l, 4l+4) of each row as one float4, so a row
 // is one coalesced 512-byte access. All R row loads are issued before any
-// arithmetic, the five steps run in registers (two warp-shuffle reductions
-// per row), and each row is written back once: the state crosses HBM exactly
+// arithmetic, the five steps run in registers (the R rows' key dots share one
+// warp reduction, and so do their output dots), and each row is written back
+// once: the state crosses HBM exactly
 // once in each direction per token. Warps walk row groups with a grid-stride
 // loop over a persistent grid of (SMs x resident CTAs), prefetching the next
 // group's rows while the current group computes.
@@ -88,29 +89,32 @@ __device__ __forceinline__ void update_rows(float4 (&m)[R], float* __restrict__ 
     }
     const float bt = beta[t.head];
     const int64_t vrow = t.head * kDv + t.row0;
-    const float v_lane = lane < R ? v[vrow + lane] : 0.0f;
     float* rows = state + vrow * kDk + lane * 4;
-    float o_lane = 0.0f;
+    // step 1 on every row, then step 2 for all R rows in one reduction:
+    // lane sum_many_lane<R>(r) receives sk of row r and forms its delta
+    float part[R];
 #pragma unroll
     for (int r = 0; r < R; ++r) {
-        float4 x = m[r];
-        // step 1: decay
-        x.x *= decay.x; x.y *= decay.y; x.z *= decay.z; x.w *= decay.w;
-        // step 2: sk = M[j].k on the decayed row
-        const float sk = warp_sum(dot4(x, k4));
-        // step 3: delta
-        const float delta = (__shfl_sync(kFull, v_lane, r) - sk) * bt;
-        // step 4: rank-1 update
-        x.x = fmaf(delta, k4.x, x.x);
-        x.y = fmaf(delta, k4.y, x.y);
-        x.z = fmaf(delta, k4.z, x.z);
-        x.w = fmaf(delta, k4.w, x.w);
-        // step 5: output from the updated row
-        const float o = warp_sum(dot4(x, q4)) * kOutScale;
-        if (lane == r) o_lane = o;
-        st_stream(rows + r * kDk, x);
+        m[r].x *= decay.x; m[r].y *= decay.y; m[r].z *= decay.z; m[r].w *= decay.w;
+        part[r] = dot4(m[r], k4);
     }
-    if (lane < R) out[vrow + lane] = o_lane;
+    const float sk_lane = warp_sum_many<R>(part, lane);
+    const int my_row = lane / (32 / R);                     // the row whose totals this lane holds
+    const float delta_lane = (v[vrow + my_row] - sk_lane) * bt;          // step 3
+#pragma unroll
+    for (int r = 0; r < R; ++r) {
+        const float delta = __shfl_sync(kFull, delta_lane, sum_many_lane<R>(r));
+        // step 4: rank-1 update
+        m[r].x = fmaf(delta, k4.x, m[r].x);
+        m[r].y = fmaf(delta, k4.y, m[r].y);
+        m[r].z = fmaf(delta, k4.z, m[r].z);
+        m[r].w = fmaf(delta, k4.w, m[r].w);
+        part[r] = dot4(m[r], q4);
+        st_stream(rows + r * kDk, m[r]);
+    }
+    // step 5: the outputs of the updated rows, again in one reduction
+    const float o_lane = warp_sum_many<R>(part, lane) * kOutScale;
+    if (lane % (32 / R) == 0) out[vrow + my_row] = o_lane;
 }
 
 template <int R, bool kChannelDecay>
