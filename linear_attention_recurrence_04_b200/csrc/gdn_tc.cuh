@@ -58,15 +58,20 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
     return ok != 0;
 }
 // Wait for the phase with the given parity to complete; false once
-// `limit_ns` of %globaltimer have passed without it.
+// `limit_ns` of %globaltimer have passed without it. The timer is read once
+// per kPollsPerCheck polls, so that reading it does not delay noticing the
+// phase.
+constexpr int kPollsPerCheck = 64;
 __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity,
                                           uint64_t limit_ns = kWaitLimitNs) {
     if (mbar_try_wait(bar, parity)) return true;
     const uint64_t t0 = global_timer();
-    while (!mbar_try_wait(bar, parity)) {
+    for (;;) {
+#pragma unroll 1
+        for (int i = 0; i < kPollsPerCheck; ++i)
+            if (mbar_try_wait(bar, parity)) return true;
         if (global_timer() - t0 > limit_ns) return false;
     }
-    return true;
 }
 
 // ---- TMA: 2D tiled load global -> shared, completing on an mbarrier --------
