@@ -404,6 +404,10 @@ prefill_kernel(float* __restrict__ state, const float* __restrict__ q,
                 s_out[n] = sc[n];
             }
             // (c) one pass: step 4 for t, then W.q_t (step 5) and W.k_{t+1}
+            // Past T the next position's key dot is never used. The scalar
+            // path zeroes its input there (measured faster); the per-channel
+            // path reads the slot anyway -- a zero-filled position or the
+            // next stage buffer, always in bounds (measured faster).
             const bool has_next = t + 1 < T;
             const float* kn = (tp + 1 < TS) ? &st.kq[gi][tp + 1][0][0] : &st_next.kq[gi][0][0][0];
             const float* kan = nullptr;     // decay * key of the next position (kCh)
@@ -430,8 +434,7 @@ prefill_kernel(float* __restrict__ state, const float* __restrict__ q,
                         const float2 dl = fma2(lo2(wv), lo2(al), z2);
                         const float2 dh = fma2(hi2(wv), hi2(al), z2);
                         wv = make_float4(dl.x, dl.y, dh.x, dh.y);
-                        next = has_next ? ld_s4(kan + n * kDk + chunk_col(i, c))
-                                        : make_float4(0.f, 0.f, 0.f, 0.f);
+                        next = ld_s4(kan + n * kDk + chunk_col(i, c));
                     }
                     const float2 lo = fma2(cf2, lo2(kv), lo2(wv));
                     const float2 hi = fma2(cf2, hi2(kv), hi2(wv));
