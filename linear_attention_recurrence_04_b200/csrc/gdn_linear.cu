@@ -8,21 +8,24 @@
 // "gdn_forward_batch", runs them as matrix-matrix products over a batch of
 // positions.
 //
-// Design (persistent: one CTA per SM walks 128 x BN output tiles, 192
-// threads; BN is 256, 128 or 64, the widest whose tile count still covers
-// every SM once -- a decode-sized product with few rows gets narrow tiles so
-// that more SMs stream the weights):
-//   warp 0      one thread issues TMA loads of 128 x 64 tiles of x and W
-//               (128-byte swizzle) into an S-stage shared-memory ring that
-//               runs on across tiles;
-//   warp 1      owns two TMEM accumulators (2 x BN fp32 columns x 128 lanes);
-//               one thread issues tcgen05.mma (bf16, M = 128, N = BN,
-//               K = 16) per 32-byte K step into the tile's accumulator; a
-//               tcgen05.commit per stage frees the slot back to the producer,
-//               one per tile hands the accumulator to the epilogue;
-//   warps 2-5   read an accumulator with tcgen05.ld (each warp its TMEM lane
-//               quarter, i.e. 32 rows), store fp32 rows, and release it: while
-//               they drain tile i, the MMAs of tile i+1 fill the other one.
+// Design (persistent: one CTA per SM walks BM x BN output tiles, 192
+// threads). The tile is the widest of 256 x 256, 128 x 256, 128 x 128 and
+// 128 x 64 whose count still covers every SM once: wide tiles take in fewer
+// bytes per MMA through TMA (which bounds this kernel), narrow ones let a
+// decode-sized product spread its weight stream over more SMs.
+//   warp 0      one thread issues TMA loads of BM x 64 tiles of x and BN x 64
+//               tiles of W (128-byte swizzle) into an S-stage shared-memory
+//               ring that runs on across tiles;
+//   warp 1      owns the TMEM accumulators -- two sets of BN fp32 columns for
+//               128-row tiles, one set of 2 x 256 for 256-row tiles (TMEM
+//               holds 512 columns); one thread issues tcgen05.mma (bf16,
+//               M = 128, N = BN, K = 16) per 32-byte K step, one per 128-row
+//               half of the tile; a tcgen05.commit per stage frees the slot
+//               back to the producer, one per tile hands the set to the
+//               epilogue;
+//   warps 2-5   read an accumulator set with tcgen05.ld (warp w its TMEM lane
+//               quarter w % 4), store fp32 rows and release the set: with two
+//               sets, tile i drains while the MMAs of tile i+1 fill the other.
 // Tiles past M, N or K are zero-filled by TMA and masked on store. An
 // element's K order never depends on the tile width, the tile's place or M,
 // so a row's result is the same in any batch. Every mbarrier wait gives up
@@ -35,35 +38,44 @@
 #include "gdn_tc.cuh"
 
 #ifndef GDN_LINEAR_BN
-#define GDN_LINEAR_BN 0          // 0: choose the tile width per launch; else force 64/128/256
-#endif
+#define GDN_LINEAR_BN 0          // 0: choose the tile per launch; else force 64/128/256 (128 rows)
+#endif                           // or 512 (256 x 256)
 
 namespace gdn {
 
 namespace {
 
-constexpr int kBM = 128;
+constexpr int kMmaM = 128;               // rows of one tcgen05.mma (cta_group::1)
 constexpr int kBK = 64;                  // 64 bf16 = one 128-byte swizzle row
-constexpr int kThreads = 192;
+constexpr int kEpilogueWarps = 4;        // one per TMEM lane quarter
+constexpr int kThreads = 64 + 32 * kEpilogueWarps;
 
-// Shared-memory ring per tile width: 4 stages of 48 KB (BN = 256), 6 of
-// 32 KB (128), 8 of 24 KB (64).
-template <int BN>
+// Shared-memory ring for a BM x BN tile: as many stages of (BM + BN) rows of
+// 128 bytes as fit 192 KB, at most 8 -- 3 of 64 KB (256 x 256), 4 of 48 KB
+// (128 x 256), 6 of 32 KB (128 x 128), 8 of 24 KB (128 x 64).
+template <int BN, int BM>
 struct LinearSmem {
-    static constexpr int kStages = BN == 256 ? 4 : (BN == 128 ? 6 : 8);
-    static constexpr uint32_t kA = kBM * kBK * 2;
+    static constexpr uint32_t kA = BM * kBK * 2;
     static constexpr uint32_t kB = BN * kBK * 2;
     static constexpr uint32_t kStage = kA + kB;
+    static constexpr int kStages = (196608 / kStage) < 8 ? static_cast<int>(196608 / kStage) : 8;
     static constexpr size_t kDynamic = static_cast<size_t>(kStage) * kStages + 1024;
 };
 
-template <int BN>
+// A tile of BM = 128 or 256 rows: with 256, two M = 128 MMAs per K step share
+// each B tile, so every byte the SM takes in through TMA feeds more MMA work
+// (the per-SM TMA intake, not the tensor pipe, bounds this kernel).
+template <int BN, int BM>
 __global__ void __launch_bounds__(kThreads, 1)
 linear_bf16_kernel(const __grid_constant__ CUtensorMap tmap_x,
                    const __grid_constant__ CUtensorMap tmap_w, float* __restrict__ y, int M,
                    int N, int K, uint32_t* __restrict__ status) {
-    using L = LinearSmem<BN>;
+    using L = LinearSmem<BN, BM>;
     constexpr int kStages = L::kStages;
+    constexpr int kHalves = BM / kMmaM;                     // MMAs per K step
+    constexpr uint32_t kAccCols = kHalves * BN;             // one tile's accumulators
+    constexpr int kNumAcc = 2 * kAccCols <= 512 ? 2 : 1;    // tiles in flight in TMEM
+    static_assert(BM == 128 || BM == 256, "tile rows");
     extern __shared__ uint8_t smem_raw[];
     __shared__ __align__(8) uint64_t full[kStages];
     __shared__ __align__(8) uint64_t empty[kStages];
@@ -81,7 +93,7 @@ linear_bf16_kernel(const __grid_constant__ CUtensorMap tmap_x,
     const int lane = threadIdx.x & 31;
     const int n_kt = (K + kBK - 1) / kBK;
     const int tiles_n = (N + BN - 1) / BN;
-    const int n_tiles = tiles_n * ((M + kBM - 1) / kBM);
+    const int n_tiles = tiles_n * ((M + BM - 1) / BM);
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < kStages; ++s) {
@@ -90,7 +102,7 @@ linear_bf16_kernel(const __grid_constant__ CUtensorMap tmap_x,
         }
         for (int a = 0; a < 2; ++a) {
             tc::mbar_init(tc::smem_u32(&acc_full[a]), 1);
-            tc::mbar_init(tc::smem_u32(&acc_empty[a]), 4);   // one arrival per epilogue warp
+            tc::mbar_init(tc::smem_u32(&acc_empty[a]), kEpilogueWarps);   // one per epilogue warp
         }
         tc::fence_mbar_init();
         issued = 0;
@@ -98,7 +110,7 @@ linear_bf16_kernel(const __grid_constant__ CUtensorMap tmap_x,
         failed = 0;
     }
     if (warp == 1) {
-        tc::tmem_alloc(tc::smem_u32(&tmem_slot), 2 * BN);
+        tc::tmem_alloc(tc::smem_u32(&tmem_slot), kNumAcc * kAccCols);
         tc::tmem_relinquish();
     }
     tc::tc_fence_before();
@@ -113,7 +125,7 @@ linear_bf16_kernel(const __grid_constant__ CUtensorMap tmap_x,
         tc::prefetch_tmap(&tmap_w);
         int64_t g = 0;                                     // k-steps issued so far
         for (int tile = blockIdx.x; tile < n_tiles && !*vfailed; tile += gridDim.x) {
-            const int m0 = (tile / tiles_n) * kBM;
+            const int m0 = (tile / tiles_n) * BM;
             const int n0 = (tile % tiles_n) * BN;
             for (int kt = 0; kt < n_kt; ++kt, ++g) {
                 const int s = static_cast<int>(g % kStages);
@@ -132,15 +144,16 @@ linear_bf16_kernel(const __grid_constant__ CUtensorMap tmap_x,
             }
         }
     } else if (warp == 1 && lane == 0) {
-        // ---- MMA issuer: tile li accumulates into accumulator li & 1 -------
-        const uint32_t idesc = tc::idesc_bf16_f32(kBM, BN);
+        // ---- MMA issuer: tile li accumulates into accumulator set li % kNumAcc
+        const uint32_t idesc = tc::idesc_bf16_f32(kMmaM, BN);
         int64_t g = 0;
         bool ok = true;
         int li = 0;
         for (int tile = blockIdx.x; ok && tile < n_tiles; tile += gridDim.x, ++li) {
-            const int acc = li & 1;
-            const uint32_t d = tmem + static_cast<uint32_t>(acc * BN);
-            if (!tc::mbar_wait(tc::smem_u32(&acc_empty[acc]), ((li >> 1) & 1) ^ 1) || *vfailed) {
+            const int acc = li % kNumAcc;
+            const int use = li / kNumAcc;                  // this set's earlier uses
+            const uint32_t d = tmem + static_cast<uint32_t>(acc) * kAccCols;
+            if (!tc::mbar_wait(tc::smem_u32(&acc_empty[acc]), (use & 1) ^ 1) || *vfailed) {
                 if (status) atomicOr(status, tc::kTimeoutMma);
                 atomicExch(&failed, 1);
                 break;
@@ -161,8 +174,13 @@ linear_bf16_kernel(const __grid_constant__ CUtensorMap tmap_x,
                 const uint32_t b = a + L::kA;
 #pragma unroll
                 for (int kk = 0; kk < kBK / 16; ++kk) {
-                    tc::mma_bf16(d, tc::desc_k_sw128(a + kk * 32), tc::desc_k_sw128(b + kk * 32),
-                                 idesc, (kt > 0 || kk > 0) ? 1u : 0u);
+#pragma unroll
+                    for (int hf = 0; hf < kHalves; ++hf) {   // rows [128 hf, 128 hf + 128)
+                        tc::mma_bf16(d + hf * BN,
+                                     tc::desc_k_sw128(a + hf * (kMmaM * kBK * 2) + kk * 32),
+                                     tc::desc_k_sw128(b + kk * 32), idesc,
+                                     (kt > 0 || kk > 0) ? 1u : 0u);
+                    }
                 }
                 tc::mma_commit(tc::smem_u32(&empty[s]));   // slot free once these MMAs finish
             }
@@ -173,41 +191,44 @@ linear_bf16_kernel(const __grid_constant__ CUtensorMap tmap_x,
         const int quarter = warp & 3;                      // TMEM lanes 32 q .. 32 q + 31
         int li = 0;
         for (int tile = blockIdx.x; tile < n_tiles; tile += gridDim.x, ++li) {
-            const int acc = li & 1;
-            if (!tc::mbar_wait(tc::smem_u32(&acc_full[acc]), (li >> 1) & 1) || *vfailed) {
+            const int acc = li % kNumAcc;
+            if (!tc::mbar_wait(tc::smem_u32(&acc_full[acc]), (li / kNumAcc) & 1) || *vfailed) {
                 if (status) atomicOr(status, tc::kTimeoutEpilogue);
                 atomicExch(&failed, 1);
                 break;
             }
             tc::tc_fence_after();
-            const int m0 = (tile / tiles_n) * kBM;
+            const int m0 = (tile / tiles_n) * BM;
             const int n0 = (tile % tiles_n) * BN;
-            const int row = m0 + quarter * 32 + lane;
-            const bool row_ok = row < M;
-            float* yrow = y + static_cast<int64_t>(row) * N;
-            const uint32_t src = tmem + static_cast<uint32_t>(acc * BN) +
-                                 (static_cast<uint32_t>(quarter * 32) << 16);
 #pragma unroll 1
-            for (int c0 = 0; c0 < BN; c0 += 32) {
-                uint32_t r[32];
-                tc::tmem_ld_32x32b_x32(src + c0, r);
-                tc::tmem_ld_wait();
-                const int col = n0 + c0;
-                if (!row_ok || col >= N) continue;
-                if (col + 32 <= N && (N & 3) == 0) {
-#pragma unroll
-                    for (int j = 0; j < 32; j += 4) {
-                        *reinterpret_cast<float4*>(yrow + col + j) =
-                            make_float4(__uint_as_float(r[j]), __uint_as_float(r[j + 1]),
-                                        __uint_as_float(r[j + 2]), __uint_as_float(r[j + 3]));
+            for (int hf = 0; hf < kHalves; ++hf) {
+                const int row = m0 + hf * kMmaM + quarter * 32 + lane;
+                const bool row_ok = row < M;
+                float* yrow = y + static_cast<int64_t>(row) * N;
+                const uint32_t src = tmem + static_cast<uint32_t>(acc) * kAccCols + hf * BN +
+                                     (static_cast<uint32_t>(quarter * 32) << 16);
+    #pragma unroll 1
+                for (int c0 = 0; c0 < BN; c0 += 32) {
+                    uint32_t r[32];
+                    tc::tmem_ld_32x32b_x32(src + c0, r);
+                    tc::tmem_ld_wait();
+                    const int col = n0 + c0;
+                    if (!row_ok || col >= N) continue;
+                    if (col + 32 <= N && (N & 3) == 0) {
+    #pragma unroll
+                        for (int j = 0; j < 32; j += 4) {
+                            *reinterpret_cast<float4*>(yrow + col + j) =
+                                make_float4(__uint_as_float(r[j]), __uint_as_float(r[j + 1]),
+                                            __uint_as_float(r[j + 2]), __uint_as_float(r[j + 3]));
+                        }
+                    } else {
+    #pragma unroll
+                        for (int j = 0; j < 32; ++j)
+                            if (col + j < N) yrow[col + j] = __uint_as_float(r[j]);
                     }
-                } else {
-#pragma unroll
-                    for (int j = 0; j < 32; ++j)
-                        if (col + j < N) yrow[col + j] = __uint_as_float(r[j]);
                 }
             }
-            // every read of this accumulator has completed: hand it back
+            // every read of this accumulator set has completed: hand it back
             tc::tc_fence_before();
             __syncwarp();
             if (lane == 0) tc::mbar_arrive(tc::smem_u32(&acc_empty[acc]));
@@ -225,7 +246,7 @@ linear_bf16_kernel(const __grid_constant__ CUtensorMap tmap_x,
     tc::tc_fence_before();
     __syncthreads();
     tc::tc_fence_after();
-    if (warp == 1) tc::tmem_dealloc(tmem, 2 * BN);
+    if (warp == 1) tc::tmem_dealloc(tmem, kNumAcc * kAccCols);
 }
 
 // cuTensorMapEncodeTiled through the runtime's driver entry point (no link
@@ -262,21 +283,21 @@ bool make_tmap(CUtensorMap* map, const void* ptr, int64_t rows, int64_t K, int b
            CUDA_SUCCESS;
 }
 
-template <int BN>
+template <int BN, int BM>
 cudaError_t launch_bn(const LinearArgs& a, cudaStream_t stream) {
     CUtensorMap tx, tw;
-    if (!make_tmap(&tx, a.x, a.M, a.K, kBM) || !make_tmap(&tw, a.w, a.N, a.K, BN))
+    if (!make_tmap(&tx, a.x, a.M, a.K, BM) || !make_tmap(&tw, a.w, a.N, a.K, BN))
         return cudaErrorInvalidValue;
-    const size_t smem = LinearSmem<BN>::kDynamic;
-    cudaError_t err = cudaFuncSetAttribute(linear_bf16_kernel<BN>,
+    const size_t smem = LinearSmem<BN, BM>::kDynamic;
+    cudaError_t err = cudaFuncSetAttribute(linear_bf16_kernel<BN, BM>,
                                            cudaFuncAttributeMaxDynamicSharedMemorySize,
                                            static_cast<int>(smem));
     if (err != cudaSuccess) return err;
-    const int64_t tiles = ((a.N + BN - 1) / BN) * ((a.M + kBM - 1) / kBM);
+    const int64_t tiles = ((a.N + BN - 1) / BN) * ((a.M + BM - 1) / BM);
     if (tiles > INT32_MAX) return cudaErrorInvalidValue;
     const int64_t sms = device_sm_count();
     const unsigned grid = static_cast<unsigned>(tiles < sms ? tiles : sms);
-    linear_bf16_kernel<BN><<<grid, kThreads, smem, stream>>>(tx, tw, a.y, static_cast<int>(a.M),
+    linear_bf16_kernel<BN, BM><<<grid, kThreads, smem, stream>>>(tx, tw, a.y, static_cast<int>(a.M),
                                                              static_cast<int>(a.N),
                                                              static_cast<int>(a.K), a.status);
     return cudaGetLastError();
@@ -286,17 +307,24 @@ cudaError_t launch_bn(const LinearArgs& a, cudaStream_t stream) {
 
 cudaError_t launch_linear_bf16(const LinearArgs& a, cudaStream_t stream) {
     if (a.M == 0 || a.N == 0) return cudaSuccess;
-    int bn = GDN_LINEAR_BN;
-    if (bn == 0) {
+    // The widest tile whose count still covers every SM once: 256 x 256,
+    // then 128 x 256, 128 x 128, 128 x 64 (decode-sized products get narrow
+    // tiles so that more SMs stream the weights).
+    int shape = GDN_LINEAR_BN;
+    if (shape == 0) {
         const int64_t sms = device_sm_count();
-        const int64_t m_tiles = (a.M + kBM - 1) / kBM;
-        bn = 64;
-        if (m_tiles * ((a.N + 255) / 256) >= sms) bn = 256;
-        else if (m_tiles * ((a.N + 127) / 128) >= sms) bn = 128;
+        auto tiles = [&](int64_t bm, int64_t bn) {
+            return ((a.M + bm - 1) / bm) * ((a.N + bn - 1) / bn);
+        };
+        shape = 64;
+        if (tiles(256, 256) >= sms) shape = 512;
+        else if (tiles(128, 256) >= sms) shape = 256;
+        else if (tiles(128, 128) >= sms) shape = 128;
     }
-    if (bn == 256) return launch_bn<256>(a, stream);
-    if (bn == 128) return launch_bn<128>(a, stream);
-    return launch_bn<64>(a, stream);
+    if (shape == 512) return launch_bn<256, 256>(a, stream);
+    if (shape == 256) return launch_bn<256, 128>(a, stream);
+    if (shape == 128) return launch_bn<128, 128>(a, stream);
+    return launch_bn<64, 128>(a, stream);
 }
 
 }  // namespace gdn
