@@ -201,3 +201,23 @@ def test_batch_b4_t4096_full_size_sampled(o):
     check_out(out[:, T - 12 + (K - 1):], ref_tail[:, K - 1:], "batch_b4_t4096 tail")
     check_ring(t["conv_ring"].cpu().numpy(), None, tail_h, d["w_in"], ref_ring, 11,
                "batch_b4_t4096 ring")
+
+
+def test_pair_b64_full_size(o):
+    """The benchmark's verify launch (64 sequences, D = 2048, K = 3), every
+    sequence against the oracle: outputs, committed and scratch rings."""
+    d = inputs.SHORT_CONV_WORKLOADS["short_conv_pair_b64"].draw()
+    t = to_dev(d)
+    scratch = torch.full_like(t["conv_ring"], float("nan"))
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    out = gdn.short_conv_pair(t["hidden"], t["w_in"], t["w_out"], t["conv_ring"], scratch,
+                              t["conv_w"], status=status)
+    torch.cuda.synchronize()
+    assert int(status.item()) == 0
+    ref_out, ref_ring, ref_scratch = o.short_conv_pair(d["hidden"], d["w_in"], d["w_out"],
+                                                       d["conv_ring"], d["conv_w"])
+    check_out(out.cpu().numpy(), ref_out, "pair_b64 out")
+    check_ring(t["conv_ring"].cpu().numpy(), d["conv_ring"], d["hidden"], d["w_in"], ref_ring, 0,
+               "pair_b64 committed ring")
+    check_ring(scratch.cpu().numpy(), d["conv_ring"], d["hidden"], d["w_in"], ref_scratch, 1,
+               "pair_b64 scratch ring")
