@@ -41,6 +41,33 @@ def test_linear_parity(M, N, K):
     check(x, w, y)
 
 
+def test_linear_wide_tiles_ragged():
+    """A product large enough for 256 x 256 tiles (at least one per SM) with M,
+    N and K all off the tile grid: every element checked."""
+    M, N, K = 3000, 3100, 200
+    x, w = bf16_pair(M, N, K, seed=11)
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    y = gdn.linear_bf16(x.cuda(), w.cuda(), status=status)
+    torch.cuda.synchronize()
+    assert int(status.item()) == 0
+    check(x, w, y)
+
+
+def test_linear_rows_independent_of_batch():
+    """A row's result does not depend on the other rows of the call or on the
+    tile shape chosen for it: rows of a 4096-row product (256 x 256 tiles)
+    equal the same rows computed alone (narrow tiles), bit for bit."""
+    M, N, K = 4096, 4096, 1024
+    x, w = bf16_pair(M, N, K, seed=13)
+    xc, wc = x.cuda(), w.cuda()
+    y = gdn.linear_bf16(xc, wc)
+    rows = [0, 255, 256, 4095]
+    for r in rows:
+        yr = gdn.linear_bf16(xc[r:r + 1].contiguous(), wc)
+        torch.cuda.synchronize()
+        assert torch.equal(yr[0], y[r]), f"row {r}"
+
+
 def test_linear_large_sampled():
     """A projection-sized product (4096 x 8192 x 2048): sampled rows checked."""
     M, N, K = 4096, 8192, 2048
