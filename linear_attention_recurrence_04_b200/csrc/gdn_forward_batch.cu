@@ -40,10 +40,17 @@ namespace {
 //    after it has read the old ring -- the only thread that reads it.
 constexpr int kConvTile = 32;
 
+// Both conv kernels move four adjacent channels per thread (16-byte
+// accesses; C is a multiple of 4), so that the pass is bound by HBM rather
+// than by load/store instruction issue.
+__device__ __forceinline__ float conv_tap(float4 w, float w0, float w1, float w2, float x) {
+    return fmaf(w.w, x, fmaf(w.z, w2, fmaf(w.y, w1, w.x * w0)));
+}
+
 __global__ void __launch_bounds__(256)
 conv_halo_kernel(const float* __restrict__ act, const float* __restrict__ ring,
                  float* __restrict__ halo, int64_t T, int64_t C, int n_tiles) {
-    const int64_t c = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+    const int64_t c = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) * 4;
     if (c >= C) return;
     const int j = blockIdx.y + 1;                        // tiles 1 .. n_tiles (n_tiles: the ring)
     const int64_t b = blockIdx.z;
@@ -52,8 +59,9 @@ conv_halo_kernel(const float* __restrict__ act, const float* __restrict__ ring,
 #pragma unroll
     for (int i = 0; i < kConvK - 1; ++i) {
         const int64_t t = end - (kConvK - 1) + i;        // raw input position (slot i)
-        dst[i * C] = t >= 0 ? act[(b * T + t) * C + c]
-                            : ring[(b * (kConvK - 1) + (kConvK - 1 + t)) * C + c];
+        const float* src = t >= 0 ? act + (b * T + t) * C + c
+                                  : ring + (b * (kConvK - 1) + (kConvK - 1 + t)) * C + c;
+        *reinterpret_cast<float4*>(dst + i * C) = *reinterpret_cast<const float4*>(src);
     }
 }
 
@@ -61,38 +69,54 @@ __global__ void __launch_bounds__(256)
 conv_tile_kernel(float* __restrict__ act, float* __restrict__ ring,
                  const float* __restrict__ halo, const float* __restrict__ conv_w, int64_t T,
                  int64_t C, int n_tiles) {
-    const int64_t c = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+    const int64_t c = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) * 4;
     if (c >= C) return;
     const int j = blockIdx.y;
     const int64_t b = blockIdx.z;
     const int64_t t0 = static_cast<int64_t>(j) * kConvTile;
     const int n = (T - t0) < kConvTile ? static_cast<int>(T - t0) : kConvTile;
-    const float4 w = ld_ro4(conv_w + c * kConvK);
+    float4 w[4];                                         // taps of channels c .. c + 3
+#pragma unroll
+    for (int q = 0; q < 4; ++q) w[q] = ld_ro4(conv_w + (c + q) * kConvK);
     const float* hs = j == 0 ? ring + b * (kConvK - 1) * C + c
                              : halo + ((b * (n_tiles + 1) + j) * (kConvK - 1)) * C + c;
-    float w0 = hs[0], w1 = hs[C], w2 = hs[2 * C];        // raw inputs, oldest first
+    // raw inputs, oldest first, of the four channels
+    float4 w0 = *reinterpret_cast<const float4*>(hs);
+    float4 w1 = *reinterpret_cast<const float4*>(hs + C);
+    float4 w2 = *reinterpret_cast<const float4*>(hs + 2 * C);
     float* col = act + (b * T + t0) * C + c;
-    float xs[kConvTile];
+    constexpr int kSub = 8;                              // positions loaded together
+#pragma unroll 1
+    for (int i0 = 0; i0 < n; i0 += kSub) {
+        float4 xs[kSub];
 #pragma unroll
-    for (int i = 0; i < kConvTile; ++i) xs[i] = (i < n) ? col[static_cast<int64_t>(i) * C] : 0.0f;
+        for (int i = 0; i < kSub; ++i)
+            if (i0 + i < n) xs[i] = *reinterpret_cast<const float4*>(col + static_cast<int64_t>(i0 + i) * C);
 #pragma unroll
-    for (int i = 0; i < kConvTile; ++i) {
-        if (i < n) {
-            const float x = xs[i];
-            const float y = fmaf(w.w, x, fmaf(w.z, w2, fmaf(w.y, w1, w.x * w0)));
-            col[static_cast<int64_t>(i) * C] = siluf_acc(y);
-            w0 = w1;
-            w1 = w2;
-            w2 = x;
+        for (int i = 0; i < kSub; ++i) {
+            if (i0 + i < n) {
+                const float4 x = xs[i];
+                float4 y;
+                y.x = siluf_acc(conv_tap(w[0], w0.x, w1.x, w2.x, x.x));
+                y.y = siluf_acc(conv_tap(w[1], w0.y, w1.y, w2.y, x.y));
+                y.z = siluf_acc(conv_tap(w[2], w0.z, w1.z, w2.z, x.z));
+                y.w = siluf_acc(conv_tap(w[3], w0.w, w1.w, w2.w, x.w));
+                *reinterpret_cast<float4*>(col + static_cast<int64_t>(i0 + i) * C) = y;
+                w0 = w1;
+                w1 = w2;
+                w2 = x;
+            }
         }
     }
     if (j == 0) {            // the ring after the call (this thread read the old one above)
         const float* nr = halo + ((b * (n_tiles + 1) + n_tiles) * (kConvK - 1)) * C + c;
         float* rg = ring + b * (kConvK - 1) * C + c;
-        const float r0 = nr[0], r1 = nr[C], r2 = nr[2 * C];
-        rg[0] = r0;
-        rg[C] = r1;
-        rg[2 * C] = r2;
+        const float4 r0 = *reinterpret_cast<const float4*>(nr);
+        const float4 r1 = *reinterpret_cast<const float4*>(nr + C);
+        const float4 r2 = *reinterpret_cast<const float4*>(nr + 2 * C);
+        *reinterpret_cast<float4*>(rg) = r0;
+        *reinterpret_cast<float4*>(rg + C) = r1;
+        *reinterpret_cast<float4*>(rg + 2 * C) = r2;
     }
 }
 
@@ -211,7 +235,7 @@ cudaError_t launch_forward_batch(const ForwardBatchArgs& a, cudaStream_t stream)
     // 2. conv over positions with the ring, SiLU (halo pass, then in place)
     {
         const int n_tiles = static_cast<int>((a.T + kConvTile - 1) / kConvTile);
-        const unsigned cblocks = static_cast<unsigned>((C + 255) / 256);
+        const unsigned cblocks = static_cast<unsigned>((C / 4 + 255) / 256);   // 4 channels a thread
         conv_halo_kernel<<<dim3(cblocks, static_cast<unsigned>(n_tiles),
                                 static_cast<unsigned>(a.B)), 256, 0, stream>>>(
             act, a.conv_ring, halo, a.T, C, n_tiles);
