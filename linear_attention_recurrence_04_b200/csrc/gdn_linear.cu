@@ -37,9 +37,11 @@
 #include "gdn_internal.h"
 #include "gdn_tc.cuh"
 
+// Tile shape: 0 chooses per launch; 64, 128 or 256 force 128 x that width;
+// 512 forces 256 x 256.
 #ifndef GDN_LINEAR_BN
-#define GDN_LINEAR_BN 0          // 0: choose the tile per launch; else force 64/128/256 (128 rows)
-#endif                           // or 512 (256 x 256)
+#define GDN_LINEAR_BN 0
+#endif
 
 namespace gdn {
 
