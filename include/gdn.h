@@ -13,28 +13,35 @@
  *   5. out[j] = dot(M[j], q) / sqrt(dk)      (the updated state)
  *
  * Conventions shared by every entry point
- *   - All tensors are dense, C-contiguous, row-major float32 in DEVICE
- *     memory of the current CUDA device; no pointer may be a host pointer.
+ *   - All tensors are dense, C-contiguous, row-major arrays in DEVICE memory
+ *     of the current CUDA device (no host pointers): float32, except the
+ *     projections' operands (hidden, x and the weight matrices), which are
+ *     bf16 bit patterns where an entry point says so.
  *   - The caller allocates and frees every buffer. The library allocates no
  *     memory, never synchronises, and enqueues its kernels on `stream`
  *     (a cudaStream_t; NULL means the legacy default stream). Results are
  *     ready once the stream reaches that point.
- *   - Supported geometry: dk = dv = 128, Hk >= 1, Hv a multiple of Hk,
- *     conv kernel K = 4. Other values return GDN_ERR_UNSUPPORTED.
+ *   - Supported geometry: dk = dv = 128, Hk >= 1, Hv a multiple of Hk, conv
+ *     kernel K = 4 for the recurrent layer's calls and K in {2, 3, 4} for the
+ *     short-conv mixer. Other values return GDN_ERR_UNSUPPORTED.
  *   - `state` and `conv_ring` are updated in place and must not overlap any
  *     other argument; `out` and the scratch outputs must not overlap any
  *     argument either (GDN_ERR_ALIAS otherwise). Read-only inputs may share
  *     memory.
- *   - Alignment: state, q, k, v, out, mixed_qkv, z, conv_ring and conv_w
- *     must be 16-byte aligned; the per-head scalars (beta, gate, a, b,
- *     A_log, dt_bias) and norm_w need 4-byte alignment.
+ *   - Alignment: state, q, k, v, g, out, mixed_qkv, z, conv_ring, conv_w,
+ *     hidden, x and the weight matrices must be 16-byte aligned, workspaces
+ *     256-byte aligned; the per-head scalars (beta, gate, a, b, A_log,
+ *     dt_bias) and norm_w need 4-byte alignment.
  *   - Arguments are checked on the host before anything is enqueued; on any
  *     error nothing is written and nothing is launched. A problem with no
  *     work (a zero size) returns GDN_OK without touching any pointer.
  *   - Sizes are int64_t. Kernel faults are asynchronous and surface at the
  *     caller's next synchronisation, as for any CUDA kernel.
  *   - Thread safety: calls from several host threads are safe; calls that
- *     update the same state buffer must be ordered by the caller.
+ *     update the same state buffer, or share a workspace, must be ordered by
+ *     the caller (gdn_forward_batch_noalloc's built-in scratch is shared by
+ *     all its calls).
+ *   - Every entry point opens an NVTX range named after itself.
  */
 #ifndef GDN_H
 #define GDN_H
