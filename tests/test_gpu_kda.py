@@ -101,3 +101,34 @@ def test_kda_prefill_b4_t4096_full_size_sampled(o):
         b, h = divmod(u, Hv)
         assert_parity(out[b, :, h], out_ref[b, :, h], f"kda prefill b{b} h{h} out")
         assert_parity(st[b, h], st_ref[b, h], f"kda prefill b{b} h{h} state")
+
+
+def test_kda_step_decay_extremes(o):
+    """Channels with g = -200 (exp underflows to 0: the column is cleared
+    before the write), g = 0 (no decay) and ordinary values in one call."""
+    d = inputs.kda_decode_inputs(1, 3, seed=1530)
+    g = d["g"].copy()
+    g[..., 0::3] = -200.0
+    g[..., 1::3] = 0.0
+    d["g"] = g
+    st_ref, out_ref = o.kda_step(d["state"], d["q"], d["k"], d["v"], d["beta"], d["g"])
+    st, out = gpu_step(d)
+    assert_parity(out, out_ref, "kda extremes out")
+    assert_parity(st, st_ref, "kda extremes state")
+
+
+def test_kda_prefill_resume_matches_one_pass(o):
+    """kda_prefill over 23 positions, then 27 more from the returned state,
+    equals the oracle over all 50."""
+    d = inputs.kda_prefill_inputs(2, 50, seed=1640, state_std=0.05)
+    t = to_dev(d)
+    cut = 23
+    sl = lambda x, a, b: x[:, a:b].contiguous()
+    o1 = gdn.kda_prefill(t["state"], sl(t["q"], 0, cut), sl(t["k"], 0, cut), sl(t["v"], 0, cut),
+                         sl(t["beta"], 0, cut), sl(t["g"], 0, cut))
+    o2 = gdn.kda_prefill(t["state"], sl(t["q"], cut, 50), sl(t["k"], cut, 50),
+                         sl(t["v"], cut, 50), sl(t["beta"], cut, 50), sl(t["g"], cut, 50))
+    torch.cuda.synchronize()
+    st_ref, out_ref = o.kda_prefill(d["state"], d["q"], d["k"], d["v"], d["beta"], d["g"])
+    assert_parity(torch.cat([o1, o2], dim=1).cpu().numpy(), out_ref, "kda resume out")
+    assert_parity(t["state"].cpu().numpy(), st_ref, "kda resume state")
