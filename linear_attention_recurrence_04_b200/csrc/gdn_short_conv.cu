@@ -21,7 +21,9 @@
 //   3. ring_update: per (sequence, channel), the ring after position
 //      n_commit - 1 goes to conv_ring and, for the two-position verify, the
 //      ring after the last position to scratch_ring (a separate kernel so
-//      that no tile of step 2 can read a ring slot that was already replaced);
+//      that no tile of step 2 can read a ring slot that was already replaced;
+//      a call of one tile -- decode, verify -- has one thread per channel,
+//      which writes the rings itself at the end of step 2);
 //   4. out = y . W_out^T              (tcgen05 GEMM).
 // u is rounded to fp32 (the ring's type) before it enters the window; the
 // window sum and the output gate run in double, and y is rounded once.
@@ -36,11 +38,15 @@ namespace {
 
 constexpr int kConvTile = 32;            // positions per thread in gate_conv
 
-template <int K>
+// kWriteRing (calls of at most kConvTile positions: one tile, so one thread
+// per (sequence, channel)): the thread that read the old ring also writes the
+// ring after position n_commit - 1 and, for the verify, the ring after the
+// last position to scratch_ring; no separate ring pass is needed.
+template <int K, bool kWriteRing>
 __global__ void __launch_bounds__(256)
-short_conv_gate_kernel(const float* __restrict__ proj, const float* __restrict__ ring,
+short_conv_gate_kernel(const float* __restrict__ proj, float* ring, float* scratch_ring,
                        const float* __restrict__ conv_w, __nv_bfloat16* __restrict__ y,
-                       int64_t B, int64_t T, int64_t D) {
+                       int64_t B, int64_t T, int64_t D, int64_t n_commit) {
     const int64_t d = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
     if (d >= D) return;
     const int64_t b = blockIdx.z;
@@ -67,6 +73,9 @@ short_conv_gate_kernel(const float* __restrict__ proj, const float* __restrict__
     // walk. A decode call (one position) runs one block, not the whole tile.
     constexpr int kSub = 8;
     __nv_bfloat16* yb = y + (b * T + t0) * D + d;
+    float committed[K - 1];                              // kWriteRing: ring after n_commit - 1
+#pragma unroll
+    for (int tau = 0; tau < K - 1; ++tau) committed[tau] = win[tau];
 #pragma unroll 1
     for (int i0 = 0; i0 < n; i0 += kSub) {
         float bg[kSub], cg[kSub], xv[kSub];
@@ -93,7 +102,21 @@ short_conv_gate_kernel(const float* __restrict__ proj, const float* __restrict__
 #pragma unroll
                 for (int tau = 0; tau < K - 2; ++tau) win[tau] = win[tau + 1];
                 win[K - 2] = u;
+                if (kWriteRing && t0 + i0 + i == n_commit - 1) {
+#pragma unroll
+                    for (int tau = 0; tau < K - 1; ++tau) committed[tau] = win[tau];
+                }
             }
+        }
+    }
+    if constexpr (kWriteRing) {
+        float* rg = ring + b * (K - 1) * D + d;
+#pragma unroll
+        for (int tau = 0; tau < K - 1; ++tau) rg[tau * D] = committed[tau];
+        if (scratch_ring) {
+            float* sg = scratch_ring + b * (K - 1) * D + d;
+#pragma unroll
+            for (int tau = 0; tau < K - 1; ++tau) sg[tau * D] = win[tau];
         }
     }
 }
@@ -144,8 +167,13 @@ cudaError_t launch_conv(const ShortConvArgs& a, float* proj, __nv_bfloat16* y,
     const dim3 grid(static_cast<unsigned>((a.D + 255) / 256),
                     static_cast<unsigned>((a.T + kConvTile - 1) / kConvTile),
                     static_cast<unsigned>(a.B));
-    short_conv_gate_kernel<K><<<grid, 256, 0, stream>>>(proj, a.conv_ring, a.conv_w, y, a.B,
-                                                        a.T, a.D);
+    if (a.T <= kConvTile) {          // one tile: the gate pass also writes the rings
+        short_conv_gate_kernel<K, true><<<grid, 256, 0, stream>>>(
+            proj, a.conv_ring, a.scratch_ring, a.conv_w, y, a.B, a.T, a.D, a.n_commit);
+        return cudaGetLastError();
+    }
+    short_conv_gate_kernel<K, false><<<grid, 256, 0, stream>>>(
+        proj, a.conv_ring, nullptr, a.conv_w, y, a.B, a.T, a.D, a.n_commit);
     cudaError_t err = cudaGetLastError();
     if (err != cudaSuccess) return err;
     const int64_t n = a.B * a.D;
