@@ -65,6 +65,9 @@
 #ifndef GDN_PREFILL_NH
 #define GDN_PREFILL_NH 0           // value heads per warp: 0 = 2 when Hv/Hk is even, else 1
 #endif
+#ifndef GDN_PREFILL_UNROLL
+#define GDN_PREFILL_UNROLL 8       // positions per unrolled block of a stage
+#endif
 
 namespace gdn {
 
@@ -73,6 +76,7 @@ namespace {
 constexpr int kTS = 16;                         // positions per stage (scalar decay)
 constexpr int kTSChannel = 8;                   // positions per stage (per-channel decay)
 constexpr int kStages = GDN_PREFILL_STAGES;
+constexpr int kUnroll = GDN_PREFILL_UNROLL;        // positions per unrolled block
 constexpr int kMaxWarps = GDN_PREFILL_MAX_WARPS;
 constexpr int kLPR = GDN_PREFILL_LPR;           // lanes sharing one state row
 constexpr int kRowsPerUnit = 32 / kLPR;         // rows of a head per warp
@@ -88,14 +92,16 @@ static_assert(kLPR == 4 || kLPR == 8, "4 or 8 lanes per row");
 
 // Shared-memory image of one stage. kCh (per-channel decay): alpha holds g
 // as copied, then exp(g); ka holds exp(g) * k. Without kCh both are stubs.
+// Slot TS of kq (k only) and of alpha / ka holds the first position of the
+// next stage, so a pass can always read the next key from its own stage.
 template <int NH, bool kCh>
 struct Stage {
     static constexpr int TS = kCh ? kTSChannel : kTS;   // positions per stage
-    float kq[kMaxGroups][TS][2][kDk];          // [group][pos][k|q][col]
+    float kq[kMaxGroups][TS + 1][2][kDk];      // [group][pos][k|q][col]
     float v[kMaxGroups][TS][NH][kMaxRows];     // rows [row_lo, row_lo + rows) of the group
     float bg[kMaxGroups][TS][NH][2];           // beta, gate
-    float alpha[kCh ? kMaxGroups : 1][kCh ? TS : 1][NH][kCh ? kDk : 4];
-    float ka[kCh ? kMaxGroups : 1][kCh ? TS : 1][NH][kCh ? kDk : 4];
+    float alpha[kCh ? kMaxGroups : 1][kCh ? TS + 1 : 1][NH][kCh ? kDk : 4];
+    float ka[kCh ? kMaxGroups : 1][kCh ? TS + 1 : 1][NH][kCh ? kDk : 4];
 };
 
 // Stages in flight: the per-channel stages carry more per position, so three.
@@ -142,7 +148,29 @@ __device__ __forceinline__ float2 fma2(float2 a, float2 b, float2 c) {
 __device__ __forceinline__ float2 lo2(float4 v) { return make_float2(v.x, v.y); }
 __device__ __forceinline__ float2 hi2(float4 v) { return make_float2(v.z, v.w); }
 __device__ __forceinline__ float4 ld_s4(const float* p) { return *reinterpret_cast<const float4*>(p); }
-__device__ __forceinline__ float sum4(float2 a, float2 b) { return (a.x + a.y) + (b.x + b.y); }
+__device__ __forceinline__ float2 mul2(float2 a, float2 b) {
+#if GDN_PREFILL_FMA2
+    return __fmul2_rn(a, b);
+#else
+    return make_float2(a.x * b.x, a.y * b.y);
+#endif
+}
+// (a.x + b.x) + (a.y + b.y): one packed add and one scalar add.
+__device__ __forceinline__ float sum4(float2 a, float2 b) {
+#if GDN_PREFILL_FMA2
+    const float2 t = __fadd2_rn(a, b);
+    return t.x + t.y;
+#else
+    return (a.x + b.x) + (a.y + b.y);
+#endif
+}
+// 1 / x to within one unit in the last place (PTX rcp.approx.ftz.f32). Used
+// for running scales in [2^-40, 2^40], where x and 1 / x are normal.
+__device__ __forceinline__ float rcp_approx(float x) {
+    float r;
+    asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(r) : "f"(x));
+    return r;
+}
 
 template <int NH, bool kCh>
 __global__ void __launch_bounds__(32 * kMaxWarps, 1)
@@ -196,9 +224,9 @@ prefill_kernel(float* __restrict__ state, const float* __restrict__ q,
         for (int gi = 0; gi < kMaxGroups; ++gi) {
             if (gi >= n_groups) break;
             const Group G = grp_of[gi];
-            for (int idx = tid; idx < TS * 64; idx += nthreads) {        // k, q rows
+            for (int idx = tid; idx < TS * 64 + 32; idx += nthreads) {   // k, q rows; k of t0 + TS
                 const int chunk = idx & 31;
-                const int which = (idx >> 5) & 1;
+                const int which = (idx >> 5) & 1;     // the extra slot gets k only
                 const int tp = idx >> 6;
                 const int64_t t = t0 + tp;
                 float* dst = &st.kq[gi][tp][which][chunk * 4];
@@ -236,7 +264,7 @@ prefill_kernel(float* __restrict__ state, const float* __restrict__ q,
                 }
             }
             if constexpr (kCh) {                                         // g rows
-                for (int idx = tid; idx < TS * NH * 32; idx += nthreads) {
+                for (int idx = tid; idx < (TS + 1) * NH * 32; idx += nthreads) {
                     const int chunk = idx & 31;
                     const int n = (idx >> 5) % NH;
                     const int tp = (idx >> 5) / NH;
@@ -256,7 +284,7 @@ prefill_kernel(float* __restrict__ state, const float* __restrict__ q,
     auto convert_stage = [&](StageT& st) {
         if constexpr (kCh) {
             for (int gi2 = 0; gi2 < n_groups; ++gi2) {
-                for (int idx = tid; idx < TS * NH * kDk; idx += nthreads) {
+                for (int idx = tid; idx < (TS + 1) * NH * kDk; idx += nthreads) {
                     const int col = idx % kDk;
                     const int n = (idx / kDk) % NH;
                     const int tp = idx / (kDk * NH);
@@ -279,11 +307,11 @@ prefill_kernel(float* __restrict__ state, const float* __restrict__ q,
     int hidx[NH];
 #pragma unroll
     for (int n = 0; n < NH; ++n) hidx[n] = G.g + (G.grp * NH + n) * Hk;
-    // out of position t, head n, row j: out_base[n] + t * out_stride
+    // Lane c < NH stores head c's outputs of row j; its pointer walks the
+    // positions (out_next: the coming position, out_prev: the pending one).
     const int64_t out_stride = static_cast<int64_t>(Hv) * kDv;
-    float* out_base[NH];
-#pragma unroll
-    for (int n = 0; n < NH; ++n) out_base[n] = out + (G.b * T * Hv + hidx[n]) * kDv + j;
+    float* out_next = out + (G.b * T * Hv + G.g + (G.grp * NH + (c < NH ? c : 0)) * Hk) * kDv + j;
+    float* out_prev = out_next;
 
     // Prologue: request the first S - 1 stages, then load the state rows.
     const int64_t n_stages = (T + TS - 1) / TS;
@@ -309,8 +337,12 @@ prefill_kernel(float* __restrict__ state, const float* __restrict__ q,
     // the previous position (its store is pending), s_out = its scale.
     float2 a_lo[NH], a_hi[NH], o_lo[NH], o_hi[NH];
     float s_out[NH];
+#pragma unroll
+    for (int n = 0; n < NH; ++n) {
+        a_lo[n] = a_hi[n] = o_lo[n] = o_hi[n] = make_float2(0.f, 0.f);
+        s_out[n] = 1.0f;
+    }
     bool out_pending = false;
-    int64_t t_out = 0;
 
     for (int64_t s = 0; s < n_stages; ++s) {
         cp_async_wait<S - 3>();             // this thread's copies of stages s, s+1 landed
@@ -329,7 +361,6 @@ prefill_kernel(float* __restrict__ state, const float* __restrict__ q,
         }
         if (!active) continue;
         const StageT& st = stages[s % S];
-        const StageT& st_next = stages[(s + 1) % S];
         const int64_t t0 = s * TS;
         const int tp_end = (T - t0) < TS ? static_cast<int>(T - t0) : TS;
 
@@ -337,116 +368,132 @@ prefill_kernel(float* __restrict__ state, const float* __restrict__ q,
         const float e_lane =
             (!kCh && lane < TS * NH) ? expf(st.bg[gi][lane % TS][lane / TS][1]) : 1.0f;
 
+        // This lane's view of the stage; position tp sits at tp * (stride).
+        constexpr int kqP = 2 * kDk;            // k and q of one position
+        constexpr int vP = NH * kMaxRows;       // v of one position
+        constexpr int bgP = 2 * NH;             // beta, gate of one position
+        constexpr int chP = NH * kDk;           // alpha or alpha * k of one position
+        constexpr int kStep = 4 * kLPR;         // columns between a lane's chunks
+        const float* kq_s = &st.kq[gi][0][0][chunk_col(0, c)];    // k; q at + kDk
+        const float* v_s = &st.v[gi][0][0][vrow];
+        const float* bg_s = &st.bg[gi][0][0][0];
+        const float* al_s = &st.alpha[gi * kCh][0][0][kCh ? chunk_col(0, c) : 0];
+        const float* ka_s = &st.ka[gi * kCh][0][0][kCh ? chunk_col(0, c) : 0];
+
         if (s == 0) {
-            // first key dot: a = W.k_0
-#pragma unroll
-            for (int n = 0; n < NH; ++n) a_lo[n] = a_hi[n] = make_float2(0.f, 0.f);
+            // first key dot: a = W.k_0 (kCh: with alpha_0 folded into k_0)
 #pragma unroll
             for (int i = 0; i < kChunks; ++i) {
 #pragma unroll
                 for (int n = 0; n < NH; ++n) {
-                    const float4 kv = kCh ? ld_s4(&st.ka[gi][0][n][chunk_col(i, c)])
-                                          : ld_s4(&st.kq[gi][0][0][chunk_col(i, c)]);
+                    const float4 kv = kCh ? ld_s4(ka_s + n * kDk + kStep * i)
+                                          : ld_s4(kq_s + kStep * i);
                     a_lo[n] = fma2(lo2(w[n][i]), lo2(kv), a_lo[n]);
                     a_hi[n] = fma2(hi2(w[n][i]), hi2(kv), a_hi[n]);
                 }
             }
         }
 
-        for (int tp = 0; tp < tp_end; ++tp) {
-            const int64_t t = t0 + tp;
+#pragma unroll(kUnroll)
+        for (int tp = 0; tp < TS; ++tp) {
+            if (tp >= tp_end) break;
             // (a) batched reductions: sk of t, and out of t-1
             float A[NH], O[NH];
 #pragma unroll
             for (int n = 0; n < NH; ++n) {
                 A[n] = sum4(a_lo[n], a_hi[n]);
-                O[n] = out_pending ? sum4(o_lo[n], o_hi[n]) : 0.0f;
+                O[n] = sum4(o_lo[n], o_hi[n]);
             }
 #pragma unroll
             for (int n = 0; n < NH; ++n) {
                 A[n] = group_sum<kLPR>(A[n]);
                 O[n] = group_sum<kLPR>(O[n]);
             }
-            if (out_pending) {
+            {   // lane c < NH stores head c's output of t - 1
+                float ov = O[0], so = s_out[0];
+#pragma unroll
+                for (int n = 1; n < NH; ++n)
+                    if (c == n) { ov = O[n]; so = s_out[n]; }
+                if (out_pending && c < NH) *out_prev = so * ov * kOutScale;
+            }
+            // (b) scalar part of position t
+            float cf[NH];
+            if constexpr (kCh) {
 #pragma unroll
                 for (int n = 0; n < NH; ++n)
-                    if (c == (n & 3)) out_base[n][t_out * out_stride] = s_out[n] * O[n] * kOutScale;
-            }
-            // (b) scalar part of position t (step 1 as a scale update, steps 2-3)
-            float cf[NH];
-            bool fold = false;
-            float s_new[NH];
-#pragma unroll
-            for (int n = 0; n < NH; ++n) {
-                const float e = kCh ? 1.0f : __shfl_sync(kFull, e_lane, tp + TS * n);
-                s_new[n] = sc[n] * e;
-                const float sk = s_new[n] * A[n];
-                cf[n] = (st.v[gi][tp][n][vrow] - sk) * st.bg[gi][tp][n][0];   // delta
-                fold |= !(s_new[n] >= kScaleLo && s_new[n] <= kScaleHi);
-            }
-            if (fold) {          // rare, and uniform across the warp
+                    cf[n] = (v_s[tp * vP + n * kMaxRows] - A[n]) * bg_s[tp * bgP + 2 * n];
+            } else {
+                // step 1 as a scale update s *= e; then, with r = 1 / s,
+                // delta / s = (v r - W.k) beta (steps 2-3)
+                float s_new[NH];
+                bool fold = false;
 #pragma unroll
                 for (int n = 0; n < NH; ++n) {
-                    if (!(s_new[n] >= kScaleLo && s_new[n] <= kScaleHi)) {
+                    s_new[n] = sc[n] * __shfl_sync(kFull, e_lane, tp + TS * n);
+                    fold |= !(s_new[n] >= kScaleLo && s_new[n] <= kScaleHi);
+                }
+                if (fold) {          // rare, and uniform across the warp
 #pragma unroll
-                        for (int i = 0; i < kChunks; ++i) {
-                            w[n][i].x *= s_new[n]; w[n][i].y *= s_new[n];
-                            w[n][i].z *= s_new[n]; w[n][i].w *= s_new[n];
+                    for (int n = 0; n < NH; ++n) {
+                        if (!(s_new[n] >= kScaleLo && s_new[n] <= kScaleHi)) {
+#pragma unroll
+                            for (int i = 0; i < kChunks; ++i) {
+                                w[n][i].x *= s_new[n]; w[n][i].y *= s_new[n];
+                                w[n][i].z *= s_new[n]; w[n][i].w *= s_new[n];
+                            }
+                            A[n] *= s_new[n];
+                            s_new[n] = 1.0f;
                         }
-                        s_new[n] = 1.0f;
                     }
                 }
-            }
 #pragma unroll
-            for (int n = 0; n < NH; ++n) {
-                sc[n] = s_new[n];
-                cf[n] *= __frcp_rn(sc[n]);                                   // delta / s
-                s_out[n] = sc[n];
+                for (int n = 0; n < NH; ++n) {
+                    sc[n] = s_new[n];
+                    s_out[n] = s_new[n];
+                    cf[n] = fmaf(v_s[tp * vP + n * kMaxRows], rcp_approx(s_new[n]), -A[n]) *
+                            bg_s[tp * bgP + 2 * n];
+                }
             }
             // (c) one pass: step 4 for t, then W.q_t (step 5) and W.k_{t+1}
-            // Past T the next position's key dot is never used. The scalar
-            // path zeroes its input there (measured faster); the per-channel
-            // path reads the slot anyway -- a zero-filled position or the
-            // next stage buffer, always in bounds (measured faster).
-            const bool has_next = t + 1 < T;
-            const float* kn = (tp + 1 < TS) ? &st.kq[gi][tp + 1][0][0] : &st_next.kq[gi][0][0][0];
-            const float* kan = nullptr;     // decay * key of the next position (kCh)
-            if constexpr (kCh)
-                kan = (tp + 1 < TS) ? &st.ka[gi][tp + 1][0][0] : &st_next.ka[gi][0][0][0];
-#pragma unroll
-            for (int n = 0; n < NH; ++n) {
-                o_lo[n] = o_hi[n] = a_lo[n] = a_hi[n] = make_float2(0.f, 0.f);
-            }
+            // (kCh: step 1 per channel first, and the next key with its decay).
+            // Slot tp + 1 always exists; past T it is zero-filled.
+            const float* kp = kq_s + tp * kqP;
 #pragma unroll
             for (int i = 0; i < kChunks; ++i) {
-                const float4 kv = ld_s4(&st.kq[gi][tp][0][chunk_col(i, c)]);
-                const float4 qv = ld_s4(&st.kq[gi][tp][1][chunk_col(i, c)]);
-                const float4 nv = has_next ? ld_s4(kn + chunk_col(i, c)) : make_float4(0.f, 0.f, 0.f, 0.f);
+                const float4 kv = ld_s4(kp + kStep * i);
+                const float4 qv = ld_s4(kp + kDk + kStep * i);
+                const float4 nv = kCh ? kv : ld_s4(kp + kqP + kStep * i);
 #pragma unroll
                 for (int n = 0; n < NH; ++n) {
                     const float2 cf2 = make_float2(cf[n], cf[n]);
                     float4 wv = w[n][i];
                     float4 next = nv;
                     if constexpr (kCh) {
-                        // step 1 per channel, and the next key with its decay
-                        const float4 al = ld_s4(&st.alpha[gi][tp][n][chunk_col(i, c)]);
-                        const float2 z2 = make_float2(0.f, 0.f);
-                        const float2 dl = fma2(lo2(wv), lo2(al), z2);
-                        const float2 dh = fma2(hi2(wv), hi2(al), z2);
+                        const float4 al = ld_s4(al_s + tp * chP + n * kDk + kStep * i);
+                        const float2 dl = mul2(lo2(wv), lo2(al));
+                        const float2 dh = mul2(hi2(wv), hi2(al));
                         wv = make_float4(dl.x, dl.y, dh.x, dh.y);
-                        next = ld_s4(kan + n * kDk + chunk_col(i, c));
+                        next = ld_s4(ka_s + (tp + 1) * chP + n * kDk + kStep * i);
                     }
                     const float2 lo = fma2(cf2, lo2(kv), lo2(wv));
                     const float2 hi = fma2(cf2, hi2(kv), hi2(wv));
                     w[n][i] = make_float4(lo.x, lo.y, hi.x, hi.y);
-                    o_lo[n] = fma2(lo, lo2(qv), o_lo[n]);
-                    o_hi[n] = fma2(hi, hi2(qv), o_hi[n]);
-                    a_lo[n] = fma2(lo, lo2(next), a_lo[n]);
-                    a_hi[n] = fma2(hi, hi2(next), a_hi[n]);
+                    if (i == 0) {
+                        o_lo[n] = mul2(lo, lo2(qv));
+                        o_hi[n] = mul2(hi, hi2(qv));
+                        a_lo[n] = mul2(lo, lo2(next));
+                        a_hi[n] = mul2(hi, hi2(next));
+                    } else {
+                        o_lo[n] = fma2(lo, lo2(qv), o_lo[n]);
+                        o_hi[n] = fma2(hi, hi2(qv), o_hi[n]);
+                        a_lo[n] = fma2(lo, lo2(next), a_lo[n]);
+                        a_hi[n] = fma2(hi, hi2(next), a_hi[n]);
+                    }
                 }
             }
             out_pending = true;
-            t_out = t;
+            out_prev = out_next;
+            out_next += out_stride;
         }
     }
     cp_async_wait<0>();
@@ -457,9 +504,11 @@ prefill_kernel(float* __restrict__ state, const float* __restrict__ q,
             float O[NH];
 #pragma unroll
             for (int n = 0; n < NH; ++n) O[n] = group_sum<kLPR>(sum4(o_lo[n], o_hi[n]));
+            float ov = O[0], so = s_out[0];
 #pragma unroll
-            for (int n = 0; n < NH; ++n)
-                if (c == (n & 3)) out_base[n][t_out * out_stride] = s_out[n] * O[n] * kOutScale;
+            for (int n = 1; n < NH; ++n)
+                if (c == n) { ov = O[n]; so = s_out[n]; }
+            if (c < NH) *out_prev = so * ov * kOutScale;
         }
         // the final state, scale folded in
 #pragma unroll
