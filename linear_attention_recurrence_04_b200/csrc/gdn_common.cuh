@@ -60,13 +60,15 @@ __device__ __forceinline__ void fold_step(T* v, int lane, int o) {
     }
 }
 
-// Sums each of the N values v[0..N-1] over the warp's 32 lanes (N a power of
-// two, at most 32) with N - 1 + log2(32 / N) shuffles instead of 5 N. Lane L
-// returns the total of value L >> (5 - log2 N).
-template <int N, typename T>
-__device__ __forceinline__ T warp_sum_many(T (&v)[N], int lane) {
-    static_assert(N >= 1 && N <= 32 && (N & (N - 1)) == 0, "N must be a power of two <= 32");
-    int o = 16;
+// Sums each of the N values v[0..N-1] over aligned groups of W lanes (N and W
+// powers of two, N <= W <= 32) with N - 1 + log2(W / N) shuffles instead of
+// N log2(W). Lane c of a group (c = lane % W) returns the total of value
+// c >> log2(W / N).
+template <int N, int W, typename T>
+__device__ __forceinline__ T group_sum_many(T (&v)[N], int lane) {
+    static_assert(N >= 1 && N <= W && W <= 32 && (N & (N - 1)) == 0 && (W & (W - 1)) == 0,
+                  "N and W must be powers of two with N <= W <= 32");
+    int o = W / 2;
     if constexpr (N >= 32) { fold_step<16>(v, lane, o); o >>= 1; }
     if constexpr (N >= 16) { fold_step<8>(v, lane, o); o >>= 1; }
     if constexpr (N >= 8) { fold_step<4>(v, lane, o); o >>= 1; }
@@ -75,6 +77,13 @@ __device__ __forceinline__ T warp_sum_many(T (&v)[N], int lane) {
     T s = v[0];
     for (; o >= 1; o >>= 1) s += __shfl_xor_sync(kFull, s, o);
     return s;
+}
+
+// The same over the whole warp: lane L returns the total of value
+// L >> (5 - log2 N).
+template <int N, typename T>
+__device__ __forceinline__ T warp_sum_many(T (&v)[N], int lane) {
+    return group_sum_many<N, 32>(v, lane);
 }
 
 // The lane that warp_sum_many<N> leaves value `i`'s total on.

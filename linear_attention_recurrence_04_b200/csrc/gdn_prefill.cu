@@ -10,11 +10,12 @@
 //  * The state never leaves the chip between positions. Row j of a head only
 //    needs k, q, v[j], beta and gate of each position, so a head's 128 x 128
 //    state splits into independent rows. A warp owns 8 rows of NH value heads
-//    that share one key head (h, h + Hk, ...): 4 lanes share a row, each
-//    holding a 32-column slice of each of its NH rows in registers, so each
-//    k/q value a lane reads serves NH rows; a row's dot products reduce over
-//    its 4 lanes with two shuffles. (Eight lanes per row, 16 columns each,
-//    doubles the resident warps but measured slower.)
+//    that share one key head (h, h + Hk, ...), held in registers: with the
+//    scalar decay 4 lanes share a row and each holds a 32-column slice of
+//    each of its NH rows, so each k/q value a lane reads serves NH rows; a
+//    row's dot products reduce over its 4 lanes with two shuffles. (Eight
+//    lanes per row, 16 columns each, doubles the resident warps but measured
+//    slower.) The per-channel decay uses the layout of struct Layout below.
 //  * Work balance: the warps ("units") are dealt to one CTA per SM in
 //    contiguous runs whose lengths differ by at most one, so every SM carries
 //    the same number of rows. A run covers at most two (sequence, key head,
@@ -42,22 +43,28 @@
 //    end, so the stored state has its ordinary meaning.
 //  * KDA ("Module linear_core", entry "kda_forward_batch"; the published Kimi
 //    Delta Attention update) is the same pipeline with a log-decay per key
-//    channel, g [B][T][Hv][dk]: no running scale, and each stage also carries
-//    alpha = exp(g) and alpha * k per value head, converted in place from the
-//    staged g one stage ahead (stages of 8 positions, so that two value heads
-//    per warp still fit). Per element and position:
+//    channel, g [B][T][Hv][dk]. Its running scale is per state column: column
+//    i of a head is held as W[.][i] with M[.][i] = S[i] W[.][i], so the decay
+//    is S *= alpha_t (per column, once per CTA and position, not per
+//    element), and with ks = S k, kd = k / S, qs = S q:
+//       sk = W.ks,  delta = (v - sk) beta,  W += delta kd,  out = W.qs,
+//    three FMAs per element and position as above. Each stage of 8 positions
+//    is converted in shared memory (convert_stage) from its staged g into
+//    ks, kd and qs. Where S times a stage's product of decays would leave
+//    [2^-40, 2^40], S is folded into W at the stage's start; where that
+//    product alone leaves the range (an underflowing decay, strong growth),
+//    the stage applies alpha element by element instead:
 //    W *= alpha_t, W += delta k_t, o += W q_t, a += W (alpha_{t+1} k_{t+1}).
+#include <type_traits>
+
 #include "gdn_common.cuh"
 #include "gdn_internal.h"
 
 #ifndef GDN_PREFILL_STAGES
-#define GDN_PREFILL_STAGES 4       // stages in flight (at least 3)
+#define GDN_PREFILL_STAGES 4       // stages in flight (at least 2)
 #endif
 #ifndef GDN_PREFILL_MAX_WARPS
 #define GDN_PREFILL_MAX_WARPS 8    // units (warps) per CTA at most
-#endif
-#ifndef GDN_PREFILL_LPR
-#define GDN_PREFILL_LPR 4          // lanes per state row (4 or 8)
 #endif
 #ifndef GDN_PREFILL_FMA2
 #define GDN_PREFILL_FMA2 1         // packed f32x2 FMAs for the per-element work
@@ -78,35 +85,63 @@ constexpr int kTSChannel = 8;                   // positions per stage (per-chan
 constexpr int kStages = GDN_PREFILL_STAGES;
 constexpr int kUnroll = GDN_PREFILL_UNROLL;        // positions per unrolled block
 constexpr int kMaxWarps = GDN_PREFILL_MAX_WARPS;
-constexpr int kLPR = GDN_PREFILL_LPR;           // lanes sharing one state row
-constexpr int kRowsPerUnit = 32 / kLPR;         // rows of a head per warp
+constexpr int kRowsPerUnit = 8;                 // rows of a head per warp
 constexpr int kUnitsPerHead = kDv / kRowsPerUnit;
-constexpr int kChunks = kDk / 4 / kLPR;         // float4 chunks per lane per row
 constexpr int kMaxGroups = 2;                   // groups one CTA's run can touch
 constexpr int kMaxRows = kMaxWarps * kRowsPerUnit;
 constexpr float kScaleLo = 0x1p-40f;
 constexpr float kScaleHi = 0x1p40f;
 static_assert(kMaxWarps <= kUnitsPerHead, "a run must span at most two groups");
-static_assert(kStages >= 3, "the pipeline reads one stage ahead");
-static_assert(kLPR == 4 || kLPR == 8, "4 or 8 lanes per row");
+static_assert(kStages >= 2, "at least double buffering");
+
+// Lane layout of a warp's 8 rows. Scalar decay: 4 lanes per row and one row
+// per lane, 32 columns each. Per-channel decay: 8 lanes per row group and two
+// rows per lane, 16 columns each, so that every staged vector value a lane
+// loads serves two rows; that kernel reads three vectors per head and is
+// bound by shared-memory wavefronts (a 16-byte load is served a quarter warp
+// per wavefront, whatever its broadcast).
+template <bool kCh>
+struct Layout {
+    static constexpr int LPR = kCh ? 8 : 4;        // lanes sharing a state row
+    static constexpr int RPL = kCh ? 2 : 1;        // state rows per lane
+    static constexpr int Chunks = kDk / 4 / LPR;   // float4 chunks per lane and row
+    static_assert(32 / LPR * RPL == kRowsPerUnit, "8 rows per warp");
+};
 
 // Shared-memory image of one stage. kCh (per-channel decay): alpha holds g
 // as copied, then exp(g); ka holds exp(g) * k. Without kCh both are stubs.
-// Slot TS of kq (k only) and of alpha / ka holds the first position of the
-// next stage, so a pass can always read the next key from its own stage.
+// Slot TS of kq (k only) holds the first position of the next stage, so a
+// pass always reads the next key from its own stage. kCh (per-channel decay)
+// adds, per value head: ks, the key-dot vectors (g as copied, then
+// converted, with slot TS as well), kd and qs, the update and output vectors,
+// mult, the scales folded into the state when the stage starts, and mode,
+// one word per group (kFold | kSlow). Without kCh those are stubs.
 template <int NH, bool kCh>
-struct Stage {
+struct alignas(16) Stage {    // stages sit back to back: each starts 16-byte aligned
     static constexpr int TS = kCh ? kTSChannel : kTS;   // positions per stage
+    static constexpr int CG = kCh ? kMaxGroups : 1;
+    static constexpr int CT = kCh ? TS : 1;
+    static constexpr int CD = kCh ? kDk : 4;
     float kq[kMaxGroups][TS + 1][2][kDk];      // [group][pos][k|q][col]
     float v[kMaxGroups][TS][NH][kMaxRows];     // rows [row_lo, row_lo + rows) of the group
     float bg[kMaxGroups][TS][NH][2];           // beta, gate
-    float alpha[kCh ? kMaxGroups : 1][kCh ? TS + 1 : 1][NH][kCh ? kDk : 4];
-    float ka[kCh ? kMaxGroups : 1][kCh ? TS + 1 : 1][NH][kCh ? kDk : 4];
+    float ks[CG][CT + 1][NH][CD];
+    float kd[CG][CT][NH][CD];
+    float qs[CG][CT][NH][CD];
+    float mult[CG][NH][CD];
+    int mode[kMaxGroups];
 };
 
-// Stages in flight: the per-channel stages carry more per position, so three.
+// Per-channel stage modes, one word per group: fold the column scales into
+// the state before the stage (kFold); apply the decays element by element
+// because a column's product of decays leaves [kScaleLo, kScaleHi] within
+// the stage (kSlow, always with kFold).
+constexpr int kFold = 1;
+constexpr int kSlow = 2;
+
+// Stages in flight: the per-channel stages carry more per position, so two.
 template <bool kCh>
-constexpr int stages_for() { return kCh ? 3 : kStages; }
+constexpr int stages_for() { return kCh ? 2 : kStages; }
 
 // One group of the CTA's run: (sequence b, key head g, head group grp) and the
 // rows of it that the run covers.
@@ -118,9 +153,10 @@ struct Group {
     int rows;
 };
 
-// Lane c of a row holds the float4 chunks {kLPR i + c}, so one warp-wide
-// 16-byte load of k or q touches 16 kLPR contiguous bytes.
-__device__ __forceinline__ int chunk_col(int i, int c) { return 4 * (kLPR * i + c); }
+// Lane c of a row holds the float4 chunks {LPR i + c}, so one warp-wide
+// 16-byte load of k or q touches 16 LPR contiguous bytes.
+template <int LPR>
+__device__ __forceinline__ int chunk_col(int i, int c) { return 4 * (LPR * i + c); }
 
 __device__ __forceinline__ void cp_async16(void* smem, const void* gmem) {
     const unsigned s = static_cast<unsigned>(__cvta_generic_to_shared(smem));
@@ -182,15 +218,21 @@ prefill_kernel(float* __restrict__ state, const float* __restrict__ q,
     constexpr int S = stages_for<kCh>();
     constexpr int TS = kCh ? kTSChannel : kTS;      // positions per stage
     using StageT = Stage<NH, kCh>;
+    constexpr int kLPR = Layout<kCh>::LPR;
+    constexpr int kRPL = Layout<kCh>::RPL;
+    constexpr int kChunks = Layout<kCh>::Chunks;
+    static_assert(sizeof(StageT) % 16 == 0, "16-byte copies and loads need aligned stages");
     extern __shared__ __align__(16) unsigned char smem_raw[];
     StageT* stages = reinterpret_cast<StageT*>(smem_raw);
     __shared__ Group grp_of[kMaxGroups];
+    // kCh: the running scale of each state column (see convert_stage)
+    __shared__ __align__(16) float s_col[kCh ? kMaxGroups : 1][NH][kCh ? kDk : 4];
 
     const int tid = threadIdx.x;
     const int nthreads = blockDim.x;
     const int warp = tid >> 5;
     const int lane = tid & 31;
-    const int p = lane / kLPR;                  // row within the warp's rows
+    const int p = lane / kLPR;                  // row group within the warp
     const int c = lane % kLPR;                  // column slice
 
     // This CTA's run of units: [u0, u0 + count).
@@ -215,11 +257,15 @@ prefill_kernel(float* __restrict__ state, const float* __restrict__ q,
         G.rows = static_cast<int>(last - first) * kRowsPerUnit;
         grp_of[tid] = G;
     }
+    if constexpr (kCh) {
+        for (int idx = tid; idx < kMaxGroups * NH * kDk; idx += nthreads) (&s_col[0][0][0])[idx] = 1.0f;
+    }
     __syncthreads();
 
     // ---- stage loader: every thread issues a share of the copies; positions
     //      at or past T are zero-filled ------------------------------------
     auto load_stage = [&](int64_t t0, StageT& st) {
+        if (kCh && tid < kMaxGroups) st.mode[tid] = 0;
 #pragma unroll
         for (int gi = 0; gi < kMaxGroups; ++gi) {
             if (gi >= n_groups) break;
@@ -269,7 +315,7 @@ prefill_kernel(float* __restrict__ state, const float* __restrict__ q,
                     const int n = (idx >> 5) % NH;
                     const int tp = (idx >> 5) / NH;
                     const int64_t t = t0 + tp;
-                    float* dst = &st.alpha[gi][tp][n][chunk * 4];
+                    float* dst = &st.ks[gi][tp][n][chunk * 4];
                     if (t < T) {
                         const int h = G.g + (G.grp * NH + n) * Hk;
                         cp_async16(dst, gate + ((G.b * T + t) * Hv + h) * kDk + chunk * 4);
@@ -280,37 +326,116 @@ prefill_kernel(float* __restrict__ state, const float* __restrict__ q,
             }
         }
     };
-    // kCh: alpha = exp(g) and ka = alpha * k of a landed stage, in place.
+    // kCh: turn a landed stage's g into the vectors of its passes. Column i
+    // of head n is held as W[j][i] with M[j][i] = S[i] W[j][i]; S (s_col)
+    // carries over between stages. A fast stage runs, per position t,
+    //   S <- S alpha_t,  ks_t = S k_t,  kd_t = k_t / S,  qs_t = S q_t,
+    // so that sk = W.ks_t, W += delta kd_t and out = W.qs_t (slot TS of ks:
+    // S alpha k of the next stage's first position). A slow stage keeps
+    // S = 1, stores kd_t = alpha_t and ks_t = alpha_t k_t, and its passes
+    // decay W element by element. Pass 1 flags each group: kFold when S
+    // times the stage's product of decays would leave [kScaleLo, kScaleHi],
+    // kSlow when that product alone does. Pass 2 writes the vectors.
     auto convert_stage = [&](StageT& st) {
         if constexpr (kCh) {
-            for (int gi2 = 0; gi2 < n_groups; ++gi2) {
-                for (int idx = tid; idx < (TS + 1) * NH * kDk; idx += nthreads) {
-                    const int col = idx % kDk;
-                    const int n = (idx / kDk) % NH;
-                    const int tp = idx / (kDk * NH);
-                    const float a = expf(st.alpha[gi2][tp][n][col]);
-                    st.alpha[gi2][tp][n][col] = a;
-                    st.ka[gi2][tp][n][col] = a * st.kq[gi2][tp][0][col];
+            const int ncols = n_groups * NH * kDk;
+            for (int idx = tid; idx < ncols; idx += nthreads) {
+                const int col = idx % kDk;
+                const int n = (idx / kDk) % NH;
+                const int gi2 = idx / (kDk * NH);
+                const float s0 = s_col[gi2][n][col];
+                float cum = 1.0f;
+                bool slow = false, fold = false;
+#pragma unroll
+                for (int tp = 0; tp <= TS; ++tp) {
+                    const float a = expf(st.ks[gi2][tp][n][col]);
+                    st.ks[gi2][tp][n][col] = a;
+                    if (tp < TS) {
+                        cum *= a;
+                        const float sc2 = s0 * cum;
+                        slow |= !(cum >= kScaleLo && cum <= kScaleHi);
+                        fold |= !(sc2 >= kScaleLo && sc2 <= kScaleHi);
+                    }
                 }
+                if (slow || fold) atomicOr(&st.mode[gi2], slow ? (kSlow | kFold) : kFold);
+            }
+            __syncthreads();
+            for (int idx = tid; idx < ncols; idx += nthreads) {
+                const int col = idx % kDk;
+                const int n = (idx / kDk) % NH;
+                const int gi2 = idx / (kDk * NH);
+                const int mode = st.mode[gi2];
+                float sv = s_col[gi2][n][col];
+                if (mode & kFold) {
+                    st.mult[gi2][n][col] = sv;
+                    sv = 1.0f;
+                }
+                if (mode & kSlow) {
+#pragma unroll
+                    for (int tp = 0; tp <= TS; ++tp) {
+                        const float a = st.ks[gi2][tp][n][col];
+                        if (tp < TS) st.kd[gi2][tp][n][col] = a;
+                        st.ks[gi2][tp][n][col] = a * st.kq[gi2][tp][0][col];
+                    }
+                } else {
+#pragma unroll
+                    for (int tp = 0; tp < TS; ++tp) {
+                        sv *= st.ks[gi2][tp][n][col];
+                        const float kv = st.kq[gi2][tp][0][col];
+                        st.ks[gi2][tp][n][col] = sv * kv;
+                        st.kd[gi2][tp][n][col] = kv * rcp_approx(sv);
+                        st.qs[gi2][tp][n][col] = sv * st.kq[gi2][tp][1][col];
+                    }
+                    st.ks[gi2][TS][n][col] = (sv * st.ks[gi2][TS][n][col]) * st.kq[gi2][TS][0][col];
+                }
+                s_col[gi2][n][col] = sv;
             }
         }
     };
 
     // ---- this warp's unit ------------------------------------------------
+    // Lane (p, c) holds rows j0 + r = rb * 8 + p * kRPL + r (r < kRPL) of
+    // the warp's NH value heads, columns chunk_col(i, c). Each position
+    // reduces the key dots A and output dots O of its (head, row) pairs over
+    // the row group's kLPR lanes.
+    //  * Scalar decay (one row per lane): every lane gets both heads' A and O
+    //    (two shuffles each) and forms both deltas; lane c < NH stores head
+    //    c's output.
+    //  * Per-channel decay: one halving reduction of all 2 NH kRPL values
+    //    leaves lane c with the total of value c >> kShift (values below
+    //    NH kRPL are the A of pair n kRPL + r, the rest the O of the same
+    //    pairs). A lane holding an A forms that pair's delta and the group
+    //    broadcasts it; a lane holding an O stores that output.
     const bool active = warp < count;
     const int64_t unit = u0 + warp;
     const int gi = active ? static_cast<int>(unit / kUnitsPerHead - gid0) : 0;
     const Group G = grp_of[gi];
     const int rb = static_cast<int>(unit % kUnitsPerHead);
-    const int j = rb * kRowsPerUnit + p;                 // row within the head
-    const int vrow = j - G.row_lo;                       // row within the staged v
+    const int j0 = rb * kRowsPerUnit + p * kRPL;         // first row within the head
     int hidx[NH];
 #pragma unroll
     for (int n = 0; n < NH; ++n) hidx[n] = G.g + (G.grp * NH + n) * Hk;
-    // Lane c < NH stores head c's outputs of row j; its pointer walks the
-    // positions (out_next: the coming position, out_prev: the pending one).
+    constexpr int kPairs = NH * kRPL;                    // (head, row) pairs per lane
+    constexpr int kVals = 2 * kPairs;                    // their A and O
+    static_assert(!kCh || kVals <= kLPR, "one reduced value per lane at least");
+    constexpr int kShift = (kLPR == 8 ? 3 : 2) - (kVals == 8 ? 3 : kVals == 4 ? 2 : 1);
+    const int grp_lane0 = lane & ~(kLPR - 1);
+    int my_n = c < NH ? c : 0, my_r = 0;                 // the pair this lane stores
+    bool my_store = c < NH;
+    if constexpr (kCh) {
+        const int my_val = c >> kShift;
+        const int my_pair = my_val < kPairs ? my_val : my_val - kPairs;
+        my_n = my_pair / kRPL;
+        my_r = my_pair % kRPL;
+        my_store = my_val >= kPairs && (c & ((1 << kShift) - 1)) == 0;
+    }
+    // staged v and beta: kCh, this lane's pair; otherwise row j0, head 0
+    const int my_v_off = kCh ? my_n * kMaxRows + (j0 + my_r - G.row_lo) : j0 - G.row_lo;
+    const int my_b_off = kCh ? 2 * my_n : 0;
+    // The pointer of this lane's output walks the positions (out_next: the
+    // coming position, out_prev: the pending one).
     const int64_t out_stride = static_cast<int64_t>(Hv) * kDv;
-    float* out_next = out + (G.b * T * Hv + G.g + (G.grp * NH + (c < NH ? c : 0)) * Hk) * kDv + j;
+    float* out_next = out + (G.b * T * Hv + G.g + (G.grp * NH + my_n) * Hk) * kDv + j0 + my_r;
     float* out_prev = out_next;
 
     // Prologue: request the first S - 1 stages, then load the state rows.
@@ -321,31 +446,36 @@ prefill_kernel(float* __restrict__ state, const float* __restrict__ q,
         cp_async_commit();
     }
 
-    float4 w[NH][kChunks];
+    float4 w[NH][kRPL][kChunks];
     float sc[NH];
     if (active) {
 #pragma unroll
         for (int n = 0; n < NH; ++n) {
-            const float* row = state + ((G.b * Hv + hidx[n]) * kDv + j) * kDk;
 #pragma unroll
-            for (int i = 0; i < kChunks; ++i) w[n][i] = ld_stream(row + chunk_col(i, c));
+            for (int r = 0; r < kRPL; ++r) {
+                const float* row = state + ((G.b * Hv + hidx[n]) * kDv + j0 + r) * kDk;
+#pragma unroll
+                for (int i = 0; i < kChunks; ++i) w[n][r][i] = ld_stream(row + chunk_col<kLPR>(i, c));
+            }
             sc[n] = 1.0f;
         }
     }
 
     // Loop-carried partial sums: a = W.k of the coming position, o = W.q of
     // the previous position (its store is pending), s_out = its scale.
-    float2 a_lo[NH], a_hi[NH], o_lo[NH], o_hi[NH];
+    float2 a_lo[NH][kRPL], a_hi[NH][kRPL], o_lo[NH][kRPL], o_hi[NH][kRPL];
     float s_out[NH];
 #pragma unroll
     for (int n = 0; n < NH; ++n) {
-        a_lo[n] = a_hi[n] = o_lo[n] = o_hi[n] = make_float2(0.f, 0.f);
+#pragma unroll
+        for (int r = 0; r < kRPL; ++r)
+            a_lo[n][r] = a_hi[n][r] = o_lo[n][r] = o_hi[n][r] = make_float2(0.f, 0.f);
         s_out[n] = 1.0f;
     }
     bool out_pending = false;
 
     for (int64_t s = 0; s < n_stages; ++s) {
-        cp_async_wait<S - 3>();             // this thread's copies of stages s, s+1 landed
+        cp_async_wait<S - 2>();             // this thread's copies of stage s landed
         __syncthreads();                     // ... and everyone's; stage s-1 is consumed
         {
             const int64_t nxt = s + S - 1;
@@ -353,10 +483,7 @@ prefill_kernel(float* __restrict__ state, const float* __restrict__ q,
             cp_async_commit();
         }
         if constexpr (kCh) {
-            // stage s+1 (and, first, stage 0) gets its decays before any warp
-            // reads its first key product for the next-position dot
-            if (s == 0) convert_stage(stages[0]);
-            if (s + 1 < n_stages) convert_stage(stages[(s + 1) % S]);
+            convert_stage(stages[s % S]);
             __syncthreads();
         }
         if (!active) continue;
@@ -364,161 +491,248 @@ prefill_kernel(float* __restrict__ state, const float* __restrict__ q,
         const int64_t t0 = s * TS;
         const int tp_end = (T - t0) < TS ? static_cast<int>(T - t0) : TS;
 
-        // decays of this stage, one per lane: lane tp + TS n holds exp(gate)
-        const float e_lane =
-            (!kCh && lane < TS * NH) ? expf(st.bg[gi][lane % TS][lane / TS][1]) : 1.0f;
-
         // This lane's view of the stage; position tp sits at tp * (stride).
         constexpr int kqP = 2 * kDk;            // k and q of one position
         constexpr int vP = NH * kMaxRows;       // v of one position
         constexpr int bgP = 2 * NH;             // beta, gate of one position
-        constexpr int chP = NH * kDk;           // alpha or alpha * k of one position
+        constexpr int chP = NH * kDk;           // ks, kd or qs of one position
         constexpr int kStep = 4 * kLPR;         // columns between a lane's chunks
-        const float* kq_s = &st.kq[gi][0][0][chunk_col(0, c)];    // k; q at + kDk
-        const float* v_s = &st.v[gi][0][0][vrow];
-        const float* bg_s = &st.bg[gi][0][0][0];
-        const float* al_s = &st.alpha[gi * kCh][0][0][kCh ? chunk_col(0, c) : 0];
-        const float* ka_s = &st.ka[gi * kCh][0][0][kCh ? chunk_col(0, c) : 0];
+        const int ccol = kCh ? chunk_col<kLPR>(0, c) : 0;
+        const float* kq_s = &st.kq[gi][0][0][chunk_col<kLPR>(0, c)];    // k; q at + kDk
+        const float* v_s = &st.v[gi][0][0][0] + my_v_off;      // see my_v_off
+        const float* bg_s = &st.bg[gi][0][0][0] + my_b_off;
+        const float* ks_s = &st.ks[gi * kCh][0][0][ccol];
+        const float* kd_s = &st.kd[gi * kCh][0][0][ccol];
+        const float* qs_s = &st.qs[gi * kCh][0][0][ccol];
 
-        if (s == 0) {
-            // first key dot: a = W.k_0 (kCh: with alpha_0 folded into k_0)
-#pragma unroll
-            for (int i = 0; i < kChunks; ++i) {
+        // decays of this stage, one per lane: lane tp + TS n holds exp(gate)
+        const float e_lane =
+            (!kCh && lane < TS * NH) ? expf(st.bg[gi][lane % TS][lane / TS][1]) : 1.0f;
+
+        int mode = 0;
+        if constexpr (kCh) {
+            mode = st.mode[gi];
+            if (mode & kFold) {             // M = S W per column: fold S into W
 #pragma unroll
                 for (int n = 0; n < NH; ++n) {
-                    const float4 kv = kCh ? ld_s4(ka_s + n * kDk + kStep * i)
-                                          : ld_s4(kq_s + kStep * i);
-                    a_lo[n] = fma2(lo2(w[n][i]), lo2(kv), a_lo[n]);
-                    a_hi[n] = fma2(hi2(w[n][i]), hi2(kv), a_hi[n]);
-                }
-            }
-        }
-
-#pragma unroll(kUnroll)
-        for (int tp = 0; tp < TS; ++tp) {
-            if (tp >= tp_end) break;
-            // (a) batched reductions: sk of t, and out of t-1
-            float A[NH], O[NH];
 #pragma unroll
-            for (int n = 0; n < NH; ++n) {
-                A[n] = sum4(a_lo[n], a_hi[n]);
-                O[n] = sum4(o_lo[n], o_hi[n]);
-            }
+                    for (int i = 0; i < kChunks; ++i) {
+                        const float4 m = ld_s4(&st.mult[gi][n][ccol + kStep * i]);
 #pragma unroll
-            for (int n = 0; n < NH; ++n) {
-                A[n] = group_sum<kLPR>(A[n]);
-                O[n] = group_sum<kLPR>(O[n]);
-            }
-            {   // lane c < NH stores head c's output of t - 1
-                float ov = O[0], so = s_out[0];
-#pragma unroll
-                for (int n = 1; n < NH; ++n)
-                    if (c == n) { ov = O[n]; so = s_out[n]; }
-                if (out_pending && c < NH) *out_prev = so * ov * kOutScale;
-            }
-            // (b) scalar part of position t
-            float cf[NH];
-            if constexpr (kCh) {
-#pragma unroll
-                for (int n = 0; n < NH; ++n)
-                    cf[n] = (v_s[tp * vP + n * kMaxRows] - A[n]) * bg_s[tp * bgP + 2 * n];
-            } else {
-                // step 1 as a scale update s *= e; then, with r = 1 / s,
-                // delta / s = (v r - W.k) beta (steps 2-3)
-                float s_new[NH];
-                bool fold = false;
-#pragma unroll
-                for (int n = 0; n < NH; ++n) {
-                    s_new[n] = sc[n] * __shfl_sync(kFull, e_lane, tp + TS * n);
-                    fold |= !(s_new[n] >= kScaleLo && s_new[n] <= kScaleHi);
-                }
-                if (fold) {          // rare, and uniform across the warp
-#pragma unroll
-                    for (int n = 0; n < NH; ++n) {
-                        if (!(s_new[n] >= kScaleLo && s_new[n] <= kScaleHi)) {
-#pragma unroll
-                            for (int i = 0; i < kChunks; ++i) {
-                                w[n][i].x *= s_new[n]; w[n][i].y *= s_new[n];
-                                w[n][i].z *= s_new[n]; w[n][i].w *= s_new[n];
-                            }
-                            A[n] *= s_new[n];
-                            s_new[n] = 1.0f;
+                        for (int r = 0; r < kRPL; ++r) {
+                            const float2 l = mul2(lo2(w[n][r][i]), lo2(m));
+                            const float2 h = mul2(hi2(w[n][r][i]), hi2(m));
+                            w[n][r][i] = make_float4(l.x, l.y, h.x, h.y);
                         }
                     }
                 }
-#pragma unroll
-                for (int n = 0; n < NH; ++n) {
-                    sc[n] = s_new[n];
-                    s_out[n] = s_new[n];
-                    cf[n] = fmaf(v_s[tp * vP + n * kMaxRows], rcp_approx(s_new[n]), -A[n]) *
-                            bg_s[tp * bgP + 2 * n];
-                }
             }
-            // (c) one pass: step 4 for t, then W.q_t (step 5) and W.k_{t+1}
-            // (kCh: step 1 per channel first, and the next key with its decay).
-            // Slot tp + 1 always exists; past T it is zero-filled.
-            const float* kp = kq_s + tp * kqP;
+        }
+
+        if (s == 0) {
+            // first key dot: a = W.k_0 (kCh: W.ks_0, the decayed key)
 #pragma unroll
             for (int i = 0; i < kChunks; ++i) {
-                const float4 kv = ld_s4(kp + kStep * i);
-                const float4 qv = ld_s4(kp + kDk + kStep * i);
-                const float4 nv = kCh ? kv : ld_s4(kp + kqP + kStep * i);
 #pragma unroll
                 for (int n = 0; n < NH; ++n) {
-                    const float2 cf2 = make_float2(cf[n], cf[n]);
-                    float4 wv = w[n][i];
-                    float4 next = nv;
-                    if constexpr (kCh) {
-                        const float4 al = ld_s4(al_s + tp * chP + n * kDk + kStep * i);
-                        const float2 dl = mul2(lo2(wv), lo2(al));
-                        const float2 dh = mul2(hi2(wv), hi2(al));
-                        wv = make_float4(dl.x, dl.y, dh.x, dh.y);
-                        next = ld_s4(ka_s + (tp + 1) * chP + n * kDk + kStep * i);
-                    }
-                    const float2 lo = fma2(cf2, lo2(kv), lo2(wv));
-                    const float2 hi = fma2(cf2, hi2(kv), hi2(wv));
-                    w[n][i] = make_float4(lo.x, lo.y, hi.x, hi.y);
-                    if (i == 0) {
-                        o_lo[n] = mul2(lo, lo2(qv));
-                        o_hi[n] = mul2(hi, hi2(qv));
-                        a_lo[n] = mul2(lo, lo2(next));
-                        a_hi[n] = mul2(hi, hi2(next));
-                    } else {
-                        o_lo[n] = fma2(lo, lo2(qv), o_lo[n]);
-                        o_hi[n] = fma2(hi, hi2(qv), o_hi[n]);
-                        a_lo[n] = fma2(lo, lo2(next), a_lo[n]);
-                        a_hi[n] = fma2(hi, hi2(next), a_hi[n]);
+                    const float4 kv = kCh ? ld_s4(ks_s + n * kDk + kStep * i)
+                                          : ld_s4(kq_s + kStep * i);
+#pragma unroll
+                    for (int r = 0; r < kRPL; ++r) {
+                        a_lo[n][r] = fma2(lo2(w[n][r][i]), lo2(kv), a_lo[n][r]);
+                        a_hi[n][r] = fma2(hi2(w[n][r][i]), hi2(kv), a_hi[n][r]);
                     }
                 }
             }
-            out_pending = true;
-            out_prev = out_next;
-            out_next += out_stride;
         }
+
+        // The positions of the stage. kSlowPath (kCh only): decay element by
+        // element with kd = alpha, update with k, output with q, next key
+        // dot with ks = alpha k.
+        auto positions = [&](auto slow_tag) {
+            constexpr bool kSlowPath = decltype(slow_tag)::value;
+#pragma unroll(kUnroll)
+            for (int tp = 0; tp < TS; ++tp) {
+                if (tp >= tp_end) break;
+                float cf[NH][kRPL];
+                if constexpr (!kCh) {
+                    // (a) batched reductions: sk of t, and out of t-1
+                    float A[NH], O[NH];
+#pragma unroll
+                    for (int n = 0; n < NH; ++n) {
+                        A[n] = sum4(a_lo[n][0], a_hi[n][0]);
+                        O[n] = sum4(o_lo[n][0], o_hi[n][0]);
+                    }
+#pragma unroll
+                    for (int n = 0; n < NH; ++n) {
+                        A[n] = group_sum<kLPR>(A[n]);
+                        O[n] = group_sum<kLPR>(O[n]);
+                    }
+                    {   // lane c < NH stores head c's output of t - 1
+                        float ov = O[0], so = s_out[0];
+#pragma unroll
+                        for (int n = 1; n < NH; ++n)
+                            if (c == n) { ov = O[n]; so = s_out[n]; }
+                        if (out_pending && my_store) *out_prev = so * ov * kOutScale;
+                    }
+                    // (b) step 1 as a scale update s *= e; then, with
+                    // r = 1 / s, delta / s = (v r - W.k) beta (steps 2-3)
+                    float s_new[NH];
+                    bool fold = false;
+#pragma unroll
+                    for (int n = 0; n < NH; ++n) {
+                        s_new[n] = sc[n] * __shfl_sync(kFull, e_lane, tp + TS * n);
+                        fold |= !(s_new[n] >= kScaleLo && s_new[n] <= kScaleHi);
+                    }
+                    if (fold) {          // rare, and uniform across the warp
+#pragma unroll
+                        for (int n = 0; n < NH; ++n) {
+                            if (!(s_new[n] >= kScaleLo && s_new[n] <= kScaleHi)) {
+#pragma unroll
+                                for (int i = 0; i < kChunks; ++i) {
+                                    w[n][0][i].x *= s_new[n]; w[n][0][i].y *= s_new[n];
+                                    w[n][0][i].z *= s_new[n]; w[n][0][i].w *= s_new[n];
+                                }
+                                A[n] *= s_new[n];
+                                s_new[n] = 1.0f;
+                            }
+                        }
+                    }
+#pragma unroll
+                    for (int n = 0; n < NH; ++n) {
+                        sc[n] = s_new[n];
+                        s_out[n] = s_new[n];
+                        cf[n][0] = fmaf(v_s[tp * vP + n * kMaxRows], rcp_approx(s_new[n]), -A[n]) *
+                                   bg_s[tp * bgP + 2 * n];
+                    }
+                } else {
+                    // (a) one halving reduction: sk of t and out of t-1 for
+                    // every pair
+                    float vals[kVals];
+#pragma unroll
+                    for (int n = 0; n < NH; ++n) {
+#pragma unroll
+                        for (int r = 0; r < kRPL; ++r) {
+                            vals[n * kRPL + r] = sum4(a_lo[n][r], a_hi[n][r]);
+                            vals[kPairs + n * kRPL + r] = sum4(o_lo[n][r], o_hi[n][r]);
+                        }
+                    }
+                    const float tot = group_sum_many<kVals, kLPR>(vals, lane);
+                    if (out_pending && my_store) *out_prev = tot * kOutScale;
+                    // (b) the key dot carries the column scales, so tot is sk
+                    // itself: this lane's pair's delta, then the broadcast
+                    const float cf_mine = (v_s[tp * vP] - tot) * bg_s[tp * bgP];
+#pragma unroll
+                    for (int n = 0; n < NH; ++n) {
+#pragma unroll
+                        for (int r = 0; r < kRPL; ++r)
+                            cf[n][r] = __shfl_sync(kFull, cf_mine,
+                                                   grp_lane0 + ((n * kRPL + r) << kShift));
+                    }
+                }
+                // (c) one pass: step 4 for t, then W.q_t (step 5) and the next
+                // position's key dot. Slot tp + 1 always exists; past T it is
+                // zero-filled.
+                const float* kp = kq_s + tp * kqP;
+#pragma unroll
+                for (int i = 0; i < kChunks; ++i) {
+                    float4 kv_sh = make_float4(0.f, 0.f, 0.f, 0.f), qv_sh = kv_sh, nv_sh = kv_sh;
+                    if constexpr (!kCh || kSlowPath) {
+                        kv_sh = ld_s4(kp + kStep * i);
+                        qv_sh = ld_s4(kp + kDk + kStep * i);
+                    }
+                    if constexpr (!kCh) nv_sh = ld_s4(kp + kqP + kStep * i);
+#pragma unroll
+                    for (int n = 0; n < NH; ++n) {
+                        float4 uv = kv_sh, qv = qv_sh, nv = nv_sh, al = kv_sh;
+                        if constexpr (kCh) {
+                            const int off = tp * chP + n * kDk + kStep * i;
+                            nv = ld_s4(ks_s + off + chP);
+                            if constexpr (kSlowPath) {
+                                al = ld_s4(kd_s + off);
+                            } else {
+                                uv = ld_s4(kd_s + off);
+                                qv = ld_s4(qs_s + off);
+                            }
+                        }
+#pragma unroll
+                        for (int r = 0; r < kRPL; ++r) {
+                            float4 wv = w[n][r][i];
+                            if constexpr (kCh && kSlowPath) {
+                                const float2 dl = mul2(lo2(wv), lo2(al));
+                                const float2 dh = mul2(hi2(wv), hi2(al));
+                                wv = make_float4(dl.x, dl.y, dh.x, dh.y);
+                            }
+                            const float2 cf2 = make_float2(cf[n][r], cf[n][r]);
+                            const float2 lo = fma2(cf2, lo2(uv), lo2(wv));
+                            const float2 hi = fma2(cf2, hi2(uv), hi2(wv));
+                            w[n][r][i] = make_float4(lo.x, lo.y, hi.x, hi.y);
+                            if (i == 0) {
+                                o_lo[n][r] = mul2(lo, lo2(qv));
+                                o_hi[n][r] = mul2(hi, hi2(qv));
+                                a_lo[n][r] = mul2(lo, lo2(nv));
+                                a_hi[n][r] = mul2(hi, hi2(nv));
+                            } else {
+                                o_lo[n][r] = fma2(lo, lo2(qv), o_lo[n][r]);
+                                o_hi[n][r] = fma2(hi, hi2(qv), o_hi[n][r]);
+                                a_lo[n][r] = fma2(lo, lo2(nv), a_lo[n][r]);
+                                a_hi[n][r] = fma2(hi, hi2(nv), a_hi[n][r]);
+                            }
+                        }
+                    }
+                }
+                out_pending = true;
+                out_prev = out_next;
+                out_next += out_stride;
+            }
+        };
+        if (kCh && (mode & kSlow)) positions(std::true_type{});
+        else positions(std::false_type{});
     }
     cp_async_wait<0>();
 
     if (active) {
         // the last position's output
         if (out_pending) {
-            float O[NH];
+            if constexpr (!kCh) {
+                float ov = 0.0f, so = s_out[0];
 #pragma unroll
-            for (int n = 0; n < NH; ++n) O[n] = group_sum<kLPR>(sum4(o_lo[n], o_hi[n]));
-            float ov = O[0], so = s_out[0];
+                for (int n = 0; n < NH; ++n) {
+                    const float O = group_sum<kLPR>(sum4(o_lo[n][0], o_hi[n][0]));
+                    if (c == n) { ov = O; so = s_out[n]; }
+                }
+                if (my_store) *out_prev = so * ov * kOutScale;
+            } else {
+                float vals[kVals];
 #pragma unroll
-            for (int n = 1; n < NH; ++n)
-                if (c == n) { ov = O[n]; so = s_out[n]; }
-            if (c < NH) *out_prev = so * ov * kOutScale;
+                for (int n = 0; n < NH; ++n) {
+#pragma unroll
+                    for (int r = 0; r < kRPL; ++r) {
+                        vals[n * kRPL + r] = 0.0f;
+                        vals[kPairs + n * kRPL + r] = sum4(o_lo[n][r], o_hi[n][r]);
+                    }
+                }
+                const float tot = group_sum_many<kVals, kLPR>(vals, lane);
+                if (my_store) *out_prev = tot * kOutScale;
+            }
         }
-        // the final state, scale folded in
+        // the final state, scale folded in (kCh: the column scales)
 #pragma unroll
         for (int n = 0; n < NH; ++n) {
-            float* row = state + ((G.b * Hv + hidx[n]) * kDv + j) * kDk;
 #pragma unroll
-            for (int i = 0; i < kChunks; ++i) {
-                float4 x = w[n][i];
-                x.x *= sc[n]; x.y *= sc[n]; x.z *= sc[n]; x.w *= sc[n];
-                st_stream(row + chunk_col(i, c), x);
+            for (int r = 0; r < kRPL; ++r) {
+                float* row = state + ((G.b * Hv + hidx[n]) * kDv + j0 + r) * kDk;
+#pragma unroll
+                for (int i = 0; i < kChunks; ++i) {
+                    float4 x = w[n][r][i];
+                    if constexpr (kCh) {
+                        const float4 m = ld_s4(&s_col[gi][n][chunk_col<kLPR>(i, c)]);
+                        x.x *= m.x; x.y *= m.y; x.z *= m.z; x.w *= m.w;
+                    } else {
+                        x.x *= sc[n]; x.y *= sc[n]; x.z *= sc[n]; x.w *= sc[n];
+                    }
+                    st_stream(row + chunk_col<kLPR>(i, c), x);
+                }
             }
         }
     }

@@ -132,3 +132,40 @@ def test_kda_prefill_resume_matches_one_pass(o):
     st_ref, out_ref = o.kda_prefill(d["state"], d["q"], d["k"], d["v"], d["beta"], d["g"])
     assert_parity(torch.cat([o1, o2], dim=1).cpu().numpy(), out_ref, "kda resume out")
     assert_parity(t["state"].cpu().numpy(), st_ref, "kda resume state")
+
+
+def test_kda_prefill_decay_extremes(o):
+    """Channels with g = -200 (exp underflows to 0) at some positions, g = 0,
+    and two positions of growth (g = +1) in one 61-position call: stages whose
+    product of decays leaves the running scale's range take the per-element
+    path, and the others resume after them. (Growth of e^6 instead of e^2
+    puts plain sequential fp32 arithmetic itself at 8e-5 relative error on
+    this input, too close to the bound to test anything.)"""
+    d = inputs.kda_prefill_inputs(2, 61, Hk=4, Hv=8, seed=1650, state_std=0.05)
+    g = d["g"].copy()
+    g[:, 10:13, :, 0::3] = -200.0
+    g[:, 20:30, :, 1::3] = 0.0
+    g[:, 40, :, 2::5] = 1.0
+    g[:, 41, :, 2::5] = 1.0
+    d["g"] = g
+    st_ref, out_ref = o.kda_prefill(d["state"], d["q"], d["k"], d["v"], d["beta"], d["g"])
+    st, out = gpu_prefill(d)
+    assert_parity(out, out_ref, "kda extremes prefill out")
+    assert_parity(st, st_ref, "kda extremes prefill state")
+
+
+@pytest.mark.parametrize("g_low,g_high", [(-4.0, -2.0), (-8.0, -5.0), (-1.0, -0.5)])
+def test_kda_prefill_strong_decay(o, g_low, g_high):
+    """Decays strong enough that the column scales fold into the state every
+    stage or two (U(-4, -2)), that a stage's own product underflows the
+    scale range (U(-8, -5)), and a fold every few stages (U(-1, -0.5)),
+    over 100 positions. (Nearly no decay over 100 positions, U(-0.05, 0),
+    leaves plain sequential fp32 arithmetic at 1.2e-4 relative error on
+    state elements just above 1e-3: beyond the bound for any fp32 order.)"""
+    d = inputs.kda_prefill_inputs(1, 100, Hk=2, Hv=4, seed=1660, state_std=0.05)
+    r = np.random.default_rng(1661)
+    d["g"] = r.uniform(g_low, g_high, d["g"].shape).astype(np.float32)
+    st_ref, out_ref = o.kda_prefill(d["state"], d["q"], d["k"], d["v"], d["beta"], d["g"])
+    st, out = gpu_prefill(d)
+    assert_parity(out, out_ref, f"kda g U({g_low},{g_high}) out")
+    assert_parity(st, st_ref, f"kda g U({g_low},{g_high}) state")
