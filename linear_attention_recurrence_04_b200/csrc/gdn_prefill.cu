@@ -749,7 +749,9 @@ cudaError_t launch_nh(const PrefillArgs& a, cudaStream_t stream) {
     if (grid < min_grid) grid = min_grid;
     const int units_lo = static_cast<int>(n_units / grid);
     const int n_big = static_cast<int>(n_units % grid);
-    const int warps = units_lo + (n_big > 0 ? 1 : 0);
+    // Per-channel decay: every CTA runs kMaxWarps warps (those past its run
+    // hold no rows) so that the per-stage conversion spreads evenly.
+    const int warps = kCh ? kMaxWarps : units_lo + (n_big > 0 ? 1 : 0);
     const size_t smem = sizeof(Stage<NH, kCh>) * stages_for<kCh>();
     cudaError_t err = cudaFuncSetAttribute(prefill_kernel<NH, kCh>,
                                            cudaFuncAttributeMaxDynamicSharedMemorySize,
