@@ -44,7 +44,7 @@
 #include "gdn_internal.h"
 
 #ifndef GDN_LAYER_MIN_CTAS
-#define GDN_LAYER_MIN_CTAS 3       // resident CTAs per SM the register budget targets
+#define GDN_LAYER_MIN_CTAS 0       // resident CTAs per SM the register budget targets (0: per variant)
 #endif
 #ifndef GDN_LAYER_ROWS
 #define GDN_LAYER_ROWS 4           // state rows per warp task
@@ -92,8 +92,17 @@ __device__ __forceinline__ double dot_fd(float4 a, const D4& b) {
 // NPOS = 1: one token, ring and state updated in place.
 // NPOS = 2: position 0 commits into conv_ring/state, position 1 continues
 //           into scratch_ring/scratch_state. Activations are [B][NPOS][...].
+// Resident CTAs per SM that the register budget targets. One position with
+// two or more value heads per key head fits four CTAs (64 registers) without
+// spilling, so more CTAs overlap their prestate / rows / tail phases (measured
+// 187.5 us against 195.1 us at B = 256); the two-position verify spills at 64
+// registers (462 us against 308 us), so it keeps three.
+constexpr int layer_min_ctas(int g, int npos) {
+    return GDN_LAYER_MIN_CTAS ? GDN_LAYER_MIN_CTAS : (npos == 1 && g >= 2) ? 4 : 3;
+}
+
 template <int G, int R, int NPOS>
-__global__ void __launch_bounds__(kLayerThreads, GDN_LAYER_MIN_CTAS)
+__global__ void __launch_bounds__(kLayerThreads, layer_min_ctas(G, NPOS))
 layer_kernel(const float* __restrict__ mixed_qkv, const float* __restrict__ z,
              const float* __restrict__ a_in, const float* __restrict__ b_in,
              float* __restrict__ conv_ring, const float* __restrict__ conv_w,
