@@ -63,8 +63,8 @@
 #ifndef GDN_PREFILL_STAGES
 #define GDN_PREFILL_STAGES 4       // stages in flight (at least 2)
 #endif
-#ifndef GDN_PREFILL_MAX_WARPS
-#define GDN_PREFILL_MAX_WARPS 8    // units (warps) per CTA at most
+#ifndef GDN_PREFILL_GDN_LPR
+#define GDN_PREFILL_GDN_LPR 4      // scalar decay: lanes per state row (4 or 8)
 #endif
 #ifndef GDN_PREFILL_FMA2
 #define GDN_PREFILL_FMA2 1         // packed f32x2 FMAs for the per-element work
@@ -84,14 +84,10 @@ constexpr int kTS = 16;                         // positions per stage (scalar d
 constexpr int kTSChannel = 8;                   // positions per stage (per-channel decay)
 constexpr int kStages = GDN_PREFILL_STAGES;
 constexpr int kUnroll = GDN_PREFILL_UNROLL;        // positions per unrolled block
-constexpr int kMaxWarps = GDN_PREFILL_MAX_WARPS;
-constexpr int kRowsPerUnit = 8;                 // rows of a head per warp
-constexpr int kUnitsPerHead = kDv / kRowsPerUnit;
 constexpr int kMaxGroups = 2;                   // groups one CTA's run can touch
-constexpr int kMaxRows = kMaxWarps * kRowsPerUnit;
+constexpr int kMaxRows = 64;                    // rows of one group a CTA holds at most
 constexpr float kScaleLo = 0x1p-40f;
 constexpr float kScaleHi = 0x1p40f;
-static_assert(kMaxWarps <= kUnitsPerHead, "a run must span at most two groups");
 static_assert(kStages >= 2, "at least double buffering");
 
 // Lane layout of a warp's 8 rows. Scalar decay: 4 lanes per row and one row
@@ -102,10 +98,17 @@ static_assert(kStages >= 2, "at least double buffering");
 // per wavefront, whatever its broadcast).
 template <bool kCh>
 struct Layout {
-    static constexpr int LPR = kCh ? 8 : 4;        // lanes sharing a state row
-    static constexpr int RPL = kCh ? 2 : 1;        // state rows per lane
-    static constexpr int Chunks = kDk / 4 / LPR;   // float4 chunks per lane and row
-    static_assert(32 / LPR * RPL == kRowsPerUnit, "8 rows per warp");
+    static constexpr int LPR = kCh ? 8 : GDN_PREFILL_GDN_LPR;   // lanes sharing a state row
+    static constexpr int RPL = kCh ? 2 : 1;                     // state rows per lane
+    static constexpr int Chunks = kDk / 4 / LPR;                // float4 chunks per lane and row
+    static constexpr int RowsPerUnit = 32 / LPR * RPL;          // rows of a head per warp
+    static constexpr int UnitsPerHead = kDv / RowsPerUnit;
+    static constexpr int MaxWarps = kMaxRows / RowsPerUnit;     // warps (units) per CTA at most
+    // One halving reduction of all key and output dots with the deltas
+    // broadcast, rather than a full reduction of each on every lane.
+    static constexpr bool Halving = kCh || LPR == 8;
+    static_assert(LPR == 4 || LPR == 8, "4 or 8 lanes per row");
+    static_assert(MaxWarps <= UnitsPerHead, "a run must span at most two groups");
 };
 
 // Shared-memory image of one stage. kCh (per-channel decay): alpha holds g
@@ -209,7 +212,7 @@ __device__ __forceinline__ float rcp_approx(float x) {
 }
 
 template <int NH, bool kCh>
-__global__ void __launch_bounds__(32 * kMaxWarps, 1)
+__global__ void __launch_bounds__(32 * Layout<kCh>::MaxWarps, 1)
 prefill_kernel(float* __restrict__ state, const float* __restrict__ q,
                const float* __restrict__ k, const float* __restrict__ v,
                const float* __restrict__ beta, const float* __restrict__ gate,
@@ -221,6 +224,9 @@ prefill_kernel(float* __restrict__ state, const float* __restrict__ q,
     constexpr int kLPR = Layout<kCh>::LPR;
     constexpr int kRPL = Layout<kCh>::RPL;
     constexpr int kChunks = Layout<kCh>::Chunks;
+    constexpr int kRowsPerUnit = Layout<kCh>::RowsPerUnit;
+    constexpr int kUnitsPerHead = Layout<kCh>::UnitsPerHead;
+    constexpr bool kHalving = Layout<kCh>::Halving;
     static_assert(sizeof(StageT) % 16 == 0, "16-byte copies and loads need aligned stages");
     extern __shared__ __align__(16) unsigned char smem_raw[];
     StageT* stages = reinterpret_cast<StageT*>(smem_raw);
@@ -398,14 +404,14 @@ prefill_kernel(float* __restrict__ state, const float* __restrict__ q,
     // the warp's NH value heads, columns chunk_col(i, c). Each position
     // reduces the key dots A and output dots O of its (head, row) pairs over
     // the row group's kLPR lanes.
-    //  * Scalar decay (one row per lane): every lane gets both heads' A and O
-    //    (two shuffles each) and forms both deltas; lane c < NH stores head
+    //  * Four lanes per row (scalar decay): every lane gets both heads' A and
+    //    O (two shuffles each) and forms both deltas; lane c < NH stores head
     //    c's output.
-    //  * Per-channel decay: one halving reduction of all 2 NH kRPL values
-    //    leaves lane c with the total of value c >> kShift (values below
-    //    NH kRPL are the A of pair n kRPL + r, the rest the O of the same
-    //    pairs). A lane holding an A forms that pair's delta and the group
-    //    broadcasts it; a lane holding an O stores that output.
+    //  * Eight lanes per row group (kHalving): one halving reduction of all
+    //    2 NH kRPL values leaves lane c with the total of value c >> kShift
+    //    (values below NH kRPL are the A of pair n kRPL + r, the rest the O of
+    //    the same pairs). A lane holding an A forms that pair's delta and the
+    //    group broadcasts it; a lane holding an O stores that output.
     const bool active = warp < count;
     const int64_t unit = u0 + warp;
     const int gi = active ? static_cast<int>(unit / kUnitsPerHead - gid0) : 0;
@@ -417,21 +423,21 @@ prefill_kernel(float* __restrict__ state, const float* __restrict__ q,
     for (int n = 0; n < NH; ++n) hidx[n] = G.g + (G.grp * NH + n) * Hk;
     constexpr int kPairs = NH * kRPL;                    // (head, row) pairs per lane
     constexpr int kVals = 2 * kPairs;                    // their A and O
-    static_assert(!kCh || kVals <= kLPR, "one reduced value per lane at least");
+    static_assert(!kHalving || kVals <= kLPR, "one reduced value per lane at least");
     constexpr int kShift = (kLPR == 8 ? 3 : 2) - (kVals == 8 ? 3 : kVals == 4 ? 2 : 1);
     const int grp_lane0 = lane & ~(kLPR - 1);
     int my_n = c < NH ? c : 0, my_r = 0;                 // the pair this lane stores
     bool my_store = c < NH;
-    if constexpr (kCh) {
+    if constexpr (kHalving) {
         const int my_val = c >> kShift;
         const int my_pair = my_val < kPairs ? my_val : my_val - kPairs;
         my_n = my_pair / kRPL;
         my_r = my_pair % kRPL;
         my_store = my_val >= kPairs && (c & ((1 << kShift) - 1)) == 0;
     }
-    // staged v and beta: kCh, this lane's pair; otherwise row j0, head 0
-    const int my_v_off = kCh ? my_n * kMaxRows + (j0 + my_r - G.row_lo) : j0 - G.row_lo;
-    const int my_b_off = kCh ? 2 * my_n : 0;
+    // staged v and beta: kHalving, this lane's pair; otherwise row j0, head 0
+    const int my_v_off = kHalving ? my_n * kMaxRows + (j0 + my_r - G.row_lo) : j0 - G.row_lo;
+    const int my_b_off = kHalving ? 2 * my_n : 0;
     // The pointer of this lane's output walks the positions (out_next: the
     // coming position, out_prev: the pending one).
     const int64_t out_stride = static_cast<int64_t>(Hv) * kDv;
@@ -555,7 +561,7 @@ prefill_kernel(float* __restrict__ state, const float* __restrict__ q,
             for (int tp = 0; tp < TS; ++tp) {
                 if (tp >= tp_end) break;
                 float cf[NH][kRPL];
-                if constexpr (!kCh) {
+                if constexpr (!kHalving) {
                     // (a) batched reductions: sk of t, and out of t-1
                     float A[NH], O[NH];
 #pragma unroll
@@ -617,11 +623,54 @@ prefill_kernel(float* __restrict__ state, const float* __restrict__ q,
                             vals[kPairs + n * kRPL + r] = sum4(o_lo[n][r], o_hi[n][r]);
                         }
                     }
-                    const float tot = group_sum_many<kVals, kLPR>(vals, lane);
-                    if (out_pending && my_store) *out_prev = tot * kOutScale;
-                    // (b) the key dot carries the column scales, so tot is sk
-                    // itself: this lane's pair's delta, then the broadcast
-                    const float cf_mine = (v_s[tp * vP] - tot) * bg_s[tp * bgP];
+                    float tot = group_sum_many<kVals, kLPR>(vals, lane);
+                    float so = s_out[0];
+#pragma unroll
+                    for (int n = 1; n < NH; ++n)
+                        if (my_n == n) so = s_out[n];
+                    if (out_pending && my_store) *out_prev = so * tot * kOutScale;
+                    // (b) this lane's pair's delta, then the broadcast
+                    float cf_mine;
+                    if constexpr (kCh) {
+                        // the key dot carries the column scales: tot is sk
+                        cf_mine = (v_s[tp * vP] - tot) * bg_s[tp * bgP];
+                    } else {
+                        // step 1 as a scale update s *= e (every lane keeps
+                        // both heads' scales); then, with r = 1 / s,
+                        // delta / s = (v r - W.k) beta (steps 2-3)
+                        float s_new[NH];
+                        bool fold = false;
+#pragma unroll
+                        for (int n = 0; n < NH; ++n) {
+                            s_new[n] = sc[n] * __shfl_sync(kFull, e_lane, tp + TS * n);
+                            fold |= !(s_new[n] >= kScaleLo && s_new[n] <= kScaleHi);
+                        }
+                        if (fold) {      // rare, and uniform across the warp
+#pragma unroll
+                            for (int n = 0; n < NH; ++n) {
+                                if (!(s_new[n] >= kScaleLo && s_new[n] <= kScaleHi)) {
+#pragma unroll
+                                    for (int r = 0; r < kRPL; ++r) {
+#pragma unroll
+                                        for (int i = 0; i < kChunks; ++i) {
+                                            w[n][r][i].x *= s_new[n]; w[n][r][i].y *= s_new[n];
+                                            w[n][r][i].z *= s_new[n]; w[n][r][i].w *= s_new[n];
+                                        }
+                                    }
+                                    if (my_n == n) tot *= s_new[n];
+                                    s_new[n] = 1.0f;
+                                }
+                            }
+                        }
+                        float s_mine = s_new[0];
+#pragma unroll
+                        for (int n = 0; n < NH; ++n) {
+                            sc[n] = s_new[n];
+                            s_out[n] = s_new[n];
+                            if (my_n == n) s_mine = s_new[n];
+                        }
+                        cf_mine = fmaf(v_s[tp * vP], rcp_approx(s_mine), -tot) * bg_s[tp * bgP];
+                    }
 #pragma unroll
                     for (int n = 0; n < NH; ++n) {
 #pragma unroll
@@ -694,7 +743,7 @@ prefill_kernel(float* __restrict__ state, const float* __restrict__ q,
     if (active) {
         // the last position's output
         if (out_pending) {
-            if constexpr (!kCh) {
+            if constexpr (!kHalving) {
                 float ov = 0.0f, so = s_out[0];
 #pragma unroll
                 for (int n = 0; n < NH; ++n) {
@@ -713,7 +762,11 @@ prefill_kernel(float* __restrict__ state, const float* __restrict__ q,
                     }
                 }
                 const float tot = group_sum_many<kVals, kLPR>(vals, lane);
-                if (my_store) *out_prev = tot * kOutScale;
+                float so = s_out[0];
+#pragma unroll
+                for (int n = 1; n < NH; ++n)
+                    if (my_n == n) so = s_out[n];
+                if (my_store) *out_prev = so * tot * kOutScale;
             }
         }
         // the final state, scale folded in (kCh: the column scales)
@@ -741,17 +794,18 @@ prefill_kernel(float* __restrict__ state, const float* __restrict__ q,
 template <int NH, bool kCh>
 cudaError_t launch_nh(const PrefillArgs& a, cudaStream_t stream) {
     const int G = a.Hv / a.Hk;
-    const int64_t n_units = a.B * a.Hk * (G / NH) * kUnitsPerHead;
+    using L = Layout<kCh>;
+    const int64_t n_units = a.B * a.Hk * (G / NH) * L::UnitsPerHead;
     if (n_units == 0) return cudaSuccess;
     const int64_t sms = device_sm_count();
     int64_t grid = n_units < sms ? n_units : sms;
-    const int64_t min_grid = (n_units + kMaxWarps - 1) / kMaxWarps;
+    const int64_t min_grid = (n_units + L::MaxWarps - 1) / L::MaxWarps;
     if (grid < min_grid) grid = min_grid;
     const int units_lo = static_cast<int>(n_units / grid);
     const int n_big = static_cast<int>(n_units % grid);
-    // Per-channel decay: every CTA runs kMaxWarps warps (those past its run
+    // Per-channel decay: every CTA runs L::MaxWarps warps (those past its run
     // hold no rows) so that the per-stage conversion spreads evenly.
-    const int warps = kCh ? kMaxWarps : units_lo + (n_big > 0 ? 1 : 0);
+    const int warps = kCh ? L::MaxWarps : units_lo + (n_big > 0 ? 1 : 0);
     const size_t smem = sizeof(Stage<NH, kCh>) * stages_for<kCh>();
     cudaError_t err = cudaFuncSetAttribute(prefill_kernel<NH, kCh>,
                                            cudaFuncAttributeMaxDynamicSharedMemorySize,
