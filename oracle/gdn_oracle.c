@@ -203,6 +203,56 @@ int oracle_gdn_prefill(double *state, const double *q, const double *k,
     return 0;
 }
 
+/*
+ * Two-position speculative verify of the bare recurrence, [B] entry
+ * "gdn_pair": position 0 commits into the state, position 1 continues from
+ * it into a scratch state that the caller swaps in when it accepts the draft.
+ * Both are the one-token recurrence [S] run in order, as in the prefill.
+ *   state   [L][B][Hv][dv][dk]  in: before position 0, out: after position 0
+ *   scratch [L][B][Hv][dv][dk]  out: after position 1 (listed units only)
+ *   q, k    [L][B][2][Hk][dk]
+ *   v       [L][B][2][Hv][dv]
+ *   beta, gate [L][B][2][Hv]
+ *   out     [L][B][2][Hv][dv]
+ * units: flat indices u = (l*B + b)*Hv + h, or NULL for all.
+ */
+int oracle_gdn_pair(double *state, double *scratch, const double *q,
+                    const double *k, const double *v, const double *beta,
+                    const double *gate, double *out, int64_t L, int64_t B,
+                    int64_t Hk, int64_t Hv, int64_t dk, int64_t dv,
+                    const int64_t *units, int64_t n_units)
+{
+    if (L < 0 || B < 0 || !dims_ok(Hk, Hv, dk, dv))
+        return -1;
+    const int64_t total = L * B * Hv;
+    const int64_t count = units ? n_units : total;
+    for (int64_t n = 0; n < count; ++n) {
+        const int64_t u = units ? units[n] : n;
+        if (u < 0 || u >= total)
+            return -1;
+    }
+    for (int64_t n = 0; n < count; ++n) {
+        const int64_t u = units ? units[n] : n;
+        const int64_t lb = u / Hv;           /* l*B + b */
+        const int64_t h = u % Hv;
+        const int64_t g = h % Hk;
+        double *live = state + u * dv * dk;
+        double *tent = scratch + u * dv * dk;
+        for (int64_t pos = 0; pos < 2; ++pos) {
+            const int64_t lbp = lb * 2 + pos;    /* (l, b, position) */
+            double *M = pos == 0 ? live : tent;
+            if (pos == 1)                        /* position 1 starts from the committed state */
+                memcpy(tent, live, (size_t)(dv * dk) * sizeof(double));
+            int rc = gdn_head_token(M, q + (lbp * Hk + g) * dk, k + (lbp * Hk + g) * dk,
+                                    v + (lbp * Hv + h) * dv, beta[lbp * Hv + h],
+                                    gate[lbp * Hv + h], out + (lbp * Hv + h) * dv, dk, dv);
+            if (rc)
+                return rc;
+        }
+    }
+    return 0;
+}
+
 /* ------------------------------------------------------------------------ */
 /* Prestate pieces, [L] and [P].                                             */
 /* ------------------------------------------------------------------------ */

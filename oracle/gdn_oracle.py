@@ -64,6 +64,8 @@ class Oracle:
         lib.oracle_gdn_prefill.restype = ctypes.c_int
         lib.oracle_gdn_prefill.argtypes = [_PD, _PD, _PD, _PD, _PD, _PD, _PD,
                                            _I64, _I64, _I64, _I64, _I64, _I64, _PI, _I64]
+        lib.oracle_gdn_pair.restype = ctypes.c_int
+        lib.oracle_gdn_pair.argtypes = [_PD] * 8 + [_I64] * 6 + [_PI, _I64]
         lib.oracle_gdn_prestate.restype = ctypes.c_int
         lib.oracle_gdn_prestate.argtypes = [_PD, _PD, _PD, _PD, _PD, _PD, _PD, _DBL,
                                             _PD, _PD, _PD, _PD, _PD,
@@ -131,6 +133,30 @@ class Oracle:
                                          _ptr(gg), _ptr(out), B, T, Hk, Hv, dk, dv, up, nu)
         _check(rc, "oracle_gdn_prefill")
         return st, out
+
+    def pair(self, state, q, k, v, beta, gate, units=None):
+        """Two positions per unit: position 0 into the state, position 1 from
+        there into a scratch state.
+
+        Shapes: state [L,B,Hv,dv,dk]; q, k [L,B,2,Hk,dk]; v [L,B,2,Hv,dv];
+        beta, gate [L,B,2,Hv]. Returns (committed_state, scratch_state,
+        out [L,B,2,Hv,dv]); units that are not listed keep their state, get a
+        zero scratch state and zero output.
+        """
+        st = _f64(state)
+        L, B, Hv, dv, dk = st.shape
+        Hk = np.shape(q)[3]
+        qq, kk, vv, bb, gg = _f64(q), _f64(k), _f64(v), _f64(beta), _f64(gate)
+        assert qq.shape == (L, B, 2, Hk, dk) and kk.shape == qq.shape
+        assert vv.shape == (L, B, 2, Hv, dv) and bb.shape == (L, B, 2, Hv)
+        assert gg.shape == bb.shape
+        scratch = np.zeros_like(st)
+        out = np.zeros((L, B, 2, Hv, dv), dtype=np.float64)
+        up, nu, _keep = _units(units)
+        rc = self.lib.oracle_gdn_pair(_ptr(st), _ptr(scratch), _ptr(qq), _ptr(kk), _ptr(vv),
+                                      _ptr(bb), _ptr(gg), _ptr(out), L, B, Hk, Hv, dk, dv, up, nu)
+        _check(rc, "oracle_gdn_pair")
+        return st, scratch, out
 
     # -- layer pieces -------------------------------------------------------
     def prestate(self, mixed_qkv, ring, conv_w, a, b, A_log, dt_bias, *, Hk, Hv, dk, dv,

@@ -240,6 +240,37 @@ def pin_prefill_textbook(o):
             _close(st[b, h], M, 1e-12, f"prefill state b{b} h{h}")
 
 
+def pin_pair_textbook(o):
+    """The two-position verify on non-square heads: the committed state, the
+    scratch state and both outputs equal the product form applied at
+    position 0 and then, from the committed state, at position 1."""
+    r = _rng(23)
+    L, B, Hk, Hv, dk, dv = 2, 2, 2, 6, 8, 6
+    S0 = r.normal(0, 0.3, (L, B, Hv, dv, dk))
+    q = _unit_rows(r.normal(size=(L, B, 2, Hk, dk)))
+    k = _unit_rows(r.normal(size=(L, B, 2, Hk, dk)))
+    v = r.normal(size=(L, B, 2, Hv, dv))
+    beta = r.uniform(0, 1, (L, B, 2, Hv))
+    gate = r.uniform(-0.5, 0, (L, B, 2, Hv))
+    live, tent, out = o.pair(S0, q, k, v, beta, gate)
+    for l in range(L):
+        for b in range(B):
+            for h in range(Hv):
+                g = h % Hk
+                M = S0[l, b, h]
+                for pos in range(2):
+                    M, on = textbook_head(M, q[l, b, pos, g], k[l, b, pos, g], v[l, b, pos, h],
+                                          beta[l, b, pos, h], gate[l, b, pos, h])
+                    _close(out[l, b, pos, h], on, 1e-12, f"pair out l{l} b{b} p{pos} h{h}")
+                    _close((live if pos == 0 else tent)[l, b, h], M, 1e-12,
+                           f"pair state l{l} b{b} p{pos} h{h}")
+    # a unit left out keeps its state and gets zero scratch and output
+    part_live, part_tent, part_out = o.pair(S0, q, k, v, beta, gate, units=[3])
+    assert np.array_equal(part_live[0, 0, 0], S0[0, 0, 0]), "unlisted unit state"
+    assert not part_tent[0, 0, 0].any() and not part_out[0, 0, :, 0].any(), "unlisted unit"
+    _close(part_tent[0, 0, 3], tent[0, 0, 3], 0.0, "listed unit scratch")
+
+
 # --------------------------------------------------------------------------
 # layer pins (torch fp64 library routines)
 # --------------------------------------------------------------------------
@@ -606,6 +637,7 @@ ALL_PINS = [
     pin_broadcast_marker,
     pin_prefill_associative_memory,
     pin_prefill_textbook,
+    pin_pair_textbook,
     pin_prestate_library,
     pin_prestate_special_values,
     pin_tail_library,

@@ -37,6 +37,14 @@ MUTATIONS = [
      "const int64_t g = h / (Hv / Hk);\n        double *M"),
     ("prefill order reversed", "const int64_t bt = b * T + t;",
      "const int64_t bt = b * T + (T - 1 - t);"),
+    # two-position verify ("Module linear_core", entry "gdn_pair")
+    ("pair position 1 from the input state",
+     "memcpy(tent, live, (size_t)(dv * dk) * sizeof(double));",
+     "memset(tent, 0, (size_t)(dv * dk) * sizeof(double));"),
+    ("pair positions swapped", "const int64_t lbp = lb * 2 + pos;",
+     "const int64_t lbp = lb * 2 + (1 - pos);"),
+    ("pair commits position 1", "double *M = pos == 0 ? live : tent;",
+     "double *M = live;"),
     # prestate
     ("conv taps reversed", "acc += w[c * K + t] * win;", "acc += w[c * K + (K - 1 - t)] * win;"),
     ("ring not refreshed", "ring[(K - 2) * C + c] = x[c];",
