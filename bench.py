@@ -55,6 +55,13 @@ def step_bytes(L: int, B: int, Hk: int = 16, Hv: int = 32, d: int = 128) -> int:
     return heads * (2 * d * d * 4 + 2 * d * 4 + 2 * 4) + L * B * Hk * 2 * d * 4
 
 
+def pair_bytes(L: int, B: int, Hk: int = 16, Hv: int = 32, d: int = 128) -> int:
+    """gdn_pair: each state row read once and written twice (committed and
+    scratch), and two positions of q/k, v, out, beta and gate."""
+    heads = L * B * Hv
+    return heads * (3 * d * d * 4 + 2 * (2 * d * 4 + 2 * 4)) + L * B * 2 * Hk * 2 * d * 4
+
+
 def prefill_bytes(B: int, T: int, Hk: int = 16, Hv: int = 32, d: int = 128) -> int:
     return (2 * B * Hv * d * d * 4 + B * T * (Hk * 2 * d * 4 + Hv * (2 * d * 4 + 2 * 4)))
 
@@ -451,6 +458,20 @@ def build_case(name: str, device):
         out = torch.empty_like(t["v"])
         return (lambda i: gdn.step(t["state"], t["q"], t["k"], t["v"], t["beta"], t["gate"],
                                    out)), dict(tensors=t)
+    if name == "pair_l1_b64":
+        # two input sets of 256 MiB of state each, so a launch's state rows
+        # are not still in L2 from the one before
+        w = inputs.PAIR_WORKLOAD
+        first = _to_dev(w.draw(), device)
+        sets = []
+        for si in range(2):
+            t = first if si == 0 else {n: x.clone() for n, x in first.items()}
+            sets.append((t, torch.empty_like(t["state"]), torch.empty_like(t["v"])))
+
+        def launch(i):
+            t, scratch, out = sets[i % len(sets)]
+            gdn.pair(t["state"], scratch, t["q"], t["k"], t["v"], t["beta"], t["gate"], out)
+        return launch, dict(sizes=w.sizes)
     if name == "prefill_b4_t4096":
         w = inputs.WORKLOADS[name]
         t = _to_dev(w.draw(), device)
@@ -532,8 +553,8 @@ def build_case(name: str, device):
     raise KeyError(f"unknown case {name!r}")
 
 
-PROFILE_CASES = ("decode_l1_b1", "decode_l1_b64", "decode_l36_b16", "prefill_b4_t4096",
-                 "layer_decode_b256", "layer_pair_b256", "forward_batch_b4_t4096",
+PROFILE_CASES = ("decode_l1_b1", "decode_l1_b64", "decode_l36_b16", "pair_l1_b64",
+                 "prefill_b4_t4096", "layer_decode_b256", "layer_pair_b256", "forward_batch_b4_t4096",
                  "linear_bf16_m16384_n8192_k2048", "short_conv_decode_b64", "short_conv_pair_b64",
                  "short_conv_batch_b4_t4096", "kda_decode_b64", "kda_prefill_b4_t4096")
 
@@ -619,6 +640,21 @@ def bench_short_conv(name: str, steps: int, warmup: int, device, peaks):
         r.update(tflops=tf, roofline={"bound": "tensor", "peak": peaks["bf16_tflops"],
                                       "unit": "TFLOP/s", "frac": tf / peaks["bf16_tflops"]})
     return r
+
+
+def bench_pair(steps: int, device, peaks):
+    """gdn_pair for 64 sequences (HBM roofline), graph-replayed over two
+    input sets."""
+    import torch
+    stream = torch.cuda.current_stream(device)
+    launch, m = build_case("pair_l1_b64", device)
+    per = time_launches(launch, 1, steps, 10, stream, graph=True) / steps
+    L, B = m["sizes"]["L"], m["sizes"]["B"]
+    gbs = pair_bytes(L, B) / per / 1e9
+    return {"ms_per_launch": per * 1e3, "layer_tokens_per_s": 2 * L * B / per, "gb_s": gbs,
+            "l2": "rotating 2 input sets",
+            "roofline": {"bound": "hbm", "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                         "frac": gbs / peaks["hbm_gbs"]}}
 
 
 def bench_kda(steps_decode: int, steps_prefill: int, device, peaks, alu_peak):
@@ -825,6 +861,8 @@ def run_ours(args) -> int:
         r2 = bench_step_workload("decode_l36_b16", 20, 3, device)
         extras["decode_l36_b16"] = _step_extra(r2, 20, peaks)
         del r2
+        torch.cuda.empty_cache()
+        extras["pair_l1_b64"] = bench_pair(400, device, peaks)
         torch.cuda.empty_cache()
         p = bench_prefill(5, 3, device)
         alu_peak = 148 * 128 * 2 * (line["clocks"]["sm_max_mhz"] or 1965) * 1e6 / 1e12

@@ -110,6 +110,32 @@ gdn_status gdn_prefill(float *state, const float *q, const float *k, const float
                        int64_t dv, void *stream);
 
 /*
+ * gdn_pair -- two-position speculative verify of the recurrence, one launch
+ * for L layers x B sequences x Hv value heads. Position 0 commits into
+ * `state`; position 1 continues from that state into `scratch_state`, which
+ * the caller takes as the new state when it accepts the draft token (by
+ * swapping the two buffers) and ignores otherwise. Each state row is read
+ * once and written twice. The results equal two gdn_step calls, bit for bit.
+ * ("Module linear_core", entry "gdn_pair": lane 1 commits, lane 2 is
+ * tentative in scratch; steps as for gdn_step.)
+ *
+ *   state          [L][B][Hv][dv][dk]  in: before position 0,
+ *                                      out: after position 0
+ *   scratch_state  [L][B][Hv][dv][dk]  out: after position 1 (never read)
+ *   q, k           [L][B][2][Hk][dk]   position p of sequence (l, b) at [l][b][p]
+ *   v              [L][B][2][Hv][dv]
+ *   beta, gate     [L][B][2][Hv]
+ *   out            [L][B][2][Hv][dv]
+ *
+ * scratch_state and out must not overlap each other or any input; state may
+ * not overlap an input.
+ */
+gdn_status gdn_pair(float *state, float *scratch_state, const float *q, const float *k,
+                    const float *v, const float *beta, const float *gate, float *out,
+                    int64_t L, int64_t B, int64_t Hk, int64_t Hv, int64_t dk, int64_t dv,
+                    void *stream);
+
+/*
  * gdn_layer_decode -- the single-token recurrent layer between the input
  * projections and the output projection, fused in one launch
  * ("Red Lite dev15e -- complete recurrent DeltaNet layer composition",

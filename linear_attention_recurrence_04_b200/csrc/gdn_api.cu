@@ -222,6 +222,41 @@ gdn_status step_call(const char* fn, float* state, const float* q, const float* 
     return launched(channel_decay ? launch_kda_step(a, s) : launch_step(a, s), fn);
 }
 
+// gdn_pair: the checks of gdn_step with two positions per sequence and a
+// second state-sized output.
+gdn_status pair_call(const char* fn, float* state, float* scratch, const float* q,
+                     const float* k, const float* v, const float* beta, const float* gate,
+                     float* out, int64_t L, int64_t B, int64_t Hk, int64_t Hv, int64_t dk,
+                     int64_t dv, void* stream) {
+    NvtxRange nvtx_range(fn);
+    if (L < 0 || B < 0) return fail(GDN_ERR_SHAPE, "%s: negative L=%lld or B=%lld", fn,
+                                    (long long)L, (long long)B);
+    gdn_status st = check_geometry(Hk, Hv, dk, dv);
+    if (st != GDN_OK) return st;
+    int64_t lb = 0, heads = 0, state_n = 0, qk_n = 0, v_n = 0;
+    if (!mul_ok(L, B, &lb) || !mul_ok(lb, Hv, &heads) || !mul_ok(heads, dv * dk, &state_n) ||
+        !mul_ok(lb, 2 * Hk * dk, &qk_n) || !mul_ok(heads, 2 * dv, &v_n) ||
+        state_n > INT64_MAX / 8 || qk_n > INT64_MAX / 8 || v_n > INT64_MAX / 8)
+        return fail(GDN_ERR_OVERFLOW, "%s: L*B*Hv*dv*dk overflows int64", fn);
+    if (heads == 0) { g_last_error[0] = '\0'; return GDN_OK; }
+    if (!state || !scratch || !q || !k || !v || !beta || !gate || !out)
+        return fail(GDN_ERR_NULL, "%s: a tensor pointer is NULL", fn);
+    if (!aligned(state, 16) || !aligned(scratch, 16) || !aligned(q, 16) || !aligned(k, 16) ||
+        !aligned(v, 16) || !aligned(out, 16) || !aligned(beta, 4) || !aligned(gate, 4))
+        return fail(GDN_ERR_ALIGN,
+                    "%s: state/scratch_state/q/k/v/out need 16-byte, beta/gate 4-byte alignment",
+                    fn);
+    const Span ins[] = {{state, state_n * 4, "state"}, {q, qk_n * 4, "q"}, {k, qk_n * 4, "k"},
+                        {v, v_n * 4, "v"}, {beta, heads * 2 * 4, "beta"},
+                        {gate, heads * 2 * 4, "gate"}, {out, v_n * 4, "out"}};
+    st = check_spans(ins, 6, 1, Span{out, v_n * 4, "out"});
+    if (st != GDN_OK) return st;
+    st = check_spans(ins, 7, 1, Span{scratch, state_n * 4, "scratch_state"});
+    if (st != GDN_OK) return st;
+    StepArgs a{state, q, k, v, beta, gate, out, heads, static_cast<int>(Hk), static_cast<int>(Hv)};
+    return launched(launch_pair(a, scratch, static_cast<cudaStream_t>(stream)), fn);
+}
+
 // Checks shared by the multi-position entries gdn_prefill and gdn_kda_prefill.
 gdn_status prefill_call(const char* fn, float* state, const float* q, const float* k,
                         const float* v, const float* beta, const float* gate, float* out,
@@ -275,6 +310,13 @@ gdn_status gdn_prefill(float* state, const float* q, const float* k, const float
                        int64_t Hk, int64_t Hv, int64_t dk, int64_t dv, void* stream) {
     return prefill_call("gdn_prefill", state, q, k, v, beta, gate, out, B, T, Hk, Hv, dk, dv,
                         false, stream);
+}
+
+gdn_status gdn_pair(float* state, float* scratch_state, const float* q, const float* k,
+                    const float* v, const float* beta, const float* gate, float* out, int64_t L,
+                    int64_t B, int64_t Hk, int64_t Hv, int64_t dk, int64_t dv, void* stream) {
+    return pair_call("gdn_pair", state, scratch_state, q, k, v, beta, gate, out, L, B, Hk, Hv, dk,
+                     dv, stream);
 }
 
 gdn_status gdn_kda_step(float* state, const float* q, const float* k, const float* v,

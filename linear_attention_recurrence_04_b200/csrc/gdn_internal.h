@@ -126,6 +126,10 @@ cudaError_t launch_step(const StepArgs& a, cudaStream_t stream);
 // channel, [..][Hv][dk] (contiguous).
 cudaError_t launch_kda_step(const StepArgs& a, cudaStream_t stream);
 cudaError_t launch_kda_prefill(const PrefillArgs& a, cudaStream_t stream);
+// Two-position verify: StepArgs with q, k, v, beta, gate and out holding two
+// positions per sequence ([L][B][2][..]); the state after position 0 goes to
+// a.state, the state after position 1 to `scratch`.
+cudaError_t launch_pair(const StepArgs& a, float* scratch, cudaStream_t stream);
 cudaError_t launch_prefill(const PrefillArgs& a, cudaStream_t stream);
 cudaError_t launch_layer_decode(const LayerArgs& a, cudaStream_t stream);
 cudaError_t launch_layer_pair(const LayerArgs& a, cudaStream_t stream);

@@ -28,7 +28,8 @@ STATUS = {
 }
 
 # Every symbol that include/gdn.h declares.
-EXPORTS = ("gdn_status_string", "gdn_last_error", "gdn_step", "gdn_prefill", "gdn_layer_decode",
+EXPORTS = ("gdn_status_string", "gdn_last_error", "gdn_step", "gdn_prefill", "gdn_pair",
+           "gdn_layer_decode",
            "gdn_layer_pair", "gdn_linear_bf16", "gdn_forward_batch_workspace_size",
            "gdn_forward_batch", "gdn_forward_batch_noalloc", "gdn_short_conv_workspace_size",
            "gdn_short_conv_forward_batch", "gdn_short_conv_forward", "gdn_short_conv_pair",
@@ -70,6 +71,8 @@ def load_library(path: Optional[str] = None) -> ctypes.CDLL:
     lib.gdn_step.argtypes = [_VP] * 7 + [_I64] * 6 + [_VP]
     lib.gdn_prefill.restype = ctypes.c_int
     lib.gdn_prefill.argtypes = [_VP] * 7 + [_I64] * 6 + [_VP]
+    lib.gdn_pair.restype = ctypes.c_int
+    lib.gdn_pair.argtypes = [_VP] * 8 + [_I64] * 6 + [_VP]
     lib.gdn_layer_decode.restype = ctypes.c_int
     lib.gdn_layer_decode.argtypes = [_VP] * 9 + [_F32, _F32] + [_VP, _VP] + [_I64] * 6 + [_VP]
     lib.gdn_layer_pair.restype = ctypes.c_int
@@ -166,6 +169,32 @@ def step(state, q, k, v, beta, gate, out=None, *, stream=None):
     st = _call(device, load_library().gdn_step, *(_ptr(t) for t in tensors), L, B, Hk, Hv, dk,
                dv, _stream(device, stream))
     _raise_on("gdn_step", st)
+    return out
+
+
+def pair(state, scratch_state, q, k, v, beta, gate, out=None, *, stream=None):
+    """Two-position verify: state [L,B,Hv,128,128] (before position 0 ->
+    after position 0, in place), scratch_state [L,B,Hv,128,128] (written:
+    after position 1), q/k [L,B,2,Hk,128], v [L,B,2,Hv,128], beta/gate
+    [L,B,2,Hv]. Returns out [L,B,2,Hv,128]."""
+    if state.dim() != 5:
+        raise ValueError("state must be [L, B, Hv, dv, dk]")
+    L, B, Hv, dv, dk = state.shape
+    Hk = q.shape[3]
+    if out is None:
+        out = torch.empty((L, B, 2, Hv, dv), dtype=torch.float32, device=state.device)
+    names = ("state", "scratch_state", "q", "k", "v", "beta", "gate", "out")
+    tensors = (state, scratch_state, q, k, v, beta, gate, out)
+    device = _dev(tensors, names)
+    expect = dict(scratch_state=(L, B, Hv, dv, dk), q=(L, B, 2, Hk, dk), k=(L, B, 2, Hk, dk),
+                  v=(L, B, 2, Hv, dv), beta=(L, B, 2, Hv), gate=(L, B, 2, Hv),
+                  out=(L, B, 2, Hv, dv))
+    for n, t in zip(names[1:], tensors[1:]):
+        if tuple(t.shape) != expect[n]:
+            raise ValueError(f"{n} has shape {tuple(t.shape)}, expected {expect[n]}")
+    st = _call(device, load_library().gdn_pair, *(_ptr(t) for t in tensors), L, B, Hk, Hv, dk,
+               dv, _stream(device, stream))
+    _raise_on("gdn_pair", st)
     return out
 
 

@@ -65,6 +65,27 @@ def decode_inputs(L: int, B: int, *, Hk: int = HK, Hv: int = HV, dk: int = DK, d
     return {n: (np.stack(p) if p else np.zeros(shapes[n], np.float32)) for n, p in parts.items()}
 
 
+def pair_inputs(L: int, B: int, *, Hk: int = HK, Hv: int = HV, dk: int = DK, dv: int = DV,
+                seed: int = 1015, state_std: float = 0.05,
+                gate_low: float = -1.0) -> Dict[str, np.ndarray]:
+    """Inputs of the two-position verify: the decode draws of decode_inputs
+    with a position axis of 2 after the sequence axis: state [L,B,Hv,dv,dk],
+    q/k [L,B,2,Hk,dk], v [L,B,2,Hv,dv], beta/gate [L,B,2,Hv] (float32)."""
+    streams = np.random.default_rng(seed).spawn(max(L, 1))
+    parts = {n: [] for n in ("state", "q", "k", "v", "beta", "gate")}
+    for l in range(L):
+        r = streams[l]
+        parts["state"].append(_f32(r.normal(0.0, state_std, (B, Hv, dv, dk))))
+        parts["q"].append(_f32(_unit_rows(r.normal(size=(B, 2, Hk, dk)))))
+        parts["k"].append(_f32(_unit_rows(r.normal(size=(B, 2, Hk, dk)))))
+        parts["v"].append(_f32(r.normal(size=(B, 2, Hv, dv))))
+        parts["beta"].append(_f32(_squash(r.normal(size=(B, 2, Hv)))))
+        parts["gate"].append(_f32(r.uniform(gate_low, 0.0, (B, 2, Hv))))
+    shapes = dict(state=(0, B, Hv, dv, dk), q=(0, B, 2, Hk, dk), k=(0, B, 2, Hk, dk),
+                  v=(0, B, 2, Hv, dv), beta=(0, B, 2, Hv), gate=(0, B, 2, Hv))
+    return {n: (np.stack(p) if p else np.zeros(shapes[n], np.float32)) for n, p in parts.items()}
+
+
 def prefill_inputs(B: int, T: int, *, Hk: int = HK, Hv: int = HV, dk: int = DK, dv: int = DV,
                    seed: int = 1003, gate_low: float = -0.5,
                    state_std: float = 0.0) -> Dict[str, np.ndarray]:
@@ -188,13 +209,15 @@ def short_conv_inputs(B: int, T: int, *, D: int = 2048, K: int = 3, seed: int = 
 class Workload:
     """One named synthetic workload and how to draw it."""
     name: str
-    kind: str                     # "step" | "prefill" | "layer" | "forward" | "short_conv" | "kda_*"
+    kind: str                     # "step" | "pair" | "prefill" | "layer" | "forward" | "short_conv" | "kda_*"
     sizes: Dict[str, int] = field(default_factory=dict)
     seed: int = 1000
 
     def draw(self) -> Dict[str, np.ndarray]:
         if self.kind == "step":
             return decode_inputs(self.sizes["L"], self.sizes["B"], seed=self.seed)
+        if self.kind == "pair":
+            return pair_inputs(self.sizes["L"], self.sizes["B"], seed=self.seed)
         if self.kind == "prefill":
             return prefill_inputs(self.sizes["B"], self.sizes["T"], seed=self.seed)
         if self.kind == "layer":
@@ -220,6 +243,9 @@ WORKLOADS = {
     "prefill_b4_t4096": Workload("prefill_b4_t4096", "prefill", dict(B=4, T=4096), seed=1003),
     "layer_decode_b256": Workload("layer_decode_b256", "layer", dict(B=256), seed=1004),
 }
+
+# The two-position speculative verify of the bare recurrence for 64 sequences.
+PAIR_WORKLOAD = Workload("pair_l1_b64", "pair", dict(L=1, B=64), seed=1015)
 
 # The batched layer forward with dense projections (D = 2048 hidden).
 FORWARD_WORKLOAD = Workload("forward_batch_b4_t4096", "forward", dict(B=4, T=4096), seed=1007)

@@ -98,6 +98,33 @@ def test_prefill_argument_checks(lib):
     assert lib.gdn_prefill(0, 0, 0, 0, 0, 0, 0, 0, 9, 16, 32, 128, 128, None) == OK
 
 
+def pair_call(lib, state=A16, scratch=fake(7), q=A16b, k=A16c, v=fake(3), beta=fake(4),
+              gate=fake(5), out=fake(6), L=1, B=1, Hk=16, Hv=32, dk=128, dv=128):
+    return lib.gdn_pair(state, scratch, q, k, v, beta, gate, out, L, B, Hk, Hv, dk, dv, None)
+
+
+def test_pair_argument_checks(lib):
+    assert pair_call(lib, B=-1) == SHAPE
+    assert pair_call(lib, Hv=20, Hk=16) == SHAPE
+    assert pair_call(lib, dk=64) == UNSUP
+    assert pair_call(lib, scratch=0) == NULL
+    assert pair_call(lib, gate=0) == NULL
+    assert pair_call(lib, scratch=fake(7) + 8) == ALIGN
+    assert pair_call(lib, gate=fake(5) + 2) == ALIGN
+    assert pair_call(lib, L=1 << 40, B=1 << 40) == OVERFLOW
+    # the scratch state inside the live state, over an input, over out
+    assert pair_call(lib, scratch=A16 + 4096) == ALIAS
+    assert pair_call(lib, scratch=fake(3) + 1024) == ALIAS
+    assert pair_call(lib, scratch=fake(6) + 256) == ALIAS
+    # out over the state; the state over q
+    assert pair_call(lib, out=A16 + 16) == ALIAS
+    assert pair_call(lib, q=A16 + 1024) == ALIAS
+    # read-only inputs may share memory
+    assert pair_call(lib, k=A16b, q=A16b, out=0) == NULL
+    assert lib.gdn_pair(0, 0, 0, 0, 0, 0, 0, 0, 0, 4, 16, 32, 128, 128, None) == OK
+    assert lib.gdn_pair(0, 0, 0, 0, 0, 0, 0, 0, 2, 0, 16, 32, 128, 128, None) == OK
+
+
 def test_layer_argument_checks(lib):
     def f(B=1, Hk=16, Hv=32, K=4, state=A16, out=fake(10), ring=fake(5)):
         return lib.gdn_layer_decode(A16b, A16c, fake(3), fake(4), ring, fake(6), fake(7),
