@@ -271,7 +271,8 @@ static double softplus(double x)
 
 /*
  * Causal depthwise conv1d over one token with the conv-state ring, [P]
- * ("conv-state shift, real F32 ssm_conv1d").
+ * section "Validation boundary" (the conv-state shift, then the fp32
+ * depthwise conv).
  *   x    [C]        this token's pre-conv input (mixed q|k|v)
  *   ring [K-1][C]   in/out; slot 0 is the oldest past input
  *   w    [C][K]     tap t multiplies window[t], window = (ring[0..K-2], x)
