@@ -98,3 +98,30 @@ def test_pair_empty_batch_is_a_no_op():
     out = gdn.pair(t["state"], scratch, t["q"], t["k"], t["v"], t["beta"], t["gate"])
     torch.cuda.synchronize()
     assert out.shape == (1, 0, 2, 32, 128)
+
+
+def test_pair_indices_past_32_bits(o):
+    """A state of 9 x 512 x 32 x 128 x 128 floats (> 2^31 elements, 9.7 GB)
+    and its scratch: units in the last layer sit past the 32-bit index range.
+    Every layer is a copy of one drawn layer, so a unit's oracle is that
+    layer's unit."""
+    base = inputs.pair_inputs(1, 512, seed=1750)
+    L, B, Hv = 9, 512, 32
+    dev = {k: torch.from_numpy(v).cuda().expand(L, *v.shape[1:]).contiguous()
+           for k, v in base.items()}
+    assert dev["state"].numel() > 2 ** 31
+    scratch = torch.empty_like(dev["state"])
+    out = gdn.pair(dev["state"], scratch, dev["q"], dev["k"], dev["v"], dev["beta"], dev["gate"])
+    torch.cuda.synchronize()
+    units = [0, 1, 777, 16383 - 5, B * Hv - 1]
+    live_ref, tent_ref, out_ref = o.pair(base["state"], base["q"], base["k"], base["v"],
+                                         base["beta"], base["gate"], units=units)
+    for u in units:
+        b, h = divmod(u, Hv)
+        assert_parity(out[L - 1, b, :, h].cpu().numpy(), out_ref[0, b, :, h], f"unit {u} out")
+        assert_parity(dev["state"][L - 1, b, h].cpu().numpy(), live_ref[0, b, h],
+                      f"unit {u} committed state")
+        assert_parity(scratch[L - 1, b, h].cpu().numpy(), tent_ref[0, b, h],
+                      f"unit {u} scratch state")
+    del dev, scratch, out
+    torch.cuda.empty_cache()
