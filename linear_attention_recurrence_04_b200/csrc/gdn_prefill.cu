@@ -72,6 +72,9 @@
 #ifndef GDN_PREFILL_NH
 #define GDN_PREFILL_NH 0           // value heads per warp: 0 = 2 when Hv/Hk is even, else 1
 #endif
+#ifndef GDN_PREFILL_LOADER_WARP
+#define GDN_PREFILL_LOADER_WARP 1  // scalar decay: one extra warp issues every stage copy
+#endif
 #ifndef GDN_PREFILL_UNROLL
 #define GDN_PREFILL_UNROLL 8       // positions per unrolled block of a stage
 #endif
@@ -103,7 +106,11 @@ struct Layout {
     static constexpr int Chunks = kDk / 4 / LPR;                // float4 chunks per lane and row
     static constexpr int RowsPerUnit = 32 / LPR * RPL;          // rows of a head per warp
     static constexpr int UnitsPerHead = kDv / RowsPerUnit;
-    static constexpr int MaxWarps = kMaxRows / RowsPerUnit;     // warps (units) per CTA at most
+    // Scalar decay with GDN_PREFILL_LOADER_WARP: one more warp, the CTA's
+    // last, issues every stage copy; the block stays at 8 warps.
+    static constexpr bool Loader = !kCh && GDN_PREFILL_LOADER_WARP;
+    static constexpr int MaxWarps = kMaxRows / RowsPerUnit - (Loader ? 1 : 0);  // units per CTA
+    static constexpr int Threads = 32 * (MaxWarps + (Loader ? 1 : 0));
     // One halving reduction of all key and output dots with the deltas
     // broadcast, rather than a full reduction of each on every lane.
     static constexpr bool Halving = kCh || LPR == 8;
@@ -212,7 +219,7 @@ __device__ __forceinline__ float rcp_approx(float x) {
 }
 
 template <int NH, bool kCh>
-__global__ void __launch_bounds__(32 * Layout<kCh>::MaxWarps, 1)
+__global__ void __launch_bounds__(Layout<kCh>::Threads, 1)
 prefill_kernel(float* __restrict__ state, const float* __restrict__ q,
                const float* __restrict__ k, const float* __restrict__ v,
                const float* __restrict__ beta, const float* __restrict__ gate,
@@ -270,13 +277,19 @@ prefill_kernel(float* __restrict__ state, const float* __restrict__ q,
 
     // ---- stage loader: every thread issues a share of the copies; positions
     //      at or past T are zero-filled ------------------------------------
+    // With a loader warp (the CTA's last warp), it alone issues the copies.
+    constexpr bool kLoaderWarp = Layout<kCh>::Loader;
+    const bool is_loader = kLoaderWarp && warp == static_cast<int>(blockDim.x >> 5) - 1;
+    const int ltid = kLoaderWarp ? lane : tid;
+    const int lstride = kLoaderWarp ? 32 : nthreads;
     auto load_stage = [&](int64_t t0, StageT& st) {
+        if (kLoaderWarp && !is_loader) return;
         if (kCh && tid < kMaxGroups) st.mode[tid] = 0;
 #pragma unroll
         for (int gi = 0; gi < kMaxGroups; ++gi) {
             if (gi >= n_groups) break;
             const Group G = grp_of[gi];
-            for (int idx = tid; idx < TS * 64 + 32; idx += nthreads) {   // k, q rows; k of t0 + TS
+            for (int idx = ltid; idx < TS * 64 + 32; idx += lstride) {   // k, q rows; k of t0 + TS
                 const int chunk = idx & 31;
                 const int which = (idx >> 5) & 1;     // the extra slot gets k only
                 const int tp = idx >> 6;
@@ -289,7 +302,7 @@ prefill_kernel(float* __restrict__ state, const float* __restrict__ q,
                 }
             }
             const int vchunks = G.rows / 4;                              // v rows
-            for (int idx = tid; idx < TS * NH * vchunks; idx += nthreads) {
+            for (int idx = ltid; idx < TS * NH * vchunks; idx += lstride) {
                 const int chunk = idx % vchunks;
                 const int n = (idx / vchunks) % NH;
                 const int tp = idx / (vchunks * NH);
@@ -302,7 +315,7 @@ prefill_kernel(float* __restrict__ state, const float* __restrict__ q,
                     *reinterpret_cast<float4*>(dst) = make_float4(0.f, 0.f, 0.f, 0.f);
                 }
             }
-            for (int idx = tid; idx < TS * NH * 2; idx += nthreads) {    // beta, gate
+            for (int idx = ltid; idx < TS * NH * 2; idx += lstride) {    // beta, gate
                 const int which = idx & 1;
                 const int n = (idx >> 1) % NH;
                 const int tp = (idx >> 1) / NH;
@@ -316,7 +329,7 @@ prefill_kernel(float* __restrict__ state, const float* __restrict__ q,
                 }
             }
             if constexpr (kCh) {                                         // g rows
-                for (int idx = tid; idx < (TS + 1) * NH * 32; idx += nthreads) {
+                for (int idx = ltid; idx < (TS + 1) * NH * 32; idx += lstride) {
                     const int chunk = idx & 31;
                     const int n = (idx >> 5) % NH;
                     const int tp = (idx >> 5) / NH;
@@ -805,7 +818,7 @@ cudaError_t launch_nh(const PrefillArgs& a, cudaStream_t stream) {
     const int n_big = static_cast<int>(n_units % grid);
     // Per-channel decay: every CTA runs L::MaxWarps warps (those past its run
     // hold no rows) so that the per-stage conversion spreads evenly.
-    const int warps = kCh ? L::MaxWarps : units_lo + (n_big > 0 ? 1 : 0);
+    const int warps = kCh ? L::MaxWarps : units_lo + (n_big > 0 ? 1 : 0) + (L::Loader ? 1 : 0);
     const size_t smem = sizeof(Stage<NH, kCh>) * stages_for<kCh>();
     cudaError_t err = cudaFuncSetAttribute(prefill_kernel<NH, kCh>,
                                            cudaFuncAttributeMaxDynamicSharedMemorySize,
