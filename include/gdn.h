@@ -103,11 +103,15 @@ gdn_status gdn_step(float *state, const float *q, const float *k, const float *v
  *   v     [B][T][Hv][dv]
  *   beta, gate [B][T][Hv]
  *   out   [B][T][Hv][dv]
+ *   status optional zero-initialised device word: the kernel's stage
+ *          pipeline waits are bounded (2 s); if one ever times out, a
+ *          non-zero bit is ORed into it and the kernel returns without
+ *          hanging (its outputs are then incomplete). NULL: not reported.
  */
 gdn_status gdn_prefill(float *state, const float *q, const float *k, const float *v,
                        const float *beta, const float *gate, float *out,
                        int64_t B, int64_t T, int64_t Hk, int64_t Hv, int64_t dk,
-                       int64_t dv, void *stream);
+                       int64_t dv, uint32_t *status, void *stream);
 
 /*
  * gdn_pair -- two-position speculative verify of the recurrence, one launch

@@ -261,7 +261,7 @@ gdn_status pair_call(const char* fn, float* state, float* scratch, const float* 
 gdn_status prefill_call(const char* fn, float* state, const float* q, const float* k,
                         const float* v, const float* beta, const float* gate, float* out,
                         int64_t B, int64_t T, int64_t Hk, int64_t Hv, int64_t dk, int64_t dv,
-                        bool channel_decay, void* stream) {
+                        bool channel_decay, uint32_t* status, void* stream) {
     NvtxRange nvtx_range(fn);
     if (B < 0 || T < 0) return fail(GDN_ERR_SHAPE, "%s: negative B=%lld or T=%lld", fn,
                                     (long long)B, (long long)T);
@@ -289,7 +289,10 @@ gdn_status prefill_call(const char* fn, float* state, const float* q, const floa
                         {gate, gate_n * 4, channel_decay ? "g" : "gate"}};
     st = check_spans(ins, 6, 1, Span{out, v_n * 4, "out"});
     if (st != GDN_OK) return st;
+    if (status && !aligned(status, 4))
+        return fail(GDN_ERR_ALIGN, "%s: status needs 4-byte alignment", fn);
     PrefillArgs a{state, q, k, v, beta, gate, out, B, T, static_cast<int>(Hk), static_cast<int>(Hv)};
+    a.status = status;
     const cudaStream_t s = static_cast<cudaStream_t>(stream);
     return launched(channel_decay ? launch_kda_prefill(a, s) : launch_prefill(a, s), fn);
 }
@@ -307,9 +310,10 @@ gdn_status gdn_step(float* state, const float* q, const float* k, const float* v
 
 gdn_status gdn_prefill(float* state, const float* q, const float* k, const float* v,
                        const float* beta, const float* gate, float* out, int64_t B, int64_t T,
-                       int64_t Hk, int64_t Hv, int64_t dk, int64_t dv, void* stream) {
+                       int64_t Hk, int64_t Hv, int64_t dk, int64_t dv, uint32_t* status,
+                       void* stream) {
     return prefill_call("gdn_prefill", state, q, k, v, beta, gate, out, B, T, Hk, Hv, dk, dv,
-                        false, stream);
+                        false, status, stream);
 }
 
 gdn_status gdn_pair(float* state, float* scratch_state, const float* q, const float* k,
@@ -330,7 +334,7 @@ gdn_status gdn_kda_prefill(float* state, const float* q, const float* k, const f
                            const float* beta, const float* g, float* out, int64_t B, int64_t T,
                            int64_t Hk, int64_t Hv, int64_t dk, int64_t dv, void* stream) {
     return prefill_call("gdn_kda_prefill", state, q, k, v, beta, g, out, B, T, Hk, Hv, dk, dv,
-                        true, stream);
+                        true, nullptr, stream);
 }
 
 namespace {

@@ -254,6 +254,7 @@ cudaError_t launch_forward_batch(const ForwardBatchArgs& a, cudaStream_t stream)
         PrefillArgs p{a.state, act, act + static_cast<int64_t>(a.Hk) * kDk,
                       act + static_cast<int64_t>(2 * a.Hk) * kDk, beta, gate, o, a.B, a.T, a.Hk,
                       a.Hv, C, C, a.Hv};
+        p.status = a.status;
         if ((err = launch_prefill(p, stream))) return err;
     }
     // 5. gated RMSNorm tail -> bf16

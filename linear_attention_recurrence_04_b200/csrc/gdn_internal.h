@@ -37,6 +37,7 @@ struct PrefillArgs {
     int64_t qk_stride = 0;
     int64_t v_stride = 0;
     int64_t bg_stride = 0;
+    uint32_t* status = nullptr;   // optional device word for timeout bits
 };
 
 struct LayerArgs {

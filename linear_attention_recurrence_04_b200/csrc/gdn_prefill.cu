@@ -59,9 +59,10 @@
 
 #include "gdn_common.cuh"
 #include "gdn_internal.h"
+#include "gdn_tc.cuh"
 
 #ifndef GDN_PREFILL_STAGES
-#define GDN_PREFILL_STAGES 4       // stages in flight (at least 2)
+#define GDN_PREFILL_STAGES 3       // stages in flight (at least 2)
 #endif
 #ifndef GDN_PREFILL_GDN_LPR
 #define GDN_PREFILL_GDN_LPR 4      // scalar decay: lanes per state row (4 or 8)
@@ -74,6 +75,9 @@
 #endif
 #ifndef GDN_PREFILL_LOADER_WARP
 #define GDN_PREFILL_LOADER_WARP 1  // scalar decay: one extra warp issues every stage copy
+#endif
+#ifndef GDN_PREFILL_MBAR
+#define GDN_PREFILL_MBAR 1         // scalar decay: stage handoff through mbarriers, no block barrier
 #endif
 #ifndef GDN_PREFILL_UNROLL
 #define GDN_PREFILL_UNROLL 8       // positions per unrolled block of a stage
@@ -224,7 +228,7 @@ prefill_kernel(float* __restrict__ state, const float* __restrict__ q,
                const float* __restrict__ k, const float* __restrict__ v,
                const float* __restrict__ beta, const float* __restrict__ gate,
                float* __restrict__ out, int64_t T, int Hk, int Hv, int units_lo, int n_big,
-               int64_t qk_stride, int64_t v_stride, int64_t bg_stride) {
+               int64_t qk_stride, int64_t v_stride, int64_t bg_stride, uint32_t* status) {
     constexpr int S = stages_for<kCh>();
     constexpr int TS = kCh ? kTSChannel : kTS;      // positions per stage
     using StageT = Stage<NH, kCh>;
@@ -240,6 +244,11 @@ prefill_kernel(float* __restrict__ state, const float* __restrict__ q,
     __shared__ Group grp_of[kMaxGroups];
     // kCh: the running scale of each state column (see convert_stage)
     __shared__ __align__(16) float s_col[kCh ? kMaxGroups : 1][NH][kCh ? kDk : 4];
+    // kPipe (scalar decay with a loader warp): stage s is full once the
+    // loader's copies of it have landed (one arrival per loader lane), and
+    // empty again once every warp with rows has finished it.
+    constexpr bool kPipe = !kCh && Layout<kCh>::Loader && GDN_PREFILL_MBAR;
+    __shared__ __align__(8) uint64_t pipe_full[kPipe ? S : 1], pipe_empty[kPipe ? S : 1];
 
     const int tid = threadIdx.x;
     const int nthreads = blockDim.x;
@@ -273,6 +282,15 @@ prefill_kernel(float* __restrict__ state, const float* __restrict__ q,
     if constexpr (kCh) {
         for (int idx = tid; idx < kMaxGroups * NH * kDk; idx += nthreads) (&s_col[0][0][0])[idx] = 1.0f;
     }
+    if constexpr (kPipe) {
+        if (tid == 0) {
+            for (int i = 0; i < S; ++i) {
+                tc::mbar_init(tc::smem_u32(&pipe_full[i]), 32);
+                tc::mbar_init(tc::smem_u32(&pipe_empty[i]), static_cast<uint32_t>(count));
+            }
+            tc::fence_mbar_init();
+        }
+    }
     __syncthreads();
 
     // ---- stage loader: every thread issues a share of the copies; positions
@@ -297,7 +315,7 @@ prefill_kernel(float* __restrict__ state, const float* __restrict__ q,
                 float* dst = &st.kq[gi][tp][which][chunk * 4];
                 if (t < T) {
                     cp_async16(dst, (which ? q : k) + (G.b * T + t) * qk_stride + G.g * kDk + chunk * 4);
-                } else {
+                } else if (!kPipe) {
                     *reinterpret_cast<float4*>(dst) = make_float4(0.f, 0.f, 0.f, 0.f);
                 }
             }
@@ -311,7 +329,7 @@ prefill_kernel(float* __restrict__ state, const float* __restrict__ q,
                 if (t < T) {
                     const int h = G.g + (G.grp * NH + n) * Hk;
                     cp_async16(dst, v + (G.b * T + t) * v_stride + h * kDv + G.row_lo + chunk * 4);
-                } else {
+                } else if (!kPipe) {
                     *reinterpret_cast<float4*>(dst) = make_float4(0.f, 0.f, 0.f, 0.f);
                 }
             }
@@ -324,7 +342,7 @@ prefill_kernel(float* __restrict__ state, const float* __restrict__ q,
                 if (t < T && !(kCh && which)) {
                     const int h = G.g + (G.grp * NH + n) * Hk;
                     cp_async4(dst, (which ? gate : beta) + (G.b * T + t) * bg_stride + h);
-                } else {
+                } else if (!kPipe) {
                     *dst = 0.0f;
                 }
             }
@@ -457,12 +475,15 @@ prefill_kernel(float* __restrict__ state, const float* __restrict__ q,
     float* out_next = out + (G.b * T * Hv + G.g + (G.grp * NH + my_n) * Hk) * kDv + j0 + my_r;
     float* out_prev = out_next;
 
-    // Prologue: request the first S - 1 stages, then load the state rows.
+    // Prologue: request the first S - 1 stages (kPipe: the loader's loop
+    // does), then load the state rows.
     const int64_t n_stages = (T + TS - 1) / TS;
+    if constexpr (!kPipe) {
 #pragma unroll
-    for (int s2 = 0; s2 < S - 1; ++s2) {
-        if (s2 < n_stages) load_stage(static_cast<int64_t>(s2) * TS, stages[s2]);
-        cp_async_commit();
+        for (int s2 = 0; s2 < S - 1; ++s2) {
+            if (s2 < n_stages) load_stage(static_cast<int64_t>(s2) * TS, stages[s2]);
+            cp_async_commit();
+        }
     }
 
     float4 w[NH][kRPL][kChunks];
@@ -493,19 +514,8 @@ prefill_kernel(float* __restrict__ state, const float* __restrict__ q,
     }
     bool out_pending = false;
 
-    for (int64_t s = 0; s < n_stages; ++s) {
-        cp_async_wait<S - 2>();             // this thread's copies of stage s landed
-        __syncthreads();                     // ... and everyone's; stage s-1 is consumed
-        {
-            const int64_t nxt = s + S - 1;
-            if (nxt < n_stages) load_stage(nxt * TS, stages[nxt % S]);
-            cp_async_commit();
-        }
-        if constexpr (kCh) {
-            convert_stage(stages[s % S]);
-            __syncthreads();
-        }
-        if (!active) continue;
+    // One stage's positions for a warp with rows (the stage has landed).
+    auto stage_body = [&](int64_t s) {
         const StageT& st = stages[s % S];
         const int64_t t0 = s * TS;
         const int tp_end = (T - t0) < TS ? static_cast<int>(T - t0) : TS;
@@ -750,8 +760,58 @@ prefill_kernel(float* __restrict__ state, const float* __restrict__ q,
         };
         if (kCh && (mode & kSlow)) positions(std::true_type{});
         else positions(std::false_type{});
+    };
+
+    if constexpr (kPipe) {
+        // The loader fills stage si once its slot is empty; each warp with
+        // rows waits for its stage to fill and frees it after its positions.
+        // Every wait is bounded: on a timeout the warp stops and reports.
+        bool timed_out = false;
+        if (is_loader) {
+            for (int64_t si = 0; si < n_stages; ++si) {
+                const int slot = static_cast<int>(si % S);
+                if (si >= S && !tc::mbar_wait(tc::smem_u32(&pipe_empty[slot]),
+                                              static_cast<uint32_t>((si / S - 1) & 1))) {
+                    timed_out = true;
+                    break;
+                }
+                load_stage(si * TS, stages[slot]);
+                asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];"
+                             ::"r"(tc::smem_u32(&pipe_full[slot])) : "memory");
+            }
+            asm volatile("cp.async.wait_all;" ::: "memory");   // nothing left in flight
+        } else if (active) {
+            for (int64_t s = 0; s < n_stages; ++s) {
+                const int slot = static_cast<int>(s % S);
+                if (!tc::mbar_wait(tc::smem_u32(&pipe_full[slot]),
+                                   static_cast<uint32_t>((s / S) & 1))) {
+                    timed_out = true;
+                    break;
+                }
+                stage_body(s);
+                __syncwarp();
+                if (lane == 0) tc::mbar_arrive(tc::smem_u32(&pipe_empty[slot]));
+            }
+        }
+        if (timed_out && status != nullptr && lane == 0) atomicOr(status, tc::kTimeoutPrefill);
+    } else {
+        for (int64_t s = 0; s < n_stages; ++s) {
+            cp_async_wait<S - 2>();             // this thread's copies of stage s landed
+            __syncthreads();                     // ... and everyone's; stage s-1 is consumed
+            {
+                const int64_t nxt = s + S - 1;
+                if (nxt < n_stages) load_stage(nxt * TS, stages[nxt % S]);
+                cp_async_commit();
+            }
+            if constexpr (kCh) {
+                convert_stage(stages[s % S]);
+                __syncthreads();
+            }
+            if (!active) continue;
+            stage_body(s);
+        }
+        cp_async_wait<0>();
     }
-    cp_async_wait<0>();
 
     if (active) {
         // the last position's output
@@ -829,7 +889,7 @@ cudaError_t launch_nh(const PrefillArgs& a, cudaStream_t stream) {
     const int64_t bg_stride = a.bg_stride ? a.bg_stride : a.Hv;
     prefill_kernel<NH, kCh><<<static_cast<unsigned>(grid), 32 * warps, smem, stream>>>(
         a.state, a.q, a.k, a.v, a.beta, a.gate, a.out, a.T, a.Hk, a.Hv, units_lo, n_big,
-        qk_stride, v_stride, bg_stride);
+        qk_stride, v_stride, bg_stride, a.status);
     return cudaGetLastError();
 }
 

@@ -19,6 +19,7 @@ namespace tc {
 constexpr uint32_t kTimeoutProducer = 1u;
 constexpr uint32_t kTimeoutMma = 2u;
 constexpr uint32_t kTimeoutEpilogue = 4u;
+constexpr uint32_t kTimeoutPrefill = 8u;     // the prefill's stage pipeline
 // Every wait gives up after this long (nanoseconds of %globaltimer).
 constexpr uint64_t kWaitLimitNs = 2000000000ull;
 

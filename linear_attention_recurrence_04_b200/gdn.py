@@ -70,7 +70,7 @@ def load_library(path: Optional[str] = None) -> ctypes.CDLL:
     lib.gdn_step.restype = ctypes.c_int
     lib.gdn_step.argtypes = [_VP] * 7 + [_I64] * 6 + [_VP]
     lib.gdn_prefill.restype = ctypes.c_int
-    lib.gdn_prefill.argtypes = [_VP] * 7 + [_I64] * 6 + [_VP]
+    lib.gdn_prefill.argtypes = [_VP] * 7 + [_I64] * 6 + [_VP, _VP]
     lib.gdn_pair.restype = ctypes.c_int
     lib.gdn_pair.argtypes = [_VP] * 8 + [_I64] * 6 + [_VP]
     lib.gdn_layer_decode.restype = ctypes.c_int
@@ -198,9 +198,11 @@ def pair(state, scratch_state, q, k, v, beta, gate, out=None, *, stream=None):
     return out
 
 
-def prefill(state, q, k, v, beta, gate, out=None, *, stream=None):
+def prefill(state, q, k, v, beta, gate, out=None, *, status=None, stream=None):
     """T positions in order: state [B,Hv,128,128] (initial -> final, in place),
-    q/k [B,T,Hk,128], v [B,T,Hv,128], beta/gate [B,T,Hv]. Returns out [B,T,Hv,128]."""
+    q/k [B,T,Hk,128], v [B,T,Hv,128], beta/gate [B,T,Hv]. Returns out [B,T,Hv,128].
+    `status`, if given, is a zero-initialised one-element int32 CUDA tensor that
+    receives timeout bits (non-zero only if a bounded wait ever gave up)."""
     if state.dim() != 4:
         raise ValueError("state must be [B, Hv, dv, dk]")
     B, Hv, dv, dk = state.shape
@@ -215,8 +217,13 @@ def prefill(state, q, k, v, beta, gate, out=None, *, stream=None):
     for n, t in zip(names[1:], tensors[1:]):
         if tuple(t.shape) != expect[n]:
             raise ValueError(f"{n} has shape {tuple(t.shape)}, expected {expect[n]}")
+    sp = None
+    if status is not None:
+        if status.dtype is not torch.int32 or status.device != device or status.numel() != 1:
+            raise TypeError("status must be a one-element int32 tensor on the same device")
+        sp = status.data_ptr()
     st = _call(device, load_library().gdn_prefill, *(_ptr(t) for t in tensors), B, T, Hk, Hv,
-               dk, dv, _stream(device, stream))
+               dk, dv, sp, _stream(device, stream))
     _raise_on("gdn_prefill", st)
     return out
 

@@ -88,14 +88,15 @@ def test_prefill_argument_checks(lib):
     f = lambda **kw: lib.gdn_prefill(kw.get("state", A16), A16b, A16c, fake(3), fake(4),
                                      fake(5), kw.get("out", fake(6)), kw.get("B", 1),
                                      kw.get("T", 4), kw.get("Hk", 16), kw.get("Hv", 32),
-                                     128, 128, None)
+                                     128, 128, kw.get("status", None), None)
     assert f(T=-1) == SHAPE
     assert f(Hv=17) == SHAPE
     assert f(state=0) == NULL
     assert f(state=A16 + 8) == ALIGN
+    assert f(status=fake(8) + 2) == ALIGN
     assert f(out=A16b) == ALIAS
-    assert lib.gdn_prefill(0, 0, 0, 0, 0, 0, 0, 2, 0, 16, 32, 128, 128, None) == OK
-    assert lib.gdn_prefill(0, 0, 0, 0, 0, 0, 0, 0, 9, 16, 32, 128, 128, None) == OK
+    assert lib.gdn_prefill(0, 0, 0, 0, 0, 0, 0, 2, 0, 16, 32, 128, 128, None, None) == OK
+    assert lib.gdn_prefill(0, 0, 0, 0, 0, 0, 0, 0, 9, 16, 32, 128, 128, None, None) == OK
 
 
 def pair_call(lib, state=A16, scratch=fake(7), q=A16b, k=A16c, v=fake(3), beta=fake(4),

@@ -20,9 +20,13 @@ def to_dev(d):
 
 
 def run_gpu(d):
+    """Runs through the C ABI with a status word, which must stay zero: no
+    bounded wait of the stage pipeline gave up."""
     t = to_dev(d)
-    out = gdn.prefill(t["state"], t["q"], t["k"], t["v"], t["beta"], t["gate"])
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    out = gdn.prefill(t["state"], t["q"], t["k"], t["v"], t["beta"], t["gate"], status=status)
     torch.cuda.synchronize()
+    assert int(status.item()) == 0, "prefill pipeline timeout bit set"
     return t["state"].cpu().numpy(), out.cpu().numpy()
 
 
