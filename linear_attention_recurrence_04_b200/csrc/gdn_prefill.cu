@@ -23,8 +23,14 @@
 //  * Inputs are staged in shared memory S stages of TS positions ahead with
 //    16-byte asynchronous copies (cp.async), shared by all warps of the CTA:
 //    k and q rows once per group and position, each warp's v rows, beta and
-//    gate. Positions past T are zero-filled. The decays exp(gate) of a stage
-//    are computed once per warp (one per lane) and broadcast by shuffle.
+//    gate. The decays exp(gate) of a stage are computed once per warp (one
+//    per lane) and broadcast by shuffle. Scalar decay: one loader warp (the
+//    CTA's last) issues every copy, and stages pass to the warps with rows
+//    through per-stage full/empty mbarriers with bounded waits, with no block
+//    barrier in the loop; positions past T are never consumed and are left
+//    unwritten. Per-channel decay: every thread issues a share of the copies,
+//    positions past T are zero-filled, and block barriers bracket each
+//    stage's conversion.
 //  * Software pipeline across positions: after the rank-1 update of position
 //    t, one pass over the register-resident rows makes both the output dot
 //    W.q_t and the next position's key dot W.k_{t+1} (both read the same
