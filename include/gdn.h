@@ -28,10 +28,15 @@
  *     other argument; `out` and the scratch outputs must not overlap any
  *     argument either (GDN_ERR_ALIAS otherwise). Read-only inputs may share
  *     memory.
- *   - Alignment: state, q, k, v, g, out, mixed_qkv, z, conv_ring, conv_w,
- *     hidden, x and the weight matrices must be 16-byte aligned, workspaces
- *     256-byte aligned; the per-head scalars (beta, gate, a, b, A_log,
- *     dt_bias) and norm_w need 4-byte alignment.
+ *   - Alignment: state, scratch_state, q, k, v, g, out, mixed_qkv, z,
+ *     conv_ring, conv_w, hidden, x and the weight matrices must be 16-byte
+ *     aligned, workspaces 256-byte aligned; the per-head scalars (beta,
+ *     gate, a, b, A_log, dt_bias), norm_w and the optional status words need
+ *     4-byte alignment.
+ *   - Status words (gdn_prefill, gdn_linear_bf16, gdn_forward_batch*,
+ *     gdn_short_conv_*): an optional zero-initialised device uint32 into
+ *     which a kernel ORs a bit if one of its bounded waits (2 s) ever gives
+ *     up; the kernel then returns without hanging. NULL: not reported.
  *   - Arguments are checked on the host before anything is enqueued; on any
  *     error nothing is written and nothing is launched. A problem with no
  *     work (a zero size) returns GDN_OK without touching any pointer.
