@@ -128,14 +128,13 @@ struct Layout {
     static_assert(MaxWarps <= UnitsPerHead, "a run must span at most two groups");
 };
 
-// Shared-memory image of one stage. kCh (per-channel decay): alpha holds g
-// as copied, then exp(g); ka holds exp(g) * k. Without kCh both are stubs.
-// Slot TS of kq (k only) holds the first position of the next stage, so a
-// pass always reads the next key from its own stage. kCh (per-channel decay)
-// adds, per value head: ks, the key-dot vectors (g as copied, then
-// converted, with slot TS as well), kd and qs, the update and output vectors,
-// mult, the scales folded into the state when the stage starts, and mode,
-// one word per group (kFold | kSlow). Without kCh those are stubs.
+// Shared-memory image of one stage. Slot TS of kq (k only) holds the first
+// position of the next stage, so a pass always reads the next key from its
+// own stage. kCh (per-channel decay) adds, per value head: ks, the key-dot
+// vectors (g as copied, then converted, with slot TS as well), kd and qs,
+// the update and output vectors, dec, the per-element decays a kSlow stage
+// applies, mult, the scales folded into the state when the stage starts, and
+// mode, one word per group (kFold | kSlow). Without kCh those are stubs.
 template <int NH, bool kCh>
 struct alignas(16) Stage {    // stages sit back to back: each starts 16-byte aligned
     static constexpr int TS = kCh ? kTSChannel : kTS;   // positions per stage
@@ -148,14 +147,16 @@ struct alignas(16) Stage {    // stages sit back to back: each starts 16-byte al
     float ks[CG][CT + 1][NH][CD];
     float kd[CG][CT][NH][CD];
     float qs[CG][CT][NH][CD];
+    float dec[CG][CT][NH][CD];
     float mult[CG][NH][CD];
     int mode[kMaxGroups];
 };
 
-// Per-channel stage modes, one word per group: fold the column scales into
-// the state before the stage (kFold); apply the decays element by element
-// because a column's product of decays leaves [kScaleLo, kScaleHi] within
-// the stage (kSlow, always with kFold).
+// Per-channel stage modes, one word per group: some column folds its scale
+// into the state before the stage (kFold; every column's mult is written, 1
+// where it does not fold); some column's product of decays leaves
+// [kScaleLo, kScaleHi] within the stage, so the stage applies dec element by
+// element (kSlow, with that column folded).
 constexpr int kFold = 1;
 constexpr int kSlow = 2;
 
@@ -371,14 +372,20 @@ prefill_kernel(float* __restrict__ state, const float* __restrict__ q,
     };
     // kCh: turn a landed stage's g into the vectors of its passes. Column i
     // of head n is held as W[j][i] with M[j][i] = S[i] W[j][i]; S (s_col)
-    // carries over between stages. A fast stage runs, per position t,
-    //   S <- S alpha_t,  ks_t = S k_t,  kd_t = k_t / S,  qs_t = S q_t,
-    // so that sk = W.ks_t, W += delta kd_t and out = W.qs_t (slot TS of ks:
-    // S alpha k of the next stage's first position). A slow stage keeps
-    // S = 1, stores kd_t = alpha_t and ks_t = alpha_t k_t, and its passes
-    // decay W element by element. Pass 1 flags each group: kFold when S
-    // times the stage's product of decays would leave [kScaleLo, kScaleHi],
-    // kSlow when that product alone does. Pass 2 writes the vectors.
+    // carries over between stages. Each column decides on its own, in one
+    // pass, so no barrier separates decision and vectors:
+    //  * a column whose S times the stage's product of decays stays within
+    //    [kScaleLo, kScaleHi] runs, per position t, S <- S alpha_t,
+    //    ks_t = S k_t, kd_t = k_t / S, qs_t = S q_t, dec_t = 1, so that
+    //    sk = W.ks_t, W += delta kd_t and out = W.qs_t (slot TS of ks: S alpha k
+    //    of the next stage's first position);
+    //  * a column whose S times that product leaves the range folds S into W
+    //    (mult = S) and runs as above from S = 1 (kFold);
+    //  * a column whose product alone leaves the range (an underflowing decay,
+    //    strong growth) folds and keeps S = 1: dec_t = alpha_t, kd_t = k_t,
+    //    qs_t = q_t, ks_t = alpha_t k_t, and a stage with such a column runs
+    //    its passes with the decay applied element by element (kSlow), which
+    //    the other columns' vectors (dec = 1) fit as well.
     auto convert_stage = [&](StageT& st) {
         if constexpr (kCh) {
             const int ncols = n_groups * NH * kDk;
@@ -400,25 +407,20 @@ prefill_kernel(float* __restrict__ state, const float* __restrict__ q,
                         fold |= !(sc2 >= kScaleLo && sc2 <= kScaleHi);
                     }
                 }
-                if (slow || fold) atomicOr(&st.mode[gi2], slow ? (kSlow | kFold) : kFold);
-            }
-            __syncthreads();
-            for (int idx = tid; idx < ncols; idx += nthreads) {
-                const int col = idx % kDk;
-                const int n = (idx / kDk) % NH;
-                const int gi2 = idx / (kDk * NH);
-                const int mode = st.mode[gi2];
-                float sv = s_col[gi2][n][col];
-                if (mode & kFold) {
-                    st.mult[gi2][n][col] = sv;
-                    sv = 1.0f;
-                }
-                if (mode & kSlow) {
+                fold |= slow;
+                st.mult[gi2][n][col] = fold ? s0 : 1.0f;
+                float sv = fold ? 1.0f : s0;
+                if (slow) {
 #pragma unroll
                     for (int tp = 0; tp <= TS; ++tp) {
                         const float a = st.ks[gi2][tp][n][col];
-                        if (tp < TS) st.kd[gi2][tp][n][col] = a;
-                        st.ks[gi2][tp][n][col] = a * st.kq[gi2][tp][0][col];
+                        const float kv = st.kq[gi2][tp][0][col];
+                        if (tp < TS) {
+                            st.dec[gi2][tp][n][col] = a;
+                            st.kd[gi2][tp][n][col] = kv;
+                            st.qs[gi2][tp][n][col] = st.kq[gi2][tp][1][col];
+                        }
+                        st.ks[gi2][tp][n][col] = a * kv;
                     }
                 } else {
 #pragma unroll
@@ -428,10 +430,12 @@ prefill_kernel(float* __restrict__ state, const float* __restrict__ q,
                         st.ks[gi2][tp][n][col] = sv * kv;
                         st.kd[gi2][tp][n][col] = kv * rcp_approx(sv);
                         st.qs[gi2][tp][n][col] = sv * st.kq[gi2][tp][1][col];
+                        st.dec[gi2][tp][n][col] = 1.0f;
                     }
                     st.ks[gi2][TS][n][col] = (sv * st.ks[gi2][TS][n][col]) * st.kq[gi2][TS][0][col];
                 }
                 s_col[gi2][n][col] = sv;
+                if (fold) atomicOr(&st.mode[gi2], slow ? (kSlow | kFold) : kFold);
             }
         }
     };
@@ -539,6 +543,7 @@ prefill_kernel(float* __restrict__ state, const float* __restrict__ q,
         const float* ks_s = &st.ks[gi * kCh][0][0][ccol];
         const float* kd_s = &st.kd[gi * kCh][0][0][ccol];
         const float* qs_s = &st.qs[gi * kCh][0][0][ccol];
+        const float* dec_s = &st.dec[gi * kCh][0][0][ccol];
 
         // decays of this stage, one per lane: lane tp + TS n holds exp(gate)
         const float e_lane =
@@ -582,8 +587,8 @@ prefill_kernel(float* __restrict__ state, const float* __restrict__ q,
         }
 
         // The positions of the stage. kSlowPath (kCh only): decay element by
-        // element with kd = alpha, update with k, output with q, next key
-        // dot with ks = alpha k.
+        // element with dec, then the same update, output and next-key vectors
+        // (kd, qs, ks) as a fast stage.
         auto positions = [&](auto slow_tag) {
             constexpr bool kSlowPath = decltype(slow_tag)::value;
 #pragma unroll(kUnroll)
@@ -711,11 +716,11 @@ prefill_kernel(float* __restrict__ state, const float* __restrict__ q,
                 // (c) one pass: step 4 for t, then W.q_t (step 5) and the next
                 // position's key dot. Slot tp + 1 always exists; past T it is
                 // zero-filled.
-                const float* kp = kq_s + tp * kqP;
+                [[maybe_unused]] const float* kp = kq_s + tp * kqP;   // scalar decay only
 #pragma unroll
                 for (int i = 0; i < kChunks; ++i) {
                     float4 kv_sh = make_float4(0.f, 0.f, 0.f, 0.f), qv_sh = kv_sh, nv_sh = kv_sh;
-                    if constexpr (!kCh || kSlowPath) {
+                    if constexpr (!kCh) {
                         kv_sh = ld_s4(kp + kStep * i);
                         qv_sh = ld_s4(kp + kDk + kStep * i);
                     }
@@ -726,12 +731,9 @@ prefill_kernel(float* __restrict__ state, const float* __restrict__ q,
                         if constexpr (kCh) {
                             const int off = tp * chP + n * kDk + kStep * i;
                             nv = ld_s4(ks_s + off + chP);
-                            if constexpr (kSlowPath) {
-                                al = ld_s4(kd_s + off);
-                            } else {
-                                uv = ld_s4(kd_s + off);
-                                qv = ld_s4(qs_s + off);
-                            }
+                            uv = ld_s4(kd_s + off);
+                            qv = ld_s4(qs_s + off);
+                            if constexpr (kSlowPath) al = ld_s4(dec_s + off);
                         }
 #pragma unroll
                         for (int r = 0; r < kRPL; ++r) {
