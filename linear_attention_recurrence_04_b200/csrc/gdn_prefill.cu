@@ -388,54 +388,65 @@ prefill_kernel(float* __restrict__ state, const float* __restrict__ q,
     //    the other columns' vectors (dec = 1) fit as well.
     auto convert_stage = [&](StageT& st) {
         if constexpr (kCh) {
-            const int ncols = n_groups * NH * kDk;
-            for (int idx = tid; idx < ncols; idx += nthreads) {
-                const int col = idx % kDk;
-                const int n = (idx / kDk) % NH;
-                const int gi2 = idx / (kDk * NH);
-                const float s0 = s_col[gi2][n][col];
-                float cum = 1.0f;
-                bool slow = false, fold = false;
+            // two adjacent columns per thread, with 8-byte shared accesses;
+            // each column decides on its own
+            auto f2 = [](float* ptr) -> float2& { return *reinterpret_cast<float2*>(ptr); };
+            const int npairs = n_groups * NH * (kDk / 2);
+            for (int pidx = tid; pidx < npairs; pidx += nthreads) {
+                const int col = (pidx % (kDk / 2)) * 2;
+                const int n = (pidx / (kDk / 2)) % NH;
+                const int gi2 = pidx / ((kDk / 2) * NH);
+                const float2 s0 = f2(&s_col[gi2][n][col]);
+                float2 cum = make_float2(1.0f, 1.0f);
+                bool slow0 = false, slow1 = false, fold0 = false, fold1 = false;
 #pragma unroll
                 for (int tp = 0; tp <= TS; ++tp) {
-                    const float a = expf(st.ks[gi2][tp][n][col]);
-                    st.ks[gi2][tp][n][col] = a;
+                    const float2 g2 = f2(&st.ks[gi2][tp][n][col]);
+                    const float2 a = make_float2(expf(g2.x), expf(g2.y));
+                    f2(&st.ks[gi2][tp][n][col]) = a;
                     if (tp < TS) {
-                        cum *= a;
-                        const float sc2 = s0 * cum;
-                        slow |= !(cum >= kScaleLo && cum <= kScaleHi);
-                        fold |= !(sc2 >= kScaleLo && sc2 <= kScaleHi);
+                        cum.x *= a.x;
+                        cum.y *= a.y;
+                        const float sx = s0.x * cum.x, sy = s0.y * cum.y;
+                        slow0 |= !(cum.x >= kScaleLo && cum.x <= kScaleHi);
+                        slow1 |= !(cum.y >= kScaleLo && cum.y <= kScaleHi);
+                        fold0 |= !(sx >= kScaleLo && sx <= kScaleHi);
+                        fold1 |= !(sy >= kScaleLo && sy <= kScaleHi);
                     }
                 }
-                fold |= slow;
-                st.mult[gi2][n][col] = fold ? s0 : 1.0f;
-                float sv = fold ? 1.0f : s0;
-                if (slow) {
+                fold0 |= slow0;
+                fold1 |= slow1;
+                f2(&st.mult[gi2][n][col]) = make_float2(fold0 ? s0.x : 1.0f, fold1 ? s0.y : 1.0f);
+                float2 sv = make_float2(fold0 ? 1.0f : s0.x, fold1 ? 1.0f : s0.y);
 #pragma unroll
-                    for (int tp = 0; tp <= TS; ++tp) {
-                        const float a = st.ks[gi2][tp][n][col];
-                        const float kv = st.kq[gi2][tp][0][col];
-                        if (tp < TS) {
-                            st.dec[gi2][tp][n][col] = a;
-                            st.kd[gi2][tp][n][col] = kv;
-                            st.qs[gi2][tp][n][col] = st.kq[gi2][tp][1][col];
-                        }
-                        st.ks[gi2][tp][n][col] = a * kv;
-                    }
-                } else {
-#pragma unroll
-                    for (int tp = 0; tp < TS; ++tp) {
-                        sv *= st.ks[gi2][tp][n][col];
-                        const float kv = st.kq[gi2][tp][0][col];
-                        st.ks[gi2][tp][n][col] = sv * kv;
-                        st.kd[gi2][tp][n][col] = kv * rcp_approx(sv);
-                        st.qs[gi2][tp][n][col] = sv * st.kq[gi2][tp][1][col];
-                        st.dec[gi2][tp][n][col] = 1.0f;
-                    }
-                    st.ks[gi2][TS][n][col] = (sv * st.ks[gi2][TS][n][col]) * st.kq[gi2][TS][0][col];
+                for (int tp = 0; tp < TS; ++tp) {
+                    const float2 a = f2(&st.ks[gi2][tp][n][col]);
+                    const float2 kv = f2(&st.kq[gi2][tp][0][col]);
+                    const float2 qv = f2(&st.kq[gi2][tp][1][col]);
+                    // fast column: S <- S alpha, ks = S k, kd = k / S, qs = S q, dec = 1;
+                    // slow column: S stays 1, ks = alpha k, kd = k, qs = q, dec = alpha
+                    if (!slow0) sv.x *= a.x;
+                    if (!slow1) sv.y *= a.y;
+                    f2(&st.ks[gi2][tp][n][col]) =
+                        make_float2((slow0 ? a.x : sv.x) * kv.x, (slow1 ? a.y : sv.y) * kv.y);
+                    f2(&st.kd[gi2][tp][n][col]) =
+                        make_float2(slow0 ? kv.x : kv.x * rcp_approx(sv.x),
+                                    slow1 ? kv.y : kv.y * rcp_approx(sv.y));
+                    f2(&st.qs[gi2][tp][n][col]) =
+                        make_float2(slow0 ? qv.x : sv.x * qv.x, slow1 ? qv.y : sv.y * qv.y);
+                    f2(&st.dec[gi2][tp][n][col]) =
+                        make_float2(slow0 ? a.x : 1.0f, slow1 ? a.y : 1.0f);
                 }
-                s_col[gi2][n][col] = sv;
-                if (fold) atomicOr(&st.mode[gi2], slow ? (kSlow | kFold) : kFold);
+                {   // slot TS: the key dot of the next stage's first position
+                    const float2 a = f2(&st.ks[gi2][TS][n][col]);
+                    const float2 kv = f2(&st.kq[gi2][TS][0][col]);
+                    f2(&st.ks[gi2][TS][n][col]) =
+                        make_float2((slow0 ? a.x : sv.x * a.x) * kv.x,
+                                    (slow1 ? a.y : sv.y * a.y) * kv.y);
+                }
+                f2(&s_col[gi2][n][col]) = sv;
+                if (fold0 || fold1)
+                    atomicOr(&st.mode[gi2], (slow0 || slow1) ? (kSlow | kFold) : kFold);
             }
         }
     };
