@@ -68,7 +68,7 @@
 #include "gdn_tc.cuh"
 
 #ifndef GDN_PREFILL_STAGES
-#define GDN_PREFILL_STAGES 3       // stages in flight (at least 2)
+#define GDN_PREFILL_STAGES 2       // stages in flight (at least 2)
 #endif
 #ifndef GDN_PREFILL_GDN_LPR
 #define GDN_PREFILL_GDN_LPR 4      // scalar decay: lanes per state row (4 or 8)
@@ -93,7 +93,10 @@ namespace gdn {
 
 namespace {
 
-constexpr int kTS = 16;                         // positions per stage (scalar decay)
+#ifndef GDN_PREFILL_TS
+#define GDN_PREFILL_TS 32          // positions per stage (scalar decay)
+#endif
+constexpr int kTS = GDN_PREFILL_TS;             // positions per stage (scalar decay)
 constexpr int kTSChannel = 8;                   // positions per stage (per-channel decay)
 constexpr int kStages = GDN_PREFILL_STAGES;
 constexpr int kUnroll = GDN_PREFILL_UNROLL;        // positions per unrolled block
@@ -556,9 +559,13 @@ prefill_kernel(float* __restrict__ state, const float* __restrict__ q,
         const float* qs_s = &st.qs[gi * kCh][0][0][ccol];
         const float* dec_s = &st.dec[gi * kCh][0][0][ccol];
 
-        // decays of this stage, one per lane: lane tp + TS n holds exp(gate)
-        const float e_lane =
-            (!kCh && lane < TS * NH) ? expf(st.bg[gi][lane % TS][lane / TS][1]) : 1.0f;
+        // decays of this stage: lane tp holds exp(gate) of position tp for
+        // each head (stages of at most 32 positions)
+        static_assert(kCh || TS <= 32, "one lane per position of a stage");
+        float e_lane[NH];
+#pragma unroll
+        for (int n = 0; n < NH; ++n)
+            e_lane[n] = (!kCh && lane < TS) ? expf(st.bg[gi][lane % TS][n][1]) : 1.0f;
 
         int mode = 0;
         if constexpr (kCh) {
@@ -632,7 +639,7 @@ prefill_kernel(float* __restrict__ state, const float* __restrict__ q,
                     bool fold = false;
 #pragma unroll
                     for (int n = 0; n < NH; ++n) {
-                        s_new[n] = sc[n] * __shfl_sync(kFull, e_lane, tp + TS * n);
+                        s_new[n] = sc[n] * __shfl_sync(kFull, e_lane[n], tp);
                         fold |= !(s_new[n] >= kScaleLo && s_new[n] <= kScaleHi);
                     }
                     if (fold) {          // rare, and uniform across the warp
@@ -687,7 +694,7 @@ prefill_kernel(float* __restrict__ state, const float* __restrict__ q,
                         bool fold = false;
 #pragma unroll
                         for (int n = 0; n < NH; ++n) {
-                            s_new[n] = sc[n] * __shfl_sync(kFull, e_lane, tp + TS * n);
+                            s_new[n] = sc[n] * __shfl_sync(kFull, e_lane[n], tp);
                             fold |= !(s_new[n] >= kScaleLo && s_new[n] <= kScaleHi);
                         }
                         if (fold) {      // rare, and uniform across the warp
