@@ -236,6 +236,20 @@ gdn_status gdn_linear_bf16(const void *x, const void *w, float *y, int64_t M, in
                            int64_t K, uint32_t *status, void *stream);
 
 /*
+ * gdn_linear_bf16_split_k -- the same product for decode-sized calls. With
+ * M <= 128 rows, K is split into S chunks (S <= 8, fixed by N, K and the
+ * device, never by M); the S CTAs of a thread-block cluster each accumulate
+ * one chunk on the tensor cores and the chunk sums are added in fp32 in chunk
+ * order through distributed shared memory. Every row is then the same in any
+ * call of at most 128 rows; it differs from gdn_linear_bf16's row by the
+ * rounding of that grouped sum (same error bound). M > 128, or a product too
+ * small to split, runs gdn_linear_bf16. Arguments, alignment, aliasing,
+ * status and errors as gdn_linear_bf16.
+ */
+gdn_status gdn_linear_bf16_split_k(const void *x, const void *w, float *y, int64_t M, int64_t N,
+                                   int64_t K, uint32_t *status, void *stream);
+
+/*
  * gdn_forward_batch -- the recurrent layer over T consecutive positions of
  * each of B sequences, with dense bf16 projections ("Module linear_core",
  * entry "gdn_forward_batch": the qkv/z/a/b and out_proj projections are

@@ -383,6 +383,38 @@ gdn_status check_layer(const char* fn, int npos, const float* mixed_qkv, const f
     return check_spans(ins, 12, 4, Span{out, z_n * 4, "out"});
 }
 
+
+// Checks shared by the two projection entries; `split` selects the split-K
+// launcher for products of at most 128 rows.
+gdn_status linear_call(const char* fn, const void* x, const void* w, float* y, int64_t M,
+                       int64_t N, int64_t K, uint32_t* status, void* stream, bool split) {
+    if (M < 0 || N < 0 || K < 0)
+        return fail(GDN_ERR_SHAPE, "%s: negative M=%lld N=%lld K=%lld", fn, (long long)M,
+                    (long long)N, (long long)K);
+    if (K % 8 != 0)
+        return fail(GDN_ERR_UNSUPPORTED, "%s: K=%lld must be a multiple of 8", fn, (long long)K);
+    if (M > (int64_t)65535 * 128 || N > INT32_MAX / 2 || K > INT32_MAX / 2)
+        return fail(GDN_ERR_OVERFLOW, "%s: M, N or K too large", fn);
+    int64_t xy = 0, xk = 0, wk = 0;
+    if (!mul_ok(M, N, &xy) || !mul_ok(M, K, &xk) || !mul_ok(N, K, &wk))
+        return fail(GDN_ERR_OVERFLOW, "%s: size overflow", fn);
+    if (M == 0 || N == 0) { g_last_error[0] = '\0'; return GDN_OK; }
+    if (!y || (K > 0 && (!x || !w)))
+        return fail(GDN_ERR_NULL, "%s: a tensor pointer is NULL", fn);
+    if (!aligned(y, 16) || (K > 0 && (!aligned(x, 16) || !aligned(w, 16))) ||
+        (status && !aligned(status, 4)))
+        return fail(GDN_ERR_ALIGN, "%s: x, w, y need 16-byte alignment", fn);
+    const Span ins[] = {{x, xk * 2, "x"}, {w, wk * 2, "w"}, {status, status ? 4 : 0, "status"}};
+    gdn_status st = check_spans(ins, 3, 0, Span{y, xy * 4, "y"});
+    if (st != GDN_OK) return st;
+    if (K == 0)    // an empty sum: y = 0
+        return launched(cudaMemsetAsync(y, 0, static_cast<size_t>(xy) * 4,
+                                        static_cast<cudaStream_t>(stream)), fn);
+    LinearArgs a{x, w, y, M, N, K, status};
+    const cudaStream_t cs = static_cast<cudaStream_t>(stream);
+    return launched(split ? launch_linear_bf16_split(a, cs) : launch_linear_bf16(a, cs), fn);
+}
+
 }  // namespace
 
 gdn_status gdn_layer_decode(const float* mixed_qkv, const float* z, const float* a,
@@ -432,30 +464,13 @@ gdn_status gdn_layer_pair(const float* mixed_qkv, const float* z, const float* a
 gdn_status gdn_linear_bf16(const void* x, const void* w, float* y, int64_t M, int64_t N,
                            int64_t K, uint32_t* status, void* stream) {
     NvtxRange nvtx_range("gdn_linear_bf16");
-    if (M < 0 || N < 0 || K < 0)
-        return fail(GDN_ERR_SHAPE, "gdn_linear_bf16: negative M=%lld N=%lld K=%lld", (long long)M,
-                    (long long)N, (long long)K);
-    if (K % 8 != 0)
-        return fail(GDN_ERR_UNSUPPORTED, "gdn_linear_bf16: K=%lld must be a multiple of 8", (long long)K);
-    if (M > (int64_t)65535 * 128 || N > INT32_MAX / 2 || K > INT32_MAX / 2)
-        return fail(GDN_ERR_OVERFLOW, "gdn_linear_bf16: M, N or K too large");
-    int64_t xy = 0, xk = 0, wk = 0;
-    if (!mul_ok(M, N, &xy) || !mul_ok(M, K, &xk) || !mul_ok(N, K, &wk))
-        return fail(GDN_ERR_OVERFLOW, "gdn_linear_bf16: size overflow");
-    if (M == 0 || N == 0) { g_last_error[0] = '\0'; return GDN_OK; }
-    if (!y || (K > 0 && (!x || !w)))
-        return fail(GDN_ERR_NULL, "gdn_linear_bf16: a tensor pointer is NULL");
-    if (!aligned(y, 16) || (K > 0 && (!aligned(x, 16) || !aligned(w, 16))) ||
-        (status && !aligned(status, 4)))
-        return fail(GDN_ERR_ALIGN, "gdn_linear_bf16: x, w, y need 16-byte alignment");
-    const Span ins[] = {{x, xk * 2, "x"}, {w, wk * 2, "w"}, {status, status ? 4 : 0, "status"}};
-    gdn_status st = check_spans(ins, 3, 0, Span{y, xy * 4, "y"});
-    if (st != GDN_OK) return st;
-    if (K == 0)    // an empty sum: y = 0
-        return launched(cudaMemsetAsync(y, 0, static_cast<size_t>(xy) * 4,
-                                        static_cast<cudaStream_t>(stream)), "gdn_linear_bf16");
-    LinearArgs a{x, w, y, M, N, K, status};
-    return launched(launch_linear_bf16(a, static_cast<cudaStream_t>(stream)), "gdn_linear_bf16");
+    return linear_call("gdn_linear_bf16", x, w, y, M, N, K, status, stream, false);
+}
+
+gdn_status gdn_linear_bf16_split_k(const void* x, const void* w, float* y, int64_t M, int64_t N,
+                                   int64_t K, uint32_t* status, void* stream) {
+    NvtxRange nvtx_range("gdn_linear_bf16_split_k");
+    return linear_call("gdn_linear_bf16_split_k", x, w, y, M, N, K, status, stream, true);
 }
 
 size_t gdn_forward_batch_workspace_size(int64_t B, int64_t T, int64_t Hk, int64_t Hv,

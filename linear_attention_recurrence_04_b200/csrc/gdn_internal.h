@@ -135,6 +135,11 @@ cudaError_t launch_prefill(const PrefillArgs& a, cudaStream_t stream);
 cudaError_t launch_layer_decode(const LayerArgs& a, cudaStream_t stream);
 cudaError_t launch_layer_pair(const LayerArgs& a, cudaStream_t stream);
 cudaError_t launch_linear_bf16(const LinearArgs& a, cudaStream_t stream);
+// The same product for M <= 128 split over K across a thread-block cluster
+// (fixed per (N, K) and device; rows are identical across such calls, and
+// differ from launch_linear_bf16's by accumulation order); M > 128, or a
+// product too small to split, goes to launch_linear_bf16.
+cudaError_t launch_linear_bf16_split(const LinearArgs& a, cudaStream_t stream);
 cudaError_t launch_forward_batch(const ForwardBatchArgs& a, cudaStream_t stream);
 cudaError_t launch_short_conv(const ShortConvArgs& a, cudaStream_t stream);
 

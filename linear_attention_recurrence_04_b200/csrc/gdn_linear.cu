@@ -31,7 +31,16 @@
 // so a row's result is the same in any batch. Every mbarrier wait gives up
 // after 2 s, ORs an error bit into the caller's status word (if given), lets
 // in-flight copies land and frees TMEM.
+//
+// Both kernels are launched with programmatic stream serialization: barrier
+// setup, TMEM allocation and an L2 prefetch of the weight boxes overlap the
+// tail of the previous kernel on the stream; every thread waits for that
+// kernel (griddepcontrol.wait) before its first global read or write or
+// bounded wait, and each CTA releases the next kernel once set up.
 #include <cuda.h>
+
+#include <algorithm>
+#include <atomic>
 
 #include "gdn_common.cuh"
 #include "gdn_internal.h"
@@ -120,11 +129,20 @@ linear_bf16_kernel(const __grid_constant__ CUtensorMap tmap_x,
     tc::tc_fence_after();
     const uint32_t tmem = tmem_slot;
     volatile int* vfailed = &failed;
+    tc::grid_dep_launch();
 
     if (warp == 0 && lane == 0) {
         // ---- producer: k-steps of every tile, through the stage ring --------
         tc::prefetch_tmap(&tmap_x);
         tc::prefetch_tmap(&tmap_w);
+        // the first tile's weight boxes head for L2 while the previous kernel
+        // on the stream finishes
+        if (static_cast<int>(blockIdx.x) < n_tiles) {
+            const int n0 = (static_cast<int>(blockIdx.x) % tiles_n) * BN;
+            for (int kt = 0; kt < n_kt && kt < kStages; ++kt)
+                tc::tma_prefetch_l2_2d(&tmap_w, kt * kBK, n0);
+        }
+        tc::grid_dep_wait();
         int64_t g = 0;                                     // k-steps issued so far
         for (int tile = blockIdx.x; tile < n_tiles && !*vfailed; tile += gridDim.x) {
             const int m0 = (tile / tiles_n) * BM;
@@ -147,6 +165,7 @@ linear_bf16_kernel(const __grid_constant__ CUtensorMap tmap_x,
         }
     } else if (warp == 1 && lane == 0) {
         // ---- MMA issuer: tile li accumulates into accumulator set li % kNumAcc
+        tc::grid_dep_wait();                       // bounded waits start from here
         const uint32_t idesc = tc::idesc_bf16_f32(kMmaM, BN);
         int64_t g = 0;
         bool ok = true;
@@ -190,6 +209,7 @@ linear_bf16_kernel(const __grid_constant__ CUtensorMap tmap_x,
         }
     } else if (warp >= 2) {
         // ---- epilogue: TMEM -> registers -> global, then release ------------
+        tc::grid_dep_wait();
         const int quarter = warp & 3;                      // TMEM lanes 32 q .. 32 q + 31
         int li = 0;
         for (int tile = blockIdx.x; tile < n_tiles; tile += gridDim.x, ++li) {
@@ -251,6 +271,219 @@ linear_bf16_kernel(const __grid_constant__ CUtensorMap tmap_x,
     if (warp == 1) tc::tmem_dealloc(tmem, kNumAcc * kAccCols);
 }
 
+// Split-K form for products of at most 128 rows (decode-sized calls).
+//
+// With few rows the persistent kernel's cost is one CTA's chain of K/16
+// dependent MMAs into one accumulator (32 k-steps x 4 MMAs for K = 2048), and
+// only N / BN SMs stream the weights. Here a cluster of `splits` CTAs shares
+// one 128 x BN output tile: CTA r runs k-steps [r n_kt / S, (r+1) n_kt / S)
+// into its own TMEM accumulator, parks the fp32 partial tile in its (then
+// idle) stage ring, and after a cluster barrier every CTA sums a 1/S slice of
+// the tile over the S partials through distributed shared memory, always in
+// rank order 0, 1, .., S-1, and stores it. The split depends on (N, K) and the
+// device alone, so a row's result is the same in any call of at most 128
+// rows; it differs from the persistent kernel's by the fp32 rounding of the
+// grouped sum.
+template <int BN>
+__global__ void __launch_bounds__(kThreads, 1)
+linear_bf16_splitk_kernel(const __grid_constant__ CUtensorMap tmap_x,
+                          const __grid_constant__ CUtensorMap tmap_w, float* __restrict__ y,
+                          int M, int N, int K, int splits, uint32_t* __restrict__ status) {
+    using L = LinearSmem<BN, kMmaM>;
+    constexpr int kStages = L::kStages;
+    constexpr int kPitch = BN + 4;        // floats per parked row: 16-byte shift per row
+    constexpr int kQuads = BN / 4;        // float4 columns of a row
+    static_assert(static_cast<size_t>(kMmaM) * kPitch * 4 + 1024 <= L::kDynamic,
+                  "the partial tile fits the stage ring");
+    extern __shared__ uint8_t smem_raw[];
+    __shared__ __align__(8) uint64_t full[kStages];
+    __shared__ __align__(8) uint64_t empty[kStages];
+    __shared__ __align__(8) uint64_t acc_full;
+    __shared__ uint32_t tmem_slot;
+    __shared__ int issued, consumed;
+    __shared__ int failed;
+
+    const uint32_t raw = tc::smem_u32(smem_raw);
+    const uint32_t base = (raw + 1023u) & ~1023u;
+    float* part = reinterpret_cast<float*>(smem_raw + (base - raw));
+
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+    const int rank = static_cast<int>(tc::cluster_ctarank());
+    const int n0 = static_cast<int>(blockIdx.x / splits) * BN;
+    const int n_kt = (K + kBK - 1) / kBK;
+    const int kb = static_cast<int>(static_cast<int64_t>(rank) * n_kt / splits);
+    const int ke = static_cast<int>(static_cast<int64_t>(rank + 1) * n_kt / splits);
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < kStages; ++s) {
+            tc::mbar_init(tc::smem_u32(&full[s]), 1);
+            tc::mbar_init(tc::smem_u32(&empty[s]), 1);
+        }
+        tc::mbar_init(tc::smem_u32(&acc_full), 1);
+        tc::fence_mbar_init();
+        issued = 0;
+        consumed = 0;
+        failed = 0;
+    }
+    if (warp == 1) {
+        tc::tmem_alloc(tc::smem_u32(&tmem_slot), BN);
+        tc::tmem_relinquish();
+    }
+    tc::tc_fence_before();
+    __syncthreads();
+    tc::tc_fence_after();
+    const uint32_t tmem = tmem_slot;
+    volatile int* vfailed = &failed;
+    tc::grid_dep_launch();
+
+    if (warp == 0 && lane == 0) {
+        // ---- producer: this rank's k-steps through the stage ring ----------
+        tc::prefetch_tmap(&tmap_x);
+        tc::prefetch_tmap(&tmap_w);
+        for (int kt = kb; kt < ke; ++kt)       // the weight stripe, into L2 early
+            tc::tma_prefetch_l2_2d(&tmap_w, kt * kBK, n0);
+        tc::grid_dep_wait();
+        for (int kt = kb, g = 0; kt < ke; ++kt, ++g) {
+            const int s = g % kStages;
+            const uint32_t ph = static_cast<uint32_t>(g / kStages) & 1u;
+            if (!tc::mbar_wait(tc::smem_u32(&empty[s]), ph ^ 1)) {
+                if (status) atomicOr(status, tc::kTimeoutProducer);
+                atomicExch(&failed, 1);
+                break;
+            }
+            if (*vfailed) break;
+            const uint32_t a = base + s * L::kStage;
+            tc::mbar_arrive_expect_tx(tc::smem_u32(&full[s]), L::kStage);
+            tc::tma_load_2d(a, &tmap_x, tc::smem_u32(&full[s]), kt * kBK, 0);
+            tc::tma_load_2d(a + L::kA, &tmap_w, tc::smem_u32(&full[s]), kt * kBK, n0);
+            issued = g + 1;
+        }
+    } else if (warp == 1 && lane == 0) {
+        // ---- MMA issuer: one accumulator, the rank's k-steps in order ------
+        tc::grid_dep_wait();
+        const uint32_t idesc = tc::idesc_bf16_f32(kMmaM, BN);
+        bool ok = true;
+        for (int kt = kb, g = 0; kt < ke; ++kt, ++g) {
+            const int s = g % kStages;
+            const uint32_t ph = static_cast<uint32_t>(g / kStages) & 1u;
+            if (!tc::mbar_wait(tc::smem_u32(&full[s]), ph) || *vfailed) {
+                if (status) atomicOr(status, tc::kTimeoutMma);
+                atomicExch(&failed, 1);
+                ok = false;
+                break;
+            }
+            consumed = g + 1;
+            tc::tc_fence_after();
+            const uint32_t a = base + s * L::kStage;
+            const uint32_t b = a + L::kA;
+#pragma unroll
+            for (int kk = 0; kk < kBK / 16; ++kk)
+                tc::mma_bf16(tmem, tc::desc_k_sw128(a + kk * 32), tc::desc_k_sw128(b + kk * 32),
+                             idesc, (g > 0 || kk > 0) ? 1u : 0u);
+            tc::mma_commit(tc::smem_u32(&empty[s]));
+        }
+        // every MMA done (so every stage read and every copy landed): the
+        // ring is free for the partial tile
+        if (ok) tc::mma_commit(tc::smem_u32(&acc_full));
+    } else if (warp >= 2) {
+        // ---- park the partial tile: TMEM -> registers -> this CTA's ring ---
+        tc::grid_dep_wait();
+        const int row = (warp & 3) * 32 + lane;            // TMEM lane quarter warp % 4
+        if (!tc::mbar_wait(tc::smem_u32(&acc_full), 0) || *vfailed) {
+            if (status) atomicOr(status, tc::kTimeoutEpilogue);
+            atomicExch(&failed, 1);
+        } else {
+            tc::tc_fence_after();
+            const uint32_t src = tmem + (static_cast<uint32_t>((warp & 3) * 32) << 16);
+#pragma unroll 1
+            for (int c0 = 0; c0 < BN; c0 += 32) {
+                uint32_t r[32];
+                tc::tmem_ld_32x32b_x32(src + c0, r);
+                tc::tmem_ld_wait();
+                if (row < M) {
+                    float4* dst = reinterpret_cast<float4*>(part + row * kPitch + c0);
+#pragma unroll
+                    for (int j = 0; j < 8; ++j)
+                        dst[j] = make_float4(__uint_as_float(r[4 * j]), __uint_as_float(r[4 * j + 1]),
+                                             __uint_as_float(r[4 * j + 2]),
+                                             __uint_as_float(r[4 * j + 3]));
+                }
+            }
+        }
+    }
+
+    // Every CTA's partial is parked; each sums its slice over the cluster.
+    // (On a timeout the partials are stale: the output is then undefined and
+    // the status word says so, but every CTA still meets both barriers.)
+    if (warp < 2 && lane != 0) tc::grid_dep_wait();   // they store below too
+    tc::tc_fence_before();
+    __syncthreads();
+    __syncwarp();
+    tc::cluster_sync();
+    {
+        const int units = M * kQuads;
+        const int lo = static_cast<int>(static_cast<int64_t>(rank) * units / splits);
+        const int hi = static_cast<int>(static_cast<int64_t>(rank + 1) * units / splits);
+        const bool vec = (N & 3) == 0;
+        // two units per pass: all 2 S remote loads are in flight together
+#pragma unroll 1
+        for (int u0 = lo + static_cast<int>(threadIdx.x); u0 < hi; u0 += 2 * kThreads) {
+            float4 v[2][8];
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+                const int u = u0 + h * kThreads;
+                const int row = u / kQuads;
+                const int c = (u - row * kQuads) * 4;
+                if (u >= hi || n0 + c >= N) continue;
+                const uint32_t off = base + static_cast<uint32_t>((row * kPitch + c) * 4);
+#pragma unroll
+                for (int s = 0; s < 8; ++s)
+                    if (s < splits) v[h][s] = tc::ld_cluster_f4(tc::map_shared_rank(off, s));
+            }
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+                const int u = u0 + h * kThreads;
+                const int row = u / kQuads;
+                const int c = (u - row * kQuads) * 4;
+                const int col = n0 + c;
+                if (u >= hi || col >= N) continue;
+                float4 acc = v[h][0];
+#pragma unroll
+                for (int s = 1; s < 8; ++s) {
+                    if (s < splits) {
+                        acc.x = __fadd_rn(acc.x, v[h][s].x);
+                        acc.y = __fadd_rn(acc.y, v[h][s].y);
+                        acc.z = __fadd_rn(acc.z, v[h][s].z);
+                        acc.w = __fadd_rn(acc.w, v[h][s].w);
+                    }
+                }
+                float* yrow = y + static_cast<int64_t>(row) * N;
+                if (vec && col + 4 <= N) {
+                    *reinterpret_cast<float4*>(yrow + col) = acc;
+                } else {
+                    const float e[4] = {acc.x, acc.y, acc.z, acc.w};
+#pragma unroll
+                    for (int j = 0; j < 4; ++j)
+                        if (col + j < N) yrow[col + j] = e[j];
+                }
+            }
+        }
+    }
+    // no CTA leaves (releasing its shared memory) while a peer still reads it
+    __syncwarp();
+    tc::cluster_sync();
+
+    if (threadIdx.x == 0 && failed) {
+        for (int g = consumed; g < issued; ++g)
+            tc::mbar_wait(tc::smem_u32(&full[g % kStages]), static_cast<uint32_t>(g / kStages) & 1u);
+    }
+    tc::tc_fence_before();
+    __syncthreads();
+    tc::tc_fence_after();
+    if (warp == 1) tc::tmem_dealloc(tmem, BN);
+}
+
 // cuTensorMapEncodeTiled through the runtime's driver entry point (no link
 // against libcuda).
 using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
@@ -299,13 +532,138 @@ cudaError_t launch_bn(const LinearArgs& a, cudaStream_t stream) {
     if (tiles > INT32_MAX) return cudaErrorInvalidValue;
     const int64_t sms = device_sm_count();
     const unsigned grid = static_cast<unsigned>(tiles < sms ? tiles : sms);
-    linear_bf16_kernel<BN, BM><<<grid, kThreads, smem, stream>>>(tx, tw, a.y, static_cast<int>(a.M),
-                                                             static_cast<int>(a.N),
-                                                             static_cast<int>(a.K), a.status);
-    return cudaGetLastError();
+    // programmatic serialization: the prologue overlaps the previous kernel
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(grid);
+    cfg.blockDim = dim3(kThreads);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr;
+    attr.id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr.val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = &attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, linear_bf16_kernel<BN, BM>, tx, tw, a.y, static_cast<int>(a.M),
+                              static_cast<int>(a.N), static_cast<int>(a.K), a.status);
+}
+
+template <int BN>
+cudaError_t set_split_smem() {
+    return cudaFuncSetAttribute(linear_bf16_splitk_kernel<BN>,
+                                cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                static_cast<int>(LinearSmem<BN, kMmaM>::kDynamic));
+}
+
+// Cluster of `splits` CTAs along x, and (`pdl`) programmatic serialization
+// so the prologue overlaps the previous kernel; attr holds two entries.
+template <int BN>
+cudaLaunchConfig_t split_config(unsigned grid, int splits, cudaStream_t stream,
+                                cudaLaunchAttribute* attr, bool pdl) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(grid);
+    cfg.blockDim = dim3(kThreads);
+    cfg.dynamicSmemBytes = LinearSmem<BN, kMmaM>::kDynamic;
+    cfg.stream = stream;
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = static_cast<unsigned>(splits);
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[1].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = pdl ? 2 : 1;
+    return cfg;
+}
+
+// Clusters of `splits` CTAs of the BN-wide split kernel that the device holds
+// at once (cached per device; 0 when the query fails).
+template <int BN>
+int max_active_clusters(int splits) {
+    constexpr int kDevs = 16;
+    static std::atomic<int> cache[kDevs][9];
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0) return 0;
+    if (dev < kDevs) {
+        const int c = cache[dev][splits].load(std::memory_order_relaxed);
+        if (c > 0) return c - 1;
+    }
+    int n = 0;
+    cudaLaunchAttribute attr[2];
+    const cudaLaunchConfig_t cfg = split_config<BN>(static_cast<unsigned>(splits), splits,
+                                                    nullptr, attr, false);
+    if (set_split_smem<BN>() != cudaSuccess ||
+        cudaOccupancyMaxActiveClusters(&n, linear_bf16_splitk_kernel<BN>, &cfg) != cudaSuccess) {
+        cudaGetLastError();
+        n = 0;
+    }
+    if (dev < kDevs) cache[dev][splits].store(n + 1, std::memory_order_relaxed);
+    return n;
+}
+
+int max_active_clusters_bn(int bn, int splits) {
+    if (bn == 256) return max_active_clusters<256>(splits);
+    if (bn == 128) return max_active_clusters<128>(splits);
+    return max_active_clusters<64>(splits);
+}
+
+struct SplitPlan {
+    int bn = 0;
+    int splits = 1;
+};
+
+// The split for an (N, K) product: for each tile width, as many K chunks (at
+// most 8, at most one per k-step) as keep tiles x chunks within one wave of
+// clusters on the device's SMs; the plan with the most CTAs wins, the wider
+// tile on a tie. (Fewer k-steps per CTA through wider tiles and more chunks
+// measured slower: the cluster reduction grows with the tile and the chunk
+// count.) A function of (N, K) and the device, never of M.
+SplitPlan split_plan(int64_t N, int64_t K) {
+    const int64_t n_kt = (K + kBK - 1) / kBK;
+    const int64_t sms = device_sm_count();
+    SplitPlan best;
+    int64_t best_ctas = 0;
+    for (const int bn : {256, 128, 64}) {
+        const int64_t tiles = (N + bn - 1) / bn;
+        int64_t s = std::min<int64_t>(std::min<int64_t>(8, n_kt), sms / tiles);
+        for (; s >= 2; --s)
+            if (tiles <= max_active_clusters_bn(bn, static_cast<int>(s))) break;
+        if (s < 2) continue;
+        if (tiles * s > best_ctas) {
+            best_ctas = tiles * s;
+            best.bn = bn;
+            best.splits = static_cast<int>(s);
+        }
+    }
+    return best;
+}
+
+template <int BN>
+cudaError_t launch_split_bn(const LinearArgs& a, int splits, cudaStream_t stream) {
+    CUtensorMap tx, tw;
+    if (!make_tmap(&tx, a.x, a.M, a.K, kMmaM) || !make_tmap(&tw, a.w, a.N, a.K, BN))
+        return cudaErrorInvalidValue;
+    cudaError_t err = set_split_smem<BN>();
+    if (err != cudaSuccess) return err;
+    const int64_t tiles = (a.N + BN - 1) / BN;
+    cudaLaunchAttribute attr[2];
+    const cudaLaunchConfig_t cfg =
+        split_config<BN>(static_cast<unsigned>(tiles * splits), splits, stream, attr, true);
+    return cudaLaunchKernelEx(&cfg, linear_bf16_splitk_kernel<BN>, tx, tw, a.y,
+                              static_cast<int>(a.M), static_cast<int>(a.N),
+                              static_cast<int>(a.K), splits, a.status);
 }
 
 }  // namespace
+
+cudaError_t launch_linear_bf16_split(const LinearArgs& a, cudaStream_t stream) {
+    if (a.M == 0 || a.N == 0) return cudaSuccess;
+    if (a.M > kMmaM) return launch_linear_bf16(a, stream);
+    const SplitPlan p = split_plan(a.N, a.K);
+    if (p.splits < 2) return launch_linear_bf16(a, stream);
+    if (p.bn == 256) return launch_split_bn<256>(a, p.splits, stream);
+    if (p.bn == 128) return launch_split_bn<128>(a, p.splits, stream);
+    return launch_split_bn<64>(a, p.splits, stream);
+}
 
 cudaError_t launch_linear_bf16(const LinearArgs& a, cudaStream_t stream) {
     if (a.M == 0 || a.N == 0) return cudaSuccess;

@@ -25,12 +25,16 @@
 //      a call of one tile -- decode, verify -- has one thread per channel,
 //      which writes the rings itself at the end of step 2);
 //   4. out = y . W_out^T              (tcgen05 GEMM).
+// Calls of at most 128 rows (B*T) run both GEMMs split over K in a
+// thread-block cluster; the rows of such calls agree bit for bit with one
+// another, and with larger calls to fp32 rounding of the accumulation order.
 // u is rounded to fp32 (the ring's type) before it enters the window; the
 // window sum and the output gate run in double, and y is rounded once.
 #include <cuda_bf16.h>
 
 #include "gdn_common.cuh"
 #include "gdn_internal.h"
+#include "gdn_tc.cuh"
 
 namespace gdn {
 
@@ -47,6 +51,8 @@ __global__ void __launch_bounds__(256)
 short_conv_gate_kernel(const float* __restrict__ proj, float* ring, float* scratch_ring,
                        const float* __restrict__ conv_w, __nv_bfloat16* __restrict__ y,
                        int64_t B, int64_t T, int64_t D, int64_t n_commit) {
+    tc::grid_dep_launch();
+    tc::grid_dep_wait();           // proj comes from the previous kernel
     const int64_t d = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
     if (d >= D) return;
     const int64_t b = blockIdx.z;
@@ -130,6 +136,8 @@ template <int K>
 __global__ void __launch_bounds__(256)
 short_conv_ring_kernel(const float* __restrict__ proj, float* ring, float* scratch_ring,
                        int64_t B, int64_t T, int64_t D, int64_t n_commit) {
+    tc::grid_dep_launch();
+    tc::grid_dep_wait();
     const int64_t idx = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
     if (idx >= B * D) return;
     const int64_t b = idx / D;
@@ -161,25 +169,40 @@ short_conv_ring_kernel(const float* __restrict__ proj, float* ring, float* scrat
 
 size_t align256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
 
+// Launch with programmatic stream serialization (each kernel here waits for
+// its predecessor with griddepcontrol.wait before touching memory).
+template <typename... Params, typename... Args>
+cudaError_t launch_pdl(void (*kernel)(Params...), dim3 grid, dim3 block, cudaStream_t stream,
+                       Args... args) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr;
+    attr.id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr.val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = &attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kernel, static_cast<Params>(args)...);
+}
+
 template <int K>
 cudaError_t launch_conv(const ShortConvArgs& a, float* proj, __nv_bfloat16* y,
                         cudaStream_t stream) {
     const dim3 grid(static_cast<unsigned>((a.D + 255) / 256),
                     static_cast<unsigned>((a.T + kConvTile - 1) / kConvTile),
                     static_cast<unsigned>(a.B));
-    if (a.T <= kConvTile) {          // one tile: the gate pass also writes the rings
-        short_conv_gate_kernel<K, true><<<grid, 256, 0, stream>>>(
-            proj, a.conv_ring, a.scratch_ring, a.conv_w, y, a.B, a.T, a.D, a.n_commit);
-        return cudaGetLastError();
-    }
-    short_conv_gate_kernel<K, false><<<grid, 256, 0, stream>>>(
-        proj, a.conv_ring, nullptr, a.conv_w, y, a.B, a.T, a.D, a.n_commit);
-    cudaError_t err = cudaGetLastError();
+    if (a.T <= kConvTile)            // one tile: the gate pass also writes the rings
+        return launch_pdl(short_conv_gate_kernel<K, true>, grid, dim3(256), stream, proj,
+                          a.conv_ring, a.scratch_ring, a.conv_w, y, a.B, a.T, a.D, a.n_commit);
+    cudaError_t err = launch_pdl(short_conv_gate_kernel<K, false>, grid, dim3(256), stream, proj,
+                                 a.conv_ring, static_cast<float*>(nullptr), a.conv_w, y, a.B,
+                                 a.T, a.D, a.n_commit);
     if (err != cudaSuccess) return err;
     const int64_t n = a.B * a.D;
-    short_conv_ring_kernel<K><<<static_cast<unsigned>((n + 255) / 256), 256, 0, stream>>>(
-        proj, a.conv_ring, a.scratch_ring, a.B, a.T, a.D, a.n_commit);
-    return cudaGetLastError();
+    return launch_pdl(short_conv_ring_kernel<K>, dim3(static_cast<unsigned>((n + 255) / 256)),
+                      dim3(256), stream, static_cast<const float*>(proj), a.conv_ring,
+                      a.scratch_ring, a.B, a.T, a.D, a.n_commit);
 }
 
 }  // namespace
@@ -200,7 +223,7 @@ cudaError_t launch_short_conv(const ShortConvArgs& a, cudaStream_t stream) {
     char* ws = static_cast<char*>(a.workspace);
     float* proj = reinterpret_cast<float*>(ws + L.proj);
     __nv_bfloat16* y = reinterpret_cast<__nv_bfloat16*>(ws + L.y);
-    cudaError_t err = launch_linear_bf16(LinearArgs{a.hidden, a.w_in, proj, BT, 3 * a.D, a.D,
+    cudaError_t err = launch_linear_bf16_split(LinearArgs{a.hidden, a.w_in, proj, BT, 3 * a.D, a.D,
                                                     a.status}, stream);
     if (err != cudaSuccess) return err;
     switch (a.K) {
@@ -210,7 +233,8 @@ cudaError_t launch_short_conv(const ShortConvArgs& a, cudaStream_t stream) {
         default: return cudaErrorInvalidValue;
     }
     if (err != cudaSuccess) return err;
-    return launch_linear_bf16(LinearArgs{y, a.w_out, a.out, BT, a.D, a.D, a.status}, stream);
+    return launch_linear_bf16_split(LinearArgs{y, a.w_out, a.out, BT, a.D, a.D, a.status},
+                                    stream);
 }
 
 }  // namespace gdn

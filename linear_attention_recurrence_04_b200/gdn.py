@@ -30,7 +30,8 @@ STATUS = {
 # Every symbol that include/gdn.h declares.
 EXPORTS = ("gdn_status_string", "gdn_last_error", "gdn_step", "gdn_prefill", "gdn_pair",
            "gdn_layer_decode",
-           "gdn_layer_pair", "gdn_linear_bf16", "gdn_forward_batch_workspace_size",
+           "gdn_layer_pair", "gdn_linear_bf16", "gdn_linear_bf16_split_k",
+           "gdn_forward_batch_workspace_size",
            "gdn_forward_batch", "gdn_forward_batch_noalloc", "gdn_short_conv_workspace_size",
            "gdn_short_conv_forward_batch", "gdn_short_conv_forward", "gdn_short_conv_pair",
            "gdn_kda_step", "gdn_kda_prefill", "gdn_selftest_bounded_wait")
@@ -79,6 +80,8 @@ def load_library(path: Optional[str] = None) -> ctypes.CDLL:
     lib.gdn_layer_pair.argtypes = [_VP] * 9 + [_F32, _F32] + [_VP] * 4 + [_I64] * 6 + [_VP]
     lib.gdn_linear_bf16.restype = ctypes.c_int
     lib.gdn_linear_bf16.argtypes = [_VP, _VP, _VP, _I64, _I64, _I64, _VP, _VP]
+    lib.gdn_linear_bf16_split_k.restype = ctypes.c_int
+    lib.gdn_linear_bf16_split_k.argtypes = [_VP, _VP, _VP, _I64, _I64, _I64, _VP, _VP]
     lib.gdn_forward_batch_workspace_size.restype = ctypes.c_size_t
     lib.gdn_forward_batch_workspace_size.argtypes = [_I64] * 6
     lib.gdn_forward_batch.restype = ctypes.c_int
@@ -296,10 +299,12 @@ def layer_pair(mixed_qkv, z, a, b, conv_ring, conv_w, A_log, dt_bias, norm_w, st
     return out, scratch_ring, scratch_state
 
 
-def linear_bf16(x, w, y=None, *, status=None, stream=None):
+def linear_bf16(x, w, y=None, *, status=None, stream=None, split_k=False):
     """y = x @ w.T on the tensor cores: x [M, K] bf16, w [N, K] bf16, y [M, N]
     fp32. `status`, if given, is a zero-initialised int32 CUDA tensor that
-    receives timeout bits (see include/gdn.h)."""
+    receives timeout bits (see include/gdn.h). split_k=True calls
+    gdn_linear_bf16_split_k (K split over a thread-block cluster when
+    M <= 128)."""
     if x.dim() != 2 or w.dim() != 2 or x.shape[1] != w.shape[1]:
         raise ValueError("x must be [M, K] and w [N, K]")
     M, K = x.shape
@@ -319,9 +324,10 @@ def linear_bf16(x, w, y=None, *, status=None, stream=None):
         if status.dtype is not torch.int32 or status.device != device or status.numel() != 1:
             raise TypeError("status must be a one-element int32 tensor on the same device")
         sp = status.data_ptr()
-    st = _call(device, load_library().gdn_linear_bf16, _ptr(x), _ptr(w), _ptr(y), M, N, K, sp,
+    name = "gdn_linear_bf16_split_k" if split_k else "gdn_linear_bf16"
+    st = _call(device, getattr(load_library(), name), _ptr(x), _ptr(w), _ptr(y), M, N, K, sp,
                _stream(device, stream))
-    _raise_on("gdn_linear_bf16", st)
+    _raise_on(name, st)
     return y
 
 

@@ -169,8 +169,10 @@ def test_layer_pair_argument_checks(lib):
                               None) == OK
 
 
-def test_linear_argument_checks(lib):
-    f = lambda x=fake(1), w=fake(2), y=fake(3), M=4, N=4, K=16, st=0: lib.gdn_linear_bf16(
+@pytest.mark.parametrize("name", ["gdn_linear_bf16", "gdn_linear_bf16_split_k"])
+def test_linear_argument_checks(lib, name):
+    fn = getattr(lib, name)
+    f = lambda x=fake(1), w=fake(2), y=fake(3), M=4, N=4, K=16, st=0: fn(
         x, w, y, M, N, K, st, None)
     assert f(K=12) == UNSUP
     assert f(M=-1) == SHAPE
@@ -178,7 +180,8 @@ def test_linear_argument_checks(lib):
     assert f(y=fake(3) + 8) == ALIGN
     assert f(y=fake(1) + 16) == ALIAS
     assert f(M=1 << 30) == OVERFLOW
-    assert lib.gdn_linear_bf16(0, 0, 0, 0, 7, 16, 0, None) == OK
+    assert f(st=fake(4) + 2) == ALIGN
+    assert fn(0, 0, 0, 0, 7, 16, 0, None) == OK
 
 
 def test_forward_batch_argument_checks(lib):

@@ -88,3 +88,53 @@ def test_linear_k_zero_and_empty():
     e = gdn.linear_bf16(torch.zeros(0, 16, dtype=torch.bfloat16, device="cuda"),
                         torch.zeros(4, 16, dtype=torch.bfloat16, device="cuda"))
     assert e.shape == (0, 4)
+
+
+# -- split-K form for decode-sized products (M <= 128) ----------------------
+
+@pytest.mark.parametrize("M,N,K", [(64, 6144, 2048), (64, 2048, 2048), (1, 8, 8), (7, 384, 128),
+                                   (100, 300, 136), (128, 257, 1000), (128, 6144 + 64, 2048),
+                                   (33, 2048, 4096), (129, 512, 512)])
+def test_linear_split_k_parity(M, N, K):
+    """Every element against the fp64 matmul with the same bound as the
+    persistent kernel: K chunks of whole and ragged 64-column steps, N off the
+    tile grid, a single k-step (no split), and M = 129 (persistent kernel)."""
+    x, w = bf16_pair(M, N, K, seed=3 * M + N + K)
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    y = gdn.linear_bf16(x.cuda(), w.cuda(), status=status, split_k=True)
+    torch.cuda.synchronize()
+    assert int(status.item()) == 0
+    check(x, w, y)
+
+
+def test_linear_split_k_rows_independent_of_batch():
+    """The split depends on N and K alone: rows of a 128-row call equal the
+    same rows of a 64-row call and computed alone, bit for bit."""
+    M, N, K = 128, 6144, 2048
+    x, w = bf16_pair(M, N, K, seed=17)
+    xc, wc = x.cuda(), w.cuda()
+    y = gdn.linear_bf16(xc, wc, split_k=True)
+    y64 = gdn.linear_bf16(xc[64:].contiguous(), wc, split_k=True)
+    torch.cuda.synchronize()
+    assert torch.equal(y64, y[64:]), "rows 64..127"
+    for r in (0, 63, 64, 127):
+        yr = gdn.linear_bf16(xc[r:r + 1].contiguous(), wc, split_k=True)
+        torch.cuda.synchronize()
+        assert torch.equal(yr[0], y[r]), f"row {r}"
+
+
+def test_linear_split_k_near_persistent_kernel():
+    """The split form and the persistent kernel differ only by the grouping of
+    the fp32 sum: within the accumulation bound of each other, and each within
+    the bound of the exact product."""
+    M, N, K = 64, 2048, 2048
+    x, w = bf16_pair(M, N, K, seed=19, scale=4.0)
+    xc, wc = x.cuda(), w.cuda()
+    ys = gdn.linear_bf16(xc, wc, split_k=True)
+    yp = gdn.linear_bf16(xc, wc)
+    torch.cuda.synchronize()
+    check(x, w, ys)
+    check(x, w, yp)
+    mag = (x.abs().double() @ w.abs().double().T).numpy()
+    diff = (ys - yp).abs().double().cpu().numpy()
+    assert np.all(diff <= 8e-7 * np.sqrt(K) * mag + 1e-30)
