@@ -119,6 +119,11 @@ struct ShortConvArgs {
 struct ShortConvLayout {
     size_t proj, y, total;
 };
+// Calls of at most 128 rows (B*T): the input projection, split over K in a
+// cluster, with the gate and conv as its epilogue -- y (bf16, [B*T][D]) and
+// both rings are written, proj is not. cudaErrorNotSupported when the call
+// is larger or the product too small to split (use the separate kernels).
+cudaError_t launch_short_conv_in_gate(const ShortConvArgs& a, void* y, cudaStream_t stream);
 ShortConvLayout short_conv_layout(int64_t B, int64_t T, int64_t D);
 
 // Each launcher enqueues its kernel on `stream` and returns the launch status.

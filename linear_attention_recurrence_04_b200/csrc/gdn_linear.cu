@@ -38,6 +38,7 @@
 // kernel (griddepcontrol.wait) before its first global read or write or
 // bounded wait, and each CTA releases the next kernel once set up.
 #include <cuda.h>
+#include <cuda_bf16.h>
 
 #include <algorithm>
 #include <atomic>
@@ -284,16 +285,42 @@ linear_bf16_kernel(const __grid_constant__ CUtensorMap tmap_x,
 // device alone, so a row's result is the same in any call of at most 128
 // rows; it differs from the persistent kernel's by the fp32 rounding of the
 // grouped sum.
-template <int BN>
+//
+// kGate = 2, 3 or 4 (conv taps): the short-conv mixer's input projection with
+// its gate and conv as the epilogue. A tile is 64 channels d0.. of the three
+// row blocks of W_in (bg | cg | xv), loaded as three 64-row boxes into one
+// 192-row B tile (N = 192, M = rows of the call). After the cluster barrier
+// CTA r takes the channel quads [16 r / S, 16 (r+1) / S) of the tile: it sums
+// bg, cg, xv over the S partials (rank order), forms u = bg * xv in fp32 and
+// keeps u and cg in its own shared memory; after a second cluster barrier one
+// thread per (sequence, channel) walks the call's positions through the conv
+// window -- the ring before position 0, u after -- exactly as the mixer's
+// gate kernel does (window sum and output gate in double, y rounded to bf16
+// once) and writes y and both rings.
+struct GateEpi {
+    float* ring;            // [B][K-1][D]
+    float* scratch_ring;    // [B][K-1][D] or null
+    const float* conv_w;    // [D][K]
+    __nv_bfloat16* y;       // [B][T][D]
+    int B, T, D, n_commit;
+};
+
+template <int BN, int kGate>
 __global__ void __launch_bounds__(kThreads, 1)
 linear_bf16_splitk_kernel(const __grid_constant__ CUtensorMap tmap_x,
                           const __grid_constant__ CUtensorMap tmap_w, float* __restrict__ y,
-                          int M, int N, int K, int splits, uint32_t* __restrict__ status) {
+                          int M, int N, int K, int splits, uint32_t* __restrict__ status,
+                          GateEpi ge) {
     using L = LinearSmem<BN, kMmaM>;
     constexpr int kStages = L::kStages;
     constexpr int kPitch = BN + 4;        // floats per parked row: 16-byte shift per row
     constexpr int kQuads = BN / 4;        // float4 columns of a row
-    static_assert(static_cast<size_t>(kMmaM) * kPitch * 4 + 1024 <= L::kDynamic,
+    constexpr uint32_t kTmemCols = BN <= 64 ? 64 : BN <= 128 ? 128 : 256;
+    static_assert(kGate == 0 || BN == 192, "the gate tile is three 64-row blocks");
+    // gate mode: u and cg of at most 8 channel quads per row after the parked tile
+    constexpr size_t kGateOff = static_cast<size_t>(kMmaM) * kPitch * 4;
+    constexpr size_t kGateBytes = kGate ? 2 * static_cast<size_t>(kMmaM) * 8 * 16 : 0;
+    static_assert(kGateOff + kGateBytes + 1024 <= L::kDynamic,
                   "the partial tile fits the stage ring");
     extern __shared__ uint8_t smem_raw[];
     __shared__ __align__(8) uint64_t full[kStages];
@@ -310,7 +337,7 @@ linear_bf16_splitk_kernel(const __grid_constant__ CUtensorMap tmap_x,
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
     const int rank = static_cast<int>(tc::cluster_ctarank());
-    const int n0 = static_cast<int>(blockIdx.x / splits) * BN;
+    const int n0 = static_cast<int>(blockIdx.x / splits) * (kGate ? 64 : BN);   // column / channel base
     const int n_kt = (K + kBK - 1) / kBK;
     const int kb = static_cast<int>(static_cast<int64_t>(rank) * n_kt / splits);
     const int ke = static_cast<int>(static_cast<int64_t>(rank + 1) * n_kt / splits);
@@ -327,7 +354,7 @@ linear_bf16_splitk_kernel(const __grid_constant__ CUtensorMap tmap_x,
         failed = 0;
     }
     if (warp == 1) {
-        tc::tmem_alloc(tc::smem_u32(&tmem_slot), BN);
+        tc::tmem_alloc(tc::smem_u32(&tmem_slot), kTmemCols);
         tc::tmem_relinquish();
     }
     tc::tc_fence_before();
@@ -341,8 +368,14 @@ linear_bf16_splitk_kernel(const __grid_constant__ CUtensorMap tmap_x,
         // ---- producer: this rank's k-steps through the stage ring ----------
         tc::prefetch_tmap(&tmap_x);
         tc::prefetch_tmap(&tmap_w);
-        for (int kt = kb; kt < ke; ++kt)       // the weight stripe, into L2 early
-            tc::tma_prefetch_l2_2d(&tmap_w, kt * kBK, n0);
+        for (int kt = kb; kt < ke; ++kt) {     // the weight stripe, into L2 early
+            if constexpr (kGate) {
+                for (int blk = 0; blk < 3; ++blk)
+                    tc::tma_prefetch_l2_2d(&tmap_w, kt * kBK, blk * ge.D + n0);
+            } else {
+                tc::tma_prefetch_l2_2d(&tmap_w, kt * kBK, n0);
+            }
+        }
         tc::grid_dep_wait();
         for (int kt = kb, g = 0; kt < ke; ++kt, ++g) {
             const int s = g % kStages;
@@ -356,7 +389,13 @@ linear_bf16_splitk_kernel(const __grid_constant__ CUtensorMap tmap_x,
             const uint32_t a = base + s * L::kStage;
             tc::mbar_arrive_expect_tx(tc::smem_u32(&full[s]), L::kStage);
             tc::tma_load_2d(a, &tmap_x, tc::smem_u32(&full[s]), kt * kBK, 0);
-            tc::tma_load_2d(a + L::kA, &tmap_w, tc::smem_u32(&full[s]), kt * kBK, n0);
+            if constexpr (kGate) {       // bg, cg, xv rows of the tile's channels
+                for (int blk = 0; blk < 3; ++blk)
+                    tc::tma_load_2d(a + L::kA + blk * 64 * kBK * 2, &tmap_w,
+                                    tc::smem_u32(&full[s]), kt * kBK, blk * ge.D + n0);
+            } else {
+                tc::tma_load_2d(a + L::kA, &tmap_w, tc::smem_u32(&full[s]), kt * kBK, n0);
+            }
             issued = g + 1;
         }
     } else if (warp == 1 && lane == 0) {
@@ -421,58 +460,150 @@ linear_bf16_splitk_kernel(const __grid_constant__ CUtensorMap tmap_x,
     __syncthreads();
     __syncwarp();
     tc::cluster_sync();
-    {
-        const int units = M * kQuads;
-        const int lo = static_cast<int>(static_cast<int64_t>(rank) * units / splits);
-        const int hi = static_cast<int>(static_cast<int64_t>(rank + 1) * units / splits);
-        const bool vec = (N & 3) == 0;
-        // two units per pass: all 2 S remote loads are in flight together
-#pragma unroll 1
-        for (int u0 = lo + static_cast<int>(threadIdx.x); u0 < hi; u0 += 2 * kThreads) {
-            float4 v[2][8];
-#pragma unroll
-            for (int h = 0; h < 2; ++h) {
-                const int u = u0 + h * kThreads;
-                const int row = u / kQuads;
-                const int c = (u - row * kQuads) * 4;
-                if (u >= hi || n0 + c >= N) continue;
-                const uint32_t off = base + static_cast<uint32_t>((row * kPitch + c) * 4);
-#pragma unroll
-                for (int s = 0; s < 8; ++s)
-                    if (s < splits) v[h][s] = tc::ld_cluster_f4(tc::map_shared_rank(off, s));
-            }
-#pragma unroll
-            for (int h = 0; h < 2; ++h) {
-                const int u = u0 + h * kThreads;
-                const int row = u / kQuads;
-                const int c = (u - row * kQuads) * 4;
-                const int col = n0 + c;
-                if (u >= hi || col >= N) continue;
-                float4 acc = v[h][0];
-#pragma unroll
-                for (int s = 1; s < 8; ++s) {
-                    if (s < splits) {
-                        acc.x = __fadd_rn(acc.x, v[h][s].x);
-                        acc.y = __fadd_rn(acc.y, v[h][s].y);
-                        acc.z = __fadd_rn(acc.z, v[h][s].z);
-                        acc.w = __fadd_rn(acc.w, v[h][s].w);
-                    }
+    if constexpr (kGate == 0) {
+        {
+            const int units = M * kQuads;
+            const int lo = static_cast<int>(static_cast<int64_t>(rank) * units / splits);
+            const int hi = static_cast<int>(static_cast<int64_t>(rank + 1) * units / splits);
+            const bool vec = (N & 3) == 0;
+            // two units per pass: all 2 S remote loads are in flight together
+    #pragma unroll 1
+            for (int u0 = lo + static_cast<int>(threadIdx.x); u0 < hi; u0 += 2 * kThreads) {
+                float4 v[2][8];
+    #pragma unroll
+                for (int h = 0; h < 2; ++h) {
+                    const int u = u0 + h * kThreads;
+                    const int row = u / kQuads;
+                    const int c = (u - row * kQuads) * 4;
+                    if (u >= hi || n0 + c >= N) continue;
+                    const uint32_t off = base + static_cast<uint32_t>((row * kPitch + c) * 4);
+    #pragma unroll
+                    for (int s = 0; s < 8; ++s)
+                        if (s < splits) v[h][s] = tc::ld_cluster_f4(tc::map_shared_rank(off, s));
                 }
-                float* yrow = y + static_cast<int64_t>(row) * N;
-                if (vec && col + 4 <= N) {
-                    *reinterpret_cast<float4*>(yrow + col) = acc;
-                } else {
-                    const float e[4] = {acc.x, acc.y, acc.z, acc.w};
-#pragma unroll
-                    for (int j = 0; j < 4; ++j)
-                        if (col + j < N) yrow[col + j] = e[j];
+    #pragma unroll
+                for (int h = 0; h < 2; ++h) {
+                    const int u = u0 + h * kThreads;
+                    const int row = u / kQuads;
+                    const int c = (u - row * kQuads) * 4;
+                    const int col = n0 + c;
+                    if (u >= hi || col >= N) continue;
+                    float4 acc = v[h][0];
+    #pragma unroll
+                    for (int s = 1; s < 8; ++s) {
+                        if (s < splits) {
+                            acc.x = __fadd_rn(acc.x, v[h][s].x);
+                            acc.y = __fadd_rn(acc.y, v[h][s].y);
+                            acc.z = __fadd_rn(acc.z, v[h][s].z);
+                            acc.w = __fadd_rn(acc.w, v[h][s].w);
+                        }
+                    }
+                    float* yrow = y + static_cast<int64_t>(row) * N;
+                    if (vec && col + 4 <= N) {
+                        *reinterpret_cast<float4*>(yrow + col) = acc;
+                    } else {
+                        const float e[4] = {acc.x, acc.y, acc.z, acc.w};
+    #pragma unroll
+                        for (int j = 0; j < 4; ++j)
+                            if (col + j < N) yrow[col + j] = e[j];
+                    }
                 }
             }
         }
+        // no CTA leaves (releasing its shared memory) while a peer still reads it
+        __syncwarp();
+        tc::cluster_sync();
+    } else {
+        // ---- gate mode: u = bg * xv and cg for this CTA's channel quads ----
+        const int q_lo = rank * 16 / splits;
+        const int nq = (rank + 1) * 16 / splits - q_lo;      // at most 8
+        float4* u_s = reinterpret_cast<float4*>(reinterpret_cast<uint8_t*>(part) + kGateOff);
+        float4* cg_s = u_s + kMmaM * 8;
+#pragma unroll 1
+        for (int it = static_cast<int>(threadIdx.x); it < M * nq; it += kThreads) {
+            const int row = it / nq;
+            const int ql = it - row * nq;
+            const int c = 4 * (q_lo + ql);
+            if (n0 + c >= ge.D) continue;
+            const uint32_t off = base + static_cast<uint32_t>((row * kPitch + c) * 4);
+            float4 v[3][8];
+#pragma unroll
+            for (int s2 = 0; s2 < 8; ++s2) {
+                if (s2 < splits) {
+#pragma unroll
+                    for (int blk = 0; blk < 3; ++blk)
+                        v[blk][s2] = tc::ld_cluster_f4(tc::map_shared_rank(off + blk * 64 * 4, s2));
+                }
+            }
+            float4 t3[3];
+#pragma unroll
+            for (int blk = 0; blk < 3; ++blk) {
+                t3[blk] = v[blk][0];
+#pragma unroll
+                for (int s2 = 1; s2 < 8; ++s2) {
+                    if (s2 < splits) {
+                        t3[blk].x = __fadd_rn(t3[blk].x, v[blk][s2].x);
+                        t3[blk].y = __fadd_rn(t3[blk].y, v[blk][s2].y);
+                        t3[blk].z = __fadd_rn(t3[blk].z, v[blk][s2].z);
+                        t3[blk].w = __fadd_rn(t3[blk].w, v[blk][s2].w);
+                    }
+                }
+            }
+            u_s[row * 8 + ql] = make_float4(__fmul_rn(t3[0].x, t3[2].x), __fmul_rn(t3[0].y, t3[2].y),
+                                            __fmul_rn(t3[0].z, t3[2].z), __fmul_rn(t3[0].w, t3[2].w));
+            cg_s[row * 8 + ql] = t3[1];
+        }
+        // no CTA leaves (releasing its shared memory) while a peer still
+        // reads it; u and cg are complete in this CTA
+        __syncwarp();
+        tc::cluster_sync();
+        // ---- the conv walk: one thread per (sequence, channel) -------------
+        constexpr int KT = kGate > 0 ? kGate : 2;
+        const int nch = 4 * nq;
+#pragma unroll 1
+        for (int it = static_cast<int>(threadIdx.x); it < ge.B * nch; it += kThreads) {
+            const int b = it / nch;
+            const int cl = it - b * nch;
+            const int d = n0 + 4 * q_lo + cl;
+            if (d >= ge.D) continue;
+            const float* u_f = reinterpret_cast<const float*>(u_s) + (cl >> 2) * 4 + (cl & 3);
+            const float* cg_f = reinterpret_cast<const float*>(cg_s) + (cl >> 2) * 4 + (cl & 3);
+            double wt[KT];
+#pragma unroll
+            for (int tau = 0; tau < KT; ++tau)
+                wt[tau] = ge.conv_w[static_cast<int64_t>(d) * KT + tau];
+            float* rg = ge.ring + static_cast<int64_t>(b) * (KT - 1) * ge.D + d;
+            float win[KT - 1], committed[KT - 1];
+#pragma unroll
+            for (int i = 0; i < KT - 1; ++i) committed[i] = win[i] = rg[static_cast<int64_t>(i) * ge.D];
+#pragma unroll 1
+            for (int t = 0; t < ge.T; ++t) {
+                const int row = b * ge.T + t;
+                const float u = u_f[row * 32];
+                double conv = 0.0;
+#pragma unroll
+                for (int tau = 0; tau < KT - 1; ++tau)
+                    conv = fma(wt[tau], static_cast<double>(win[tau]), conv);
+                conv = fma(wt[KT - 1], static_cast<double>(u), conv);
+                ge.y[static_cast<int64_t>(row) * ge.D + d] =
+                    __double2bfloat16(static_cast<double>(cg_f[row * 32]) * conv);
+#pragma unroll
+                for (int tau = 0; tau < KT - 2; ++tau) win[tau] = win[tau + 1];
+                win[KT - 2] = u;
+                if (t == ge.n_commit - 1) {
+#pragma unroll
+                    for (int tau = 0; tau < KT - 1; ++tau) committed[tau] = win[tau];
+                }
+            }
+#pragma unroll
+            for (int tau = 0; tau < KT - 1; ++tau) rg[static_cast<int64_t>(tau) * ge.D] = committed[tau];
+            if (ge.scratch_ring) {
+                float* sg = ge.scratch_ring + static_cast<int64_t>(b) * (KT - 1) * ge.D + d;
+#pragma unroll
+                for (int tau = 0; tau < KT - 1; ++tau) sg[static_cast<int64_t>(tau) * ge.D] = win[tau];
+            }
+        }
     }
-    // no CTA leaves (releasing its shared memory) while a peer still reads it
-    __syncwarp();
-    tc::cluster_sync();
 
     if (threadIdx.x == 0 && failed) {
         for (int g = consumed; g < issued; ++g)
@@ -481,7 +612,7 @@ linear_bf16_splitk_kernel(const __grid_constant__ CUtensorMap tmap_x,
     tc::tc_fence_before();
     __syncthreads();
     tc::tc_fence_after();
-    if (warp == 1) tc::tmem_dealloc(tmem, BN);
+    if (warp == 1) tc::tmem_dealloc(tmem, kTmemCols);
 }
 
 // cuTensorMapEncodeTiled through the runtime's driver entry point (no link
@@ -547,9 +678,9 @@ cudaError_t launch_bn(const LinearArgs& a, cudaStream_t stream) {
                               static_cast<int>(a.N), static_cast<int>(a.K), a.status);
 }
 
-template <int BN>
+template <int BN, int kGate = 0>
 cudaError_t set_split_smem() {
-    return cudaFuncSetAttribute(linear_bf16_splitk_kernel<BN>,
+    return cudaFuncSetAttribute(linear_bf16_splitk_kernel<BN, kGate>,
                                 cudaFuncAttributeMaxDynamicSharedMemorySize,
                                 static_cast<int>(LinearSmem<BN, kMmaM>::kDynamic));
 }
@@ -577,7 +708,7 @@ cudaLaunchConfig_t split_config(unsigned grid, int splits, cudaStream_t stream,
 
 // Clusters of `splits` CTAs of the BN-wide split kernel that the device holds
 // at once (cached per device; 0 when the query fails).
-template <int BN>
+template <int BN, int kGate = 0>
 int max_active_clusters(int splits) {
     constexpr int kDevs = 16;
     static std::atomic<int> cache[kDevs][9];
@@ -591,8 +722,9 @@ int max_active_clusters(int splits) {
     cudaLaunchAttribute attr[2];
     const cudaLaunchConfig_t cfg = split_config<BN>(static_cast<unsigned>(splits), splits,
                                                     nullptr, attr, false);
-    if (set_split_smem<BN>() != cudaSuccess ||
-        cudaOccupancyMaxActiveClusters(&n, linear_bf16_splitk_kernel<BN>, &cfg) != cudaSuccess) {
+    if (set_split_smem<BN, kGate>() != cudaSuccess ||
+        cudaOccupancyMaxActiveClusters(&n, linear_bf16_splitk_kernel<BN, kGate>, &cfg) !=
+            cudaSuccess) {
         cudaGetLastError();
         n = 0;
     }
@@ -648,12 +780,57 @@ cudaError_t launch_split_bn(const LinearArgs& a, int splits, cudaStream_t stream
     cudaLaunchAttribute attr[2];
     const cudaLaunchConfig_t cfg =
         split_config<BN>(static_cast<unsigned>(tiles * splits), splits, stream, attr, true);
-    return cudaLaunchKernelEx(&cfg, linear_bf16_splitk_kernel<BN>, tx, tw, a.y,
+    return cudaLaunchKernelEx(&cfg, linear_bf16_splitk_kernel<BN, 0>, tx, tw, a.y,
                               static_cast<int>(a.M), static_cast<int>(a.N),
-                              static_cast<int>(a.K), splits, a.status);
+                              static_cast<int>(a.K), splits, a.status, GateEpi{});
+}
+
+// The short-conv input projection with the gate and conv as its epilogue:
+// tiles of 64 channels, each split over K like the plain form (most chunks
+// that keep the clusters in one wave, at most 8).
+template <int KT>
+cudaError_t launch_gate_k(const ShortConvArgs& a, void* y, cudaStream_t stream) {
+    const int64_t M = a.B * a.T, D = a.D;
+    const int64_t n_kt = (D + kBK - 1) / kBK;
+    const int64_t tiles = (D + 63) / 64;
+    int64_t s = std::min<int64_t>(std::min<int64_t>(8, n_kt), device_sm_count() / tiles);
+    for (; s >= 2; --s)
+        if (tiles <= max_active_clusters<192, KT>(static_cast<int>(s))) break;
+    if (s < 2) return cudaErrorNotSupported;
+    CUtensorMap tx, tw;
+    if (!make_tmap(&tx, a.hidden, M, D, kMmaM) || !make_tmap(&tw, a.w_in, 3 * D, D, 64))
+        return cudaErrorInvalidValue;
+    cudaError_t err = set_split_smem<192, KT>();
+    if (err != cudaSuccess) return err;
+    cudaLaunchAttribute attr[2];
+    const cudaLaunchConfig_t cfg = split_config<192>(static_cast<unsigned>(tiles * s),
+                                                     static_cast<int>(s), stream, attr, true);
+    GateEpi ge;
+    ge.ring = a.conv_ring;
+    ge.scratch_ring = a.scratch_ring;
+    ge.conv_w = a.conv_w;
+    ge.y = static_cast<__nv_bfloat16*>(y);
+    ge.B = static_cast<int>(a.B);
+    ge.T = static_cast<int>(a.T);
+    ge.D = static_cast<int>(D);
+    ge.n_commit = static_cast<int>(a.n_commit);
+    return cudaLaunchKernelEx(&cfg, linear_bf16_splitk_kernel<192, KT>, tx, tw,
+                              static_cast<float*>(nullptr), static_cast<int>(M),
+                              static_cast<int>(3 * D), static_cast<int>(D), static_cast<int>(s),
+                              a.status, ge);
 }
 
 }  // namespace
+
+cudaError_t launch_short_conv_in_gate(const ShortConvArgs& a, void* y, cudaStream_t stream) {
+    if (a.B * a.T > kMmaM) return cudaErrorNotSupported;
+    switch (a.K) {
+        case 2: return launch_gate_k<2>(a, y, stream);
+        case 3: return launch_gate_k<3>(a, y, stream);
+        case 4: return launch_gate_k<4>(a, y, stream);
+        default: return cudaErrorInvalidValue;
+    }
+}
 
 cudaError_t launch_linear_bf16_split(const LinearArgs& a, cudaStream_t stream) {
     if (a.M == 0 || a.N == 0) return cudaSuccess;

@@ -25,9 +25,12 @@
 //      a call of one tile -- decode, verify -- has one thread per channel,
 //      which writes the rings itself at the end of step 2);
 //   4. out = y . W_out^T              (tcgen05 GEMM).
-// Calls of at most 128 rows (B*T) run both GEMMs split over K in a
-// thread-block cluster; the rows of such calls agree bit for bit with one
-// another, and with larger calls to fp32 rounding of the accumulation order.
+// Calls of at most 128 rows (B*T) run stages 1-3 as one kernel: the input
+// projection split over K in a thread-block cluster, whose epilogue sums the
+// partials and does the gate, conv and rings for its 64 channels (the same
+// arithmetic as the gate kernel below); stage 4 is split the same way. The
+// rows of such calls agree bit for bit with one another, and with larger
+// calls to fp32 rounding of the projections' accumulation order.
 // u is rounded to fp32 (the ring's type) before it enters the window; the
 // window sum and the output gate run in double, and y is rounded once.
 #include <cuda_bf16.h>
@@ -223,7 +226,14 @@ cudaError_t launch_short_conv(const ShortConvArgs& a, cudaStream_t stream) {
     char* ws = static_cast<char*>(a.workspace);
     float* proj = reinterpret_cast<float*>(ws + L.proj);
     __nv_bfloat16* y = reinterpret_cast<__nv_bfloat16*>(ws + L.y);
-    cudaError_t err = launch_linear_bf16_split(LinearArgs{a.hidden, a.w_in, proj, BT, 3 * a.D, a.D,
+    // at most 128 rows: stages 1-3 in one kernel (the split-K projection with
+    // the gate, conv and rings as its epilogue), then stage 4
+    cudaError_t err = launch_short_conv_in_gate(a, y, stream);
+    if (err == cudaSuccess)
+        return launch_linear_bf16_split(LinearArgs{y, a.w_out, a.out, BT, a.D, a.D, a.status},
+                                        stream);
+    if (err != cudaErrorNotSupported) return err;
+    err = launch_linear_bf16_split(LinearArgs{a.hidden, a.w_in, proj, BT, 3 * a.D, a.D,
                                                     a.status}, stream);
     if (err != cudaSuccess) return err;
     switch (a.K) {
