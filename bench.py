@@ -721,6 +721,65 @@ def cpu_oracle_baseline(name: str, budget_s: float, max_units: Optional[int] = N
                 seconds=elapsed, units=int(len(units)), reps=reps)
 
 
+def cpu_oracle_baseline_parallel(name: str, budget_s: float):
+    """The same fp64 C oracle on every host core this process may use: its
+    step entry is called from one thread per core on disjoint unit lists
+    (ctypes releases the GIL during the call), over inputs converted to fp64
+    once and shared. Whole decode steps over all units, repeated until
+    `budget_s` has elapsed (at least once)."""
+    import ctypes
+    from concurrent.futures import ThreadPoolExecutor
+    import oracle
+    from linear_attention_recurrence_04_b200 import inputs
+    o = oracle.load()
+    w = inputs.WORKLOADS[name]
+    L, B = w.sizes["L"], w.sizes["B"]
+    d = inputs.decode_inputs(L, B, seed=w.seed)
+    f64 = {k: np.ascontiguousarray(v, dtype=np.float64) for k, v in d.items()}
+    L, B, Hv, dv, dk = f64["state"].shape
+    Hk = f64["q"].shape[2]
+    total_units = L * B * Hv
+    n = max(1, len(os.sched_getaffinity(0)))
+    chunks = [np.ascontiguousarray(c, dtype=np.int64)
+              for c in np.array_split(np.arange(total_units), n) if c.size]
+    outs = [np.zeros((L, B, Hv, dv)) for _ in chunks]
+    pd = ctypes.POINTER(ctypes.c_double)
+    pi = ctypes.POINTER(ctypes.c_int64)
+    ptr = lambda a: a.ctypes.data_as(pd)
+
+    def work(j):
+        u = chunks[j]
+        rc = o.lib.oracle_gdn_step(ptr(f64["state"]), ptr(f64["q"]), ptr(f64["k"]),
+                                   ptr(f64["v"]), ptr(f64["beta"]), ptr(f64["gate"]),
+                                   ptr(outs[j]), L, B, Hk, Hv, dk, dv,
+                                   u.ctypes.data_as(pi), int(u.size))
+        if rc != 0:
+            raise RuntimeError(f"oracle_gdn_step returned {rc}")
+
+    def timed(threads, budget):
+        reps, elapsed = 0, 0.0
+        with ThreadPoolExecutor(threads) as ex:
+            while reps == 0 or elapsed < budget:
+                t0 = time.perf_counter()
+                if threads == 1:
+                    for j in range(len(chunks)):
+                        work(j)
+                else:
+                    list(ex.map(work, range(len(chunks))))
+                elapsed += time.perf_counter() - t0
+                reps += 1
+        return reps, elapsed, reps * total_units * STATE_BYTES_PER_HEAD * 2 / elapsed / 1e9
+
+    r1, e1, v1 = timed(1, budget_s / 2)           # the same calls on one thread
+    rn, en, vn = timed(len(chunks), budget_s / 2)
+    return dict(value=vn, unit=UNIT, cores=len(chunks), kind="oracle",
+                value_one_thread=v1,
+                sample=(f"{rn} pass(es) of the fp64 C oracle over all {total_units} "
+                        f"value-head units of {name}, {len(chunks)} threads on disjoint units, "
+                        f"inputs converted to fp64 once and shared, {en:.1f} s; the same "
+                        f"calls on one thread: {r1} pass(es), {e1:.1f} s"))
+
+
 # --------------------------------------------------------------------------
 # arms
 # --------------------------------------------------------------------------
@@ -923,6 +982,9 @@ def run_ours(args) -> int:
     if env["rank"] == 0 and env["world"] == 1 and not args.no_cpu_baseline:
         cb = cpu_oracle_baseline(HEADLINE, args.cpu_budget)
         line["cpu_baseline"] = {k: cb[k] for k in ("value", "unit", "cores", "kind", "sample")}
+        # the same oracle on every host core (independent units, no exchange)
+        line["cpu_baseline_all_cores"] = cpu_oracle_baseline_parallel(HEADLINE,
+                                                                      args.cpu_budget)
 
     if env["world"] > 1:
         barrier()

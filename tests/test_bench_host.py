@@ -98,3 +98,15 @@ def test_reference_arm_line():
     assert line["impl"] == "reference" and line["unit"] == "GB/s" and line["value"] > 0
     assert line["metric"] == bench.METRIC and line["steps"] == 3
     assert line["e2e"]["h2d_bytes_per_step"] == 0 and line["cpu_baseline"]["kind"] == "oracle"
+
+
+def test_cpu_baselines_time_the_oracle():
+    """One pass each: the single-thread leg and the all-cores leg (the oracle's
+    C entry on disjoint units from one thread per core) both report the state
+    bandwidth of the headline workload."""
+    one = bench.cpu_oracle_baseline(bench.HEADLINE, 0.0, max_units=64)
+    assert one["cores"] == 1 and one["kind"] == "oracle" and one["value"] > 0
+    allc = bench.cpu_oracle_baseline_parallel(bench.HEADLINE, 0.0)
+    assert allc["kind"] == "oracle" and allc["unit"] == bench.UNIT
+    assert 1 <= allc["cores"] <= len(os.sched_getaffinity(0))
+    assert allc["value"] > 0 and allc["value_one_thread"] > 0
