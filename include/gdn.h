@@ -371,6 +371,14 @@ gdn_status gdn_kda_prefill(float *state, const float *q, const float *k, const f
  * Limits: B <= 65535, T <= 65535 * 32, B*T <= 65535 * 128 (GDN_ERR_OVERFLOW
  * otherwise). gdn_short_conv_workspace_size returns 0 for an invalid shape.
  *
+ * Calls of at most 128 rows (B*T) run the input projection split over K in a
+ * thread-block cluster, with the gate, conv and ring update as its epilogue,
+ * and the output projection split the same way (see gdn_linear_bf16_split_k).
+ * Outputs and rings are then identical, bit for bit, across all such calls
+ * (any chunking into calls, single positions, the verify). Between a call of
+ * at most 128 rows and a larger one they differ by the fp32 rounding of the
+ * projections' accumulation order.
+ *
  * gdn_short_conv_forward_batch runs T positions in order; conv_ring ends as
  * the ring after position T-1 (T = 0 does nothing).
  * gdn_short_conv_forward is the same call for one position per sequence:

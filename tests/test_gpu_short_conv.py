@@ -114,8 +114,8 @@ def test_chunks_and_single_positions_are_elementwise_identical():
 
 @pytest.mark.parametrize("B,T,D", [(3, 5, 1024), (2, 1, 1088), (7, 9, 1088)])
 def test_wide_hidden_matches_oracle(o, B, T, D):
-    """Hidden sizes of 16 and 17 k-steps of 64 (the last one ragged in
-    groups of 8), one position and several."""
+    """Hidden sizes of 16 and 17 k-steps of 64 (17 64-channel tiles for the
+    fused projection-and-gate kernel), one position and several."""
     d = inputs.short_conv_inputs(B, T, D=D, K=3, seed=1480 + D + T)
     t = to_dev(d)
     out = gpu_batch(t)
@@ -149,6 +149,62 @@ def test_pair_matches_oracle(o, K):
     out2 = gpu_batch(t2)
     assert torch.equal(out, out2), "pair vs two-position batch"
     assert torch.equal(scratch, t2["conv_ring"]), "scratch ring vs two-position batch ring"
+
+
+@pytest.mark.parametrize("B,T,D,K", [(3, 5, 200, 3), (2, 1, 1096, 4), (64, 1, 200, 2),
+                                     (4, 30, 200, 3)])
+def test_ragged_channel_tiles_match_oracle(o, B, T, D, K):
+    """Hidden sizes off the 64-channel tile of the fused projection-and-gate
+    kernel that calls of at most 128 rows take (200 = 3 x 64 + 8,
+    1096 = 17 x 64 + 8); B*T of 15, 2, 64 and 120 rows."""
+    d = inputs.short_conv_inputs(B, T, D=D, K=K, seed=1490 + D + T)
+    t = to_dev(d)
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    out = gdn.short_conv_forward_batch(t["hidden"], t["w_in"], t["w_out"], t["conv_ring"],
+                                       t["conv_w"], status=status)
+    torch.cuda.synchronize()
+    assert int(status.item()) == 0
+    ref_out, ref_ring = o.short_conv_forward_batch(d["hidden"], d["w_in"], d["w_out"],
+                                                   d["conv_ring"], d["conv_w"])
+    check_out(out.cpu().numpy(), ref_out, f"B{B} T{T} D{D} K{K} out")
+    check_ring(t["conv_ring"].cpu().numpy(), d["conv_ring"], d["hidden"], d["w_in"], ref_ring,
+               T - 1, f"B{B} T{T} D{D} K{K} ring")
+
+
+def test_pair_ragged_channel_tile_matches_oracle(o):
+    B, D, K = 6, 200, 4
+    d = inputs.short_conv_inputs(B, 2, D=D, K=K, seed=1495)
+    t = to_dev(d)
+    scratch = torch.full_like(t["conv_ring"], float("nan"))
+    out = gdn.short_conv_pair(t["hidden"], t["w_in"], t["w_out"], t["conv_ring"], scratch,
+                              t["conv_w"])
+    torch.cuda.synchronize()
+    ref_out, ref_ring, ref_scratch = o.short_conv_pair(d["hidden"], d["w_in"], d["w_out"],
+                                                       d["conv_ring"], d["conv_w"])
+    check_out(out.cpu().numpy(), ref_out, "pair D200 out")
+    check_ring(t["conv_ring"].cpu().numpy(), d["conv_ring"], d["hidden"], d["w_in"], ref_ring, 0,
+               "pair D200 committed ring")
+    check_ring(scratch.cpu().numpy(), d["conv_ring"], d["hidden"], d["w_in"], ref_scratch, 1,
+               "pair D200 scratch ring")
+
+
+def test_rows_of_calls_up_to_128_rows_are_batch_invariant():
+    """Calls of at most 128 rows share one split of K (fixed by D): the
+    sequences of a 64-sequence decode equal the same sequences decoded in a
+    call of their own, bit for bit (outputs and rings)."""
+    B, D = 64, 2048
+    d = inputs.short_conv_inputs(B, 1, D=D, K=3, seed=1497)
+    whole = to_dev(d)
+    out_all = gdn.short_conv_forward(whole["hidden"][:, 0].contiguous(), whole["w_in"],
+                                     whole["w_out"], whole["conv_ring"], whole["conv_w"])
+    for b in (0, 37, 63):
+        one = to_dev({k: (v[b:b + 1] if k in ("hidden", "conv_ring") else v)
+                      for k, v in d.items()})
+        o1 = gdn.short_conv_forward(one["hidden"][:, 0].contiguous(), one["w_in"], one["w_out"],
+                                    one["conv_ring"], one["conv_w"])
+        torch.cuda.synchronize()
+        assert torch.equal(o1[0], out_all[b]), f"sequence {b} output"
+        assert torch.equal(one["conv_ring"][0], whole["conv_ring"][b]), f"sequence {b} ring"
 
 
 def test_empty_batch_is_a_no_op():
