@@ -87,7 +87,7 @@ def test_pair_accept_then_reject(o):
     ref = {k: v.astype(np.float64) for k, v in d.items()}
     out, sring, sstate = run_pair(t, 16)
     out_r, ring_r, st_r, sring_r, sst_r = oracle_pair(o, ref, 16)
-    assert_parity(out.cpu().numpy(), out_r, "round 1 out")
+    assert_parity(out.cpu().numpy(), out_r, "first verify out")
     t["conv_ring"], t["state"] = sring, sstate            # accept
     ref["conv_ring"], ref["state"] = sring_r, sst_r
     d2 = pair_inputs(3, seed=931)
@@ -96,9 +96,9 @@ def test_pair_accept_then_reject(o):
         ref[n] = d2[n]
     out, sring, sstate = run_pair(t, 16)
     out_r, ring_r, st_r, sring_r, sst_r = oracle_pair(o, ref, 16)
-    assert_parity(out.cpu().numpy(), out_r, "round 2 out")
-    assert_parity(t["state"].cpu().numpy(), st_r, "round 2 committed (draft rejected)")
-    assert_parity(t["conv_ring"].cpu().numpy(), ring_r, "round 2 ring")
+    assert_parity(out.cpu().numpy(), out_r, "second verify out")
+    assert_parity(t["state"].cpu().numpy(), st_r, "second verify committed (draft rejected)")
+    assert_parity(t["conv_ring"].cpu().numpy(), ring_r, "second verify ring")
 
 
 def test_pair_full_workload_sampled(o):
