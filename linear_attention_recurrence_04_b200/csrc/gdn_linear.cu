@@ -52,6 +52,10 @@
 #ifndef GDN_LINEAR_BN
 #define GDN_LINEAR_BN 0
 #endif
+// 1: products with enough 256 x 256 tiles take the pair-CTA (cta_group::2) form.
+#ifndef GDN_LINEAR_PAIR
+#define GDN_LINEAR_PAIR 1
+#endif
 
 namespace gdn {
 
@@ -615,6 +619,208 @@ linear_bf16_splitk_kernel(const __grid_constant__ CUtensorMap tmap_x,
     if (warp == 1) tc::tmem_dealloc(tmem, kTmemCols);
 }
 
+// Pair-CTA form for large products: a cluster of two CTAs on two SMs owns a
+// 256 x 256 output tile and runs it as M = 256 tcgen05.mma (cta_group::2)
+// issued by the leader (rank 0). Each CTA stages its own 128 rows of x and its
+// own 128 rows of W per k-step (32 KB), so each SM takes in half the bytes of
+// a single-CTA 256 x 256 tile, and holds only its 128 x 256 quarter of the
+// accumulator: two accumulator sets fit in TMEM and a tile's epilogue runs
+// while the next tile's MMAs fill the other set.
+//   full[s]     leader only: one arrival (the leader's expect-tx of both
+//               CTAs' bytes); both CTAs' TMA loads complete on it;
+//   empty[s]    both CTAs: the leader's per-stage commit, multicast;
+//   acc_full    both CTAs: the leader's per-tile commit, multicast;
+//   acc_empty   leader only: the four epilogue warps of both CTAs (the
+//               peer's arrive remotely).
+// Rows of a tile accumulate over K in the same order as the other forms.
+// Every wait is bounded (2 s); every path meets the cluster barriers at the
+// end, after which the leader lets copies addressed to its barriers land.
+constexpr int kPairStages = 6;
+constexpr uint32_t kPairHalf = 128 * kBK * 2;                 // 128 rows x 64 bf16
+constexpr uint32_t kPairStage = 2 * kPairHalf;                // x half + W half
+constexpr size_t kPairDynamic = static_cast<size_t>(kPairStage) * kPairStages + 1024;
+
+__global__ void __launch_bounds__(kThreads, 1)
+linear_bf16_pair_kernel(const __grid_constant__ CUtensorMap tmap_x,
+                        const __grid_constant__ CUtensorMap tmap_w, float* __restrict__ y, int M,
+                        int N, int K, uint32_t* __restrict__ status) {
+    extern __shared__ uint8_t smem_raw[];
+    __shared__ __align__(8) uint64_t full[kPairStages];
+    __shared__ __align__(8) uint64_t empty[kPairStages];
+    __shared__ __align__(8) uint64_t acc_full[2];
+    __shared__ __align__(8) uint64_t acc_empty[2];
+    __shared__ uint32_t tmem_slot;
+    __shared__ int issued, consumed;
+    __shared__ int failed;
+
+    const uint32_t raw = tc::smem_u32(smem_raw);
+    const uint32_t base = (raw + 1023u) & ~1023u;
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+    const int rank = static_cast<int>(tc::cluster_ctarank());   // 0: leader
+    const int pair = static_cast<int>(blockIdx.x >> 1);
+    const int n_pairs = static_cast<int>(gridDim.x >> 1);
+    const int n_kt = (K + kBK - 1) / kBK;
+    const int tiles_n = (N + 255) / 256;
+    const int n_tiles = tiles_n * ((M + 255) / 256);
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < kPairStages; ++s) {
+            tc::mbar_init(tc::smem_u32(&full[s]), 1);
+            tc::mbar_init(tc::smem_u32(&empty[s]), 1);
+        }
+        for (int a = 0; a < 2; ++a) {
+            tc::mbar_init(tc::smem_u32(&acc_full[a]), 1);
+            tc::mbar_init(tc::smem_u32(&acc_empty[a]), 2 * kEpilogueWarps);
+        }
+        tc::fence_mbar_init();
+        issued = 0;
+        consumed = 0;
+        failed = 0;
+    }
+    if (warp == 1) {
+        tc::tmem_alloc_pair(tc::smem_u32(&tmem_slot), 512);
+        tc::tmem_relinquish_pair();
+    }
+    // both CTAs' barriers exist before either signals the other's
+    tc::tc_fence_before();
+    __syncthreads();
+    __syncwarp();
+    tc::cluster_sync();
+    tc::tc_fence_after();
+    const uint32_t tmem = tmem_slot;
+    volatile int* vfailed = &failed;
+    tc::grid_dep_launch();
+
+    if (warp == 0 && lane == 0) {
+        // ---- producer (both CTAs): this CTA's halves of every k-step -------
+        tc::prefetch_tmap(&tmap_x);
+        tc::prefetch_tmap(&tmap_w);
+        tc::grid_dep_wait();
+        int g = 0;
+        for (int tile = pair; tile < n_tiles && !*vfailed; tile += n_pairs) {
+            const int m0 = (tile / tiles_n) * 256 + rank * 128;
+            const int n0 = (tile % tiles_n) * 256 + rank * 128;
+            for (int kt = 0; kt < n_kt; ++kt, ++g) {
+                const int s = g % kPairStages;
+                const uint32_t ph = static_cast<uint32_t>(g / kPairStages) & 1u;
+                if (!tc::mbar_wait(tc::smem_u32(&empty[s]), ph ^ 1)) {
+                    if (status) atomicOr(status, tc::kTimeoutProducer);
+                    atomicExch(&failed, 1);
+                    break;
+                }
+                if (*vfailed) break;
+                const uint32_t a = base + s * kPairStage;
+                const uint32_t fb = tc::map_shared_rank(tc::smem_u32(&full[s]), 0);
+                if (rank == 0) tc::mbar_arrive_expect_tx(tc::smem_u32(&full[s]), 2 * kPairStage);
+                tc::tma_load_2d_pair(a, &tmap_x, fb, kt * kBK, m0);
+                tc::tma_load_2d_pair(a + kPairHalf, &tmap_w, fb, kt * kBK, n0);
+                issued = g + 1;
+            }
+        }
+    } else if (warp == 1 && lane == 0 && rank == 0) {
+        // ---- MMA issuer (leader): tile li into accumulator set li % 2 -------
+        tc::grid_dep_wait();
+        const uint32_t idesc = tc::idesc_bf16_f32(256, 256);
+        int g = 0;
+        bool ok = true;
+        int li = 0;
+        for (int tile = pair; ok && tile < n_tiles; tile += n_pairs, ++li) {
+            const int acc = li & 1;
+            const uint32_t d = tmem + static_cast<uint32_t>(acc) * 256;
+            if (!tc::mbar_wait(tc::smem_u32(&acc_empty[acc]), ((li >> 1) & 1) ^ 1) || *vfailed) {
+                if (status) atomicOr(status, tc::kTimeoutMma);
+                atomicExch(&failed, 1);
+                break;
+            }
+            tc::tc_fence_after();
+            for (int kt = 0; kt < n_kt; ++kt, ++g) {
+                const int s = g % kPairStages;
+                const uint32_t ph = static_cast<uint32_t>(g / kPairStages) & 1u;
+                if (!tc::mbar_wait(tc::smem_u32(&full[s]), ph) || *vfailed) {
+                    if (status) atomicOr(status, tc::kTimeoutMma);
+                    atomicExch(&failed, 1);
+                    ok = false;
+                    break;
+                }
+                consumed = g + 1;
+                tc::tc_fence_after();
+                const uint32_t a = base + s * kPairStage;
+#pragma unroll
+                for (int kk = 0; kk < kBK / 16; ++kk)
+                    tc::mma_bf16_pair(d, tc::desc_k_sw128(a + kk * 32),
+                                      tc::desc_k_sw128(a + kPairHalf + kk * 32), idesc,
+                                      (kt > 0 || kk > 0) ? 1u : 0u);
+                tc::mma_commit_pair(tc::smem_u32(&empty[s]), 0x3);   // both CTAs' slots
+            }
+            if (ok) tc::mma_commit_pair(tc::smem_u32(&acc_full[acc]), 0x3);
+        }
+    } else if (warp >= 2) {
+        // ---- epilogue (both CTAs): this CTA's 128 rows of each tile ---------
+        tc::grid_dep_wait();
+        const int quarter = warp & 3;
+        const uint32_t ae0 = tc::map_shared_rank(tc::smem_u32(&acc_empty[0]), 0);
+        const uint32_t ae1 = tc::map_shared_rank(tc::smem_u32(&acc_empty[1]), 0);
+        int li = 0;
+        for (int tile = pair; tile < n_tiles; tile += n_pairs, ++li) {
+            const int acc = li & 1;
+            if (!tc::mbar_wait(tc::smem_u32(&acc_full[acc]), (li >> 1) & 1) || *vfailed) {
+                if (status) atomicOr(status, tc::kTimeoutEpilogue);
+                atomicExch(&failed, 1);
+                break;
+            }
+            tc::tc_fence_after();
+            const int row = (tile / tiles_n) * 256 + rank * 128 + quarter * 32 + lane;
+            const int n0 = (tile % tiles_n) * 256;
+            const bool row_ok = row < M;
+            float* yrow = y + static_cast<int64_t>(row) * N;
+            const uint32_t src = tmem + static_cast<uint32_t>(acc) * 256 +
+                                 (static_cast<uint32_t>(quarter * 32) << 16);
+#pragma unroll 1
+            for (int c0 = 0; c0 < 256; c0 += 32) {
+                uint32_t r[32];
+                tc::tmem_ld_32x32b_x32(src + c0, r);
+                tc::tmem_ld_wait();
+                const int col = n0 + c0;
+                if (!row_ok || col >= N) continue;
+                if (col + 32 <= N && (N & 3) == 0) {
+#pragma unroll
+                    for (int j = 0; j < 32; j += 4)
+                        *reinterpret_cast<float4*>(yrow + col + j) =
+                            make_float4(__uint_as_float(r[j]), __uint_as_float(r[j + 1]),
+                                        __uint_as_float(r[j + 2]), __uint_as_float(r[j + 3]));
+                } else {
+#pragma unroll
+                    for (int j = 0; j < 32; ++j)
+                        if (col + j < N) yrow[col + j] = __uint_as_float(r[j]);
+                }
+            }
+            tc::tc_fence_before();
+            __syncwarp();
+            if (lane == 0) tc::mbar_arrive_cluster(acc ? ae1 : ae0);   // the leader's set is free
+        }
+    }
+
+    // Both CTAs meet here; then the leader lets any copy still addressed to
+    // its barriers land (a timeout path only), and both meet again before
+    // TMEM and shared memory are released.
+    if (warp < 2 && lane != 0) tc::grid_dep_wait();
+    tc::tc_fence_before();
+    __syncthreads();
+    __syncwarp();
+    tc::cluster_sync();
+    if (threadIdx.x == 0 && rank == 0 && failed) {
+        for (int g = consumed; g < issued; ++g)
+            tc::mbar_wait(tc::smem_u32(&full[g % kPairStages]),
+                          static_cast<uint32_t>(g / kPairStages) & 1u);
+    }
+    __syncthreads();
+    __syncwarp();
+    tc::cluster_sync();
+    tc::tc_fence_after();
+    if (warp == 1) tc::tmem_dealloc_pair(tmem, 512);
+}
+
 // cuTensorMapEncodeTiled through the runtime's driver entry point (no link
 // against libcuda).
 using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
@@ -785,6 +991,65 @@ cudaError_t launch_split_bn(const LinearArgs& a, int splits, cudaStream_t stream
                               static_cast<int>(a.K), splits, a.status, GateEpi{});
 }
 
+// Pairs of the pair-CTA kernel the device holds at once (cached per device).
+int max_active_pairs() {
+    constexpr int kDevs = 16;
+    static std::atomic<int> cache[kDevs];
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0) return 0;
+    if (dev < kDevs) {
+        const int c = cache[dev].load(std::memory_order_relaxed);
+        if (c > 0) return c - 1;
+    }
+    int n = 0;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(2);
+    cfg.blockDim = dim3(kThreads);
+    cfg.dynamicSmemBytes = kPairDynamic;
+    cudaLaunchAttribute attr;
+    attr.id = cudaLaunchAttributeClusterDimension;
+    attr.val.clusterDim.x = 2;
+    attr.val.clusterDim.y = 1;
+    attr.val.clusterDim.z = 1;
+    cfg.attrs = &attr;
+    cfg.numAttrs = 1;
+    if (cudaFuncSetAttribute(linear_bf16_pair_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             static_cast<int>(kPairDynamic)) != cudaSuccess ||
+        cudaOccupancyMaxActiveClusters(&n, linear_bf16_pair_kernel, &cfg) != cudaSuccess) {
+        cudaGetLastError();
+        n = 0;
+    }
+    if (dev < kDevs) cache[dev].store(n + 1, std::memory_order_relaxed);
+    return n;
+}
+
+cudaError_t launch_pair_gemm(const LinearArgs& a, int64_t tiles, int pairs, cudaStream_t stream) {
+    CUtensorMap tx, tw;
+    if (!make_tmap(&tx, a.x, a.M, a.K, 128) || !make_tmap(&tw, a.w, a.N, a.K, 128))
+        return cudaErrorInvalidValue;
+    cudaError_t err = cudaFuncSetAttribute(linear_bf16_pair_kernel,
+                                           cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                           static_cast<int>(kPairDynamic));
+    if (err != cudaSuccess) return err;
+    const int64_t n = tiles < pairs ? tiles : pairs;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(static_cast<unsigned>(2 * n));
+    cfg.blockDim = dim3(kThreads);
+    cfg.dynamicSmemBytes = kPairDynamic;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[2];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 2;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[1].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 2;
+    return cudaLaunchKernelEx(&cfg, linear_bf16_pair_kernel, tx, tw, a.y, static_cast<int>(a.M),
+                              static_cast<int>(a.N), static_cast<int>(a.K), a.status);
+}
+
 // The short-conv input projection with the gate and conv as its epilogue:
 // tiles of 64 channels, each split over K like the plain form (most chunks
 // that keep the clusters in one wave, at most 8).
@@ -857,6 +1122,12 @@ cudaError_t launch_linear_bf16(const LinearArgs& a, cudaStream_t stream) {
         if (tiles(256, 256) >= sms) shape = 512;
         else if (tiles(128, 256) >= sms) shape = 256;
         else if (tiles(128, 128) >= sms) shape = 128;
+    }
+    if (shape == 512 && GDN_LINEAR_PAIR && GDN_LINEAR_BN == 0 && a.N >= 256) {
+        // 256 x 256 tiles for every pair of SMs: the pair-CTA form
+        const int64_t tiles = ((a.M + 255) / 256) * ((a.N + 255) / 256);
+        const int pairs = max_active_pairs();
+        if (pairs > 0 && tiles >= pairs) return launch_pair_gemm(a, tiles, pairs, stream);
     }
     if (shape == 512) return launch_bn<256, 256>(a, stream);
     if (shape == 256) return launch_bn<256, 128>(a, stream);
