@@ -28,7 +28,12 @@
 //               sets, tile i drains while the MMAs of tile i+1 fill the other.
 // Tiles past M, N or K are zero-filled by TMA and masked on store. An
 // element's K order never depends on the tile width, the tile's place or M,
-// so a row's result is the same in any batch. Every mbarrier wait gives up
+// so a row's result is the same in any batch.
+//
+// Two more forms follow the persistent kernel: the pair-CTA kernel
+// (cta_group::2, one 256 x 256 tile per pair of SMs) that products with
+// enough such tiles take -- same K order, same rows -- and the split-K
+// cluster kernel for calls of at most 128 rows (its own fixed K grouping). Every mbarrier wait gives up
 // after 2 s, ORs an error bit into the caller's status word (if given), lets
 // in-flight copies land and frees TMEM.
 //
@@ -628,8 +633,8 @@ linear_bf16_splitk_kernel(const __grid_constant__ CUtensorMap tmap_x,
 // while the next tile's MMAs fill the other set.
 //   full[s]     leader only: one arrival (the leader's expect-tx of both
 //               CTAs' bytes); both CTAs' TMA loads complete on it;
-//   empty[s]    both CTAs: the leader's per-stage commit, multicast;
-//   acc_full    both CTAs: the leader's per-tile commit, multicast;
+//   empty[s]    both CTAs: the leader's per-stage commit, sent to both;
+//   acc_full    both CTAs: the leader's per-tile commit, sent to both;
 //   acc_empty   leader only: the four epilogue warps of both CTAs (the
 //               peer's arrive remotely).
 // Rows of a tile accumulate over K in the same order as the other forms.

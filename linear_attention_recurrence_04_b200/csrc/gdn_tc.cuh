@@ -6,7 +6,8 @@
 // tile stored with the 128-byte swizzle (TMA CU_TENSOR_MAP_SWIZZLE_128B) is
 // described by start address >> 4, leading byte offset 1 (unused for swizzled
 // K-major), stride byte offset 1024 B >> 4 (between 8-row groups), version 1
-// and layout type 2 (128-byte swizzle). No load here uses cluster multicast.
+// and layout type 2 (128-byte swizzle). Every TMA load here fills only the
+// issuing CTA's own shared memory.
 #pragma once
 
 #include <cstdint>
@@ -186,7 +187,8 @@ __device__ __forceinline__ void tma_prefetch_l2_2d(const void* tmap, int32_t x, 
 
 // ---- pair-CTA (cta_group::2) forms: one MMA over two SMs of a cluster pair --
 // TMA tile load into this CTA's shared memory whose byte count completes on
-// `bar`, a shared::cluster address (the pair leader's barrier). No multicast.
+// `bar`, a shared::cluster address (the pair leader's barrier); only this
+// CTA's shared memory is written.
 __device__ __forceinline__ void tma_load_2d_pair(uint32_t dst, const void* tmap, uint32_t bar,
                                                  int32_t x, int32_t y) {
     asm volatile(
