@@ -780,6 +780,55 @@ def cpu_oracle_baseline_parallel(name: str, budget_s: float):
                         f"calls on one thread: {r1} pass(es), {e1:.1f} s"))
 
 
+def cpu_oracle_prefill_parallel(budget_s: float):
+    """The fp64 C oracle on prefill_b4_t4096, parallel over (sequence, value
+    head) units: one thread per host core, each running whole units through
+    all T positions (ctypes releases the GIL during the call), over inputs
+    converted to fp64 once. Repeats passes over a sample of one unit per
+    thread until `budget_s` has elapsed (at least once); reports tokens/s of
+    the workload (a token is one position of one sequence, all 32 heads) and
+    the fp64 rate."""
+    import ctypes
+    from concurrent.futures import ThreadPoolExecutor
+    import oracle
+    from linear_attention_recurrence_04_b200 import inputs
+    o = oracle.load()
+    w = inputs.WORKLOADS["prefill_b4_t4096"]
+    d = w.draw()
+    f64 = {k: np.ascontiguousarray(v, dtype=np.float64) for k, v in d.items()}
+    B, Hv, dv, dk = f64["state"].shape
+    T, Hk = f64["q"].shape[1], f64["q"].shape[2]
+    n = max(1, min(len(os.sched_getaffinity(0)), B * Hv))
+    units = [np.array([u], dtype=np.int64) for u in range(n)]
+    states = [f64["state"].copy() for _ in range(n)]
+    outs = [np.zeros((B, T, Hv, dv)) for _ in range(n)]
+    pd = ctypes.POINTER(ctypes.c_double)
+    pi = ctypes.POINTER(ctypes.c_int64)
+    ptr = lambda a: a.ctypes.data_as(pd)
+
+    def work(j):
+        rc = o.lib.oracle_gdn_prefill(ptr(states[j]), ptr(f64["q"]), ptr(f64["k"]),
+                                      ptr(f64["v"]), ptr(f64["beta"]), ptr(f64["gate"]),
+                                      ptr(outs[j]), B, T, Hk, Hv, dk, dv,
+                                      units[j].ctypes.data_as(pi), 1)
+        if rc != 0:
+            raise RuntimeError(f"oracle_gdn_prefill returned {rc}")
+
+    reps, elapsed = 0, 0.0
+    with ThreadPoolExecutor(n) as ex:
+        while reps == 0 or elapsed < budget_s:
+            t0 = time.perf_counter()
+            list(ex.map(work, range(n)))
+            elapsed += time.perf_counter() - t0
+            reps += 1
+    unit_positions = reps * n * T
+    return dict(value=unit_positions / Hv / elapsed, unit="tokens/s", cores=n, kind="oracle",
+                fp64_gflops=unit_positions * 7 * dk * dv / elapsed / 1e9,
+                sample=(f"{reps} pass(es) over {n} of the {B * Hv} (sequence, head) units of "
+                        f"prefill_b4_t4096, each through all {T} positions, one unit per "
+                        f"thread, {n} threads, {elapsed:.1f} s"))
+
+
 # --------------------------------------------------------------------------
 # arms
 # --------------------------------------------------------------------------
@@ -985,6 +1034,9 @@ def run_ours(args) -> int:
         # the same oracle on every host core (independent units, no exchange)
         line["cpu_baseline_all_cores"] = cpu_oracle_baseline_parallel(HEADLINE,
                                                                       args.cpu_budget)
+        if "prefill_b4_t4096" in line.get("workloads", {}):
+            line["workloads"]["prefill_b4_t4096"]["cpu_baseline_all_cores"] = \
+                cpu_oracle_prefill_parallel(args.cpu_budget / 2)
 
     if env["world"] > 1:
         barrier()

@@ -110,3 +110,6 @@ def test_cpu_baselines_time_the_oracle():
     assert allc["kind"] == "oracle" and allc["unit"] == bench.UNIT
     assert 1 <= allc["cores"] <= len(os.sched_getaffinity(0))
     assert allc["value"] > 0 and allc["value_one_thread"] > 0
+    pre = bench.cpu_oracle_prefill_parallel(0.0)
+    assert pre["unit"] == "tokens/s" and pre["value"] > 0 and pre["fp64_gflops"] > 0
+    assert 1 <= pre["cores"] <= len(os.sched_getaffinity(0))
