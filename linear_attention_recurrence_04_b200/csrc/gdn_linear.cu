@@ -640,10 +640,14 @@ linear_bf16_splitk_kernel(const __grid_constant__ CUtensorMap tmap_x,
 // Rows of a tile accumulate over K in the same order as the other forms.
 // Every wait is bounded (2 s); every path meets the cluster barriers at the
 // end, after which the leader lets copies addressed to its barriers land.
-constexpr int kPairStages = 6;
+#ifndef GDN_LINEAR_PAIR_STAGES
+#define GDN_LINEAR_PAIR_STAGES 6
+#endif
+constexpr int kPairStages = GDN_LINEAR_PAIR_STAGES;
 constexpr uint32_t kPairHalf = 128 * kBK * 2;                 // 128 rows x 64 bf16
 constexpr uint32_t kPairStage = 2 * kPairHalf;                // x half + W half
 constexpr size_t kPairDynamic = static_cast<size_t>(kPairStage) * kPairStages + 1024;
+static_assert(kPairDynamic <= 232448, "the stage ring fits the shared memory of a CTA");
 
 __global__ void __launch_bounds__(kThreads, 1)
 linear_bf16_pair_kernel(const __grid_constant__ CUtensorMap tmap_x,
