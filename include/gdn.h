@@ -33,7 +33,7 @@
  *     aligned, workspaces 256-byte aligned; the per-head scalars (beta,
  *     gate, a, b, A_log, dt_bias), norm_w and the optional status words need
  *     4-byte alignment.
- *   - Status words (gdn_prefill, gdn_linear_bf16, gdn_forward_batch*,
+ *   - Status words (gdn_prefill, gdn_linear_bf16*, gdn_forward_batch*,
  *     gdn_short_conv_*): an optional zero-initialised device uint32 into
  *     which a kernel ORs a bit if one of its bounded waits (2 s) ever gives
  *     up; the kernel then returns without hanging. NULL: not reported.
