@@ -283,9 +283,10 @@ linear_bf16_kernel(const __grid_constant__ CUtensorMap tmap_x,
 
 // Split-K form for products of at most 128 rows (decode-sized calls).
 //
-// With few rows the persistent kernel's cost is one CTA's chain of K/16
-// dependent MMAs into one accumulator (32 k-steps x 4 MMAs for K = 2048), and
-// only N / BN SMs stream the weights. Here a cluster of `splits` CTAs shares
+// With few rows the persistent kernel's cost is one CTA's K/16 MMA
+// instructions (32 k-steps x 4 for K = 2048), each about 87 ns of issue
+// whatever the tile's width or rows (interleaved accumulators do not shorten
+// it), and only N / BN SMs stream the weights. Here a cluster of `splits` CTAs shares
 // one 128 x BN output tile: CTA r runs k-steps [r n_kt / S, (r+1) n_kt / S)
 // into its own TMEM accumulator, parks the fp32 partial tile in its (then
 // idle) stage ring, and after a cluster barrier every CTA sums a 1/S slice of
