@@ -7,16 +7,23 @@ workload (64 sequences x 32 value heads x 128 x 128 fp32 state, one layer).
 The timed region holds exactly K steps, bracketed by a barrier and a device
 synchronisation on both sides and timed with CUDA events on the launching
 stream; with N ranks each rank runs its own B = 64 batch (weak scaling, no
-collective on the data path) and the slowest rank's time is used.
+collective on the data path) and the slowest rank's time is used. Without a
+launcher, ``--gpus N`` (N > 1) starts N ranks itself through torchrun; under
+a launcher, N must equal WORLD_SIZE.
+
+The metric is state GB/s: each value head's 64 KiB state read once and
+written once per token, counted the same way in every figure (the GPU step,
+the end-to-end leg, the CPU baselines and the reference arm).
 
 Printed (rank 0, one JSON line): state GB/s over all ranks, layer-tokens/s,
 the roofline of the step kernel against the measured HBM copy bandwidth, an
 end-to-end figure through the C ABI with the per-step inputs copied from
-pinned host memory and the output copied back, NVML clock samples taken
-during the timed region, the fp64 CPU oracle timed on this host as a
-reported baseline, and (N = 1) the other workloads (36-layer and B = 1 decode,
-prefill, fused layer and verify, batched forward, KDA core, short-conv mixer)
-measured the same way, each with its roofline.
+pinned host memory and the output copied back (graph-replayed and eager),
+NVML clock samples taken during the timed region, the CPU oracle timed on
+this host as a reported baseline (its literal fp32 instantiation, and the
+fp64 parity oracle beside it), and (N = 1) the other workloads (36-layer and
+B = 1 decode, prefill, fused layer and verify, batched forward, KDA core,
+short-conv mixer) measured the same way, each with its roofline.
 
 ``--impl reference`` times the CPU oracle alone on the same workload and
 metric (rank 0 only; other ranks exit at once).
@@ -53,6 +60,20 @@ E2E_SLOTS = 2            # device buffer slots of the end-to-end pipeline
 def step_bytes(L: int, B: int, Hk: int = 16, Hv: int = 32, d: int = 128) -> int:
     heads = L * B * Hv
     return heads * (2 * d * d * 4 + 2 * d * 4 + 2 * 4) + L * B * Hk * 2 * d * 4
+
+
+def state_rw_bytes(L: int, B: int, Hv: int = 32, d: int = 128) -> int:
+    """State bytes one decode token moves: every value head's d x d fp32 state
+    read once and written once. The headline metric (state GB/s) is this
+    figure per second, in every arm: the GPU step, the end-to-end leg, the
+    CPU oracle baselines and the reference arm."""
+    return 2 * L * B * Hv * d * d * 4
+
+
+def state_gb_s(units: int, seconds: float, n_ranks: int = 1, d: int = 128) -> float:
+    """State GB/s of `units` value-head tokens per rank over `seconds` (the
+    slowest rank's time): read + write of each unit's d x d fp32 state."""
+    return throughput(units * 2 * d * d * 4 / 1e9, n_ranks, seconds)
 
 
 def pair_bytes(L: int, B: int, Hk: int = 16, Hv: int = 32, d: int = 128) -> int:
@@ -255,6 +276,13 @@ def _to_dev(d: Dict[str, np.ndarray], device) -> Dict[str, "torch.Tensor"]:
     return {k: torch.from_numpy(np.ascontiguousarray(v)).to(device) for k, v in d.items()}
 
 
+def step_footprint(L: int, B: int, Hk: int = 16, Hv: int = 32, d: int = 128) -> int:
+    """Bytes of one decode input set (state, q, k, v, beta, gate) and its
+    output, the unit the timed launches rotate over."""
+    return (L * B * Hv * d * d * 4 + 2 * L * B * Hk * d * 4 + 2 * L * B * Hv * d * 4
+            + 2 * L * B * Hv * 4)
+
+
 def _sets_for(bytes_per_set: int) -> int:
     """Rotating input sets so the sets together exceed 4x the L2."""
     return max(1, min(64, math.ceil(4 * L2_BYTES / max(bytes_per_set, 1))))
@@ -308,7 +336,8 @@ def bench_step_workload(name: str, steps: int, warmup: int, device, seed_offset:
     d = inputs.decode_inputs(L, B, seed=w.seed + seed_offset)
     base = _to_dev(d, device)
     nbytes = step_bytes(L, B)
-    footprint = sum(v.nbytes for v in d.values()) + d["v"].nbytes   # inputs + out
+    footprint = step_footprint(L, B)
+    assert footprint == sum(v.nbytes for v in d.values()) + d["v"].nbytes   # inputs + out
     n_sets = _sets_for(footprint)
     sets = [base] + [{k: v.clone() for k, v in base.items()} for _ in range(n_sets - 1)]
     outs = [torch.empty_like(s["v"]) for s in sets]
@@ -319,7 +348,7 @@ def bench_step_workload(name: str, steps: int, warmup: int, device, seed_offset:
         gdn.step(s["state"], s["q"], s["k"], s["v"], s["beta"], s["gate"], outs[i])
 
     secs = time_launches(launch, n_sets, steps, warmup, stream, graph=graph)
-    return dict(seconds=secs, bytes=nbytes, state_bytes=L * B * 32 * STATE_BYTES_PER_HEAD,
+    return dict(seconds=secs, bytes=nbytes, units=L * B * 32, state_rw=state_rw_bytes(L, B),
                 layer_tokens=L * B, n_sets=n_sets, set_bytes=footprint, sets=sets, outs=outs,
                 d=d)
 
@@ -334,11 +363,14 @@ def bench_e2e(d: Dict[str, np.ndarray], steps: int, warmup: int, device):
     copy per step). Copy-in, compute and copy-out run on three streams with
     two device buffer slots, so step i+1's inputs travel while step i
     computes and step i-1's output travels back; events order every reuse of
-    a slot. The K steps of that loop -- each one's copy-in, gdn_step call
-    through the C ABI and copy-out -- are captured once into a CUDA graph
-    (as a serving loop would, so host-side issue does not pace the GPU) and
-    replayed; the timed region runs from the first copy-in to the last
-    copy-out."""
+    a slot. The same K-step loop is timed twice:
+      - graph: the K steps (each one's copy-in, gdn_step call through the C
+        ABI and copy-out) captured once into a CUDA graph and replayed, as a
+        serving loop would, so host-side issue does not pace the GPU;
+      - eager: the K steps issued from Python, each one a ctypes call of
+        gdn_step with the library's argument checks and launch on the host.
+    Each timed region runs from before the first copy-in to after the last
+    copy-out. Returns (graph_seconds, eager_seconds, h2d_bytes, d2h_bytes)."""
     import torch
     from linear_attention_recurrence_04_b200 import gdn
     names = ("q", "k", "v", "beta", "gate")
@@ -383,35 +415,44 @@ def bench_e2e(d: Dict[str, np.ndarray], steps: int, warmup: int, device):
             out_done[sl].record(s_out)
         used[sl] = True
 
+    def loop(origin):
+        # the three streams fork from `origin` and join it again at the end
+        for s in (s_in, s_comp, s_out):
+            s.wait_stream(origin)
+        for i in range(steps):
+            step(warmup + i)
+        for s in (s_in, s_comp, s_out):
+            origin.wait_stream(s)
+
     for i in range(warmup):
         step(i)
     torch.cuda.synchronize()
-    # Capture the K steps: the three streams fork from the capture stream and
-    # join it again at the end; slot reuse inside the graph waits only on
-    # events recorded inside it.
+    # graph: slot reuse inside the graph waits only on events recorded inside it
     graph = torch.cuda.CUDAGraph()
     cap = torch.cuda.Stream(device)
     used[:] = [False] * n_slots
     with torch.cuda.graph(graph, stream=cap):
-        for s in (s_in, s_comp, s_out):
-            s.wait_stream(cap)
-        for i in range(steps):
-            step(warmup + i)
-        for s in (s_in, s_comp, s_out):
-            cap.wait_stream(s)
+        loop(cap)
     torch.cuda.synchronize()
+    replay = torch.cuda.current_stream(device)
     start = torch.cuda.Event(enable_timing=True)
     end = torch.cuda.Event(enable_timing=True)
-    replay = torch.cuda.current_stream(device)
     start.record(replay)
     graph.replay()
     end.record(replay)
     torch.cuda.synchronize()
-    secs = start.elapsed_time(end) / 1e3
+    graph_secs = start.elapsed_time(end) / 1e3
     del graph
+    # eager: the same loop issued call by call
+    used[:] = [False] * n_slots
+    start.record(replay)
+    loop(replay)
+    end.record(replay)
+    torch.cuda.synchronize()
+    eager_secs = start.elapsed_time(end) / 1e3
     h2d = host_in.numel() * host_in.element_size()
     d2h = host_out[0].numel() * host_out[0].element_size()
-    return secs, h2d, d2h
+    return graph_secs, eager_secs, h2d, d2h
 
 
 def bench_prefill(steps: int, warmup: int, device):
@@ -694,67 +735,87 @@ def bench_kda(steps_decode: int, steps_prefill: int, device, peaks, alu_peak):
     return res
 
 
-def cpu_oracle_baseline(name: str, budget_s: float, max_units: Optional[int] = None):
-    """Time the fp64 oracle as it stands on a bounded sample of the workload:
-    whole decode steps over the first `units` (layer, sequence, head) units,
-    repeated until `budget_s` has elapsed (at least once)."""
-    import oracle
-    from linear_attention_recurrence_04_b200 import inputs
-    o = oracle.load()
-    w = inputs.WORKLOADS[name]
-    L, B = w.sizes["L"], w.sizes["B"]
-    d = inputs.decode_inputs(L, B, seed=w.seed)
-    total_units = L * B * 32
-    units = np.arange(total_units if max_units is None else min(max_units, total_units))
-    st = d["state"]
+class OracleDecode:
+    """The C oracle's decode entry on one decode workload, with the inputs
+    converted once (outside any timing) to the instantiation's type:
+    precision "f32" is the literal fp32 instantiation (``gdn_oracle_f32.c``,
+    the pages' F32 CPU step), "f64" the double parity oracle. `run(units)`
+    advances the listed (layer, sequence, head) units by one token in place;
+    calls on disjoint unit lists may run from several threads at once
+    (ctypes releases the GIL during the call)."""
+
+    def __init__(self, name: str, precision: str = "f32"):
+        import ctypes
+        import oracle
+        from linear_attention_recurrence_04_b200 import inputs
+        w = inputs.WORKLOADS[name]
+        d = inputs.decode_inputs(w.sizes["L"], w.sizes["B"], seed=w.seed)
+        if precision == "f32":
+            lib, ctype, dt = oracle.load_f32().lib, ctypes.c_float, np.float32
+            self._fn = lib.oracle_gdn_step_f32
+        elif precision == "f64":
+            lib, ctype, dt = oracle.load().lib, ctypes.c_double, np.float64
+            self._fn = lib.oracle_gdn_step
+        else:
+            raise ValueError(precision)
+        self.precision = precision
+        self.a = {k: np.array(v, dtype=dt, order="C") for k, v in d.items()}
+        self.out = np.zeros(self.a["v"].shape, dtype=dt)
+        self.L, self.B, self.Hv, self.dv, self.dk = self.a["state"].shape
+        self.Hk = self.a["q"].shape[2]
+        self.total_units = self.L * self.B * self.Hv
+        self._pt = ctypes.POINTER(ctype)
+        self._pi = ctypes.POINTER(ctypes.c_int64)
+
+    def run(self, units: np.ndarray) -> None:
+        u = np.ascontiguousarray(units, dtype=np.int64)
+        p = lambda x: x.ctypes.data_as(self._pt)
+        a = self.a
+        rc = self._fn(p(a["state"]), p(a["q"]), p(a["k"]), p(a["v"]), p(a["beta"]),
+                      p(a["gate"]), p(self.out), self.L, self.B, self.Hk, self.Hv, self.dk,
+                      self.dv, u.ctypes.data_as(self._pi), int(u.size))
+        if rc != 0:
+            raise RuntimeError(f"oracle decode entry returned {rc}")
+
+
+def _label(precision: str) -> str:
+    return ("the fp32 instantiation of the C oracle (literal F32 step)" if precision == "f32"
+            else "the fp64 C oracle")
+
+
+def cpu_oracle_baseline(name: str, budget_s: float, max_units: Optional[int] = None,
+                        precision: str = "f32"):
+    """Time the oracle as it stands, on one thread, over a bounded sample of
+    the workload: whole decode steps over the first `units` (layer, sequence,
+    head) units, repeated until `budget_s` has elapsed (at least once). The
+    inputs are converted once, before timing."""
+    od = OracleDecode(name, precision)
+    units = np.arange(od.total_units if max_units is None else
+                      min(max_units, od.total_units), dtype=np.int64)
     reps, elapsed = 0, 0.0
     while reps == 0 or elapsed < budget_s:
         t0 = time.perf_counter()
-        o.step(st, d["q"], d["k"], d["v"], d["beta"], d["gate"], units=units)
+        od.run(units)
         elapsed += time.perf_counter() - t0
         reps += 1
-    state_bytes = reps * len(units) * STATE_BYTES_PER_HEAD * 2
-    return dict(value=state_bytes / elapsed / 1e9, unit=UNIT, cores=1, kind="oracle",
-                sample=(f"{reps} pass(es) of the fp64 C oracle over {len(units)} of "
-                        f"{total_units} value-head units of {name}, single thread, "
-                        f"{elapsed:.1f} s"),
+    return dict(value=state_gb_s(reps * len(units), elapsed), unit=UNIT, cores=1,
+                kind="oracle", precision=precision,
+                sample=(f"{reps} pass(es) of {_label(precision)} over {len(units)} of "
+                        f"{od.total_units} value-head units of {name}, single thread, inputs "
+                        f"converted once before timing, {elapsed:.1f} s"),
                 seconds=elapsed, units=int(len(units)), reps=reps)
 
 
-def cpu_oracle_baseline_parallel(name: str, budget_s: float):
-    """The same fp64 C oracle on every host core this process may use: its
-    step entry is called from one thread per core on disjoint unit lists
-    (ctypes releases the GIL during the call), over inputs converted to fp64
+def cpu_oracle_baseline_parallel(name: str, budget_s: float, precision: str = "f32"):
+    """The same oracle entry on every host core this process may use: called
+    from one thread per core on disjoint unit lists, over inputs converted
     once and shared. Whole decode steps over all units, repeated until
-    `budget_s` has elapsed (at least once)."""
-    import ctypes
+    `budget_s` has elapsed (at least once); half the budget times the same
+    calls on one thread."""
     from concurrent.futures import ThreadPoolExecutor
-    import oracle
-    from linear_attention_recurrence_04_b200 import inputs
-    o = oracle.load()
-    w = inputs.WORKLOADS[name]
-    L, B = w.sizes["L"], w.sizes["B"]
-    d = inputs.decode_inputs(L, B, seed=w.seed)
-    f64 = {k: np.ascontiguousarray(v, dtype=np.float64) for k, v in d.items()}
-    L, B, Hv, dv, dk = f64["state"].shape
-    Hk = f64["q"].shape[2]
-    total_units = L * B * Hv
+    od = OracleDecode(name, precision)
     n = max(1, len(os.sched_getaffinity(0)))
-    chunks = [np.ascontiguousarray(c, dtype=np.int64)
-              for c in np.array_split(np.arange(total_units), n) if c.size]
-    outs = [np.zeros((L, B, Hv, dv)) for _ in chunks]
-    pd = ctypes.POINTER(ctypes.c_double)
-    pi = ctypes.POINTER(ctypes.c_int64)
-    ptr = lambda a: a.ctypes.data_as(pd)
-
-    def work(j):
-        u = chunks[j]
-        rc = o.lib.oracle_gdn_step(ptr(f64["state"]), ptr(f64["q"]), ptr(f64["k"]),
-                                   ptr(f64["v"]), ptr(f64["beta"]), ptr(f64["gate"]),
-                                   ptr(outs[j]), L, B, Hk, Hv, dk, dv,
-                                   u.ctypes.data_as(pi), int(u.size))
-        if rc != 0:
-            raise RuntimeError(f"oracle_gdn_step returned {rc}")
+    chunks = [c for c in np.array_split(np.arange(od.total_units, dtype=np.int64), n) if c.size]
 
     def timed(threads, budget):
         reps, elapsed = 0, 0.0
@@ -762,57 +823,55 @@ def cpu_oracle_baseline_parallel(name: str, budget_s: float):
             while reps == 0 or elapsed < budget:
                 t0 = time.perf_counter()
                 if threads == 1:
-                    for j in range(len(chunks)):
-                        work(j)
+                    for c in chunks:
+                        od.run(c)
                 else:
-                    list(ex.map(work, range(len(chunks))))
+                    list(ex.map(od.run, chunks))
                 elapsed += time.perf_counter() - t0
                 reps += 1
-        return reps, elapsed, reps * total_units * STATE_BYTES_PER_HEAD * 2 / elapsed / 1e9
+        return reps, elapsed, state_gb_s(reps * od.total_units, elapsed)
 
-    r1, e1, v1 = timed(1, budget_s / 2)           # the same calls on one thread
+    r1, e1, v1 = timed(1, budget_s / 2)
     rn, en, vn = timed(len(chunks), budget_s / 2)
-    return dict(value=vn, unit=UNIT, cores=len(chunks), kind="oracle",
+    return dict(value=vn, unit=UNIT, cores=len(chunks), kind="oracle", precision=precision,
                 value_one_thread=v1,
-                sample=(f"{rn} pass(es) of the fp64 C oracle over all {total_units} "
+                sample=(f"{rn} pass(es) of {_label(precision)} over all {od.total_units} "
                         f"value-head units of {name}, {len(chunks)} threads on disjoint units, "
-                        f"inputs converted to fp64 once and shared, {en:.1f} s; the same "
-                        f"calls on one thread: {r1} pass(es), {e1:.1f} s"))
+                        f"inputs converted once and shared, {en:.1f} s; the same calls on one "
+                        f"thread: {r1} pass(es), {e1:.1f} s"))
 
 
-def cpu_oracle_prefill_parallel(budget_s: float):
-    """The fp64 C oracle on prefill_b4_t4096, parallel over (sequence, value
-    head) units: one thread per host core, each running whole units through
-    all T positions (ctypes releases the GIL during the call), over inputs
-    converted to fp64 once. Repeats passes over a sample of one unit per
-    thread until `budget_s` has elapsed (at least once); reports tokens/s of
-    the workload (a token is one position of one sequence, all 32 heads) and
-    the fp64 rate."""
+def cpu_oracle_prefill_parallel(budget_s: float, precision: str = "f32"):
+    """The oracle's prefill entry on prefill_b4_t4096, parallel over
+    (sequence, value head) units: one thread per host core, each running
+    whole units through all T positions, over inputs converted once. Repeats
+    passes over a sample of one unit per thread until `budget_s` has elapsed
+    (at least once); reports tokens/s of the workload (a token is one
+    position of one sequence, all 32 heads) and the arithmetic rate."""
     import ctypes
     from concurrent.futures import ThreadPoolExecutor
     import oracle
     from linear_attention_recurrence_04_b200 import inputs
-    o = oracle.load()
+    if precision == "f32":
+        fn, ctype, dt = oracle.load_f32().lib.oracle_gdn_prefill_f32, ctypes.c_float, np.float32
+    else:
+        fn, ctype, dt = oracle.load().lib.oracle_gdn_prefill, ctypes.c_double, np.float64
     w = inputs.WORKLOADS["prefill_b4_t4096"]
-    d = w.draw()
-    f64 = {k: np.ascontiguousarray(v, dtype=np.float64) for k, v in d.items()}
-    B, Hv, dv, dk = f64["state"].shape
-    T, Hk = f64["q"].shape[1], f64["q"].shape[2]
+    a = {k: np.array(v, dtype=dt, order="C") for k, v in w.draw().items()}
+    B, Hv, dv, dk = a["state"].shape
+    T, Hk = a["q"].shape[1], a["q"].shape[2]
     n = max(1, min(len(os.sched_getaffinity(0)), B * Hv))
     units = [np.array([u], dtype=np.int64) for u in range(n)]
-    states = [f64["state"].copy() for _ in range(n)]
-    outs = [np.zeros((B, T, Hv, dv)) for _ in range(n)]
-    pd = ctypes.POINTER(ctypes.c_double)
-    pi = ctypes.POINTER(ctypes.c_int64)
-    ptr = lambda a: a.ctypes.data_as(pd)
+    states = [a["state"].copy() for _ in range(n)]
+    outs = [np.zeros((B, T, Hv, dv), dtype=dt) for _ in range(n)]
+    pt, pi = ctypes.POINTER(ctype), ctypes.POINTER(ctypes.c_int64)
+    p = lambda x: x.ctypes.data_as(pt)
 
     def work(j):
-        rc = o.lib.oracle_gdn_prefill(ptr(states[j]), ptr(f64["q"]), ptr(f64["k"]),
-                                      ptr(f64["v"]), ptr(f64["beta"]), ptr(f64["gate"]),
-                                      ptr(outs[j]), B, T, Hk, Hv, dk, dv,
-                                      units[j].ctypes.data_as(pi), 1)
+        rc = fn(p(states[j]), p(a["q"]), p(a["k"]), p(a["v"]), p(a["beta"]), p(a["gate"]),
+                p(outs[j]), B, T, Hk, Hv, dk, dv, units[j].ctypes.data_as(pi), 1)
         if rc != 0:
-            raise RuntimeError(f"oracle_gdn_prefill returned {rc}")
+            raise RuntimeError(f"oracle prefill entry returned {rc}")
 
     reps, elapsed = 0, 0.0
     with ThreadPoolExecutor(n) as ex:
@@ -823,54 +882,57 @@ def cpu_oracle_prefill_parallel(budget_s: float):
             reps += 1
     unit_positions = reps * n * T
     return dict(value=unit_positions / Hv / elapsed, unit="tokens/s", cores=n, kind="oracle",
-                fp64_gflops=unit_positions * 7 * dk * dv / elapsed / 1e9,
-                sample=(f"{reps} pass(es) over {n} of the {B * Hv} (sequence, head) units of "
-                        f"prefill_b4_t4096, each through all {T} positions, one unit per "
-                        f"thread, {n} threads, {elapsed:.1f} s"))
+                precision=precision,
+                gflops=unit_positions * 7 * dk * dv / elapsed / 1e9,
+                sample=(f"{reps} pass(es) of {_label(precision)} over {n} of the {B * Hv} "
+                        f"(sequence, head) units of prefill_b4_t4096, each through all {T} "
+                        f"positions, one unit per thread, {n} threads, {elapsed:.1f} s"))
 
 
 # --------------------------------------------------------------------------
 # arms
 # --------------------------------------------------------------------------
-def config_block(n_sets: int, set_bytes: int) -> Dict[str, object]:
+def config_block() -> Dict[str, object]:
+    """The headline workload, identical in both arms."""
+    n_sets = _sets_for(step_footprint(1, 64))
     return {"workload": HEADLINE, "L": 1, "B": 64, "Hk": 16, "Hv": 32, "dk": 128, "dv": 128,
             "state_bytes": 64 * 32 * STATE_BYTES_PER_HEAD,
-            "l2": f"rotating {n_sets} input sets of {set_bytes / 2**20:.0f} MiB "
+            "l2": f"rotating {n_sets} input sets of {step_footprint(1, 64) / 2**20:.0f} MiB "
                   f"(> 4x the 126 MB L2)",
             "parallelism": "independent batches per rank"}
 
 
 def run_reference(args) -> int:
+    """The oracle as the reference arm: the fp32 instantiation of the C
+    oracle's decode step (the pages' F32 CPU path), one host thread, each
+    step a bounded sample of the headline workload's units, sized so that
+    the whole run stays within about two minutes."""
     env = dist_env()
     if env["rank"] != 0:
         return 0
     n_steps = args.steps + args.warmup
-    # size each step so the whole run stays within about two minutes
-    probe = cpu_oracle_baseline(HEADLINE, 0.0, max_units=64)
-    per_unit = probe["seconds"] / probe["units"]
-    units = int(max(1, min(2048, 120.0 / max(n_steps, 1) / per_unit)))
-    import oracle
-    from linear_attention_recurrence_04_b200 import inputs
-    o = oracle.load()
-    w = inputs.WORKLOADS[HEADLINE]
-    d = inputs.decode_inputs(1, 64, seed=w.seed)
-    sel = np.arange(units)
-    st = d["state"]
+    od = OracleDecode(HEADLINE, "f32")
+    probe = np.arange(64, dtype=np.int64)
+    t0 = time.perf_counter()
+    od.run(probe)
+    per_unit = (time.perf_counter() - t0) / probe.size
+    units = int(max(1, min(od.total_units, 120.0 / max(n_steps, 1) / per_unit)))
+    sel = np.arange(units, dtype=np.int64)
     for _ in range(args.warmup):
-        st, _out = o.step(st, d["q"], d["k"], d["v"], d["beta"], d["gate"], units=sel)
+        od.run(sel)
     t0 = time.perf_counter()
     for _ in range(args.steps):
-        st, _out = o.step(st, d["q"], d["k"], d["v"], d["beta"], d["gate"], units=sel)
+        od.run(sel)
     secs = time.perf_counter() - t0
-    value = args.steps * units * STATE_BYTES_PER_HEAD * 2 / secs / 1e9
-    sample = (f"each step: the fp64 C oracle over {units} of 2048 value-head units of "
-              f"{HEADLINE}, single thread")
+    value = state_gb_s(args.steps * units, secs)
+    sample = (f"each step: {_label('f32')} over {units} of {od.total_units} value-head units "
+              f"of {HEADLINE}, single thread, inputs converted once before timing")
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": env["world"],
         "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": secs / max(args.steps, 1) * 1e3, "higher_is_better": True,
-        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": config_block(1, 0) | {"l2": "n/a (host)"}, "impl": "reference",
+        "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+        "config": config_block(), "impl": "reference",
         "cpu_baseline": {"value": value, "unit": UNIT, "cores": 1, "kind": "oracle",
                          "sample": sample},
         "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
@@ -928,8 +990,7 @@ def run_ours(args) -> int:
     del graph
     eager_secs = max_over_ranks(time_launches(launch, n_sets, args.steps, 3, stream), device)
     per_launch = secs / max(args.steps, 1)
-    state_total = res["state_bytes"] * args.steps
-    value = throughput(state_total / 1e9, env["world"], secs)
+    value = state_gb_s(res["units"] * args.steps, secs, env["world"])
     tokens_per_s = throughput(res["layer_tokens"] * args.steps, env["world"], secs)
     peaks = measured_peaks()
     achieved = res["bytes"] / per_launch / 1e9
@@ -938,9 +999,11 @@ def run_ours(args) -> int:
     # ---- end to end through the C ABI with host buffers --------------
     e2e_steps = max(args.steps, 1)
     barrier()
-    e2e_secs, h2d, d2h = bench_e2e(res["d"], e2e_steps, args.warmup, device)
+    e2e_secs, e2e_eager_secs, h2d, d2h = bench_e2e(res["d"], e2e_steps, args.warmup, device)
     e2e_secs = max_over_ranks(e2e_secs, device)
-    e2e_value = throughput(res["state_bytes"] * e2e_steps / 1e9, env["world"], e2e_secs)
+    e2e_eager_secs = max_over_ranks(e2e_eager_secs, device)
+    e2e_value = state_gb_s(res["units"] * e2e_steps, e2e_secs, env["world"])
+    e2e_eager = state_gb_s(res["units"] * e2e_steps, e2e_eager_secs, env["world"])
     del sets, outs, res["sets"], res["outs"]
     torch.cuda.empty_cache()
 
@@ -950,7 +1013,7 @@ def run_ours(args) -> int:
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
         "data": "synthetic (seeded numpy draws: state N(0,0.05^2), unit q/k, v N(0,1), "
                 "beta sigmoid(N(0,1)), gate U(-1,0))",
-        "config": config_block(n_sets, res["set_bytes"]),
+        "config": config_block(),
         "layer_tokens_per_s": tokens_per_s,
         "timing": "CUDA graph of the K launches, replayed once between CUDA events",
         "eager_ms_per_step": eager_secs / max(args.steps, 1) * 1e3,
@@ -966,7 +1029,11 @@ def run_ours(args) -> int:
                 "d2h_bytes_per_step": d2h, "ms_per_step": e2e_secs / e2e_steps * 1e3,
                 "timing": "K pipelined steps (pinned copy-in, gdn_step through the C ABI, "
                           "copy-out to pinned memory) captured in one CUDA graph, replayed "
-                          "between CUDA events"},
+                          "between CUDA events",
+                "eager": {"value": e2e_eager, "unit": UNIT,
+                          "ms_per_step": e2e_eager_secs / e2e_steps * 1e3,
+                          "timing": "the same K steps issued from Python, one ctypes call of "
+                                    "gdn_step per step, between CUDA events"}},
         "gpu_launches": args.steps,
         "clocks": clocks.summary(),
     }
@@ -1029,14 +1096,20 @@ def run_ours(args) -> int:
         line["workloads"] = extras
 
     if env["rank"] == 0 and env["world"] == 1 and not args.no_cpu_baseline:
-        cb = cpu_oracle_baseline(HEADLINE, args.cpu_budget)
+        budget = args.cpu_budget
+        cb = cpu_oracle_baseline(HEADLINE, budget / 2, precision="f32")
         line["cpu_baseline"] = {k: cb[k] for k in ("value", "unit", "cores", "kind", "sample")}
-        # the same oracle on every host core (independent units, no exchange)
-        line["cpu_baseline_all_cores"] = cpu_oracle_baseline_parallel(HEADLINE,
-                                                                      args.cpu_budget)
+        # the same instantiation on every host core (independent units, no exchange)
+        line["cpu_baseline_all_cores"] = cpu_oracle_baseline_parallel(HEADLINE, budget / 2,
+                                                                      precision="f32")
+        # the double parity oracle, for reference
+        c64 = cpu_oracle_baseline(HEADLINE, budget / 4, precision="f64")
+        line["cpu_baseline_fp64"] = {
+            "one_thread": {k: c64[k] for k in ("value", "unit", "cores", "sample")},
+            "all_cores": cpu_oracle_baseline_parallel(HEADLINE, budget / 4, precision="f64")}
         if "prefill_b4_t4096" in line.get("workloads", {}):
             line["workloads"]["prefill_b4_t4096"]["cpu_baseline_all_cores"] = \
-                cpu_oracle_prefill_parallel(args.cpu_budget / 2)
+                cpu_oracle_prefill_parallel(budget / 3, precision="f32")
 
     if env["world"] > 1:
         barrier()
@@ -1049,11 +1122,28 @@ def run_ours(args) -> int:
 def _step_extra(r, steps, peaks):
     per = r["seconds"] / steps
     gbs = r["bytes"] / per / 1e9
-    return {"ms_per_launch": per * 1e3, "state_gb_s": r["state_bytes"] / per / 1e9,
+    return {"ms_per_launch": per * 1e3, "state_gb_s": state_gb_s(r["units"], per),
             "layer_tokens_per_s": r["layer_tokens"] / per, "gb_s": gbs,
             "roofline": {"bound": "hbm", "peak": peaks["hbm_gbs"], "unit": "GB/s",
                          "frac": gbs / peaks["hbm_gbs"]},
             "l2": f"rotating {r['n_sets']} input sets"}
+
+
+def launcher_command(argv: List[str], n_gpus: int, port: int) -> List[str]:
+    """torchrun command that starts one rank of this script per GPU."""
+    return [sys.executable, "-m", "torch.distributed.run", "--nnodes=1",
+            f"--nproc-per-node={n_gpus}", "--master-addr", "127.0.0.1",
+            "--master-port", str(port), os.path.abspath(__file__), *argv]
+
+
+def world_mismatch(gpus: int, environ) -> Optional[str]:
+    """Why `--gpus` and the launcher's WORLD_SIZE disagree, or None."""
+    world = int(environ.get("WORLD_SIZE", 1))
+    if world != gpus:
+        return (f"--gpus {gpus} but this process is one of WORLD_SIZE={world} ranks: run "
+                f"`bench.py --gpus N` without a launcher (it starts N ranks itself) or "
+                f"under torchrun with --nproc-per-node N")
+    return None
 
 
 def main(argv=None) -> int:
@@ -1073,6 +1163,20 @@ def main(argv=None) -> int:
     args = ap.parse_args(argv)
     if args.profile_case:
         return run_profile_case(args.profile_case, args.launches)
+    if args.gpus < 1:
+        ap.error("--gpus must be at least 1")
+    if args.gpus > 1 and "WORLD_SIZE" not in os.environ:
+        # not under a launcher: one rank per GPU, started here
+        import socket
+        import subprocess
+        with socket.socket() as sk:
+            sk.bind(("127.0.0.1", 0))
+            port = sk.getsockname()[1]
+        argv = sys.argv[1:] if argv is None else list(argv)
+        return subprocess.call(launcher_command(argv, args.gpus, port))
+    why = world_mismatch(args.gpus, os.environ)
+    if why:
+        ap.error(why)
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")
     if args.impl == "reference":
