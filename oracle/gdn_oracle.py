@@ -41,6 +41,31 @@ class OracleError(RuntimeError):
     pass
 
 
+def _chunks(units: Optional[Sequence[int]], total: int, threads: int):
+    """The listed units (all when None) split into `threads` contiguous
+    lists for parallel calls; each chunk is written by one call only."""
+    arr = np.arange(total, dtype=np.int64) if units is None else \
+        np.ascontiguousarray(np.asarray(units, dtype=np.int64))
+    return [np.ascontiguousarray(c) for c in np.array_split(arr, max(1, threads)) if c.size]
+
+
+def _run_split(fn, units, total: int, threads: int, what: str) -> None:
+    """Call `fn(units_ptr, n_units)` over disjoint unit lists, from `threads`
+    host threads at once (ctypes releases the GIL during each call). The C
+    entry points write only the state, outputs and rings of the units they
+    are given, so the calls touch disjoint memory."""
+    if threads <= 1:
+        up, nu, _keep = _units(units)
+        _check(fn(up, nu), what)
+        return
+    from concurrent.futures import ThreadPoolExecutor
+    parts = _chunks(units, total, threads)
+    with ThreadPoolExecutor(len(parts)) as ex:
+        rcs = list(ex.map(lambda c: fn(c.ctypes.data_as(_PI), int(c.size)), parts))
+    for rc in rcs:
+        _check(rc, what)
+
+
 def _check(rc: int, what: str) -> None:
     if rc == -1:
         raise OracleError(f"{what}: bad argument")
@@ -95,12 +120,13 @@ class Oracle:
         self.lib = lib
 
     # -- recurrence ---------------------------------------------------------
-    def step(self, state, q, k, v, beta, gate, units=None):
+    def step(self, state, q, k, v, beta, gate, units=None, threads=1):
         """One token for every (layer, sequence, value head) unit.
 
         Shapes: state [L,B,Hv,dv,dk]; q, k [L,B,Hk,dk]; v [L,B,Hv,dv];
         beta, gate [L,B,Hv]. Returns (new_state, out [L,B,Hv,dv]); units that
-        are not listed keep their state and get zero output.
+        are not listed keep their state and get zero output. `threads` > 1
+        splits the units over that many host threads (same results).
         """
         st = _f64(state)
         L, B, Hv, dv, dk = st.shape
@@ -109,14 +135,15 @@ class Oracle:
         assert qq.shape == (L, B, Hk, dk) and kk.shape == qq.shape
         assert vv.shape == (L, B, Hv, dv) and bb.shape == (L, B, Hv) and gg.shape == bb.shape
         out = np.zeros((L, B, Hv, dv), dtype=np.float64)
-        up, nu, _keep = _units(units)
-        rc = self.lib.oracle_gdn_step(_ptr(st), _ptr(qq), _ptr(kk), _ptr(vv), _ptr(bb),
-                                      _ptr(gg), _ptr(out), L, B, Hk, Hv, dk, dv, up, nu)
-        _check(rc, "oracle_gdn_step")
+        fn = lambda up, nu: self.lib.oracle_gdn_step(_ptr(st), _ptr(qq), _ptr(kk), _ptr(vv),
+                                                     _ptr(bb), _ptr(gg), _ptr(out),
+                                                     L, B, Hk, Hv, dk, dv, up, nu)
+        _run_split(fn, units, L * B * Hv, threads, "oracle_gdn_step")
         return st, out
 
-    def prefill(self, state, q, k, v, beta, gate, units=None):
-        """T positions in order, for every (sequence, value head) unit.
+    def prefill(self, state, q, k, v, beta, gate, units=None, threads=1):
+        """T positions in order, for every (sequence, value head) unit
+        (`threads` > 1: the units split over that many host threads).
 
         Shapes: state [B,Hv,dv,dk]; q, k [B,T,Hk,dk]; v [B,T,Hv,dv];
         beta, gate [B,T,Hv]. Returns (final_state, out [B,T,Hv,dv]).
@@ -128,10 +155,10 @@ class Oracle:
         assert qq.shape == (B, T, Hk, dk) and kk.shape == qq.shape
         assert vv.shape == (B, T, Hv, dv) and bb.shape == (B, T, Hv) and gg.shape == bb.shape
         out = np.zeros((B, T, Hv, dv), dtype=np.float64)
-        up, nu, _keep = _units(units)
-        rc = self.lib.oracle_gdn_prefill(_ptr(st), _ptr(qq), _ptr(kk), _ptr(vv), _ptr(bb),
-                                         _ptr(gg), _ptr(out), B, T, Hk, Hv, dk, dv, up, nu)
-        _check(rc, "oracle_gdn_prefill")
+        fn = lambda up, nu: self.lib.oracle_gdn_prefill(_ptr(st), _ptr(qq), _ptr(kk), _ptr(vv),
+                                                        _ptr(bb), _ptr(gg), _ptr(out),
+                                                        B, T, Hk, Hv, dk, dv, up, nu)
+        _run_split(fn, units, B * Hv, threads, "oracle_gdn_prefill")
         return st, out
 
     def pair(self, state, q, k, v, beta, gate, units=None):
@@ -194,7 +221,7 @@ class Oracle:
         return y
 
     def layer_decode(self, mixed_qkv, z, a, b, ring, conv_w, A_log, dt_bias, norm_w, state,
-                     *, Hk, l2_eps=1e-6, norm_eps=1e-6, seqs=None):
+                     *, Hk, l2_eps=1e-6, norm_eps=1e-6, seqs=None, threads=1):
         """Prestate -> recurrence -> gated RMSNorm tail, one token per sequence.
 
         Shapes: mixed_qkv [B,C]; z [B,Hv*dv]; a, b [B,Hv]; ring [B,K-1,C];
@@ -209,17 +236,16 @@ class Oracle:
         assert x.shape == (B, C) and C == 2 * Hk * dk + Hv * dv
         assert zz.shape == (B, Hv * dv) and rg.shape == (B, K - 1, C) and nw.shape == (dv,)
         out = np.zeros((B, Hv * dv))
-        sp, ns, _keep = _units(seqs)
-        rc = self.lib.oracle_gdn_layer_decode(_ptr(x), _ptr(zz), _ptr(aa), _ptr(bb), _ptr(rg),
-                                              _ptr(w), _ptr(al), _ptr(dt), _ptr(nw),
-                                              float(l2_eps), float(norm_eps), _ptr(st),
-                                              _ptr(out), B, Hk, Hv, dk, dv, K, sp, ns)
-        _check(rc, "oracle_gdn_layer_decode")
+        fn = lambda sp, ns: self.lib.oracle_gdn_layer_decode(
+            _ptr(x), _ptr(zz), _ptr(aa), _ptr(bb), _ptr(rg), _ptr(w), _ptr(al), _ptr(dt),
+            _ptr(nw), float(l2_eps), float(norm_eps), _ptr(st), _ptr(out),
+            B, Hk, Hv, dk, dv, K, sp, ns)
+        _run_split(fn, seqs, B, threads, "oracle_gdn_layer_decode")
         return out, rg, st
 
 
     def layer_pair(self, mixed_qkv, z, a, b, ring, conv_w, A_log, dt_bias, norm_w, state, *,
-                   Hk, l2_eps=1e-6, norm_eps=1e-6, seqs=None):
+                   Hk, l2_eps=1e-6, norm_eps=1e-6, seqs=None, threads=1):
         """Two positions per sequence: position 1 commits, position 2 is tentative.
 
         Shapes: mixed_qkv [B,2,C]; z [B,2,Hv*dv]; a, b [B,2,Hv]; ring [B,K-1,C];
@@ -238,12 +264,11 @@ class Oracle:
         out = np.zeros((B, 2, Hv * dv))
         srg = np.zeros_like(rg)
         sst = np.zeros_like(st)
-        sp, ns, _keep = _units(seqs)
-        rc = self.lib.oracle_gdn_layer_pair(_ptr(x), _ptr(zz), _ptr(aa), _ptr(bb), _ptr(rg),
-                                            _ptr(w), _ptr(al), _ptr(dt), _ptr(nw), float(l2_eps),
-                                            float(norm_eps), _ptr(st), _ptr(srg), _ptr(sst),
-                                            _ptr(out), B, Hk, Hv, dk, dv, K, sp, ns)
-        _check(rc, "oracle_gdn_layer_pair")
+        fn = lambda sp, ns: self.lib.oracle_gdn_layer_pair(
+            _ptr(x), _ptr(zz), _ptr(aa), _ptr(bb), _ptr(rg), _ptr(w), _ptr(al), _ptr(dt),
+            _ptr(nw), float(l2_eps), float(norm_eps), _ptr(st), _ptr(srg), _ptr(sst),
+            _ptr(out), B, Hk, Hv, dk, dv, K, sp, ns)
+        _run_split(fn, seqs, B, threads, "oracle_gdn_layer_pair")
         return out, rg, st, srg, sst
 
 
@@ -298,7 +323,7 @@ class Oracle:
         _check(rc, "oracle_kda_step")
         return st, out
 
-    def kda_prefill(self, state, q, k, v, beta, g, units=None):
+    def kda_prefill(self, state, q, k, v, beta, g, units=None, threads=1):
         """T KDA positions in order. Shapes: state [B,Hv,dv,dk]; q, k
         [B,T,Hk,dk]; v [B,T,Hv,dv]; beta [B,T,Hv]; g [B,T,Hv,dk].
         Returns (final_state, out [B,T,Hv,dv])."""
@@ -310,10 +335,10 @@ class Oracle:
         assert vv.shape == (B, T, Hv, dv) and bb.shape == (B, T, Hv)
         assert gg.shape == (B, T, Hv, dk)
         out = np.zeros((B, T, Hv, dv), dtype=np.float64)
-        up, nu, _keep = _units(units)
-        rc = self.lib.oracle_kda_prefill(_ptr(st), _ptr(qq), _ptr(kk), _ptr(vv), _ptr(bb),
-                                         _ptr(gg), _ptr(out), B, T, Hk, Hv, dk, dv, up, nu)
-        _check(rc, "oracle_kda_prefill")
+        fn = lambda up, nu: self.lib.oracle_kda_prefill(_ptr(st), _ptr(qq), _ptr(kk), _ptr(vv),
+                                                        _ptr(bb), _ptr(gg), _ptr(out),
+                                                        B, T, Hk, Hv, dk, dv, up, nu)
+        _run_split(fn, units, B * Hv, threads, "oracle_kda_prefill")
         return st, out
 
     # -- LFM2 short-convolution mixer ----------------------------------------
@@ -371,3 +396,65 @@ def load() -> Oracle:
     if _DEFAULT is None:
         _DEFAULT = Oracle()
     return _DEFAULT
+
+
+class OracleF32:
+    """The literal fp32 instantiation of the recurrence (``gdn_oracle_f32.c``):
+    decode and prefill with every value in float. Only the benchmark's CPU
+    baseline times it; parity is judged against the double oracle above."""
+
+    def __init__(self, so_path: Optional[str] = None):
+        if so_path is None:
+            so_path = _build.build_f32()
+        self.path = so_path
+        lib = ctypes.CDLL(os.path.abspath(so_path))
+        pf = ctypes.POINTER(ctypes.c_float)
+        for name in ("oracle_gdn_step_f32", "oracle_gdn_prefill_f32"):
+            fn = getattr(lib, name)
+            fn.restype = ctypes.c_int
+            fn.argtypes = [pf] * 7 + [_I64] * 6 + [_PI, _I64]
+        self.lib = lib
+        self._pf = pf
+
+    def ptr(self, a: np.ndarray):
+        assert a.dtype == np.float32 and a.flags.c_contiguous
+        return a.ctypes.data_as(self._pf)
+
+    def step(self, state, q, k, v, beta, gate, units=None):
+        """As Oracle.step, in float32 (returns float32 arrays)."""
+        f = lambda a: np.ascontiguousarray(np.asarray(a, dtype=np.float32)).copy()
+        st, qq, kk, vv, bb, gg = f(state), f(q), f(k), f(v), f(beta), f(gate)
+        L, B, Hv, dv, dk = st.shape
+        Hk = qq.shape[2]
+        out = np.zeros((L, B, Hv, dv), dtype=np.float32)
+        up, nu, _keep = _units(units)
+        rc = self.lib.oracle_gdn_step_f32(self.ptr(st), self.ptr(qq), self.ptr(kk), self.ptr(vv),
+                                          self.ptr(bb), self.ptr(gg), self.ptr(out),
+                                          L, B, Hk, Hv, dk, dv, up, nu)
+        _check(rc, "oracle_gdn_step_f32")
+        return st, out
+
+    def prefill(self, state, q, k, v, beta, gate, units=None):
+        """As Oracle.prefill, in float32 (returns float32 arrays)."""
+        f = lambda a: np.ascontiguousarray(np.asarray(a, dtype=np.float32)).copy()
+        st, qq, kk, vv, bb, gg = f(state), f(q), f(k), f(v), f(beta), f(gate)
+        B, Hv, dv, dk = st.shape
+        T, Hk = qq.shape[1], qq.shape[2]
+        out = np.zeros((B, T, Hv, dv), dtype=np.float32)
+        up, nu, _keep = _units(units)
+        rc = self.lib.oracle_gdn_prefill_f32(self.ptr(st), self.ptr(qq), self.ptr(kk),
+                                             self.ptr(vv), self.ptr(bb), self.ptr(gg),
+                                             self.ptr(out), B, T, Hk, Hv, dk, dv, up, nu)
+        _check(rc, "oracle_gdn_prefill_f32")
+        return st, out
+
+
+_DEFAULT_F32: Optional[OracleF32] = None
+
+
+def load_f32() -> OracleF32:
+    """The fp32 instantiation built from this directory's source."""
+    global _DEFAULT_F32
+    if _DEFAULT_F32 is None:
+        _DEFAULT_F32 = OracleF32()
+    return _DEFAULT_F32

@@ -1,5 +1,7 @@
 """gdn_layer_pair (two-position speculative verify) on the GPU against the
 fp64 oracle, through the C ABI."""
+import os
+
 import numpy as np
 import pytest
 import torch
@@ -101,9 +103,11 @@ def test_pair_accept_then_reject(o):
     assert_parity(t["conv_ring"].cpu().numpy(), ring_r, "second verify ring")
 
 
-def test_pair_full_workload_sampled(o):
-    """B = 256 sequences, two positions each; 6 sequences recomputed by the
-    oracle, both rings checked exactly everywhere."""
+def test_pair_full_workload_full_parity(o):
+    """B = 256 sequences, two positions each: both outputs, the committed and
+    scratch states and both rings of every sequence against the oracle (its
+    sequences split over the host cores); the rings also checked exactly
+    against the inputs they must hold."""
     d = pair_inputs(256, seed=941)
     t = to_dev(d)
     out, sring, sstate = run_pair(t, 16)
@@ -114,10 +118,12 @@ def test_pair_full_workload_sampled(o):
     assert np.array_equal(sr[:, 0], d["conv_ring"][:, 2])
     assert np.array_equal(sr[:, 1], d["mixed_qkv"][:, 0])
     assert np.array_equal(sr[:, 2], d["mixed_qkv"][:, 1])
-    seqs = [0, 5, 100, 128, 254, 255]
-    sub = {k: (v[seqs] if k not in ("conv_w", "A_log", "dt_bias", "norm_w") else v)
-           for k, v in d.items()}
-    out_r, _, st_r, _, sst_r = oracle_pair(o, sub, 16)
-    assert_parity(out[seqs].cpu().numpy(), out_r, "B256 pair out (sampled)")
-    assert_parity(t["state"][seqs].cpu().numpy(), st_r, "B256 committed (sampled)")
-    assert_parity(sstate[seqs].cpu().numpy(), sst_r, "B256 scratch (sampled)")
+    out_r, ring_r, st_r, sring_r, sst_r = o.layer_pair(
+        *(d[n] for n in ORDER), Hk=16, threads=max(1, len(os.sched_getaffinity(0))))
+    assert np.array_equal(ring.astype(np.float64), ring_r), "B256 committed ring"
+    assert np.array_equal(sr.astype(np.float64), sring_r), "B256 scratch ring"
+    assert_parity(out.cpu().numpy(), out_r, "B256 pair out")
+    st, sst = t["state"].cpu().numpy(), sstate.cpu().numpy()
+    for b0 in range(0, 256, 64):
+        assert_parity(st[b0:b0 + 64], st_r[b0:b0 + 64], f"B256 committed, sequences {b0}..")
+        assert_parity(sst[b0:b0 + 64], sst_r[b0:b0 + 64], f"B256 scratch, sequences {b0}..")
