@@ -72,10 +72,17 @@ typedef enum gdn_status {
 /* Static English text for a status code (never NULL). */
 const char *gdn_status_string(int status);
 
-/* Text describing the last failed call on this host thread ("" if none).
- * The pointer stays valid until the next call of this library on the same
- * thread. */
+/* Text describing the last failed call on this host thread ("" if none):
+ * any status, cleared by a call that succeeds. The pointer stays valid until
+ * the next call of this library on the same thread. */
 const char *gdn_last_error(void);
+
+/* Text of the last call on this host thread that returned GDN_ERR_CUDA ("" if
+ * none has): the CUDA runtime's name and description of the refused launch.
+ * Unlike gdn_last_error() it only changes when another call returns
+ * GDN_ERR_CUDA; argument errors and later successful calls leave it as it is.
+ * Thread-local; the pointer stays valid for the life of the thread. */
+const char *gdn_last_cuda_error(void);
 
 /*
  * gdn_step -- one decode token for L layers x B sequences x Hv value heads,
@@ -299,11 +306,18 @@ gdn_status gdn_forward_batch(const void *hidden, const void *w_qkv, const void *
  * those of gdn_forward_batch without `workspace` and `workspace_bytes`.
  *
  * The workspace is a 16 MiB array built into the library (held on every GPU
- * that loads the library until the process exits). B*T positions whose
- * gdn_forward_batch_workspace_size() exceeds 16 MiB (about 215 positions at
- * Hk = 16, Hv = 32, dk = dv = 128) are rejected with GDN_ERR_UNSUPPORTED and
- * a message; nothing is launched. The first call on a device looks up the
- * array's device address; make that call before any stream capture. Every
+ * that loads the library until the process exits). A call is accepted when
+ * gdn_forward_batch_workspace_size(B, T, ...) fits in 16 MiB: at Hk = 16,
+ * Hv = 32, dk = dv = 128 that is about 72.5 KiB per position plus 96 KiB per
+ * started 32-position tile of each sequence, so B = 1 with T <= 216, B = 67
+ * with T = 2, B = 97 with T = 1. Larger calls are rejected with
+ * GDN_ERR_UNSUPPORTED and a message; nothing is launched.
+ *
+ * The array's device address is looked up with cudaGetSymbolAddress in the
+ * current context and cached per device under the driver's ID of that
+ * context; the first call in a context (the first on a device, and the
+ * first after cudaDeviceReset or in another context the caller made
+ * current) does that lookup, so make it before any stream capture. Every
  * call uses the same array, so calls whose GPU work overlaps (other streams,
  * other host threads on the same device) race and must be ordered by the
  * caller. The library performs no allocation of any kind for this call.

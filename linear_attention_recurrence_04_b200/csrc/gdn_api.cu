@@ -18,6 +18,8 @@ namespace gdn {
 namespace {
 
 thread_local char g_last_error[512] = "";
+// The text of the last GDN_ERR_CUDA on this thread; kept until the next one.
+thread_local char g_last_cuda_error[512] = "";
 
 // An NVTX range over one entry point (named after it), so a timeline tool
 // shows each library call; free when no tool is attached.
@@ -33,6 +35,7 @@ gdn_status fail(gdn_status st, const char* fmt, ...) {
     va_start(ap, fmt);
     vsnprintf(g_last_error, sizeof(g_last_error), fmt, ap);
     va_end(ap);
+    if (st == GDN_ERR_CUDA) snprintf(g_last_cuda_error, sizeof(g_last_cuda_error), "%s", g_last_error);
     return st;
 }
 
@@ -100,6 +103,7 @@ gdn_status launched(cudaError_t err, const char* what) {
 
 int report_error(int status, const char* message) {
     snprintf(g_last_error, sizeof(g_last_error), "%s", message);
+    if (status == GDN_ERR_CUDA) snprintf(g_last_cuda_error, sizeof(g_last_cuda_error), "%s", message);
     return status;
 }
 
@@ -184,6 +188,8 @@ const char* gdn_status_string(int status) {
 }
 
 const char* gdn_last_error(void) { return g_last_error; }
+
+const char* gdn_last_cuda_error(void) { return g_last_cuda_error; }
 
 }  // extern "C"
 

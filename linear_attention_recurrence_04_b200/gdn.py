@@ -28,7 +28,7 @@ STATUS = {
 }
 
 # Every symbol that include/gdn.h declares.
-EXPORTS = ("gdn_status_string", "gdn_last_error", "gdn_step", "gdn_prefill", "gdn_pair",
+EXPORTS = ("gdn_status_string", "gdn_last_error", "gdn_last_cuda_error", "gdn_step", "gdn_prefill", "gdn_pair",
            "gdn_layer_decode",
            "gdn_layer_pair", "gdn_linear_bf16", "gdn_linear_bf16_split_k",
            "gdn_forward_batch_workspace_size",
@@ -68,6 +68,8 @@ def load_library(path: Optional[str] = None) -> ctypes.CDLL:
     lib.gdn_status_string.argtypes = [ctypes.c_int]
     lib.gdn_last_error.restype = ctypes.c_char_p
     lib.gdn_last_error.argtypes = []
+    lib.gdn_last_cuda_error.restype = ctypes.c_char_p
+    lib.gdn_last_cuda_error.argtypes = []
     lib.gdn_step.restype = ctypes.c_int
     lib.gdn_step.argtypes = [_VP] * 7 + [_I64] * 6 + [_VP]
     lib.gdn_prefill.restype = ctypes.c_int

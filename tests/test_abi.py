@@ -42,6 +42,18 @@ def test_library_exports_every_declared_symbol(lib):
         assert hasattr(lib, name)
 
 
+def test_last_cuda_error_keeps_only_cuda_failures(lib):
+    """gdn_last_cuda_error (the scope table's name for the CUDA error text)
+    is exported, starts empty and is not touched by argument errors, which
+    gdn_last_error reports instead."""
+    lib.gdn_last_cuda_error.restype = ctypes.c_char_p
+    before = lib.gdn_last_cuda_error()
+    assert before == b""
+    assert step_call(lib, dk=64) == UNSUP
+    assert b"dk=64" in lib.gdn_last_error()
+    assert lib.gdn_last_cuda_error() == before
+
+
 def test_status_strings(lib):
     for code in range(8):
         assert gdn.status_string(code)
