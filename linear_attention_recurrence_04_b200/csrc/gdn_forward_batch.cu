@@ -35,9 +35,11 @@ namespace {
 //    run in parallel in tiles of kConvTile; to convolve in place, the K-1 raw
 //    inputs before each tile are copied out first (conv_halo_kernel), then
 //    every (sequence, tile, channel) thread convolves its tile
-//    (conv_tile_kernel). The halo pass also forms the ring the call leaves
-//    behind (slot n_tiles), which the tile-0 thread of each channel writes
-//    after it has read the old ring -- the only thread that reads it.
+//    (conv_tile_kernel). Tile 0 reads its K-1 inputs from the old ring, so
+//    the halo holds n_tiles slots per sequence: slot j - 1 for tile j >= 1,
+//    and slot n_tiles - 1 (the inputs before position T) is also the ring the
+//    call leaves behind, which the tile-0 thread of each channel writes after
+//    it has read the old ring -- the only thread that reads it.
 constexpr int kConvTile = 32;
 
 // Both conv kernels move four adjacent channels per thread (16-byte
@@ -55,7 +57,7 @@ conv_halo_kernel(const float* __restrict__ act, const float* __restrict__ ring,
     const int j = blockIdx.y + 1;                        // tiles 1 .. n_tiles (n_tiles: the ring)
     const int64_t b = blockIdx.z;
     const int64_t end = j < n_tiles ? static_cast<int64_t>(j) * kConvTile : T;
-    float* dst = halo + ((b * (n_tiles + 1) + j) * (kConvK - 1)) * C + c;
+    float* dst = halo + ((b * n_tiles + (j - 1)) * (kConvK - 1)) * C + c;
 #pragma unroll
     for (int i = 0; i < kConvK - 1; ++i) {
         const int64_t t = end - (kConvK - 1) + i;        // raw input position (slot i)
@@ -79,7 +81,7 @@ conv_tile_kernel(float* __restrict__ act, float* __restrict__ ring,
 #pragma unroll
     for (int q = 0; q < 4; ++q) w[q] = ld_ro4(conv_w + (c + q) * kConvK);
     const float* hs = j == 0 ? ring + b * (kConvK - 1) * C + c
-                             : halo + ((b * (n_tiles + 1) + j) * (kConvK - 1)) * C + c;
+                             : halo + ((b * n_tiles + (j - 1)) * (kConvK - 1)) * C + c;
     // raw inputs, oldest first, of the four channels
     float4 w0 = *reinterpret_cast<const float4*>(hs);
     float4 w1 = *reinterpret_cast<const float4*>(hs + C);
@@ -109,7 +111,7 @@ conv_tile_kernel(float* __restrict__ act, float* __restrict__ ring,
         }
     }
     if (j == 0) {            // the ring after the call (this thread read the old one above)
-        const float* nr = halo + ((b * (n_tiles + 1) + n_tiles) * (kConvK - 1)) * C + c;
+        const float* nr = halo + ((b * n_tiles + (n_tiles - 1)) * (kConvK - 1)) * C + c;
         float* rg = ring + b * (kConvK - 1) * C + c;
         const float4 r0 = *reinterpret_cast<const float4*>(nr);
         const float4 r1 = *reinterpret_cast<const float4*>(nr + C);
@@ -202,7 +204,7 @@ ForwardBatchLayout forward_batch_layout(int64_t B, int64_t T, int Hk, int Hv) {
     L.o = off;     off = align256(off + BT * HD * 4);
     L.y = off;     off = align256(off + BT * HD * 2);
     const int64_t n_tiles = (T + kConvTile - 1) / kConvTile;
-    L.halo = off;  off = align256(off + B * (n_tiles + 1) * (kConvK - 1) * C * 4);
+    L.halo = off;  off = align256(off + B * n_tiles * (kConvK - 1) * C * 4);
     L.total = off;
     return L;
 }
