@@ -499,6 +499,16 @@ def build_case(name: str, device):
         out = torch.empty_like(t["v"])
         return (lambda i: gdn.step(t["state"], t["q"], t["k"], t["v"], t["beta"], t["gate"],
                                    out)), dict(tensors=t)
+    if name == "decode_l1_b64_rotated":
+        # the benchmark's rotation: launch i uses input set i % n_sets, so a
+        # run of launches shows each one's DRAM traffic in steady state (the
+        # write-backs a launch leaves in L2 are paid by the ones after it)
+        r = bench_step_workload("decode_l1_b64", 0, 0, device)
+        sets, outs = r["sets"], r["outs"]
+        return (lambda i: gdn.step(sets[i % len(sets)]["state"], sets[i % len(sets)]["q"],
+                                   sets[i % len(sets)]["k"], sets[i % len(sets)]["v"],
+                                   sets[i % len(sets)]["beta"], sets[i % len(sets)]["gate"],
+                                   outs[i % len(sets)])), dict(n_sets=len(sets))
     if name == "pair_l1_b64":
         # two input sets of 256 MiB of state each, so a launch's state rows
         # are not still in L2 from the one before
@@ -602,7 +612,8 @@ def build_case(name: str, device):
     raise KeyError(f"unknown case {name!r}")
 
 
-PROFILE_CASES = ("decode_l1_b1", "decode_l1_b64", "decode_l36_b16", "pair_l1_b64",
+PROFILE_CASES = ("decode_l1_b1", "decode_l1_b64", "decode_l1_b64_rotated", "decode_l36_b16",
+                 "pair_l1_b64",
                  "prefill_b4_t4096", "layer_decode_b256", "layer_pair_b256", "forward_batch_b4_t4096",
                  "linear_bf16_m16384_n8192_k2048", "short_conv_decode_b64", "short_conv_pair_b64",
                  "short_conv_batch_b4_t4096", "kda_decode_b64", "kda_prefill_b4_t4096")

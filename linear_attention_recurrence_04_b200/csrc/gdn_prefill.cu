@@ -36,7 +36,11 @@
 //    W.q_t and the next position's key dot W.k_{t+1} (both read the same
 //    updated row), and the 4-lane reductions of out_t and sk_{t+1} run as one
 //    batch at the top of the next iteration. The dependency chain per
-//    position is then: reduce -> scalar delta -> one fused pass.
+//    position is then: reduce -> scalar delta -> one fused pass. With the
+//    scalar decay the next key read by pass t stays in registers as pass
+//    t + 1's update vector, so each position reads two staged vectors (its q
+//    and the next k) instead of three: the pass is bound by register-operand
+//    bandwidth and shared-memory delivery to the lanes, not by the chain.
 //  * Algebra in place of step 1 (same result up to rounding): head h's state
 //    is held as s * W with a per-head scalar s, so the decay is s *= e (one
 //    multiply per head, not per element). With W held:
@@ -73,6 +77,13 @@
 #ifndef GDN_PREFILL_GDN_LPR
 #define GDN_PREFILL_GDN_LPR 4      // scalar decay: lanes per state row (4 or 8)
 #endif
+#ifndef GDN_PREFILL_GDN_RPL
+#define GDN_PREFILL_GDN_RPL 1      // scalar decay: state rows per lane (2 needs 8 lanes per row)
+#endif
+#ifndef GDN_PREFILL_KREUSE
+#define GDN_PREFILL_KREUSE 1       // scalar decay: the next key read by a pass is kept in
+                                   // registers as the following pass's update vector
+#endif
 #ifndef GDN_PREFILL_FMA2
 #define GDN_PREFILL_FMA2 1         // packed f32x2 FMAs for the per-element work
 #endif
@@ -86,7 +97,10 @@
 #define GDN_PREFILL_MBAR 1         // scalar decay: stage handoff through mbarriers, no block barrier
 #endif
 #ifndef GDN_PREFILL_UNROLL
-#define GDN_PREFILL_UNROLL 8       // positions per unrolled block of a stage
+#define GDN_PREFILL_UNROLL 4       // scalar decay: positions per unrolled block of a stage
+#endif
+#ifndef GDN_PREFILL_KDA_UNROLL
+#define GDN_PREFILL_KDA_UNROLL 8   // per-channel decay: positions per unrolled block
 #endif
 
 namespace gdn {
@@ -99,7 +113,8 @@ namespace {
 constexpr int kTS = GDN_PREFILL_TS;             // positions per stage (scalar decay)
 constexpr int kTSChannel = 8;                   // positions per stage (per-channel decay)
 constexpr int kStages = GDN_PREFILL_STAGES;
-constexpr int kUnroll = GDN_PREFILL_UNROLL;        // positions per unrolled block
+template <bool kCh>
+constexpr int unroll_for() { return kCh ? GDN_PREFILL_KDA_UNROLL : GDN_PREFILL_UNROLL; }
 constexpr int kMaxGroups = 2;                   // groups one CTA's run can touch
 constexpr int kMaxRows = 64;                    // rows of one group a CTA holds at most
 constexpr float kScaleLo = 0x1p-40f;
@@ -115,7 +130,7 @@ static_assert(kStages >= 2, "at least double buffering");
 template <bool kCh>
 struct Layout {
     static constexpr int LPR = kCh ? 8 : GDN_PREFILL_GDN_LPR;   // lanes sharing a state row
-    static constexpr int RPL = kCh ? 2 : 1;                     // state rows per lane
+    static constexpr int RPL = kCh ? 2 : GDN_PREFILL_GDN_RPL;   // state rows per lane
     static constexpr int Chunks = kDk / 4 / LPR;                // float4 chunks per lane and row
     static constexpr int RowsPerUnit = 32 / LPR * RPL;          // rows of a head per warp
     static constexpr int UnitsPerHead = kDv / RowsPerUnit;
@@ -128,6 +143,11 @@ struct Layout {
     // broadcast, rather than a full reduction of each on every lane.
     static constexpr bool Halving = kCh || LPR == 8;
     static_assert(LPR == 4 || LPR == 8, "4 or 8 lanes per row");
+    static_assert(Halving || RPL == 1, "two rows per lane use the halving reduction");
+    // The key of position t + 1, read by pass t for the next key dot, is the
+    // update vector of pass t + 1: kept in registers, it is read from shared
+    // memory once instead of twice.
+    static constexpr bool KReuse = !kCh && GDN_PREFILL_KREUSE;
     static_assert(MaxWarps <= UnitsPerHead, "a run must span at most two groups");
 };
 
@@ -537,6 +557,8 @@ prefill_kernel(float* __restrict__ state, const float* __restrict__ q,
         s_out[n] = 1.0f;
     }
     bool out_pending = false;
+    constexpr bool kKReuse = Layout<kCh>::KReuse;
+    float4 kreg[kKReuse ? kChunks : 1];      // kKReuse: this lane's chunks of the coming key
 
     // One stage's positions for a warp with rows (the stage has landed).
     auto stage_body = [&](int64_t s) {
@@ -595,6 +617,7 @@ prefill_kernel(float* __restrict__ state, const float* __restrict__ q,
                 for (int n = 0; n < NH; ++n) {
                     const float4 kv = kCh ? ld_s4(ks_s + n * kDk + kStep * i)
                                           : ld_s4(kq_s + kStep * i);
+                    if constexpr (kKReuse) kreg[i] = kv;
 #pragma unroll
                     for (int r = 0; r < kRPL; ++r) {
                         a_lo[n][r] = fma2(lo2(w[n][r][i]), lo2(kv), a_lo[n][r]);
@@ -609,7 +632,7 @@ prefill_kernel(float* __restrict__ state, const float* __restrict__ q,
         // (kd, qs, ks) as a fast stage.
         auto positions = [&](auto slow_tag) {
             constexpr bool kSlowPath = decltype(slow_tag)::value;
-#pragma unroll(kUnroll)
+#pragma unroll(unroll_for<kCh>())
             for (int tp = 0; tp < TS; ++tp) {
                 if (tp >= tp_end) break;
                 float cf[NH][kRPL];
@@ -739,10 +762,12 @@ prefill_kernel(float* __restrict__ state, const float* __restrict__ q,
                 for (int i = 0; i < kChunks; ++i) {
                     float4 kv_sh = make_float4(0.f, 0.f, 0.f, 0.f), qv_sh = kv_sh, nv_sh = kv_sh;
                     if constexpr (!kCh) {
-                        kv_sh = ld_s4(kp + kStep * i);
+                        if constexpr (kKReuse) kv_sh = kreg[i];
+                        else kv_sh = ld_s4(kp + kStep * i);
                         qv_sh = ld_s4(kp + kDk + kStep * i);
                     }
                     if constexpr (!kCh) nv_sh = ld_s4(kp + kqP + kStep * i);
+                    if constexpr (kKReuse) kreg[i] = nv_sh;
 #pragma unroll
                     for (int n = 0; n < NH; ++n) {
                         float4 uv = kv_sh, qv = qv_sh, nv = nv_sh, al = kv_sh;
