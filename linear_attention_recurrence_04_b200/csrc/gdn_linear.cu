@@ -307,6 +307,18 @@ linear_bf16_kernel(const __grid_constant__ CUtensorMap tmap_x,
 // window -- the ring before position 0, u after -- exactly as the mixer's
 // gate kernel does (window sum and output gate in double, y rounded to bf16
 // once) and writes y and both rings.
+// Gate mode: the ring entries and conv taps of the CTA's channels are read
+// into shared memory past the stage ring while the main loop runs (they do not
+// depend on the product), so the conv walk after the reduction reads no
+// global memory. Used when the CTA's share fits kRingCache bytes.
+constexpr size_t kRingCache = 16384;
+constexpr size_t kTapCache = 32 * 4 * 4;          // at most 32 channels x 4 taps
+
+template <int BN, int kGate>
+constexpr size_t split_smem_bytes() {
+    return LinearSmem<BN, kMmaM>::kDynamic + (kGate ? kRingCache + kTapCache : 0);
+}
+
 struct GateEpi {
     float* ring;            // [B][K-1][D]
     float* scratch_ring;    // [B][K-1][D] or null
@@ -351,6 +363,17 @@ linear_bf16_splitk_kernel(const __grid_constant__ CUtensorMap tmap_x,
     const int n_kt = (K + kBK - 1) / kBK;
     const int kb = static_cast<int>(static_cast<int64_t>(rank) * n_kt / splits);
     const int ke = static_cast<int>(static_cast<int64_t>(rank + 1) * n_kt / splits);
+    // gate mode: this CTA's channel quads [q_lo, q_lo + nq) of the tile, and
+    // the shared-memory copies of their ring entries and taps (past the ring)
+    constexpr int KT = kGate > 0 ? kGate : 2;
+    const int q_lo = rank * 16 / splits;
+    const int nq = (rank + 1) * 16 / splits - q_lo;      // at most 8
+    const int nch = 4 * nq;
+    const bool ring_cached =
+        kGate > 0 && static_cast<size_t>(ge.B) * (KT - 1) * nch * 4 <= kRingCache;
+    float* ring_c = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(part) +
+                                             static_cast<size_t>(kStages) * L::kStage);
+    float* taps_c = ring_c + kRingCache / 4;
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < kStages; ++s) {
@@ -436,8 +459,27 @@ linear_bf16_splitk_kernel(const __grid_constant__ CUtensorMap tmap_x,
         // ring is free for the partial tile
         if (ok) tc::mma_commit(tc::smem_u32(&acc_full));
     } else if (warp >= 2) {
-        // ---- park the partial tile: TMEM -> registers -> this CTA's ring ---
         tc::grid_dep_wait();
+        if (kGate > 0 && ring_cached) {
+            // ---- gate mode, while the MMAs run: the ring entries and taps of
+            //      this CTA's channels into shared memory (the ring was
+            //      written by earlier kernels on the stream: after the wait)
+            const int et = static_cast<int>(threadIdx.x) - 64;
+            const int n4 = ge.B * (KT - 1) * nq;
+            for (int it = et; it < n4; it += 32 * kEpilogueWarps) {
+                const int bt = it / nq;                        // b (K-1) + slot
+                const int ql = it - bt * nq;
+                const int d = n0 + 4 * (q_lo + ql);
+                if (d < ge.D)
+                    reinterpret_cast<float4*>(ring_c)[it] = *reinterpret_cast<const float4*>(
+                        ge.ring + static_cast<int64_t>(bt) * ge.D + d);
+            }
+            for (int it = et; it < nch * KT; it += 32 * kEpilogueWarps) {
+                const int d = n0 + 4 * q_lo + it / KT;
+                if (d < ge.D) taps_c[it] = ge.conv_w[static_cast<int64_t>(d) * KT + it % KT];
+            }
+        }
+        // ---- park the partial tile: TMEM -> registers -> this CTA's ring ---
         const int row = (warp & 3) * 32 + lane;            // TMEM lane quarter warp % 4
         if (!tc::mbar_wait(tc::smem_u32(&acc_full), 0) || *vfailed) {
             if (status) atomicOr(status, tc::kTimeoutEpilogue);
@@ -470,6 +512,11 @@ linear_bf16_splitk_kernel(const __grid_constant__ CUtensorMap tmap_x,
     __syncthreads();
     __syncwarp();
     tc::cluster_sync();
+    // every rank's partial tile, addressed through its mapped base (an offset
+    // into a peer's shared memory maps like the base)
+    uint32_t peer[8];
+#pragma unroll
+    for (int s = 0; s < 8; ++s) peer[s] = s < splits ? tc::map_shared_rank(base, s) : 0u;
     if constexpr (kGate == 0) {
         {
             const int units = M * kQuads;
@@ -486,10 +533,10 @@ linear_bf16_splitk_kernel(const __grid_constant__ CUtensorMap tmap_x,
                     const int row = u / kQuads;
                     const int c = (u - row * kQuads) * 4;
                     if (u >= hi || n0 + c >= N) continue;
-                    const uint32_t off = base + static_cast<uint32_t>((row * kPitch + c) * 4);
+                    const uint32_t off = static_cast<uint32_t>((row * kPitch + c) * 4);
     #pragma unroll
                     for (int s = 0; s < 8; ++s)
-                        if (s < splits) v[h][s] = tc::ld_cluster_f4(tc::map_shared_rank(off, s));
+                        if (s < splits) v[h][s] = tc::ld_cluster_f4(peer[s] + off);
                 }
     #pragma unroll
                 for (int h = 0; h < 2; ++h) {
@@ -523,10 +570,102 @@ linear_bf16_splitk_kernel(const __grid_constant__ CUtensorMap tmap_x,
         // no CTA leaves (releasing its shared memory) while a peer still reads it
         __syncwarp();
         tc::cluster_sync();
+    } else if (ge.T <= 2 && ring_cached) {
+        // ---- gate mode, calls of one or two positions (decode, verify): one
+        //      thread per (sequence, channel quad) sums bg, cg and xv over the
+        //      S partials (rank order), forms u = bg * xv, walks its four
+        //      channels' conv windows through the positions (the ring from the
+        //      shared copy) and writes y and both rings. The arithmetic, and so
+        //      every bit of y and the rings, is that of the general path below.
+#pragma unroll 1
+        for (int it = static_cast<int>(threadIdx.x); it < ge.B * nq; it += kThreads) {
+            const int b = it / nq;
+            const int ql = it - b * nq;
+            const int c = 4 * (q_lo + ql);
+            const int d = n0 + c;
+            if (d >= ge.D) continue;
+            double wt[4][KT];
+            float win[4][KT - 1], committed[4][KT - 1];
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+#pragma unroll
+                for (int tau = 0; tau < KT; ++tau) wt[j][tau] = taps_c[(4 * ql + j) * KT + tau];
+#pragma unroll
+                for (int i = 0; i < KT - 1; ++i)
+                    committed[j][i] = win[j][i] = ring_c[(b * (KT - 1) + i) * nch + 4 * ql + j];
+            }
+            for (int t = 0; t < ge.T; ++t) {
+                const int row = b * ge.T + t;
+                const uint32_t off = static_cast<uint32_t>((row * kPitch + c) * 4);
+                float4 v[3][8];
+#pragma unroll
+                for (int s2 = 0; s2 < 8; ++s2) {
+                    if (s2 < splits) {
+#pragma unroll
+                        for (int blk = 0; blk < 3; ++blk)
+                            v[blk][s2] = tc::ld_cluster_f4(peer[s2] + off + blk * 64 * 4);
+                    }
+                }
+                float4 t3[3];
+#pragma unroll
+                for (int blk = 0; blk < 3; ++blk) {
+                    t3[blk] = v[blk][0];
+#pragma unroll
+                    for (int s2 = 1; s2 < 8; ++s2) {
+                        if (s2 < splits) {
+                            t3[blk].x = __fadd_rn(t3[blk].x, v[blk][s2].x);
+                            t3[blk].y = __fadd_rn(t3[blk].y, v[blk][s2].y);
+                            t3[blk].z = __fadd_rn(t3[blk].z, v[blk][s2].z);
+                            t3[blk].w = __fadd_rn(t3[blk].w, v[blk][s2].w);
+                        }
+                    }
+                }
+                const float uu[4] = {__fmul_rn(t3[0].x, t3[2].x), __fmul_rn(t3[0].y, t3[2].y),
+                                     __fmul_rn(t3[0].z, t3[2].z), __fmul_rn(t3[0].w, t3[2].w)};
+                const float cgv[4] = {t3[1].x, t3[1].y, t3[1].z, t3[1].w};
+                __nv_bfloat16 yv[4];
+#pragma unroll
+                for (int j = 0; j < 4; ++j) {
+                    double conv = 0.0;
+#pragma unroll
+                    for (int tau = 0; tau < KT - 1; ++tau)
+                        conv = fma(wt[j][tau], static_cast<double>(win[j][tau]), conv);
+                    conv = fma(wt[j][KT - 1], static_cast<double>(uu[j]), conv);
+                    yv[j] = __double2bfloat16(static_cast<double>(cgv[j]) * conv);
+#pragma unroll
+                    for (int tau = 0; tau < KT - 2; ++tau) win[j][tau] = win[j][tau + 1];
+                    win[j][KT - 2] = uu[j];
+                    if (t == ge.n_commit - 1) {
+#pragma unroll
+                        for (int tau = 0; tau < KT - 1; ++tau) committed[j][tau] = win[j][tau];
+                    }
+                }
+                uint2 packed;
+                packed.x = static_cast<uint32_t>(__bfloat16_as_ushort(yv[0])) |
+                           (static_cast<uint32_t>(__bfloat16_as_ushort(yv[1])) << 16);
+                packed.y = static_cast<uint32_t>(__bfloat16_as_ushort(yv[2])) |
+                           (static_cast<uint32_t>(__bfloat16_as_ushort(yv[3])) << 16);
+                *reinterpret_cast<uint2*>(ge.y + static_cast<int64_t>(row) * ge.D + d) = packed;
+            }
+            float* rg = ge.ring + static_cast<int64_t>(b) * (KT - 1) * ge.D + d;
+#pragma unroll
+            for (int tau = 0; tau < KT - 1; ++tau)
+                *reinterpret_cast<float4*>(rg + static_cast<int64_t>(tau) * ge.D) =
+                    make_float4(committed[0][tau], committed[1][tau], committed[2][tau],
+                                committed[3][tau]);
+            if (ge.scratch_ring) {
+                float* sg = ge.scratch_ring + static_cast<int64_t>(b) * (KT - 1) * ge.D + d;
+#pragma unroll
+                for (int tau = 0; tau < KT - 1; ++tau)
+                    *reinterpret_cast<float4*>(sg + static_cast<int64_t>(tau) * ge.D) =
+                        make_float4(win[0][tau], win[1][tau], win[2][tau], win[3][tau]);
+            }
+        }
+        // no CTA leaves (releasing its shared memory) while a peer still reads it
+        __syncwarp();
+        tc::cluster_sync();
     } else {
         // ---- gate mode: u = bg * xv and cg for this CTA's channel quads ----
-        const int q_lo = rank * 16 / splits;
-        const int nq = (rank + 1) * 16 / splits - q_lo;      // at most 8
         float4* u_s = reinterpret_cast<float4*>(reinterpret_cast<uint8_t*>(part) + kGateOff);
         float4* cg_s = u_s + kMmaM * 8;
 #pragma unroll 1
@@ -535,14 +674,14 @@ linear_bf16_splitk_kernel(const __grid_constant__ CUtensorMap tmap_x,
             const int ql = it - row * nq;
             const int c = 4 * (q_lo + ql);
             if (n0 + c >= ge.D) continue;
-            const uint32_t off = base + static_cast<uint32_t>((row * kPitch + c) * 4);
+            const uint32_t off = static_cast<uint32_t>((row * kPitch + c) * 4);
             float4 v[3][8];
 #pragma unroll
             for (int s2 = 0; s2 < 8; ++s2) {
                 if (s2 < splits) {
 #pragma unroll
                     for (int blk = 0; blk < 3; ++blk)
-                        v[blk][s2] = tc::ld_cluster_f4(tc::map_shared_rank(off + blk * 64 * 4, s2));
+                        v[blk][s2] = tc::ld_cluster_f4(peer[s2] + off + blk * 64 * 4);
                 }
             }
             float4 t3[3];
@@ -568,25 +707,26 @@ linear_bf16_splitk_kernel(const __grid_constant__ CUtensorMap tmap_x,
         __syncwarp();
         tc::cluster_sync();
         // ---- the conv walk: one thread per (sequence, channel) -------------
-        constexpr int KT = kGate > 0 ? kGate : 2;
-        const int nch = 4 * nq;
-#pragma unroll 1
-        for (int it = static_cast<int>(threadIdx.x); it < ge.B * nch; it += kThreads) {
+        // (two items per pass, so that the two independent chains of shared
+        // loads, double-precision window sums and stores overlap)
+        auto walk = [&](int it) {
             const int b = it / nch;
             const int cl = it - b * nch;
             const int d = n0 + 4 * q_lo + cl;
-            if (d >= ge.D) continue;
+            if (d >= ge.D) return;
             const float* u_f = reinterpret_cast<const float*>(u_s) + (cl >> 2) * 4 + (cl & 3);
             const float* cg_f = reinterpret_cast<const float*>(cg_s) + (cl >> 2) * 4 + (cl & 3);
             double wt[KT];
 #pragma unroll
             for (int tau = 0; tau < KT; ++tau)
-                wt[tau] = ge.conv_w[static_cast<int64_t>(d) * KT + tau];
+                wt[tau] = ring_cached ? taps_c[cl * KT + tau]
+                                      : ge.conv_w[static_cast<int64_t>(d) * KT + tau];
             float* rg = ge.ring + static_cast<int64_t>(b) * (KT - 1) * ge.D + d;
             float win[KT - 1], committed[KT - 1];
 #pragma unroll
-            for (int i = 0; i < KT - 1; ++i) committed[i] = win[i] = rg[static_cast<int64_t>(i) * ge.D];
-#pragma unroll 1
+            for (int i = 0; i < KT - 1; ++i)
+                committed[i] = win[i] = ring_cached ? ring_c[(b * (KT - 1) + i) * nch + cl]
+                                                    : rg[static_cast<int64_t>(i) * ge.D];
             for (int t = 0; t < ge.T; ++t) {
                 const int row = b * ge.T + t;
                 const float u = u_f[row * 32];
@@ -612,6 +752,12 @@ linear_bf16_splitk_kernel(const __grid_constant__ CUtensorMap tmap_x,
 #pragma unroll
                 for (int tau = 0; tau < KT - 1; ++tau) sg[static_cast<int64_t>(tau) * ge.D] = win[tau];
             }
+        };
+        const int n_items = ge.B * nch;
+#pragma unroll 1
+        for (int it = static_cast<int>(threadIdx.x); it < n_items; it += 2 * kThreads) {
+            walk(it);
+            if (it + kThreads < n_items) walk(it + kThreads);
         }
     }
 
@@ -898,18 +1044,18 @@ template <int BN, int kGate = 0>
 cudaError_t set_split_smem() {
     return cudaFuncSetAttribute(linear_bf16_splitk_kernel<BN, kGate>,
                                 cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                static_cast<int>(LinearSmem<BN, kMmaM>::kDynamic));
+                                static_cast<int>(split_smem_bytes<BN, kGate>()));
 }
 
 // Cluster of `splits` CTAs along x, and (`pdl`) programmatic serialization
 // so the prologue overlaps the previous kernel; attr holds two entries.
-template <int BN>
+template <int BN, int kGate = 0>
 cudaLaunchConfig_t split_config(unsigned grid, int splits, cudaStream_t stream,
                                 cudaLaunchAttribute* attr, bool pdl) {
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(grid);
     cfg.blockDim = dim3(kThreads);
-    cfg.dynamicSmemBytes = LinearSmem<BN, kMmaM>::kDynamic;
+    cfg.dynamicSmemBytes = split_smem_bytes<BN, kGate>();
     cfg.stream = stream;
     attr[0].id = cudaLaunchAttributeClusterDimension;
     attr[0].val.clusterDim.x = static_cast<unsigned>(splits);
@@ -936,8 +1082,8 @@ int max_active_clusters(int splits) {
     }
     int n = 0;
     cudaLaunchAttribute attr[2];
-    const cudaLaunchConfig_t cfg = split_config<BN>(static_cast<unsigned>(splits), splits,
-                                                    nullptr, attr, false);
+    const cudaLaunchConfig_t cfg = split_config<BN, kGate>(static_cast<unsigned>(splits),
+                                                           splits, nullptr, attr, false);
     if (set_split_smem<BN, kGate>() != cudaSuccess ||
         cudaOccupancyMaxActiveClusters(&n, linear_bf16_splitk_kernel<BN, kGate>, &cfg) !=
             cudaSuccess) {
@@ -1078,8 +1224,8 @@ cudaError_t launch_gate_k(const ShortConvArgs& a, void* y, cudaStream_t stream) 
     cudaError_t err = set_split_smem<192, KT>();
     if (err != cudaSuccess) return err;
     cudaLaunchAttribute attr[2];
-    const cudaLaunchConfig_t cfg = split_config<192>(static_cast<unsigned>(tiles * s),
-                                                     static_cast<int>(s), stream, attr, true);
+    const cudaLaunchConfig_t cfg = split_config<192, KT>(static_cast<unsigned>(tiles * s),
+                                                         static_cast<int>(s), stream, attr, true);
     GateEpi ge;
     ge.ring = a.conv_ring;
     ge.scratch_ring = a.scratch_ring;
