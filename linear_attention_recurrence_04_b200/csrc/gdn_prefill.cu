@@ -53,18 +53,16 @@
 //    end, so the stored state has its ordinary meaning.
 //  * KDA ("Module linear_core", entry "kda_forward_batch"; the published Kimi
 //    Delta Attention update) is the same pipeline with a log-decay per key
-//    channel, g [B][T][Hv][dk]. Its running scale is per state column: column
-//    i of a head is held as W[.][i] with M[.][i] = S[i] W[.][i], so the decay
-//    is S *= alpha_t (per column, once per CTA and position, not per
-//    element), and with ks = S k, kd = k / S, qs = S q:
-//       sk = W.ks,  delta = (v - sk) beta,  W += delta kd,  out = W.qs,
-//    three FMAs per element and position as above. Each stage of 8 positions
-//    is converted in shared memory (convert_stage) from its staged g into
-//    ks, kd and qs. Where S times a stage's product of decays would leave
-//    [2^-40, 2^40], S is folded into W at the stage's start; where that
-//    product alone leaves the range (an underflowing decay, strong growth),
-//    the stage applies alpha element by element instead:
-//    W *= alpha_t, W += delta k_t, o += W q_t, a += W (alpha_{t+1} k_{t+1}).
+//    channel, g [B][T][Hv][dk], applied element by element as step 1 reads:
+//    the registers hold D = alpha_t (.) M_{t-1}, the state already decayed
+//    for the coming position, and pass t runs
+//       M = D + delta_t k_t,  o += M.q_t,  D = alpha_{t+1} (.) M,  a += D.k_{t+1},
+//    four packed operations per element pair and position. k and q are
+//    shared by the two value heads of a warp and k_t is kept in registers
+//    from the previous pass, so each position reads q_t, k_{t+1} and each
+//    head's alpha_{t+1} from shared memory. The loader warp turns each
+//    staged g into alpha = exp(g) once its copies have landed (alpha = 1 past
+//    the last position, so the final registers hold M_{T-1}).
 #include <type_traits>
 
 #include "gdn_common.cuh"
@@ -100,7 +98,7 @@
 #define GDN_PREFILL_UNROLL 4       // scalar decay: positions per unrolled block of a stage
 #endif
 #ifndef GDN_PREFILL_KDA_UNROLL
-#define GDN_PREFILL_KDA_UNROLL 8   // per-channel decay: positions per unrolled block
+#define GDN_PREFILL_KDA_UNROLL 4   // per-channel decay: positions per unrolled block
 #endif
 
 namespace gdn {
@@ -111,22 +109,34 @@ namespace {
 #define GDN_PREFILL_TS 32          // positions per stage (scalar decay)
 #endif
 constexpr int kTS = GDN_PREFILL_TS;             // positions per stage (scalar decay)
-constexpr int kTSChannel = 8;                   // positions per stage (per-channel decay)
+#ifndef GDN_PREFILL_KDA_TS
+#define GDN_PREFILL_KDA_TS 20      // positions per stage (per-channel decay)
+#endif
+#ifndef GDN_PREFILL_KDA_CONVERTER
+#define GDN_PREFILL_KDA_CONVERTER 1  // per-channel decay: a second warp shares the alpha conversion
+#endif
+#ifndef GDN_PREFILL_KDA_FASTEXP
+#define GDN_PREFILL_KDA_FASTEXP 0  // per-channel decay: alpha by the fast exponential intrinsic
+#endif
+#ifndef GDN_PREFILL_KDA_STAGES
+#define GDN_PREFILL_KDA_STAGES 2   // stages in flight (per-channel decay)
+#endif
+constexpr int kTSChannel = GDN_PREFILL_KDA_TS;  // positions per stage (per-channel decay)
 constexpr int kStages = GDN_PREFILL_STAGES;
 template <bool kCh>
 constexpr int unroll_for() { return kCh ? GDN_PREFILL_KDA_UNROLL : GDN_PREFILL_UNROLL; }
 constexpr int kMaxGroups = 2;                   // groups one CTA's run can touch
 constexpr int kMaxRows = 64;                    // rows of one group a CTA holds at most
-constexpr float kScaleLo = 0x1p-40f;
+constexpr float kScaleLo = 0x1p-40f;           // scalar decay: fold-back bounds of the scale
 constexpr float kScaleHi = 0x1p40f;
 static_assert(kStages >= 2, "at least double buffering");
 
 // Lane layout of a warp's 8 rows. Scalar decay: 4 lanes per row and one row
 // per lane, 32 columns each. Per-channel decay: 8 lanes per row group and two
 // rows per lane, 16 columns each, so that every staged vector value a lane
-// loads serves two rows; that kernel reads three vectors per head and is
-// bound by shared-memory wavefronts (a 16-byte load is served a quarter warp
-// per wavefront, whatever its broadcast).
+// loads serves two rows of each head; that kernel reads a decay vector per
+// head besides q and k, and a 16-byte shared load is served a quarter warp
+// per wavefront, whatever its broadcast.
 template <bool kCh>
 struct Layout {
     static constexpr int LPR = kCh ? 8 : GDN_PREFILL_GDN_LPR;   // lanes sharing a state row
@@ -134,11 +144,17 @@ struct Layout {
     static constexpr int Chunks = kDk / 4 / LPR;                // float4 chunks per lane and row
     static constexpr int RowsPerUnit = 32 / LPR * RPL;          // rows of a head per warp
     static constexpr int UnitsPerHead = kDv / RowsPerUnit;
-    // Scalar decay with GDN_PREFILL_LOADER_WARP: one more warp, the CTA's
-    // last, issues every stage copy; the block stays at 8 warps.
-    static constexpr bool Loader = !kCh && GDN_PREFILL_LOADER_WARP;
+    // One more warp, the CTA's last, issues every stage copy. Per-channel
+    // decay: it then turns the landed stage's g into alpha, it and a
+    // converter warp (the one before it) taking half each; the alpha
+    // conversion sits between a stage's copies landing and its release, so
+    // halving it shortens the loader's path (build option
+    // GDN_PREFILL_KDA_CONVERTER=0: the loader alone).
+    static constexpr bool Loader = kCh || GDN_PREFILL_LOADER_WARP;
+    static constexpr bool Converter = kCh && GDN_PREFILL_KDA_CONVERTER;
+    static constexpr int Helpers = (Loader ? 1 : 0) + (Converter ? 1 : 0);   // warps without rows
     static constexpr int MaxWarps = kMaxRows / RowsPerUnit - (Loader ? 1 : 0);  // units per CTA
-    static constexpr int Threads = 32 * (MaxWarps + (Loader ? 1 : 0));
+    static constexpr int Threads = 32 * (MaxWarps + Helpers);
     // One halving reduction of all key and output dots with the deltas
     // broadcast, rather than a full reduction of each on every lane.
     static constexpr bool Halving = kCh || LPR == 8;
@@ -147,45 +163,30 @@ struct Layout {
     // The key of position t + 1, read by pass t for the next key dot, is the
     // update vector of pass t + 1: kept in registers, it is read from shared
     // memory once instead of twice.
-    static constexpr bool KReuse = !kCh && GDN_PREFILL_KREUSE;
+    static constexpr bool KReuse = kCh || GDN_PREFILL_KREUSE;
     static_assert(MaxWarps <= UnitsPerHead, "a run must span at most two groups");
 };
 
 // Shared-memory image of one stage. Slot TS of kq (k only) holds the first
 // position of the next stage, so a pass always reads the next key from its
-// own stage. kCh (per-channel decay) adds, per value head: ks, the key-dot
-// vectors (g as copied, then converted, with slot TS as well), kd and qs,
-// the update and output vectors, dec, the per-element decays a kSlow stage
-// applies, mult, the scales folded into the state when the stage starts, and
-// mode, one word per group (kFold | kSlow). Without kCh those are stubs.
+// own stage. kCh (per-channel decay) adds al, per value head and position the
+// decay alpha = exp(g) (g as copied, then converted in place), with slot TS
+// as well; without kCh it is a stub.
 template <int NH, bool kCh>
 struct alignas(16) Stage {    // stages sit back to back: each starts 16-byte aligned
     static constexpr int TS = kCh ? kTSChannel : kTS;   // positions per stage
     static constexpr int CG = kCh ? kMaxGroups : 1;
-    static constexpr int CT = kCh ? TS : 1;
+    static constexpr int CT = kCh ? TS : 0;
     static constexpr int CD = kCh ? kDk : 4;
     float kq[kMaxGroups][TS + 1][2][kDk];      // [group][pos][k|q][col]
     float v[kMaxGroups][TS][NH][kMaxRows];     // rows [row_lo, row_lo + rows) of the group
     float bg[kMaxGroups][TS][NH][2];           // beta, gate
-    float ks[CG][CT + 1][NH][CD];
-    float kd[CG][CT][NH][CD];
-    float qs[CG][CT][NH][CD];
-    float dec[CG][CT][NH][CD];
-    float mult[CG][NH][CD];
-    int mode[kMaxGroups];
+    float al[CG][CT + 1][NH][CD];              // kCh: alpha of positions t0 .. t0 + TS
 };
 
-// Per-channel stage modes, one word per group: some column folds its scale
-// into the state before the stage (kFold; every column's mult is written, 1
-// where it does not fold); some column's product of decays leaves
-// [kScaleLo, kScaleHi] within the stage, so the stage applies dec element by
-// element (kSlow, with that column folded).
-constexpr int kFold = 1;
-constexpr int kSlow = 2;
-
-// Stages in flight: the per-channel stages carry more per position, so two.
+// Stages in flight.
 template <bool kCh>
-constexpr int stages_for() { return kCh ? 2 : kStages; }
+constexpr int stages_for() { return kCh ? GDN_PREFILL_KDA_STAGES : kStages; }
 
 // One group of the CTA's run: (sequence b, key head g, head group grp) and the
 // rows of it that the run covers.
@@ -272,13 +273,17 @@ prefill_kernel(float* __restrict__ state, const float* __restrict__ q,
     extern __shared__ __align__(16) unsigned char smem_raw[];
     StageT* stages = reinterpret_cast<StageT*>(smem_raw);
     __shared__ Group grp_of[kMaxGroups];
-    // kCh: the running scale of each state column (see convert_stage)
-    __shared__ __align__(16) float s_col[kCh ? kMaxGroups : 1][NH][kCh ? kDk : 4];
-    // kPipe (scalar decay with a loader warp): stage s is full once the
-    // loader's copies of it have landed (one arrival per loader lane), and
-    // empty again once every warp with rows has finished it.
-    constexpr bool kPipe = !kCh && Layout<kCh>::Loader && GDN_PREFILL_MBAR;
+    // kPipe (a loader warp): stage s is full once the loader's copies of it
+    // have landed (and, kCh, its g has become alpha; one arrival per loader
+    // lane), and empty again once every warp with rows has finished it.
+    constexpr bool kPipe = Layout<kCh>::Loader && (kCh || GDN_PREFILL_MBAR);
+    static_assert(!kCh || kPipe, "the per-channel decay runs on the loader-warp pipeline");
+    constexpr bool kConverter = Layout<kCh>::Converter;
     __shared__ __align__(8) uint64_t pipe_full[kPipe ? S : 1], pipe_empty[kPipe ? S : 1];
+    // kCh: the loader's copies of stage s have landed (one arrival per loader
+    // lane); the loader and the converter then each convert half of it and
+    // arrive on pipe_full (one arrival per warp).
+    __shared__ __align__(8) uint64_t pipe_landed[kCh ? S : 1];
 
     const int tid = threadIdx.x;
     const int nthreads = blockDim.x;
@@ -309,13 +314,13 @@ prefill_kernel(float* __restrict__ state, const float* __restrict__ q,
         G.rows = static_cast<int>(last - first) * kRowsPerUnit;
         grp_of[tid] = G;
     }
-    if constexpr (kCh) {
-        for (int idx = tid; idx < kMaxGroups * NH * kDk; idx += nthreads) (&s_col[0][0][0])[idx] = 1.0f;
-    }
     if constexpr (kPipe) {
         if (tid == 0) {
             for (int i = 0; i < S; ++i) {
-                tc::mbar_init(tc::smem_u32(&pipe_full[i]), 32);
+                tc::mbar_init(tc::smem_u32(&pipe_full[i]), kCh ? (kConverter ? 2 : 1) : 32);
+                // kCh: each loader lane arrives twice, once with the bytes of
+                // its bulk copies and once when its 4-byte copies land
+                if (kCh) tc::mbar_init(tc::smem_u32(&pipe_landed[i]), 64);
                 tc::mbar_init(tc::smem_u32(&pipe_empty[i]), static_cast<uint32_t>(count));
             }
             tc::fence_mbar_init();
@@ -328,11 +333,76 @@ prefill_kernel(float* __restrict__ state, const float* __restrict__ q,
     // With a loader warp (the CTA's last warp), it alone issues the copies.
     constexpr bool kLoaderWarp = Layout<kCh>::Loader;
     const bool is_loader = kLoaderWarp && warp == static_cast<int>(blockDim.x >> 5) - 1;
+    const bool is_converter = kConverter && warp == static_cast<int>(blockDim.x >> 5) - 2;
     const int ltid = kLoaderWarp ? lane : tid;
     const int lstride = kLoaderWarp ? 32 : nthreads;
+    // kCh: the stage's rows (512-byte k, q and g rows, the v rows of the run)
+    // as bulk copies that complete on pipe_landed, beta as 4-byte copies;
+    // alpha slots past the last position get g = 0. The lane then arrives on
+    // pipe_landed twice (with the bytes of its bulk copies, and when its
+    // 4-byte copies have landed).
+    auto load_stage_bulk = [&](int64_t t0, StageT& st, uint32_t landed) {
+        uint32_t bytes = 0;
+        for (int gi = 0; gi < n_groups; ++gi) {
+            const Group G = grp_of[gi];
+            const int kq_items = 2 * TS + 1;              // k of t0 .. t0+TS, q of t0 .. t0+TS-1
+            const int g_items = (TS + 1) * NH;
+            const int v_items = TS * NH;
+            const int n_items = kq_items + g_items + v_items;
+            for (int it = lane; it < n_items; it += 32) {
+                const float* src = nullptr;
+                float* dst = nullptr;
+                uint32_t size = 0;
+                int64_t t = 0;
+                if (it < kq_items) {
+                    const int tp = it >> 1, which = it & 1;
+                    t = t0 + tp;
+                    src = (which ? q : k) + (G.b * T + t) * qk_stride + G.g * kDk;
+                    dst = &st.kq[gi][tp][which][0];
+                    size = kDk * 4;
+                } else if (it < kq_items + g_items) {
+                    const int j = it - kq_items;
+                    const int tp = j / NH, n = j - (j / NH) * NH;
+                    t = t0 + tp;
+                    const int h = G.g + (G.grp * NH + n) * Hk;
+                    src = gate + ((G.b * T + t) * Hv + h) * kDk;
+                    dst = &st.al[gi][tp][n][0];
+                    size = kDk * 4;
+                    if (t >= T) {                         // g = 0: alpha = 1 past the end
+                        float4* z = reinterpret_cast<float4*>(dst);
+                        for (int c4 = 0; c4 < kDk / 4; ++c4) z[c4] = make_float4(0.f, 0.f, 0.f, 0.f);
+                    }
+                } else {
+                    const int j = it - kq_items - g_items;
+                    const int tp = j / NH, n = j - (j / NH) * NH;
+                    t = t0 + tp;
+                    const int h = G.g + (G.grp * NH + n) * Hk;
+                    src = v + (G.b * T + t) * v_stride + h * kDv + G.row_lo;
+                    dst = &st.v[gi][tp][n][0];
+                    size = static_cast<uint32_t>(G.rows) * 4;
+                }
+                if (t < T) {
+                    asm volatile(
+                        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes "
+                        "[%0], [%1], %2, [%3];"
+                        ::"r"(tc::smem_u32(dst)), "l"(src), "r"(size), "r"(landed) : "memory");
+                    bytes += size;
+                }
+            }
+            for (int idx = lane; idx < TS * NH; idx += 32) {          // beta
+                const int n = idx % NH, tp = idx / NH;
+                const int64_t t = t0 + tp;
+                if (t < T) {
+                    const int h = G.g + (G.grp * NH + n) * Hk;
+                    cp_async4(&st.bg[gi][tp][n][0], beta + (G.b * T + t) * bg_stride + h);
+                }
+            }
+        }
+        tc::mbar_arrive_expect_tx(landed, bytes);
+        asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(landed) : "memory");
+    };
     auto load_stage = [&](int64_t t0, StageT& st) {
         if (kLoaderWarp && !is_loader) return;
-        if (kCh && tid < kMaxGroups) st.mode[tid] = 0;
 #pragma unroll
         for (int gi = 0; gi < kMaxGroups; ++gi) {
             if (gi >= n_groups) break;
@@ -382,94 +452,33 @@ prefill_kernel(float* __restrict__ state, const float* __restrict__ q,
                     const int n = (idx >> 5) % NH;
                     const int tp = (idx >> 5) / NH;
                     const int64_t t = t0 + tp;
-                    float* dst = &st.ks[gi][tp][n][chunk * 4];
+                    float* dst = &st.al[gi][tp][n][chunk * 4];
                     if (t < T) {
                         const int h = G.g + (G.grp * NH + n) * Hk;
                         cp_async16(dst, gate + ((G.b * T + t) * Hv + h) * kDk + chunk * 4);
-                    } else {
+                    } else {     // g = 0: alpha = 1 past the last position
                         *reinterpret_cast<float4*>(dst) = make_float4(0.f, 0.f, 0.f, 0.f);
                     }
                 }
             }
         }
     };
-    // kCh: turn a landed stage's g into the vectors of its passes. Column i
-    // of head n is held as W[j][i] with M[j][i] = S[i] W[j][i]; S (s_col)
-    // carries over between stages. Each column decides on its own, in one
-    // pass, so no barrier separates decision and vectors:
-    //  * a column whose S times the stage's product of decays stays within
-    //    [kScaleLo, kScaleHi] runs, per position t, S <- S alpha_t,
-    //    ks_t = S k_t, kd_t = k_t / S, qs_t = S q_t, dec_t = 1, so that
-    //    sk = W.ks_t, W += delta kd_t and out = W.qs_t (slot TS of ks: S alpha k
-    //    of the next stage's first position);
-    //  * a column whose S times that product leaves the range folds S into W
-    //    (mult = S) and runs as above from S = 1 (kFold);
-    //  * a column whose product alone leaves the range (an underflowing decay,
-    //    strong growth) folds and keeps S = 1: dec_t = alpha_t, kd_t = k_t,
-    //    qs_t = q_t, ks_t = alpha_t k_t, and a stage with such a column runs
-    //    its passes with the decay applied element by element (kSlow), which
-    //    the other columns' vectors (dec = 1) fit as well.
-    auto convert_stage = [&](StageT& st) {
+    // kCh: alpha = exp(g) in place, once the loader's copies of the stage have
+    // landed: half 0 by the loader warp, half 1 by the converter warp
+    auto alpha_stage = [&](StageT& st, int half) {
         if constexpr (kCh) {
-            // two adjacent columns per thread, with 8-byte shared accesses;
-            // each column decides on its own
-            auto f2 = [](float* ptr) -> float2& { return *reinterpret_cast<float2*>(ptr); };
-            const int npairs = n_groups * NH * (kDk / 2);
-            for (int pidx = tid; pidx < npairs; pidx += nthreads) {
-                const int col = (pidx % (kDk / 2)) * 2;
-                const int n = (pidx / (kDk / 2)) % NH;
-                const int gi2 = pidx / ((kDk / 2) * NH);
-                const float2 s0 = f2(&s_col[gi2][n][col]);
-                float2 cum = make_float2(1.0f, 1.0f);
-                bool slow0 = false, slow1 = false, fold0 = false, fold1 = false;
-#pragma unroll
-                for (int tp = 0; tp <= TS; ++tp) {
-                    const float2 g2 = f2(&st.ks[gi2][tp][n][col]);
-                    const float2 a = make_float2(expf(g2.x), expf(g2.y));
-                    f2(&st.ks[gi2][tp][n][col]) = a;
-                    if (tp < TS) {
-                        cum.x *= a.x;
-                        cum.y *= a.y;
-                        const float sx = s0.x * cum.x, sy = s0.y * cum.y;
-                        slow0 |= !(cum.x >= kScaleLo && cum.x <= kScaleHi);
-                        slow1 |= !(cum.y >= kScaleLo && cum.y <= kScaleHi);
-                        fold0 |= !(sx >= kScaleLo && sx <= kScaleHi);
-                        fold1 |= !(sy >= kScaleLo && sy <= kScaleHi);
-                    }
-                }
-                fold0 |= slow0;
-                fold1 |= slow1;
-                f2(&st.mult[gi2][n][col]) = make_float2(fold0 ? s0.x : 1.0f, fold1 ? s0.y : 1.0f);
-                float2 sv = make_float2(fold0 ? 1.0f : s0.x, fold1 ? 1.0f : s0.y);
-#pragma unroll
-                for (int tp = 0; tp < TS; ++tp) {
-                    const float2 a = f2(&st.ks[gi2][tp][n][col]);
-                    const float2 kv = f2(&st.kq[gi2][tp][0][col]);
-                    const float2 qv = f2(&st.kq[gi2][tp][1][col]);
-                    // fast column: S <- S alpha, ks = S k, kd = k / S, qs = S q, dec = 1;
-                    // slow column: S stays 1, ks = alpha k, kd = k, qs = q, dec = alpha
-                    if (!slow0) sv.x *= a.x;
-                    if (!slow1) sv.y *= a.y;
-                    f2(&st.ks[gi2][tp][n][col]) =
-                        make_float2((slow0 ? a.x : sv.x) * kv.x, (slow1 ? a.y : sv.y) * kv.y);
-                    f2(&st.kd[gi2][tp][n][col]) =
-                        make_float2(slow0 ? kv.x : kv.x * rcp_approx(sv.x),
-                                    slow1 ? kv.y : kv.y * rcp_approx(sv.y));
-                    f2(&st.qs[gi2][tp][n][col]) =
-                        make_float2(slow0 ? qv.x : sv.x * qv.x, slow1 ? qv.y : sv.y * qv.y);
-                    f2(&st.dec[gi2][tp][n][col]) =
-                        make_float2(slow0 ? a.x : 1.0f, slow1 ? a.y : 1.0f);
-                }
-                {   // slot TS: the key dot of the next stage's first position
-                    const float2 a = f2(&st.ks[gi2][TS][n][col]);
-                    const float2 kv = f2(&st.kq[gi2][TS][0][col]);
-                    f2(&st.ks[gi2][TS][n][col]) =
-                        make_float2((slow0 ? a.x : sv.x * a.x) * kv.x,
-                                    (slow1 ? a.y : sv.y * a.y) * kv.y);
-                }
-                f2(&s_col[gi2][n][col]) = sv;
-                if (fold0 || fold1)
-                    atomicOr(&st.mode[gi2], (slow0 || slow1) ? (kSlow | kFold) : kFold);
+            const int n4 = n_groups * (TS + 1) * NH * (kDk / 4);
+            const int lo = !kConverter ? 0 : half ? n4 / 2 : 0;
+            const int hi = !kConverter ? n4 : half ? n4 : n4 / 2;
+            float4* a4 = reinterpret_cast<float4*>(&st.al[0][0][0][0]);
+            for (int idx = lo + lane; idx < hi; idx += 32) {
+                float4 g4 = a4[idx];
+#if GDN_PREFILL_KDA_FASTEXP
+                g4.x = __expf(g4.x); g4.y = __expf(g4.y); g4.z = __expf(g4.z); g4.w = __expf(g4.w);
+#else
+                g4.x = expf(g4.x); g4.y = expf(g4.y); g4.z = expf(g4.z); g4.w = expf(g4.w);
+#endif
+                a4[idx] = g4;
             }
         }
     };
@@ -570,16 +579,13 @@ prefill_kernel(float* __restrict__ state, const float* __restrict__ q,
         constexpr int kqP = 2 * kDk;            // k and q of one position
         constexpr int vP = NH * kMaxRows;       // v of one position
         constexpr int bgP = 2 * NH;             // beta, gate of one position
-        constexpr int chP = NH * kDk;           // ks, kd or qs of one position
+        constexpr int alP = NH * kDk;           // kCh: alpha of one position
         constexpr int kStep = 4 * kLPR;         // columns between a lane's chunks
         const int ccol = kCh ? chunk_col<kLPR>(0, c) : 0;
         const float* kq_s = &st.kq[gi][0][0][chunk_col<kLPR>(0, c)];    // k; q at + kDk
         const float* v_s = &st.v[gi][0][0][0] + my_v_off;      // see my_v_off
         const float* bg_s = &st.bg[gi][0][0][0] + my_b_off;
-        const float* ks_s = &st.ks[gi * kCh][0][0][ccol];
-        const float* kd_s = &st.kd[gi * kCh][0][0][ccol];
-        const float* qs_s = &st.qs[gi * kCh][0][0][ccol];
-        const float* dec_s = &st.dec[gi * kCh][0][0][ccol];
+        const float* al_s = &st.al[gi * kCh][0][0][ccol];     // kCh only
 
         // decays of this stage: lane tp holds exp(gate) of position tp for
         // each head (stages of at most 32 positions)
@@ -589,35 +595,24 @@ prefill_kernel(float* __restrict__ state, const float* __restrict__ q,
         for (int n = 0; n < NH; ++n)
             e_lane[n] = (!kCh && lane < TS) ? expf(st.bg[gi][lane % TS][n][1]) : 1.0f;
 
-        int mode = 0;
-        if constexpr (kCh) {
-            mode = st.mode[gi];
-            if (mode & kFold) {             // M = S W per column: fold S into W
+        if (s == 0) {
+            // first key dot: a = W.k_0 (kCh: first the decay of position 0,
+            // D = alpha_0 (.) M, then a = D.k_0)
+#pragma unroll
+            for (int i = 0; i < kChunks; ++i) {
+                const float4 kv = ld_s4(kq_s + kStep * i);
+                if constexpr (kKReuse) kreg[i] = kv;
 #pragma unroll
                 for (int n = 0; n < NH; ++n) {
-#pragma unroll
-                    for (int i = 0; i < kChunks; ++i) {
-                        const float4 m = ld_s4(&st.mult[gi][n][ccol + kStep * i]);
+                    if constexpr (kCh) {
+                        const float4 al = ld_s4(al_s + n * kDk + kStep * i);
 #pragma unroll
                         for (int r = 0; r < kRPL; ++r) {
-                            const float2 l = mul2(lo2(w[n][r][i]), lo2(m));
-                            const float2 h = mul2(hi2(w[n][r][i]), hi2(m));
+                            const float2 l = mul2(lo2(w[n][r][i]), lo2(al));
+                            const float2 h = mul2(hi2(w[n][r][i]), hi2(al));
                             w[n][r][i] = make_float4(l.x, l.y, h.x, h.y);
                         }
                     }
-                }
-            }
-        }
-
-        if (s == 0) {
-            // first key dot: a = W.k_0 (kCh: W.ks_0, the decayed key)
-#pragma unroll
-            for (int i = 0; i < kChunks; ++i) {
-#pragma unroll
-                for (int n = 0; n < NH; ++n) {
-                    const float4 kv = kCh ? ld_s4(ks_s + n * kDk + kStep * i)
-                                          : ld_s4(kq_s + kStep * i);
-                    if constexpr (kKReuse) kreg[i] = kv;
 #pragma unroll
                     for (int r = 0; r < kRPL; ++r) {
                         a_lo[n][r] = fma2(lo2(w[n][r][i]), lo2(kv), a_lo[n][r]);
@@ -627,11 +622,8 @@ prefill_kernel(float* __restrict__ state, const float* __restrict__ q,
             }
         }
 
-        // The positions of the stage. kSlowPath (kCh only): decay element by
-        // element with dec, then the same update, output and next-key vectors
-        // (kd, qs, ks) as a fast stage.
-        auto positions = [&](auto slow_tag) {
-            constexpr bool kSlowPath = decltype(slow_tag)::value;
+        // The positions of the stage.
+        auto positions = [&]() {
 #pragma unroll(unroll_for<kCh>())
             for (int tp = 0; tp < TS; ++tp) {
                 if (tp >= tp_end) break;
@@ -707,7 +699,7 @@ prefill_kernel(float* __restrict__ state, const float* __restrict__ q,
                     // (b) this lane's pair's delta, then the broadcast
                     float cf_mine;
                     if constexpr (kCh) {
-                        // the key dot carries the column scales: tot is sk
+                        // the state is held unscaled: tot is sk
                         cf_mine = (v_s[tp * vP] - tot) * bg_s[tp * bgP];
                     } else {
                         // step 1 as a scale update s *= e (every lane keeps
@@ -755,51 +747,44 @@ prefill_kernel(float* __restrict__ state, const float* __restrict__ q,
                     }
                 }
                 // (c) one pass: step 4 for t, then W.q_t (step 5) and the next
-                // position's key dot. Slot tp + 1 always exists; past T it is
-                // zero-filled.
-                [[maybe_unused]] const float* kp = kq_s + tp * kqP;   // scalar decay only
+                // position's key dot; kCh: the next position's decay (step 1)
+                // between the two, D = alpha_{t+1} (.) M. Slot tp + 1 always
+                // exists (kCh: alpha = 1 past the last position).
+                const float* kp = kq_s + tp * kqP;
 #pragma unroll
                 for (int i = 0; i < kChunks; ++i) {
-                    float4 kv_sh = make_float4(0.f, 0.f, 0.f, 0.f), qv_sh = kv_sh, nv_sh = kv_sh;
-                    if constexpr (!kCh) {
-                        if constexpr (kKReuse) kv_sh = kreg[i];
-                        else kv_sh = ld_s4(kp + kStep * i);
-                        qv_sh = ld_s4(kp + kDk + kStep * i);
-                    }
-                    if constexpr (!kCh) nv_sh = ld_s4(kp + kqP + kStep * i);
-                    if constexpr (kKReuse) kreg[i] = nv_sh;
+                    float4 kv_sh;
+                    if constexpr (kKReuse) kv_sh = kreg[i];
+                    else kv_sh = ld_s4(kp + kStep * i);
+                    const float4 qv = ld_s4(kp + kDk + kStep * i);
+                    const float4 nv = ld_s4(kp + kqP + kStep * i);
+                    if constexpr (kKReuse) kreg[i] = nv;
 #pragma unroll
                     for (int n = 0; n < NH; ++n) {
-                        float4 uv = kv_sh, qv = qv_sh, nv = nv_sh, al = kv_sh;
-                        if constexpr (kCh) {
-                            const int off = tp * chP + n * kDk + kStep * i;
-                            nv = ld_s4(ks_s + off + chP);
-                            uv = ld_s4(kd_s + off);
-                            qv = ld_s4(qs_s + off);
-                            if constexpr (kSlowPath) al = ld_s4(dec_s + off);
-                        }
+                        [[maybe_unused]] float4 al;
+                        if constexpr (kCh) al = ld_s4(al_s + (tp + 1) * alP + n * kDk + kStep * i);
 #pragma unroll
                         for (int r = 0; r < kRPL; ++r) {
-                            float4 wv = w[n][r][i];
-                            if constexpr (kCh && kSlowPath) {
-                                const float2 dl = mul2(lo2(wv), lo2(al));
-                                const float2 dh = mul2(hi2(wv), hi2(al));
-                                wv = make_float4(dl.x, dl.y, dh.x, dh.y);
-                            }
+                            const float4 wv = w[n][r][i];
                             const float2 cf2 = make_float2(cf[n][r], cf[n][r]);
-                            const float2 lo = fma2(cf2, lo2(uv), lo2(wv));
-                            const float2 hi = fma2(cf2, hi2(uv), hi2(wv));
-                            w[n][r][i] = make_float4(lo.x, lo.y, hi.x, hi.y);
+                            const float2 lo = fma2(cf2, lo2(kv_sh), lo2(wv));
+                            const float2 hi = fma2(cf2, hi2(kv_sh), hi2(wv));
+                            float2 dlo = lo, dhi = hi;
+                            if constexpr (kCh) {
+                                dlo = mul2(lo, lo2(al));
+                                dhi = mul2(hi, hi2(al));
+                            }
+                            w[n][r][i] = make_float4(dlo.x, dlo.y, dhi.x, dhi.y);
                             if (i == 0) {
                                 o_lo[n][r] = mul2(lo, lo2(qv));
                                 o_hi[n][r] = mul2(hi, hi2(qv));
-                                a_lo[n][r] = mul2(lo, lo2(nv));
-                                a_hi[n][r] = mul2(hi, hi2(nv));
+                                a_lo[n][r] = mul2(dlo, lo2(nv));
+                                a_hi[n][r] = mul2(dhi, hi2(nv));
                             } else {
                                 o_lo[n][r] = fma2(lo, lo2(qv), o_lo[n][r]);
                                 o_hi[n][r] = fma2(hi, hi2(qv), o_hi[n][r]);
-                                a_lo[n][r] = fma2(lo, lo2(nv), a_lo[n][r]);
-                                a_hi[n][r] = fma2(hi, hi2(nv), a_hi[n][r]);
+                                a_lo[n][r] = fma2(dlo, lo2(nv), a_lo[n][r]);
+                                a_hi[n][r] = fma2(dhi, hi2(nv), a_hi[n][r]);
                             }
                         }
                     }
@@ -809,8 +794,7 @@ prefill_kernel(float* __restrict__ state, const float* __restrict__ q,
                 out_next += out_stride;
             }
         };
-        if (kCh && (mode & kSlow)) positions(std::true_type{});
-        else positions(std::false_type{});
+        positions();
     };
 
     if constexpr (kPipe) {
@@ -826,11 +810,44 @@ prefill_kernel(float* __restrict__ state, const float* __restrict__ q,
                     timed_out = true;
                     break;
                 }
-                load_stage(si * TS, stages[slot]);
-                asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];"
-                             ::"r"(tc::smem_u32(&pipe_full[slot])) : "memory");
+                if constexpr (kCh) {
+                    // the copies land on pipe_landed; then this warp converts
+                    // half 0 of the stage (all of it without a converter warp)
+                    // and publishes its part
+                    load_stage_bulk(si * TS, stages[slot], tc::smem_u32(&pipe_landed[slot]));
+                    __syncwarp();                  // the zero-filled alpha slots
+                    if (!tc::mbar_wait(tc::smem_u32(&pipe_landed[slot]),
+                                       static_cast<uint32_t>((si / S) & 1))) {
+                        // give the copies in flight one more bounded wait
+                        // before this CTA can leave
+                        tc::mbar_wait(tc::smem_u32(&pipe_landed[slot]),
+                                      static_cast<uint32_t>((si / S) & 1));
+                        timed_out = true;
+                        break;
+                    }
+                    alpha_stage(stages[slot], 0);
+                    __syncwarp();
+                    if (lane == 0) tc::mbar_arrive(tc::smem_u32(&pipe_full[slot]));
+                } else {
+                    load_stage(si * TS, stages[slot]);
+                    asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];"
+                                 ::"r"(tc::smem_u32(&pipe_full[slot])) : "memory");
+                }
             }
             asm volatile("cp.async.wait_all;" ::: "memory");   // nothing left in flight
+        } else if (is_converter) {
+            // kCh: half 1 of every stage, once its copies have landed
+            for (int64_t si = 0; si < n_stages; ++si) {
+                const int slot = static_cast<int>(si % S);
+                if (!tc::mbar_wait(tc::smem_u32(&pipe_landed[slot]),
+                                   static_cast<uint32_t>((si / S) & 1))) {
+                    timed_out = true;
+                    break;
+                }
+                alpha_stage(stages[slot], 1);
+                __syncwarp();
+                if (lane == 0) tc::mbar_arrive(tc::smem_u32(&pipe_full[slot]));
+            }
         } else if (active) {
             for (int64_t s = 0; s < n_stages; ++s) {
                 const int slot = static_cast<int>(s % S);
@@ -853,10 +870,6 @@ prefill_kernel(float* __restrict__ state, const float* __restrict__ q,
                 const int64_t nxt = s + S - 1;
                 if (nxt < n_stages) load_stage(nxt * TS, stages[nxt % S]);
                 cp_async_commit();
-            }
-            if constexpr (kCh) {
-                convert_stage(stages[s % S]);
-                __syncthreads();
             }
             if (!active) continue;
             stage_body(s);
@@ -893,7 +906,8 @@ prefill_kernel(float* __restrict__ state, const float* __restrict__ q,
                 if (my_store) *out_prev = so * tot * kOutScale;
             }
         }
-        // the final state, scale folded in (kCh: the column scales)
+        // the final state (scalar decay: with the scale folded in; kCh: the
+        // registers hold M_{T-1}, decayed by alpha = 1)
 #pragma unroll
         for (int n = 0; n < NH; ++n) {
 #pragma unroll
@@ -902,10 +916,7 @@ prefill_kernel(float* __restrict__ state, const float* __restrict__ q,
 #pragma unroll
                 for (int i = 0; i < kChunks; ++i) {
                     float4 x = w[n][r][i];
-                    if constexpr (kCh) {
-                        const float4 m = ld_s4(&s_col[gi][n][chunk_col<kLPR>(i, c)]);
-                        x.x *= m.x; x.y *= m.y; x.z *= m.z; x.w *= m.w;
-                    } else {
+                    if constexpr (!kCh) {
                         x.x *= sc[n]; x.y *= sc[n]; x.z *= sc[n]; x.w *= sc[n];
                     }
                     st_stream(row + chunk_col<kLPR>(i, c), x);
@@ -927,9 +938,7 @@ cudaError_t launch_nh(const PrefillArgs& a, cudaStream_t stream) {
     if (grid < min_grid) grid = min_grid;
     const int units_lo = static_cast<int>(n_units / grid);
     const int n_big = static_cast<int>(n_units % grid);
-    // Per-channel decay: every CTA runs L::MaxWarps warps (those past its run
-    // hold no rows) so that the per-stage conversion spreads evenly.
-    const int warps = kCh ? L::MaxWarps : units_lo + (n_big > 0 ? 1 : 0) + (L::Loader ? 1 : 0);
+    const int warps = units_lo + (n_big > 0 ? 1 : 0) + L::Helpers;
     const size_t smem = sizeof(Stage<NH, kCh>) * stages_for<kCh>();
     cudaError_t err = cudaFuncSetAttribute(prefill_kernel<NH, kCh>,
                                            cudaFuncAttributeMaxDynamicSharedMemorySize,
