@@ -97,6 +97,9 @@
 #ifndef GDN_PREFILL_UNROLL
 #define GDN_PREFILL_UNROLL 4       // scalar decay: positions per unrolled block of a stage
 #endif
+#ifndef GDN_PREFILL_BULK
+#define GDN_PREFILL_BULK 1         // scalar decay: the loader's rows as bulk copies
+#endif
 #ifndef GDN_PREFILL_KDA_UNROLL
 #define GDN_PREFILL_KDA_UNROLL 4   // per-channel decay: positions per unrolled block
 #endif
@@ -317,7 +320,8 @@ prefill_kernel(float* __restrict__ state, const float* __restrict__ q,
     if constexpr (kPipe) {
         if (tid == 0) {
             for (int i = 0; i < S; ++i) {
-                tc::mbar_init(tc::smem_u32(&pipe_full[i]), kCh ? (kConverter ? 2 : 1) : 32);
+                tc::mbar_init(tc::smem_u32(&pipe_full[i]),
+                              kCh ? (kConverter ? 2 : 1) : (GDN_PREFILL_BULK ? 64 : 32));
                 // kCh: each loader lane arrives twice, once with the bytes of
                 // its bulk copies and once when its 4-byte copies land
                 if (kCh) tc::mbar_init(tc::smem_u32(&pipe_landed[i]), 64);
@@ -336,17 +340,17 @@ prefill_kernel(float* __restrict__ state, const float* __restrict__ q,
     const bool is_converter = kConverter && warp == static_cast<int>(blockDim.x >> 5) - 2;
     const int ltid = kLoaderWarp ? lane : tid;
     const int lstride = kLoaderWarp ? 32 : nthreads;
-    // kCh: the stage's rows (512-byte k, q and g rows, the v rows of the run)
-    // as bulk copies that complete on pipe_landed, beta as 4-byte copies;
-    // alpha slots past the last position get g = 0. The lane then arrives on
-    // pipe_landed twice (with the bytes of its bulk copies, and when its
-    // 4-byte copies have landed).
+    // The stage's rows (512-byte k and q rows, kCh: g rows, the v rows of the
+    // run) as bulk copies that complete on `landed`, beta (and the scalar
+    // gate) as 4-byte copies; kCh: alpha slots past the last position get
+    // g = 0. The lane then arrives on `landed` twice (with the bytes of its
+    // bulk copies, and when its 4-byte copies have landed).
     auto load_stage_bulk = [&](int64_t t0, StageT& st, uint32_t landed) {
         uint32_t bytes = 0;
         for (int gi = 0; gi < n_groups; ++gi) {
             const Group G = grp_of[gi];
             const int kq_items = 2 * TS + 1;              // k of t0 .. t0+TS, q of t0 .. t0+TS-1
-            const int g_items = (TS + 1) * NH;
+            const int g_items = kCh ? (TS + 1) * NH : 0;
             const int v_items = TS * NH;
             const int n_items = kq_items + g_items + v_items;
             for (int it = lane; it < n_items; it += 32) {
@@ -389,12 +393,15 @@ prefill_kernel(float* __restrict__ state, const float* __restrict__ q,
                     bytes += size;
                 }
             }
-            for (int idx = lane; idx < TS * NH; idx += 32) {          // beta
-                const int n = idx % NH, tp = idx / NH;
+            constexpr int kScalars = kCh ? 1 : 2;                       // beta (, gate)
+            for (int idx = lane; idx < TS * NH * kScalars; idx += 32) {
+                const int which = idx % kScalars;
+                const int n = (idx / kScalars) % NH, tp = idx / (kScalars * NH);
                 const int64_t t = t0 + tp;
                 if (t < T) {
                     const int h = G.g + (G.grp * NH + n) * Hk;
-                    cp_async4(&st.bg[gi][tp][n][0], beta + (G.b * T + t) * bg_stride + h);
+                    cp_async4(&st.bg[gi][tp][n][which],
+                              (which ? gate : beta) + (G.b * T + t) * bg_stride + h);
                 }
             }
         }
@@ -828,6 +835,8 @@ prefill_kernel(float* __restrict__ state, const float* __restrict__ q,
                     alpha_stage(stages[slot], 0);
                     __syncwarp();
                     if (lane == 0) tc::mbar_arrive(tc::smem_u32(&pipe_full[slot]));
+                } else if constexpr (GDN_PREFILL_BULK != 0) {
+                    load_stage_bulk(si * TS, stages[slot], tc::smem_u32(&pipe_full[slot]));
                 } else {
                     load_stage(si * TS, stages[slot]);
                     asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];"
