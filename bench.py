@@ -619,6 +619,61 @@ PROFILE_CASES = ("decode_l1_b1", "decode_l1_b64", "decode_l1_b64_rotated", "deco
                  "short_conv_batch_b4_t4096", "kda_decode_b64", "kda_prefill_b4_t4096")
 
 
+CUBLAS_SHAPES = ((16384, 8192, 2048), (16384, 4096, 2048), (16384, 2048, 4096), (16384, 64, 2048),
+                 (8192, 8192, 8192), (64, 6144, 2048), (64, 2048, 2048))
+
+
+def run_cublas_compare(reps: int = 20) -> int:
+    """gdn_linear_bf16 (and, for at most 128 rows, its split-K form) against
+    cuBLAS (torch.mm with bf16 inputs and fp32 output) on the layer's
+    projection shapes, each graph-replayed `reps` times between CUDA events;
+    products of at most 128 rows rotate 16 weight sets (more than the L2).
+    Prints one JSON line per shape with both times and the largest absolute
+    difference of the two outputs."""
+    import torch
+    from linear_attention_recurrence_04_b200 import gdn
+    if not torch.cuda.is_available():
+        raise SystemExit("bench.py needs a CUDA device (there is no CPU path)")
+    dev = torch.device("cuda", 0)
+    gen = torch.Generator(device=dev).manual_seed(1011)
+
+    def timed(fn, n_sets):
+        for i in range(3):
+            fn(i % n_sets)
+        torch.cuda.synchronize()
+        g = capture([(lambda j=j: fn(j % n_sets)) for j in range(reps)], dev)
+        torch.cuda.synchronize()
+        a = torch.cuda.Event(enable_timing=True)
+        b = torch.cuda.Event(enable_timing=True)
+        a.record()
+        g.replay()
+        b.record()
+        torch.cuda.synchronize()
+        return a.elapsed_time(b) / reps * 1e3
+
+    for M, N, K in CUBLAS_SHAPES:
+        n_sets = 16 if M <= 128 else 1
+        x = torch.randn(M, K, device=dev, generator=gen).to(torch.bfloat16)
+        ws = [torch.randn(N, K, device=dev, generator=gen).mul(K ** -0.5).to(torch.bfloat16)
+              for _ in range(n_sets)]
+        y = torch.empty(M, N, device=dev, dtype=torch.float32)
+        yc = torch.empty_like(y)
+        line = {"M": M, "N": N, "K": K,
+                "gdn_linear_bf16_us": timed(lambda i: gdn.linear_bf16(x, ws[i], y), n_sets)}
+        if M <= 128:
+            line["gdn_linear_bf16_split_k_us"] = timed(
+                lambda i: gdn.linear_bf16(x, ws[i], y, split_k=True), n_sets)
+        line["cublas_us"] = timed(lambda i: torch.mm(x, ws[i].t(), out_dtype=torch.float32,
+                                                      out=yc), n_sets)
+        ours = min(line["gdn_linear_bf16_us"], line.get("gdn_linear_bf16_split_k_us", float("inf")))
+        line["ours_tflops"] = 2.0 * M * N * K / ours / 1e6
+        line["cublas_tflops"] = 2.0 * M * N * K / line["cublas_us"] / 1e6
+        line["ours_over_cublas_time"] = ours / line["cublas_us"]
+        line["max_abs_diff"] = float((y - yc).abs().max())
+        print(json.dumps(line), flush=True)
+    return 0
+
+
 def run_profile_case(name: str, launches: int) -> int:
     """Run `launches` calls of one case and exit (no timing): the program
     that ncu captures for the summaries kept with the sources."""
@@ -1169,11 +1224,15 @@ def main(argv=None) -> int:
     ap.add_argument("--profile-case", choices=PROFILE_CASES, default=None,
                     help="run --launches calls of one case without timing (for ncu) and exit")
     ap.add_argument("--launches", type=int, default=3)
+    ap.add_argument("--cublas-compare", action="store_true",
+                    help="time the projection kernels against cuBLAS on the layer's shapes and exit")
     ap.add_argument("--no-extras", action="store_true",
                     help="skip the other four workloads (headline only)")
     args = ap.parse_args(argv)
     if args.profile_case:
         return run_profile_case(args.profile_case, args.launches)
+    if args.cublas_compare:
+        return run_cublas_compare()
     if args.gpus < 1:
         ap.error("--gpus must be at least 1")
     if args.gpus > 1 and "WORLD_SIZE" not in os.environ:
