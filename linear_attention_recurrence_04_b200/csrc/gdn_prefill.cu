@@ -118,6 +118,10 @@ constexpr int kTS = GDN_PREFILL_TS;             // positions per stage (scalar d
 #ifndef GDN_PREFILL_KDA_CONVERTER
 #define GDN_PREFILL_KDA_CONVERTER 1  // per-channel decay: a second warp shares the alpha conversion
 #endif
+#ifndef GDN_PREFILL_KDA_LOADER_SHARE
+#define GDN_PREFILL_KDA_LOADER_SHARE 0  // per-channel decay: eighths of the alpha conversion
+                                        // the loader takes (the converter warp the rest)
+#endif
 #ifndef GDN_PREFILL_KDA_FASTEXP
 #define GDN_PREFILL_KDA_FASTEXP 0  // per-channel decay: alpha by the fast exponential intrinsic
 #endif
@@ -148,11 +152,13 @@ struct Layout {
     static constexpr int RowsPerUnit = 32 / LPR * RPL;          // rows of a head per warp
     static constexpr int UnitsPerHead = kDv / RowsPerUnit;
     // One more warp, the CTA's last, issues every stage copy. Per-channel
-    // decay: it then turns the landed stage's g into alpha, it and a
-    // converter warp (the one before it) taking half each; the alpha
-    // conversion sits between a stage's copies landing and its release, so
-    // halving it shortens the loader's path (build option
-    // GDN_PREFILL_KDA_CONVERTER=0: the loader alone).
+    // decay: a converter warp (the one before it) turns each landed stage's
+    // g into alpha. Warps issue on sub-partition warp % 4, so with 7 warps
+    // with rows the converter (warp 7) shares the sub-partition that holds
+    // only one of them, and the loader (warp 8, bulk copies only) one that
+    // holds two (build options: GDN_PREFILL_KDA_LOADER_SHARE, the eighths of
+    // the conversion the loader takes; GDN_PREFILL_KDA_CONVERTER=0, the
+    // loader alone).
     static constexpr bool Loader = kCh || GDN_PREFILL_LOADER_WARP;
     static constexpr bool Converter = kCh && GDN_PREFILL_KDA_CONVERTER;
     static constexpr int Helpers = (Loader ? 1 : 0) + (Converter ? 1 : 0);   // warps without rows
@@ -471,12 +477,13 @@ prefill_kernel(float* __restrict__ state, const float* __restrict__ q,
         }
     };
     // kCh: alpha = exp(g) in place, once the loader's copies of the stage have
-    // landed: half 0 by the loader warp, half 1 by the converter warp
+    // landed: part 0 by the loader warp, part 1 by the converter warp
     auto alpha_stage = [&](StageT& st, int half) {
         if constexpr (kCh) {
             const int n4 = n_groups * (TS + 1) * NH * (kDk / 4);
-            const int lo = !kConverter ? 0 : half ? n4 / 2 : 0;
-            const int hi = !kConverter ? n4 : half ? n4 : n4 / 2;
+            const int cut = n4 * GDN_PREFILL_KDA_LOADER_SHARE / 8;
+            const int lo = !kConverter ? 0 : half ? cut : 0;
+            const int hi = !kConverter ? n4 : half ? n4 : cut;
             float4* a4 = reinterpret_cast<float4*>(&st.al[0][0][0][0]);
             for (int idx = lo + lane; idx < hi; idx += 32) {
                 float4 g4 = a4[idx];
@@ -819,8 +826,8 @@ prefill_kernel(float* __restrict__ state, const float* __restrict__ q,
                 }
                 if constexpr (kCh) {
                     // the copies land on pipe_landed; then this warp converts
-                    // half 0 of the stage (all of it without a converter warp)
-                    // and publishes its part
+                    // its part of the stage (all of it without a converter
+                    // warp) and publishes it
                     load_stage_bulk(si * TS, stages[slot], tc::smem_u32(&pipe_landed[slot]));
                     __syncwarp();                  // the zero-filled alpha slots
                     if (!tc::mbar_wait(tc::smem_u32(&pipe_landed[slot]),
@@ -845,7 +852,7 @@ prefill_kernel(float* __restrict__ state, const float* __restrict__ q,
             }
             asm volatile("cp.async.wait_all;" ::: "memory");   // nothing left in flight
         } else if (is_converter) {
-            // kCh: half 1 of every stage, once its copies have landed
+            // kCh: the converter's part of every stage, once its copies have landed
             for (int64_t si = 0; si < n_stages; ++si) {
                 const int slot = static_cast<int>(si % S);
                 if (!tc::mbar_wait(tc::smem_u32(&pipe_landed[slot]),
