@@ -100,6 +100,12 @@
 #ifndef GDN_PREFILL_BULK
 #define GDN_PREFILL_BULK 1         // scalar decay: the loader's rows as bulk copies
 #endif
+#ifndef GDN_PREFILL_KDA_LPR
+#define GDN_PREFILL_KDA_LPR 8      // per-channel decay: lanes per state row (4 or 8)
+#endif
+#ifndef GDN_PREFILL_KDA_RPL
+#define GDN_PREFILL_KDA_RPL 2      // per-channel decay: state rows per lane (2 needs 8 lanes)
+#endif
 #ifndef GDN_PREFILL_KDA_UNROLL
 #define GDN_PREFILL_KDA_UNROLL 4   // per-channel decay: positions per unrolled block
 #endif
@@ -146,8 +152,8 @@ static_assert(kStages >= 2, "at least double buffering");
 // per wavefront, whatever its broadcast.
 template <bool kCh>
 struct Layout {
-    static constexpr int LPR = kCh ? 8 : GDN_PREFILL_GDN_LPR;   // lanes sharing a state row
-    static constexpr int RPL = kCh ? 2 : GDN_PREFILL_GDN_RPL;   // state rows per lane
+    static constexpr int LPR = kCh ? GDN_PREFILL_KDA_LPR : GDN_PREFILL_GDN_LPR;   // lanes per row
+    static constexpr int RPL = kCh ? GDN_PREFILL_KDA_RPL : GDN_PREFILL_GDN_RPL;   // rows per lane
     static constexpr int Chunks = kDk / 4 / LPR;                // float4 chunks per lane and row
     static constexpr int RowsPerUnit = 32 / LPR * RPL;          // rows of a head per warp
     static constexpr int UnitsPerHead = kDv / RowsPerUnit;
@@ -166,7 +172,7 @@ struct Layout {
     static constexpr int Threads = 32 * (MaxWarps + Helpers);
     // One halving reduction of all key and output dots with the deltas
     // broadcast, rather than a full reduction of each on every lane.
-    static constexpr bool Halving = kCh || LPR == 8;
+    static constexpr bool Halving = LPR == 8;
     static_assert(LPR == 4 || LPR == 8, "4 or 8 lanes per row");
     static_assert(Halving || RPL == 1, "two rows per lane use the halving reduction");
     // The key of position t + 1, read by pass t for the next key dot, is the
@@ -662,6 +668,11 @@ prefill_kernel(float* __restrict__ state, const float* __restrict__ q,
                             if (c == n) { ov = O[n]; so = s_out[n]; }
                         if (out_pending && my_store) *out_prev = so * ov * kOutScale;
                     }
+                    if constexpr (kCh) {     // the state is held unscaled: A is sk
+#pragma unroll
+                        for (int n = 0; n < NH; ++n)
+                            cf[n][0] = (v_s[tp * vP + n * kMaxRows] - A[n]) * bg_s[tp * bgP + 2 * n];
+                    } else {
                     // (b) step 1 as a scale update s *= e; then, with
                     // r = 1 / s, delta / s = (v r - W.k) beta (steps 2-3)
                     float s_new[NH];
@@ -691,6 +702,7 @@ prefill_kernel(float* __restrict__ state, const float* __restrict__ q,
                         s_out[n] = s_new[n];
                         cf[n][0] = fmaf(v_s[tp * vP + n * kMaxRows], rcp_approx(s_new[n]), -A[n]) *
                                    bg_s[tp * bgP + 2 * n];
+                    }
                     }
                 } else {
                     // (a) one halving reduction: sk of t and out of t-1 for
