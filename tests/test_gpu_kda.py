@@ -70,7 +70,8 @@ def test_kda_uniform_decay_equals_gdn_step():
 
 @pytest.mark.parametrize("B,T,Hk,Hv,std", [(2, 37, 16, 32, 0.05), (1, 16, 4, 4, 0.0),
                                            (3, 9, 2, 6, 0.05), (1, 1, 16, 32, 0.05),
-                                           (1, 49, 8, 8, 0.05)])
+                                           (1, 49, 8, 8, 0.05),
+                                           (10, 41, 16, 32, 0.05)])   # two waves of CTAs
 def test_kda_prefill_parity(o, B, T, Hk, Hv, std):
     d = inputs.kda_prefill_inputs(B, T, Hk=Hk, Hv=Hv, seed=1600 + T, state_std=std)
     st_ref, out_ref = o.kda_prefill(d["state"], d["q"], d["k"], d["v"], d["beta"], d["g"])

@@ -36,7 +36,8 @@ def run_gpu(d):
 
 @pytest.mark.parametrize("B,T,Hk,Hv,std", [(2, 37, 16, 32, 0.05), (1, 5, 4, 4, 0.05),
                                            (3, 9, 2, 6, 0.0), (1, 16, 2, 8, 0.05),
-                                           (1, 1, 16, 32, 0.05)])
+                                           (1, 1, 16, 32, 0.05),
+                                           (10, 70, 16, 32, 0.05)])   # two waves of CTAs
 def test_prefill_small_full_parity(o, B, T, Hk, Hv, std):
     d = inputs.prefill_inputs(B, T, Hk=Hk, Hv=Hv, seed=500 + B * 100 + T, state_std=std)
     st_ref, out_ref = o.prefill(d["state"], d["q"], d["k"], d["v"], d["beta"], d["gate"])
