@@ -377,7 +377,8 @@ gdn_status gdn_kda_prefill(float *state, const float *q, const float *k, const f
  *   out       [B][T][D] fp32
  *   workspace device scratch of gdn_short_conv_workspace_size(B, T, D) bytes,
  *             256-byte aligned, owned by the caller; contents on entry do
- *             not matter and are undefined afterwards
+ *             not matter and are undefined afterwards (its last 256 bytes
+ *             hold the one-kernel form's barrier word, below)
  *   status    optional zero-initialised device word for timeout bits (see
  *             gdn_linear_bf16)
  * All pointers are device pointers, 16-byte aligned. conv_ring is updated in
@@ -392,6 +393,18 @@ gdn_status gdn_kda_prefill(float *state, const float *q, const float *k, const f
  * (any chunking into calls, single positions, the verify). Between a call of
  * at most 128 rows and a larger one they differ by the fp32 rounding of the
  * projections' accumulation order.
+ *
+ * One-kernel form: calls of one or two positions (decode, verify) with D a
+ * multiple of 64 whose two projections take the same K split run the whole
+ * mixer as one kernel, with the same bits. Between the conv and the output
+ * projection its CTAs meet at a grid-wide barrier: a 64-bit word at offset
+ * workspace_size - 256 that the call tags with a number of its own (any
+ * earlier content is replaced; a CUDA graph replay finds and replaces its
+ * own completed count). The barrier needs every CTA of the grid resident at
+ * once (one per SM, at most 148): a kernel on another stream that holds SMs
+ * for longer than the 2 s wait limit makes the call time out, ORing 16 into
+ * `status` (the outputs are then undefined). Two calls that share a
+ * workspace must be ordered, as for any workspace.
  *
  * gdn_short_conv_forward_batch runs T positions in order; conv_ring ends as
  * the ring after position T-1 (T = 0 does nothing).

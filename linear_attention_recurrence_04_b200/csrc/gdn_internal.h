@@ -117,13 +117,19 @@ struct ShortConvArgs {
     uint32_t* status;
 };
 struct ShortConvLayout {
-    size_t proj, y, total;
+    size_t proj, y, bar, total;   // bar: the one-kernel form's barrier word
 };
 // Calls of at most 128 rows (B*T): the input projection, split over K in a
 // cluster, with the gate and conv as its epilogue -- y (bf16, [B*T][D]) and
 // both rings are written, proj is not. cudaErrorNotSupported when the call
 // is larger or the product too small to split (use the separate kernels).
 cudaError_t launch_short_conv_in_gate(const ShortConvArgs& a, void* y, cudaStream_t stream);
+// Calls of one or two positions and at most 128 rows: the whole mixer as one
+// kernel (both projections split as above, a grid-wide barrier on the word
+// `bar` of the workspace between the conv and the output projection).
+// cudaErrorNotSupported when the shape does not fit that form.
+cudaError_t launch_short_conv_fused(const ShortConvArgs& a, void* y, unsigned long long* bar,
+                                    cudaStream_t stream);
 ShortConvLayout short_conv_layout(int64_t B, int64_t T, int64_t D);
 
 // Each launcher enqueues its kernel on `stream` and returns the launch status.

@@ -45,8 +45,11 @@
 #include <cuda.h>
 #include <cuda_bf16.h>
 
+#include <unistd.h>
+
 #include <algorithm>
 #include <atomic>
+#include <chrono>
 
 #include "gdn_common.cuh"
 #include "gdn_internal.h"
@@ -56,6 +59,13 @@
 // 512 forces 256 x 256.
 #ifndef GDN_LINEAR_BN
 #define GDN_LINEAR_BN 0
+#endif
+// Split-K form: k-steps of each CTA's weight stripe prefetched into L2 before
+// the dependency wait (-1: all of them). The first two measured best: the
+// whole stripe of every CTA at once queues the first stages behind it
+// (short-conv decode 22.2 against 21.2 us).
+#ifndef GDN_SPLIT_PREFETCH
+#define GDN_SPLIT_PREFETCH 2
 #endif
 // 1: products with enough 256 x 256 tiles take the pair-CTA (cta_group::2) form.
 #ifndef GDN_LINEAR_PAIR
@@ -314,9 +324,32 @@ linear_bf16_kernel(const __grid_constant__ CUtensorMap tmap_x,
 constexpr size_t kRingCache = 16384;
 constexpr size_t kTapCache = 32 * 4 * 4;          // at most 32 channels x 4 taps
 
-template <int BN, int kGate>
+//
+// kFuse (gate mode, one or two positions, every channel tile's conv ring in
+// shared memory): the whole mixer in one kernel. The output projection
+// out = y W_out^T is split exactly as the split-K form splits it on its own
+// (64-column tiles, the same K chunks, the same rank-order reduction), so
+// its bits are those of the two-kernel path: CTA r of cluster c owns output
+// columns [64 c, 64 c + 64) and y channels of the k-steps it owned in the
+// input projection. Its W_out chunks stream into shared memory as soon as
+// the input projection's MMAs are done (into the freed stage ring and a
+// region past the ring cache), while the partials are reduced and the conv
+// walked. Every CTA's y (all channels of every sequence) is written before
+// any CTA reads it: after the walk one thread per CTA passes a grid-wide
+// barrier (a tagged counter in the caller's workspace, every wait bounded),
+// then loads the CTA's y chunks with TMA into the freed ring; the MMAs run
+// as each chunk lands, and the partial tiles are reduced over the cluster
+// like any split-K product and stored as out.
+constexpr int split_threads(bool fuse) { return fuse ? kThreads + 64 : kThreads; }
+constexpr uint32_t kWoChunk = 64 * kBK * 2;       // 64 W_out rows of one k-step
+constexpr int kFuseMaxSteps = 8;                  // k-steps per CTA the fused form holds
+// W_out chunks 4..7 past the caches, on a 1024-byte boundary (the swizzle atom)
+constexpr size_t kWoSpare = 4 * static_cast<size_t>(kWoChunk) + 1024;
+
+template <int BN, int kGate, bool kFuse = false>
 constexpr size_t split_smem_bytes() {
-    return LinearSmem<BN, kMmaM>::kDynamic + (kGate ? kRingCache + kTapCache : 0);
+    return LinearSmem<BN, kMmaM>::kDynamic + (kGate ? kRingCache + kTapCache : 0) +
+           (kFuse ? kWoSpare : 0);
 }
 
 struct GateEpi {
@@ -327,18 +360,35 @@ struct GateEpi {
     int B, T, D, n_commit;
 };
 
-template <int BN, int kGate>
-__global__ void __launch_bounds__(kThreads, 1)
+// The fused form's output projection: y as the A operand (128-row boxes of
+// 64 channels; rows past B*T read as zero), W_out as the B operand (64-row
+// boxes), out [B*T][D] fp32, the barrier word and this call's tag.
+struct alignas(64) FuseMaps {
+    CUtensorMap y;
+    CUtensorMap wo;
+};
+struct FuseOut {
+    float* out;
+    unsigned long long* bar;
+    uint64_t tag;
+};
+
+template <int BN, int kGate, bool kFuse = false>
+__global__ void __launch_bounds__(split_threads(kFuse), 1)
 linear_bf16_splitk_kernel(const __grid_constant__ CUtensorMap tmap_x,
                           const __grid_constant__ CUtensorMap tmap_w, float* __restrict__ y,
                           int M, int N, int K, int splits, uint32_t* __restrict__ status,
-                          GateEpi ge) {
+                          GateEpi ge, const __grid_constant__ FuseMaps fm, FuseOut fo) {
     using L = LinearSmem<BN, kMmaM>;
+    // the fused form has two more warps, for the walk and the reductions
+    constexpr int kThr = split_threads(kFuse);
     constexpr int kStages = L::kStages;
     constexpr int kPitch = BN + 4;        // floats per parked row: 16-byte shift per row
     constexpr int kQuads = BN / 4;        // float4 columns of a row
     constexpr uint32_t kTmemCols = BN <= 64 ? 64 : BN <= 128 ? 128 : 256;
     static_assert(kGate == 0 || BN == 192, "the gate tile is three 64-row blocks");
+    static_assert(!kFuse || (kGate > 0 && kStages * L::kStage >= 16 * 8192 + 4 * kWoChunk),
+                  "the fused form's y chunks and W_out chunks 0..3 fit the stage ring");
     // gate mode: u and cg of at most 8 channel quads per row after the parked tile
     constexpr size_t kGateOff = static_cast<size_t>(kMmaM) * kPitch * 4;
     constexpr size_t kGateBytes = kGate ? 2 * static_cast<size_t>(kMmaM) * 8 * 16 : 0;
@@ -348,9 +398,14 @@ linear_bf16_splitk_kernel(const __grid_constant__ CUtensorMap tmap_x,
     __shared__ __align__(8) uint64_t full[kStages];
     __shared__ __align__(8) uint64_t empty[kStages];
     __shared__ __align__(8) uint64_t acc_full;
+    // fused form: W_out chunks landed, each y chunk landed, output MMAs done
+    __shared__ __align__(8) uint64_t wo_full;
+    __shared__ __align__(8) uint64_t y_full[kFuseMaxSteps];
+    __shared__ __align__(8) uint64_t out_full;
     __shared__ uint32_t tmem_slot;
     __shared__ int issued, consumed;
     __shared__ int failed;
+    __shared__ int wo_issued, y_issued;
 
     const uint32_t raw = tc::smem_u32(smem_raw);
     const uint32_t base = (raw + 1023u) & ~1023u;
@@ -374,6 +429,15 @@ linear_bf16_splitk_kernel(const __grid_constant__ CUtensorMap tmap_x,
     float* ring_c = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(part) +
                                              static_cast<size_t>(kStages) * L::kStage);
     float* taps_c = ring_c + kRingCache / 4;
+    // fused form: y chunk g at base + g * 16 KB (after the grid barrier);
+    // W_out chunks 0..3 in the ring's last 32 KB, 4..7 past the caches
+    const uint32_t wo_lo = base + kFuseMaxSteps * L::kA;
+    const uint32_t wo_hi =
+        (base + static_cast<uint32_t>(kStages * L::kStage + kRingCache + kTapCache) + 1023u) &
+        ~1023u;
+    auto wo_addr = [&](int g) -> uint32_t {
+        return g < 4 ? wo_lo + g * kWoChunk : wo_hi + (g - 4) * kWoChunk;
+    };
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < kStages; ++s) {
@@ -381,10 +445,17 @@ linear_bf16_splitk_kernel(const __grid_constant__ CUtensorMap tmap_x,
             tc::mbar_init(tc::smem_u32(&empty[s]), 1);
         }
         tc::mbar_init(tc::smem_u32(&acc_full), 1);
+        if constexpr (kFuse) {
+            tc::mbar_init(tc::smem_u32(&wo_full), 1);
+            for (int j = 0; j < kFuseMaxSteps; ++j) tc::mbar_init(tc::smem_u32(&y_full[j]), 1);
+            tc::mbar_init(tc::smem_u32(&out_full), 1);
+        }
         tc::fence_mbar_init();
         issued = 0;
         consumed = 0;
         failed = 0;
+        wo_issued = 0;
+        y_issued = 0;
     }
     if (warp == 1) {
         tc::tmem_alloc(tc::smem_u32(&tmem_slot), kTmemCols);
@@ -401,7 +472,11 @@ linear_bf16_splitk_kernel(const __grid_constant__ CUtensorMap tmap_x,
         // ---- producer: this rank's k-steps through the stage ring ----------
         tc::prefetch_tmap(&tmap_x);
         tc::prefetch_tmap(&tmap_w);
-        for (int kt = kb; kt < ke; ++kt) {     // the weight stripe, into L2 early
+        // the rank's x boxes, then the weight stripe, into L2 early (x
+        // first: its few boxes would otherwise queue behind the stripe)
+        for (int kt = kb; kt < ke; ++kt) tc::tma_prefetch_l2_2d(&tmap_x, kt * kBK, 0);
+        const int pf_end = GDN_SPLIT_PREFETCH < 0 ? ke : min(ke, kb + GDN_SPLIT_PREFETCH);
+        for (int kt = kb; kt < pf_end; ++kt) {
             if constexpr (kGate) {
                 for (int blk = 0; blk < 3; ++blk)
                     tc::tma_prefetch_l2_2d(&tmap_w, kt * kBK, blk * ge.D + n0);
@@ -431,6 +506,25 @@ linear_bf16_splitk_kernel(const __grid_constant__ CUtensorMap tmap_x,
             }
             issued = g + 1;
         }
+        if constexpr (kFuse) {
+            // this call's tag into the barrier word (the previous kernel on
+            // the stream is complete, so no launch still polls it)
+            tc::grid_barrier_install(fo.bar, fo.tag, gridDim.x);
+            // the input projection's MMAs are done, so its stages are free:
+            // this CTA's W_out chunks (rows n0.., its k-steps), while the
+            // partials are parked and reduced
+            if (!*vfailed) {
+                if (!tc::mbar_wait(tc::smem_u32(&acc_full), 0)) {
+                    atomicExch(&failed, 1);
+                } else if (!*vfailed) {
+                    tc::mbar_arrive_expect_tx(tc::smem_u32(&wo_full),
+                                              static_cast<uint32_t>(ke - kb) * kWoChunk);
+                    for (int kt = kb, g = 0; kt < ke; ++kt, ++g)
+                        tc::tma_load_2d(wo_addr(g), &fm.wo, tc::smem_u32(&wo_full), kt * kBK, n0);
+                    wo_issued = 1;
+                }
+            }
+        }
     } else if (warp == 1 && lane == 0) {
         // ---- MMA issuer: one accumulator, the rank's k-steps in order ------
         tc::grid_dep_wait();
@@ -458,7 +552,7 @@ linear_bf16_splitk_kernel(const __grid_constant__ CUtensorMap tmap_x,
         // every MMA done (so every stage read and every copy landed): the
         // ring is free for the partial tile
         if (ok) tc::mma_commit(tc::smem_u32(&acc_full));
-    } else if (warp >= 2) {
+    } else if (warp >= 2 && warp < 2 + kEpilogueWarps) {
         tc::grid_dep_wait();
         if (kGate > 0 && ring_cached) {
             // ---- gate mode, while the MMAs run: the ring entries and taps of
@@ -487,15 +581,16 @@ linear_bf16_splitk_kernel(const __grid_constant__ CUtensorMap tmap_x,
         } else {
             tc::tc_fence_after();
             const uint32_t src = tmem + (static_cast<uint32_t>((warp & 3) * 32) << 16);
+            static_assert(BN % 64 == 0, "the partial is parked 64 columns at a time");
 #pragma unroll 1
-            for (int c0 = 0; c0 < BN; c0 += 32) {
-                uint32_t r[32];
-                tc::tmem_ld_32x32b_x32(src + c0, r);
+            for (int c0 = 0; c0 < BN; c0 += 64) {
+                uint32_t r[64];
+                tc::tmem_ld_32x32b_x64(src + c0, r);
                 tc::tmem_ld_wait();
                 if (row < M) {
                     float4* dst = reinterpret_cast<float4*>(part + row * kPitch + c0);
 #pragma unroll
-                    for (int j = 0; j < 8; ++j)
+                    for (int j = 0; j < 16; ++j)
                         dst[j] = make_float4(__uint_as_float(r[4 * j]), __uint_as_float(r[4 * j + 1]),
                                              __uint_as_float(r[4 * j + 2]),
                                              __uint_as_float(r[4 * j + 3]));
@@ -507,7 +602,8 @@ linear_bf16_splitk_kernel(const __grid_constant__ CUtensorMap tmap_x,
     // Every CTA's partial is parked; each sums its slice over the cluster.
     // (On a timeout the partials are stale: the output is then undefined and
     // the status word says so, but every CTA still meets both barriers.)
-    if (warp < 2 && lane != 0) tc::grid_dep_wait();   // they store below too
+    if ((warp < 2 && lane != 0) || warp >= 2 + kEpilogueWarps)
+        tc::grid_dep_wait();                           // they store below too
     tc::tc_fence_before();
     __syncthreads();
     __syncwarp();
@@ -525,11 +621,11 @@ linear_bf16_splitk_kernel(const __grid_constant__ CUtensorMap tmap_x,
             const bool vec = (N & 3) == 0;
             // two units per pass: all 2 S remote loads are in flight together
     #pragma unroll 1
-            for (int u0 = lo + static_cast<int>(threadIdx.x); u0 < hi; u0 += 2 * kThreads) {
+            for (int u0 = lo + static_cast<int>(threadIdx.x); u0 < hi; u0 += 2 * kThr) {
                 float4 v[2][8];
     #pragma unroll
                 for (int h = 0; h < 2; ++h) {
-                    const int u = u0 + h * kThreads;
+                    const int u = u0 + h * kThr;
                     const int row = u / kQuads;
                     const int c = (u - row * kQuads) * 4;
                     if (u >= hi || n0 + c >= N) continue;
@@ -540,7 +636,7 @@ linear_bf16_splitk_kernel(const __grid_constant__ CUtensorMap tmap_x,
                 }
     #pragma unroll
                 for (int h = 0; h < 2; ++h) {
-                    const int u = u0 + h * kThreads;
+                    const int u = u0 + h * kThr;
                     const int row = u / kQuads;
                     const int c = (u - row * kQuads) * 4;
                     const int col = n0 + c;
@@ -578,7 +674,7 @@ linear_bf16_splitk_kernel(const __grid_constant__ CUtensorMap tmap_x,
         //      shared copy) and writes y and both rings. The arithmetic, and so
         //      every bit of y and the rings, is that of the general path below.
 #pragma unroll 1
-        for (int it = static_cast<int>(threadIdx.x); it < ge.B * nq; it += kThreads) {
+        for (int it = static_cast<int>(threadIdx.x); it < ge.B * nq; it += kThr) {
             const int b = it / nq;
             const int ql = it - b * nq;
             const int c = 4 * (q_lo + ql);
@@ -661,6 +757,129 @@ linear_bf16_splitk_kernel(const __grid_constant__ CUtensorMap tmap_x,
                         make_float4(win[0][tau], win[1][tau], win[2][tau], win[3][tau]);
             }
         }
+        if constexpr (kFuse) {
+            // ---- the output projection ------------------------------------
+            // This CTA's y is stored (generic proxy); every CTA's must be
+            // before any is loaded (async proxy). Passing the grid barrier
+            // also means every peer has finished reading this CTA's parked
+            // partial, so TMA may overwrite the ring (the proxy fences order
+            // the parked partial's generic stores before those writes).
+            tc::fence_proxy_async();
+            __syncthreads();
+            const int nk = ke - kb;
+            if (threadIdx.x == 0) {
+                if (!tc::grid_barrier_wait(fo.bar, fo.tag, gridDim.x)) {
+                    if (status) atomicOr(status, tc::kTimeoutGrid);
+                    atomicExch(&failed, 1);
+                } else if (!*vfailed) {
+                    tc::fence_proxy_async();
+                    for (int kt = kb, g = 0; kt < ke; ++kt, ++g) {
+                        tc::mbar_arrive_expect_tx(tc::smem_u32(&y_full[g]), L::kA);
+                        tc::tma_load_2d(base + g * L::kA, &fm.y, tc::smem_u32(&y_full[g]),
+                                        kt * kBK, 0);
+                    }
+                    y_issued = nk;
+                }
+            }
+            __syncthreads();
+            const bool run_out = y_issued > 0;
+            if (run_out && warp == 1 && lane == 0) {
+                // y chunk g (A, 128 rows) times W_out chunk g (B, 64 rows)
+                // into TMEM columns [0, 64), in k order, as each chunk lands
+                bool ok = tc::mbar_wait(tc::smem_u32(&wo_full), 0) && !*vfailed;
+                const uint32_t idesc = tc::idesc_bf16_f32(kMmaM, 64);
+                for (int g = 0; ok && g < nk; ++g) {
+                    if (!tc::mbar_wait(tc::smem_u32(&y_full[g]), 0)) {
+                        ok = false;
+                        break;
+                    }
+                    tc::tc_fence_after();
+                    const uint32_t a = base + g * L::kA;
+                    const uint32_t b = wo_addr(g);
+#pragma unroll
+                    for (int kk = 0; kk < kBK / 16; ++kk)
+                        tc::mma_bf16(tmem, tc::desc_k_sw128(a + kk * 32),
+                                     tc::desc_k_sw128(b + kk * 32), idesc,
+                                     (g > 0 || kk > 0) ? 1u : 0u);
+                }
+                if (ok) {
+                    tc::mma_commit(tc::smem_u32(&out_full));
+                } else {
+                    if (status) atomicOr(status, tc::kTimeoutMma);
+                    atomicExch(&failed, 1);
+                }
+            } else if (run_out && warp >= 2 && warp < 2 + kEpilogueWarps) {
+                // park the output partial (rows < M, 64 columns, rows padded
+                // by 16 bytes) at the ring's start: every y chunk was read
+                constexpr int kPitchO = 64 + 4;
+                const int row = (warp & 3) * 32 + lane;
+                if (!tc::mbar_wait(tc::smem_u32(&out_full), 0) || *vfailed) {
+                    if (status) atomicOr(status, tc::kTimeoutEpilogue);
+                    atomicExch(&failed, 1);
+                } else {
+                    tc::tc_fence_after();
+                    const uint32_t src = tmem + (static_cast<uint32_t>((warp & 3) * 32) << 16);
+                    uint32_t r[64];
+                    tc::tmem_ld_32x32b_x64(src, r);
+                    tc::tmem_ld_wait();
+                    if (row < M) {
+                        float4* dst = reinterpret_cast<float4*>(part + row * kPitchO);
+#pragma unroll
+                        for (int j = 0; j < 16; ++j)
+                            dst[j] = make_float4(
+                                __uint_as_float(r[4 * j]), __uint_as_float(r[4 * j + 1]),
+                                __uint_as_float(r[4 * j + 2]), __uint_as_float(r[4 * j + 3]));
+                    }
+                }
+            }
+            tc::tc_fence_before();
+            __syncthreads();
+            __syncwarp();
+            tc::cluster_sync();
+            // every CTA sums a 1/S slice of the 64-column tile over the S
+            // partials in rank order and stores it: the split-K form's sum
+            {
+                constexpr int kPitchO = 64 + 4;
+                constexpr int kQuadsO = 16;
+                const int units = run_out ? M * kQuadsO : 0;
+                const int lo = static_cast<int>(static_cast<int64_t>(rank) * units / splits);
+                const int hi = static_cast<int>(static_cast<int64_t>(rank + 1) * units / splits);
+#pragma unroll 1
+                for (int u0 = lo + static_cast<int>(threadIdx.x); u0 < hi; u0 += 2 * kThr) {
+                    float4 v[2][8];
+#pragma unroll
+                    for (int h = 0; h < 2; ++h) {
+                        const int u = u0 + h * kThr;
+                        if (u >= hi) continue;
+                        const int row = u / kQuadsO;
+                        const int c = (u - row * kQuadsO) * 4;
+                        const uint32_t off = static_cast<uint32_t>((row * kPitchO + c) * 4);
+#pragma unroll
+                        for (int s2 = 0; s2 < 8; ++s2)
+                            if (s2 < splits) v[h][s2] = tc::ld_cluster_f4(peer[s2] + off);
+                    }
+#pragma unroll
+                    for (int h = 0; h < 2; ++h) {
+                        const int u = u0 + h * kThr;
+                        if (u >= hi) continue;
+                        const int row = u / kQuadsO;
+                        const int c = (u - row * kQuadsO) * 4;
+                        float4 acc = v[h][0];
+#pragma unroll
+                        for (int s2 = 1; s2 < 8; ++s2) {
+                            if (s2 < splits) {
+                                acc.x = __fadd_rn(acc.x, v[h][s2].x);
+                                acc.y = __fadd_rn(acc.y, v[h][s2].y);
+                                acc.z = __fadd_rn(acc.z, v[h][s2].z);
+                                acc.w = __fadd_rn(acc.w, v[h][s2].w);
+                            }
+                        }
+                        *reinterpret_cast<float4*>(fo.out + static_cast<int64_t>(row) * ge.D + n0 +
+                                                   c) = acc;
+                    }
+                }
+            }
+        }
         // no CTA leaves (releasing its shared memory) while a peer still reads it
         __syncwarp();
         tc::cluster_sync();
@@ -669,7 +888,7 @@ linear_bf16_splitk_kernel(const __grid_constant__ CUtensorMap tmap_x,
         float4* u_s = reinterpret_cast<float4*>(reinterpret_cast<uint8_t*>(part) + kGateOff);
         float4* cg_s = u_s + kMmaM * 8;
 #pragma unroll 1
-        for (int it = static_cast<int>(threadIdx.x); it < M * nq; it += kThreads) {
+        for (int it = static_cast<int>(threadIdx.x); it < M * nq; it += kThr) {
             const int row = it / nq;
             const int ql = it - row * nq;
             const int c = 4 * (q_lo + ql);
@@ -755,15 +974,19 @@ linear_bf16_splitk_kernel(const __grid_constant__ CUtensorMap tmap_x,
         };
         const int n_items = ge.B * nch;
 #pragma unroll 1
-        for (int it = static_cast<int>(threadIdx.x); it < n_items; it += 2 * kThreads) {
+        for (int it = static_cast<int>(threadIdx.x); it < n_items; it += 2 * kThr) {
             walk(it);
-            if (it + kThreads < n_items) walk(it + kThreads);
+            if (it + kThr < n_items) walk(it + kThr);
         }
     }
 
     if (threadIdx.x == 0 && failed) {
         for (int g = consumed; g < issued; ++g)
             tc::mbar_wait(tc::smem_u32(&full[g % kStages]), static_cast<uint32_t>(g / kStages) & 1u);
+        if constexpr (kFuse) {      // the fused form's copies in flight land first
+            if (wo_issued) tc::mbar_wait(tc::smem_u32(&wo_full), 0);
+            for (int g = 0; g < y_issued; ++g) tc::mbar_wait(tc::smem_u32(&y_full[g]), 0);
+        }
     }
     tc::tc_fence_before();
     __syncthreads();
@@ -1040,22 +1263,22 @@ cudaError_t launch_bn(const LinearArgs& a, cudaStream_t stream) {
                               static_cast<int>(a.N), static_cast<int>(a.K), a.status);
 }
 
-template <int BN, int kGate = 0>
+template <int BN, int kGate = 0, bool kFuse = false>
 cudaError_t set_split_smem() {
-    return cudaFuncSetAttribute(linear_bf16_splitk_kernel<BN, kGate>,
+    return cudaFuncSetAttribute(linear_bf16_splitk_kernel<BN, kGate, kFuse>,
                                 cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                static_cast<int>(split_smem_bytes<BN, kGate>()));
+                                static_cast<int>(split_smem_bytes<BN, kGate, kFuse>()));
 }
 
 // Cluster of `splits` CTAs along x, and (`pdl`) programmatic serialization
 // so the prologue overlaps the previous kernel; attr holds two entries.
-template <int BN, int kGate = 0>
+template <int BN, int kGate = 0, bool kFuse = false>
 cudaLaunchConfig_t split_config(unsigned grid, int splits, cudaStream_t stream,
                                 cudaLaunchAttribute* attr, bool pdl) {
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(grid);
-    cfg.blockDim = dim3(kThreads);
-    cfg.dynamicSmemBytes = split_smem_bytes<BN, kGate>();
+    cfg.blockDim = dim3(split_threads(kFuse));
+    cfg.dynamicSmemBytes = split_smem_bytes<BN, kGate, kFuse>();
     cfg.stream = stream;
     attr[0].id = cudaLaunchAttributeClusterDimension;
     attr[0].val.clusterDim.x = static_cast<unsigned>(splits);
@@ -1070,7 +1293,7 @@ cudaLaunchConfig_t split_config(unsigned grid, int splits, cudaStream_t stream,
 
 // Clusters of `splits` CTAs of the BN-wide split kernel that the device holds
 // at once (cached per device; 0 when the query fails).
-template <int BN, int kGate = 0>
+template <int BN, int kGate = 0, bool kFuse = false>
 int max_active_clusters(int splits) {
     constexpr int kDevs = 16;
     static std::atomic<int> cache[kDevs][9];
@@ -1082,10 +1305,10 @@ int max_active_clusters(int splits) {
     }
     int n = 0;
     cudaLaunchAttribute attr[2];
-    const cudaLaunchConfig_t cfg = split_config<BN, kGate>(static_cast<unsigned>(splits),
+    const cudaLaunchConfig_t cfg = split_config<BN, kGate, kFuse>(static_cast<unsigned>(splits),
                                                            splits, nullptr, attr, false);
-    if (set_split_smem<BN, kGate>() != cudaSuccess ||
-        cudaOccupancyMaxActiveClusters(&n, linear_bf16_splitk_kernel<BN, kGate>, &cfg) !=
+    if (set_split_smem<BN, kGate, kFuse>() != cudaSuccess ||
+        cudaOccupancyMaxActiveClusters(&n, linear_bf16_splitk_kernel<BN, kGate, kFuse>, &cfg) !=
             cudaSuccess) {
         cudaGetLastError();
         n = 0;
@@ -1144,7 +1367,8 @@ cudaError_t launch_split_bn(const LinearArgs& a, int splits, cudaStream_t stream
         split_config<BN>(static_cast<unsigned>(tiles * splits), splits, stream, attr, true);
     return cudaLaunchKernelEx(&cfg, linear_bf16_splitk_kernel<BN, 0>, tx, tw, a.y,
                               static_cast<int>(a.M), static_cast<int>(a.N),
-                              static_cast<int>(a.K), splits, a.status, GateEpi{});
+                              static_cast<int>(a.K), splits, a.status, GateEpi{}, FuseMaps{},
+                              FuseOut{});
 }
 
 // Pairs of the pair-CTA kernel the device holds at once (cached per device).
@@ -1206,17 +1430,38 @@ cudaError_t launch_pair_gemm(const LinearArgs& a, int64_t tiles, int pairs, cuda
                               static_cast<int>(a.N), static_cast<int>(a.K), a.status);
 }
 
-// The short-conv input projection with the gate and conv as its epilogue:
-// tiles of 64 channels, each split over K like the plain form (most chunks
-// that keep the clusters in one wave, at most 8).
-template <int KT>
-cudaError_t launch_gate_k(const ShortConvArgs& a, void* y, cudaStream_t stream) {
-    const int64_t M = a.B * a.T, D = a.D;
+// The gate form's split of K for D channels: tiles of 64 channels, each split
+// over K like the plain form (the most chunks that keep the clusters in one
+// wave, at most 8); below 2 the form does not apply.
+template <int KT, bool kFuse = false>
+int64_t gate_splits(int64_t D) {
     const int64_t n_kt = (D + kBK - 1) / kBK;
     const int64_t tiles = (D + 63) / 64;
     int64_t s = std::min<int64_t>(std::min<int64_t>(8, n_kt), device_sm_count() / tiles);
     for (; s >= 2; --s)
-        if (tiles <= max_active_clusters<192, KT>(static_cast<int>(s))) break;
+        if (tiles <= max_active_clusters<192, KT, kFuse>(static_cast<int>(s))) break;
+    return s;
+}
+
+GateEpi gate_epi(const ShortConvArgs& a, void* y) {
+    GateEpi ge;
+    ge.ring = a.conv_ring;
+    ge.scratch_ring = a.scratch_ring;
+    ge.conv_w = a.conv_w;
+    ge.y = static_cast<__nv_bfloat16*>(y);
+    ge.B = static_cast<int>(a.B);
+    ge.T = static_cast<int>(a.T);
+    ge.D = static_cast<int>(a.D);
+    ge.n_commit = static_cast<int>(a.n_commit);
+    return ge;
+}
+
+// The short-conv input projection with the gate and conv as its epilogue.
+template <int KT>
+cudaError_t launch_gate_k(const ShortConvArgs& a, void* y, cudaStream_t stream) {
+    const int64_t M = a.B * a.T, D = a.D;
+    const int64_t tiles = (D + 63) / 64;
+    const int64_t s = gate_splits<KT>(D);
     if (s < 2) return cudaErrorNotSupported;
     CUtensorMap tx, tw;
     if (!make_tmap(&tx, a.hidden, M, D, kMmaM) || !make_tmap(&tw, a.w_in, 3 * D, D, 64))
@@ -1226,19 +1471,66 @@ cudaError_t launch_gate_k(const ShortConvArgs& a, void* y, cudaStream_t stream) 
     cudaLaunchAttribute attr[2];
     const cudaLaunchConfig_t cfg = split_config<192, KT>(static_cast<unsigned>(tiles * s),
                                                          static_cast<int>(s), stream, attr, true);
-    GateEpi ge;
-    ge.ring = a.conv_ring;
-    ge.scratch_ring = a.scratch_ring;
-    ge.conv_w = a.conv_w;
-    ge.y = static_cast<__nv_bfloat16*>(y);
-    ge.B = static_cast<int>(a.B);
-    ge.T = static_cast<int>(a.T);
-    ge.D = static_cast<int>(D);
-    ge.n_commit = static_cast<int>(a.n_commit);
     return cudaLaunchKernelEx(&cfg, linear_bf16_splitk_kernel<192, KT>, tx, tw,
                               static_cast<float*>(nullptr), static_cast<int>(M),
                               static_cast<int>(3 * D), static_cast<int>(D), static_cast<int>(s),
-                              a.status, ge);
+                              a.status, gate_epi(a, y), FuseMaps{}, FuseOut{});
+}
+
+// A 48-bit tag, never 0, for each fused launch enqueued by this process
+// (SplitMix64 over a counter seeded from the clock and the process id), so
+// that the barrier word of a workspace never holds a stale tag of a later
+// call.
+uint64_t next_call_tag() {
+    static std::atomic<uint64_t> seq{0};
+    static const uint64_t seed = static_cast<uint64_t>(
+        std::chrono::steady_clock::now().time_since_epoch().count()) ^
+        (static_cast<uint64_t>(getpid()) << 32);
+    uint64_t z = seed + 0x9E3779B97F4A7C15ull * (seq.fetch_add(1, std::memory_order_relaxed) + 1);
+    z = (z ^ (z >> 30)) * 0xBF58476D1CE4E5B9ull;
+    z = (z ^ (z >> 27)) * 0x94D049BB133111EBull;
+    z ^= z >> 31;
+    z &= (1ull << 48) - 1;
+    return z ? z : 1;
+}
+
+// The whole mixer in one kernel (the split kernel's kFuse form), for calls of
+// one or two positions whose split is the one the two-kernel path takes for
+// both projections, so that its bits are that path's.
+template <int KT>
+cudaError_t launch_fused_k(const ShortConvArgs& a, void* y, unsigned long long* bar,
+                           cudaStream_t stream) {
+    const int64_t M = a.B * a.T, D = a.D;
+    if (a.T > 2 || M > kMmaM || D % 64 != 0 || (reinterpret_cast<uintptr_t>(bar) & 7) != 0)
+        return cudaErrorNotSupported;
+    const int64_t n_kt = D / kBK, tiles = D / 64;
+    const int64_t s = gate_splits<KT>(D);
+    if (s < 2 || gate_splits<KT, true>(D) != s) return cudaErrorNotSupported;
+    const SplitPlan p = split_plan(D, D);
+    if (p.bn != 64 || p.splits != s) return cudaErrorNotSupported;
+    if ((n_kt + s - 1) / s > kFuseMaxSteps) return cudaErrorNotSupported;
+    // every rank's conv rings in shared memory (the walk the fused form runs)
+    const int64_t nq_max = (16 + s - 1) / s;
+    if (a.B * (KT - 1) * 4 * nq_max * 4 > static_cast<int64_t>(kRingCache))
+        return cudaErrorNotSupported;
+    CUtensorMap tx, tw;
+    FuseMaps fm;
+    if (!make_tmap(&tx, a.hidden, M, D, kMmaM) || !make_tmap(&tw, a.w_in, 3 * D, D, 64) ||
+        !make_tmap(&fm.y, y, M, D, kMmaM) || !make_tmap(&fm.wo, a.w_out, D, D, 64))
+        return cudaErrorInvalidValue;
+    cudaError_t err = set_split_smem<192, KT, true>();
+    if (err != cudaSuccess) return err;
+    cudaLaunchAttribute attr[2];
+    const cudaLaunchConfig_t cfg = split_config<192, KT, true>(
+        static_cast<unsigned>(tiles * s), static_cast<int>(s), stream, attr, true);
+    FuseOut fo;
+    fo.out = a.out;
+    fo.bar = bar;
+    fo.tag = next_call_tag();
+    return cudaLaunchKernelEx(&cfg, linear_bf16_splitk_kernel<192, KT, true>, tx, tw,
+                              static_cast<float*>(nullptr), static_cast<int>(M),
+                              static_cast<int>(3 * D), static_cast<int>(D), static_cast<int>(s),
+                              a.status, gate_epi(a, y), fm, fo);
 }
 
 }  // namespace
@@ -1249,6 +1541,16 @@ cudaError_t launch_short_conv_in_gate(const ShortConvArgs& a, void* y, cudaStrea
         case 2: return launch_gate_k<2>(a, y, stream);
         case 3: return launch_gate_k<3>(a, y, stream);
         case 4: return launch_gate_k<4>(a, y, stream);
+        default: return cudaErrorInvalidValue;
+    }
+}
+
+cudaError_t launch_short_conv_fused(const ShortConvArgs& a, void* y, unsigned long long* bar,
+                                    cudaStream_t stream) {
+    switch (a.K) {
+        case 2: return launch_fused_k<2>(a, y, bar, stream);
+        case 3: return launch_fused_k<3>(a, y, bar, stream);
+        case 4: return launch_fused_k<4>(a, y, bar, stream);
         default: return cudaErrorInvalidValue;
     }
 }

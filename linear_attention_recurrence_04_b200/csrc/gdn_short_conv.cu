@@ -30,7 +30,10 @@
 // partials and does the gate, conv and rings for its 64 channels (the same
 // arithmetic as the gate kernel below); stage 4 is split the same way. The
 // rows of such calls agree bit for bit with one another, and with larger
-// calls to fp32 rounding of the projections' accumulation order.
+// calls to fp32 rounding of the projections' accumulation order. Calls of
+// one or two positions whose two splits agree run all four stages as one
+// kernel (the split kernel's fused form: a grid-wide barrier on a word of the
+// workspace between the conv and the output projection), with the same bits.
 // u is rounded to fp32 (the ring's type) before it enters the window; the
 // window sum and the output gate run in double, and y is rounded once.
 #include <cuda_bf16.h>
@@ -38,6 +41,12 @@
 #include "gdn_common.cuh"
 #include "gdn_internal.h"
 #include "gdn_tc.cuh"
+
+// 1: calls of one or two positions run the whole mixer as one kernel; 0:
+// they take the two-kernel path (the same bits).
+#ifndef GDN_SHORT_CONV_FUSED
+#define GDN_SHORT_CONV_FUSED 1
+#endif
 
 namespace gdn {
 
@@ -215,7 +224,8 @@ ShortConvLayout short_conv_layout(int64_t B, int64_t T, int64_t D) {
     ShortConvLayout L;
     L.proj = 0;
     L.y = align256(static_cast<size_t>(BT) * 3 * D * 4);
-    L.total = align256(L.y + static_cast<size_t>(BT) * D * 2);
+    L.bar = align256(L.y + static_cast<size_t>(BT) * D * 2);
+    L.total = L.bar + 256;
     return L;
 }
 
@@ -226,9 +236,15 @@ cudaError_t launch_short_conv(const ShortConvArgs& a, cudaStream_t stream) {
     char* ws = static_cast<char*>(a.workspace);
     float* proj = reinterpret_cast<float*>(ws + L.proj);
     __nv_bfloat16* y = reinterpret_cast<__nv_bfloat16*>(ws + L.y);
+    // one or two positions, at most 128 rows: the whole mixer in one kernel
+    cudaError_t err = cudaErrorNotSupported;
+    if (GDN_SHORT_CONV_FUSED)
+        err = launch_short_conv_fused(a, y, reinterpret_cast<unsigned long long*>(ws + L.bar),
+                                      stream);
+    if (err != cudaErrorNotSupported) return err;
     // at most 128 rows: stages 1-3 in one kernel (the split-K projection with
     // the gate, conv and rings as its epilogue), then stage 4
-    cudaError_t err = launch_short_conv_in_gate(a, y, stream);
+    err = launch_short_conv_in_gate(a, y, stream);
     if (err == cudaSuccess)
         return launch_linear_bf16_split(LinearArgs{y, a.w_out, a.out, BT, a.D, a.D, a.status},
                                         stream);

@@ -21,6 +21,7 @@ constexpr uint32_t kTimeoutProducer = 1u;
 constexpr uint32_t kTimeoutMma = 2u;
 constexpr uint32_t kTimeoutEpilogue = 4u;
 constexpr uint32_t kTimeoutPrefill = 8u;     // the prefill's stage pipeline
+constexpr uint32_t kTimeoutGrid = 16u;       // a grid-wide barrier (one-kernel mixer)
 // Every wait gives up after this long (nanoseconds of %globaltimer).
 constexpr uint64_t kWaitLimitNs = 2000000000ull;
 
@@ -162,6 +163,11 @@ __device__ __forceinline__ void tmem_ld_32x32b_x32(uint32_t taddr, uint32_t (&r)
         : "r"(taddr)
         : "memory");
 }
+// 32 lanes x 64 consecutive 32-bit columns (one round trip for 64 columns).
+__device__ __forceinline__ void tmem_ld_32x32b_x64(uint32_t taddr, uint32_t (&r)[64]) {
+    tmem_ld_32x32b_x32(taddr, *reinterpret_cast<uint32_t(*)[32]>(&r[0]));
+    tmem_ld_32x32b_x32(taddr + 32, *reinterpret_cast<uint32_t(*)[32]>(&r[32]));
+}
 __device__ __forceinline__ void tmem_ld_wait() {
     asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
 }
@@ -258,6 +264,51 @@ __device__ __forceinline__ float4 ld_cluster_f4(uint32_t addr) {
     asm volatile("ld.shared::cluster.v4.f32 {%0, %1, %2, %3}, [%4];"
                  : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w) : "r"(addr) : "memory");
     return v;
+}
+
+// ---- grid-wide barrier on one 64-bit word of global memory -------------------
+// Orders this thread's generic-proxy accesses (global and shared) with
+// async-proxy (TMA) ones: a TMA load of data that generic stores wrote, or
+// into shared memory that generic stores wrote before.
+__device__ __forceinline__ void fence_proxy_async() {
+    asm volatile("fence.proxy.async;" ::: "memory");
+}
+// The word holds (tag << 16) | count, where `tag` (48 bits, never 0) names
+// one call. Install: a CTA that finds the word holding anything but this
+// call's tag with a count below `n` replaces it with (tag, 0) -- either
+// another call's word or this tag's word left complete by an earlier launch
+// of the same call (a CUDA graph replay), never this launch's, which cannot
+// reach n before this CTA arrives. Wait: the CTA adds 1 (release) and waits
+// (acquire) until the count reaches `n`; the word is left as (tag, n). A CTA
+// whose wait runs past kWaitLimitNs clears the word and returns false: the
+// others then time out too, and nothing of the failed launch survives it.
+// Each CTA installs once (after the previous kernel on the stream has
+// completed) and then waits once, on every path, from one thread; every CTA
+// of the grid must become resident (n CTAs on distinct SMs, nothing that
+// waits on this grid occupying the rest).
+__device__ __forceinline__ void grid_barrier_install(unsigned long long* word, uint64_t tag,
+                                                     uint32_t n) {
+    const unsigned long long mine = static_cast<unsigned long long>(tag) << 16;
+    unsigned long long v = *reinterpret_cast<volatile unsigned long long*>(word);
+    while (!((v >> 16) == tag && (v & 0xffffull) < n)) {
+        const unsigned long long prev = atomicCAS(word, v, mine);
+        if (prev == v) break;
+        v = prev;
+    }
+}
+__device__ __forceinline__ bool grid_barrier_wait(unsigned long long* word, uint64_t tag,
+                                                  uint32_t n) {
+    asm volatile("red.release.gpu.global.add.u64 [%0], 1;" ::"l"(word) : "memory");
+    const uint64_t t0 = global_timer();
+    for (int polls = 0;; ++polls) {
+        unsigned long long w;
+        asm volatile("ld.acquire.gpu.global.u64 %0, [%1];" : "=l"(w) : "l"(word) : "memory");
+        if ((w >> 16) == tag && (w & 0xffffull) >= n) return true;
+        if ((polls & 15) == 15 && global_timer() - t0 > kWaitLimitNs) break;
+        __nanosleep(32);
+    }
+    atomicExch(word, 0ull);
+    return false;
 }
 
 }  // namespace tc
