@@ -449,6 +449,27 @@ gdn_status gdn_short_conv_pair(const void *hidden, const void *w_in, const void 
 gdn_status gdn_selftest_bounded_wait(uint32_t *result, uint64_t limit_ns, int arrive,
                                      void *stream);
 
+/*
+ * gdn_selftest_grid_barrier -- the same check for the grid-wide barrier of
+ * the one-kernel short-conv mixer (see gdn_short_conv_forward), with no
+ * counterpart on the source pages. `ctas` CTAs (1..32, one thread each)
+ * install `tag` into `word` and wait, each with the limit limit_ns
+ * (0 < limit_ns <= 2e9), until `expect` (1..64) have arrived.
+ *   word    device uint64, 8-byte aligned: (tag << 16) | count; on entry
+ *           anything (another tag, a completed count of this tag); on
+ *           return (tag << 16) | ctas when every wait completed, and 0 after
+ *           a wait ran out (expect > ctas makes every wait run out)
+ *   result  device words [2 * ctas]: result[i] = 0 (CTA i passed) or 16
+ *           (timed out: the bit the mixer ORs into its status word);
+ *           result[ctas + i] = microseconds CTA i waited. 4-byte aligned.
+ *   tag     0 < tag < 2^48; as in the mixer, a tag names one grid: a word
+ *           left as (tag, c) with c < expect counts as that grid in progress
+ * Errors: GDN_ERR_NULL, GDN_ERR_UNSUPPORTED (a size, the tag or the limit
+ * out of range), GDN_ERR_ALIGN, GDN_ERR_CUDA (launch refused).
+ */
+gdn_status gdn_selftest_grid_barrier(unsigned long long *word, uint32_t *result, uint64_t tag,
+                                     int ctas, int expect, uint64_t limit_ns, void *stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -274,7 +274,7 @@ __device__ __forceinline__ void fence_proxy_async() {
     asm volatile("fence.proxy.async;" ::: "memory");
 }
 // The word holds (tag << 16) | count, where `tag` (48 bits, never 0) names
-// one call. Install: a CTA that finds the word holding anything but this
+// one call and so one grid size `n` (a replay repeats both). Install: a CTA that finds the word holding anything but this
 // call's tag with a count below `n` replaces it with (tag, 0) -- either
 // another call's word or this tag's word left complete by an earlier launch
 // of the same call (a CUDA graph replay), never this launch's, which cannot
@@ -297,14 +297,14 @@ __device__ __forceinline__ void grid_barrier_install(unsigned long long* word, u
     }
 }
 __device__ __forceinline__ bool grid_barrier_wait(unsigned long long* word, uint64_t tag,
-                                                  uint32_t n) {
+                                                  uint32_t n, uint64_t limit_ns = kWaitLimitNs) {
     asm volatile("red.release.gpu.global.add.u64 [%0], 1;" ::"l"(word) : "memory");
     const uint64_t t0 = global_timer();
     for (int polls = 0;; ++polls) {
         unsigned long long w;
         asm volatile("ld.acquire.gpu.global.u64 %0, [%1];" : "=l"(w) : "l"(word) : "memory");
         if ((w >> 16) == tag && (w & 0xffffull) >= n) return true;
-        if ((polls & 15) == 15 && global_timer() - t0 > kWaitLimitNs) break;
+        if ((polls & 15) == 15 && global_timer() - t0 > limit_ns) break;
         __nanosleep(32);
     }
     atomicExch(word, 0ull);

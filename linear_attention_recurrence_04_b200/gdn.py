@@ -34,7 +34,8 @@ EXPORTS = ("gdn_status_string", "gdn_last_error", "gdn_last_cuda_error", "gdn_st
            "gdn_forward_batch_workspace_size",
            "gdn_forward_batch", "gdn_forward_batch_noalloc", "gdn_short_conv_workspace_size",
            "gdn_short_conv_forward_batch", "gdn_short_conv_forward", "gdn_short_conv_pair",
-           "gdn_kda_step", "gdn_kda_prefill", "gdn_selftest_bounded_wait")
+           "gdn_kda_step", "gdn_kda_prefill", "gdn_selftest_bounded_wait",
+           "gdn_selftest_grid_barrier")
 
 
 class GdnError(RuntimeError):
@@ -97,6 +98,9 @@ def load_library(path: Optional[str] = None) -> ctypes.CDLL:
         getattr(lib, name).argtypes = [_VP] * 7 + [_I64] * 6 + [_VP]
     lib.gdn_selftest_bounded_wait.restype = ctypes.c_int
     lib.gdn_selftest_bounded_wait.argtypes = [_VP, ctypes.c_uint64, ctypes.c_int, _VP]
+    lib.gdn_selftest_grid_barrier.restype = ctypes.c_int
+    lib.gdn_selftest_grid_barrier.argtypes = [_VP, _VP, ctypes.c_uint64, ctypes.c_int,
+                                              ctypes.c_int, ctypes.c_uint64, _VP]
     lib.gdn_short_conv_workspace_size.restype = ctypes.c_size_t
     lib.gdn_short_conv_workspace_size.argtypes = [_I64] * 3
     lib.gdn_short_conv_forward_batch.restype = ctypes.c_int
@@ -554,3 +558,21 @@ def selftest_bounded_wait(limit_ns: int, arrive: bool = False, *, device=None, s
     torch.cuda.synchronize(device)
     r = result.cpu().tolist()
     return bool(r[0]), int(r[1]) & 0xFFFFFFFF
+
+
+def selftest_grid_barrier(word, tag: int, ctas: int, expect: int, limit_ns: int, *,
+                          stream=None):
+    """Run the one-kernel mixer's grid-wide barrier in `ctas` CTAs on `word`
+    (a CUDA int64 tensor of one element) expecting `expect` arrivals. Returns
+    (status bits per CTA, microseconds waited per CTA) after synchronising."""
+    if word.dtype is not torch.int64 or not word.is_cuda or word.numel() != 1:
+        raise TypeError("word must be a one-element int64 CUDA tensor")
+    device = word.device
+    result = torch.zeros(2 * ctas, dtype=torch.int32, device=device)
+    st = _call(device, load_library().gdn_selftest_grid_barrier, word.data_ptr(),
+               result.data_ptr(), int(tag), int(ctas), int(expect), int(limit_ns),
+               _stream(device, stream))
+    _raise_on("gdn_selftest_grid_barrier", st)
+    torch.cuda.synchronize(device)
+    r = result.cpu().tolist()
+    return [x & 0xFFFFFFFF for x in r[:ctas]], [x & 0xFFFFFFFF for x in r[ctas:]]

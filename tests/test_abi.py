@@ -277,3 +277,21 @@ def test_selftest_bounded_wait_argument_checks(lib):
     assert lib.gdn_selftest_bounded_wait(fake(1), 0, 0, None) == UNSUP
     assert lib.gdn_selftest_bounded_wait(fake(1), 2_000_000_001, 0, None) == UNSUP
     assert lib.gdn_selftest_bounded_wait(fake(1) + 2, 1000, 0, None) == ALIGN
+
+
+def test_selftest_grid_barrier_argument_checks(lib):
+    """Refused on the host before any launch: null pointers, sizes, a zero or
+    over-wide tag, the limit, misalignment."""
+    w, r = fake(1), fake(2)
+    assert lib.gdn_selftest_grid_barrier(0, r, 5, 2, 2, 1000, None) == NULL
+    assert lib.gdn_selftest_grid_barrier(w, 0, 5, 2, 2, 1000, None) == NULL
+    assert lib.gdn_selftest_grid_barrier(w, r, 5, 0, 2, 1000, None) == UNSUP
+    assert lib.gdn_selftest_grid_barrier(w, r, 5, 33, 2, 1000, None) == UNSUP
+    assert lib.gdn_selftest_grid_barrier(w, r, 5, 2, 0, 1000, None) == UNSUP
+    assert lib.gdn_selftest_grid_barrier(w, r, 5, 2, 65, 1000, None) == UNSUP
+    assert lib.gdn_selftest_grid_barrier(w, r, 0, 2, 2, 1000, None) == UNSUP
+    assert lib.gdn_selftest_grid_barrier(w, r, 1 << 48, 2, 2, 1000, None) == UNSUP
+    assert lib.gdn_selftest_grid_barrier(w, r, 5, 2, 2, 0, None) == UNSUP
+    assert lib.gdn_selftest_grid_barrier(w, r, 5, 2, 2, 2_000_000_001, None) == UNSUP
+    assert lib.gdn_selftest_grid_barrier(w + 4, r, 5, 2, 2, 1000, None) == ALIGN
+    assert lib.gdn_selftest_grid_barrier(w, r + 2, 5, 2, 2, 1000, None) == ALIGN

@@ -39,3 +39,33 @@ def test_context_is_usable_after_a_timeout():
     y = gdn.linear_bf16(x, w, status=status)
     torch.cuda.synchronize()
     assert int(status.item()) == 0 and not bool(y.any())
+
+
+def _word_value(word):
+    return int(word.item()) & 0xFFFFFFFFFFFFFFFF
+
+
+def test_grid_barrier_passes_runs_out_and_resets():
+    """The one-kernel short-conv mixer's grid-wide barrier, run on its own.
+    A tag always comes with one grid size (one tag per enqueued call, which a
+    graph replay repeats). 8 CTAs meet on a word that holds stale bytes and,
+    on the second run, this tag's own completed count (as a replay finds it),
+    and pass. With a new tag and one CTA fewer than expected, every wait runs
+    out after its limit, reports bit 16 and leaves the word cleared; that
+    call then completes when replayed with its full grid, and another tag
+    replaces its completed word."""
+    tag = 0x5EED_0000_1234
+    word = torch.full((1,), 0x0123_4567_89AB_CDEF, dtype=torch.int64, device="cuda")
+    for _ in range(2):
+        bits, waited = gdn.selftest_grid_barrier(word, tag, 8, 8, 50_000_000)
+        assert bits == [0] * 8, bits
+        assert max(waited) < 50_000, waited
+        assert _word_value(word) == (tag << 16) | 8
+    bits, waited = gdn.selftest_grid_barrier(word, tag + 1, 8, 9, 30_000_000)   # 30 ms limit
+    assert bits == [16] * 8, bits
+    assert all(30_000 <= w < 1_000_000 for w in waited), waited
+    assert _word_value(word) == 0
+    bits, _ = gdn.selftest_grid_barrier(word, tag + 1, 9, 9, 50_000_000)
+    assert bits == [0] * 9 and _word_value(word) == ((tag + 1) << 16) | 9
+    bits, _ = gdn.selftest_grid_barrier(word, tag, 3, 3, 50_000_000)
+    assert bits == [0] * 3 and _word_value(word) == (tag << 16) | 3
