@@ -75,6 +75,10 @@
 #ifndef GDN_PREFILL_GDN_LPR
 #define GDN_PREFILL_GDN_LPR 4      // scalar decay: lanes per state row (4 or 8)
 #endif
+#ifndef GDN_PREFILL_GDN_HALVING
+#define GDN_PREFILL_GDN_HALVING 0  // scalar decay, 4 lanes per row: one halving reduction of
+                                   // the A and O values with the deltas broadcast
+#endif
 #ifndef GDN_PREFILL_GDN_RPL
 #define GDN_PREFILL_GDN_RPL 1      // scalar decay: state rows per lane (2 needs 8 lanes per row)
 #endif
@@ -172,7 +176,7 @@ struct Layout {
     static constexpr int Threads = 32 * (MaxWarps + Helpers);
     // One halving reduction of all key and output dots with the deltas
     // broadcast, rather than a full reduction of each on every lane.
-    static constexpr bool Halving = LPR == 8;
+    static constexpr bool Halving = LPR == 8 || (!kCh && GDN_PREFILL_GDN_HALVING);
     static_assert(LPR == 4 || LPR == 8, "4 or 8 lanes per row");
     static_assert(Halving || RPL == 1, "two rows per lane use the halving reduction");
     // The key of position t + 1, read by pass t for the next key dot, is the
