@@ -404,7 +404,9 @@ gdn_status gdn_kda_prefill(float *state, const float *q, const float *k, const f
  * once (one per SM, at most 148): a kernel on another stream that holds SMs
  * for longer than the 2 s wait limit makes the call time out, ORing 16 into
  * `status` (the outputs are then undefined). Two calls that share a
- * workspace must be ordered, as for any workspace.
+ * workspace must be ordered, as for any workspace. The environment variable
+ * GDN_SHORT_CONV_ONE_KERNEL=0, read at every call, selects the two-kernel
+ * path instead (the same bits), e.g. where other work holds SMs for long.
  *
  * gdn_short_conv_forward_batch runs T positions in order; conv_ring ends as
  * the ring after position T-1 (T = 0 does nothing).

@@ -38,6 +38,8 @@
 // window sum and the output gate run in double, and y is rounded once.
 #include <cuda_bf16.h>
 
+#include <cstdlib>
+
 #include "gdn_common.cuh"
 #include "gdn_internal.h"
 #include "gdn_tc.cuh"
@@ -236,9 +238,12 @@ cudaError_t launch_short_conv(const ShortConvArgs& a, cudaStream_t stream) {
     char* ws = static_cast<char*>(a.workspace);
     float* proj = reinterpret_cast<float*>(ws + L.proj);
     __nv_bfloat16* y = reinterpret_cast<__nv_bfloat16*>(ws + L.y);
-    // one or two positions, at most 128 rows: the whole mixer in one kernel
+    // one or two positions, at most 128 rows: the whole mixer in one kernel,
+    // unless the environment turns it off (GDN_SHORT_CONV_ONE_KERNEL=0; read
+    // at every call)
     cudaError_t err = cudaErrorNotSupported;
-    if (GDN_SHORT_CONV_FUSED)
+    const char* one = std::getenv("GDN_SHORT_CONV_ONE_KERNEL");
+    if (GDN_SHORT_CONV_FUSED && !(one && one[0] == '0' && one[1] == '\0'))
         err = launch_short_conv_fused(a, y, reinterpret_cast<unsigned long long*>(ws + L.bar),
                                       stream);
     if (err != cudaErrorNotSupported) return err;

@@ -335,3 +335,38 @@ def test_one_kernel_decode_graph_replay_and_stale_workspace():
     assert torch.equal(g["conv_ring"], eager["conv_ring"]), "ring after the replays"
     check_word(ws, need, D)
     del graph
+
+
+@pytest.mark.parametrize("T", [1, 2])
+def test_one_kernel_and_two_kernel_paths_are_bit_identical(monkeypatch, T):
+    """GDN_SHORT_CONV_ONE_KERNEL=0 selects the two-kernel path for decode and
+    verify calls; both paths give the same outputs and rings bit for bit
+    (64 sequences, D = 2048, K = 3)."""
+    B, D, K = 64, 2048, 3
+    d = inputs.short_conv_inputs(B, T, D=D, K=K, seed=1499 + T)
+    runs = {}
+    for flag in ("1", "0"):
+        monkeypatch.setenv("GDN_SHORT_CONV_ONE_KERNEL", flag)
+        t = to_dev(d)
+        need = gdn.short_conv_workspace_size(B, T, D)
+        ws = torch.zeros(need, dtype=torch.uint8, device="cuda")
+        status = torch.zeros(1, dtype=torch.int32, device="cuda")
+        if T == 1:
+            out = gdn.short_conv_forward(t["hidden"][:, 0].contiguous(), t["w_in"], t["w_out"],
+                                         t["conv_ring"], t["conv_w"], workspace=ws,
+                                         status=status)
+            scratch = None
+        else:
+            scratch = torch.full_like(t["conv_ring"], float("nan"))
+            out = gdn.short_conv_pair(t["hidden"], t["w_in"], t["w_out"], t["conv_ring"],
+                                      scratch, t["conv_w"], workspace=ws, status=status)
+        torch.cuda.synchronize()
+        assert int(status.item()) == 0
+        word = int.from_bytes(bytes(ws[need - 256:need - 248].cpu().numpy()), "little")
+        runs[flag] = (out, t["conv_ring"], scratch, word)
+    one, two = runs["1"], runs["0"]
+    assert one[3] != 0 and two[3] == 0, "the barrier word shows which path ran"
+    assert torch.equal(one[0], two[0]), "outputs"
+    assert torch.equal(one[1], two[1]), "committed ring"
+    if T == 2:
+        assert torch.equal(one[2], two[2]), "scratch ring"
