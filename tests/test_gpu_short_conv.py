@@ -370,3 +370,36 @@ def test_one_kernel_and_two_kernel_paths_are_bit_identical(monkeypatch, T):
     assert torch.equal(one[1], two[1]), "committed ring"
     if T == 2:
         assert torch.equal(one[2], two[2]), "scratch ring"
+
+
+@pytest.mark.parametrize("K", [3, 4])
+def test_decode_b128_full_rows_matches_oracle(o, monkeypatch, K):
+    """128 sequences, one position: the largest call of the split forms. With
+    K = 3 it runs as one kernel (all 128 rows of every partial and y box
+    real) and equals the two-kernel path bit for bit; with K = 4 the rings of
+    a CTA's channels no longer fit its shared-memory cache and the call takes
+    the two kernels. Both against the oracle."""
+    B, D = 128, 2048
+    d = inputs.short_conv_inputs(B, 1, D=D, K=K, seed=1510 + K)
+    ref_out, ref_ring = o.short_conv_forward_batch(d["hidden"], d["w_in"], d["w_out"],
+                                                   d["conv_ring"], d["conv_w"])
+    results = {}
+    for flag in ("1", "0"):
+        monkeypatch.setenv("GDN_SHORT_CONV_ONE_KERNEL", flag)
+        t = to_dev(d)
+        need = gdn.short_conv_workspace_size(B, 1, D)
+        ws = torch.zeros(need, dtype=torch.uint8, device="cuda")
+        status = torch.zeros(1, dtype=torch.int32, device="cuda")
+        out = gdn.short_conv_forward(t["hidden"][:, 0].contiguous(), t["w_in"], t["w_out"],
+                                     t["conv_ring"], t["conv_w"], workspace=ws, status=status)
+        torch.cuda.synchronize()
+        assert int(status.item()) == 0
+        word = int.from_bytes(bytes(ws[need - 256:need - 248].cpu().numpy()), "little")
+        results[flag] = (out, t["conv_ring"], word)
+        check_out(out.cpu().numpy(), ref_out[:, 0], f"decode_b128 K{K} out ({flag})")
+        check_ring(t["conv_ring"].cpu().numpy(), d["conv_ring"], d["hidden"], d["w_in"],
+                   ref_ring, 0, f"decode_b128 K{K} ring ({flag})")
+    one, two = results["1"], results["0"]
+    assert two[2] == 0
+    assert (one[2] != 0) == (K == 3), "one kernel for K = 3 only"
+    assert torch.equal(one[0], two[0]) and torch.equal(one[1], two[1])
