@@ -75,6 +75,12 @@
 #ifndef GDN_PREFILL_GDN_LPR
 #define GDN_PREFILL_GDN_LPR 4      // scalar decay: lanes per state row (4 or 8)
 #endif
+#ifndef GDN_PREFILL_STAGE_FOLD_CHECK
+#define GDN_PREFILL_STAGE_FOLD_CHECK 0  // scalar decay, 1: one check per stage of whether the
+                                        // running scale can leave its range, the per-position
+                                        // check skipped when it cannot (measured slower: the
+                                        // branch splits the unrolled positions)
+#endif
 #ifndef GDN_PREFILL_GDN_HALVING
 #define GDN_PREFILL_GDN_HALVING 0  // scalar decay, 4 lanes per row: one halving reduction of
                                    // the A and O values with the deltas broadcast
@@ -618,6 +624,26 @@ prefill_kernel(float* __restrict__ state, const float* __restrict__ q,
 #pragma unroll
         for (int n = 0; n < NH; ++n)
             e_lane[n] = (!kCh && lane < TS) ? expf(st.bg[gi][lane % TS][n][1]) : 1.0f;
+        // Scalar decay: whether the running scale can leave its range within
+        // this stage. Without a fold every prefix product of the stage's
+        // decays lies between the product of their parts below 1 and the
+        // product of their parts above 1; with a factor-2 margin for rounding,
+        // a stage whose bounds stay inside needs no per-position check (and
+        // no position of it would fold: the results are the same).
+        bool may_fold = true;
+        if constexpr (!kCh && GDN_PREFILL_STAGE_FOLD_CHECK) {
+            may_fold = false;
+#pragma unroll
+            for (int n = 0; n < NH; ++n) {
+                float lo = fminf(e_lane[n], 1.0f), hi = fmaxf(e_lane[n], 1.0f);
+#pragma unroll
+                for (int off = 16; off > 0; off >>= 1) {
+                    lo *= __shfl_xor_sync(kFull, lo, off);
+                    hi *= __shfl_xor_sync(kFull, hi, off);
+                }
+                may_fold |= !(sc[n] * lo >= 2.0f * kScaleLo && sc[n] * hi <= 0.5f * kScaleHi);
+            }
+        }
 
         if (s == 0) {
             // first key dot: a = W.k_0 (kCh: first the decay of position 0,
@@ -682,9 +708,12 @@ prefill_kernel(float* __restrict__ state, const float* __restrict__ q,
                     float s_new[NH];
                     bool fold = false;
 #pragma unroll
-                    for (int n = 0; n < NH; ++n) {
+                    for (int n = 0; n < NH; ++n)
                         s_new[n] = sc[n] * __shfl_sync(kFull, e_lane[n], tp);
-                        fold |= !(s_new[n] >= kScaleLo && s_new[n] <= kScaleHi);
+                    if (may_fold) {      // uniform across the warp
+#pragma unroll
+                        for (int n = 0; n < NH; ++n)
+                            fold |= !(s_new[n] >= kScaleLo && s_new[n] <= kScaleHi);
                     }
                     if (fold) {          // rare, and uniform across the warp
 #pragma unroll
@@ -738,9 +767,12 @@ prefill_kernel(float* __restrict__ state, const float* __restrict__ q,
                         float s_new[NH];
                         bool fold = false;
 #pragma unroll
-                        for (int n = 0; n < NH; ++n) {
+                        for (int n = 0; n < NH; ++n)
                             s_new[n] = sc[n] * __shfl_sync(kFull, e_lane[n], tp);
-                            fold |= !(s_new[n] >= kScaleLo && s_new[n] <= kScaleHi);
+                        if (may_fold) {  // uniform across the warp
+#pragma unroll
+                            for (int n = 0; n < NH; ++n)
+                                fold |= !(s_new[n] >= kScaleLo && s_new[n] <= kScaleHi);
                         }
                         if (fold) {      // rare, and uniform across the warp
 #pragma unroll
